@@ -1,0 +1,418 @@
+/*
+ * hyb_oracle.c -- CPU oracle for the hybrid_v2 two-tier KV cache.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
+ * cpu_baseline / reference legs of bench.py may load this library.  The GPU
+ * library never links, calls or includes anything from here, and this file
+ * includes nothing from the GPU side.
+ *
+ * What it computes (source: the web page "DeepSeek V4混合式KV Cache推理优化实战解析",
+ * cited below as [hybrid_v2 page] with its section numbers):
+ *   - The hybrid_v2 cache contract (section 3.1): hot zone of 32 tokens kept in
+ *     FP16 and never quantized; cold zone in 64-token blocks of INT8 (INT4 for
+ *     "L2" cold blocks) with a block-wise scale (sections 2.1, 2.2, 3.2).
+ *   - The hot zone is the MOST RECENT 32 tokens (section 2.1).  (The vLLM
+ *     snippet of section 4.2 slices the first 32 instead; the prose wins.)
+ *   - Quantization of the cold part (section 4.2, "quantize_int8"): symmetric
+ *     absmax scaling, one FP32 scale per (block, kv-head, K|V),
+ *     scale = absmax / Q with Q = 127 (INT8) or 7 (INT4), codes =
+ *     clamp(round-half-even(x / scale), -Q, Q).
+ *   - A block that is filled over several calls keeps one scale: when newly
+ *     sealed tokens need a larger scale, the codes already in the block are
+ *     re-quantized to the new scale in place (section 3.2 says a re-tiered
+ *     block gets a new INT8 scale assigned in the kernel; the page is silent on
+ *     partial blocks -- this is the plainest reading that keeps the block
+ *     layout fixed).
+ *   - Attention (section 4.2, steps 3-5): one softmax over hot and cold keys
+ *     together, on the dequantized cold values (code * scale) and the FP16 hot
+ *     values, evaluated here in FP64.  The page's torch.cat of two separately
+ *     normalised outputs is not a softmax over the union; the exact softmax
+ *     over the union is the definition used.
+ *
+ * Everything here is deliberately plain: per-element loops, no blocking, no
+ * vectorisation, FP32 arithmetic exactly where the quantizer defines it (IEEE
+ * division, rintf under the default round-to-nearest-even mode; build with
+ * -ffp-contract=off so no multiply-add is fused) and FP64 for attention.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORA_OK 0
+#define ORA_ERR_INVALID -1
+#define ORA_ERR_NOMEM -2
+
+/* ------------------------------------------------------------------ */
+/* IEEE 754 binary16 -> double, written from the format definition:   */
+/* 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits.            */
+/* ------------------------------------------------------------------ */
+double ora_half_to_double(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int expo = (h >> 10) & 0x1f;
+  int frac = h & 0x3ff;
+  double v;
+  if (expo == 0) {
+    v = ldexp((double)frac, -24); /* subnormal: frac * 2^-24 */
+  } else if (expo == 31) {
+    v = frac ? NAN : INFINITY;
+  } else {
+    v = ldexp((double)(1024 + frac), expo - 25); /* (1 + frac/1024) * 2^(expo-15) */
+  }
+  return sign ? -v : v;
+}
+
+static float half_to_float(uint16_t h) { return (float)ora_half_to_double(h); }
+
+/* ------------------------------------------------------------------ */
+/* Cache state, kept in LOGICAL form: per sequence, per logical block. */
+/* ------------------------------------------------------------------ */
+typedef struct {
+  int batch, hkv, hq, d, hot, block, max_blocks, quant_bits;
+  int32_t *len;     /* [batch] tokens in the cache                      */
+  int32_t *n_int4;  /* [batch] logical blocks < n_int4 are INT4 ("L2")  */
+  uint16_t *ring;   /* [batch][hkv][hot][2][d] FP16 bits, slot = pos % hot */
+  /* per (batch, logical block): NULL until the first token is sealed */
+  int8_t **codes;   /* each [hkv][2][block][d], unpacked codes          */
+  float **scale;    /* each [hkv][2]                                    */
+  int *qmax;        /* [batch*max_blocks] 127 or 7 once sealed, else 0  */
+} ora_cache;
+
+void ora_free(ora_cache *c);
+
+ora_cache *ora_new(int batch, int hkv, int hq, int d, int hot, int block,
+                   int max_blocks, int quant_bits) {
+  if (batch <= 0 || hkv <= 0 || hq <= 0 || hq % hkv || d <= 0 || hot <= 0 ||
+      block <= 0 || max_blocks < 0 || (quant_bits != 8 && quant_bits != 4))
+    return NULL;
+  ora_cache *c = (ora_cache *)calloc(1, sizeof(ora_cache));
+  if (!c) return NULL;
+  c->batch = batch; c->hkv = hkv; c->hq = hq; c->d = d; c->hot = hot;
+  c->block = block; c->max_blocks = max_blocks; c->quant_bits = quant_bits;
+  size_t nb = (size_t)batch * (max_blocks > 0 ? max_blocks : 1);
+  c->len = (int32_t *)calloc(batch, sizeof(int32_t));
+  c->n_int4 = (int32_t *)calloc(batch, sizeof(int32_t));
+  c->ring = (uint16_t *)calloc((size_t)batch * hkv * hot * 2 * d, sizeof(uint16_t));
+  c->codes = (int8_t **)calloc(nb, sizeof(int8_t *));
+  c->scale = (float **)calloc(nb, sizeof(float *));
+  c->qmax = (int *)calloc(nb, sizeof(int));
+  if (!c->len || !c->n_int4 || !c->ring || !c->codes || !c->scale || !c->qmax) {
+    ora_free(c);
+    return NULL;
+  }
+  return c;
+}
+
+void ora_free(ora_cache *c) {
+  if (!c) return;
+  size_t nb = (size_t)c->batch * (c->max_blocks > 0 ? c->max_blocks : 1);
+  if (c->codes)
+    for (size_t i = 0; i < nb; i++) free(c->codes[i]);
+  if (c->scale)
+    for (size_t i = 0; i < nb; i++) free(c->scale[i]);
+  free(c->codes); free(c->scale); free(c->qmax);
+  free(c->len); free(c->n_int4); free(c->ring);
+  free(c);
+}
+
+int ora_set_n_int4(ora_cache *c, const int32_t *n_int4) {
+  for (int b = 0; b < c->batch; b++) c->n_int4[b] = n_int4 ? n_int4[b] : 0;
+  return ORA_OK;
+}
+
+int32_t ora_len(const ora_cache *c, int b) { return c->len[b]; }
+
+static uint16_t *ring_row(ora_cache *c, int b, int h, int slot, int kv) {
+  return c->ring + ((((size_t)b * c->hkv + h) * c->hot + slot) * 2 + kv) * c->d;
+}
+
+/* Round half to even on FP32, as the IEEE default rounding mode does. */
+static float rne(float x) { return rintf(x); }
+
+static int clampi(int v, int q) { return v > q ? q : (v < -q ? -q : v); }
+
+/*
+ * One append call for the whole batch, [hybrid_v2 page] sections 2.1, 3.2, 4.2:
+ * n_new[b] new tokens for sequence b, FP16 K and V laid out
+ * [batch][max_new][hkv][d].  Tokens that leave the hot zone are sealed into
+ * their cold block; the newest (up to hot) tokens go to the hot ring.
+ * Returns ORA_ERR_INVALID (and changes nothing) when any n_new is negative or
+ * above max_new or when a sequence would outgrow max_blocks cold blocks.
+ */
+int ora_append(ora_cache *c, const int32_t *n_new, int max_new,
+               const uint16_t *k_new, const uint16_t *v_new) {
+  const int d = c->d, hot = c->hot, blk = c->block, hkv = c->hkv;
+  for (int b = 0; b < c->batch; b++) {
+    int n = n_new[b];
+    if (n < 0 || n > max_new) return ORA_ERR_INVALID;
+    long L_new = (long)c->len[b] + n;
+    long cold_new = L_new > hot ? L_new - hot : 0;
+    if (cold_new > (long)c->max_blocks * blk) return ORA_ERR_INVALID;
+  }
+  for (int b = 0; b < c->batch; b++) {
+    const int n = n_new[b];
+    const int L_old = c->len[b];
+    const int L_new = L_old + n;
+    const int e0 = L_old > hot ? L_old - hot : 0; /* first position leaving */
+    const int e1 = L_new > hot ? L_new - hot : 0; /* one past the last      */
+    /* FP16 bits of position p, channel ch, for head h and K (kv=0) or V (1). */
+#define SRC(p, h, kv, ch)                                                      \
+  ((p) < L_old ? ring_row(c, b, h, (p) % hot, kv)[ch]                          \
+               : ((kv) == 0 ? k_new : v_new)[(((size_t)b * max_new + ((p) - L_old)) * hkv + (h)) * d + (ch)])
+    /* group the evicted positions by logical block, ascending */
+    for (int p0 = e0; p0 < e1;) {
+      const int i = p0 / blk;
+      const int p1 = (i + 1) * blk < e1 ? (i + 1) * blk : e1;
+      const size_t bi = (size_t)b * c->max_blocks + i;
+      const int first_slot = p0 - i * blk;
+      const int q = (c->quant_bits == 4 || i < c->n_int4[b]) ? 7 : 127;
+      if (!c->codes[bi]) {
+        c->codes[bi] = (int8_t *)calloc((size_t)hkv * 2 * blk * d, 1);
+        c->scale[bi] = (float *)calloc((size_t)hkv * 2, sizeof(float));
+        if (!c->codes[bi] || !c->scale[bi]) return ORA_ERR_NOMEM;
+        c->qmax[bi] = q;
+      }
+      for (int h = 0; h < hkv; h++) {
+        for (int kv = 0; kv < 2; kv++) {
+          int8_t *cd = c->codes[bi] + ((size_t)h * 2 + kv) * blk * d;
+          float *sp = c->scale[bi] + h * 2 + kv;
+          /* absmax over the group's tokens x channels (exact in FP32) */
+          float a = 0.0f;
+          for (int p = p0; p < p1; p++)
+            for (int ch = 0; ch < d; ch++) {
+              float x = fabsf(half_to_float(SRC(p, h, kv, ch)));
+              if (x > a) a = x;
+            }
+          float s_c = a / (float)q;
+          float s;
+          if (first_slot == 0) {
+            s = s_c; /* empty block: its scale comes from these tokens */
+          } else {
+            s = *sp;
+            if (s_c > s) {
+              /* grow the scale; re-quantize the codes already sealed */
+              for (int t = 0; t < first_slot; t++)
+                for (int ch = 0; ch < d; ch++) {
+                  float old = (float)cd[t * d + ch] * s;
+                  cd[t * d + ch] = (int8_t)clampi((int)rne(old / s_c), q);
+                }
+              s = s_c;
+            }
+          }
+          *sp = s;
+          for (int p = p0; p < p1; p++)
+            for (int ch = 0; ch < d; ch++) {
+              float x = half_to_float(SRC(p, h, kv, ch));
+              int code = (s == 0.0f) ? 0 : clampi((int)rne(x / s), q);
+              cd[(p - i * blk) * d + ch] = (int8_t)code;
+            }
+        }
+      }
+      p0 = p1;
+    }
+    /* newest min(n, hot) tokens into the hot ring, slot = position % hot */
+    const int first_hot = L_new - (n < hot ? n : hot);
+    for (int p = first_hot; p < L_new; p++)
+      for (int h = 0; h < hkv; h++)
+        for (int kv = 0; kv < 2; kv++) {
+          const uint16_t *src = ((kv == 0) ? k_new : v_new) +
+                                (((size_t)b * max_new + (p - L_old)) * hkv + h) * d;
+          memcpy(ring_row(c, b, h, p % hot, kv), src, (size_t)d * sizeof(uint16_t));
+        }
+#undef SRC
+    c->len[b] = L_new;
+  }
+  return ORA_OK;
+}
+
+/* Value of position p (channel ch) of head h, K (kv=0) or V (kv=1), in FP64:
+ * hot FP16 value, or code * scale for a cold position. */
+static double kv_value(const ora_cache *c, int b, int h, int kv, int p, int ch) {
+  const int L = c->len[b];
+  const int cold = L > c->hot ? L - c->hot : 0;
+  if (p >= cold)
+    return ora_half_to_double(
+        c->ring[((((size_t)b * c->hkv + h) * c->hot + p % c->hot) * 2 + kv) * c->d + ch]);
+  const int i = p / c->block;
+  const size_t bi = (size_t)b * c->max_blocks + i;
+  const int8_t code = c->codes[bi][(((size_t)h * 2 + kv) * c->block + (p - i * c->block)) * c->d + ch];
+  return (double)code * (double)c->scale[bi][h * 2 + kv];
+}
+
+/*
+ * Single-query decode attention, FP64, for the (b, query head) pairs listed in
+ * `pairs` (2*npairs ints) or for all pairs when pairs == NULL.
+ * q: FP16 [batch][hq][d].  Query head h reads kv head h / (hq/hkv).
+ * out: [batch][hq][d], lse: [batch][hq] (natural log); entries of pairs not
+ * listed are left untouched.  An empty sequence gives out = 0, lse = -inf.
+ */
+int ora_decode(const ora_cache *c, const uint16_t *q, double softmax_scale,
+               const int32_t *pairs, int npairs, double *out, double *lse,
+               int nthreads) {
+  const int d = c->d, g = c->hq / c->hkv;
+  const int total = pairs ? npairs : c->batch * c->hq;
+  if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+  for (int w = 0; w < total; w++) {
+    const int b = pairs ? pairs[2 * w] : w / c->hq;
+    const int hh = pairs ? pairs[2 * w + 1] : w % c->hq;
+    const int hk = hh / g;
+    const int L = c->len[b];
+    double *o = out + ((size_t)b * c->hq + hh) * d;
+    if (L == 0) {
+      for (int ch = 0; ch < d; ch++) o[ch] = 0.0;
+      lse[(size_t)b * c->hq + hh] = -INFINITY;
+      continue;
+    }
+    double *z = (double *)malloc(sizeof(double) * L);
+    const uint16_t *qh = q + ((size_t)b * c->hq + hh) * d;
+    double m = -INFINITY;
+    for (int j = 0; j < L; j++) {
+      double acc = 0.0;
+      for (int ch = 0; ch < d; ch++)
+        acc += ora_half_to_double(qh[ch]) * kv_value(c, b, hk, 0, j, ch);
+      z[j] = softmax_scale * acc;
+      if (z[j] > m) m = z[j];
+    }
+    double l = 0.0;
+    for (int j = 0; j < L; j++) {
+      z[j] = exp(z[j] - m);
+      l += z[j];
+    }
+    for (int ch = 0; ch < d; ch++) {
+      double acc = 0.0;
+      for (int j = 0; j < L; j++) acc += z[j] * kv_value(c, b, hk, 1, j, ch);
+      o[ch] = acc / l;
+    }
+    lse[(size_t)b * c->hq + hh] = m + log(l);
+    free(z);
+  }
+  return ORA_OK;
+}
+
+/*
+ * Log-sum-exp merge of per-split partial results, FP64 (the split-KV
+ * "flash-decoding" combine; the merge of softmax pieces that the page's
+ * torch.cat of section 4.2 stands in for).  o_part: [rows][n_splits][d],
+ * each the softmax-normalised output of one split; lse_part: [rows][n_splits]
+ * (natural log, -inf for an empty split).  out: [rows][d]; lse: [rows].
+ */
+int ora_combine(int rows, int n_splits, int d, const double *o_part,
+                const double *lse_part, double *out, double *lse) {
+  for (int r = 0; r < rows; r++) {
+    double m = -INFINITY;
+    for (int s = 0; s < n_splits; s++)
+      if (lse_part[(size_t)r * n_splits + s] > m) m = lse_part[(size_t)r * n_splits + s];
+    double *o = out + (size_t)r * d;
+    if (m == -INFINITY) {
+      for (int ch = 0; ch < d; ch++) o[ch] = 0.0;
+      lse[r] = -INFINITY;
+      continue;
+    }
+    double wsum = 0.0;
+    for (int ch = 0; ch < d; ch++) o[ch] = 0.0;
+    for (int s = 0; s < n_splits; s++) {
+      double w = exp(lse_part[(size_t)r * n_splits + s] - m);
+      wsum += w;
+      for (int ch = 0; ch < d; ch++) o[ch] += w * o_part[((size_t)r * n_splits + s) * d + ch];
+    }
+    for (int ch = 0; ch < d; ch++) o[ch] /= wsum;
+    lse[r] = m + log(wsum);
+  }
+  return ORA_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Inspection of the logical state (for the oracle's own tests).       */
+/* ------------------------------------------------------------------ */
+
+/* Logical block i of sequence b: codes [hkv][2][block][d] (slots not yet
+ * sealed are 0) and scales [hkv][2].  Returns Q (127 or 7), or 0 if the
+ * block holds no sealed token. */
+int ora_get_block(const ora_cache *c, int b, int i, int8_t *codes, float *scales) {
+  const size_t bi = (size_t)b * c->max_blocks + i;
+  if (b < 0 || b >= c->batch || i < 0 || i >= c->max_blocks || !c->codes[bi]) return 0;
+  memcpy(codes, c->codes[bi], (size_t)c->hkv * 2 * c->block * c->d);
+  memcpy(scales, c->scale[bi], (size_t)c->hkv * 2 * sizeof(float));
+  return c->qmax[bi];
+}
+
+/* Hot ring of sequence b: FP16 bits [hkv][hot][2][d]. */
+int ora_get_ring(const ora_cache *c, int b, uint16_t *ring) {
+  memcpy(ring, c->ring + (size_t)b * c->hkv * c->hot * 2 * c->d,
+         (size_t)c->hkv * c->hot * 2 * c->d * sizeof(uint16_t));
+  return ORA_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* The device memory format, written out from its definition:          */
+/*   cold pool bytes [num_phys][hkv][2][tile] with tile = block*d bytes */
+/*   (K tile, then V tile, per physical block and kv head).            */
+/*   K tile, INT8: token-major, byte (t, ch) at t*d + ch.              */
+/*   V tile, INT8: channel-major, 64 token bytes per channel row, the  */
+/*     four 16-byte chunks of row ch stored at chunk index             */
+/*     (t/16) XOR ((ch/2) % 4): byte (t, ch) at                        */
+/*     ch*64 + (((t/16) ^ ((ch/2) % 4)) * 16) + t%16.                  */
+/*   INT4 tiles use the first half of the tile.  Eight consecutive     */
+/*   codes e=0..7 along the packed axis share one 32-bit word: code e  */
+/*   sits in byte e%4, low nibble for e<4, high nibble for e>=4, as a  */
+/*   4-bit two's complement number.                                    */
+/*   K tile, INT4: token-major, 64 bytes per token; channel ch of      */
+/*     token t in word t*16 + ch/8 (bytes), element ch%8.              */
+/*   V tile, INT4: channel-major, 32 bytes per channel row in four     */
+/*     8-byte units of 16 tokens, unit u stored at u XOR ((ch/4) % 4); */
+/*     within a unit, tokens 0..7 in its first word, 8..15 in the      */
+/*     second.                                                         */
+/*   scales: float [num_phys][hkv][2].                                 */
+/*   hot ring: FP16 [batch][hkv][hot][2][d] (K row, then V row).       */
+/* Only sealed slots are written; other bytes are left as they are.    */
+/* ------------------------------------------------------------------ */
+static void put_nibble(uint8_t *word4, int e, int code) {
+  uint8_t *byte = word4 + (e & 3);
+  uint8_t nib = (uint8_t)(code & 0xf);
+  if (e < 4) *byte = (uint8_t)((*byte & 0xf0) | nib);
+  else *byte = (uint8_t)((*byte & 0x0f) | (nib << 4));
+}
+
+int ora_export(const ora_cache *c, const int32_t *block_table, int num_phys,
+               uint8_t *cold, float *scales, uint16_t *hot, int32_t *seq_lens) {
+  const int d = c->d, blk = c->block, hkv = c->hkv;
+  const size_t tile = (size_t)blk * d;
+  if (d != 128 || blk != 64) return ORA_ERR_INVALID; /* format defined for 64 x 128 */
+  for (int b = 0; b < c->batch; b++) {
+    const int L = c->len[b];
+    const int cold_len = L > c->hot ? L - c->hot : 0;
+    const int nblk = (cold_len + blk - 1) / blk;
+    for (int i = 0; i < nblk; i++) {
+      const size_t bi = (size_t)b * c->max_blocks + i;
+      const int phys = block_table[(size_t)b * c->max_blocks + i];
+      if (phys < 0 || phys >= num_phys) return ORA_ERR_INVALID;
+      const int sealed = cold_len - i * blk < blk ? cold_len - i * blk : blk;
+      for (int h = 0; h < hkv; h++) {
+        for (int kv = 0; kv < 2; kv++) {
+          const int8_t *cd = c->codes[bi] + ((size_t)h * 2 + kv) * blk * d;
+          uint8_t *t8 = cold + (((size_t)phys * hkv + h) * 2 + kv) * tile;
+          scales[((size_t)phys * hkv + h) * 2 + kv] = c->scale[bi][h * 2 + kv];
+          for (int t = 0; t < sealed; t++)
+            for (int ch = 0; ch < d; ch++) {
+              const int code = cd[t * d + ch];
+              if (c->qmax[bi] == 127) {
+                if (kv == 0) t8[t * d + ch] = (uint8_t)code;
+                else t8[ch * 64 + (((t / 16) ^ ((ch / 2) % 4)) * 16) + t % 16] = (uint8_t)code;
+              } else {
+                if (kv == 0) put_nibble(t8 + t * 64 + (ch / 8) * 4, ch % 8, code);
+                else {
+                  const int unit = (t / 16) ^ ((ch / 4) % 4);
+                  const int in_unit = t % 16;
+                  put_nibble(t8 + ch * 32 + unit * 8 + (in_unit / 8) * 4, in_unit % 8, code);
+                }
+              }
+            }
+        }
+      }
+    }
+    seq_lens[b] = L;
+  }
+  memcpy(hot, c->ring, (size_t)c->batch * hkv * c->hot * 2 * d * sizeof(uint16_t));
+  return ORA_OK;
+}
