@@ -1,0 +1,259 @@
+/*
+ * hyb_kv.h -- C ABI of the B200 (sm_100a) hybrid_v2 KV-cache decode library.
+ *
+ * The method: web page "DeepSeek V4混合式KV Cache推理优化实战解析" (cited as
+ * [hybrid_v2 page] below).  A sequence's KV cache has two tiers:
+ *   - a hot zone holding the most recent 32 tokens in FP16, never quantized,
+ *     K and V interleaved per token, 512-byte aligned (sections 2.1, 3.1, 3.2);
+ *   - a cold zone holding all earlier tokens in 64-token blocks of symmetric
+ *     INT8 with a block-wise scale, INT4 for the "L2" cold blocks (sections
+ *     2.1, 2.2, 3.1), reached through a block table (section 3.2, block header).
+ * The three fields of the hybrid_v2 contract are hot_tokens (power of two),
+ * quantization_bits (4 or 8) and block_size (a multiple of 8); the example
+ * set 32 / 8 / 64 is the only one this library implements (section 3.1;
+ * section 5.1 for the invalid-value error).
+ *
+ * Calls:
+ *   hyb_kv_append      seal tokens leaving the hot zone into cold blocks
+ *                      (absmax / RNE / clamp quantization) and write the new
+ *                      tokens into the hot ring ([hybrid_v2 page] 4.2, step 2)
+ *   hyb_decode_attn    single-query attention of q[B][Hq][d] over hot + cold,
+ *                      GQA, split-KV, FP32 accumulation, FP16 output
+ *                      ([hybrid_v2 page] 4.2, steps 3-5)
+ *   hyb_combine        log-sum-exp merge of split partial results (the merge
+ *                      that replaces the page's torch.cat of step 5)
+ *
+ * Conventions for every call:
+ *   - Pointers named "device" are CUDA device pointers the caller allocated;
+ *     the library allocates no memory and keeps no pointer after a call
+ *     returns.  Buffers must stay alive until the stream work completes.
+ *   - Work is enqueued asynchronously on `stream` (0 = legacy default stream).
+ *   - Return value: HYB_OK (0) or a negative HYB_ERR_* code; on an error
+ *     return nothing was enqueued (HYB_ERR_CUDA: a launch failed; the CUDA
+ *     error is kept for hyb_last_cuda_error()).
+ *   - Errors found on the device (a block-table entry out of range, an n_new
+ *     above max_new, a sequence outgrowing its block table, a bounded wait
+ *     that ran out) never trap: the kernel skips the affected unit and records
+ *     the first such HYB_STATUS_* code in the sticky device word desc->status
+ *     (atomic compare-and-swap from 0).  Read it with hyb_read_status().
+ *   - Not thread-safe with respect to the same cache: calls on one cache must
+ *     be ordered on one stream (or by events).
+ */
+#ifndef HYB_KV_H
+#define HYB_KV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *hyb_stream_t; /* same type as cudaStream_t */
+
+/* return codes */
+#define HYB_OK 0
+#define HYB_ERR_INVALID_VALUE (-1) /* bad config value, shape, null or misaligned pointer;
+                                      named after the page's CUDA_ERROR_INVALID_VALUE (3.1) */
+#define HYB_ERR_UNSUPPORTED (-2)   /* valid per the page but not built: hot_tokens != 32,
+                                      block_size != 64, head_dim != 128, Hq/Hkv > 8 */
+#define HYB_ERR_WORKSPACE (-3)     /* workspace missing or smaller than required */
+#define HYB_ERR_CUDA (-4)          /* a CUDA runtime call or launch failed */
+
+/* device status codes (sticky, first error wins) */
+#define HYB_STATUS_OK 0
+#define HYB_STATUS_BAD_BLOCK 1     /* block-table entry < 0 or >= num_phys_blocks; block skipped */
+#define HYB_STATUS_BAD_N_NEW 2     /* n_new[b] < 0 or > max_new; sequence b left unchanged */
+#define HYB_STATUS_CAPACITY 3      /* append would need more than max_blocks_per_seq blocks;
+                                      sequence b left unchanged */
+#define HYB_STATUS_SEQ_LEN 4       /* seq_lens[b] < 0 or > max_seq_len at decode; b skipped */
+#define HYB_STATUS_TIMEOUT 5       /* a bounded wait inside a kernel gave up; unit skipped */
+
+/*
+ * The cache descriptor (host struct; the pointers inside are device memory).
+ *
+ * Geometry: hot_tokens HOT = 32, block_size BLK = 64, head_dim D = 128,
+ * num_kv_heads Hkv >= 1, num_q_heads Hq a multiple of Hkv with Hq/Hkv <= 8
+ * (query head h reads kv head h / (Hq/Hkv)), quant_bits 8 (INT8 cold blocks;
+ * logical blocks below n_int4_blocks[b] are INT4) or 4 (every cold block INT4).
+ *
+ * Token positions 0..L-1 of sequence b (L = seq_lens[b]): positions >= L-32
+ * are hot, the others cold; cold position p lives in logical block p/64,
+ * slot p%64, of physical block block_table[b][p/64].
+ *
+ * Memory layouts (all little-endian, all device memory):
+ *   hot    FP16 [batch][Hkv][HOT][2][D]: per (sequence, kv head) a ring of 32
+ *          token slots, slot = position % 32, each slot the K row (D halves)
+ *          followed by the V row (D halves) -- 512 B per token, 16 KB per
+ *          (sequence, kv head).  Base 512-byte aligned ([hybrid_v2 page] 3.2).
+ *   cold   bytes [num_phys_blocks][Hkv][2][8192]: per physical block and kv
+ *          head a K tile then a V tile of 64 tokens x 128 channels.  Base
+ *          16-byte aligned.
+ *            K, INT8: token-major, code of (slot t, channel c) at t*128 + c.
+ *            V, INT8: channel-major rows of 64 bytes; the 16-byte chunk
+ *              holding slots 16j..16j+15 of channel c is stored at chunk
+ *              position j ^ ((c/2) % 4): byte c*64 + 16*(j ^ ((c/2)%4)) + t%16.
+ *            INT4 tiles use the first 4096 bytes: 4-bit two's complement
+ *              codes, eight consecutive codes e = 0..7 along the packed axis
+ *              per 32-bit word, code e in byte e%4, low nibble for e < 4 and
+ *              high nibble for e >= 4.
+ *            K, INT4: 64 bytes per token; channel c in word t*16 + c/8.
+ *            V, INT4: channel-major rows of 32 bytes in four 8-byte units of
+ *              16 slots, unit j stored at unit position j ^ ((c/4) % 4);
+ *              slots 16j..16j+7 in the unit's first word, the rest in its
+ *              second.
+ *          Codes are in [-127, 127] (INT8) or [-7, 7] (INT4); -128 / -8 are
+ *          never produced.  Bytes of slots not yet sealed are never written.
+ *   scales FP32 [num_phys_blocks][Hkv][2]: K scale, V scale of each tile;
+ *          the value of a cold element is code * scale.
+ *   block_table int32 [batch][max_blocks_per_seq]; entries for blocks a
+ *          sequence does not reach are ignored.  A block that appends write
+ *          into must belong to one sequence only.
+ *   seq_lens int32 [batch]: tokens in each sequence; hyb_kv_append advances it.
+ *   n_int4_blocks int32 [batch] or NULL: logical blocks below it are INT4
+ *          ("L2" blocks, [hybrid_v2 page] 2.2 / 3.1).  A block's format is
+ *          fixed when its first token is sealed; do not change n_int4_blocks
+ *          for blocks that already hold tokens.
+ *   status int32 device word, 0 = ok (see HYB_STATUS_*).
+ * A fresh cache is: seq_lens all 0, status 0 (contents of hot / cold / scales
+ * do not matter).
+ */
+typedef struct hyb_cache_desc {
+  int32_t hot_tokens;         /* must be 32 */
+  int32_t block_size;         /* must be 64 */
+  int32_t head_dim;           /* must be 128 */
+  int32_t quant_bits;         /* 8 or 4 */
+  int32_t num_kv_heads;       /* Hkv >= 1 */
+  int32_t num_q_heads;        /* Hq, multiple of Hkv, Hq/Hkv <= 8 */
+  int32_t num_phys_blocks;    /* physical blocks in `cold` / `scales` */
+  int32_t max_blocks_per_seq; /* columns of block_table */
+  int32_t batch;              /* sequences */
+  int32_t reserved;           /* set to 0 */
+  void *hot;                  /* device, see above */
+  void *cold;                 /* device */
+  float *scales;              /* device */
+  const int32_t *block_table; /* device */
+  int32_t *seq_lens;          /* device */
+  const int32_t *n_int4_blocks; /* device or NULL */
+  int32_t *status;            /* device */
+} hyb_cache_desc;
+
+/*
+ * Host-only check of a descriptor (no GPU needed, nothing enqueued).
+ * Returns HYB_OK, HYB_ERR_INVALID_VALUE (hot_tokens not a power of two in
+ * {16, 32, 64, 128}, block_size not a multiple of 8, quant_bits not 4 or 8,
+ * non-positive sizes, Hq not a multiple of Hkv, null or misaligned pointers)
+ * or HYB_ERR_UNSUPPORTED (a valid configuration other than 32 / 64 / D=128,
+ * or Hq/Hkv > 8).  The contract is the page's section 3.1 and 5.1.
+ */
+int hyb_check_desc(const hyb_cache_desc *desc);
+
+/*
+ * Append n_new[b] tokens to every sequence b ([hybrid_v2 page] 4.2 step 2,
+ * quantize_int8, and 2.1 / 3.2 for the tiers).
+ *   n_new  device int32 [batch], each in [0, max_new].
+ *   k_new, v_new  device FP16 [batch][max_new][Hkv][D]; row j of sequence b
+ *          is position seq_lens[b] + j.  Rows j >= n_new[b] are not read.
+ *          16-byte aligned.
+ * For L_old = seq_lens[b] and L_new = L_old + n_new[b], the positions
+ * max(0, L_old-32) .. max(0, L_new-32)-1 leave the hot zone in ascending
+ * order (their FP16 values come from the hot ring, or straight from k_new /
+ * v_new for new tokens that never become hot).  They are grouped by logical
+ * block; per group, kv head and K|V:
+ *   a   = max |x| over the group's tokens and channels (FP32, exact),
+ *   s_c = a / Q in IEEE FP32 (Q = 127, or 7 for INT4 blocks),
+ *   if the block held no token: s = s_c;
+ *   else if s_c > s_old: every code c already in the block becomes
+ *        clamp(rint((c * s_old) / s_c), -Q, Q) and s = s_c;
+ *   else s = s_old;
+ *   new codes = (s == 0) ? 0 : clamp(rint(x / s), -Q, Q)   (rint: half to even).
+ * Then the newest min(n_new[b], 32) tokens are written to hot slots
+ * position % 32 and seq_lens[b] = L_new.  The result is bit-exact and does
+ * not depend on the launch configuration.
+ * Device errors: HYB_STATUS_BAD_N_NEW or HYB_STATUS_CAPACITY (sequence
+ * untouched), HYB_STATUS_BAD_BLOCK (that block skipped, seq_lens still
+ * advanced -- the cache is then damaged and must be rebuilt).
+ */
+int hyb_kv_append(const hyb_cache_desc *desc, const int32_t *n_new, int32_t max_new,
+                  const void *k_new, const void *v_new, hyb_stream_t stream);
+
+/*
+ * Split planning for hyb_decode_attn (host only).  max_seq_len is a host
+ * upper bound of seq_lens[b]; split_tokens is a multiple of 64 (tokens per
+ * split of the cold range) or 0 for automatic.  Writes the split size used
+ * and the number of splits per sequence, n_splits = max(1,
+ * ceil(max(0, max_seq_len - 32) / split_tokens)).  Returns HYB_OK or
+ * HYB_ERR_INVALID_VALUE.  The automatic choice depends on the GPU's SM count
+ * (device 0 of the current context when none is current).
+ */
+int hyb_decode_plan(const hyb_cache_desc *desc, int32_t max_seq_len, int32_t split_tokens,
+                    int32_t *split_tokens_out, int32_t *n_splits_out);
+
+/* Bytes of workspace hyb_decode_attn needs for these arguments (0 when a
+ * single split suffices), or 0 with an invalid descriptor. */
+size_t hyb_decode_workspace_bytes(const hyb_cache_desc *desc, int32_t max_seq_len,
+                                  int32_t split_tokens);
+
+/*
+ * Single-query decode attention over hot + cold ([hybrid_v2 page] 4.2 steps
+ * 3-5; one softmax over all L keys of each sequence, no mask):
+ *   out[b][h] = sum_j softmax_j(z) V_j,  z_j = softmax_scale * (q[b][h] . K_j),
+ *   K_j, V_j = FP16 hot values, or code * scale for cold positions, of kv
+ *   head h / (Hq/Hkv).
+ *   q        device FP16 [batch][Hq][D], 16-byte aligned.
+ *   softmax_scale  finite, usually 1/sqrt(D).
+ *   max_seq_len    host upper bound of seq_lens (a larger device value sets
+ *            HYB_STATUS_SEQ_LEN and that sequence is skipped).
+ *   split_tokens   multiple of 64, or 0 = automatic (hyb_decode_plan).
+ *   workspace, workspace_bytes  device scratch of at least
+ *            hyb_decode_workspace_bytes() bytes (may be NULL when that is 0),
+ *            16-byte aligned; its contents need no initialisation.
+ *   out      device FP16 [batch][Hq][D] (round to nearest even), 16-byte aligned.
+ *   lse_out  device FP32 [batch][Hq] natural-log log-sum-exp of the logits, or NULL.
+ * An empty sequence (L = 0) gives out = 0 and lse = -inf.
+ * Arithmetic: cold dot products run exactly in integers (16-bit fixed-point q
+ * per head, 16-bit fixed-point softmax weights per 16-token group); hot
+ * tokens in FP32; the online softmax, the per-block scale products and all
+ * merges in FP32.  Accuracy versus exact FP64 attention on the same cache:
+ * max-abs error <= 2e-3 and per-row relative L2 <= 1e-3 on the measured
+ * workloads.
+ */
+int hyb_decode_attn(const hyb_cache_desc *desc, const void *q, float softmax_scale,
+                    int32_t max_seq_len, int32_t split_tokens, void *workspace,
+                    size_t workspace_bytes, void *out, float *lse_out, hyb_stream_t stream);
+
+/*
+ * Log-sum-exp merge of split partial results ([hybrid_v2 page] 4.2 step 5,
+ * done as a softmax merge):
+ *   rows = batch * num_q_heads;  o_partial device FP32 [rows][n_splits][D],
+ *   each split's normalised output; lse_partial device FP32 [rows][n_splits]
+ *   (natural log, -inf for an empty split).
+ *   out[r] = sum_s w_s o_s / sum_s w_s with w_s = exp(lse_s - max_s lse_s),
+ *   written as FP16 [rows][D]; lse_out[r] = max + log(sum_s w_s) (FP32, or
+ *   NULL).  All-empty rows give 0 and -inf.
+ * head_dim must be 128; n_splits >= 1.
+ */
+int hyb_combine(int32_t batch, int32_t num_q_heads, int32_t head_dim, int32_t n_splits,
+                const float *o_partial, const float *lse_partial, void *out, float *lse_out,
+                hyb_stream_t stream);
+
+/* Copy the device status word to *host_status (waits for `stream`), and
+ * reset it to 0 when `clear` is nonzero. */
+int hyb_read_status(const hyb_cache_desc *desc, int32_t *host_status, int32_t clear,
+                    hyb_stream_t stream);
+
+/* Text of a HYB_ERR_* return code or HYB_STATUS_* code (status codes are
+ * passed as 100 + code). Never NULL. */
+const char *hyb_strerror(int code);
+
+/* CUDA error number behind the last HYB_ERR_CUDA of this thread (0 if none). */
+int hyb_last_cuda_error(void);
+
+/* Library version, 10000*major + 100*minor + patch. */
+int hyb_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HYB_KV_H */

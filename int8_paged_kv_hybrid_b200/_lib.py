@@ -1,0 +1,163 @@
+"""ctypes binding of libhybkv.so (the C ABI in include/hyb_kv.h).
+
+Argument marshalling only: every step of the decode path runs in the CUDA
+library.  Tensors are PyTorch CUDA tensors (PyTorch provides device memory
+and streams); their data pointers go straight to the C functions.  There is
+no CPU fallback: if the library cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libhybkv.so")
+
+HYB_OK = 0
+HYB_ERR_INVALID_VALUE = -1
+HYB_ERR_UNSUPPORTED = -2
+HYB_ERR_WORKSPACE = -3
+HYB_ERR_CUDA = -4
+
+HYB_STATUS_OK = 0
+HYB_STATUS_BAD_BLOCK = 1
+HYB_STATUS_BAD_N_NEW = 2
+HYB_STATUS_CAPACITY = 3
+HYB_STATUS_SEQ_LEN = 4
+HYB_STATUS_TIMEOUT = 5
+
+EXPORTED = (
+    "hyb_check_desc", "hyb_kv_append", "hyb_decode_plan", "hyb_decode_workspace_bytes",
+    "hyb_decode_attn", "hyb_combine", "hyb_read_status", "hyb_strerror",
+    "hyb_last_cuda_error", "hyb_version",
+)
+
+
+class HybError(RuntimeError):
+    def __init__(self, code, what=""):
+        self.code = code
+        super().__init__("%s failed: %s (%d)" % (what, strerror(code), code))
+
+
+class CacheDesc(ctypes.Structure):
+    """Mirror of hyb_cache_desc."""
+    _fields_ = [
+        ("hot_tokens", ctypes.c_int32),
+        ("block_size", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("quant_bits", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("num_q_heads", ctypes.c_int32),
+        ("num_phys_blocks", ctypes.c_int32),
+        ("max_blocks_per_seq", ctypes.c_int32),
+        ("batch", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("hot", ctypes.c_void_p),
+        ("cold", ctypes.c_void_p),
+        ("scales", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p),
+        ("seq_lens", ctypes.c_void_p),
+        ("n_int4_blocks", ctypes.c_void_p),
+        ("status", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libhybkv.so (building it first if it is missing and nvcc exists)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        from . import build as _build
+        _build.build()
+    lib = ctypes.CDLL(path)
+    P, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    D = ctypes.POINTER(CacheDesc)
+    lib.hyb_check_desc.argtypes = [D]
+    lib.hyb_kv_append.argtypes = [D, P, i32, P, P, P]
+    lib.hyb_decode_plan.argtypes = [D, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
+    lib.hyb_decode_workspace_bytes.argtypes = [D, i32, i32]
+    lib.hyb_decode_workspace_bytes.restype = sz
+    lib.hyb_decode_attn.argtypes = [D, P, ctypes.c_float, i32, i32, P, sz, P, P, P]
+    lib.hyb_combine.argtypes = [i32, i32, i32, i32, P, P, P, P, P]
+    lib.hyb_read_status.argtypes = [D, ctypes.POINTER(i32), i32, P]
+    lib.hyb_strerror.argtypes = [ctypes.c_int]
+    lib.hyb_strerror.restype = ctypes.c_char_p
+    for name in ("hyb_check_desc", "hyb_kv_append", "hyb_decode_plan", "hyb_decode_attn",
+                 "hyb_combine", "hyb_read_status", "hyb_last_cuda_error", "hyb_version"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def strerror(code: int) -> str:
+    return load().hyb_strerror(int(code)).decode()
+
+
+def _check(rc, what):
+    if rc != HYB_OK:
+        raise HybError(rc, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def hyb_check_desc(desc: CacheDesc) -> int:
+    return load().hyb_check_desc(ctypes.byref(desc))
+
+
+def hyb_kv_append(desc, n_new, max_new, k_new, v_new, stream=None):
+    _check(load().hyb_kv_append(ctypes.byref(desc), _ptr(n_new), int(max_new), _ptr(k_new),
+                                _ptr(v_new), _stream(stream)), "hyb_kv_append")
+
+
+def hyb_decode_plan(desc, max_seq_len, split_tokens=0):
+    st, ns = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(load().hyb_decode_plan(ctypes.byref(desc), int(max_seq_len), int(split_tokens),
+                                  ctypes.byref(st), ctypes.byref(ns)), "hyb_decode_plan")
+    return st.value, ns.value
+
+
+def hyb_decode_workspace_bytes(desc, max_seq_len, split_tokens=0) -> int:
+    return int(load().hyb_decode_workspace_bytes(ctypes.byref(desc), int(max_seq_len), int(split_tokens)))
+
+
+def hyb_decode_attn(desc, q, softmax_scale, max_seq_len, split_tokens, workspace, out,
+                    lse_out=None, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().hyb_decode_attn(ctypes.byref(desc), _ptr(q), float(softmax_scale), int(max_seq_len),
+                                  int(split_tokens), _ptr(workspace), ws_bytes, _ptr(out),
+                                  _ptr(lse_out), _stream(stream)), "hyb_decode_attn")
+
+
+def hyb_combine(batch, num_q_heads, head_dim, n_splits, o_partial, lse_partial, out,
+                lse_out=None, stream=None):
+    _check(load().hyb_combine(int(batch), int(num_q_heads), int(head_dim), int(n_splits),
+                              _ptr(o_partial), _ptr(lse_partial), _ptr(out), _ptr(lse_out),
+                              _stream(stream)), "hyb_combine")
+
+
+def hyb_read_status(desc, clear=False, stream=None) -> int:
+    v = ctypes.c_int32(0)
+    _check(load().hyb_read_status(ctypes.byref(desc), ctypes.byref(v), 1 if clear else 0,
+                                  _stream(stream)), "hyb_read_status")
+    return v.value
+
+
+def hyb_last_cuda_error() -> int:
+    return load().hyb_last_cuda_error()
+
+
+def hyb_version() -> int:
+    return load().hyb_version()

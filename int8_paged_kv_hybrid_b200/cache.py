@@ -1,0 +1,92 @@
+"""HybridKVCache: device buffers of one hybrid_v2 cache plus its descriptor.
+
+PyTorch only allocates the buffers and supplies the stream; appends and
+attention go through the C ABI (libhybkv.so).  Layouts are those of
+include/hyb_kv.h.
+"""
+from __future__ import annotations
+
+import math
+
+from . import _lib
+
+HOT, BLOCK, HEAD_DIM = 32, 64, 128
+TILE_BYTES = BLOCK * HEAD_DIM
+
+
+class HybridKVCache:
+    def __init__(self, batch, num_kv_heads, num_q_heads, num_phys_blocks, max_blocks_per_seq,
+                 quant_bits=8, block_table=None, n_int4=None, device="cuda"):
+        import torch
+        self.batch, self.hkv, self.hq = int(batch), int(num_kv_heads), int(num_q_heads)
+        self.num_phys, self.max_blocks = int(num_phys_blocks), int(max_blocks_per_seq)
+        self.quant_bits = int(quant_bits)
+        dev = torch.device(device)
+        self.device = dev
+        self.hot = torch.zeros((self.batch, self.hkv, HOT, 2, HEAD_DIM), dtype=torch.float16, device=dev)
+        self.cold = torch.zeros((self.num_phys, self.hkv, 2, TILE_BYTES), dtype=torch.uint8, device=dev)
+        self.scales = torch.zeros((self.num_phys, self.hkv, 2), dtype=torch.float32, device=dev)
+        if block_table is None:
+            self.block_table = torch.full((self.batch, self.max_blocks), -1, dtype=torch.int32, device=dev)
+        else:
+            self.block_table = torch.as_tensor(block_table, dtype=torch.int32).to(dev).contiguous()
+            assert tuple(self.block_table.shape) == (self.batch, self.max_blocks)
+        self.seq_lens = torch.zeros(self.batch, dtype=torch.int32, device=dev)
+        self.n_int4 = None
+        if n_int4 is not None:
+            self.n_int4 = torch.as_tensor(n_int4, dtype=torch.int32).to(dev).contiguous()
+        self.status_word = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.desc = self._make_desc()
+        rc = _lib.hyb_check_desc(self.desc)
+        if rc != _lib.HYB_OK:
+            raise _lib.HybError(rc, "hyb_check_desc")
+
+    def _make_desc(self):
+        d = _lib.CacheDesc()
+        d.hot_tokens, d.block_size, d.head_dim = HOT, BLOCK, HEAD_DIM
+        d.quant_bits = self.quant_bits
+        d.num_kv_heads, d.num_q_heads = self.hkv, self.hq
+        d.num_phys_blocks, d.max_blocks_per_seq, d.batch = self.num_phys, self.max_blocks, self.batch
+        d.reserved = 0
+        d.hot = self.hot.data_ptr()
+        d.cold = self.cold.data_ptr()
+        d.scales = self.scales.data_ptr()
+        d.block_table = self.block_table.data_ptr()
+        d.seq_lens = self.seq_lens.data_ptr()
+        d.n_int4_blocks = None if self.n_int4 is None else self.n_int4.data_ptr()
+        d.status = self.status_word.data_ptr()
+        return d
+
+    # ---- the three calls ----
+    def append(self, n_new, k_new, v_new, stream=None):
+        """n_new: int32 CUDA [batch]; k_new, v_new: FP16 CUDA [batch][max_new][Hkv][128]."""
+        assert k_new.is_contiguous() and v_new.is_contiguous() and n_new.is_contiguous()
+        _lib.hyb_kv_append(self.desc, n_new, k_new.shape[1], k_new, v_new, stream)
+
+    def plan(self, max_seq_len, split_tokens=0):
+        return _lib.hyb_decode_plan(self.desc, max_seq_len, split_tokens)
+
+    def workspace(self, max_seq_len, split_tokens=0):
+        import torch
+        n = _lib.hyb_decode_workspace_bytes(self.desc, max_seq_len, split_tokens)
+        return None if n == 0 else torch.empty(n, dtype=torch.uint8, device=self.device)
+
+    def decode(self, q, softmax_scale, max_seq_len, split_tokens=0, out=None, lse=None,
+               workspace=None, stream=None):
+        """q: FP16 CUDA [batch][Hq][128] -> out FP16 [batch][Hq][128] (and lse FP32 [batch][Hq])."""
+        import torch
+        assert q.is_contiguous()
+        if out is None:
+            out = torch.empty((self.batch, self.hq, HEAD_DIM), dtype=torch.float16, device=self.device)
+        if workspace is None:
+            workspace = self.workspace(max_seq_len, split_tokens)
+        _lib.hyb_decode_attn(self.desc, q, softmax_scale, max_seq_len, split_tokens, workspace,
+                             out, lse, stream)
+        return out
+
+    def status(self, clear=False, stream=None):
+        return _lib.hyb_read_status(self.desc, clear, stream)
+
+
+def default_softmax_scale(head_dim=HEAD_DIM):
+    return 1.0 / math.sqrt(head_dim)

@@ -1,0 +1,223 @@
+// append.cu -- hyb_kv_append: seal tokens leaving the hot zone into cold
+// blocks and write the newest tokens into the hot ring.
+//
+// Method: web page "DeepSeek V4混合式KV Cache推理优化实战解析", section 4.2
+// (quantize_int8 of the cold part), sections 2.1 / 3.1 (INT8, INT4 for L2
+// blocks, block size 64, hot zone = most recent 32 tokens in FP16) and 3.2
+// (per-block scale held in the block header, re-assigned inside the kernel).
+//
+// One CTA per sequence; warp w handles (kv head, K|V) pairs w, w+nwarps, ...
+// A warp owns everything it writes (its tiles' bytes, its scale words and its
+// hot-ring rows), so no inter-warp ordering is needed until seq_lens[b] is
+// advanced after the final barrier.  Lane l covers channels 4l..4l+3.
+//
+// Bit-exactness: absmax is exact; the scale is an IEEE FP32 division; codes
+// use IEEE division and round-half-even conversion; the re-quantization is an
+// FP32 multiply followed by an IEEE division.  No contraction into FMA can
+// occur in these expressions (__fmul_rn / __fdiv_rn are never fused).
+#include "kernels.cuh"
+
+namespace hyb {
+
+__device__ __forceinline__ int quantize(float x, float s, int q) {
+  if (s == 0.f) return 0;
+  return clamp_code(__float2int_rn(__fdiv_rn(x, s)), q);
+}
+
+__device__ __forceinline__ int requantize(int c, float s_old, float s_new, int q) {
+  return clamp_code(__float2int_rn(__fdiv_rn(__fmul_rn(static_cast<float>(c), s_old), s_new)), q);
+}
+
+__device__ __forceinline__ int nib_get(uint32_t w, int e) {
+  const int v = (w >> (8 * (e & 3) + 4 * (e >> 2))) & 0xf;
+  return v >= 8 ? v - 16 : v;
+}
+
+__device__ __forceinline__ uint32_t nib_put(uint32_t w, int e, int c) {
+  const int sh = 8 * (e & 3) + 4 * (e >> 2);
+  return (w & ~(0xfu << sh)) | (static_cast<uint32_t>(c & 0xf) << sh);
+}
+
+// Re-quantize the codes of slots [0, first) of one tile from s_old to s_new.
+__device__ void requant_tile(uint8_t *tile, int kv, bool int4, int first, float s_old,
+                             float s_new, int q, int lane) {
+  uint32_t *w32 = reinterpret_cast<uint32_t *>(tile);
+  if (!int4 && kv == 0) {
+    // token-major rows of 128 bytes: word w holds 4 channels of slot w / 32
+    for (int w = lane; w < first * 32; w += 32) {
+      uint32_t x = w32[w], y = 0;
+      for (int e = 0; e < 4; e++) {
+        const int c = static_cast<int8_t>((x >> (8 * e)) & 0xff);
+        y |= static_cast<uint32_t>(requantize(c, s_old, s_new, q) & 0xff) << (8 * e);
+      }
+      w32[w] = y;
+    }
+  } else if (!int4) {
+    // channel-major rows of 64 bytes with swizzled 16-byte chunks
+    for (int w = lane; w < kTileBytes / 4; w += 32) {
+      const int row = w >> 4;
+      const int j = ((w >> 2) & 3) ^ ((row >> 1) & 3);
+      const int base = 16 * j + 4 * (w & 3);
+      if (base >= first) continue;
+      uint32_t x = w32[w], y = x;
+      for (int e = 0; e < 4; e++) {
+        if (base + e >= first) break;
+        const int c = static_cast<int8_t>((x >> (8 * e)) & 0xff);
+        y = (y & ~(0xffu << (8 * e))) |
+            (static_cast<uint32_t>(requantize(c, s_old, s_new, q) & 0xff) << (8 * e));
+      }
+      w32[w] = y;
+    }
+  } else if (kv == 0) {
+    // INT4 token-major rows of 64 bytes: word w holds 8 channels of slot w / 16
+    for (int w = lane; w < first * 16; w += 32) {
+      uint32_t x = w32[w], y = 0;
+      for (int e = 0; e < 8; e++) y = nib_put(y, e, requantize(nib_get(x, e), s_old, s_new, q));
+      w32[w] = y;
+    }
+  } else {
+    // INT4 channel-major rows of 32 bytes, swizzled 8-byte units of 16 slots
+    for (int w = lane; w < kTileBytes / 8; w += 32) {
+      const int row = w >> 3;
+      const int j = ((w >> 1) & 3) ^ ((row >> 2) & 3);
+      const int base = 16 * j + 8 * (w & 1);
+      if (base >= first) continue;
+      uint32_t x = w32[w], y = x;
+      for (int e = 0; e < 8; e++) {
+        if (base + e >= first) break;
+        y = nib_put(y, e, requantize(nib_get(x, e), s_old, s_new, q));
+      }
+      w32[w] = y;
+    }
+  }
+}
+
+// Four FP16 channels 4*lane..4*lane+3 of position t (K if kv == 0, else V).
+__device__ __forceinline__ void load4(const AppendArgs &a, int b, int h, int kv, int L_old, int t,
+                                      int lane, float x[4]) {
+  const __half *src;
+  if (t < L_old)
+    src = a.hot + ((((size_t)b * a.hkv + h) * kHot + (t % kHot)) * 2 + kv) * kDim;
+  else
+    src = (kv ? a.v_new : a.k_new) + (((size_t)b * a.max_new + (t - L_old)) * a.hkv + h) * kDim;
+  const uint2 raw = *reinterpret_cast<const uint2 *>(src + 4 * lane);
+  const __half2 lo = *reinterpret_cast<const __half2 *>(&raw.x);
+  const __half2 hi = *reinterpret_cast<const __half2 *>(&raw.y);
+  x[0] = __low2float(lo);
+  x[1] = __high2float(lo);
+  x[2] = __low2float(hi);
+  x[3] = __high2float(hi);
+}
+
+__global__ void __launch_bounds__(1024) append_kernel(AppendArgs a) {
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  const int L_old = a.seq_lens[b];
+  const int n = a.n_new[b];
+  if (n < 0 || n > a.max_new || L_old < 0) {
+    if (threadIdx.x == 0) set_status(a.status, HYB_STATUS_BAD_N_NEW);
+    return;
+  }
+  const long long L_new_ll = static_cast<long long>(L_old) + n;
+  if (L_new_ll - kHot > static_cast<long long>(a.max_blocks) * kBlock || L_new_ll > 0x7fffffffLL) {
+    if (threadIdx.x == 0) set_status(a.status, HYB_STATUS_CAPACITY);
+    return;
+  }
+  if (n == 0) return;
+  const int L_new = static_cast<int>(L_new_ll);
+  const int e0 = max(0, L_old - kHot), e1 = max(0, L_new - kHot);
+
+  for (int pair = warp; pair < 2 * a.hkv; pair += nwarps) {
+    const int h = pair >> 1, kv = pair & 1;
+    for (int p0 = e0; p0 < e1;) {
+      const int i = p0 / kBlock;
+      const int p1 = min((i + 1) * kBlock, e1);
+      const int first = p0 - i * kBlock;
+      const int phys = a.block_table[(size_t)b * a.max_blocks + i];
+      if (phys < 0 || phys >= a.num_phys) {
+        if (lane == 0) set_status(a.status, HYB_STATUS_BAD_BLOCK);
+        p0 = p1;
+        continue;
+      }
+      const bool int4 = a.quant_bits == 4 || (a.n_int4 != nullptr && i < a.n_int4[b]);
+      const int q = int4 ? 7 : 127;
+      // absmax over the group's tokens and channels
+      float amax = 0.f;
+      for (int t = p0; t < p1; t++) {
+        float x[4];
+        load4(a, b, h, kv, L_old, t, lane, x);
+        for (int j = 0; j < 4; j++) amax = fmaxf(amax, fabsf(x[j]));
+      }
+      for (int m = 16; m > 0; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+      const float s_c = __fdiv_rn(amax, static_cast<float>(q));
+      uint8_t *tile = a.cold + (((size_t)phys * a.hkv + h) * 2 + kv) * kTileBytes;
+      float *sp = a.scales + ((size_t)phys * a.hkv + h) * 2 + kv;
+      float s = s_c;
+      if (first != 0) {
+        const float s_old = *sp;
+        if (s_c > s_old)
+          requant_tile(tile, kv, int4, first, s_old, s_c, q, lane);
+        else
+          s = s_old;
+      }
+      __syncwarp();
+      for (int t = p0; t < p1; t++) {
+        const int slot = t - i * kBlock;
+        float x[4];
+        load4(a, b, h, kv, L_old, t, lane, x);
+        int c[4];
+        for (int j = 0; j < 4; j++) c[j] = quantize(x[j], s, q);
+        if (!int4 && kv == 0) {
+          uint32_t w = 0;
+          for (int j = 0; j < 4; j++) w |= static_cast<uint32_t>(c[j] & 0xff) << (8 * j);
+          *reinterpret_cast<uint32_t *>(tile + slot * kDim + 4 * lane) = w;
+        } else if (!int4) {
+          for (int j = 0; j < 4; j++) {
+            const int ch = 4 * lane + j;
+            tile[ch * 64 + 16 * ((slot >> 4) ^ ((ch >> 1) & 3)) + (slot & 15)] =
+                static_cast<uint8_t>(c[j]);
+          }
+        } else if (kv == 0) {
+          uint32_t nib = 0;
+          for (int j = 0; j < 4; j++) nib |= static_cast<uint32_t>(c[j] & 0xf) << (8 * j);
+          const uint32_t other = __shfl_xor_sync(0xffffffffu, nib, 1);
+          if ((lane & 1) == 0)
+            *reinterpret_cast<uint32_t *>(tile + slot * 64 + 4 * (lane >> 1)) = nib | (other << 4);
+        } else {
+          for (int j = 0; j < 4; j++) {
+            const int ch = 4 * lane + j;
+            const int unit = (slot >> 4) ^ ((ch >> 2) & 3);
+            const int in = slot & 15;
+            uint8_t *byte = tile + ch * 32 + unit * 8 + (in >> 3) * 4 + (in & 3);
+            const uint8_t old = *byte;
+            *byte = (in & 4) ? static_cast<uint8_t>((old & 0x0f) | ((c[j] & 0xf) << 4))
+                             : static_cast<uint8_t>((old & 0xf0) | (c[j] & 0xf));
+          }
+        }
+      }
+      if (lane == 0) *sp = s;
+      __syncwarp();
+      p0 = p1;
+    }
+    // newest min(n, 32) tokens into the hot ring (after their slots' old
+    // occupants were read above)
+    const int nh = min(n, kHot);
+    for (int t = L_new - nh; t < L_new; t++) {
+      const __half *src =
+          (kv ? a.v_new : a.k_new) + (((size_t)b * a.max_new + (t - L_old)) * a.hkv + h) * kDim;
+      __half *dst = a.hot + ((((size_t)b * a.hkv + h) * kHot + (t % kHot)) * 2 + kv) * kDim;
+      *reinterpret_cast<uint2 *>(dst + 4 * lane) = *reinterpret_cast<const uint2 *>(src + 4 * lane);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) a.seq_lens[b] = L_new;
+}
+
+cudaError_t launch_append(const AppendArgs &a, int batch, cudaStream_t stream) {
+  const int nwarps = min(2 * a.hkv, 32);
+  append_kernel<<<batch, 32 * nwarps, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace hyb

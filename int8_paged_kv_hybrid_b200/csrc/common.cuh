@@ -1,0 +1,101 @@
+// common.cuh -- device helpers shared by the hybrid_v2 kernels (sm_100a).
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+
+#include "hyb_kv.h"
+
+namespace hyb {
+
+constexpr int kHot = 32;          // hot-zone tokens per sequence
+constexpr int kBlock = 64;        // tokens per cold block
+constexpr int kDim = 128;         // head dimension
+constexpr int kTileBytes = kBlock * kDim;        // one K or V tile, INT8
+constexpr int kTilePairBytes = 2 * kTileBytes;   // K tile + V tile of one (block, kv head)
+constexpr int kHotTokenBytes = 2 * kDim * 2;     // K row + V row, FP16
+constexpr int kHotBytes = kHot * kHotTokenBytes; // 16 KB per (sequence, kv head)
+
+// First error wins; later errors leave the word unchanged.
+__device__ __forceinline__ void set_status(int32_t *status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---- mbarrier (CTA scope) ----
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t tx) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(
+                   smem_addr(bar)),
+               "r"(tx)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of `bar` to complete, giving up after about
+// `limit_cycles` SM clock cycles.  Returns false on timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+                                                  long long limit_cycles) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > limit_cycles) return false;
+  }
+  return true;
+}
+
+// ---- 1-D bulk copy global -> shared (TMA engine), completes on an mbarrier.
+// No cluster multicast.  dst and src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
+                                         uint64_t *bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+// L2 policy for data read once per decode step (KV tiles): evict first.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// ---- integer helpers ----
+// Sign-extend the four 4-bit values held in the low nibbles of the bytes of
+// u (high nibbles zero) to four int8 bytes.
+__device__ __forceinline__ uint32_t sext_nibbles(uint32_t u) {
+  return ((u ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+}
+
+__device__ __forceinline__ int clamp_code(int v, int q) { return v > q ? q : (v < -q ? -q : v); }
+
+}  // namespace hyb

@@ -1,0 +1,236 @@
+// hyb_host.cu -- the C ABI declared in include/hyb_kv.h: argument checks,
+// split planning, workspace sizing and kernel launches.  No memory is
+// allocated here; every buffer belongs to the caller.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "kernels.cuh"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = static_cast<int>(e);
+  return HYB_ERR_CUDA;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();  // clear the sticky-free error this query may leave
+    n = 148;             // B200
+  }
+  return n;
+}
+
+constexpr size_t kWsAlign = 256;
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace
+
+extern "C" {
+
+int hyb_version(void) { return 10000; }
+
+int hyb_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char *hyb_strerror(int code) {
+  switch (code) {
+    case HYB_OK: return "ok";
+    case HYB_ERR_INVALID_VALUE: return "invalid value (configuration, shape, null or misaligned pointer)";
+    case HYB_ERR_UNSUPPORTED: return "unsupported configuration (only hot 32 / block 64 / head_dim 128, Hq/Hkv <= 8)";
+    case HYB_ERR_WORKSPACE: return "workspace missing or too small";
+    case HYB_ERR_CUDA: return "CUDA error (see hyb_last_cuda_error)";
+    case 100 + HYB_STATUS_OK: return "device status: ok";
+    case 100 + HYB_STATUS_BAD_BLOCK: return "device status: block-table entry out of range";
+    case 100 + HYB_STATUS_BAD_N_NEW: return "device status: n_new out of range";
+    case 100 + HYB_STATUS_CAPACITY: return "device status: sequence outgrew its block table";
+    case 100 + HYB_STATUS_SEQ_LEN: return "device status: seq_lens out of range for decode";
+    case 100 + HYB_STATUS_TIMEOUT: return "device status: a bounded wait in a kernel ran out";
+    default: return "unknown code";
+  }
+}
+
+int hyb_check_desc(const hyb_cache_desc *d) {
+  if (!d) return HYB_ERR_INVALID_VALUE;
+  // hybrid_v2 contract (page sections 3.1 / 5.1)
+  const int h = d->hot_tokens;
+  if (!(h == 16 || h == 32 || h == 64 || h == 128)) return HYB_ERR_INVALID_VALUE;
+  if (d->block_size <= 0 || d->block_size % 8 != 0) return HYB_ERR_INVALID_VALUE;
+  if (d->quant_bits != 8 && d->quant_bits != 4) return HYB_ERR_INVALID_VALUE;
+  if (d->head_dim <= 0 || d->num_kv_heads <= 0 || d->num_q_heads <= 0 || d->batch <= 0 ||
+      d->num_phys_blocks < 0 || d->max_blocks_per_seq <= 0)
+    return HYB_ERR_INVALID_VALUE;
+  if (d->num_q_heads % d->num_kv_heads != 0) return HYB_ERR_INVALID_VALUE;
+  if (d->reserved != 0) return HYB_ERR_INVALID_VALUE;
+  if (!d->hot || !d->cold || !d->scales || !d->block_table || !d->seq_lens || !d->status)
+    return HYB_ERR_INVALID_VALUE;
+  if (!aligned(d->hot, 512) || !aligned(d->cold, 16) || !aligned(d->scales, 8) ||
+      !aligned(d->block_table, 4) || !aligned(d->seq_lens, 4) || !aligned(d->status, 4) ||
+      (d->n_int4_blocks && !aligned(d->n_int4_blocks, 4)))
+    return HYB_ERR_INVALID_VALUE;
+  // what this library builds
+  if (h != hyb::kHot || d->block_size != hyb::kBlock || d->head_dim != hyb::kDim)
+    return HYB_ERR_UNSUPPORTED;
+  if (d->num_q_heads / d->num_kv_heads > 8) return HYB_ERR_UNSUPPORTED;
+  return HYB_OK;
+}
+
+int hyb_kv_append(const hyb_cache_desc *d, const int32_t *n_new, int32_t max_new, const void *k_new,
+                  const void *v_new, hyb_stream_t stream) {
+  const int rc = hyb_check_desc(d);
+  if (rc != HYB_OK) return rc;
+  if (!n_new || !k_new || !v_new || max_new <= 0 || !aligned(n_new, 4) || !aligned(k_new, 16) ||
+      !aligned(v_new, 16))
+    return HYB_ERR_INVALID_VALUE;
+  hyb::AppendArgs a;
+  a.hot = static_cast<__half *>(d->hot);
+  a.cold = static_cast<uint8_t *>(d->cold);
+  a.scales = d->scales;
+  a.block_table = d->block_table;
+  a.seq_lens = d->seq_lens;
+  a.n_int4 = d->quant_bits == 8 ? d->n_int4_blocks : nullptr;
+  a.status = d->status;
+  a.n_new = n_new;
+  a.k_new = static_cast<const __half *>(k_new);
+  a.v_new = static_cast<const __half *>(v_new);
+  a.hkv = d->num_kv_heads;
+  a.num_phys = d->num_phys_blocks;
+  a.max_blocks = d->max_blocks_per_seq;
+  a.quant_bits = d->quant_bits;
+  a.max_new = max_new;
+  const cudaError_t e = hyb::launch_append(a, d->batch, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HYB_OK : cuda_fail(e);
+}
+
+int hyb_decode_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens,
+                    int32_t *split_tokens_out, int32_t *n_splits_out) {
+  const int rc = hyb_check_desc(d);
+  if (rc != HYB_OK) return rc;
+  if (max_seq_len < 0) return HYB_ERR_INVALID_VALUE;
+  const long long max_blocks_needed = (static_cast<long long>(max_seq_len) - hyb::kHot > 0)
+                                          ? (max_seq_len - hyb::kHot + hyb::kBlock - 1) / hyb::kBlock
+                                          : 0;
+  if (max_blocks_needed > d->max_blocks_per_seq) return HYB_ERR_INVALID_VALUE;
+  int tb;  // cold blocks per split
+  if (split_tokens == 0) {
+    // enough CTAs for about three per SM over the whole grid, at least two
+    // blocks per split, at most the kernel's limit
+    const long long units = static_cast<long long>(d->batch) * d->num_kv_heads;
+    const long long target = 3LL * sm_count();
+    const long long s_target = (target + units - 1) / units;
+    long long t = s_target > 0 ? (max_blocks_needed + s_target - 1) / s_target : max_blocks_needed;
+    if (t < 2) t = 2;
+    if (t > hyb::decode_max_split_blocks()) t = hyb::decode_max_split_blocks();
+    tb = static_cast<int>(t);
+  } else {
+    if (split_tokens < 0 || split_tokens % hyb::kBlock != 0) return HYB_ERR_INVALID_VALUE;
+    tb = split_tokens / hyb::kBlock;
+    if (tb < 1 || tb > hyb::decode_max_split_blocks()) return HYB_ERR_INVALID_VALUE;
+  }
+  long long ns = (max_blocks_needed + tb - 1) / tb;
+  if (ns < 1) ns = 1;
+  if (ns > 65535) return HYB_ERR_INVALID_VALUE;
+  if (split_tokens_out) *split_tokens_out = tb * hyb::kBlock;
+  if (n_splits_out) *n_splits_out = static_cast<int32_t>(ns);
+  return HYB_OK;
+}
+
+static size_t workspace_for(const hyb_cache_desc *d, int ns) {
+  if (ns <= 1) return 0;
+  const size_t rows = static_cast<size_t>(d->batch) * d->num_q_heads;
+  return round_up(rows * ns * hyb::kDim * sizeof(float), kWsAlign) +
+         round_up(rows * ns * sizeof(float), kWsAlign);
+}
+
+size_t hyb_decode_workspace_bytes(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens) {
+  int32_t st = 0, ns = 0;
+  if (hyb_decode_plan(d, max_seq_len, split_tokens, &st, &ns) != HYB_OK) return 0;
+  return workspace_for(d, ns);
+}
+
+int hyb_decode_attn(const hyb_cache_desc *d, const void *q, float softmax_scale, int32_t max_seq_len,
+                    int32_t split_tokens, void *workspace, size_t workspace_bytes, void *out,
+                    float *lse_out, hyb_stream_t stream) {
+  int32_t st = 0, ns = 0;
+  const int rc = hyb_decode_plan(d, max_seq_len, split_tokens, &st, &ns);
+  if (rc != HYB_OK) return rc;
+  if (!q || !out || !aligned(q, 16) || !aligned(out, 16) || (lse_out && !aligned(lse_out, 4)) ||
+      !std::isfinite(softmax_scale))
+    return HYB_ERR_INVALID_VALUE;
+  const size_t need = workspace_for(d, ns);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16)))
+    return HYB_ERR_WORKSPACE;
+  const size_t rows = static_cast<size_t>(d->batch) * d->num_q_heads;
+  hyb::DecodeArgs a;
+  a.hot = static_cast<const uint8_t *>(d->hot);
+  a.cold = static_cast<const uint8_t *>(d->cold);
+  a.scales = d->scales;
+  a.block_table = d->block_table;
+  a.seq_lens = d->seq_lens;
+  a.n_int4 = d->quant_bits == 8 ? d->n_int4_blocks : nullptr;
+  a.status = d->status;
+  a.q = static_cast<const __half *>(q);
+  a.out = static_cast<__half *>(out);
+  a.lse_out = lse_out;
+  a.o_part = ns > 1 ? static_cast<float *>(workspace) : nullptr;
+  a.lse_part = ns > 1 ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                                  round_up(rows * ns * hyb::kDim * sizeof(float), kWsAlign))
+                      : nullptr;
+  a.hkv = d->num_kv_heads;
+  a.hq = d->num_q_heads;
+  a.num_phys = d->num_phys_blocks;
+  a.max_blocks = d->max_blocks_per_seq;
+  a.quant_bits = d->quant_bits;
+  a.n_splits = ns;
+  a.split_blocks = st / hyb::kBlock;
+  a.max_seq_len = max_seq_len;
+  a.qk_scale = softmax_scale * 1.4426950408889634f;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = hyb::launch_decode(a, d->num_q_heads / d->num_kv_heads, d->batch, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (ns > 1) {
+    hyb::CombineArgs c{a.o_part, a.lse_part, static_cast<__half *>(out), lse_out, ns};
+    e = hyb::launch_combine(c, static_cast<int>(rows), s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return HYB_OK;
+}
+
+int hyb_combine(int32_t batch, int32_t num_q_heads, int32_t head_dim, int32_t n_splits,
+                const float *o_partial, const float *lse_partial, void *out, float *lse_out,
+                hyb_stream_t stream) {
+  if (batch <= 0 || num_q_heads <= 0 || n_splits < 1 || !o_partial || !lse_partial || !out ||
+      !aligned(o_partial, 16) || !aligned(lse_partial, 4) || !aligned(out, 16) ||
+      (lse_out && !aligned(lse_out, 4)))
+    return HYB_ERR_INVALID_VALUE;
+  if (head_dim != hyb::kDim) return HYB_ERR_UNSUPPORTED;
+  const long long rows = static_cast<long long>(batch) * num_q_heads;
+  if (rows > 0x7fffffffLL) return HYB_ERR_INVALID_VALUE;
+  hyb::CombineArgs c{o_partial, lse_partial, static_cast<__half *>(out), lse_out, n_splits};
+  const cudaError_t e = hyb::launch_combine(c, static_cast<int>(rows), reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HYB_OK : cuda_fail(e);
+}
+
+int hyb_read_status(const hyb_cache_desc *d, int32_t *host_status, int32_t clear, hyb_stream_t stream) {
+  if (!d || !d->status || !host_status) return HYB_ERR_INVALID_VALUE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(host_status, d->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess && clear) {
+    e = cudaMemsetAsync(d->status, 0, sizeof(int32_t), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  }
+  return e == cudaSuccess ? HYB_OK : cuda_fail(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,55 @@
+// kernels.cuh -- argument blocks and launchers of the hybrid_v2 kernels
+// (shared by the kernels and the C-ABI layer).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace hyb {
+
+struct AppendArgs {
+  __half *hot;                // FP16 [batch][Hkv][32][2][128]
+  uint8_t *cold;              // [num_phys][Hkv][2][8192]
+  float *scales;              // [num_phys][Hkv][2]
+  const int32_t *block_table; // [batch][max_blocks]
+  int32_t *seq_lens;          // [batch]
+  const int32_t *n_int4;      // [batch] or null
+  int32_t *status;
+  const int32_t *n_new;       // [batch]
+  const __half *k_new;        // FP16 [batch][max_new][Hkv][128]
+  const __half *v_new;
+  int hkv, num_phys, max_blocks, quant_bits, max_new;
+};
+
+struct DecodeArgs {
+  const uint8_t *hot;
+  const uint8_t *cold;
+  const float *scales;
+  const int32_t *block_table;
+  const int32_t *seq_lens;
+  const int32_t *n_int4;
+  int32_t *status;
+  const __half *q;            // FP16 [batch][Hq][128]
+  __half *out;                // FP16 [batch][Hq][128]
+  float *lse_out;             // [batch][Hq] or null
+  float *o_part;              // [batch][Hq][n_splits][128] (n_splits > 1)
+  float *lse_part;            // [batch][Hq][n_splits]
+  int hkv, hq, num_phys, max_blocks, quant_bits, n_splits, split_blocks, max_seq_len;
+  float qk_scale;             // softmax_scale * log2(e)
+};
+
+struct CombineArgs {
+  const float *o_part;        // [rows][n_splits][128]
+  const float *lse_part;      // [rows][n_splits]
+  __half *out;                // [rows][128]
+  float *lse_out;             // [rows] or null
+  int n_splits;
+};
+
+cudaError_t launch_append(const AppendArgs &a, int batch, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, cudaStream_t stream);
+cudaError_t launch_combine(const CombineArgs &a, int rows, cudaStream_t stream);
+int decode_max_split_blocks();
+
+}  // namespace hyb

@@ -174,17 +174,23 @@ def step_tokens(w: Workload, step: int, n_new: np.ndarray, max_new: Optional[int
     """FP16 K and V for append call `step`: [batch][max_new][hkv][d] each.
     Rows beyond n_new[b] are zero (never read)."""
     mx = w.max_new if max_new is None else max_new
+    n_new = np.asarray(n_new, np.int64)
     rng = np.random.default_rng([w.seed, 1, step])
-    shape = (w.batch, mx, w.num_kv_heads, w.head_dim)
-    k = rng.standard_normal(shape, dtype=np.float32)
-    v = rng.standard_normal(shape, dtype=np.float32)
+    rows = (w.num_kv_heads, w.head_dim)
+    total = int(n_new.sum())
+    kd = rng.standard_normal((total,) + rows, dtype=np.float32)
+    vd = rng.standard_normal((total,) + rows, dtype=np.float32)
     if w.outlier_channels is not None:
         for h in range(w.num_kv_heads):
-            k[:, :, h, w.outlier_channels[h]] *= 10.0
-    mask = np.arange(mx)[None, :] < np.asarray(n_new)[:, None]
-    k *= mask[:, :, None, None]
-    v *= mask[:, :, None, None]
-    return k.astype(np.float16), v.astype(np.float16)
+            kd[:, h, w.outlier_channels[h]] *= 10.0
+    k = np.zeros((w.batch, mx) + rows, np.float16)
+    v = np.zeros((w.batch, mx) + rows, np.float16)
+    o = 0
+    for b, n in enumerate(n_new):
+        k[b, :n] = kd[o:o + n]
+        v[b, :n] = vd[o:o + n]
+        o += n
+    return k, v
 
 
 def query(w: Workload, step: int = 0) -> np.ndarray:
@@ -219,3 +225,36 @@ def kv_bytes(w: Workload, lens: Optional[np.ndarray] = None) -> int:
         total += nblk * 4                          # block table entries
     total += w.batch * w.num_q_heads * d * 2 * 2   # q in, out
     return total
+
+
+def custom_workload(name, lens, num_q_heads, num_kv_heads, seed, softmax_scale=None,
+                    schedule="random", chunk=64, max_step=64, pool_extra=3, n_int4=None,
+                    outliers=False, split_tokens=0) -> Workload:
+    """A small workload with the given final lengths (for parity tests).
+    schedule: "random" (U[1, max_step] tokens per call), "chunk" (prefill in
+    `chunk`-token calls then one 1-token call) or "one" (a single call)."""
+    rng = np.random.default_rng([seed, 0])
+    lens = np.asarray(lens, np.int64)
+    B = len(lens)
+    nblk = np.array([cold_blocks_for(int(L)) for L in lens])
+    pool = int(nblk.sum()) + pool_extra
+    bt = _block_table(rng, nblk, pool)
+    if schedule == "random":
+        sched = _random_step_schedule(rng, lens, 1, max_step)
+        mx = max_step
+    elif schedule == "chunk":
+        sched = _chunk_schedule(lens, chunk)
+        mx = chunk
+    else:
+        sched = [lens.astype(np.int32)]
+        mx = max(1, int(lens.max()))
+    outl = None
+    if outliers:
+        outl = np.stack([rng.choice(HEAD_DIM, 4, replace=False) for _ in range(num_kv_heads)])
+    sm = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(HEAD_DIM)
+    return Workload(name=name, batch=B, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads,
+                    lens=lens.astype(np.int32), softmax_scale=sm, q_std=1.0,
+                    num_phys_blocks=pool, block_table=bt,
+                    n_int4=None if n_int4 is None else np.asarray(n_int4, np.int32),
+                    schedule=sched, max_new=mx, seed=seed, outlier_channels=outl,
+                    split_tokens=split_tokens)

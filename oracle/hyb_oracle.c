@@ -62,7 +62,17 @@ double ora_half_to_double(uint16_t h) {
   return sign ? -v : v;
 }
 
-static float half_to_float(uint16_t h) { return (float)ora_half_to_double(h); }
+/* All 65536 binary16 values as float, filled from the definition above. */
+static float half_table[65536];
+static int half_table_ready = 0;
+
+static void build_half_table(void) {
+  if (half_table_ready) return;
+  for (int i = 0; i < 65536; i++) half_table[i] = (float)ora_half_to_double((uint16_t)i);
+  half_table_ready = 1;
+}
+
+static float half_to_float(uint16_t h) { return half_table[h]; }
 
 /* ------------------------------------------------------------------ */
 /* Cache state, kept in LOGICAL form: per sequence, per logical block. */
@@ -85,6 +95,7 @@ ora_cache *ora_new(int batch, int hkv, int hq, int d, int hot, int block,
   if (batch <= 0 || hkv <= 0 || hq <= 0 || hq % hkv || d <= 0 || hot <= 0 ||
       block <= 0 || max_blocks < 0 || (quant_bits != 8 && quant_bits != 4))
     return NULL;
+  build_half_table();
   ora_cache *c = (ora_cache *)calloc(1, sizeof(ora_cache));
   if (!c) return NULL;
   c->batch = batch; c->hkv = hkv; c->hq = hq; c->d = d; c->hot = hot;
@@ -231,7 +242,7 @@ static double kv_value(const ora_cache *c, int b, int h, int kv, int p, int ch) 
   const int L = c->len[b];
   const int cold = L > c->hot ? L - c->hot : 0;
   if (p >= cold)
-    return ora_half_to_double(
+    return (double)half_to_float(
         c->ring[((((size_t)b * c->hkv + h) * c->hot + p % c->hot) * 2 + kv) * c->d + ch]);
   const int i = p / c->block;
   const size_t bi = (size_t)b * c->max_blocks + i;
@@ -270,7 +281,7 @@ int ora_decode(const ora_cache *c, const uint16_t *q, double softmax_scale,
     for (int j = 0; j < L; j++) {
       double acc = 0.0;
       for (int ch = 0; ch < d; ch++)
-        acc += ora_half_to_double(qh[ch]) * kv_value(c, b, hk, 0, j, ch);
+        acc += (double)half_to_float(qh[ch]) * kv_value(c, b, hk, 0, j, ch);
       z[j] = softmax_scale * acc;
       if (z[j] > m) m = z[j];
     }

@@ -1,0 +1,133 @@
+"""Host-side checks of the C ABI (no GPU): exported symbols, the hybrid_v2
+configuration contract, split planning and workspace sizing."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import int8_paged_kv_hybrid_b200 as hk
+from int8_paged_kv_hybrid_b200 import _lib, synth
+from golden_cases import GOLDEN
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn), encoding="utf-8").read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"^[A-Za-z_][\w \*]*?\b(hyb_\w+)\s*\(", text, flags=re.M))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = hk.load()
+    declared = _declared_functions()
+    assert {"hyb_kv_append", "hyb_decode_attn", "hyb_combine"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(_lib.EXPORTED) <= declared
+
+
+def _desc(hot=32, block=64, qbits=8, d=128, hkv=8, hq=32, batch=2, phys=16, maxb=4):
+    x = _lib.CacheDesc()
+    x.hot_tokens, x.block_size, x.head_dim, x.quant_bits = hot, block, d, qbits
+    x.num_kv_heads, x.num_q_heads, x.num_phys_blocks = hkv, hq, phys
+    x.max_blocks_per_seq, x.batch, x.reserved = maxb, batch, 0
+    base = 0x7f0000000000
+    x.hot, x.cold, x.scales = base, base + 0x100000, base + 0x200000
+    x.block_table, x.seq_lens, x.status = base + 0x300000, base + 0x310000, base + 0x320000
+    x.n_int4_blocks = None
+    return x
+
+
+def test_config_contract_golden():
+    """hot_tokens / block_size / quantization_bits per the page (sections 3.1, 5.1)."""
+    codes = {"ok": 0, "invalid": _lib.HYB_ERR_INVALID_VALUE, "unsupported": _lib.HYB_ERR_UNSUPPORTED}
+    n = 0
+    for line in open(os.path.join(GOLDEN, "config_contract.txt"), encoding="utf-8"):
+        f = line.split("#", 1)[0].split()
+        if not f:
+            continue
+        hot, block, qbits, want = int(f[0]), int(f[1]), int(f[2]), f[3]
+        assert hk.hyb_check_desc(_desc(hot=hot, block=block, qbits=qbits)) == codes[want], f
+        n += 1
+    assert n >= 10
+
+
+def test_descriptor_rejections():
+    ok = _desc()
+    assert hk.hyb_check_desc(ok) == 0
+    for field, val, want in [
+        ("head_dim", 64, _lib.HYB_ERR_UNSUPPORTED),
+        ("num_q_heads", 30, _lib.HYB_ERR_INVALID_VALUE),    # not a multiple of Hkv
+        ("num_q_heads", 72, _lib.HYB_ERR_UNSUPPORTED),      # group of 9
+        ("batch", 0, _lib.HYB_ERR_INVALID_VALUE),
+        ("max_blocks_per_seq", 0, _lib.HYB_ERR_INVALID_VALUE),
+        ("reserved", 1, _lib.HYB_ERR_INVALID_VALUE),
+        ("hot", 0x7f0000000100, _lib.HYB_ERR_INVALID_VALUE),  # hot zone not 512-byte aligned
+        ("cold", 0x7f0000100008, _lib.HYB_ERR_INVALID_VALUE),
+        ("status", None, _lib.HYB_ERR_INVALID_VALUE),
+    ]:
+        d = _desc()
+        setattr(d, field, val)
+        assert hk.hyb_check_desc(d) == want, (field, val)
+    assert hk.load().hyb_check_desc(None) == _lib.HYB_ERR_INVALID_VALUE
+
+
+def test_plan_and_workspace():
+    d = _desc(batch=4, maxb=2048, phys=8192)
+    st, ns = hk.hyb_decode_plan(d, 131072, 512)
+    assert st == 512 and ns == 256      # ceil((131072 - 32) / 512)
+    st, ns = hk.hyb_decode_plan(d, 32768, 512)
+    assert ns == 64                     # the page's 32K context: >= 64 splits at 512 tokens
+    st, ns = hk.hyb_decode_plan(d, 32, 512)
+    assert ns == 1 and hk.hyb_decode_workspace_bytes(d, 32, 512) == 0
+    ws = hk.hyb_decode_workspace_bytes(d, 131072, 512)
+    rows = 4 * 32
+    assert ws >= rows * 256 * 128 * 4 + rows * 256 * 4
+    for bad in (100, -64, 64 * 129):
+        with pytest.raises(hk.HybError):
+            hk.hyb_decode_plan(d, 4096, bad)
+    with pytest.raises(hk.HybError):
+        hk.hyb_decode_plan(d, 64 * 2048 + 33, 0)  # longer than the block table allows
+    # automatic splits: a multiple of 64 tokens, at least two blocks
+    for L in (33, 1000, 2048, 131072):
+        st, ns = hk.hyb_decode_plan(d, L, 0)
+        assert st % 64 == 0 and st >= 128 and ns >= 1
+        assert ns == max(1, -(-max(0, L - 32) // st))
+
+
+def test_strerror_covers_codes():
+    for c in (0, -1, -2, -3, -4, 100, 101, 102, 103, 104, 105):
+        assert hk.strerror(c) and hk.strerror(c) != "unknown code"
+    assert hk.strerror(12345) == "unknown code"
+
+
+def test_kv_bytes_formula():
+    """Algorithmic bytes of config 2: 8 x 8 heads x (2016 cold tokens x 256 B +
+    32 hot x 512 B + 32 blocks x 8 B) + 8 x 32 block-table entries x 4 B +
+    q and out (8 x 32 x 128 x 2 B each)."""
+    w = synth.make_workload(2)
+    want = 8 * 8 * (2016 * 256 + 32 * 512 + 32 * 8) + 8 * 32 * 4 + 2 * 8 * 32 * 128 * 2
+    assert synth.kv_bytes(w) == want
+    assert abs(want / 1e6 - 34.2) < 0.5   # "34.2 MB"
+
+
+def test_workload_shapes():
+    w = synth.make_workload(4)
+    assert list(w.lens) == [32768, 32768, 131072, 131072] and w.split_tokens == 512
+    w5 = synth.make_workload(5)
+    assert w5.num_q_heads == 28 and w5.num_kv_heads == 4 and w5.batch == 128
+    nb = w5.cold_blocks()
+    assert np.array_equal(w5.n_int4, nb // 4)
+    w3 = synth.make_workload(3)
+    assert w3.lens.min() >= 256 and w3.lens.max() <= 8192 and w3.outlier_channels.shape == (8, 4)
+    for w in (synth.make_workload(i) for i in (1, 2, 3, 4, 5)):
+        used = w.block_table[w.block_table >= 0]
+        assert len(np.unique(used)) == len(used) and used.max() < w.num_phys_blocks
+        assert sum(int(s.sum()) for s in w.schedule) == int(w.lens.sum())

@@ -1,0 +1,113 @@
+"""hyb_decode_attn (+ hyb_combine) on the GPU against the FP64 oracle:
+max-abs <= 2e-3 and per-row relative L2 <= 1e-3 on the same cache contents.
+Small cases span several splits, ragged tails, empty and all-hot sequences;
+the five measured workloads run at full size with sampled rows."""
+import numpy as np
+import pytest
+
+from harness import assert_cache_equal, assert_decode_close, decode_both, errors, make_pair, replay
+from int8_paged_kv_hybrid_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+SMALL_LENS = [0, 1, 5, 31, 32, 33, 64, 95, 96, 97, 130, 255, 1000, 2047, 3001]
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 4), (32, 8), (28, 4), (16, 2)])
+@pytest.mark.parametrize("split", [0, 64, 192])
+def test_small_parity(hq, hkv, split):
+    w = synth.custom_workload("small", SMALL_LENS, hq, hkv, seed=hq * 31 + hkv, max_step=64)
+    cache, ora = make_pair(w)
+    replay(w, cache, ora)
+    got, lse, ref, ref_lse = decode_both(w, cache, ora, split_tokens=split)
+    assert_decode_close(w, got, lse, ref, ref_lse, what="G=%d split=%d" % (hq // hkv, split))
+    assert cache.status() == 0
+
+
+@pytest.mark.parametrize("qbits,int4", [(4, False), (8, True)])
+def test_int4_parity(qbits, int4):
+    lens = [40, 200, 777, 2100]
+    nb = [synth.cold_blocks_for(L) for L in lens]
+    w = synth.custom_workload("int4", lens, 28, 4, seed=3 + qbits, schedule="chunk",
+                              n_int4=[n // 4 for n in nb] if int4 else None)
+    cache, ora = make_pair(w, quant_bits=qbits)
+    replay(w, cache, ora)
+    assert_cache_equal(w, cache, ora)
+    for split in (0, 128):
+        got, lse, ref, ref_lse = decode_both(w, cache, ora, split_tokens=split)
+        assert_decode_close(w, got, lse, ref, ref_lse, what="int4 split=%d" % split)
+
+
+def test_softmax_scale_one_with_scaled_q():
+    """Config-2 convention: q ~ N(0,1)/sqrt(d) and softmax_scale = 1."""
+    w = synth.custom_workload("s1", [300, 2048], 32, 8, seed=9, softmax_scale=1.0, schedule="chunk")
+    w.q_std = 1.0 / np.sqrt(128)
+    cache, ora = make_pair(w)
+    replay(w, cache, ora)
+    got, lse, ref, ref_lse = decode_both(w, cache, ora)
+    assert_decode_close(w, got, lse, ref, ref_lse, what="scale 1")
+
+
+def test_split_invariance():
+    """One split per sequence vs 64-token splits: same result within FP32 merges."""
+    w = synth.custom_workload("inv", [5000, 700, 33], 32, 8, seed=21)
+    cache, ora = make_pair(w)
+    replay(w, cache, ora)
+    import torch
+    q = torch.from_numpy(synth.query(w)).cuda()
+    a = cache.decode(q, w.softmax_scale, 5000, 64 * 79).float()
+    b = cache.decode(q, w.softmax_scale, 5000, 64).float()
+    torch.cuda.synchronize()
+    assert float((a - b).abs().max()) <= 1e-3
+
+
+def test_peaked_attention():
+    """Large logits (q scaled x8): the softmax is nearly one-hot; the 16-bit
+    weights keep their relative precision per 16-token group."""
+    w = synth.custom_workload("peak", [1500, 90], 8, 2, seed=4)
+    cache, ora = make_pair(w)
+    replay(w, cache, ora)
+    q = (synth.query(w).astype(np.float32) * 8).astype(np.float16)
+    got, lse, ref, ref_lse = decode_both(w, cache, ora, q=q)
+    assert_decode_close(w, got, lse, ref, ref_lse, what="peaked")
+
+
+def test_seq_len_beyond_bound_sets_status():
+    import torch
+    from int8_paged_kv_hybrid_b200 import _lib
+    w = synth.custom_workload("bound", [100, 300], 8, 8, seed=2)
+    cache, ora = make_pair(w)
+    replay(w, cache, ora)
+    q = torch.from_numpy(synth.query(w)).cuda()
+    out = cache.decode(q, w.softmax_scale, 200, 64)     # sequence 1 is longer than 200
+    torch.cuda.synchronize()
+    assert cache.status(clear=True) == _lib.HYB_STATUS_SEQ_LEN
+    ref, _ = ora.decode(synth.query(w), w.softmax_scale)
+    assert errors(out.float().cpu().numpy()[:1], ref[:1])[0] <= 2e-3   # sequence 0 unaffected
+    assert float(out[1].float().abs().max()) == 0.0                    # sequence 1 skipped
+
+
+def _sample_pairs(w, n, seed):
+    rng = np.random.default_rng(seed)
+    pairs = {(int(b), int(h)) for b, h in zip(rng.integers(0, w.batch, n), rng.integers(0, w.num_q_heads, n))}
+    # always include the longest and the shortest sequence
+    for b in (int(np.argmax(w.lens)), int(np.argmin(w.lens))):
+        pairs.add((b, 0))
+        pairs.add((b, w.num_q_heads - 1))
+    return sorted(pairs)
+
+
+@pytest.mark.parametrize("idx", [1, 2, 3, 4, 5])
+def test_workload_full_size(idx):
+    """The measured workloads at full size, in the launch configuration the
+    benchmark uses (automatic splits, or 512-token splits for the long-context
+    workload): appends bit-exact over the whole pool, attention on sampled rows
+    (all rows for workloads 1 and 2)."""
+    w = synth.make_workload(idx)
+    cache, ora = make_pair(w)
+    replay(w, cache, ora)
+    assert_cache_equal(w, cache, ora, w.name)
+    pairs = None if idx in (1, 2) else _sample_pairs(w, 24, idx)
+    got, lse, ref, ref_lse = decode_both(w, cache, ora, pairs=pairs)
+    mabs, rel = assert_decode_close(w, got, lse, ref, ref_lse, pairs=pairs, what=w.name)
+    print("%s: max-abs %.3g rel-L2 %.3g" % (w.name, mabs, rel))
