@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Benchmark of the hybrid_v2 decode path on B200.
+
+One step = one pass of the whole hot path over one batch: hyb_kv_append of
+the step's token (hot-ring write + sealing of the token that leaves the hot
+zone, with quantization) followed by hyb_decode_attn (split-KV attention over
+the hot ring and the INT8 cold blocks, with the log-sum-exp merge of its
+splits).  Workload: Llama-3-8B attention shapes, one layer, batch 8, Hq 32,
+Hkv 8, d 128, every sequence 2048 tokens (32 FP16 hot + 2016 INT8 cold in a
+4096-block pool), seeded synthetic N(0,1) data.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Prints one JSON line (rank 0).  With N > 1 (torchrun), every rank runs its
+own batch (weak scaling, no data-path collective); times are the max over
+ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn KV GB/s (frac of HBM peak) and tokens/s at 1 B200 vs CPU oracle"
+UNIT = "GB/s"
+WORKLOAD = 2
+PROFILE = os.path.join(ROOT, "profiles", "decode_splitkv_llama8b_b8_L2048.md")
+KERNEL_SOURCES = ["decode.cu", "common.cuh", "kernels.cuh"]
+FLUSH_BYTES = 512 << 20   # > 126 MB L2
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=400)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="native", choices=["native", "reference"])
+    p.add_argument("--split", type=int, default=0, help="split_tokens (0 = automatic)")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--lean", action="store_true",
+                   help="profiling run: no state restore, L2 flush, e2e or CPU baseline")
+    return p.parse_args()
+
+
+def workload_config(w, split, ns):
+    return {"workload": "llama3-8b decode attention, 1 layer: batch %d, Hq %d, Hkv %d, d 128, "
+                        "L %d (32 FP16 hot + %d INT8 cold in 64-token blocks), %d-block pool"
+                        % (w.batch, w.num_q_heads, w.num_kv_heads, int(w.lens[0]),
+                           int(w.lens[0]) - 32, w.num_phys_blocks),
+            "batch": int(w.batch), "seq_len": int(w.lens[0]), "num_q_heads": w.num_q_heads,
+            "num_kv_heads": w.num_kv_heads, "head_dim": 128, "hot_tokens": 32, "block_size": 64,
+            "quant_bits": 8, "split_tokens": split, "n_splits": ns,
+            "step": "hyb_kv_append (1 token/seq) + hyb_decode_attn",
+            "l2": "flushed between timed steps (512 MB write)",
+            "parallelism": "replicas (independent batch per GPU)"}
+
+
+def kernel_sha():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "int8_paged_kv_hybrid_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel source."""
+    try:
+        text = open(PROFILE, encoding="utf-8").read()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha") != kernel_sha():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 10 ms; stop() summarises
+    the samples taken after mark() (the timed region)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.t_mark = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), "--query-gpu=timestamp," + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "10"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def mark(self):
+        self.t_mark = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        t_stop = time.time()
+        time.sleep(0.05)
+        self.proc.terminate()
+        try:
+            text, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        import datetime
+        rows = []
+        for line in text.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(f[2]), float(f[3]), [x.lower() == "active" for x in f[6:10]]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        # samples taken from the start of the timed region on (nvidia-smi's
+        # timestamps are wall-clock local time, as datetime parses them)
+        t0 = self.t_mark or 0.0
+        timed = [r for r in rows if t0 <= r[0] <= t_stop] or rows[-3:]
+        sm = sorted(r[1] for r in timed)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in timed for i in range(4) if r[3][i]})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": rows[0][2], "reasons": reasons,
+                "samples_timed": len(timed), "samples": len(rows)}
+
+
+def build_gpu_state(w, torch):
+    from int8_paged_kv_hybrid_b200 import HybridKVCache, synth
+    cache = HybridKVCache(w.batch, w.num_kv_heads, w.num_q_heads, w.num_phys_blocks, w.max_blocks,
+                          block_table=w.block_table, n_int4=w.n_int4)
+    for si, n in enumerate(w.schedule[:-1]):
+        k, v = synth.step_tokens(w, si, n)
+        cache.append(torch.from_numpy(n).cuda(), torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
+    last = len(w.schedule) - 1
+    n_last = w.schedule[-1]
+    k_last, v_last = synth.step_tokens(w, last, n_last, max_new=int(n_last.max()))
+    q = synth.query(w)
+    torch.cuda.synchronize()
+    return cache, n_last, k_last, v_last, q
+
+
+def _touched_blocks(w, n_last):
+    """Physical blocks the step's append can write (the blocks holding the
+    positions that leave the hot zone)."""
+    import numpy as np
+    phys = []
+    for b in range(w.batch):
+        L_new = int(w.lens[b])
+        L_old = L_new - int(n_last[b])
+        e0, e1 = max(0, L_old - 32), max(0, L_new - 32)
+        for i in range(e0 // 64, (e1 + 63) // 64):
+            if e1 > e0:
+                phys.append(int(w.block_table[b, i]))
+    return np.array(sorted(set(phys)), np.int64)
+
+
+def run_native(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from int8_paged_kv_hybrid_b200 import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    clocks = ClockSampler(local_rank) if rank == 0 and not args.lean else None
+    w = synth.make_workload(WORKLOAD, seed_offset=1000 * rank)
+    L = int(w.lens.max())
+    cache, n_last, k_last, v_last, q = build_gpu_state(w, torch)
+    if args.lean:
+        L += args.warmup + args.steps  # the lean run lets the cache grow one token per step
+    split, ns = cache.plan(L, args.split)
+    n_d = torch.from_numpy(n_last).to(dev)
+    k_d = torch.from_numpy(k_last).to(dev)
+    v_d = torch.from_numpy(v_last).to(dev)
+    q_d = torch.from_numpy(q).to(dev)
+    out = torch.empty((w.batch, w.num_q_heads, 128), dtype=torch.float16, device=dev)
+    lse = torch.empty((w.batch, w.num_q_heads), dtype=torch.float32, device=dev)
+    ws = cache.workspace(L, split)
+
+    # state the step changes, restored before every step (untimed)
+    touched = torch.from_numpy(_touched_blocks(w, n_last)).to(dev)
+    snap = None
+    if not args.lean:
+        snap = {"hot": cache.hot.clone(), "scales": cache.scales.clone(),
+                "seq_lens": cache.seq_lens.clone(), "cold": cache.cold.index_select(0, touched)}
+    flush = torch.empty(0 if args.lean else FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def restore():
+        if snap is None:
+            return
+        cache.hot.copy_(snap["hot"])
+        cache.scales.copy_(snap["scales"])
+        cache.seq_lens.copy_(snap["seq_lens"])
+        cache.cold.index_copy_(0, touched, snap["cold"])
+
+    # one eager run (sets kernel attributes, checks the path), then capture the
+    # append and the decode as two CUDA graphs on a side stream
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        restore()
+        cache.append(n_d, k_d, v_d)
+        cache.decode(q_d, w.softmax_scale, L, split, out=out, lse=lse, workspace=ws)
+        restore()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g_app, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_app, stream=side):
+        cache.append(n_d, k_d, v_d)
+    with torch.cuda.graph(g_dec, stream=side):
+        cache.decode(q_d, w.softmax_scale, L, split, out=out, lse=lse, workspace=ws)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def timed_steps(n):
+        evs = []
+        for _ in range(n):
+            restore()
+            flush.zero_()
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0.record(stream)
+            g_app.replay()
+            e1.record(stream)
+            g_dec.replay()
+            e2.record(stream)
+            evs.append((e0, e1, e2))
+        return evs
+
+    timed_steps(args.warmup)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.mark()
+    evs = timed_steps(args.steps)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop() if clocks else None
+    ms_step = sum(a.elapsed_time(c) for a, b, c in evs) / len(evs)
+    ms_dec = sum(b.elapsed_time(c) for a, b, c in evs) / len(evs)
+    ms_app = sum(a.elapsed_time(b) for a, b, c in evs) / len(evs)
+    if world > 1:
+        t = torch.tensor([ms_step, ms_dec, ms_app], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, ms_dec, ms_app = t.tolist()
+    assert torch.isfinite(out.float()).all() and cache.status() == 0
+    if args.lean:
+        return {"lean": True, "ms_per_step": ms_step, "ms_decode": ms_dec, "ms_append": ms_app}, w
+
+    # end to end with host buffers: pinned H2D of the step's inputs, the two
+    # library calls, D2H of the output -- all inside the timed span
+    h_n = torch.from_numpy(n_last).pin_memory()
+    h_k = torch.from_numpy(k_last).pin_memory()
+    h_v = torch.from_numpy(v_last).pin_memory()
+    h_q = torch.from_numpy(q).pin_memory()
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_n, h_k, h_v, h_q))
+    d2h = h_out.numel() * h_out.element_size()
+    e2e = []
+    for i in range(args.warmup + args.steps):
+        restore()
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        n_d.copy_(h_n, non_blocking=True)
+        k_d.copy_(h_k, non_blocking=True)
+        v_d.copy_(h_v, non_blocking=True)
+        q_d.copy_(h_q, non_blocking=True)
+        g_app.replay()
+        g_dec.replay()
+        h_out.copy_(out, non_blocking=True)
+        e1.record(stream)
+        if i >= args.warmup:
+            e2e.append((e0, e1))
+    torch.cuda.synchronize()
+    ms_e2e = sum(a.elapsed_time(b) for a, b in e2e) / len(e2e)
+    if world > 1:
+        t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = t.item()
+    del g_app, g_dec
+
+    kvb = synth.kv_bytes(w)
+    peak, peak_kind = measured_peaks()
+    total_bytes = kvb * world
+    value = total_bytes / (ms_step * 1e-3) / 1e9
+    tokens_s = w.batch * world / (ms_step * 1e-3)
+    achieved = kvb / (ms_dec * 1e-3) / 1e9
+    res = None
+    if rank == 0:
+        res = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+            "data": "synthetic (seeded N(0,1) FP16 K/V/q; caches built by the library's own appends)",
+            "config": workload_config(w, split, ns),
+            "tokens_per_s": round(tokens_s, 1),
+            "tokens_per_s_model_equiv": round(tokens_s / 32, 1),
+            "kv_bytes_per_step": kvb,
+            "frac_of_hbm_peak_step": round(value / world / peak, 4),
+            "ms_decode": round(ms_dec, 5), "ms_append": round(ms_app, 5),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": profiled_traffic(),
+                         "kernel": "hyb::decode_kernel<4>", "peak_kind": peak_kind,
+                         "achieved_bytes": "algorithmic KV bytes per launch (%d)" % kvb},
+            "e2e": {"value": round(total_bytes / (ms_e2e * 1e-3) / 1e9, 1), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(ms_e2e, 5)},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clk,
+        }
+    return res, w
+
+
+def oracle_step_rate(w, steps, warmup, budget_s=None):
+    """Time the CPU oracle (as it stands) on the same workload: per step the
+    1-token append plus FP64 attention of every (sequence, head).  The state
+    grows by one token per step (bounded sample)."""
+    import numpy as np
+    import oracle
+    from int8_paged_kv_hybrid_b200 import synth
+    threads = os.cpu_count() or 1
+    ora = oracle.OracleCache(w.batch, w.num_kv_heads, w.num_q_heads, w.max_blocks + 16)
+    for si, n in enumerate(w.schedule[:-1]):
+        k, v = synth.step_tokens(w, si, n)
+        ora.append(n, k, v)
+    last = len(w.schedule) - 1
+    n_last = w.schedule[-1]
+    k_last, v_last = synth.step_tokens(w, last, n_last, max_new=int(n_last.max()))
+    q = synth.query(w)
+    times = []
+    for i in range(warmup + steps):
+        t0 = time.perf_counter()
+        ora.append(n_last, k_last, v_last)
+        ora.decode(q, w.softmax_scale, nthreads=threads)
+        t1 = time.perf_counter()
+        if i >= warmup:
+            times.append(t1 - t0)
+        if budget_s is not None and sum(times) > budget_s and len(times) >= 1:
+            break
+    return sum(times) / len(times), len(times), threads
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and world == 1 and args.gpus > 1:
+        print(json.dumps({"error": "run N > 1 under torchrun"}))
+        return 2
+    from int8_paged_kv_hybrid_b200 import synth
+
+    if args.impl == "reference":
+        # the CPU oracle on the host cores: rank 0 alone
+        if rank != 0:
+            return 0
+        w = synth.make_workload(WORKLOAD)
+        sec, n, threads = oracle_step_rate(w, args.steps, args.warmup, budget_s=150.0)
+        kvb = synth.kv_bytes(w)
+        val = kvb / sec / 1e9
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": UNIT, "n_gpus": world,
+            "steps": n, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w, 0, 0),
+            "tokens_per_s": round(w.batch / sec, 3),
+            "cpu_baseline": {"value": round(val, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": "%d full steps of the workload (append 1 token/seq + FP64 attention "
+                                       "of all 256 rows), state growing 1 token per step" % n},
+            "e2e": {"value": round(val, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
+        return 0
+
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local_rank))
+    res, w = run_native(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.lean:
+        sec, n, threads = oracle_step_rate(w, 3, 0, budget_s=30.0)
+        res["cpu_baseline"] = {"value": round(synth.kv_bytes(w) / sec / 1e9, 4), "unit": UNIT,
+                               "cores": threads, "kind": "oracle",
+                               "sample": "%d full steps of the same workload (1-token append + FP64 "
+                                         "attention of all rows) on the host, OpenMP over rows" % n}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -189,8 +189,10 @@ int hyb_kv_append(const hyb_cache_desc *desc, const int32_t *n_new, int32_t max_
 int hyb_decode_plan(const hyb_cache_desc *desc, int32_t max_seq_len, int32_t split_tokens,
                     int32_t *split_tokens_out, int32_t *n_splits_out);
 
-/* Bytes of workspace hyb_decode_attn needs for these arguments (0 when a
- * single split suffices), or 0 with an invalid descriptor. */
+/* Bytes of workspace hyb_decode_attn needs for these arguments, or 0 with an
+ * invalid descriptor.  It is 0 when each sequence takes at most 8 splits:
+ * the splits of a (sequence, kv head) then run as one thread-block cluster
+ * and are merged through distributed shared memory. */
 size_t hyb_decode_workspace_bytes(const hyb_cache_desc *desc, int32_t max_seq_len,
                                   int32_t split_tokens);
 
@@ -207,10 +209,18 @@ size_t hyb_decode_workspace_bytes(const hyb_cache_desc *desc, int32_t max_seq_le
  *   split_tokens   multiple of 64, or 0 = automatic (hyb_decode_plan).
  *   workspace, workspace_bytes  device scratch of at least
  *            hyb_decode_workspace_bytes() bytes (may be NULL when that is 0),
- *            16-byte aligned; its contents need no initialisation.
+ *            16-byte aligned.  It must be zero-filled before its first use;
+ *            every completed call leaves it ready for the next one (its
+ *            arrival counters back at zero).  Calls that share a workspace
+ *            must not overlap on the GPU.
  *   out      device FP16 [batch][Hq][D] (round to nearest even), 16-byte aligned.
  *   lse_out  device FP32 [batch][Hq] natural-log log-sum-exp of the logits, or NULL.
  * An empty sequence (L = 0) gives out = 0 and lse = -inf.
+ * One kernel launch: one CTA per (split, kv head, sequence).  With at most 8
+ * splits the splits of a (sequence, kv head) form a thread-block cluster and
+ * are merged by log-sum-exp (the same merge as hyb_combine) through
+ * distributed shared memory; with more, the last CTA of a (sequence, kv head)
+ * to finish merges them through the workspace.
  * Arithmetic: cold dot products run exactly in integers (16-bit fixed-point q
  * per head, 16-bit fixed-point softmax weights per 16-token group); hot
  * tokens in FP32; the online softmax, the per-block scale products and all

@@ -69,7 +69,7 @@ class HybridKVCache:
     def workspace(self, max_seq_len, split_tokens=0):
         import torch
         n = _lib.hyb_decode_workspace_bytes(self.desc, max_seq_len, split_tokens)
-        return None if n == 0 else torch.empty(n, dtype=torch.uint8, device=self.device)
+        return None if n == 0 else torch.zeros(n, dtype=torch.uint8, device=self.device)
 
     def decode(self, q, softmax_scale, max_seq_len, split_tokens=0, out=None, lse=None,
                workspace=None, stream=None):

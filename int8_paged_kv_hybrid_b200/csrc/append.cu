@@ -39,57 +39,53 @@ __device__ __forceinline__ uint32_t nib_put(uint32_t w, int e, int c) {
 }
 
 // Re-quantize the codes of slots [0, first) of one tile from s_old to s_new.
+// Every possible code is re-quantized once (table in shared memory, same
+// arithmetic as requantize()); the tile is then rewritten by lookup, with
+// its words loaded 16 at a time so their latencies overlap.
 __device__ void requant_tile(uint8_t *tile, int kv, bool int4, int first, float s_old,
-                             float s_new, int q, int lane) {
+                             float s_new, int q, int lane, int8_t *tbl) {
+  for (int c = lane - 127; c <= 127; c += 32)
+    tbl[c + 127] = static_cast<int8_t>(requantize(c, s_old, s_new, q));
+  __syncwarp();
   uint32_t *w32 = reinterpret_cast<uint32_t *>(tile);
-  if (!int4 && kv == 0) {
-    // token-major rows of 128 bytes: word w holds 4 channels of slot w / 32
-    for (int w = lane; w < first * 32; w += 32) {
-      uint32_t x = w32[w], y = 0;
-      for (int e = 0; e < 4; e++) {
-        const int c = static_cast<int8_t>((x >> (8 * e)) & 0xff);
-        y |= static_cast<uint32_t>(requantize(c, s_old, s_new, q) & 0xff) << (8 * e);
-      }
-      w32[w] = y;
+  // words of the tile that can hold sealed slots, by layout
+  const int nwords = !int4 ? (kv == 0 ? first * 32 : kTileBytes / 4) : (kv == 0 ? first * 16 : kTileBytes / 8);
+  constexpr int kBatch = 16;
+  for (int w0 = lane; w0 < nwords; w0 += 32 * kBatch) {
+    uint32_t x[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; j++) {
+      const int w = w0 + 32 * j;
+      x[j] = w < nwords ? w32[w] : 0u;
     }
-  } else if (!int4) {
-    // channel-major rows of 64 bytes with swizzled 16-byte chunks
-    for (int w = lane; w < kTileBytes / 4; w += 32) {
-      const int row = w >> 4;
-      const int j = ((w >> 2) & 3) ^ ((row >> 1) & 3);
-      const int base = 16 * j + 4 * (w & 3);
-      if (base >= first) continue;
-      uint32_t x = w32[w], y = x;
-      for (int e = 0; e < 4; e++) {
-        if (base + e >= first) break;
-        const int c = static_cast<int8_t>((x >> (8 * e)) & 0xff);
-        y = (y & ~(0xffu << (8 * e))) |
-            (static_cast<uint32_t>(requantize(c, s_old, s_new, q) & 0xff) << (8 * e));
-      }
-      w32[w] = y;
-    }
-  } else if (kv == 0) {
-    // INT4 token-major rows of 64 bytes: word w holds 8 channels of slot w / 16
-    for (int w = lane; w < first * 16; w += 32) {
-      uint32_t x = w32[w], y = 0;
-      for (int e = 0; e < 8; e++) y = nib_put(y, e, requantize(nib_get(x, e), s_old, s_new, q));
-      w32[w] = y;
-    }
-  } else {
-    // INT4 channel-major rows of 32 bytes, swizzled 8-byte units of 16 slots
-    for (int w = lane; w < kTileBytes / 8; w += 32) {
-      const int row = w >> 3;
-      const int j = ((w >> 1) & 3) ^ ((row >> 2) & 3);
-      const int base = 16 * j + 8 * (w & 1);
-      if (base >= first) continue;
-      uint32_t x = w32[w], y = x;
-      for (int e = 0; e < 8; e++) {
-        if (base + e >= first) break;
-        y = nib_put(y, e, requantize(nib_get(x, e), s_old, s_new, q));
+#pragma unroll
+    for (int j = 0; j < kBatch; j++) {
+      const int w = w0 + 32 * j;
+      if (w >= nwords) continue;
+      uint32_t y = x[j];
+      if (!int4) {
+        // slot of byte e: token-major -> all sealed; channel-major -> 16*chunk + 4*(w%4) + e
+        const int row = w >> 4;
+        const int base = kv == 0 ? 0 : 16 * (((w >> 2) & 3) ^ ((row >> 1) & 3)) + 4 * (w & 3);
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          if (kv != 0 && base + e >= first) continue;
+          const int c = static_cast<int8_t>((x[j] >> (8 * e)) & 0xff);
+          y = (y & ~(0xffu << (8 * e))) | (static_cast<uint32_t>(static_cast<uint8_t>(tbl[c + 127])) << (8 * e));
+        }
+      } else {
+        const int row = w >> 3;
+        const int base = kv == 0 ? 0 : 16 * (((w >> 1) & 3) ^ ((row >> 2) & 3)) + 8 * (w & 1);
+#pragma unroll
+        for (int e = 0; e < 8; e++) {
+          if (kv != 0 && base + e >= first) continue;
+          y = nib_put(y, e, tbl[nib_get(x[j], e) + 127]);
+        }
       }
       w32[w] = y;
     }
   }
+  __syncwarp();
 }
 
 // Four FP16 channels 4*lane..4*lane+3 of position t (K if kv == 0, else V).
@@ -109,7 +105,7 @@ __device__ __forceinline__ void load4(const AppendArgs &a, int b, int h, int kv,
   x[3] = __high2float(hi);
 }
 
-__global__ void __launch_bounds__(1024) append_kernel(AppendArgs a) {
+__global__ void __launch_bounds__(512) append_kernel(AppendArgs a) {
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = blockDim.x >> 5;
@@ -127,6 +123,7 @@ __global__ void __launch_bounds__(1024) append_kernel(AppendArgs a) {
   if (n == 0) return;
   const int L_new = static_cast<int>(L_new_ll);
   const int e0 = max(0, L_old - kHot), e1 = max(0, L_new - kHot);
+  __shared__ int8_t s_tbl[16][256];  // per-warp re-quantization tables
 
   for (int pair = warp; pair < 2 * a.hkv; pair += nwarps) {
     const int h = pair >> 1, kv = pair & 1;
@@ -144,10 +141,15 @@ __global__ void __launch_bounds__(1024) append_kernel(AppendArgs a) {
       const int q = int4 ? 7 : 127;
       // absmax over the group's tokens and channels
       float amax = 0.f;
-      for (int t = p0; t < p1; t++) {
-        float x[4];
-        load4(a, b, h, kv, L_old, t, lane, x);
-        for (int j = 0; j < 4; j++) amax = fmaxf(amax, fabsf(x[j]));
+      for (int t0 = p0; t0 < p1; t0 += 8) {
+        float x[8][4];
+#pragma unroll
+        for (int u = 0; u < 8; u++)
+          if (t0 + u < p1) load4(a, b, h, kv, L_old, t0 + u, lane, x[u]);
+#pragma unroll
+        for (int u = 0; u < 8; u++)
+          if (t0 + u < p1)
+            for (int j = 0; j < 4; j++) amax = fmaxf(amax, fabsf(x[u][j]));
       }
       for (int m = 16; m > 0; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
       const float s_c = __fdiv_rn(amax, static_cast<float>(q));
@@ -157,17 +159,23 @@ __global__ void __launch_bounds__(1024) append_kernel(AppendArgs a) {
       if (first != 0) {
         const float s_old = *sp;
         if (s_c > s_old)
-          requant_tile(tile, kv, int4, first, s_old, s_c, q, lane);
+          requant_tile(tile, kv, int4, first, s_old, s_c, q, lane, s_tbl[warp]);
         else
           s = s_old;
       }
       __syncwarp();
-      for (int t = p0; t < p1; t++) {
+      for (int t0 = p0; t0 < p1; t0 += 8) {
+        float xb[8][4];
+#pragma unroll
+        for (int u = 0; u < 8; u++)
+          if (t0 + u < p1) load4(a, b, h, kv, L_old, t0 + u, lane, xb[u]);
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+        const int t = t0 + u;
+        if (t >= p1) break;
         const int slot = t - i * kBlock;
-        float x[4];
-        load4(a, b, h, kv, L_old, t, lane, x);
         int c[4];
-        for (int j = 0; j < 4; j++) c[j] = quantize(x[j], s, q);
+        for (int j = 0; j < 4; j++) c[j] = quantize(xb[u][j], s, q);
         if (!int4 && kv == 0) {
           uint32_t w = 0;
           for (int j = 0; j < 4; j++) w |= static_cast<uint32_t>(c[j] & 0xff) << (8 * j);
@@ -195,6 +203,7 @@ __global__ void __launch_bounds__(1024) append_kernel(AppendArgs a) {
                              : static_cast<uint8_t>((old & 0xf0) | (c[j] & 0xf));
           }
         }
+        }
       }
       if (lane == 0) *sp = s;
       __syncwarp();
@@ -215,7 +224,7 @@ __global__ void __launch_bounds__(1024) append_kernel(AppendArgs a) {
 }
 
 cudaError_t launch_append(const AppendArgs &a, int batch, cudaStream_t stream) {
-  const int nwarps = min(2 * a.hkv, 32);
+  const int nwarps = min(2 * a.hkv, 16);
   append_kernel<<<batch, 32 * nwarps, 0, stream>>>(a);
   return cudaGetLastError();
 }

@@ -11,24 +11,28 @@
 // split is a run of up to `split_blocks` cold blocks; the split that holds
 // the sequence's last cold block also attends the hot ring.  Each cold block
 // (K tile 8 KB + V tile 8 KB, or 4 + 4 KB for INT4) and the hot ring (16 KB)
-// is one pipeline item, brought into a 4-stage shared-memory ring by the TMA
+// is one pipeline item, brought into a 3-stage shared-memory ring by the TMA
 // engine with one 1-D bulk copy (no cluster multicast) completing on an
-// mbarrier; every wait is bounded.
+// mbarrier; every wait is bounded.  Four CTAs fit on an SM (16 warps).
 //
 // Arithmetic (per kv head, for its G = Hq/Hkv query heads):
 //  * q is turned into 16-bit fixed point per query head (q_i = rint(q * 32767
 //    / max|q|)); a cold logit is the exact int32 dot product of q_i with the
 //    K codes (dp2a: two 16x8-bit products per instruction), times
-//    max|q|/32767 * K-scale * softmax_scale * log2(e).
+//    max|q|/32767 * K-scale * softmax_scale * log2(e).  Eight lanes share a
+//    token (16 channels each); each lane keeps its heads in a lane-dependent
+//    order (head = k XOR x(lane)) so the cross-lane reduction that leaves one
+//    head's total in each lane needs no selects.
 //  * Warp w owns tokens 16w..16w+15 of every block and keeps its own online
-//    softmax state (running max, sum, FP32 output accumulator) per head.  Its
-//    softmax weights relative to the 16-token maximum are 16-bit fixed point
-//    (p_i = rint(32767 * 2^(z - max))); P.V is again an exact int32 dp2a sum
-//    over the V codes, folded into the FP32 state with the V scale.
+//    softmax state (running max, sum, FP32 output accumulator) per head,
+//    rescaling only when the running max grows.  Its softmax weights relative
+//    to the 16-token maximum are 16-bit fixed point (p_i = rint(32767 *
+//    2^(z - max))); P.V is again an exact int32 dp2a sum over the V codes,
+//    folded into the FP32 state with the V scale.
 //  * Hot tokens are attended in FP32 from the FP16 values (never quantized).
-//  * The 4 warp states are merged in FP32 at the end of the split; the
-//    split's normalised output and log-sum-exp go to the workspace for
-//    hyb_combine, or straight to the FP16 output when there is one split.
+//  * The 4 warp states are merged in FP32 at the end of the split; the last
+//    CTA of a (sequence, kv head) to finish merges the splits (log-sum-exp)
+//    and writes the FP16 output.
 // Tensor cores are not used: per byte of KV the work is a few integer
 // multiply-adds, and the kernel is bound by HBM bandwidth.
 #include <cfloat>
@@ -39,82 +43,91 @@ namespace hyb {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = 32 * kWarps;
-constexpr int kStages = 4;
-constexpr int kMaxSplitBlocks = 128;
+constexpr int kStages = 3;
+constexpr int kMaxSplitBlocks = 128;  // == kThreads: one block-table entry per thread
 constexpr long long kWaitCycles = 1ll << 31;  // ~1 s at B200 clocks
 constexpr float kLn2 = 0.69314718055994531f;
 
 template <int G>
+__host__ __device__ constexpr int pow2_heads() {
+  return G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : 8));
+}
+
+template <int G>
 struct DecodeSmem {
+  static constexpr int P = pow2_heads<G>();
   alignas(128) uint8_t ring[kStages][kTilePairBytes];
-  uint64_t full[kStages];
+  uint64_t full[kStages];   // data of the stage landed (TMA transaction count)
+  uint64_t empty[kStages];  // every warp is done with the stage
   int32_t phys[kMaxSplitBlocks];
-  float sk[kMaxSplitBlocks];
-  float sv[kMaxSplitBlocks];
-  alignas(16) float qf[G][kDim];
-  alignas(16) int16_t qi[G][kDim];
-  float sq[G];
+  float2 scl[kMaxSplitBlocks];  // (K scale, V scale) of each block of the split
+  alignas(16) float qf[P][kDim];     // q in FP32 (rows >= G are zero)
+  alignas(16) int16_t qi[P][kDim];   // q in 16-bit fixed point (rows >= G are zero)
+  float sq[P];                       // fixed-point step of each head's q
   alignas(16) uint16_t pcode[kWarps][G][16];
   alignas(16) float phot[kWarps][G][8];
   float wmax[kWarps][G];
   float wsum[kWarps][G];
   float mrun[kWarps][G];
   float lrun[kWarps][G];
+  float cl_l[G];   // this split's log2-sum-exp per head, read by the cluster's merge
+  float mfin[G];   // final merge: max and sum of the split weights per head
+  float dfin[G];
+  int last;
+  int abort_flag;
 };
 
-template <int G>
-constexpr int pow2_heads() {
-  return G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : 8));
+// 2^x on the SFU (max relative error ~2^-22); 2^-inf = +0.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
-// One level of the head-transposing reduction across lanes (xor m): lanes
-// with bit m set keep the upper half of the C live values, the others the
-// lower half, and each adds its partner's copy of the half it keeps.
-template <int C, int P, typename T>
-__device__ __forceinline__ void tr_level(T (&v)[P], int lane, int m) {
-  const bool up = (lane & m) != 0;
-#pragma unroll
-  for (int k = 0; k < C / 2; k++) {
-    const T send = up ? v[k] : v[k + C / 2];
-    const T keep = up ? v[k + C / 2] : v[k];
-    v[k] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-  }
-}
-
-// Sum each of P per-lane values over the 8 lanes of a lane octet; on return
-// v[0] holds the octet total of head head_of_lane<P>(lane).
+// Sum P per-lane values over the 8 lanes of a lane octet.  Lane l holds its
+// values in the order head = k ^ x(l) (see head_xor); at each level a lane
+// keeps its lower half and adds the partner's upper half, which (because the
+// partner's order differs in exactly that bit) holds the same heads.  On
+// return v[0] is the octet total for head x(l).
 template <int P, typename T>
-__device__ __forceinline__ void transpose_reduce(T (&v)[P], int lane) {
-  if constexpr (P == 8) {
-    tr_level<8>(v, lane, 4);
-    tr_level<4>(v, lane, 2);
-    tr_level<2>(v, lane, 1);
-  } else if constexpr (P == 4) {
-    tr_level<4>(v, lane, 4);
-    tr_level<2>(v, lane, 2);
-    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
-  } else if constexpr (P == 2) {
-    tr_level<2>(v, lane, 4);
-    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 2);
-    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
-  } else {
-    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 4);
-    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 2);
-    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
-  }
-}
-
-template <int P>
-__device__ __forceinline__ int head_of_lane(int lane) {
-  int hd = 0, c = P;
+__device__ __forceinline__ void transpose_reduce(T (&v)[P]) {
+  int c = P;
 #pragma unroll
   for (int m = 4; m >= 1; m >>= 1) {
     if (c > 1) {
-      if (lane & m) hd += c / 2;
+#pragma unroll
+      for (int k = 0; k < c / 2; k++) v[k] += __shfl_xor_sync(0xffffffffu, v[k + c / 2], m);
       c /= 2;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
     }
   }
-  return hd;
+}
+
+// Head order of a lane: value k of the lane is head k ^ head_xor(lane).
+template <int P>
+__device__ __forceinline__ int head_xor(int lane) {
+  if constexpr (P == 8) return lane & 7;
+  if constexpr (P == 4) return (lane >> 1) & 3;
+  if constexpr (P == 2) return (lane >> 2) & 1;
+  return 0;
+}
+
+// Barrier over all threads of all CTAs of the cluster (release / acquire).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Load a float from the shared memory of CTA `rank` of this cluster, at the
+// offset `local` has in this CTA's shared memory.
+__device__ __forceinline__ float ld_cluster_f32(const float *local, int rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
 }
 
 __device__ __forceinline__ void unpack_int4(uint32_t x, uint32_t &lo, uint32_t &hi) {
@@ -122,8 +135,11 @@ __device__ __forceinline__ void unpack_int4(uint32_t x, uint32_t &lo, uint32_t &
   hi = sext_nibbles((x >> 4) & 0x0f0f0f0fu);
 }
 
-template <int G>
-__global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(const DecodeArgs a) {
+// kCluster: the grid is launched in clusters of n_splits CTAs (the splits of
+// one (sequence, kv head)); splits are merged through distributed shared
+// memory instead of the workspace.
+template <int G, bool kCluster>
+__global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 2)) decode_kernel(const DecodeArgs a) {
   constexpr int P = pow2_heads<G>();
   extern __shared__ __align__(128) uint8_t smem_raw[];
   DecodeSmem<G> &sm = *reinterpret_cast<DecodeSmem<G> *>(smem_raw);
@@ -132,54 +148,53 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int S = a.n_splits;
   const int hq0 = h * G;
+  const int i0 = s * a.split_blocks;
 
+  // independent loads first: the sequence length, this split's block-table
+  // entries (one per thread, clamped to the row) and q
   int L = a.seq_lens[b];
+  const int i_tid = i0 + tid;
+  const int phys_raw =
+      (tid < a.split_blocks && i_tid < a.max_blocks) ? a.block_table[(size_t)b * a.max_blocks + i_tid] : -1;
+  float qv[G];
+#pragma unroll
+  for (int j = 0; j < G; j++) qv[j] = __half2float(a.q[((size_t)b * a.hq + hq0) * kDim + j * kDim + tid]);
+
   if (L < 0 || L > a.max_seq_len) {
+    // sequence skipped: treated as empty (zero output, lse -inf)
     if (tid == 0 && s == 0 && h == 0) set_status(a.status, HYB_STATUS_SEQ_LEN);
-    L = -1;
+    L = 0;
   }
   const int Lc = max(0, L - kHot);
   const int nblk = (Lc + kBlock - 1) / kBlock;
   const int Sb = max(1, (nblk + a.split_blocks - 1) / a.split_blocks);
-  if (L < 0 || s >= Sb) {
-    // nothing to attend in this split: neutral partial result
-    for (int e = tid; e < G * kDim; e += kThreads) {
-      const int hh = e / kDim, c = e % kDim;
-      const size_t row = (size_t)b * a.hq + hq0 + hh;
-      if (S > 1)
-        a.o_part[(row * S + s) * kDim + c] = 0.f;
-      else
-        a.out[row * kDim + c] = __float2half_rn(0.f);
-      if (c == 0) {
-        if (S > 1)
-          a.lse_part[row * S + s] = -INFINITY;
-        else if (a.lse_out)
-          a.lse_out[row] = -INFINITY;
-      }
-    }
-    return;
-  }
-  const int i0 = s * a.split_blocks;
-  const int ncold = min(nblk, i0 + a.split_blocks) - i0;
+  // past this sequence's last split: no work and no partial (a cluster member
+  // still takes part in the cluster's merge, with an empty state)
+  if (!kCluster && s >= Sb) return;
+  const int ncold = max(0, min(nblk, i0 + a.split_blocks) - i0);
   const int nhot = (s == Sb - 1) ? min(L, kHot) : 0;
   const int nitems = ncold + (nhot > 0 ? 1 : 0);
   const int n_int4_b = a.quant_bits == 4 ? 0x7fffffff : (a.n_int4 ? a.n_int4[b] : 0);
 
   if (tid == 0) {
 #pragma unroll
-    for (int st = 0; st < kStages; st++) mbar_init(&sm.full[st], 1);
+    for (int st = 0; st < kStages; st++) {
+      mbar_init(&sm.full[st], 1);
+      mbar_init(&sm.empty[st], kWarps);
+    }
+    sm.abort_flag = 0;
     mbar_fence_init();
   }
-  for (int k = tid; k < ncold; k += kThreads) {
-    int phys = a.block_table[(size_t)b * a.max_blocks + i0 + k];
+  if (tid < ncold) {
+    int phys = phys_raw;
     if (phys < 0 || phys >= a.num_phys) {
       set_status(a.status, HYB_STATUS_BAD_BLOCK);
       phys = -1;
     }
-    sm.phys[k] = phys;
+    sm.phys[tid] = phys;
   }
-  for (int e = tid; e < G * kDim; e += kThreads)
-    sm.qf[e / kDim][e % kDim] = __half2float(a.q[((size_t)b * a.hq + hq0) * kDim + e]);
+#pragma unroll
+  for (int j = 0; j < P; j++) sm.qf[j][tid] = j < G ? qv[j] : 0.f;
   __syncthreads();
 
   const uint64_t pol = l2_policy_evict_first();
@@ -208,46 +223,44 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
       bulk_g2s(dst, src, bytes, &sm.full[st], pol);
     }
   };
+  // block scales: requested before the bulk copies so that they do not queue
+  // behind them; stored once they arrive (overlapping the copies)
+  float2 sc_ld = make_float2(0.f, 0.f);
+  if (tid < ncold && sm.phys[tid] >= 0)
+    sc_ld = __ldg(reinterpret_cast<const float2 *>(a.scales + ((size_t)sm.phys[tid] * a.hkv + h) * 2));
   int issued = 0;
   if (tid == 0) {
     issued = min(nitems, kStages);
     for (int k = 0; k < issued; k++) issue(k);
   }
-
-  // block scales (their loads overlap the first copies)
-  for (int k = tid; k < ncold; k += kThreads) {
-    const int phys = sm.phys[k];
-    float2 sc = make_float2(0.f, 0.f);
-    if (phys >= 0) sc = *reinterpret_cast<const float2 *>(a.scales + ((size_t)phys * a.hkv + h) * 2);
-    sm.sk[k] = sc.x;
-    sm.sv[k] = sc.y;
-  }
-  // q in 16-bit fixed point per head
-  for (int hh = warp; hh < G; hh += kWarps) {
+  if (tid < ncold) sm.scl[tid] = sc_ld;
+  // q in 16-bit fixed point per head (padding heads stay zero)
+  for (int j = warp; j < P; j += kWarps) {
     float amax = 0.f;
-    for (int c = lane; c < kDim; c += 32) amax = fmaxf(amax, fabsf(sm.qf[hh][c]));
+    for (int c = lane; c < kDim; c += 32) amax = fmaxf(amax, fabsf(sm.qf[j][c]));
+#pragma unroll
     for (int m = 16; m > 0; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
     const float inv = amax > 0.f ? 32767.f / amax : 0.f;
     for (int c = lane; c < kDim; c += 32) {
-      const int v = __float2int_rn(sm.qf[hh][c] * inv);
-      sm.qi[hh][c] = static_cast<int16_t>(max(-32767, min(32767, v)));
+      const int v = __float2int_rn(sm.qf[j][c] * inv);
+      sm.qi[j][c] = static_cast<int16_t>(max(-32767, min(32767, v)));
     }
-    if (lane == 0) sm.sq[hh] = amax > 0.f ? amax / 32767.f : 0.f;
+    if (lane == 0) sm.sq[j] = amax > 0.f ? amax / 32767.f : 0.f;
   }
   __syncthreads();
 
   const int tg = lane >> 3, cs = lane & 7;
-  const int hd = head_of_lane<P>(lane);
-  const bool owner = (lane & (8 / P - 1)) == 0 && hd < G;
-  const float sq_hd = hd < G ? sm.sq[hd] : 0.f;
+  const int hx = head_xor<P>(lane);   // this lane's value k is head k ^ hx; its final head is hx
+  const bool owner = (lane & (8 / P - 1)) == 0 && hx < G;
+  const float sq_hd = sm.sq[hx];
 
-  uint32_t qp[G][8];
+  uint32_t qp[P][8];  // q pairs of this lane's 16 channels, in the lane's head order
 #pragma unroll
-  for (int hh = 0; hh < G; hh++) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(&sm.qi[hh][16 * cs]);
+  for (int k = 0; k < P; k++) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(&sm.qi[k ^ hx][16 * cs]);
     const uint4 x0 = src[0], x1 = src[1];
-    qp[hh][0] = x0.x; qp[hh][1] = x0.y; qp[hh][2] = x0.z; qp[hh][3] = x0.w;
-    qp[hh][4] = x1.x; qp[hh][5] = x1.y; qp[hh][6] = x1.z; qp[hh][7] = x1.w;
+    qp[k][0] = x0.x; qp[k][1] = x0.y; qp[k][2] = x0.z; qp[k][3] = x0.w;
+    qp[k][4] = x1.x; qp[k][5] = x1.y; qp[k][6] = x1.z; qp[k][7] = x1.w;
   }
 
   float m_run[G], l_run[G], acc[G][4];
@@ -260,11 +273,30 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
   }
 
   bool aborted = false;
-  int k_stop = nitems;
+  int next_issue = issued;  // thread 0: next item to bring in
   for (int k = 0; k < nitems; k++) {
     const int st = k % kStages;
-    const bool ok = mbar_wait_bounded(&sm.full[st], (k / kStages) & 1, kWaitCycles);
+    // thread 0 refills stages the warps have released: item k must be in
+    // flight before anyone waits for it, later ones only if already free
+    if (tid == 0) {
+      for (; next_issue < min(nitems, k + kStages); next_issue++) {
+        const int j = next_issue - kStages;  // previous item of that stage
+        if (next_issue <= k) {
+          if (!mbar_wait_bounded(&sm.empty[j % kStages], (j / kStages) & 1, kWaitCycles)) {
+            set_status(a.status, HYB_STATUS_TIMEOUT);
+            sm.abort_flag = 1;
+            break;
+          }
+        } else if (!mbar_try_wait(&sm.empty[j % kStages], (j / kStages) & 1)) {
+          break;
+        }
+        issue(next_issue);
+      }
+      issued = next_issue;
+    }
+    bool ok = mbar_wait_bounded(&sm.full[st], (k / kStages) & 1, kWaitCycles);
     if (!ok && lane == 0) set_status(a.status, HYB_STATUS_TIMEOUT);
+    ok = ok && *reinterpret_cast<volatile int *>(&sm.abort_flag) == 0;
     const uint8_t *stage = sm.ring[st];
     if (ok && k < ncold) {
       // ---------------- cold block ----------------
@@ -273,7 +305,8 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
       const int nv = nvalid - 16 * warp;
       if (nv > 0) {
         const bool int4 = i < n_int4_b;
-        const float coef = sq_hd * sm.sk[k] * a.qk_scale;
+        const float2 sc = sm.scl[k];
+        const float coef = sq_hd * sc.x * a.qk_scale;
         float z[4];
 #pragma unroll
         for (int step = 0; step < 4; step++) {
@@ -289,40 +322,40 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
           }
           int dot[P];
 #pragma unroll
-          for (int hh = 0; hh < P; hh++) {
-            int d = 0;
-            if (hh < G) {
+          for (int kk = 0; kk < P; kk++) dot[kk] = 0;
 #pragma unroll
-              for (int j = 0; j < 4; j++) {
-                d = __dp2a_lo(static_cast<int>(qp[hh][2 * j]), static_cast<int>(kw[j]), d);
-                d = __dp2a_hi(static_cast<int>(qp[hh][2 * j + 1]), static_cast<int>(kw[j]), d);
-              }
-            }
-            dot[hh] = d;
+          for (int j = 0; j < 4; j++) {
+#pragma unroll
+            for (int kk = 0; kk < P; kk++)
+              dot[kk] = __dp2a_lo(static_cast<int>(qp[kk][2 * j]), static_cast<int>(kw[j]), dot[kk]);
+#pragma unroll
+            for (int kk = 0; kk < P; kk++)
+              dot[kk] = __dp2a_hi(static_cast<int>(qp[kk][2 * j + 1]), static_cast<int>(kw[j]), dot[kk]);
           }
-          transpose_reduce<P>(dot, lane);
-          z[step] = (4 * step + tg < nv && hd < G) ? static_cast<float>(dot[0]) * coef : -INFINITY;
+          transpose_reduce<P>(dot);
+          z[step] = (4 * step + tg < nv) ? static_cast<float>(dot[0]) * coef : -INFINITY;
         }
         float mb = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
         mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 8));
         mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 16));
+        // 16-bit weights: round(32767 * 2^(z - mb)) via the 1.5*2^23 magic add
         int psum = 0;
-        int pc[4];
+        uint32_t pc[4];
 #pragma unroll
         for (int step = 0; step < 4; step++) {
-          const float pv = z[step] == -INFINITY ? 0.f : exp2f(z[step] - mb);
-          pc[step] = __float2int_rn(pv * 32767.f);
-          psum += pc[step];
+          const float pq = fmaf(ex2(z[step] - mb), 32767.f, 12582912.f);
+          pc[step] = __float_as_uint(pq) - 0x4B400000u;
+          psum += static_cast<int>(pc[step]);
         }
         psum += __shfl_xor_sync(0xffffffffu, psum, 8);
         psum += __shfl_xor_sync(0xffffffffu, psum, 16);
         if (owner) {
 #pragma unroll
           for (int step = 0; step < 4; step++)
-            sm.pcode[warp][hd][4 * step + tg] = static_cast<uint16_t>(pc[step]);
+            sm.pcode[warp][hx][4 * step + tg] = static_cast<uint16_t>(pc[step]);
           if (tg == 0) {
-            sm.wmax[warp][hd] = mb;
-            sm.wsum[warp][hd] = static_cast<float>(psum);
+            sm.wmax[warp][hx] = mb;
+            sm.wsum[warp][hx] = static_cast<float>(psum);
           }
         }
         __syncwarp();
@@ -342,32 +375,40 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
             unpack_int4(v.y, vw[kk][2], vw[kk][3]);
           }
         }
-        const float sv = sm.sv[k];
+        int ai[G][4];
+#pragma unroll
+        for (int hh = 0; hh < G; hh++)
+#pragma unroll
+          for (int kk = 0; kk < 4; kk++) ai[hh][kk] = 0;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+#pragma unroll
+          for (int hh = 0; hh < G; hh++) {
+            // p codes of tokens 4j..4j+3 of this warp's 16, as two 16-bit pairs
+            const uint2 pp = *reinterpret_cast<const uint2 *>(&sm.pcode[warp][hh][4 * j]);
+#pragma unroll
+            for (int kk = 0; kk < 4; kk++) {
+              ai[hh][kk] = __dp2a_lo(static_cast<int>(pp.x), static_cast<int>(vw[kk][j]), ai[hh][kk]);
+              ai[hh][kk] = __dp2a_hi(static_cast<int>(pp.y), static_cast<int>(vw[kk][j]), ai[hh][kk]);
+            }
+          }
+        }
 #pragma unroll
         for (int hh = 0; hh < G; hh++) {
-          const uint4 pa = *reinterpret_cast<const uint4 *>(&sm.pcode[warp][hh][0]);
-          const uint4 pb = *reinterpret_cast<const uint4 *>(&sm.pcode[warp][hh][8]);
-          const uint32_t pp[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
-          int ai[4];
-#pragma unroll
-          for (int kk = 0; kk < 4; kk++) {
-            int d = 0;
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-              d = __dp2a_lo(static_cast<int>(pp[2 * j]), static_cast<int>(vw[kk][j]), d);
-              d = __dp2a_hi(static_cast<int>(pp[2 * j + 1]), static_cast<int>(vw[kk][j]), d);
-            }
-            ai[kk] = d;
-          }
           const float mbh = sm.wmax[warp][hh];
-          const float m_new = fmaxf(m_run[hh], mbh);
-          const float alpha = exp2f(m_run[hh] - m_new);
-          const float beta = exp2f(mbh - m_new) * (1.f / 32767.f);
-          l_run[hh] = l_run[hh] * alpha + beta * sm.wsum[warp][hh];
-          const float cv = beta * sv;
+          if (mbh > m_run[hh]) {  // warp-uniform: rescale only when the max grows
+            const float alpha = ex2(m_run[hh] - mbh);
+            l_run[hh] *= alpha;
 #pragma unroll
-          for (int kk = 0; kk < 4; kk++) acc[hh][kk] = acc[hh][kk] * alpha + cv * static_cast<float>(ai[kk]);
-          m_run[hh] = m_new;
+            for (int kk = 0; kk < 4; kk++) acc[hh][kk] *= alpha;
+            m_run[hh] = mbh;
+          }
+          const float beta = ex2(mbh - m_run[hh]) * (1.f / 32767.f);
+          l_run[hh] = fmaf(beta, sm.wsum[warp][hh], l_run[hh]);
+          const float cv = beta * sc.y;
+#pragma unroll
+          for (int kk = 0; kk < 4; kk++)
+            acc[hh][kk] = fmaf(cv, static_cast<float>(ai[hh][kk]), acc[hh][kk]);
         }
       }
     } else if (ok) {
@@ -390,23 +431,21 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
           }
           float dot[P];
 #pragma unroll
-          for (int hh = 0; hh < P; hh++) {
+          for (int kk = 0; kk < P; kk++) {
+            const float4 *qv4 = reinterpret_cast<const float4 *>(&sm.qf[kk ^ hx][16 * cs]);
             float d = 0.f;
-            if (hh < G) {
-              const float4 *qv = reinterpret_cast<const float4 *>(&sm.qf[hh][16 * cs]);
 #pragma unroll
-              for (int j = 0; j < 4; j++) {
-                const float4 qq = qv[j];
-                d = fmaf(qq.x, kf[4 * j], d);
-                d = fmaf(qq.y, kf[4 * j + 1], d);
-                d = fmaf(qq.z, kf[4 * j + 2], d);
-                d = fmaf(qq.w, kf[4 * j + 3], d);
-              }
+            for (int j = 0; j < 4; j++) {
+              const float4 qq = qv4[j];
+              d = fmaf(qq.x, kf[4 * j], d);
+              d = fmaf(qq.y, kf[4 * j + 1], d);
+              d = fmaf(qq.z, kf[4 * j + 2], d);
+              d = fmaf(qq.w, kf[4 * j + 3], d);
             }
-            dot[hh] = d;
+            dot[kk] = d;
           }
-          transpose_reduce<P>(dot, lane);
-          z[step] = (4 * step + tg < nv && hd < G) ? dot[0] * a.qk_scale : -INFINITY;
+          transpose_reduce<P>(dot);
+          z[step] = (4 * step + tg < nv) ? dot[0] * a.qk_scale : -INFINITY;
         }
         float mb = fmaxf(z[0], z[1]);
         mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 8));
@@ -414,17 +453,17 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
         float pv[2], psum = 0.f;
 #pragma unroll
         for (int step = 0; step < 2; step++) {
-          pv[step] = z[step] == -INFINITY ? 0.f : exp2f(z[step] - mb);
+          pv[step] = ex2(z[step] - mb);
           psum += pv[step];
         }
         psum += __shfl_xor_sync(0xffffffffu, psum, 8);
         psum += __shfl_xor_sync(0xffffffffu, psum, 16);
         if (owner) {
-          sm.phot[warp][hd][tg] = pv[0];
-          sm.phot[warp][hd][4 + tg] = pv[1];
+          sm.phot[warp][hx][tg] = pv[0];
+          sm.phot[warp][hx][4 + tg] = pv[1];
           if (tg == 0) {
-            sm.wmax[warp][hd] = mb;
-            sm.wsum[warp][hd] = psum;
+            sm.wmax[warp][hx] = mb;
+            sm.wsum[warp][hx] = psum;
           }
         }
         __syncwarp();
@@ -450,52 +489,62 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
 #pragma unroll
         for (int hh = 0; hh < G; hh++) {
           const float mbh = sm.wmax[warp][hh];
-          const float m_new = fmaxf(m_run[hh], mbh);
-          const float alpha = exp2f(m_run[hh] - m_new);
-          const float beta = exp2f(mbh - m_new);
-          l_run[hh] = l_run[hh] * alpha + beta * sm.wsum[warp][hh];
+          if (mbh > m_run[hh]) {
+            const float alpha = ex2(m_run[hh] - mbh);
+            l_run[hh] *= alpha;
 #pragma unroll
-          for (int kk = 0; kk < 4; kk++) acc[hh][kk] = acc[hh][kk] * alpha + beta * ah[hh][kk];
-          m_run[hh] = m_new;
+            for (int kk = 0; kk < 4; kk++) acc[hh][kk] *= alpha;
+            m_run[hh] = mbh;
+          }
+          const float beta = ex2(mbh - m_run[hh]);
+          l_run[hh] = fmaf(beta, sm.wsum[warp][hh], l_run[hh]);
+#pragma unroll
+          for (int kk = 0; kk < 4; kk++) acc[hh][kk] = fmaf(beta, ah[hh][kk], acc[hh][kk]);
         }
       }
     }
-    if (__syncthreads_or(!ok)) {
+    __syncwarp();
+    if (!ok) {
+      sm.abort_flag = 1;
       aborted = true;
-      k_stop = k;
       break;
     }
-    if (tid == 0 && k + kStages < nitems) {
-      issue(k + kStages);
-      issued = k + kStages + 1;
-    }
+    if (lane == 0) mbar_arrive(&sm.empty[st]);
   }
+  aborted = __syncthreads_or(aborted) != 0;
 
   if (aborted) {
-    // let every copy still in flight land before the CTA's shared memory is released
+    // let every copy still in flight land before the CTA's shared memory is
+    // released: the last item issued into each stage
     if (tid == 0) {
-      for (int k = k_stop; k < issued; k++)
-        (void)mbar_wait_bounded(&sm.full[k % kStages], (k / kStages) & 1, kWaitCycles);
+      for (int j = max(0, issued - kStages); j < issued; j++)
+        (void)mbar_wait_bounded(&sm.full[j % kStages], (j / kStages) & 1, kWaitCycles);
     }
     __syncthreads();
-    return;
-  }
-
-  // ---------------- merge the 4 warp states ----------------
-  float *mbuf = reinterpret_cast<float *>(&sm.ring[0][0]);  // [kWarps][G][kDim]
+  } else {
+    // ---------------- merge the 4 warp states ----------------
+    float *mbuf = reinterpret_cast<float *>(&sm.ring[0][0]);  // [kWarps][G][kDim]
 #pragma unroll
-  for (int hh = 0; hh < G; hh++)
+    for (int hh = 0; hh < G; hh++)
 #pragma unroll
-    for (int kk = 0; kk < 4; kk++) mbuf[(warp * G + hh) * kDim + lane + 32 * kk] = acc[hh][kk];
-  if (lane == 0) {
+      for (int kk = 0; kk < 4; kk++) mbuf[(warp * G + hh) * kDim + lane + 32 * kk] = acc[hh][kk];
+    if (lane == 0) {
 #pragma unroll
-    for (int hh = 0; hh < G; hh++) {
-      sm.mrun[warp][hh] = m_run[hh];
-      sm.lrun[warp][hh] = l_run[hh];
+      for (int hh = 0; hh < G; hh++) {
+        sm.mrun[warp][hh] = m_run[hh];
+        sm.lrun[warp][hh] = l_run[hh];
+      }
     }
+    __syncthreads();
   }
-  __syncthreads();
+  // this split's normalised output (channel tid) and log2-sum-exp per head
+  float o_s[G], lse2_s[G];
+#pragma unroll
   for (int hh = 0; hh < G; hh++) {
+    o_s[hh] = 0.f;
+    lse2_s[hh] = -INFINITY;
+    if (aborted) continue;
+    const float *mbuf = reinterpret_cast<const float *>(&sm.ring[0][0]);
     float mm = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kWarps; w++) mm = fmaxf(mm, sm.mrun[w][hh]);
@@ -503,23 +552,150 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
     if (mm != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < kWarps; w++) {
-        const float f = exp2f(sm.mrun[w][hh] - mm);
+        const float f = ex2(sm.mrun[w][hh] - mm);
         num = fmaf(f, mbuf[(w * G + hh) * kDim + tid], num);
         den = fmaf(f, sm.lrun[w][hh], den);
       }
     }
-    const float o = den > 0.f ? num / den : 0.f;
-    const float lse = den > 0.f ? (mm + log2f(den)) * kLn2 : -INFINITY;
+    if (den > 0.f) {
+      o_s[hh] = num * __frcp_rn(den);
+      lse2_s[hh] = mm + __log2f(den);
+    }
+  }
+  if constexpr (kCluster) {
+    // ---------------- split merge across the cluster (distributed shared memory) ----------------
+    float *cl_o = reinterpret_cast<float *>(&sm.ring[0][0]);  // [G][kDim], this split's output
+    __syncthreads();  // the warp-merge buffer above is no longer read
+#pragma unroll
+    for (int hh = 0; hh < G; hh++) cl_o[hh * kDim + tid] = o_s[hh];
+    if (tid == 0) {
+#pragma unroll
+      for (int hh = 0; hh < G; hh++) sm.cl_l[hh] = lse2_s[hh];
+    }
+    cluster_sync_all();
+    // CTA s of the cluster merges output elements [s*per, (s+1)*per)
+    const int per = (G * kDim + S - 1) / S;
+    for (int e = s * per + tid; e < min((s + 1) * per, G * kDim); e += kThreads) {
+      const int hh = e / kDim, c = e - hh * kDim;
+      float lj[16];
+      float m = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 16; j++) {
+        lj[j] = j < S ? ld_cluster_f32(&sm.cl_l[hh], j) : -INFINITY;
+        m = fmaxf(m, lj[j]);
+      }
+      float num = 0.f, den = 0.f;
+      if (m != -INFINITY) {
+#pragma unroll
+        for (int j = 0; j < 16; j++) {
+          if (j < S) {
+            const float wgt = ex2(lj[j] - m);
+            num = fmaf(wgt, ld_cluster_f32(&cl_o[hh * kDim + c], j), num);
+            den += wgt;
+          }
+        }
+      }
+      const size_t row = (size_t)b * a.hq + hq0 + hh;
+      a.out[row * kDim + c] = __float2half_rn(den > 0.f ? num / den : 0.f);
+      if (c == 0 && a.lse_out) a.lse_out[row] = den > 0.f ? (m + log2f(den)) * kLn2 : -INFINITY;
+    }
+    cluster_sync_all();  // no CTA leaves while its shared memory may still be read
+    return;
+  }
+  if (Sb == 1) {
+#pragma unroll
+    for (int hh = 0; hh < G; hh++) {
+      const size_t row = (size_t)b * a.hq + hq0 + hh;
+      a.out[row * kDim + tid] = __float2half_rn(o_s[hh]);
+      if (tid == 0 && a.lse_out) a.lse_out[row] = lse2_s[hh] * kLn2;
+    }
+    return;
+  }
+  // ---------------- split merge by the last CTA of (sequence, kv head) ----------------
+#pragma unroll
+  for (int hh = 0; hh < G; hh++) {
     const size_t row = (size_t)b * a.hq + hq0 + hh;
-    if (S == 1) {
-      a.out[row * kDim + tid] = __float2half_rn(o);
-      if (tid == 0 && a.lse_out) a.lse_out[row] = lse;
-    } else {
-      a.o_part[(row * S + s) * kDim + tid] = o;
-      if (tid == 0) a.lse_part[row * S + s] = lse;
+    a.o_part[(row * S + s) * kDim + tid] = o_s[hh];
+    if (tid == 0) a.lse_part[row * S + s] = lse2_s[hh];
+  }
+  __syncthreads();  // all partial stores of the CTA precede thread 0's release below
+  if (tid == 0) {
+    __threadfence();
+    const int ticket = atomicAdd(&a.counters[(size_t)b * a.hkv + h], 1);
+    sm.last = (ticket == Sb - 1) ? 1 : 0;
+    if (sm.last) {
+      __threadfence();
+      a.counters[(size_t)b * a.hkv + h] = 0;  // ready for the next call
+    }
+  }
+  __syncthreads();
+  if (!sm.last) return;
+  __threadfence();
+  // split weights: lse of every (head, split) into shared memory, then per
+  // head the max and the weights 2^(lse - max) (0 for empty splits)
+  float *wts = reinterpret_cast<float *>(&sm.ring[0][0]);  // [G][Sb]
+  const bool fits = G * Sb <= kStages * kTilePairBytes / 4;
+  if (fits) {
+    for (int e = tid; e < G * Sb; e += kThreads) {
+      const int hh = e / Sb, j = e - hh * Sb;
+      wts[e] = __ldcg(a.lse_part + ((size_t)b * a.hq + hq0 + hh) * S + j);
+    }
+    __syncthreads();
+    for (int hh = warp; hh < G; hh += kWarps) {
+      float m = -INFINITY;
+      for (int j = lane; j < Sb; j += 32) m = fmaxf(m, wts[hh * Sb + j]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float den = 0.f;
+      for (int j = lane; j < Sb; j += 32) {
+        const float wv = m == -INFINITY ? 0.f : ex2(wts[hh * Sb + j] - m);
+        wts[hh * Sb + j] = wv;
+        den += wv;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+      if (lane == 0) {
+        sm.mfin[hh] = m;
+        sm.dfin[hh] = den;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int hh = 0; hh < G; hh++) {
+      const size_t row = (size_t)b * a.hq + hq0 + hh;
+      const float *op = a.o_part + row * S * kDim + tid;
+      float num = 0.f;
+#pragma unroll 8
+      for (int j = 0; j < Sb; j++) num = fmaf(wts[hh * Sb + j], __ldcg(op + (size_t)j * kDim), num);
+      const float den = sm.dfin[hh];
+      a.out[row * kDim + tid] = __float2half_rn(den > 0.f ? num / den : 0.f);
+      if (tid == 0 && a.lse_out) a.lse_out[row] = den > 0.f ? (sm.mfin[hh] + log2f(den)) * kLn2 : -INFINITY;
+    }
+  } else {
+    // very many splits: two passes over global memory per head
+#pragma unroll 1
+    for (int hh = 0; hh < G; hh++) {
+      const size_t row = (size_t)b * a.hq + hq0 + hh;
+      const float *lp = a.lse_part + row * S;
+      const float *op = a.o_part + row * S * kDim + tid;
+      float m = -INFINITY;
+      for (int j = 0; j < Sb; j++) m = fmaxf(m, __ldcg(lp + j));
+      float num = 0.f, den = 0.f;
+      if (m != -INFINITY) {
+        for (int j = 0; j < Sb; j++) {
+          const float wgt = ex2(__ldcg(lp + j) - m);
+          num = fmaf(wgt, __ldcg(op + (size_t)j * kDim), num);
+          den += wgt;
+        }
+      }
+      a.out[row * kDim + tid] = __float2half_rn(den > 0.f ? num / den : 0.f);
+      if (tid == 0 && a.lse_out) a.lse_out[row] = den > 0.f ? (m + log2f(den)) * kLn2 : -INFINITY;
     }
   }
 }
+
+// Largest cluster the decode kernel is launched with (portable size).
+constexpr int kMaxCluster = 8;
 
 template <int G>
 static cudaError_t launch_decode_g(const DecodeArgs &a, int batch, cudaStream_t stream) {
@@ -529,13 +705,33 @@ static cudaError_t launch_decode_g(const DecodeArgs &a, int batch, cudaStream_t 
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 31 && !(configured_dev_mask & (1 << dev))) {
-    e = cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(decode_kernel<G, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(decode_kernel<G, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     configured_dev_mask |= 1 << dev;
   }
   dim3 grid(a.n_splits, a.hkv, batch);
-  decode_kernel<G><<<grid, kThreads, smem, stream>>>(a);
+  if (a.n_splits >= 2 && a.n_splits <= kMaxCluster) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = a.n_splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_kernel<G, true>, a);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
+  decode_kernel<G, false><<<grid, kThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -553,6 +749,42 @@ cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, cudaStream_
   }
 }
 
+int decode_max_cluster() { return kMaxCluster; }
+
 int decode_max_split_blocks() { return kMaxSplitBlocks; }
+
+// CTAs of the decode kernel one SM holds at once for this head group (0 if
+// the device cannot be queried).
+int decode_ctas_per_sm(int group) {
+  static int cached[32][9];  // [device][group], 0 = not yet known
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (dev >= 0 && dev < 32 && group >= 1 && group <= 8 && cached[dev][group] > 0)
+    return cached[dev][group];
+  int n = 0;
+  cudaError_t e = cudaErrorInvalidValue;
+  switch (group) {
+#define HYB_OCC(g)                                                                          \
+  case g:                                                                                   \
+    e = cudaFuncSetAttribute(decode_kernel<g, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             static_cast<int>(sizeof(DecodeSmem<g>)));                      \
+    if (e == cudaSuccess)                                                                   \
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<g, false>, kThreads, \
+                                                        sizeof(DecodeSmem<g>));             \
+    break;
+    HYB_OCC(1) HYB_OCC(2) HYB_OCC(3) HYB_OCC(4) HYB_OCC(5) HYB_OCC(6) HYB_OCC(7) HYB_OCC(8)
+#undef HYB_OCC
+    default: break;
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (dev >= 0 && dev < 32 && group >= 1 && group <= 8) cached[dev][group] = n;
+  return n;
+}
 
 }  // namespace hyb

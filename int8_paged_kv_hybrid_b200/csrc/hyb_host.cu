@@ -123,13 +123,22 @@ int hyb_decode_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_
   if (max_blocks_needed > d->max_blocks_per_seq) return HYB_ERR_INVALID_VALUE;
   int tb;  // cold blocks per split
   if (split_tokens == 0) {
-    // enough CTAs for about three per SM over the whole grid, at least two
-    // blocks per split, at most the kernel's limit
+    // Automatic: with few (sequence, kv head) units, enough splits of the
+    // longest sequence to fill one wave of resident CTAs and no more; with
+    // many units, splits of about a quarter wave's share so that sequences of
+    // different lengths even out over several waves.
+    const int group = d->num_q_heads / d->num_kv_heads;
+    int occ = hyb::decode_ctas_per_sm(group);
+    if (occ <= 0) occ = group <= 4 ? 4 : 2;
+    const long long slots = static_cast<long long>(sm_count()) * occ;
     const long long units = static_cast<long long>(d->batch) * d->num_kv_heads;
-    const long long target = 3LL * sm_count();
-    const long long s_target = (target + units - 1) / units;
-    long long t = s_target > 0 ? (max_blocks_needed + s_target - 1) / s_target : max_blocks_needed;
-    if (t < 2) t = 2;
+    const long long s_wave = slots / units;
+    long long t;
+    if (s_wave >= 2)
+      t = (max_blocks_needed + s_wave - 1) / s_wave;
+    else
+      t = (max_blocks_needed * units + 4 * slots - 1) / (4 * slots);
+    if (t < 1) t = 1;
     if (t > hyb::decode_max_split_blocks()) t = hyb::decode_max_split_blocks();
     tb = static_cast<int>(t);
   } else {
@@ -145,12 +154,26 @@ int hyb_decode_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_
   return HYB_OK;
 }
 
-static size_t workspace_for(const hyb_cache_desc *d, int ns) {
-  if (ns <= 1) return 0;
+// Workspace layout (ns > 1): arrival counters int32 [batch][Hkv], then the
+// split outputs FP32 [batch][Hq][ns][128], then their log2-sum-exp FP32
+// [batch][Hq][ns]; each part starts on a 256-byte boundary.
+struct WsLayout {
+  size_t counters, o_part, lse_part, total;
+};
+
+static WsLayout ws_layout(const hyb_cache_desc *d, int ns) {
+  WsLayout w{0, 0, 0, 0};
+  // one split, or few enough to merge inside a thread-block cluster: none
+  if (ns <= hyb::decode_max_cluster()) return w;
   const size_t rows = static_cast<size_t>(d->batch) * d->num_q_heads;
-  return round_up(rows * ns * hyb::kDim * sizeof(float), kWsAlign) +
-         round_up(rows * ns * sizeof(float), kWsAlign);
+  w.counters = 0;
+  w.o_part = round_up(static_cast<size_t>(d->batch) * d->num_kv_heads * sizeof(int32_t), kWsAlign);
+  w.lse_part = w.o_part + round_up(rows * ns * hyb::kDim * sizeof(float), kWsAlign);
+  w.total = w.lse_part + round_up(rows * ns * sizeof(float), kWsAlign);
+  return w;
 }
+
+static size_t workspace_for(const hyb_cache_desc *d, int ns) { return ws_layout(d, ns).total; }
 
 size_t hyb_decode_workspace_bytes(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens) {
   int32_t st = 0, ns = 0;
@@ -170,7 +193,6 @@ int hyb_decode_attn(const hyb_cache_desc *d, const void *q, float softmax_scale,
   const size_t need = workspace_for(d, ns);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16)))
     return HYB_ERR_WORKSPACE;
-  const size_t rows = static_cast<size_t>(d->batch) * d->num_q_heads;
   hyb::DecodeArgs a;
   a.hot = static_cast<const uint8_t *>(d->hot);
   a.cold = static_cast<const uint8_t *>(d->cold);
@@ -182,10 +204,12 @@ int hyb_decode_attn(const hyb_cache_desc *d, const void *q, float softmax_scale,
   a.q = static_cast<const __half *>(q);
   a.out = static_cast<__half *>(out);
   a.lse_out = lse_out;
-  a.o_part = ns > 1 ? static_cast<float *>(workspace) : nullptr;
-  a.lse_part = ns > 1 ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
-                                                  round_up(rows * ns * hyb::kDim * sizeof(float), kWsAlign))
-                      : nullptr;
+  const WsLayout wl = ws_layout(d, ns);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const bool use_ws = wl.total > 0;
+  a.counters = use_ws ? reinterpret_cast<int32_t *>(ws + wl.counters) : nullptr;
+  a.o_part = use_ws ? reinterpret_cast<float *>(ws + wl.o_part) : nullptr;
+  a.lse_part = use_ws ? reinterpret_cast<float *>(ws + wl.lse_part) : nullptr;
   a.hkv = d->num_kv_heads;
   a.hq = d->num_q_heads;
   a.num_phys = d->num_phys_blocks;
@@ -196,13 +220,8 @@ int hyb_decode_attn(const hyb_cache_desc *d, const void *q, float softmax_scale,
   a.max_seq_len = max_seq_len;
   a.qk_scale = softmax_scale * 1.4426950408889634f;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = hyb::launch_decode(a, d->num_q_heads / d->num_kv_heads, d->batch, s);
+  const cudaError_t e = hyb::launch_decode(a, d->num_q_heads / d->num_kv_heads, d->batch, s);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (ns > 1) {
-    hyb::CombineArgs c{a.o_part, a.lse_part, static_cast<__half *>(out), lse_out, ns};
-    e = hyb::launch_combine(c, static_cast<int>(rows), s);
-    if (e != cudaSuccess) return cuda_fail(e);
-  }
   return HYB_OK;
 }
 

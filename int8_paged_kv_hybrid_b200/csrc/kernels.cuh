@@ -34,7 +34,8 @@ struct DecodeArgs {
   __half *out;                // FP16 [batch][Hq][128]
   float *lse_out;             // [batch][Hq] or null
   float *o_part;              // [batch][Hq][n_splits][128] (n_splits > 1)
-  float *lse_part;            // [batch][Hq][n_splits]
+  float *lse_part;            // [batch][Hq][n_splits], log2 domain
+  int32_t *counters;          // [batch][Hkv] arrivals per (sequence, kv head), zero between calls
   int hkv, hq, num_phys, max_blocks, quant_bits, n_splits, split_blocks, max_seq_len;
   float qk_scale;             // softmax_scale * log2(e)
 };
@@ -51,5 +52,7 @@ cudaError_t launch_append(const AppendArgs &a, int batch, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, cudaStream_t stream);
 cudaError_t launch_combine(const CombineArgs &a, int rows, cudaStream_t stream);
 int decode_max_split_blocks();
+int decode_ctas_per_sm(int group);
+int decode_max_cluster();
 
 }  // namespace hyb

@@ -94,10 +94,11 @@ def _random_step_schedule(rng, lens: np.ndarray, lo: int, hi: int) -> List[np.nd
     return sched
 
 
-def make_workload(idx: int, scale_down: int = 1) -> Workload:
+def make_workload(idx: int, scale_down: int = 1, seed_offset: int = 0) -> Workload:
     """Workload `idx` in 1..5.  scale_down > 1 shrinks lengths and batch (same
-    structure) for quick tests."""
-    seed = 1000 + idx
+    structure) for quick tests; seed_offset gives an independent replica of
+    the same shapes (one per GPU in the multi-GPU benchmark)."""
+    seed = 1000 + idx + seed_offset
     rng = np.random.default_rng([seed, 0])
     d = HEAD_DIM
     n_int4 = None

@@ -95,10 +95,10 @@ def test_plan_and_workspace():
             hk.hyb_decode_plan(d, 4096, bad)
     with pytest.raises(hk.HybError):
         hk.hyb_decode_plan(d, 64 * 2048 + 33, 0)  # longer than the block table allows
-    # automatic splits: a multiple of 64 tokens, at least two blocks
+    # automatic splits: a multiple of 64 tokens, at most 8192
     for L in (33, 1000, 2048, 131072):
         st, ns = hk.hyb_decode_plan(d, L, 0)
-        assert st % 64 == 0 and st >= 128 and ns >= 1
+        assert st % 64 == 0 and 64 <= st <= 8192 and ns >= 1
         assert ns == max(1, -(-max(0, L - 32) // st))
 
 
