@@ -33,7 +33,7 @@ METRIC = "decode-attn KV GB/s (frac of HBM peak) and tokens/s at 1 B200 vs CPU o
 UNIT = "GB/s"
 WORKLOAD = 2
 PROFILE = os.path.join(ROOT, "profiles", "decode_splitkv_llama8b_b8_L2048.md")
-KERNEL_SOURCES = ["decode.cu", "common.cuh", "kernels.cuh"]
+KERNEL_SOURCES = ["decode.cu", "common.cuh", "kernels.cuh"]  # the profiled kernel's sources
 FLUSH_BYTES = 512 << 20   # > 126 MB L2
 
 
@@ -58,7 +58,7 @@ def workload_config(w, split, ns):
             "batch": int(w.batch), "seq_len": int(w.lens[0]), "num_q_heads": w.num_q_heads,
             "num_kv_heads": w.num_kv_heads, "head_dim": 128, "hot_tokens": 32, "block_size": 64,
             "quant_bits": 8, "split_tokens": split, "n_splits": ns,
-            "step": "hyb_kv_append (1 token/seq) + hyb_decode_attn",
+            "step": "hyb_decode_step: append 1 token/seq + split-KV attention, one launch",
             "l2": "flushed between timed steps (512 MB write)",
             "parallelism": "replicas (independent batch per GPU)"}
 
@@ -209,7 +209,7 @@ def run_native(args, rank, world, local_rank):
     q_d = torch.from_numpy(q).to(dev)
     out = torch.empty((w.batch, w.num_q_heads, 128), dtype=torch.float16, device=dev)
     lse = torch.empty((w.batch, w.num_q_heads), dtype=torch.float32, device=dev)
-    ws = cache.workspace(L, split)
+    ws = cache.step_workspace(L, split)
 
     # state the step changes, restored before every step (untimed)
     touched = torch.from_numpy(_touched_blocks(w, n_last)).to(dev)
@@ -228,21 +228,19 @@ def run_native(args, rank, world, local_rank):
         cache.cold.index_copy_(0, touched, snap["cold"])
 
     # one eager run (sets kernel attributes, checks the path), then capture the
-    # append and the decode as two CUDA graphs on a side stream
+    # step -- hyb_decode_step: append of the step's token + attention, one
+    # launch -- as a CUDA graph on a side stream
     side = torch.cuda.Stream(device=dev)
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
         restore()
-        cache.append(n_d, k_d, v_d)
-        cache.decode(q_d, w.softmax_scale, L, split, out=out, lse=lse, workspace=ws)
+        cache.step(n_d, k_d, v_d, q_d, w.softmax_scale, L, split, out=out, lse=lse, workspace=ws)
         restore()
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
-    g_app, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_app, stream=side):
-        cache.append(n_d, k_d, v_d)
-    with torch.cuda.graph(g_dec, stream=side):
-        cache.decode(q_d, w.softmax_scale, L, split, out=out, lse=lse, workspace=ws)
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=side):
+        cache.step(n_d, k_d, v_d, q_d, w.softmax_scale, L, split, out=out, lse=lse, workspace=ws)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
@@ -251,13 +249,11 @@ def run_native(args, rank, world, local_rank):
         for _ in range(n):
             restore()
             flush.zero_()
-            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            g_app.replay()
+            g_step.replay()
             e1.record(stream)
-            g_dec.replay()
-            e2.record(stream)
-            evs.append((e0, e1, e2))
+            evs.append((e0, e1))
         return evs
 
     timed_steps(args.warmup)
@@ -273,16 +269,14 @@ def run_native(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop() if clocks else None
-    ms_step = sum(a.elapsed_time(c) for a, b, c in evs) / len(evs)
-    ms_dec = sum(b.elapsed_time(c) for a, b, c in evs) / len(evs)
-    ms_app = sum(a.elapsed_time(b) for a, b, c in evs) / len(evs)
+    ms_step = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
     if world > 1:
-        t = torch.tensor([ms_step, ms_dec, ms_app], dtype=torch.float64, device=dev)
+        t = torch.tensor([ms_step], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, ms_dec, ms_app = t.tolist()
+        ms_step = t.item()
     assert torch.isfinite(out.float()).all() and cache.status() == 0
     if args.lean:
-        return {"lean": True, "ms_per_step": ms_step, "ms_decode": ms_dec, "ms_append": ms_app}, w
+        return {"lean": True, "ms_per_step": ms_step}, w
 
     # end to end with host buffers: pinned H2D of the step's inputs, the two
     # library calls, D2H of the output -- all inside the timed span
@@ -303,8 +297,7 @@ def run_native(args, rank, world, local_rank):
         k_d.copy_(h_k, non_blocking=True)
         v_d.copy_(h_v, non_blocking=True)
         q_d.copy_(h_q, non_blocking=True)
-        g_app.replay()
-        g_dec.replay()
+        g_step.replay()
         h_out.copy_(out, non_blocking=True)
         e1.record(stream)
         if i >= args.warmup:
@@ -315,14 +308,15 @@ def run_native(args, rank, world, local_rank):
         t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_e2e = t.item()
-    del g_app, g_dec
+    del g_step
 
     kvb = synth.kv_bytes(w)
+    stepb = kvb + synth.append_bytes(w, n_last)
     peak, peak_kind = measured_peaks()
     total_bytes = kvb * world
     value = total_bytes / (ms_step * 1e-3) / 1e9
     tokens_s = w.batch * world / (ms_step * 1e-3)
-    achieved = kvb / (ms_dec * 1e-3) / 1e9
+    achieved = stepb / (ms_step * 1e-3) / 1e9
     res = None
     if rank == 0:
         res = {
@@ -335,15 +329,16 @@ def run_native(args, rank, world, local_rank):
             "tokens_per_s_model_equiv": round(tokens_s / 32, 1),
             "kv_bytes_per_step": kvb,
             "frac_of_hbm_peak_step": round(value / world / peak, 4),
-            "ms_decode": round(ms_dec, 5), "ms_append": round(ms_app, 5),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": profiled_traffic(),
-                         "kernel": "hyb::decode_kernel<4>", "peak_kind": peak_kind,
-                         "achieved_bytes": "algorithmic KV bytes per launch (%d)" % kvb},
+                         "kernel": "hyb::decode_kernel<4,true> (fused append + attention, the step's "
+                                   "only launch)", "peak_kind": peak_kind,
+                         "achieved_bytes": "algorithmic bytes per launch: attention %d + append %d"
+                                           % (kvb, stepb - kvb)},
             "e2e": {"value": round(total_bytes / (ms_e2e * 1e-3) / 1e9, 1), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(ms_e2e, 5)},
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": args.steps,
             "clocks": clk,
         }
     return res, w

@@ -20,6 +20,8 @@
  *   hyb_decode_attn    single-query attention of q[B][Hq][d] over hot + cold,
  *                      GQA, split-KV, FP32 accumulation, FP16 output
  *                      ([hybrid_v2 page] 4.2, steps 3-5)
+ *   hyb_decode_step    the two above fused: append of one token per sequence
+ *                      and attention in a single launch
  *   hyb_combine        log-sum-exp merge of split partial results (the merge
  *                      that replaces the page's torch.cat of step 5)
  *
@@ -231,6 +233,34 @@ size_t hyb_decode_workspace_bytes(const hyb_cache_desc *desc, int32_t max_seq_le
 int hyb_decode_attn(const hyb_cache_desc *desc, const void *q, float softmax_scale,
                     int32_t max_seq_len, int32_t split_tokens, void *workspace,
                     size_t workspace_bytes, void *out, float *lse_out, hyb_stream_t stream);
+
+/*
+ * One decode step in one launch: hyb_kv_append of n_new[b] in {0, 1} tokens
+ * followed by hyb_decode_attn over the grown cache ([hybrid_v2 page] 4.2,
+ * steps 2-5 fused).  The CTA that attends a sequence's tail block and hot ring
+ * seals the token leaving the hot zone inside its staged copies (same
+ * arithmetic as hyb_kv_append, bit-exact), writes the changed codes, scale
+ * and ring slot back, and attends the updated copies; seq_lens[b] is
+ * advanced by the last CTA of the sequence.
+ *   n_new    device int32 [batch], each 0 or 1 (other values: that sequence
+ *            gets HYB_STATUS_BAD_N_NEW and is attended without appending).
+ *   k_new, v_new  device FP16 [batch][1][Hkv][D] (the hyb_kv_append layout
+ *            with max_new = 1), 16-byte aligned.
+ *   max_seq_len   host upper bound of the lengths AFTER the append.
+ *   workspace     at least hyb_decode_step_workspace_bytes() bytes (never 0:
+ *            it holds a counter per sequence), zero-filled before first use,
+ *            left ready for the next call; calls sharing it must not overlap.
+ * Other arguments and the result as for hyb_decode_attn.
+ */
+int hyb_decode_step(const hyb_cache_desc *desc, const int32_t *n_new, const void *k_new,
+                    const void *v_new, const void *q, float softmax_scale, int32_t max_seq_len,
+                    int32_t split_tokens, void *workspace, size_t workspace_bytes, void *out,
+                    float *lse_out, hyb_stream_t stream);
+
+/* Bytes of workspace hyb_decode_step needs for these arguments (0 with an
+ * invalid descriptor). */
+size_t hyb_decode_step_workspace_bytes(const hyb_cache_desc *desc, int32_t max_seq_len,
+                                       int32_t split_tokens);
 
 /*
  * Log-sum-exp merge of split partial results ([hybrid_v2 page] 4.2 step 5,

@@ -8,6 +8,7 @@ combine.  This package is its thin Python binding.
 """
 from ._lib import (  # noqa: F401
     CacheDesc, HybError, hyb_check_desc, hyb_combine, hyb_decode_attn, hyb_decode_plan,
+    hyb_decode_step, hyb_decode_step_workspace_bytes,
     hyb_decode_workspace_bytes, hyb_kv_append, hyb_last_cuda_error, hyb_read_status,
     hyb_version, load, strerror,
 )

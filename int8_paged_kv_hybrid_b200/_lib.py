@@ -28,7 +28,8 @@ HYB_STATUS_TIMEOUT = 5
 
 EXPORTED = (
     "hyb_check_desc", "hyb_kv_append", "hyb_decode_plan", "hyb_decode_workspace_bytes",
-    "hyb_decode_attn", "hyb_combine", "hyb_read_status", "hyb_strerror",
+    "hyb_decode_attn", "hyb_decode_step", "hyb_decode_step_workspace_bytes", "hyb_combine",
+    "hyb_read_status", "hyb_strerror",
     "hyb_last_cuda_error", "hyb_version",
 )
 
@@ -82,11 +83,14 @@ def load(path: str = LIB_PATH):
     lib.hyb_decode_workspace_bytes.argtypes = [D, i32, i32]
     lib.hyb_decode_workspace_bytes.restype = sz
     lib.hyb_decode_attn.argtypes = [D, P, ctypes.c_float, i32, i32, P, sz, P, P, P]
+    lib.hyb_decode_step.argtypes = [D, P, P, P, P, ctypes.c_float, i32, i32, P, sz, P, P, P]
+    lib.hyb_decode_step_workspace_bytes.argtypes = [D, i32, i32]
+    lib.hyb_decode_step_workspace_bytes.restype = sz
     lib.hyb_combine.argtypes = [i32, i32, i32, i32, P, P, P, P, P]
     lib.hyb_read_status.argtypes = [D, ctypes.POINTER(i32), i32, P]
     lib.hyb_strerror.argtypes = [ctypes.c_int]
     lib.hyb_strerror.restype = ctypes.c_char_p
-    for name in ("hyb_check_desc", "hyb_kv_append", "hyb_decode_plan", "hyb_decode_attn",
+    for name in ("hyb_check_desc", "hyb_kv_append", "hyb_decode_plan", "hyb_decode_attn", "hyb_decode_step",
                  "hyb_combine", "hyb_read_status", "hyb_last_cuda_error", "hyb_version"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -139,6 +143,19 @@ def hyb_decode_attn(desc, q, softmax_scale, max_seq_len, split_tokens, workspace
     _check(load().hyb_decode_attn(ctypes.byref(desc), _ptr(q), float(softmax_scale), int(max_seq_len),
                                   int(split_tokens), _ptr(workspace), ws_bytes, _ptr(out),
                                   _ptr(lse_out), _stream(stream)), "hyb_decode_attn")
+
+
+def hyb_decode_step_workspace_bytes(desc, max_seq_len, split_tokens=0) -> int:
+    return int(load().hyb_decode_step_workspace_bytes(ctypes.byref(desc), int(max_seq_len), int(split_tokens)))
+
+
+def hyb_decode_step(desc, n_new, k_new, v_new, q, softmax_scale, max_seq_len, split_tokens, workspace,
+                    out, lse_out=None, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().hyb_decode_step(ctypes.byref(desc), _ptr(n_new), _ptr(k_new), _ptr(v_new), _ptr(q),
+                                  float(softmax_scale), int(max_seq_len), int(split_tokens),
+                                  _ptr(workspace), ws_bytes, _ptr(out), _ptr(lse_out), _stream(stream)),
+           "hyb_decode_step")
 
 
 def hyb_combine(batch, num_q_heads, head_dim, n_splits, o_partial, lse_partial, out,

@@ -84,6 +84,25 @@ class HybridKVCache:
                              out, lse, stream)
         return out
 
+    def step_workspace(self, max_seq_len, split_tokens=0):
+        import torch
+        n = _lib.hyb_decode_step_workspace_bytes(self.desc, max_seq_len, split_tokens)
+        return torch.zeros(max(n, 16), dtype=torch.uint8, device=self.device)
+
+    def step(self, n_new, k_new, v_new, q, softmax_scale, max_seq_len, split_tokens=0, out=None,
+             lse=None, workspace=None, stream=None):
+        """Fused decode step: append n_new[b] in {0, 1} tokens (k_new, v_new FP16
+        [batch][1][Hkv][128]) and attend q; max_seq_len bounds the new lengths."""
+        import torch
+        assert q.is_contiguous() and k_new.is_contiguous() and v_new.is_contiguous()
+        if out is None:
+            out = torch.empty((self.batch, self.hq, HEAD_DIM), dtype=torch.float16, device=self.device)
+        if workspace is None:
+            workspace = self.step_workspace(max_seq_len, split_tokens)
+        _lib.hyb_decode_step(self.desc, n_new, k_new, v_new, q, softmax_scale, max_seq_len, split_tokens,
+                             workspace, out, lse, stream)
+        return out
+
     def status(self, clear=False, stream=None):
         return _lib.hyb_read_status(self.desc, clear, stream)
 

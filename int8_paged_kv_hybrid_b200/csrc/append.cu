@@ -19,25 +19,6 @@
 
 namespace hyb {
 
-__device__ __forceinline__ int quantize(float x, float s, int q) {
-  if (s == 0.f) return 0;
-  return clamp_code(__float2int_rn(__fdiv_rn(x, s)), q);
-}
-
-__device__ __forceinline__ int requantize(int c, float s_old, float s_new, int q) {
-  return clamp_code(__float2int_rn(__fdiv_rn(__fmul_rn(static_cast<float>(c), s_old), s_new)), q);
-}
-
-__device__ __forceinline__ int nib_get(uint32_t w, int e) {
-  const int v = (w >> (8 * (e & 3) + 4 * (e >> 2))) & 0xf;
-  return v >= 8 ? v - 16 : v;
-}
-
-__device__ __forceinline__ uint32_t nib_put(uint32_t w, int e, int c) {
-  const int sh = 8 * (e & 3) + 4 * (e >> 2);
-  return (w & ~(0xfu << sh)) | (static_cast<uint32_t>(c & 0xf) << sh);
-}
-
 // Re-quantize the codes of slots [0, first) of one tile from s_old to s_new.
 // Every possible code is re-quantized once (table in shared memory, same
 // arithmetic as requantize()); the tile is then rewritten by lookup, with
@@ -48,8 +29,7 @@ __device__ void requant_tile(uint8_t *tile, int kv, bool int4, int first, float 
     tbl[c + 127] = static_cast<int8_t>(requantize(c, s_old, s_new, q));
   __syncwarp();
   uint32_t *w32 = reinterpret_cast<uint32_t *>(tile);
-  // words of the tile that can hold sealed slots, by layout
-  const int nwords = !int4 ? (kv == 0 ? first * 32 : kTileBytes / 4) : (kv == 0 ? first * 16 : kTileBytes / 8);
+  const int nwords = requant_nwords(kv, int4, first);
   constexpr int kBatch = 16;
   for (int w0 = lane; w0 < nwords; w0 += 32 * kBatch) {
     uint32_t x[kBatch];
@@ -61,28 +41,7 @@ __device__ void requant_tile(uint8_t *tile, int kv, bool int4, int first, float 
 #pragma unroll
     for (int j = 0; j < kBatch; j++) {
       const int w = w0 + 32 * j;
-      if (w >= nwords) continue;
-      uint32_t y = x[j];
-      if (!int4) {
-        // slot of byte e: token-major -> all sealed; channel-major -> 16*chunk + 4*(w%4) + e
-        const int row = w >> 4;
-        const int base = kv == 0 ? 0 : 16 * (((w >> 2) & 3) ^ ((row >> 1) & 3)) + 4 * (w & 3);
-#pragma unroll
-        for (int e = 0; e < 4; e++) {
-          if (kv != 0 && base + e >= first) continue;
-          const int c = static_cast<int8_t>((x[j] >> (8 * e)) & 0xff);
-          y = (y & ~(0xffu << (8 * e))) | (static_cast<uint32_t>(static_cast<uint8_t>(tbl[c + 127])) << (8 * e));
-        }
-      } else {
-        const int row = w >> 3;
-        const int base = kv == 0 ? 0 : 16 * (((w >> 1) & 3) ^ ((row >> 2) & 3)) + 8 * (w & 1);
-#pragma unroll
-        for (int e = 0; e < 8; e++) {
-          if (kv != 0 && base + e >= first) continue;
-          y = nib_put(y, e, tbl[nib_get(x[j], e) + 127]);
-        }
-      }
-      w32[w] = y;
+      if (w < nwords) w32[w] = requant_word(x[j], w, kv, int4, first, tbl);
     }
   }
   __syncwarp();

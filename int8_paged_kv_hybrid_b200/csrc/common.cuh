@@ -98,4 +98,63 @@ __device__ __forceinline__ uint32_t sext_nibbles(uint32_t u) {
 
 __device__ __forceinline__ int clamp_code(int v, int q) { return v > q ? q : (v < -q ? -q : v); }
 
+// ---- the cold-zone quantizer (IEEE division, round half to even, clamp) ----
+// code of x under scale s; a zero scale (all-zero group) gives code 0
+__device__ __forceinline__ int quantize(float x, float s, int q) {
+  if (s == 0.f) return 0;
+  return clamp_code(__float2int_rn(__fdiv_rn(x, s)), q);
+}
+
+// a code sealed under s_old, re-expressed under the larger scale s_new
+__device__ __forceinline__ int requantize(int c, float s_old, float s_new, int q) {
+  return clamp_code(__float2int_rn(__fdiv_rn(__fmul_rn(static_cast<float>(c), s_old), s_new)), q);
+}
+
+// INT4 packing: element e (0..7) of a 32-bit word is byte e%4, low nibble for
+// e < 4, high nibble for e >= 4 (4-bit two's complement)
+__device__ __forceinline__ int nib_get(uint32_t w, int e) {
+  const int v = (w >> (8 * (e & 3) + 4 * (e >> 2))) & 0xf;
+  return v >= 8 ? v - 16 : v;
+}
+
+__device__ __forceinline__ uint32_t nib_put(uint32_t w, int e, int c) {
+  const int sh = 8 * (e & 3) + 4 * (e >> 2);
+  return (w & ~(0xfu << sh)) | (static_cast<uint32_t>(c & 0xf) << sh);
+}
+
+// Re-quantization of the codes already in a tile.  `tbl` maps every code c
+// to its re-quantized value tbl[c + 127]; only codes of slots < first change.
+// Words of a tile, by layout: INT8 K token-major (32 words per slot), INT8 V
+// channel-major with swizzled 16-byte chunks (16 words per channel row), INT4
+// K (16 words per slot), INT4 V (8 words per channel row, swizzled 8-byte
+// units).  requant_nwords() is the number of leading words that can hold
+// sealed codes.
+__device__ __forceinline__ int requant_nwords(int kv, bool int4, int first) {
+  return !int4 ? (kv == 0 ? first * 32 : kTileBytes / 4) : (kv == 0 ? first * 16 : kTileBytes / 8);
+}
+
+__device__ __forceinline__ uint32_t requant_word(uint32_t x, int w, int kv, bool int4, int first,
+                                                 const int8_t *tbl) {
+  uint32_t y = x;
+  if (!int4) {
+    const int row = w >> 4;
+    const int base = kv == 0 ? 0 : 16 * (((w >> 2) & 3) ^ ((row >> 1) & 3)) + 4 * (w & 3);
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      if (kv != 0 && base + e >= first) continue;
+      const int c = static_cast<int8_t>((x >> (8 * e)) & 0xff);
+      y = (y & ~(0xffu << (8 * e))) | (static_cast<uint32_t>(static_cast<uint8_t>(tbl[c + 127])) << (8 * e));
+    }
+  } else {
+    const int row = w >> 3;
+    const int base = kv == 0 ? 0 : 16 * (((w >> 1) & 3) ^ ((row >> 2) & 3)) + 8 * (w & 1);
+#pragma unroll
+    for (int e = 0; e < 8; e++) {
+      if (kv != 0 && base + e >= first) continue;
+      y = nib_put(y, e, tbl[nib_get(x, e) + 127]);
+    }
+  }
+  return y;
+}
+
 }  // namespace hyb

@@ -70,6 +70,9 @@ struct DecodeSmem {
   float wsum[kWarps][G];
   float mrun[kWarps][G];
   float lrun[kWarps][G];
+  int8_t rqt[2][256];  // fused step: re-quantization tables of the tail block (K, V)
+  float seal_s[2];     // fused step: the tail block's scales after sealing
+  int seal_rq[2];      // fused step: 1 if the tail block's codes were re-quantized
   float cl_l[G];   // this split's log2-sum-exp per head, read by the cluster's merge
   float mfin[G];   // final merge: max and sum of the split weights per head
   float dfin[G];
@@ -135,6 +138,122 @@ __device__ __forceinline__ void unpack_int4(uint32_t x, uint32_t &lo, uint32_t &
   hi = sext_nibbles((x >> 4) & 0x0f0f0f0fu);
 }
 
+// Fused decode step: append the sequence's new token inside the staged copies
+// of the tail block (item ncold-1) and the hot ring (item ncold), with the
+// arithmetic of hyb_kv_append (bit-exact), and write back what changed.  All
+// threads of the CTA call it.
+template <int G>
+__device__ __noinline__ void fused_append(DecodeSmem<G> &sm, const DecodeArgs &a, int b, int h, int L_old,
+                                          int i0, int ncold, int n_int4_b, bool do_seal, __half2 new_kv,
+                                          int tid, int warp, int lane) {
+  uint8_t *hot_st = sm.ring[ncold % kStages];
+  const int rs = L_old % kHot;  // ring slot of the evicted and of the new token
+  const int e = L_old - kHot;   // position sealed (when do_seal)
+  const int slot = do_seal ? e % kBlock : 0;
+  const int ti = do_seal ? ncold - 1 : 0;  // tail item of this split
+  const bool int4 = do_seal && (i0 + ti) < n_int4_b;
+  const int Q = int4 ? 7 : 127;
+  uint8_t *tile_st = sm.ring[ti % kStages];
+  if (do_seal && warp < 2) {
+    // warp 0: K, warp 1: V -- absmax of the evicted token, new scale
+    const int kv = warp;
+    const __half *row = reinterpret_cast<const __half *>(hot_st + rs * kHotTokenBytes) + kv * kDim;
+    float amax = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; j++) amax = fmaxf(amax, fabsf(__half2float(row[4 * lane + j])));
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+    const float s_c = __fdiv_rn(amax, static_cast<float>(Q));
+    const float s_old = kv ? sm.scl[ti].y : sm.scl[ti].x;
+    float s_new = s_c;
+    int rq = 0;
+    if (slot != 0) {
+      if (s_c > s_old) rq = 1;
+      else s_new = s_old;
+    }
+    if (rq)
+      for (int c = lane - 127; c <= 127; c += 32)
+        sm.rqt[kv][c + 127] = static_cast<int8_t>(requantize(c, s_old, s_new, Q));
+    if (lane == 0) {
+      sm.seal_s[kv] = s_new;
+      sm.seal_rq[kv] = rq;
+    }
+  }
+  __syncthreads();
+  if (do_seal && tid == 0) sm.scl[ti] = make_float2(sm.seal_s[0], sm.seal_s[1]);  // attention uses these
+  if (do_seal) {
+    // codes already in the tail block, under a grown scale
+#pragma unroll
+    for (int kv = 0; kv < 2; kv++) {
+      if (!sm.seal_rq[kv]) continue;
+      uint32_t *w32 = reinterpret_cast<uint32_t *>(tile_st + kv * kTileBytes);
+      const int nw = requant_nwords(kv, int4, slot);
+      for (int w = tid; w < nw; w += kThreads) w32[w] = requant_word(w32[w], w, kv, int4, slot, sm.rqt[kv]);
+    }
+  }
+  __syncthreads();
+  const int c = tid;  // channel
+  if (do_seal) {
+    // the evicted token's codes into slot `slot`
+    const __half *krow = reinterpret_cast<const __half *>(hot_st + rs * kHotTokenBytes);
+    const int ck = quantize(__half2float(krow[c]), sm.seal_s[0], Q);
+    const int cv = quantize(__half2float(krow[kDim + c]), sm.seal_s[1], Q);
+    if (!int4) {
+      tile_st[slot * kDim + c] = static_cast<uint8_t>(ck);
+      tile_st[kTileBytes + c * 64 + 16 * ((slot >> 4) ^ ((c >> 1) & 3)) + (slot & 15)] = static_cast<uint8_t>(cv);
+    } else {
+      // K: channels c and c+4 of an 8-channel group share a byte; the thread of
+      // the lower one writes both (its partner's code comes by shuffle)
+      const int ck_hi = __shfl_down_sync(0xffffffffu, ck, 4);
+      if ((c & 4) == 0) {
+        uint8_t *byte = tile_st + slot * 64 + 4 * (c >> 3) + (c & 3);
+        *byte = static_cast<uint8_t>((ck & 0xf) | ((ck_hi & 0xf) << 4));
+      }
+      const int unit = (slot >> 4) ^ ((c >> 2) & 3);
+      const int in = slot & 15;
+      uint8_t *byte = tile_st + kTileBytes + c * 32 + unit * 8 + (in >> 3) * 4 + (in & 3);
+      *byte = (in & 4) ? static_cast<uint8_t>((*byte & 0x0f) | ((cv & 0xf) << 4))
+                       : static_cast<uint8_t>((*byte & 0xf0) | (cv & 0xf));
+    }
+  }
+  __syncthreads();
+  // the new token into the ring slot: the staged copy (for this attention) and the cache
+  {
+    __half *srow = reinterpret_cast<__half *>(hot_st + rs * kHotTokenBytes);
+    srow[c] = __low2half(new_kv);
+    srow[kDim + c] = __high2half(new_kv);
+    __half *grow = reinterpret_cast<__half *>(a.hot) + ((((size_t)b * a.hkv + h) * kHot + rs) * 2) * kDim;
+    grow[c] = __low2half(new_kv);
+    grow[kDim + c] = __high2half(new_kv);
+  }
+  if (do_seal) {
+    // write back what changed in the tail block: scales, then the whole tile
+    // if its codes were re-quantized, else the sealed token's codes
+    const int phys = sm.phys[ti];
+    uint8_t *gtile = a.cold + ((size_t)phys * a.hkv + h) * kTilePairBytes;
+    if (tid < 2) a.scales[((size_t)phys * a.hkv + h) * 2 + tid] = sm.seal_s[tid];
+#pragma unroll
+    for (int kv = 0; kv < 2; kv++) {
+      uint8_t *g = gtile + kv * kTileBytes;
+      const uint8_t *t = tile_st + kv * kTileBytes;
+      if (sm.seal_rq[kv]) {
+        const int nvec = (int4 ? kTileBytes / 2 : kTileBytes) / 16;
+        for (int v = tid; v < nvec; v += kThreads)
+          reinterpret_cast<uint4 *>(g)[v] = reinterpret_cast<const uint4 *>(t)[v];
+      } else if (kv == 0) {
+        const int rowb = int4 ? 64 : kDim;
+        if (tid * 16 < rowb)
+          reinterpret_cast<uint4 *>(g + slot * rowb)[tid] = reinterpret_cast<const uint4 *>(t + slot * rowb)[tid];
+      } else {
+        const int off = !int4 ? c * 64 + 16 * ((slot >> 4) ^ ((c >> 1) & 3)) + (slot & 15)
+                              : c * 32 + 8 * ((slot >> 4) ^ ((c >> 2) & 3)) + ((slot & 15) >> 3) * 4 + (slot & 3);
+        g[off] = t[off];
+      }
+    }
+  }
+  __syncthreads();
+}
+
 // kCluster: the grid is launched in clusters of n_splits CTAs (the splits of
 // one (sequence, kv head)); splits are merged through distributed shared
 // memory instead of the workspace.
@@ -152,7 +271,8 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 2)) decode_kernel(cons
 
   // independent loads first: the sequence length, this split's block-table
   // entries (one per thread, clamped to the row) and q
-  int L = a.seq_lens[b];
+  const int L_old = a.seq_lens[b];
+  int n_app = a.n_new ? a.n_new[b] : 0;  // fused step: tokens appended to this sequence
   const int i_tid = i0 + tid;
   const int phys_raw =
       (tid < a.split_blocks && i_tid < a.max_blocks) ? a.block_table[(size_t)b * a.max_blocks + i_tid] : -1;
@@ -160,10 +280,25 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 2)) decode_kernel(cons
 #pragma unroll
   for (int j = 0; j < G; j++) qv[j] = __half2float(a.q[((size_t)b * a.hq + hq0) * kDim + j * kDim + tid]);
 
-  if (L < 0 || L > a.max_seq_len) {
-    // sequence skipped: treated as empty (zero output, lse -inf)
+  if (n_app < 0 || n_app > 1) {
+    if (tid == 0 && s == 0 && h == 0) set_status(a.status, HYB_STATUS_BAD_N_NEW);
+    n_app = 0;
+  }
+  int L = L_old + n_app;
+  if (L_old < 0 || L > a.max_seq_len) {
+    // sequence skipped: treated as empty (zero output, lse -inf), not appended to
     if (tid == 0 && s == 0 && h == 0) set_status(a.status, HYB_STATUS_SEQ_LEN);
     L = 0;
+    n_app = 0;
+  }
+  if (a.n_new && tid == 32) {
+    // every CTA of the grid has read seq_lens[b] once this count is complete;
+    // the last one advances it
+    const int ticket = atomicAdd(&a.seq_cnt[b], 1);
+    if (ticket == static_cast<int>(gridDim.x * gridDim.y) - 1) {
+      a.seq_lens[b] = L_old + n_app;
+      a.seq_cnt[b] = 0;
+    }
   }
   const int Lc = max(0, L - kHot);
   const int nblk = (Lc + kBlock - 1) / kBlock;
@@ -174,6 +309,17 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 2)) decode_kernel(cons
   const int ncold = max(0, min(nblk, i0 + a.split_blocks) - i0);
   const int nhot = (s == Sb - 1) ? min(L, kHot) : 0;
   const int nitems = ncold + (nhot > 0 ? 1 : 0);
+  // fused step, in the split that holds the tail block and the hot ring: the
+  // new token goes to ring slot L_old % 32 (whose old occupant, position
+  // L_old - 32, is sealed into the tail block first)
+  const bool do_ring = n_app == 1 && nhot > 0;
+  const bool do_seal = do_ring && L_old >= kHot;
+  const int k_fused = do_seal ? ncold - 1 : ncold;  // item at which the append is done
+  __half2 new_kv = __halves2half2(__float2half_rn(0.f), __float2half_rn(0.f));
+  if (do_ring) {
+    const size_t o = ((size_t)b * a.hkv + h) * kDim + tid;
+    new_kv = __halves2half2(a.k_new[o], a.v_new[o]);
+  }
   const int n_int4_b = a.quant_bits == 4 ? 0x7fffffff : (a.n_int4 ? a.n_int4[b] : 0);
 
   if (tid == 0) {
@@ -281,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 2)) decode_kernel(cons
     if (tid == 0) {
       for (; next_issue < min(nitems, k + kStages); next_issue++) {
         const int j = next_issue - kStages;  // previous item of that stage
-        if (next_issue <= k) {
+        if (next_issue <= k + ((do_ring && k == k_fused) ? 1 : 0)) {
           if (!mbar_wait_bounded(&sm.empty[j % kStages], (j / kStages) & 1, kWaitCycles)) {
             set_status(a.status, HYB_STATUS_TIMEOUT);
             sm.abort_flag = 1;
@@ -296,6 +442,13 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 2)) decode_kernel(cons
     }
     bool ok = mbar_wait_bounded(&sm.full[st], (k / kStages) & 1, kWaitCycles);
     if (!ok && lane == 0) set_status(a.status, HYB_STATUS_TIMEOUT);
+    if (do_ring && k == k_fused) {
+      // ---------------- fused append (whole CTA, in the staged copies) ----------------
+      const int kh = ncold;  // the hot item
+      if (k != kh) ok = ok && mbar_wait_bounded(&sm.full[kh % kStages], (kh / kStages) & 1, kWaitCycles);
+      ok = __syncthreads_and(ok) != 0;
+      if (ok) fused_append<G>(sm, a, b, h, L_old, i0, ncold, n_int4_b, do_seal, new_kv, tid, warp, lane);
+    }
     ok = ok && *reinterpret_cast<volatile int *>(&sm.abort_flag) == 0;
     const uint8_t *stage = sm.ring[st];
     if (ok && k < ncold) {

@@ -154,26 +154,33 @@ int hyb_decode_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_
   return HYB_OK;
 }
 
-// Workspace layout (ns > 1): arrival counters int32 [batch][Hkv], then the
+// Workspace layout.  Fused step only: read counters int32 [batch].  With more
+// splits than one cluster holds: arrival counters int32 [batch][Hkv], then the
 // split outputs FP32 [batch][Hq][ns][128], then their log2-sum-exp FP32
-// [batch][Hq][ns]; each part starts on a 256-byte boundary.
+// [batch][Hq][ns].  Each part starts on a 256-byte boundary.
 struct WsLayout {
-  size_t counters, o_part, lse_part, total;
+  size_t seq_cnt, counters, o_part, lse_part, total;
 };
 
-static WsLayout ws_layout(const hyb_cache_desc *d, int ns) {
-  WsLayout w{0, 0, 0, 0};
-  // one split, or few enough to merge inside a thread-block cluster: none
-  if (ns <= hyb::decode_max_cluster()) return w;
-  const size_t rows = static_cast<size_t>(d->batch) * d->num_q_heads;
-  w.counters = 0;
-  w.o_part = round_up(static_cast<size_t>(d->batch) * d->num_kv_heads * sizeof(int32_t), kWsAlign);
-  w.lse_part = w.o_part + round_up(rows * ns * hyb::kDim * sizeof(float), kWsAlign);
-  w.total = w.lse_part + round_up(rows * ns * sizeof(float), kWsAlign);
+static WsLayout ws_layout(const hyb_cache_desc *d, int ns, bool step) {
+  WsLayout w{0, 0, 0, 0, 0};
+  size_t off = 0;
+  if (step) {
+    w.seq_cnt = 0;
+    off = round_up(static_cast<size_t>(d->batch) * sizeof(int32_t), kWsAlign);
+  }
+  if (ns > hyb::decode_max_cluster()) {
+    const size_t rows = static_cast<size_t>(d->batch) * d->num_q_heads;
+    w.counters = off;
+    w.o_part = off + round_up(static_cast<size_t>(d->batch) * d->num_kv_heads * sizeof(int32_t), kWsAlign);
+    w.lse_part = w.o_part + round_up(rows * ns * hyb::kDim * sizeof(float), kWsAlign);
+    off = w.lse_part + round_up(rows * ns * sizeof(float), kWsAlign);
+  }
+  w.total = off;
   return w;
 }
 
-static size_t workspace_for(const hyb_cache_desc *d, int ns) { return ws_layout(d, ns).total; }
+static size_t workspace_for(const hyb_cache_desc *d, int ns) { return ws_layout(d, ns, false).total; }
 
 size_t hyb_decode_workspace_bytes(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens) {
   int32_t st = 0, ns = 0;
@@ -181,21 +188,25 @@ size_t hyb_decode_workspace_bytes(const hyb_cache_desc *d, int32_t max_seq_len, 
   return workspace_for(d, ns);
 }
 
-int hyb_decode_attn(const hyb_cache_desc *d, const void *q, float softmax_scale, int32_t max_seq_len,
-                    int32_t split_tokens, void *workspace, size_t workspace_bytes, void *out,
-                    float *lse_out, hyb_stream_t stream) {
+static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_scale, int32_t max_seq_len,
+                         int32_t split_tokens, void *workspace, size_t workspace_bytes, void *out,
+                         float *lse_out, hyb_stream_t stream, const int32_t *n_new, const void *k_new,
+                         const void *v_new) {
   int32_t st = 0, ns = 0;
   const int rc = hyb_decode_plan(d, max_seq_len, split_tokens, &st, &ns);
   if (rc != HYB_OK) return rc;
   if (!q || !out || !aligned(q, 16) || !aligned(out, 16) || (lse_out && !aligned(lse_out, 4)) ||
       !std::isfinite(softmax_scale))
     return HYB_ERR_INVALID_VALUE;
-  const size_t need = workspace_for(d, ns);
-  if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16)))
+  const bool step = n_new != nullptr;
+  if (step && (!aligned(n_new, 4) || !k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)))
+    return HYB_ERR_INVALID_VALUE;
+  const WsLayout wl = ws_layout(d, ns, step);
+  if (wl.total > 0 && (!workspace || workspace_bytes < wl.total || !aligned(workspace, 16)))
     return HYB_ERR_WORKSPACE;
   hyb::DecodeArgs a;
-  a.hot = static_cast<const uint8_t *>(d->hot);
-  a.cold = static_cast<const uint8_t *>(d->cold);
+  a.hot = static_cast<uint8_t *>(d->hot);
+  a.cold = static_cast<uint8_t *>(d->cold);
   a.scales = d->scales;
   a.block_table = d->block_table;
   a.seq_lens = d->seq_lens;
@@ -204,12 +215,11 @@ int hyb_decode_attn(const hyb_cache_desc *d, const void *q, float softmax_scale,
   a.q = static_cast<const __half *>(q);
   a.out = static_cast<__half *>(out);
   a.lse_out = lse_out;
-  const WsLayout wl = ws_layout(d, ns);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  const bool use_ws = wl.total > 0;
-  a.counters = use_ws ? reinterpret_cast<int32_t *>(ws + wl.counters) : nullptr;
-  a.o_part = use_ws ? reinterpret_cast<float *>(ws + wl.o_part) : nullptr;
-  a.lse_part = use_ws ? reinterpret_cast<float *>(ws + wl.lse_part) : nullptr;
+  const bool merge_ws = ns > hyb::decode_max_cluster();
+  a.counters = merge_ws ? reinterpret_cast<int32_t *>(ws + wl.counters) : nullptr;
+  a.o_part = merge_ws ? reinterpret_cast<float *>(ws + wl.o_part) : nullptr;
+  a.lse_part = merge_ws ? reinterpret_cast<float *>(ws + wl.lse_part) : nullptr;
   a.hkv = d->num_kv_heads;
   a.hq = d->num_q_heads;
   a.num_phys = d->num_phys_blocks;
@@ -219,10 +229,35 @@ int hyb_decode_attn(const hyb_cache_desc *d, const void *q, float softmax_scale,
   a.split_blocks = st / hyb::kBlock;
   a.max_seq_len = max_seq_len;
   a.qk_scale = softmax_scale * 1.4426950408889634f;
+  a.n_new = n_new;
+  a.k_new = static_cast<const __half *>(k_new);
+  a.v_new = static_cast<const __half *>(v_new);
+  a.seq_cnt = step ? reinterpret_cast<int32_t *>(ws + wl.seq_cnt) : nullptr;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const cudaError_t e = hyb::launch_decode(a, d->num_q_heads / d->num_kv_heads, d->batch, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return HYB_OK;
+}
+
+int hyb_decode_attn(const hyb_cache_desc *d, const void *q, float softmax_scale, int32_t max_seq_len,
+                    int32_t split_tokens, void *workspace, size_t workspace_bytes, void *out,
+                    float *lse_out, hyb_stream_t stream) {
+  return decode_launch(d, q, softmax_scale, max_seq_len, split_tokens, workspace, workspace_bytes, out,
+                       lse_out, stream, nullptr, nullptr, nullptr);
+}
+
+size_t hyb_decode_step_workspace_bytes(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens) {
+  int32_t st = 0, ns = 0;
+  if (hyb_decode_plan(d, max_seq_len, split_tokens, &st, &ns) != HYB_OK) return 0;
+  return ws_layout(d, ns, true).total;
+}
+
+int hyb_decode_step(const hyb_cache_desc *d, const int32_t *n_new, const void *k_new, const void *v_new,
+                    const void *q, float softmax_scale, int32_t max_seq_len, int32_t split_tokens,
+                    void *workspace, size_t workspace_bytes, void *out, float *lse_out, hyb_stream_t stream) {
+  if (!n_new) return HYB_ERR_INVALID_VALUE;
+  return decode_launch(d, q, softmax_scale, max_seq_len, split_tokens, workspace, workspace_bytes, out,
+                       lse_out, stream, n_new, k_new, v_new);
 }
 
 int hyb_combine(int32_t batch, int32_t num_q_heads, int32_t head_dim, int32_t n_splits,

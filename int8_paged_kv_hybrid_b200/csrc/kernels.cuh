@@ -23,11 +23,11 @@ struct AppendArgs {
 };
 
 struct DecodeArgs {
-  const uint8_t *hot;
-  const uint8_t *cold;
-  const float *scales;
+  uint8_t *hot;               // written only by the fused step (new token)
+  uint8_t *cold;              // written only by the fused step (sealed token)
+  float *scales;
   const int32_t *block_table;
-  const int32_t *seq_lens;
+  int32_t *seq_lens;          // advanced only by the fused step
   const int32_t *n_int4;
   int32_t *status;
   const __half *q;            // FP16 [batch][Hq][128]
@@ -38,6 +38,13 @@ struct DecodeArgs {
   int32_t *counters;          // [batch][Hkv] arrivals per (sequence, kv head), zero between calls
   int hkv, hq, num_phys, max_blocks, quant_bits, n_splits, split_blocks, max_seq_len;
   float qk_scale;             // softmax_scale * log2(e)
+  // fused decode step (null for attention only): append n_new[b] in {0, 1}
+  // tokens first; k_new / v_new FP16 [batch][Hkv][128]; seq_cnt [batch]
+  // counts the CTAs that have read seq_lens[b] (zero between calls)
+  const int32_t *n_new;
+  const __half *k_new;
+  const __half *v_new;
+  int32_t *seq_cnt;
 };
 
 struct CombineArgs {

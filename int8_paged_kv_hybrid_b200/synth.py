@@ -259,3 +259,19 @@ def custom_workload(name, lens, num_q_heads, num_kv_heads, seed, softmax_scale=N
                     n_int4=None if n_int4 is None else np.asarray(n_int4, np.int32),
                     schedule=sched, max_new=mx, seed=seed, outlier_channels=outl,
                     split_tokens=split_tokens)
+
+
+def append_bytes(w: Workload, n_new: np.ndarray) -> int:
+    """Algorithmic bytes of appending n_new[b] in {0, 1} tokens beyond what the
+    attention pass reads anyway (the evicted token and the tail block are in
+    the attention bytes): the new token's FP16 K and V read (512 B per kv
+    head) and written to the hot ring (512 B), the sealed token's codes
+    written (256 B at INT8) and the two scales (8 B), per kv head."""
+    total = 0
+    for b, n in enumerate(np.asarray(n_new)):
+        if int(n) == 0:
+            continue
+        L_old = int(w.lens[b]) - int(n)
+        per_head = 512 + 512 + ((256 + 8) if L_old >= HOT else 0)
+        total += w.num_kv_heads * per_head
+    return total
