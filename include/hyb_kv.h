@@ -61,6 +61,8 @@ typedef struct CUstream_st *hyb_stream_t; /* same type as cudaStream_t */
                                       block_size != 64, head_dim != 128, Hq/Hkv > 8 */
 #define HYB_ERR_WORKSPACE (-3)     /* workspace missing or smaller than required */
 #define HYB_ERR_CUDA (-4)          /* a CUDA runtime call or launch failed */
+#define HYB_ERR_SCRATCH_LIMIT (-5) /* hyb_decode_attn_noalloc: the call needs more scratch
+                                      than the library's static buffer holds */
 
 /* device status codes (sticky, first error wins) */
 #define HYB_STATUS_OK 0
@@ -233,6 +235,34 @@ size_t hyb_decode_workspace_bytes(const hyb_cache_desc *desc, int32_t max_seq_le
 int hyb_decode_attn(const hyb_cache_desc *desc, const void *q, float softmax_scale,
                     int32_t max_seq_len, int32_t split_tokens, void *workspace,
                     size_t workspace_bytes, void *out, float *lse_out, hyb_stream_t stream);
+
+/*
+ * hyb_decode_attn without a caller-provided workspace (the pages have no
+ * counterpart: this is an integration convenience).  For callers that cannot
+ * allocate device memory when they run attention -- code handed a fixed
+ * device-memory budget at start-up, plugins whose host application owns the
+ * allocator, decode loops where an allocation could block or fail -- the
+ * scratch comes from one static device array compiled into the library
+ * (hyb_noalloc_scratch_limit() bytes, 4 MiB, held by every GPU that loads the
+ * library until the process exits).  Same arguments and results as
+ * hyb_decode_attn minus the workspace.
+ *   - Allocates nothing (no cudaMalloc / cudaFree).
+ *   - The first call on a device looks up the array's device address for that
+ *     device; make that first call before any stream capture on the device.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     contents; each call clears the part that must start at zero.  Calls
+ *     that overlap on the GPU race on the array: order them (one stream, or
+ *     events).
+ *   - Returns HYB_ERR_SCRATCH_LIMIT, enqueuing nothing, when the problem
+ *     needs more scratch than the limit (hyb_decode_workspace_bytes() >
+ *     hyb_noalloc_scratch_limit()).
+ */
+int hyb_decode_attn_noalloc(const hyb_cache_desc *desc, const void *q, float softmax_scale,
+                            int32_t max_seq_len, int32_t split_tokens, void *out, float *lse_out,
+                            hyb_stream_t stream);
+
+/* Bytes of the static scratch array behind hyb_decode_attn_noalloc. */
+size_t hyb_noalloc_scratch_limit(void);
 
 /*
  * One decode step in one launch: hyb_kv_append of n_new[b] in {0, 1} tokens

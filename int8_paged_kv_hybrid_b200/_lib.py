@@ -18,6 +18,7 @@ HYB_ERR_INVALID_VALUE = -1
 HYB_ERR_UNSUPPORTED = -2
 HYB_ERR_WORKSPACE = -3
 HYB_ERR_CUDA = -4
+HYB_ERR_SCRATCH_LIMIT = -5
 
 HYB_STATUS_OK = 0
 HYB_STATUS_BAD_BLOCK = 1
@@ -30,7 +31,7 @@ EXPORTED = (
     "hyb_check_desc", "hyb_kv_append", "hyb_decode_plan", "hyb_decode_workspace_bytes",
     "hyb_decode_attn", "hyb_decode_step", "hyb_decode_step_workspace_bytes", "hyb_combine",
     "hyb_read_status", "hyb_strerror",
-    "hyb_last_cuda_error", "hyb_version",
+    "hyb_last_cuda_error", "hyb_version", "hyb_decode_attn_noalloc", "hyb_noalloc_scratch_limit",
 )
 
 
@@ -87,6 +88,10 @@ def load(path: str = LIB_PATH):
     lib.hyb_decode_step_workspace_bytes.argtypes = [D, i32, i32]
     lib.hyb_decode_step_workspace_bytes.restype = sz
     lib.hyb_combine.argtypes = [i32, i32, i32, i32, P, P, P, P, P]
+    lib.hyb_decode_attn_noalloc.argtypes = [D, P, ctypes.c_float, i32, i32, P, P, P]
+    lib.hyb_decode_attn_noalloc.restype = ctypes.c_int
+    lib.hyb_noalloc_scratch_limit.argtypes = []
+    lib.hyb_noalloc_scratch_limit.restype = sz
     lib.hyb_read_status.argtypes = [D, ctypes.POINTER(i32), i32, P]
     lib.hyb_strerror.argtypes = [ctypes.c_int]
     lib.hyb_strerror.restype = ctypes.c_char_p
@@ -156,6 +161,19 @@ def hyb_decode_step(desc, n_new, k_new, v_new, q, softmax_scale, max_seq_len, sp
                                   float(softmax_scale), int(max_seq_len), int(split_tokens),
                                   _ptr(workspace), ws_bytes, _ptr(out), _ptr(lse_out), _stream(stream)),
            "hyb_decode_step")
+
+
+def hyb_decode_attn_noalloc(desc, q, softmax_scale, max_seq_len, split_tokens, out, lse_out=None,
+                            stream=None):
+    """hyb_decode_attn with the library's static scratch buffer instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    _check(load().hyb_decode_attn_noalloc(ctypes.byref(desc), _ptr(q), float(softmax_scale),
+                                          int(max_seq_len), int(split_tokens), _ptr(out), _ptr(lse_out),
+                                          _stream(stream)), "hyb_decode_attn_noalloc")
+
+
+def hyb_noalloc_scratch_limit() -> int:
+    return int(load().hyb_noalloc_scratch_limit())
 
 
 def hyb_combine(batch, num_q_heads, head_dim, n_splits, o_partial, lse_partial, out,

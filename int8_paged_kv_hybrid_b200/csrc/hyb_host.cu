@@ -50,6 +50,7 @@ const char *hyb_strerror(int code) {
     case HYB_ERR_UNSUPPORTED: return "unsupported configuration (only hot 32 / block 64 / head_dim 128, Hq/Hkv <= 8)";
     case HYB_ERR_WORKSPACE: return "workspace missing or too small";
     case HYB_ERR_CUDA: return "CUDA error (see hyb_last_cuda_error)";
+    case HYB_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the static buffer of hyb_decode_attn_noalloc";
     case 100 + HYB_STATUS_OK: return "device status: ok";
     case 100 + HYB_STATUS_BAD_BLOCK: return "device status: block-table entry out of range";
     case 100 + HYB_STATUS_BAD_N_NEW: return "device status: n_new out of range";
@@ -181,6 +182,19 @@ static WsLayout ws_layout(const hyb_cache_desc *d, int ns, bool step) {
 }
 
 static size_t workspace_for(const hyb_cache_desc *d, int ns) { return ws_layout(d, ns, false).total; }
+
+}  // extern "C"
+
+namespace hyb {
+// Leading bytes of the hyb_decode_attn workspace that must be zero before a
+// call (the arrival counters); 0 when the workspace is not used.
+size_t decode_ws_zero_prefix(const hyb_cache_desc *d, int ns) {
+  const WsLayout w = ws_layout(d, ns, false);
+  return w.total > 0 ? w.o_part : 0;
+}
+}  // namespace hyb
+
+extern "C" {
 
 size_t hyb_decode_workspace_bytes(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens) {
   int32_t st = 0, ns = 0;

@@ -61,5 +61,6 @@ cudaError_t launch_combine(const CombineArgs &a, int rows, cudaStream_t stream);
 int decode_max_split_blocks();
 int decode_ctas_per_sm(int group);
 int decode_max_cluster();
+size_t decode_ws_zero_prefix(const hyb_cache_desc *d, int ns);
 
 }  // namespace hyb
