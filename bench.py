@@ -44,6 +44,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--split", type=int, default=0, help="split_tokens (0 = automatic)")
+    p.add_argument("--workload", type=int, default=WORKLOAD,
+                   help="1..5: the measured shapes (2, the default, is the headline workload)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--lean", action="store_true",
                    help="profiling run: no state restore, L2 flush, e2e or CPU baseline")
@@ -51,13 +53,19 @@ def parse():
 
 
 def workload_config(w, split, ns):
-    return {"workload": "llama3-8b decode attention, 1 layer: batch %d, Hq %d, Hkv %d, d 128, "
-                        "L %d (32 FP16 hot + %d INT8 cold in 64-token blocks), %d-block pool"
-                        % (w.batch, w.num_q_heads, w.num_kv_heads, int(w.lens[0]),
-                           int(w.lens[0]) - 32, w.num_phys_blocks),
-            "batch": int(w.batch), "seq_len": int(w.lens[0]), "num_q_heads": w.num_q_heads,
-            "num_kv_heads": w.num_kv_heads, "head_dim": 128, "hot_tokens": 32, "block_size": 64,
-            "quant_bits": 8, "split_tokens": split, "n_splits": ns,
+    lens = w.lens
+    if w.name == "config2":
+        what = ("llama3-8b decode attention, 1 layer: batch %d, Hq %d, Hkv %d, d 128, L %d (32 FP16 hot + "
+                "%d INT8 cold in 64-token blocks), %d-block pool"
+                % (w.batch, w.num_q_heads, w.num_kv_heads, int(lens[0]), int(lens[0]) - 32, w.num_phys_blocks))
+    else:
+        what = ("decode attention, 1 layer: batch %d, Hq %d, Hkv %d, d 128, L %d..%d (mean %.0f), 32 FP16 hot "
+                "+ %s cold in 64-token blocks, %d-block pool"
+                % (w.batch, w.num_q_heads, w.num_kv_heads, int(lens.min()), int(lens.max()), float(lens.mean()),
+                   "INT8 (oldest quarter INT4)" if w.n_int4 is not None else "INT8", w.num_phys_blocks))
+    return {"workload": what, "batch": int(w.batch), "seq_len": int(lens.max()),
+            "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads, "head_dim": 128, "hot_tokens": 32,
+            "block_size": 64, "quant_bits": 8, "split_tokens": split, "n_splits": ns,
             "step": "hyb_decode_step: append 1 token/seq + split-KV attention, one launch",
             "l2": "flushed between timed steps (512 MB write)",
             "parallelism": "replicas (independent batch per GPU)"}
@@ -162,12 +170,14 @@ def build_gpu_state(w, torch):
     from int8_paged_kv_hybrid_b200 import HybridKVCache, synth
     cache = HybridKVCache(w.batch, w.num_kv_heads, w.num_q_heads, w.num_phys_blocks, w.max_blocks,
                           block_table=w.block_table, n_int4=w.n_int4)
-    for si, n in enumerate(w.schedule[:-1]):
-        k, v = synth.step_tokens(w, si, n)
+    # prefill to L-1 in 64-token appends; the benchmarked step appends the last token
+    sched = synth._chunk_schedule(w.lens, 64)
+    for si, n in enumerate(sched[:-1]):
+        k, v = synth.step_tokens(w, si, n, max_new=64)
         cache.append(torch.from_numpy(n).cuda(), torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
-    last = len(w.schedule) - 1
-    n_last = w.schedule[-1]
-    k_last, v_last = synth.step_tokens(w, last, n_last, max_new=int(n_last.max()))
+    last = len(sched) - 1
+    n_last = sched[-1]
+    k_last, v_last = synth.step_tokens(w, last, n_last, max_new=1)
     q = synth.query(w)
     torch.cuda.synchronize()
     return cache, n_last, k_last, v_last, q
@@ -197,12 +207,12 @@ def run_native(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     clocks = ClockSampler(local_rank) if rank == 0 and not args.lean else None
-    w = synth.make_workload(WORKLOAD, seed_offset=1000 * rank)
+    w = synth.make_workload(args.workload, seed_offset=1000 * rank)
     L = int(w.lens.max())
     cache, n_last, k_last, v_last, q = build_gpu_state(w, torch)
     if args.lean:
         L += args.warmup + args.steps  # the lean run lets the cache grow one token per step
-    split, ns = cache.plan(L, args.split)
+    split, ns = cache.plan(L, args.split or w.split_tokens)
     n_d = torch.from_numpy(n_last).to(dev)
     k_d = torch.from_numpy(k_last).to(dev)
     v_d = torch.from_numpy(v_last).to(dev)
@@ -353,12 +363,13 @@ def oracle_step_rate(w, steps, warmup, budget_s=None):
     from int8_paged_kv_hybrid_b200 import synth
     threads = os.cpu_count() or 1
     ora = oracle.OracleCache(w.batch, w.num_kv_heads, w.num_q_heads, w.max_blocks + 16)
-    for si, n in enumerate(w.schedule[:-1]):
-        k, v = synth.step_tokens(w, si, n)
+    sched = synth._chunk_schedule(w.lens, 64)
+    for si, n in enumerate(sched[:-1]):
+        k, v = synth.step_tokens(w, si, n, max_new=64)
         ora.append(n, k, v)
-    last = len(w.schedule) - 1
-    n_last = w.schedule[-1]
-    k_last, v_last = synth.step_tokens(w, last, n_last, max_new=int(n_last.max()))
+    last = len(sched) - 1
+    n_last = sched[-1]
+    k_last, v_last = synth.step_tokens(w, last, n_last, max_new=1)
     q = synth.query(w)
     times = []
     for i in range(warmup + steps):
@@ -387,7 +398,7 @@ def main():
         # the CPU oracle on the host cores: rank 0 alone
         if rank != 0:
             return 0
-        w = synth.make_workload(WORKLOAD)
+        w = synth.make_workload(args.workload)
         sec, n, threads = oracle_step_rate(w, args.steps, args.warmup, budget_s=150.0)
         kvb = synth.kv_bytes(w)
         val = kvb / sec / 1e9

@@ -143,7 +143,7 @@ __device__ __forceinline__ void unpack_int4(uint32_t x, uint32_t &lo, uint32_t &
 // arithmetic of hyb_kv_append (bit-exact), and write back what changed.  All
 // threads of the CTA call it.
 template <int G>
-__device__ __noinline__ void fused_append(DecodeSmem<G> &sm, const DecodeArgs &a, int b, int h, int L_old,
+__device__ __forceinline__ void fused_append(DecodeSmem<G> &sm, const DecodeArgs &a, int b, int h, int L_old,
                                           int i0, int ncold, int n_int4_b, bool do_seal, __half2 new_kv,
                                           int tid, int warp, int lane) {
   uint8_t *hot_st = sm.ring[ncold % kStages];
@@ -254,11 +254,40 @@ __device__ __noinline__ void fused_append(DecodeSmem<G> &sm, const DecodeArgs &a
   __syncthreads();
 }
 
+// Raise a warp's running max to cover an item's logits, whose maximum over a
+// lane's tokens is zmax (lane's head hx): m_run per head, the accumulators
+// and the lane's denominator (l_lane + psum_lane / 32767) are rescaled.
+// Warp-uniform call; rare once the first blocks are seen.
+template <int G, int P>
+__device__ __forceinline__ void raise_max(float zmax, float (&m_run)[G], float (&acc)[G][4], float &m_hx,
+                                          float &l_lane, int &psum_lane, int hx) {
+  float mb = zmax;
+  mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 8));
+  mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 16));
+  float alpha_hx = 1.f;
+#pragma unroll
+  for (int hh = 0; hh < G; hh++) {
+    const float mbh = __shfl_sync(0xffffffffu, mb, hh * (8 / P));  // a lane holding head hh
+    if (mbh > m_run[hh]) {
+      const float alpha = ex2(m_run[hh] - mbh);
+#pragma unroll
+      for (int kk = 0; kk < 4; kk++) acc[hh][kk] *= alpha;
+      if (hh == hx) alpha_hx = alpha;
+      m_run[hh] = mbh;
+    }
+    if (hh == hx) m_hx = m_run[hh];
+  }
+  if (alpha_hx != 1.f) {
+    l_lane = (l_lane + static_cast<float>(psum_lane) * (1.f / 32767.f)) * alpha_hx;
+    psum_lane = 0;
+  }
+}
+
 // kCluster: the grid is launched in clusters of n_splits CTAs (the splits of
 // one (sequence, kv head)); splits are merged through distributed shared
 // memory instead of the workspace.
 template <int G, bool kCluster>
-__global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 2)) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(const DecodeArgs a) {
   constexpr int P = pow2_heads<G>();
   extern __shared__ __align__(128) uint8_t smem_raw[];
   DecodeSmem<G> &sm = *reinterpret_cast<DecodeSmem<G> *>(smem_raw);
@@ -409,14 +438,21 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 2)) decode_kernel(cons
     qp[k][4] = x1.x; qp[k][5] = x1.y; qp[k][6] = x1.z; qp[k][7] = x1.w;
   }
 
-  float m_run[G], l_run[G], acc[G][4];
+  // Online-softmax state of this warp.  m_run: running max per head (the
+  // same in every lane); acc: unnormalised output of the lane's channels;
+  // weights are taken relative to m_run, so the denominator can be summed
+  // per lane (head hx, its own tokens) and reduced across lanes only at the
+  // end: l_lane (FP32) plus psum_lane (integer sum of 16-bit weight codes).
+  float m_run[G], acc[G][4];
 #pragma unroll
   for (int hh = 0; hh < G; hh++) {
     m_run[hh] = -INFINITY;
-    l_run[hh] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < 4; kk++) acc[hh][kk] = 0.f;
   }
+  float m_hx = hx < G ? -INFINITY : INFINITY;  // m_run of this lane's head (+inf: padding head)
+  float l_lane = 0.f;
+  int psum_lane = 0;
 
   bool aborted = false;
   int next_issue = issued;  // thread 0: next item to bring in
@@ -488,28 +524,24 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 2)) decode_kernel(cons
           transpose_reduce<P>(dot);
           z[step] = (4 * step + tg < nv) ? static_cast<float>(dot[0]) * coef : -INFINITY;
         }
-        float mb = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
-        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 8));
-        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 16));
-        // 16-bit weights: round(32767 * 2^(z - mb)) via the 1.5*2^23 magic add
-        int psum = 0;
+        // the running max must cover these logits (rare after the first blocks)
+        {
+          const float zmax = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
+          if (__any_sync(0xffffffffu, zmax > m_hx)) raise_max<G, P>(zmax, m_run, acc, m_hx, l_lane, psum_lane, hx);
+        }
+        // 16-bit weights relative to the running max: round(32767 * 2^(z - m))
+        // via the 1.5*2^23 magic add
         uint32_t pc[4];
 #pragma unroll
         for (int step = 0; step < 4; step++) {
-          const float pq = fmaf(ex2(z[step] - mb), 32767.f, 12582912.f);
+          const float pq = fmaf(ex2(z[step] - m_hx), 32767.f, 12582912.f);
           pc[step] = __float_as_uint(pq) - 0x4B400000u;
-          psum += static_cast<int>(pc[step]);
+          psum_lane += static_cast<int>(pc[step]);
         }
-        psum += __shfl_xor_sync(0xffffffffu, psum, 8);
-        psum += __shfl_xor_sync(0xffffffffu, psum, 16);
         if (owner) {
 #pragma unroll
           for (int step = 0; step < 4; step++)
             sm.pcode[warp][hx][4 * step + tg] = static_cast<uint16_t>(pc[step]);
-          if (tg == 0) {
-            sm.wmax[warp][hx] = mb;
-            sm.wsum[warp][hx] = static_cast<float>(psum);
-          }
         }
         __syncwarp();
         // P.V over this warp's 16 tokens; lane owns channels lane + 32*kk
@@ -528,40 +560,24 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 2)) decode_kernel(cons
             unpack_int4(v.y, vw[kk][2], vw[kk][3]);
           }
         }
-        int ai[G][4];
-#pragma unroll
-        for (int hh = 0; hh < G; hh++)
-#pragma unroll
-          for (int kk = 0; kk < 4; kk++) ai[hh][kk] = 0;
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-#pragma unroll
-          for (int hh = 0; hh < G; hh++) {
-            // p codes of tokens 4j..4j+3 of this warp's 16, as two 16-bit pairs
-            const uint2 pp = *reinterpret_cast<const uint2 *>(&sm.pcode[warp][hh][4 * j]);
-#pragma unroll
-            for (int kk = 0; kk < 4; kk++) {
-              ai[hh][kk] = __dp2a_lo(static_cast<int>(pp.x), static_cast<int>(vw[kk][j]), ai[hh][kk]);
-              ai[hh][kk] = __dp2a_hi(static_cast<int>(pp.y), static_cast<int>(vw[kk][j]), ai[hh][kk]);
-            }
-          }
-        }
+        const float cv = sc.y * (1.f / 32767.f);
 #pragma unroll
         for (int hh = 0; hh < G; hh++) {
-          const float mbh = sm.wmax[warp][hh];
-          if (mbh > m_run[hh]) {  // warp-uniform: rescale only when the max grows
-            const float alpha = ex2(m_run[hh] - mbh);
-            l_run[hh] *= alpha;
+          // p codes of this warp's 16 tokens, as 16-bit pairs (tokens 2i, 2i+1)
+          const uint4 pa = *reinterpret_cast<const uint4 *>(&sm.pcode[warp][hh][0]);
+          const uint4 pb = *reinterpret_cast<const uint4 *>(&sm.pcode[warp][hh][8]);
+          const uint32_t pp[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+          int ai[4] = {0, 0, 0, 0};
 #pragma unroll
-            for (int kk = 0; kk < 4; kk++) acc[hh][kk] *= alpha;
-            m_run[hh] = mbh;
+          for (int j = 0; j < 4; j++) {
+#pragma unroll
+            for (int kk = 0; kk < 4; kk++) {
+              ai[kk] = __dp2a_lo(static_cast<int>(pp[2 * j]), static_cast<int>(vw[kk][j]), ai[kk]);
+              ai[kk] = __dp2a_hi(static_cast<int>(pp[2 * j + 1]), static_cast<int>(vw[kk][j]), ai[kk]);
+            }
           }
-          const float beta = ex2(mbh - m_run[hh]) * (1.f / 32767.f);
-          l_run[hh] = fmaf(beta, sm.wsum[warp][hh], l_run[hh]);
-          const float cv = beta * sc.y;
 #pragma unroll
-          for (int kk = 0; kk < 4; kk++)
-            acc[hh][kk] = fmaf(cv, static_cast<float>(ai[hh][kk]), acc[hh][kk]);
+          for (int kk = 0; kk < 4; kk++) acc[hh][kk] = fmaf(cv, static_cast<float>(ai[kk]), acc[hh][kk]);
         }
       }
     } else if (ok) {
@@ -600,24 +616,19 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 2)) decode_kernel(cons
           transpose_reduce<P>(dot);
           z[step] = (4 * step + tg < nv) ? dot[0] * a.qk_scale : -INFINITY;
         }
-        float mb = fmaxf(z[0], z[1]);
-        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 8));
-        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 16));
-        float pv[2], psum = 0.f;
+        {
+          const float zmax = fmaxf(z[0], z[1]);
+          if (__any_sync(0xffffffffu, zmax > m_hx)) raise_max<G, P>(zmax, m_run, acc, m_hx, l_lane, psum_lane, hx);
+        }
+        float pv[2];
 #pragma unroll
         for (int step = 0; step < 2; step++) {
-          pv[step] = ex2(z[step] - mb);
-          psum += pv[step];
+          pv[step] = ex2(z[step] - m_hx);
+          l_lane += pv[step];
         }
-        psum += __shfl_xor_sync(0xffffffffu, psum, 8);
-        psum += __shfl_xor_sync(0xffffffffu, psum, 16);
         if (owner) {
           sm.phot[warp][hx][tg] = pv[0];
           sm.phot[warp][hx][4 + tg] = pv[1];
-          if (tg == 0) {
-            sm.wmax[warp][hx] = mb;
-            sm.wsum[warp][hx] = psum;
-          }
         }
         __syncwarp();
         float ah[G][4];
@@ -640,20 +651,9 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 2)) decode_kernel(cons
           }
         }
 #pragma unroll
-        for (int hh = 0; hh < G; hh++) {
-          const float mbh = sm.wmax[warp][hh];
-          if (mbh > m_run[hh]) {
-            const float alpha = ex2(m_run[hh] - mbh);
-            l_run[hh] *= alpha;
+        for (int hh = 0; hh < G; hh++)
 #pragma unroll
-            for (int kk = 0; kk < 4; kk++) acc[hh][kk] *= alpha;
-            m_run[hh] = mbh;
-          }
-          const float beta = ex2(mbh - m_run[hh]);
-          l_run[hh] = fmaf(beta, sm.wsum[warp][hh], l_run[hh]);
-#pragma unroll
-          for (int kk = 0; kk < 4; kk++) acc[hh][kk] = fmaf(beta, ah[hh][kk], acc[hh][kk]);
-        }
+          for (int kk = 0; kk < 4; kk++) acc[hh][kk] += ah[hh][kk];
       }
     }
     __syncwarp();
@@ -665,6 +665,16 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 2)) decode_kernel(cons
     if (lane == 0) mbar_arrive(&sm.empty[st]);
   }
   aborted = __syncthreads_or(aborted) != 0;
+  // denominators: this lane's partial for head hx, summed over the 4 token
+  // groups, then gathered per head from a lane that holds it
+  float l_run[G];
+  {
+    float lt = l_lane + static_cast<float>(psum_lane) * (1.f / 32767.f);
+    lt += __shfl_xor_sync(0xffffffffu, lt, 8);
+    lt += __shfl_xor_sync(0xffffffffu, lt, 16);
+#pragma unroll
+    for (int hh = 0; hh < G; hh++) l_run[hh] = __shfl_sync(0xffffffffu, lt, hh * (8 / P));
+  }
 
   if (aborted) {
     // let every copy still in flight land before the CTA's shared memory is

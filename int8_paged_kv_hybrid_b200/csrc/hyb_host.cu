@@ -130,7 +130,7 @@ int hyb_decode_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_
     // different lengths even out over several waves.
     const int group = d->num_q_heads / d->num_kv_heads;
     int occ = hyb::decode_ctas_per_sm(group);
-    if (occ <= 0) occ = group <= 4 ? 4 : 2;
+    if (occ <= 0) occ = group <= 4 ? 3 : 2;
     const long long slots = static_cast<long long>(sm_count()) * occ;
     const long long units = static_cast<long long>(d->batch) * d->num_kv_heads;
     const long long s_wave = slots / units;
