@@ -13,7 +13,8 @@
 // (K tile 8 KB + V tile 8 KB, or 4 + 4 KB for INT4) and the hot ring (16 KB)
 // is one pipeline item, brought into a 3-stage shared-memory ring by the TMA
 // engine with one 1-D bulk copy (no cluster multicast) completing on an
-// mbarrier; every wait is bounded.  Four CTAs fit on an SM (16 warps).
+// mbarrier; every wait is bounded.  Three CTAs fit on an SM for up to 4 query
+// heads per kv head (two above that).
 //
 // Arithmetic (per kv head, for its G = Hq/Hkv query heads):
 //  * q is turned into 16-bit fixed point per query head (q_i = rint(q * 32767
@@ -283,6 +284,78 @@ __device__ __forceinline__ void raise_max(float zmax, float (&m_run)[G], float (
   }
 }
 
+// One full INT8 cold block (all 64 tokens valid), for one warp.  The warp's
+// tokens are 16w..16w+15; lane (tg, cs) takes tokens 16w + 4tg + step, step
+// 0..3 (channels 16cs..16cs+15), so the four weight codes an owner lane
+// produces for its head are adjacent and leave in one 8-byte store.  k_lane
+// and v_lane are the lane's byte offsets of its K row (step 0) and of its V
+// words inside a stage; pc is this warp's weight-code rows.  Same arithmetic
+// as the general path; no masks, no INT4 branches, offsets fixed per lane.
+template <int G, int P>
+__device__ __forceinline__ void cold_block_full(const uint8_t *stage, int k_lane, int v_lane,
+                                                const uint32_t (&qp)[P][8], float coef, float cv,
+                                                uint16_t (*pc_rows)[16], int hx, int tg, bool owner,
+                                                float (&m_run)[G], float (&acc)[G][4], float &m_hx,
+                                                float &l_lane, int &psum_lane) {
+  float z[4];
+#pragma unroll
+  for (int step = 0; step < 4; step++) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(stage + k_lane + step * kDim);
+    const uint32_t kw[4] = {v.x, v.y, v.z, v.w};
+    int dot[P];
+#pragma unroll
+    for (int kk = 0; kk < P; kk++) dot[kk] = 0;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+#pragma unroll
+      for (int kk = 0; kk < P; kk++)
+        dot[kk] = __dp2a_lo(static_cast<int>(qp[kk][2 * j]), static_cast<int>(kw[j]), dot[kk]);
+#pragma unroll
+      for (int kk = 0; kk < P; kk++)
+        dot[kk] = __dp2a_hi(static_cast<int>(qp[kk][2 * j + 1]), static_cast<int>(kw[j]), dot[kk]);
+    }
+    transpose_reduce<P>(dot);
+    z[step] = static_cast<float>(dot[0]) * coef;
+  }
+  {
+    const float zmax = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
+    if (__any_sync(0xffffffffu, zmax > m_hx)) raise_max<G, P>(zmax, m_run, acc, m_hx, l_lane, psum_lane, hx);
+  }
+  uint32_t pc[4];
+#pragma unroll
+  for (int step = 0; step < 4; step++) {
+    const float pq = fmaf(ex2(z[step] - m_hx), 32767.f, 12582912.f);
+    pc[step] = __float_as_uint(pq) - 0x4B400000u;
+    psum_lane += static_cast<int>(pc[step]);
+  }
+  if (owner)
+    *reinterpret_cast<uint2 *>(&pc_rows[hx][4 * tg]) = make_uint2(pc[0] | (pc[1] << 16), pc[2] | (pc[3] << 16));
+  __syncwarp();
+  uint32_t vw[4][4];
+#pragma unroll
+  for (int kk = 0; kk < 4; kk++) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(stage + v_lane + 32 * kBlock * kk);
+    vw[kk][0] = v.x; vw[kk][1] = v.y; vw[kk][2] = v.z; vw[kk][3] = v.w;
+  }
+#pragma unroll
+  for (int hh = 0; hh < G; hh++) {
+    const uint4 pa = *reinterpret_cast<const uint4 *>(&pc_rows[hh][0]);
+    const uint4 pb = *reinterpret_cast<const uint4 *>(&pc_rows[hh][8]);
+    const uint32_t pp[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+    int ai[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+#pragma unroll
+      for (int kk = 0; kk < 4; kk++) {
+        ai[kk] = __dp2a_lo(static_cast<int>(pp[2 * j]), static_cast<int>(vw[kk][j]), ai[kk]);
+        ai[kk] = __dp2a_hi(static_cast<int>(pp[2 * j + 1]), static_cast<int>(vw[kk][j]), ai[kk]);
+      }
+    }
+#pragma unroll
+    for (int kk = 0; kk < 4; kk++) acc[hh][kk] = fmaf(cv, static_cast<float>(ai[kk]), acc[hh][kk]);
+  }
+}
+
 // kCluster: the grid is launched in clusters of n_splits CTAs (the splits of
 // one (sequence, kv head)); splits are merged through distributed shared
 // memory instead of the workspace.
@@ -428,6 +501,9 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
   const int hx = head_xor<P>(lane);   // this lane's value k is head k ^ hx; its final head is hx
   const bool owner = (lane & (8 / P - 1)) == 0 && hx < G;
   const float sq_hd = sm.sq[hx];
+  // full-block path: the lane's K row (tokens 16w + 4tg + step) and V words
+  const int k_lane = (16 * warp + 4 * tg) * kDim + 16 * cs;
+  const int v_lane = kTileBytes + lane * kBlock + 16 * (warp ^ ((lane >> 1) & 3));
 
   uint32_t qp[P][8];  // q pairs of this lane's 16 channels, in the lane's head order
 #pragma unroll
@@ -492,10 +568,13 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
       const int i = i0 + k;
       const int nvalid = sm.phys[k] < 0 ? 0 : min(kBlock, Lc - i * kBlock);
       const int nv = nvalid - 16 * warp;
-      if (nv > 0) {
-        const bool int4 = i < n_int4_b;
-        const float2 sc = sm.scl[k];
-        const float coef = sq_hd * sc.x * a.qk_scale;
+      const bool int4 = i < n_int4_b;
+      const float2 sc = sm.scl[k];
+      const float coef = sq_hd * sc.x * a.qk_scale;
+      if (nvalid == kBlock && !int4) {
+        cold_block_full<G, P>(stage, k_lane, v_lane, qp, coef, sc.y * (1.f / 32767.f), sm.pcode[warp], hx, tg,
+                              owner, m_run, acc, m_hx, l_lane, psum_lane);
+      } else if (nv > 0) {
         float z[4];
 #pragma unroll
         for (int step = 0; step < 4; step++) {
