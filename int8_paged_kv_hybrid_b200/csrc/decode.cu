@@ -67,16 +67,12 @@ struct DecodeSmem {
   float sq[P];                       // fixed-point step of each head's q
   alignas(16) uint16_t pcode[kWarps][G][16];
   alignas(16) float phot[kWarps][G][8];
-  float wmax[kWarps][G];
-  float wsum[kWarps][G];
   float mrun[kWarps][G];
   float lrun[kWarps][G];
   int8_t rqt[2][256];  // fused step: re-quantization tables of the tail block (K, V)
   float seal_s[2];     // fused step: the tail block's scales after sealing
   int seal_rq[2];      // fused step: 1 if the tail block's codes were re-quantized
   float cl_l[G];   // this split's log2-sum-exp per head, read by the cluster's merge
-  float mfin[G];   // final merge: max and sum of the split weights per head
-  float dfin[G];
   int last;
   int abort_flag;
 };
@@ -281,6 +277,72 @@ __device__ __forceinline__ void raise_max(float zmax, float (&m_run)[G], float (
   if (alpha_hx != 1.f) {
     l_lane = (l_lane + static_cast<float>(psum_lane) * (1.f / 32767.f)) * alpha_hx;
     psum_lane = 0;
+  }
+}
+
+// Log-sum-exp merge of n partial results of the G query heads of one kv head
+// (read from global memory through L2).  Partial j of head hh: 128 FP32 at
+// o + hh * o_hs + j * 128 and its log2-sum-exp at lse + hh * l_hs + j (-inf:
+// empty, output 0).  Warp w merges heads w, w + 4, ...; lane l channels
+// 4l..4l+3; the loads of kMergeFan partials are issued together.  Writes the
+// FP16 output rows [G][128] at out (and the natural-log lse at lse_out), or,
+// when out is null, the merged FP32 rows at p_o (row stride p_s * 128) with
+// their log2-sum-exp at p_lse (stride p_s).
+template <int G>
+__device__ __forceinline__ void merge_splits(const float *o, size_t o_hs, const float *lse, size_t l_hs, int n,
+                                             int warp, int lane, __half *out, float *lse_out, float *p_o,
+                                             float *p_lse, int p_s) {
+  for (int hh = warp; hh < G; hh += kWarps) {
+    const float *oh = o + hh * o_hs + 4 * lane;
+    const float *lh = lse + hh * l_hs;
+    float m = -INFINITY, den = 0.f;
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = 0; j0 < n; j0 += kMergeFan) {
+      const int nj = min(kMergeFan, n - j0);
+      float4 ov[kMergeFan];
+#pragma unroll
+      for (int j = 0; j < kMergeFan; j++)
+        ov[j] = j < nj ? __ldcg(reinterpret_cast<const float4 *>(oh + (size_t)(j0 + j) * kDim))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float lj = lane < nj ? __ldcg(lh + j0 + lane) : -INFINITY;
+      float mr = lj;
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, d));
+      const float mn = fmaxf(m, mr);
+      if (mn == -INFINITY) continue;  // nothing but empty partials so far
+      const float sc = ex2(m - mn);
+      num.x *= sc; num.y *= sc; num.z *= sc; num.w *= sc;
+      den *= sc;
+      m = mn;
+      const float wl = ex2(lj - m);  // lane j's weight (0 for an empty partial)
+      float ws = wl;
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, d);
+      den += ws;
+#pragma unroll
+      for (int j = 0; j < kMergeFan; j++) {
+        const float wj = __shfl_sync(0xffffffffu, wl, j);
+        num.x = fmaf(wj, ov[j].x, num.x);
+        num.y = fmaf(wj, ov[j].y, num.y);
+        num.z = fmaf(wj, ov[j].z, num.z);
+        num.w = fmaf(wj, ov[j].w, num.w);
+      }
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    const float lse2 = den > 0.f ? m + log2f(den) : -INFINITY;
+    if (out) {
+      __half2 h01 = __floats2half2_rn(num.x * inv, num.y * inv);
+      __half2 h23 = __floats2half2_rn(num.z * inv, num.w * inv);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t *>(&h01);
+      pk.y = *reinterpret_cast<uint32_t *>(&h23);
+      *reinterpret_cast<uint2 *>(out + hh * kDim + 4 * lane) = pk;
+      if (lane == 0 && lse_out) lse_out[hh] = lse2 * kLn2;
+    } else {
+      *reinterpret_cast<float4 *>(p_o + (size_t)hh * p_s * kDim + 4 * lane) =
+          make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+      if (lane == 0) p_lse[(size_t)hh * p_s] = lse2;
+    }
   }
 }
 
@@ -853,87 +915,55 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
     }
     return;
   }
-  // ---------------- split merge by the last CTA of (sequence, kv head) ----------------
+  // ---------------- split merge in global memory ----------------
+  // The last CTA of (sequence, kv head) to finish merges the splits; with
+  // more than kMergeFan splits, the last CTA of each group of kMergeFan
+  // splits merges the group first and the last group merges the groups.
+  const size_t row0 = (size_t)b * a.hq + hq0;
 #pragma unroll
   for (int hh = 0; hh < G; hh++) {
-    const size_t row = (size_t)b * a.hq + hq0 + hh;
-    a.o_part[(row * S + s) * kDim + tid] = o_s[hh];
-    if (tid == 0) a.lse_part[row * S + s] = lse2_s[hh];
+    a.o_part[((row0 + hh) * S + s) * kDim + tid] = o_s[hh];
+    if (tid == 0) a.lse_part[(row0 + hh) * S + s] = lse2_s[hh];
   }
-  __syncthreads();  // all partial stores of the CTA precede thread 0's release below
+  const int unit = b * a.hkv + h;
+  const bool grouped = Sb > kMergeFan;
+  const int grp = s / kMergeFan;
+  __threadfence();
+  __syncthreads();
   if (tid == 0) {
-    __threadfence();
-    const int ticket = atomicAdd(&a.counters[(size_t)b * a.hkv + h], 1);
-    sm.last = (ticket == Sb - 1) ? 1 : 0;
-    if (sm.last) {
-      __threadfence();
-      a.counters[(size_t)b * a.hkv + h] = 0;  // ready for the next call
-    }
+    int32_t *cnt = grouped ? &a.g_counters[(size_t)unit * a.n_groups + grp] : &a.counters[unit];
+    const int need = grouped ? min(kMergeFan, Sb - grp * kMergeFan) : Sb;
+    const int last = atomicAdd(cnt, 1) == need - 1;
+    if (last) *cnt = 0;  // ready for the next call
+    sm.last = last;
   }
   __syncthreads();
   if (!sm.last) return;
   __threadfence();
-  // split weights: lse of every (head, split) into shared memory, then per
-  // head the max and the weights 2^(lse - max) (0 for empty splits)
-  float *wts = reinterpret_cast<float *>(&sm.ring[0][0]);  // [G][Sb]
-  const bool fits = G * Sb <= kStages * kTilePairBytes / 4;
-  if (fits) {
-    for (int e = tid; e < G * Sb; e += kThreads) {
-      const int hh = e / Sb, j = e - hh * Sb;
-      wts[e] = __ldcg(a.lse_part + ((size_t)b * a.hq + hq0 + hh) * S + j);
-    }
-    __syncthreads();
-    for (int hh = warp; hh < G; hh += kWarps) {
-      float m = -INFINITY;
-      for (int j = lane; j < Sb; j += 32) m = fmaxf(m, wts[hh * Sb + j]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      float den = 0.f;
-      for (int j = lane; j < Sb; j += 32) {
-        const float wv = m == -INFINITY ? 0.f : ex2(wts[hh * Sb + j] - m);
-        wts[hh * Sb + j] = wv;
-        den += wv;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-      if (lane == 0) {
-        sm.mfin[hh] = m;
-        sm.dfin[hh] = den;
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int hh = 0; hh < G; hh++) {
-      const size_t row = (size_t)b * a.hq + hq0 + hh;
-      const float *op = a.o_part + row * S * kDim + tid;
-      float num = 0.f;
-#pragma unroll 8
-      for (int j = 0; j < Sb; j++) num = fmaf(wts[hh * Sb + j], __ldcg(op + (size_t)j * kDim), num);
-      const float den = sm.dfin[hh];
-      a.out[row * kDim + tid] = __float2half_rn(den > 0.f ? num / den : 0.f);
-      if (tid == 0 && a.lse_out) a.lse_out[row] = den > 0.f ? (sm.mfin[hh] + log2f(den)) * kLn2 : -INFINITY;
-    }
-  } else {
-    // very many splits: two passes over global memory per head
-#pragma unroll 1
-    for (int hh = 0; hh < G; hh++) {
-      const size_t row = (size_t)b * a.hq + hq0 + hh;
-      const float *lp = a.lse_part + row * S;
-      const float *op = a.o_part + row * S * kDim + tid;
-      float m = -INFINITY;
-      for (int j = 0; j < Sb; j++) m = fmaxf(m, __ldcg(lp + j));
-      float num = 0.f, den = 0.f;
-      if (m != -INFINITY) {
-        for (int j = 0; j < Sb; j++) {
-          const float wgt = ex2(__ldcg(lp + j) - m);
-          num = fmaf(wgt, __ldcg(op + (size_t)j * kDim), num);
-          den += wgt;
-        }
-      }
-      a.out[row * kDim + tid] = __float2half_rn(den > 0.f ? num / den : 0.f);
-      if (tid == 0 && a.lse_out) a.lse_out[row] = den > 0.f ? (m + log2f(den)) * kLn2 : -INFINITY;
-    }
+  if (!grouped) {
+    merge_splits<G>(a.o_part + row0 * S * kDim, (size_t)S * kDim, a.lse_part + row0 * S, S, Sb, warp, lane,
+                    a.out + row0 * kDim, a.lse_out ? a.lse_out + row0 : nullptr, nullptr, nullptr, 0);
+    return;
   }
+  const int NG = a.n_groups;
+  const int j0 = grp * kMergeFan;
+  merge_splits<G>(a.o_part + (row0 * S + j0) * kDim, (size_t)S * kDim, a.lse_part + row0 * S + j0, S,
+                  min(kMergeFan, Sb - j0), warp, lane, nullptr, nullptr, a.g_part + (row0 * NG + grp) * kDim,
+                  a.g_lse + row0 * NG + grp, NG);
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int ngb = (Sb + kMergeFan - 1) / kMergeFan;
+    const int last = atomicAdd(&a.counters[unit], 1) == ngb - 1;
+    if (last) a.counters[unit] = 0;
+    sm.last = last;
+  }
+  __syncthreads();
+  if (!sm.last) return;
+  __threadfence();
+  merge_splits<G>(a.g_part + row0 * NG * kDim, (size_t)NG * kDim, a.g_lse + row0 * NG, NG,
+                  (Sb + kMergeFan - 1) / kMergeFan, warp, lane, a.out + row0 * kDim,
+                  a.lse_out ? a.lse_out + row0 : nullptr, nullptr, nullptr, 0);
 }
 
 // Largest cluster the decode kernel is launched with (portable size).

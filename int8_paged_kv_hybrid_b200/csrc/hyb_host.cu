@@ -156,15 +156,19 @@ int hyb_decode_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_
 }
 
 // Workspace layout.  Fused step only: read counters int32 [batch].  With more
-// splits than one cluster holds: arrival counters int32 [batch][Hkv], then the
-// split outputs FP32 [batch][Hq][ns][128], then their log2-sum-exp FP32
-// [batch][Hq][ns].  Each part starts on a 256-byte boundary.
+// splits than one cluster holds: arrival counters int32 [batch][Hkv] and, with
+// more than kMergeFan splits, group arrival counters int32 [batch][Hkv][ng]
+// (ng = ceil(ns / kMergeFan)); then the split outputs FP32
+// [batch][Hq][ns][128] and their log2-sum-exp FP32 [batch][Hq][ns]; then the
+// group outputs FP32 [batch][Hq][ng][128] and their log2-sum-exp [batch][Hq][ng].
+// Each part starts on a 256-byte boundary; the counters come first.
 struct WsLayout {
-  size_t seq_cnt, counters, o_part, lse_part, total;
+  size_t seq_cnt, counters, g_counters, o_part, lse_part, g_part, g_lse, total;
+  int n_groups;
 };
 
 static WsLayout ws_layout(const hyb_cache_desc *d, int ns, bool step) {
-  WsLayout w{0, 0, 0, 0, 0};
+  WsLayout w{0, 0, 0, 0, 0, 0, 0, 0, 0};
   size_t off = 0;
   if (step) {
     w.seq_cnt = 0;
@@ -172,10 +176,19 @@ static WsLayout ws_layout(const hyb_cache_desc *d, int ns, bool step) {
   }
   if (ns > hyb::decode_max_cluster()) {
     const size_t rows = static_cast<size_t>(d->batch) * d->num_q_heads;
+    const size_t units = static_cast<size_t>(d->batch) * d->num_kv_heads;
+    const size_t ng = ns > hyb::kMergeFan ? (ns + hyb::kMergeFan - 1) / hyb::kMergeFan : 0;
+    w.n_groups = static_cast<int>(ng);
     w.counters = off;
-    w.o_part = off + round_up(static_cast<size_t>(d->batch) * d->num_kv_heads * sizeof(int32_t), kWsAlign);
+    off += round_up(units * sizeof(int32_t), kWsAlign);
+    w.g_counters = off;
+    off += round_up(units * ng * sizeof(int32_t), kWsAlign);
+    w.o_part = off;
     w.lse_part = w.o_part + round_up(rows * ns * hyb::kDim * sizeof(float), kWsAlign);
     off = w.lse_part + round_up(rows * ns * sizeof(float), kWsAlign);
+    w.g_part = off;
+    w.g_lse = w.g_part + round_up(rows * ng * hyb::kDim * sizeof(float), kWsAlign);
+    off = w.g_lse + round_up(rows * ng * sizeof(float), kWsAlign);
   }
   w.total = off;
   return w;
@@ -234,6 +247,10 @@ static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_s
   a.counters = merge_ws ? reinterpret_cast<int32_t *>(ws + wl.counters) : nullptr;
   a.o_part = merge_ws ? reinterpret_cast<float *>(ws + wl.o_part) : nullptr;
   a.lse_part = merge_ws ? reinterpret_cast<float *>(ws + wl.lse_part) : nullptr;
+  a.n_groups = merge_ws ? wl.n_groups : 0;
+  a.g_counters = a.n_groups > 0 ? reinterpret_cast<int32_t *>(ws + wl.g_counters) : nullptr;
+  a.g_part = a.n_groups > 0 ? reinterpret_cast<float *>(ws + wl.g_part) : nullptr;
+  a.g_lse = a.n_groups > 0 ? reinterpret_cast<float *>(ws + wl.g_lse) : nullptr;
   a.hkv = d->num_kv_heads;
   a.hq = d->num_q_heads;
   a.num_phys = d->num_phys_blocks;

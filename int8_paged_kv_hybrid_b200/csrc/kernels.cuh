@@ -36,6 +36,13 @@ struct DecodeArgs {
   float *o_part;              // [batch][Hq][n_splits][128] (n_splits > 1)
   float *lse_part;            // [batch][Hq][n_splits], log2 domain
   int32_t *counters;          // [batch][Hkv] arrivals per (sequence, kv head), zero between calls
+  // more than kMergeFan splits: the splits are merged in groups of kMergeFan
+  // first; group results [batch][Hq][n_groups][128] and their log2-sum-exp,
+  // arrival counters per group [batch][Hkv][n_groups] (zero between calls)
+  float *g_part;
+  float *g_lse;
+  int32_t *g_counters;
+  int n_groups;
   int hkv, hq, num_phys, max_blocks, quant_bits, n_splits, split_blocks, max_seq_len;
   float qk_scale;             // softmax_scale * log2(e)
   // fused decode step (null for attention only): append n_new[b] in {0, 1}
@@ -54,6 +61,9 @@ struct CombineArgs {
   float *lse_out;             // [rows] or null
   int n_splits;
 };
+
+// Partial results merged per round (and per group when there are more).
+constexpr int kMergeFan = 16;
 
 cudaError_t launch_append(const AppendArgs &a, int batch, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, cudaStream_t stream);
