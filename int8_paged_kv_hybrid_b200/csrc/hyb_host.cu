@@ -113,79 +113,138 @@ int hyb_kv_append(const hyb_cache_desc *d, const int32_t *n_new, int32_t max_new
   return e == cudaSuccess ? HYB_OK : cuda_fail(e);
 }
 
-int hyb_decode_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens,
-                    int32_t *split_tokens_out, int32_t *n_splits_out) {
+}  // extern "C"
+
+namespace {
+
+// Use the persistent kernel for plans that do not fit in one wave (off: the
+// one-wave kernel over several waves of short splits measured faster).
+constexpr bool kPersistent = false;
+// Cold blocks per split when the splits take several waves.
+constexpr int kMultiWaveSplit = 16;
+
+// How a decode call runs.  One-wave kernel (decode.cu): grid (ns, Hkv, batch),
+// every split of every (sequence, kv head) resident at once -- chosen when
+// that fits on the GPU.  Otherwise the persistent kernel (decode_sk.cu): as
+// many CTAs as are resident at once, each taking an equal share of the cold
+// blocks of all sequences (batch <= its sequence table).
+struct Plan {
+  bool sk;       // persistent kernel
+  bool cluster;  // one-wave kernel in clusters of ns CTAs (split merge in distributed shared memory)
+  int tb;        // cold blocks per split (persistent kernel: positions per split)
+  int ns;    // splits per (sequence, kv head), at most
+  int grid;  // persistent kernel: CTAs
+};
+
+int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens, Plan *p) {
   const int rc = hyb_check_desc(d);
   if (rc != HYB_OK) return rc;
   if (max_seq_len < 0) return HYB_ERR_INVALID_VALUE;
-  const long long max_blocks_needed = (static_cast<long long>(max_seq_len) - hyb::kHot > 0)
-                                          ? (max_seq_len - hyb::kHot + hyb::kBlock - 1) / hyb::kBlock
-                                          : 0;
-  if (max_blocks_needed > d->max_blocks_per_seq) return HYB_ERR_INVALID_VALUE;
-  int tb;  // cold blocks per split
+  const long long nblk = (static_cast<long long>(max_seq_len) - hyb::kHot > 0)
+                             ? (max_seq_len - hyb::kHot + hyb::kBlock - 1) / hyb::kBlock
+                             : 0;
+  if (nblk > d->max_blocks_per_seq) return HYB_ERR_INVALID_VALUE;
+  const long long npos = nblk > 0 ? nblk : 1;  // positions of a (sequence, kv head) in the persistent kernel
+  const int group = d->num_q_heads / d->num_kv_heads;
+  const int sms = sm_count();
+  int occ = hyb::decode_ctas_per_sm(group);
+  if (occ <= 0) occ = group <= 4 ? 3 : 2;
+  const long long slots = static_cast<long long>(sms) * occ;
+  const long long units = static_cast<long long>(d->batch) * d->num_kv_heads;
+  // persistent kernel: batch within its sequence table, positions in 32 bits
+  const bool sk_ok = d->batch <= hyb::decode_sk_max_batch() && units * npos < (1ll << 30);
+  const int max_tb = hyb::decode_max_split_blocks();
+  long long tb = 0;
   if (split_tokens == 0) {
-    // Automatic: with few (sequence, kv head) units, enough splits of the
-    // longest sequence to fill one wave of resident CTAs and no more; with
-    // many units, splits of about a quarter wave's share so that sequences of
-    // different lengths even out over several waves.
-    const int group = d->num_q_heads / d->num_kv_heads;
-    int occ = hyb::decode_ctas_per_sm(group);
-    if (occ <= 0) occ = group <= 4 ? 3 : 2;
-    const long long slots = static_cast<long long>(sm_count()) * occ;
-    const long long units = static_cast<long long>(d->batch) * d->num_kv_heads;
+    // one wave: enough splits of the longest sequence to fill the GPU, no more
     const long long s_wave = slots / units;
-    long long t;
-    if (s_wave >= 2)
-      t = (max_blocks_needed + s_wave - 1) / s_wave;
-    else
-      t = (max_blocks_needed * units + 4 * slots - 1) / (4 * slots);
-    if (t < 1) t = 1;
-    if (t > hyb::decode_max_split_blocks()) t = hyb::decode_max_split_blocks();
-    tb = static_cast<int>(t);
+    if (s_wave >= 1) {
+      tb = (nblk + s_wave - 1) / s_wave;
+      if (tb < 1) tb = 1;
+      if (tb > max_tb) tb = max_tb;
+    }
+    if (tb == 0 || units * ((nblk + tb - 1) / tb) > slots) {
+      if (sk_ok && kPersistent) {
+        tb = npos;  // persistent kernel, no split boundaries of its own
+      } else {
+        // several waves: short splits, so that the CTA scheduler evens out
+        // sequences of different lengths and CTAs of different speeds
+        tb = kMultiWaveSplit;
+        if (tb > nblk) tb = nblk > 0 ? nblk : 1;
+      }
+    }
   } else {
     if (split_tokens < 0 || split_tokens % hyb::kBlock != 0) return HYB_ERR_INVALID_VALUE;
     tb = split_tokens / hyb::kBlock;
-    if (tb < 1 || tb > hyb::decode_max_split_blocks()) return HYB_ERR_INVALID_VALUE;
+    if (tb < 1) return HYB_ERR_INVALID_VALUE;
   }
-  long long ns = (max_blocks_needed + tb - 1) / tb;
+  long long ns = (nblk + tb - 1) / tb;
   if (ns < 1) ns = 1;
-  if (ns > 65535) return HYB_ERR_INVALID_VALUE;
-  if (split_tokens_out) *split_tokens_out = tb * hyb::kBlock;
-  if (n_splits_out) *n_splits_out = static_cast<int32_t>(ns);
+  const bool one_wave = tb <= max_tb && units * ns <= slots;
+  p->sk = !one_wave && sk_ok && kPersistent;
+  // clusters only when every split is resident at once: a cluster holds its
+  // CTAs until the slowest split is done
+  p->cluster = !p->sk && one_wave && ns >= 2 && ns <= hyb::decode_max_cluster();
+  if (!p->sk && (tb > max_tb || ns > 65535)) return HYB_ERR_INVALID_VALUE;
+  if (p->sk) {
+    ns = (npos + tb - 1) / tb;
+    int occ_sk = hyb::decode_sk_ctas_per_sm(group);
+    if (occ_sk <= 0) occ_sk = group <= 4 ? 3 : 2;
+    long long grid = static_cast<long long>(sms) * occ_sk;
+    if (grid > units * npos) grid = units * npos;
+    p->grid = static_cast<int>(grid);
+  } else {
+    p->grid = 0;
+  }
+  if (tb * hyb::kBlock > 0x7fffffffLL || units * ns > 0x7fffffffLL) return HYB_ERR_INVALID_VALUE;
+  p->tb = static_cast<int>(tb);
+  p->ns = static_cast<int>(ns);
   return HYB_OK;
 }
 
-// Workspace layout.  Fused step only: read counters int32 [batch].  With more
-// splits than one cluster holds: arrival counters int32 [batch][Hkv] and, with
-// more than kMergeFan splits, group arrival counters int32 [batch][Hkv][ng]
-// (ng = ceil(ns / kMergeFan)); then the split outputs FP32
-// [batch][Hq][ns][128] and their log2-sum-exp FP32 [batch][Hq][ns]; then the
-// group outputs FP32 [batch][Hq][ng][128] and their log2-sum-exp [batch][Hq][ng].
+// Workspace layout.  Fused step: read counters int32 [batch] first.
+// One-wave kernel with more splits than one cluster holds: arrival counters
+// int32 [batch][Hkv] and, with more than kMergeFan splits, group arrival
+// counters int32 [batch][Hkv][ng] (ng = ceil(ns / kMergeFan)); then the split
+// outputs FP32 [batch][Hq][ns][128] and their log2-sum-exp FP32
+// [batch][Hq][ns]; then the group outputs FP32 [batch][Hq][ng][128] and their
+// log2-sum-exp [batch][Hq][ng].
+// Persistent kernel: arrival counters per (sequence, kv head) and per group as
+// above, then per split int32 [batch][Hkv][ns]; then one partial result per
+// slot (slots = batch * Hkv * ns + grid): FP32 [slot][Hq/Hkv][128] and the
+// log2-sum-exp [slot][Hq/Hkv]; then the group outputs.
 // Each part starts on a 256-byte boundary; the counters come first.
 struct WsLayout {
-  size_t seq_cnt, counters, g_counters, o_part, lse_part, g_part, g_lse, total;
+  size_t seq_cnt, counters, g_counters, split_cnt, o_part, lse_part, g_part, g_lse, total;
   int n_groups;
 };
 
-static WsLayout ws_layout(const hyb_cache_desc *d, int ns, bool step) {
-  WsLayout w{0, 0, 0, 0, 0, 0, 0, 0, 0};
+WsLayout ws_layout(const hyb_cache_desc *d, const Plan &pl, bool step) {
+  WsLayout w{0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
   size_t off = 0;
   if (step) {
     w.seq_cnt = 0;
     off = round_up(static_cast<size_t>(d->batch) * sizeof(int32_t), kWsAlign);
   }
-  if (ns > hyb::decode_max_cluster()) {
-    const size_t rows = static_cast<size_t>(d->batch) * d->num_q_heads;
-    const size_t units = static_cast<size_t>(d->batch) * d->num_kv_heads;
-    const size_t ng = ns > hyb::kMergeFan ? (ns + hyb::kMergeFan - 1) / hyb::kMergeFan : 0;
+  const size_t rows = static_cast<size_t>(d->batch) * d->num_q_heads;
+  const size_t units = static_cast<size_t>(d->batch) * d->num_kv_heads;
+  const size_t ns = static_cast<size_t>(pl.ns);
+  const size_t ng = ns > static_cast<size_t>(hyb::kMergeFan) ? (ns + hyb::kMergeFan - 1) / hyb::kMergeFan : 0;
+  if (pl.sk || (!pl.cluster && ns > 1)) {
     w.n_groups = static_cast<int>(ng);
     w.counters = off;
     off += round_up(units * sizeof(int32_t), kWsAlign);
     w.g_counters = off;
     off += round_up(units * ng * sizeof(int32_t), kWsAlign);
+    if (pl.sk) {
+      w.split_cnt = off;
+      off += round_up(units * ns * sizeof(int32_t), kWsAlign);
+    }
+    // partial results: [rows][ns] (one-wave) or [slots][Hq/Hkv] (persistent)
+    const size_t parts = pl.sk ? (units * ns + static_cast<size_t>(pl.grid)) * (rows / units) : rows * ns;
     w.o_part = off;
-    w.lse_part = w.o_part + round_up(rows * ns * hyb::kDim * sizeof(float), kWsAlign);
-    off = w.lse_part + round_up(rows * ns * sizeof(float), kWsAlign);
+    w.lse_part = w.o_part + round_up(parts * hyb::kDim * sizeof(float), kWsAlign);
+    off = w.lse_part + round_up(parts * sizeof(float), kWsAlign);
     w.g_part = off;
     w.g_lse = w.g_part + round_up(rows * ng * hyb::kDim * sizeof(float), kWsAlign);
     off = w.g_lse + round_up(rows * ng * sizeof(float), kWsAlign);
@@ -194,33 +253,43 @@ static WsLayout ws_layout(const hyb_cache_desc *d, int ns, bool step) {
   return w;
 }
 
-static size_t workspace_for(const hyb_cache_desc *d, int ns) { return ws_layout(d, ns, false).total; }
-
-}  // extern "C"
+}  // namespace
 
 namespace hyb {
 // Leading bytes of the hyb_decode_attn workspace that must be zero before a
 // call (the arrival counters); 0 when the workspace is not used.
-size_t decode_ws_zero_prefix(const hyb_cache_desc *d, int ns) {
-  const WsLayout w = ws_layout(d, ns, false);
+size_t decode_ws_zero_prefix(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens) {
+  Plan pl;
+  if (make_plan(d, max_seq_len, split_tokens, &pl) != HYB_OK) return 0;
+  const WsLayout w = ws_layout(d, pl, false);
   return w.total > 0 ? w.o_part : 0;
 }
 }  // namespace hyb
 
 extern "C" {
 
+int hyb_decode_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens,
+                    int32_t *split_tokens_out, int32_t *n_splits_out) {
+  Plan pl;
+  const int rc = make_plan(d, max_seq_len, split_tokens, &pl);
+  if (rc != HYB_OK) return rc;
+  if (split_tokens_out) *split_tokens_out = pl.tb * hyb::kBlock;
+  if (n_splits_out) *n_splits_out = pl.ns;
+  return HYB_OK;
+}
+
 size_t hyb_decode_workspace_bytes(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens) {
-  int32_t st = 0, ns = 0;
-  if (hyb_decode_plan(d, max_seq_len, split_tokens, &st, &ns) != HYB_OK) return 0;
-  return workspace_for(d, ns);
+  Plan pl;
+  if (make_plan(d, max_seq_len, split_tokens, &pl) != HYB_OK) return 0;
+  return ws_layout(d, pl, false).total;
 }
 
 static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_scale, int32_t max_seq_len,
                          int32_t split_tokens, void *workspace, size_t workspace_bytes, void *out,
                          float *lse_out, hyb_stream_t stream, const int32_t *n_new, const void *k_new,
                          const void *v_new) {
-  int32_t st = 0, ns = 0;
-  const int rc = hyb_decode_plan(d, max_seq_len, split_tokens, &st, &ns);
+  Plan pl;
+  const int rc = make_plan(d, max_seq_len, split_tokens, &pl);
   if (rc != HYB_OK) return rc;
   if (!q || !out || !aligned(q, 16) || !aligned(out, 16) || (lse_out && !aligned(lse_out, 4)) ||
       !std::isfinite(softmax_scale))
@@ -228,7 +297,7 @@ static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_s
   const bool step = n_new != nullptr;
   if (step && (!aligned(n_new, 4) || !k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)))
     return HYB_ERR_INVALID_VALUE;
-  const WsLayout wl = ws_layout(d, ns, step);
+  const WsLayout wl = ws_layout(d, pl, step);
   if (wl.total > 0 && (!workspace || workspace_bytes < wl.total || !aligned(workspace, 16)))
     return HYB_ERR_WORKSPACE;
   hyb::DecodeArgs a;
@@ -243,7 +312,7 @@ static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_s
   a.out = static_cast<__half *>(out);
   a.lse_out = lse_out;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  const bool merge_ws = ns > hyb::decode_max_cluster();
+  const bool merge_ws = pl.sk || (!pl.cluster && pl.ns > 1);
   a.counters = merge_ws ? reinterpret_cast<int32_t *>(ws + wl.counters) : nullptr;
   a.o_part = merge_ws ? reinterpret_cast<float *>(ws + wl.o_part) : nullptr;
   a.lse_part = merge_ws ? reinterpret_cast<float *>(ws + wl.lse_part) : nullptr;
@@ -251,13 +320,15 @@ static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_s
   a.g_counters = a.n_groups > 0 ? reinterpret_cast<int32_t *>(ws + wl.g_counters) : nullptr;
   a.g_part = a.n_groups > 0 ? reinterpret_cast<float *>(ws + wl.g_part) : nullptr;
   a.g_lse = a.n_groups > 0 ? reinterpret_cast<float *>(ws + wl.g_lse) : nullptr;
+  a.sk_split_cnt = pl.sk ? reinterpret_cast<int32_t *>(ws + wl.split_cnt) : nullptr;
+  a.batch = d->batch;
   a.hkv = d->num_kv_heads;
   a.hq = d->num_q_heads;
   a.num_phys = d->num_phys_blocks;
   a.max_blocks = d->max_blocks_per_seq;
   a.quant_bits = d->quant_bits;
-  a.n_splits = ns;
-  a.split_blocks = st / hyb::kBlock;
+  a.n_splits = pl.ns;
+  a.split_blocks = pl.tb;
   a.max_seq_len = max_seq_len;
   a.qk_scale = softmax_scale * 1.4426950408889634f;
   a.n_new = n_new;
@@ -265,7 +336,9 @@ static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_s
   a.v_new = static_cast<const __half *>(v_new);
   a.seq_cnt = step ? reinterpret_cast<int32_t *>(ws + wl.seq_cnt) : nullptr;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const cudaError_t e = hyb::launch_decode(a, d->num_q_heads / d->num_kv_heads, d->batch, s);
+  const int group = d->num_q_heads / d->num_kv_heads;
+  const cudaError_t e =
+      pl.sk ? hyb::launch_decode_sk(a, group, pl.grid, s) : hyb::launch_decode(a, group, d->batch, pl.cluster, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return HYB_OK;
 }
@@ -278,9 +351,9 @@ int hyb_decode_attn(const hyb_cache_desc *d, const void *q, float softmax_scale,
 }
 
 size_t hyb_decode_step_workspace_bytes(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens) {
-  int32_t st = 0, ns = 0;
-  if (hyb_decode_plan(d, max_seq_len, split_tokens, &st, &ns) != HYB_OK) return 0;
-  return ws_layout(d, ns, true).total;
+  Plan pl;
+  if (make_plan(d, max_seq_len, split_tokens, &pl) != HYB_OK) return 0;
+  return ws_layout(d, pl, true).total;
 }
 
 int hyb_decode_step(const hyb_cache_desc *d, const int32_t *n_new, const void *k_new, const void *v_new,

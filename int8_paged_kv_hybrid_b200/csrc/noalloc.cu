@@ -72,7 +72,7 @@ int hyb_decode_attn_noalloc(const hyb_cache_desc *desc, const void *q, float sof
       cudaGetLastError();
       return HYB_ERR_CUDA;
     }
-    const size_t zero = hyb::decode_ws_zero_prefix(desc, ns);
+    const size_t zero = hyb::decode_ws_zero_prefix(desc, max_seq_len, split_tokens);
     if (zero > 0) {
       const cudaError_t m = cudaMemsetAsync(ws, 0, zero, reinterpret_cast<cudaStream_t>(stream));
       if (m != cudaSuccess) {

@@ -100,6 +100,8 @@ def test_plan_and_workspace():
         st, ns = hk.hyb_decode_plan(d, L, 0)
         assert st % 64 == 0 and 64 <= st <= 8192 and ns >= 1
         assert ns == max(1, -(-max(0, L - 32) // st))
+    # one wave when every split fits on the GPU at once (4 x 8 units x 16 <= 444)
+    assert hk.hyb_decode_plan(d, 2048, 0)[1] >= 8
 
 
 def test_strerror_covers_codes():
