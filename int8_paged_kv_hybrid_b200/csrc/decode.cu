@@ -14,7 +14,10 @@
 // is one pipeline item, brought into a 3-stage shared-memory ring by the TMA
 // engine with one 1-D bulk copy (no cluster multicast) completing on an
 // mbarrier; every wait is bounded.  Three CTAs fit on an SM for up to 4 query
-// heads per kv head (two above that).
+// heads per kv head (two above that).  When all splits are resident at once
+// (one wave) 2..8 splits of a (sequence, kv head) run as one thread-block
+// cluster and merge through distributed shared memory; otherwise the last
+// split to finish merges them from the workspace.
 //
 // Arithmetic (per kv head, for its G = Hq/Hkv query heads):
 //  * q is turned into 16-bit fixed point per query head (q_i = rint(q * 32767
@@ -27,7 +30,7 @@
 //  * Warp w owns tokens 16w..16w+15 of every block and keeps its own online
 //    softmax state (running max, sum, FP32 output accumulator) per head,
 //    rescaling only when the running max grows.  Its softmax weights relative
-//    to the 16-token maximum are 16-bit fixed point (p_i = rint(32767 *
+//    to the running maximum are 16-bit fixed point (p_i = rint(32767 *
 //    2^(z - max))); P.V is again an exact int32 dp2a sum over the V codes,
 //    folded into the FP32 state with the V scale.
 //  * Hot tokens are attended in FP32 from the FP16 values (never quantized).

@@ -1,6 +1,5 @@
-// decode_dev.cuh -- device building blocks of the decode kernels (the
-// one-wave kernel in decode.cu and the persistent kernel in decode_sk.cu):
-// the per-item arithmetic on a staged cold block or hot ring, the fused
+// decode_dev.cuh -- device building blocks of the decode kernel
+// (decode.cu): the per-item arithmetic on a staged cold block or hot ring, the fused
 // append of the decode step, the merge of the four warps' softmax states and
 // the log-sum-exp merge of partial results.  The arithmetic is described at
 // the top of decode.cu.

@@ -117,23 +117,18 @@ int hyb_kv_append(const hyb_cache_desc *d, const int32_t *n_new, int32_t max_new
 
 namespace {
 
-// Use the persistent kernel for plans that do not fit in one wave (off: the
-// one-wave kernel over several waves of short splits measured faster).
-constexpr bool kPersistent = false;
 // Cold blocks per split when the splits take several waves.
 constexpr int kMultiWaveSplit = 16;
 
-// How a decode call runs.  One-wave kernel (decode.cu): grid (ns, Hkv, batch),
-// every split of every (sequence, kv head) resident at once -- chosen when
-// that fits on the GPU.  Otherwise the persistent kernel (decode_sk.cu): as
-// many CTAs as are resident at once, each taking an equal share of the cold
-// blocks of all sequences (batch <= its sequence table).
+// How a decode call runs: grid (ns, Hkv, batch) of the decode kernel.  When
+// every split fits on the GPU at once (one wave), automatic plans cut the
+// longest sequence into as many splits as fill the GPU, and 2..8 splits are
+// merged inside a thread-block cluster.  Otherwise the splits are short and
+// run in several waves, merged through the workspace.
 struct Plan {
-  bool sk;       // persistent kernel
-  bool cluster;  // one-wave kernel in clusters of ns CTAs (split merge in distributed shared memory)
-  int tb;        // cold blocks per split (persistent kernel: positions per split)
-  int ns;    // splits per (sequence, kv head), at most
-  int grid;  // persistent kernel: CTAs
+  bool cluster;  // clusters of ns CTAs (split merge in distributed shared memory)
+  int tb;        // cold blocks per split
+  int ns;        // splits per (sequence, kv head), at most
 };
 
 int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens, Plan *p) {
@@ -144,15 +139,12 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
                              ? (max_seq_len - hyb::kHot + hyb::kBlock - 1) / hyb::kBlock
                              : 0;
   if (nblk > d->max_blocks_per_seq) return HYB_ERR_INVALID_VALUE;
-  const long long npos = nblk > 0 ? nblk : 1;  // positions of a (sequence, kv head) in the persistent kernel
   const int group = d->num_q_heads / d->num_kv_heads;
   const int sms = sm_count();
   int occ = hyb::decode_ctas_per_sm(group);
   if (occ <= 0) occ = group <= 4 ? 3 : 2;
   const long long slots = static_cast<long long>(sms) * occ;
   const long long units = static_cast<long long>(d->batch) * d->num_kv_heads;
-  // persistent kernel: batch within its sequence table, positions in 32 bits
-  const bool sk_ok = d->batch <= hyb::decode_sk_max_batch() && units * npos < (1ll << 30);
   const int max_tb = hyb::decode_max_split_blocks();
   long long tb = 0;
   if (split_tokens == 0) {
@@ -164,14 +156,11 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
       if (tb > max_tb) tb = max_tb;
     }
     if (tb == 0 || units * ((nblk + tb - 1) / tb) > slots) {
-      if (sk_ok && kPersistent) {
-        tb = npos;  // persistent kernel, no split boundaries of its own
-      } else {
-        // several waves: short splits, so that the CTA scheduler evens out
-        // sequences of different lengths and CTAs of different speeds
-        tb = kMultiWaveSplit;
-        if (tb > nblk) tb = nblk > 0 ? nblk : 1;
-      }
+      // several waves: short splits, so that the CTA scheduler evens out
+      // sequences of different lengths and CTAs that run at different speeds
+      // (the last CTA placed on an SM gets the fewest issue slots)
+      tb = kMultiWaveSplit;
+      if (tb > nblk) tb = nblk > 0 ? nblk : 1;
     }
   } else {
     if (split_tokens < 0 || split_tokens % hyb::kBlock != 0) return HYB_ERR_INVALID_VALUE;
@@ -180,47 +169,30 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
   }
   long long ns = (nblk + tb - 1) / tb;
   if (ns < 1) ns = 1;
-  const bool one_wave = tb <= max_tb && units * ns <= slots;
-  p->sk = !one_wave && sk_ok && kPersistent;
+  if (tb > max_tb || ns > 65535) return HYB_ERR_INVALID_VALUE;
   // clusters only when every split is resident at once: a cluster holds its
-  // CTAs until the slowest split is done
-  p->cluster = !p->sk && one_wave && ns >= 2 && ns <= hyb::decode_max_cluster();
-  if (!p->sk && (tb > max_tb || ns > 65535)) return HYB_ERR_INVALID_VALUE;
-  if (p->sk) {
-    ns = (npos + tb - 1) / tb;
-    int occ_sk = hyb::decode_sk_ctas_per_sm(group);
-    if (occ_sk <= 0) occ_sk = group <= 4 ? 3 : 2;
-    long long grid = static_cast<long long>(sms) * occ_sk;
-    if (grid > units * npos) grid = units * npos;
-    p->grid = static_cast<int>(grid);
-  } else {
-    p->grid = 0;
-  }
-  if (tb * hyb::kBlock > 0x7fffffffLL || units * ns > 0x7fffffffLL) return HYB_ERR_INVALID_VALUE;
+  // CTAs until its slowest split is done
+  p->cluster = units * ns <= slots && ns >= 2 && ns <= hyb::decode_max_cluster();
   p->tb = static_cast<int>(tb);
   p->ns = static_cast<int>(ns);
   return HYB_OK;
 }
 
-// Workspace layout.  Fused step: read counters int32 [batch] first.
-// One-wave kernel with more splits than one cluster holds: arrival counters
-// int32 [batch][Hkv] and, with more than kMergeFan splits, group arrival
-// counters int32 [batch][Hkv][ng] (ng = ceil(ns / kMergeFan)); then the split
-// outputs FP32 [batch][Hq][ns][128] and their log2-sum-exp FP32
-// [batch][Hq][ns]; then the group outputs FP32 [batch][Hq][ng][128] and their
-// log2-sum-exp [batch][Hq][ng].
-// Persistent kernel: arrival counters per (sequence, kv head) and per group as
-// above, then per split int32 [batch][Hkv][ns]; then one partial result per
-// slot (slots = batch * Hkv * ns + grid): FP32 [slot][Hq/Hkv][128] and the
-// log2-sum-exp [slot][Hq/Hkv]; then the group outputs.
-// Each part starts on a 256-byte boundary; the counters come first.
+// Workspace layout.  Fused step: read counters int32 [batch] first.  Splits
+// merged through the workspace (not in a cluster): arrival counters int32
+// [batch][Hkv] and, with more than kMergeFan splits, group arrival counters
+// int32 [batch][Hkv][ng] (ng = ceil(ns / kMergeFan)); then the split outputs
+// FP32 [batch][Hq][ns][128] and their log2-sum-exp FP32 [batch][Hq][ns]; then
+// the group outputs FP32 [batch][Hq][ng][128] and their log2-sum-exp
+// [batch][Hq][ng].  Each part starts on a 256-byte boundary; the counters
+// come first.
 struct WsLayout {
-  size_t seq_cnt, counters, g_counters, split_cnt, o_part, lse_part, g_part, g_lse, total;
+  size_t seq_cnt, counters, g_counters, o_part, lse_part, g_part, g_lse, total;
   int n_groups;
 };
 
 WsLayout ws_layout(const hyb_cache_desc *d, const Plan &pl, bool step) {
-  WsLayout w{0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
+  WsLayout w{0, 0, 0, 0, 0, 0, 0, 0, 0};
   size_t off = 0;
   if (step) {
     w.seq_cnt = 0;
@@ -230,18 +202,13 @@ WsLayout ws_layout(const hyb_cache_desc *d, const Plan &pl, bool step) {
   const size_t units = static_cast<size_t>(d->batch) * d->num_kv_heads;
   const size_t ns = static_cast<size_t>(pl.ns);
   const size_t ng = ns > static_cast<size_t>(hyb::kMergeFan) ? (ns + hyb::kMergeFan - 1) / hyb::kMergeFan : 0;
-  if (pl.sk || (!pl.cluster && ns > 1)) {
+  if (!pl.cluster && ns > 1) {
     w.n_groups = static_cast<int>(ng);
     w.counters = off;
     off += round_up(units * sizeof(int32_t), kWsAlign);
     w.g_counters = off;
     off += round_up(units * ng * sizeof(int32_t), kWsAlign);
-    if (pl.sk) {
-      w.split_cnt = off;
-      off += round_up(units * ns * sizeof(int32_t), kWsAlign);
-    }
-    // partial results: [rows][ns] (one-wave) or [slots][Hq/Hkv] (persistent)
-    const size_t parts = pl.sk ? (units * ns + static_cast<size_t>(pl.grid)) * (rows / units) : rows * ns;
+    const size_t parts = rows * ns;
     w.o_part = off;
     w.lse_part = w.o_part + round_up(parts * hyb::kDim * sizeof(float), kWsAlign);
     off = w.lse_part + round_up(parts * sizeof(float), kWsAlign);
@@ -312,7 +279,7 @@ static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_s
   a.out = static_cast<__half *>(out);
   a.lse_out = lse_out;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  const bool merge_ws = pl.sk || (!pl.cluster && pl.ns > 1);
+  const bool merge_ws = !pl.cluster && pl.ns > 1;
   a.counters = merge_ws ? reinterpret_cast<int32_t *>(ws + wl.counters) : nullptr;
   a.o_part = merge_ws ? reinterpret_cast<float *>(ws + wl.o_part) : nullptr;
   a.lse_part = merge_ws ? reinterpret_cast<float *>(ws + wl.lse_part) : nullptr;
@@ -320,8 +287,6 @@ static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_s
   a.g_counters = a.n_groups > 0 ? reinterpret_cast<int32_t *>(ws + wl.g_counters) : nullptr;
   a.g_part = a.n_groups > 0 ? reinterpret_cast<float *>(ws + wl.g_part) : nullptr;
   a.g_lse = a.n_groups > 0 ? reinterpret_cast<float *>(ws + wl.g_lse) : nullptr;
-  a.sk_split_cnt = pl.sk ? reinterpret_cast<int32_t *>(ws + wl.split_cnt) : nullptr;
-  a.batch = d->batch;
   a.hkv = d->num_kv_heads;
   a.hq = d->num_q_heads;
   a.num_phys = d->num_phys_blocks;
@@ -337,8 +302,7 @@ static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_s
   a.seq_cnt = step ? reinterpret_cast<int32_t *>(ws + wl.seq_cnt) : nullptr;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int group = d->num_q_heads / d->num_kv_heads;
-  const cudaError_t e =
-      pl.sk ? hyb::launch_decode_sk(a, group, pl.grid, s) : hyb::launch_decode(a, group, d->batch, pl.cluster, s);
+  const cudaError_t e = hyb::launch_decode(a, group, d->batch, pl.cluster, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return HYB_OK;
 }

@@ -43,10 +43,6 @@ struct DecodeArgs {
   float *g_lse;
   int32_t *g_counters;
   int n_groups;
-  // persistent kernel: arrivals per split [n_split_slots] (zero between calls);
-  // o_part / lse_part then hold one partial per slot, [slot][Hq/Hkv][128]
-  int32_t *sk_split_cnt;
-  int batch;
   int hkv, hq, num_phys, max_blocks, quant_bits, n_splits, split_blocks, max_seq_len;
   float qk_scale;             // softmax_scale * log2(e)
   // fused decode step (null for attention only): append n_new[b] in {0, 1}
@@ -71,9 +67,6 @@ constexpr int kMergeFan = 16;
 
 cudaError_t launch_append(const AppendArgs &a, int batch, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream);
-cudaError_t launch_decode_sk(const DecodeArgs &a, int group, int grid, cudaStream_t stream);
-int decode_sk_max_batch();
-int decode_sk_ctas_per_sm(int group);
 cudaError_t launch_combine(const CombineArgs &a, int rows, cudaStream_t stream);
 int decode_max_split_blocks();
 int decode_ctas_per_sm(int group);
