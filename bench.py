@@ -33,7 +33,7 @@ METRIC = "decode-attn KV GB/s (frac of HBM peak) and tokens/s at 1 B200 vs CPU o
 UNIT = "GB/s"
 WORKLOAD = 2
 PROFILE = os.path.join(ROOT, "profiles", "decode_splitkv_llama8b_b8_L2048.md")
-KERNEL_SOURCES = ["decode.cu", "common.cuh", "kernels.cuh"]  # the profiled kernel's sources
+KERNEL_SOURCES = ["decode.cu", "decode_dev.cuh", "common.cuh", "kernels.cuh"]  # the profiled kernel's sources
 FLUSH_BYTES = 512 << 20   # > 126 MB L2
 
 
