@@ -62,6 +62,12 @@ def _load():
     lib.ora_get_block.argtypes = [P, i32, i32, P, P]
     lib.ora_get_ring.argtypes = [P, i32, P]
     lib.ora_export.argtypes = [P, P, i32, P, P, P, P]
+    lib.ora_migrate.argtypes = [P, P]
+    lib.ora_n_int4.argtypes = [P, i32]
+    lib.ora_n_int4.restype = ctypes.c_int32
+    lib.ora_migration_threshold_ms.argtypes = [P, i32]
+    lib.ora_migration_threshold_ms.restype = ctypes.c_double
+    lib.ora_migration_decision.argtypes = [ctypes.c_double, ctypes.c_double, i32]
     lib.ora_half_to_double.argtypes = [ctypes.c_uint16]
     lib.ora_half_to_double.restype = ctypes.c_double
     _lib = lib
@@ -116,6 +122,17 @@ class OracleCache:
         if rc != 0:
             raise ValueError("oracle append rejected (rc=%d)" % rc)
 
+    def migrate(self, target_n_int4):
+        """Move each sequence's INT4 block count to target_n_int4[b],
+        re-quantizing the blocks in between (see ora_migrate)."""
+        t = _c(target_n_int4, np.int32)
+        rc = self._lib.ora_migrate(self._h, _ptr(t))
+        if rc != 0:
+            raise ValueError("oracle migrate rejected (rc=%d)" % rc)
+
+    def n_int4(self):
+        return np.array([self._lib.ora_n_int4(self._h, b) for b in range(self.batch)], np.int32)
+
     def lens(self):
         return np.array([self._lib.ora_len(self._h, b) for b in range(self.batch)], np.int32)
 
@@ -164,6 +181,17 @@ class OracleCache:
         if rc != 0:
             raise ValueError("oracle export failed (rc=%d)" % rc)
         return dict(cold=cold, scales=sc, hot=hot.view(np.float16), seq_lens=sl)
+
+
+def migration_threshold_ms(lens):
+    """Adaptive migration threshold in ms (see ora_migration_threshold_ms)."""
+    a = _c(np.asarray(lens, np.int32), np.int32)
+    return float(_load().ora_migration_threshold_ms(_ptr(a), a.size))
+
+
+def migration_decision(avg_interval_ms, threshold_ms, is_int4):
+    """+1 promote (INT4 -> INT8), -1 demote (INT8 -> INT4), 0 keep."""
+    return int(_load().ora_migration_decision(float(avg_interval_ms), float(threshold_ms), 1 if is_int4 else 0))
 
 
 def combine(o_part, lse_part):

@@ -236,6 +236,91 @@ int ora_append(ora_cache *c, const int32_t *n_new, int max_new,
   return ORA_OK;
 }
 
+/*
+ * Tier migration, [hybrid_v2 page] section 3.3: a cold block moves between
+ * the INT8 ("L1") and the INT4 ("L2") tier and is given a new scale in place
+ * (section 3.2).  The tier is kept as a count per sequence -- logical blocks
+ * below n_int4[b] are INT4 -- so a migration moves that count to target[b]:
+ * every sealed block between the old and the new count is re-quantized to
+ * the other width, per (kv head, K|V):
+ *   a = max over the block of |code * scale|          (FP32)
+ *   scale' = a / Q'                                    (Q' = 7 or 127)
+ *   code' = clamp(round-half-even(code * scale / scale'), -Q', Q')
+ * (the arithmetic ora_append uses to re-quantize a tail block; a block of
+ * zeros gets scale 0 and codes 0).  Blocks with no sealed token only change
+ * tier.  Returns ORA_ERR_INVALID and changes nothing for a target outside
+ * [0, max_blocks], or for a cache whose cold zone is all INT4.
+ */
+int ora_migrate(ora_cache *c, const int32_t *target) {
+  const int d = c->d, blk = c->block, hkv = c->hkv;
+  if (c->quant_bits != 8) return ORA_ERR_INVALID;
+  for (int b = 0; b < c->batch; b++)
+    if (target[b] < 0 || target[b] > c->max_blocks) return ORA_ERR_INVALID;
+  for (int b = 0; b < c->batch; b++) {
+    const int cur = c->n_int4[b], tgt = target[b];
+    const int lo = cur < tgt ? cur : tgt, hi = cur < tgt ? tgt : cur;
+    for (int i = lo; i < hi; i++) {
+      const size_t bi = (size_t)b * c->max_blocks + i;
+      if (!c->codes[bi]) continue; /* nothing sealed yet */
+      const int q = i < tgt ? 7 : 127;
+      for (int h = 0; h < hkv; h++) {
+        for (int kv = 0; kv < 2; kv++) {
+          int8_t *cd = c->codes[bi] + ((size_t)h * 2 + kv) * blk * d;
+          float *sp = c->scale[bi] + h * 2 + kv;
+          const float s_old = *sp;
+          float a = 0.0f;
+          for (int t = 0; t < blk; t++)
+            for (int ch = 0; ch < d; ch++) {
+              float x = fabsf((float)cd[t * d + ch] * s_old);
+              if (x > a) a = x;
+            }
+          const float s_new = a / (float)q;
+          for (int t = 0; t < blk; t++)
+            for (int ch = 0; ch < d; ch++) {
+              float v = (float)cd[t * d + ch] * s_old;
+              cd[t * d + ch] = (int8_t)(s_new == 0.0f ? 0 : clampi((int)rne(v / s_new), q));
+            }
+          *sp = s_new;
+        }
+      }
+      c->qmax[bi] = q;
+    }
+    c->n_int4[b] = tgt;
+  }
+  return ORA_OK;
+}
+
+int32_t ora_n_int4(const ora_cache *c, int b) { return c->n_int4[b]; }
+
+/*
+ * Adaptive migration threshold, [hybrid_v2 page] section 3.3, in ms:
+ * 3000 * (1 + 0.2 * load_factor), load_factor = geometric mean of the
+ * batch's sequence lengths / 512.  Sequences of length 0 are left out of the
+ * mean (no sequence at all: load_factor 0).
+ */
+double ora_migration_threshold_ms(const int32_t *lens, int n) {
+  double log_sum = 0.0;
+  int m = 0;
+  for (int i = 0; i < n; i++)
+    if (lens[i] > 0) {
+      log_sum += log((double)lens[i]);
+      m++;
+    }
+  const double load_factor = m > 0 ? exp(log_sum / m) / 512.0 : 0.0;
+  return 3000.0 * (1.0 + 0.2 * load_factor);
+}
+
+/*
+ * Per-block decision of section 3.3: an INT4 ("L2") block whose mean access
+ * interval is below the threshold moves up (+1); an INT8 ("L1") block whose
+ * mean interval is above 1.5 x the threshold moves down (-1); otherwise 0.
+ */
+int ora_migration_decision(double avg_interval_ms, double threshold_ms, int is_int4) {
+  if (is_int4 && avg_interval_ms < threshold_ms) return 1;
+  if (!is_int4 && avg_interval_ms > 1.5 * threshold_ms) return -1;
+  return 0;
+}
+
 /* Value of position p (channel ch) of head h, K (kv=0) or V (kv=1), in FP64:
  * hot FP16 value, or code * scale for a cold position. */
 static double kv_value(const ora_cache *c, int b, int h, int kv, int p, int ch) {

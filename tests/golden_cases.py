@@ -37,6 +37,8 @@ def parse_cases(fname):
                 cur["tokens"][(pos, kv)] = vals
             elif tok[0] == "append":
                 cur["ops"].append(("append", int(tok[1].split("=")[1])))
+            elif tok[0] == "migrate":
+                cur["ops"].append(("migrate", int(tok[1].split("=")[1])))
             elif tok[0] == "check":
                 spec = {}
                 codes = None
