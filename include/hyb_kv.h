@@ -22,6 +22,10 @@
  *                      ([hybrid_v2 page] 4.2, steps 3-5)
  *   hyb_decode_step    the two above fused: append of one token per sequence
  *                      and attention in a single launch
+ *   hyb_kv_migrate     move cold blocks between the INT8 and the INT4 tier in
+ *                      place with new scales ([hybrid_v2 page] 3.2, 3.3), and
+ *                      hyb_migration_threshold_ms / hyb_migration_decision,
+ *                      the page's adaptive migration policy (host functions)
  *   hyb_combine        log-sum-exp merge of split partial results (the merge
  *                      that replaces the page's torch.cat of step 5)
  *
@@ -72,6 +76,9 @@ typedef struct CUstream_st *hyb_stream_t; /* same type as cudaStream_t */
                                       sequence b left unchanged */
 #define HYB_STATUS_SEQ_LEN 4       /* seq_lens[b] < 0 or > max_seq_len at decode; b skipped */
 #define HYB_STATUS_TIMEOUT 5       /* a bounded wait inside a kernel gave up; unit skipped */
+#define HYB_STATUS_BAD_TIER 6      /* hyb_kv_migrate: target[b] outside [0, max_blocks_per_seq] or
+                                      more than max_delta blocks from n_int4_blocks[b]; sequence
+                                      left unchanged */
 
 /*
  * The cache descriptor (host struct; the pointers inside are device memory).
@@ -306,6 +313,58 @@ size_t hyb_decode_step_workspace_bytes(const hyb_cache_desc *desc, int32_t max_s
 int hyb_combine(int32_t batch, int32_t num_q_heads, int32_t head_dim, int32_t n_splits,
                 const float *o_partial, const float *lse_partial, void *out, float *lse_out,
                 hyb_stream_t stream);
+
+/*
+ * hyb_kv_migrate -- move cold blocks between the INT8 ("L1") and the INT4
+ * ("L2") tier in place ([hybrid_v2 page] 3.3: blocks are promoted or demoted
+ * by their access interval; 3.2: a block that changes tier is given a new
+ * scale inside the kernel, with no host copy).
+ *
+ * The tier is a count per sequence: logical blocks below n_int4_blocks[b]
+ * are INT4.  For every sequence that count moves to target_n_int4[b]; each
+ * block holding a sealed token between the old and the new count is
+ * re-quantized to the other width, per (kv head, K|V):
+ *   scale' = max|code * scale| / Q'   (Q' = 7 or 127, IEEE FP32 division)
+ *   code'  = clamp(round-half-even(code * scale / scale'), -Q', Q')
+ * -- the arithmetic of a tail block's re-quantization in hyb_kv_append; an
+ * all-zero tile gets scale 0.  A demoted tile is rewritten in INT4 in its
+ * first 4096 bytes and its other 4096 bytes are zeroed; a promoted tile is
+ * rewritten whole; slots not yet sealed get code 0.  Blocks with nothing
+ * sealed only change tier (later appends seal into them at the new width).
+ * Then n_int4_blocks[b] = target_n_int4[b].  Moving a tier back does not
+ * restore precision an INT4 round lost.
+ *
+ *   desc           quant_bits 8 and n_int4_blocks non-NULL; this is the one
+ *                  call that writes through desc->n_int4_blocks.
+ *   target_n_int4  device int32 [batch], 4-byte aligned, each in
+ *                  [0, max_blocks_per_seq].
+ *   max_delta      host upper bound of |target_n_int4[b] - n_int4_blocks[b]|
+ *                  over the batch (it sizes the grid), 0..max_blocks_per_seq.
+ * Returns HYB_OK, HYB_ERR_INVALID_VALUE (bad descriptor, NULL n_int4_blocks,
+ * NULL or misaligned target, max_delta out of range), HYB_ERR_UNSUPPORTED
+ * (quant_bits 4: every block is INT4 already) or HYB_ERR_CUDA.  Device
+ * errors: HYB_STATUS_BAD_TIER (that sequence left unchanged) and
+ * HYB_STATUS_BAD_BLOCK (that block skipped).  Asynchronous on `stream`; it
+ * must not overlap on the GPU with any other call on the same cache.
+ */
+int hyb_kv_migrate(const hyb_cache_desc *desc, const int32_t *target_n_int4, int32_t max_delta,
+                   hyb_stream_t stream);
+
+/*
+ * The adaptive migration threshold of [hybrid_v2 page] 3.3, in ms (host
+ * function, no GPU): 3000 * (1 + 0.2 * load_factor), load_factor = geometric
+ * mean of the batch's sequence lengths / 512.  seq_lens is a HOST array of n
+ * entries; lengths <= 0 are left out of the mean (none left: load_factor 0).
+ * Returns 3000 for n <= 0 or a NULL array.
+ */
+double hyb_migration_threshold_ms(const int32_t *seq_lens, int32_t n);
+
+/*
+ * The page's decision for one block (host function): +1 promote an INT4
+ * block whose mean access interval is below the threshold, -1 demote an INT8
+ * block whose mean interval is above 1.5 x the threshold, 0 otherwise.
+ */
+int hyb_migration_decision(double avg_interval_ms, double threshold_ms, int32_t block_is_int4);
 
 /* Copy the device status word to *host_status (waits for `stream`), and
  * reset it to 0 when `clear` is nonzero. */

@@ -3,13 +3,14 @@
 The hot zone keeps the most recent 32 tokens of every sequence in FP16; older
 tokens live in 64-token INT8 (or INT4) cold blocks behind a block table.  The
 library (libhybkv.so, C ABI in include/hyb_kv.h) provides the append /
-quantize kernel, the split-KV decode attention kernel and the log-sum-exp
-combine.  This package is its thin Python binding.
+quantize kernel, the split-KV decode attention kernel, the log-sum-exp
+combine and the INT8 <-> INT4 tier migration.  This package is its thin
+Python binding.
 """
 from ._lib import (  # noqa: F401
     CacheDesc, HybError, hyb_check_desc, hyb_combine, hyb_decode_attn, hyb_decode_plan,
     hyb_decode_step, hyb_decode_step_workspace_bytes,
-    hyb_decode_workspace_bytes, hyb_kv_append, hyb_last_cuda_error, hyb_read_status,
-    hyb_version, load, strerror,
+    hyb_decode_workspace_bytes, hyb_kv_append, hyb_kv_migrate, hyb_last_cuda_error,
+    hyb_migration_decision, hyb_migration_threshold_ms, hyb_read_status, hyb_version, load, strerror,
 )
 from .cache import HybridKVCache  # noqa: F401

@@ -26,12 +26,14 @@ HYB_STATUS_BAD_N_NEW = 2
 HYB_STATUS_CAPACITY = 3
 HYB_STATUS_SEQ_LEN = 4
 HYB_STATUS_TIMEOUT = 5
+HYB_STATUS_BAD_TIER = 6
 
 EXPORTED = (
     "hyb_check_desc", "hyb_kv_append", "hyb_decode_plan", "hyb_decode_workspace_bytes",
     "hyb_decode_attn", "hyb_decode_step", "hyb_decode_step_workspace_bytes", "hyb_combine",
     "hyb_read_status", "hyb_strerror",
     "hyb_last_cuda_error", "hyb_version", "hyb_decode_attn_noalloc", "hyb_noalloc_scratch_limit",
+    "hyb_kv_migrate", "hyb_migration_threshold_ms", "hyb_migration_decision",
 )
 
 
@@ -92,11 +94,16 @@ def load(path: str = LIB_PATH):
     lib.hyb_decode_attn_noalloc.restype = ctypes.c_int
     lib.hyb_noalloc_scratch_limit.argtypes = []
     lib.hyb_noalloc_scratch_limit.restype = sz
+    lib.hyb_kv_migrate.argtypes = [D, P, i32, P]
+    lib.hyb_migration_threshold_ms.argtypes = [ctypes.POINTER(i32), i32]
+    lib.hyb_migration_threshold_ms.restype = ctypes.c_double
+    lib.hyb_migration_decision.argtypes = [ctypes.c_double, ctypes.c_double, i32]
+    lib.hyb_migration_decision.restype = ctypes.c_int
     lib.hyb_read_status.argtypes = [D, ctypes.POINTER(i32), i32, P]
     lib.hyb_strerror.argtypes = [ctypes.c_int]
     lib.hyb_strerror.restype = ctypes.c_char_p
     for name in ("hyb_check_desc", "hyb_kv_append", "hyb_decode_plan", "hyb_decode_attn", "hyb_decode_step",
-                 "hyb_combine", "hyb_read_status", "hyb_last_cuda_error", "hyb_version"):
+                 "hyb_combine", "hyb_read_status", "hyb_last_cuda_error", "hyb_version", "hyb_kv_migrate"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -181,6 +188,24 @@ def hyb_combine(batch, num_q_heads, head_dim, n_splits, o_partial, lse_partial, 
     _check(load().hyb_combine(int(batch), int(num_q_heads), int(head_dim), int(n_splits),
                               _ptr(o_partial), _ptr(lse_partial), _ptr(out), _ptr(lse_out),
                               _stream(stream)), "hyb_combine")
+
+
+def hyb_kv_migrate(desc, target_n_int4, max_delta, stream=None):
+    """target_n_int4: int32 CUDA tensor [batch]; max_delta: host bound on the move."""
+    _check(load().hyb_kv_migrate(ctypes.byref(desc), _ptr(target_n_int4), int(max_delta), _stream(stream)),
+           "hyb_kv_migrate")
+
+
+def hyb_migration_threshold_ms(seq_lens) -> float:
+    """Adaptive migration threshold (ms) for host sequence lengths."""
+    lens = [int(x) for x in seq_lens]
+    arr = (ctypes.c_int32 * max(1, len(lens)))(*lens)
+    return float(load().hyb_migration_threshold_ms(arr, len(lens)))
+
+
+def hyb_migration_decision(avg_interval_ms, threshold_ms, block_is_int4) -> int:
+    """+1 promote (INT4 -> INT8), -1 demote (INT8 -> INT4), 0 keep."""
+    return int(load().hyb_migration_decision(float(avg_interval_ms), float(threshold_ms), 1 if block_is_int4 else 0))
 
 
 def hyb_read_status(desc, clear=False, stream=None) -> int:

@@ -63,6 +63,18 @@ class HybridKVCache:
         assert k_new.is_contiguous() and v_new.is_contiguous() and n_new.is_contiguous()
         _lib.hyb_kv_append(self.desc, n_new, k_new.shape[1], k_new, v_new, stream)
 
+    def migrate(self, target_n_int4, max_delta=None, stream=None):
+        """Move every sequence's INT4 block count to target_n_int4 (int32
+        [batch], host or CUDA), re-quantizing the blocks in between in place
+        (hyb_kv_migrate).  max_delta: bound on the move (default: the table width)."""
+        import torch
+        if self.n_int4 is None:
+            self.n_int4 = torch.zeros(self.batch, dtype=torch.int32, device=self.device)
+            self.desc = self._make_desc()
+        tgt = torch.as_tensor(target_n_int4, dtype=torch.int32).to(self.device).contiguous()
+        md = self.max_blocks if max_delta is None else int(max_delta)
+        _lib.hyb_kv_migrate(self.desc, tgt, md, stream)
+
     def plan(self, max_seq_len, split_tokens=0):
         return _lib.hyb_decode_plan(self.desc, max_seq_len, split_tokens)
 

@@ -57,6 +57,8 @@ const char *hyb_strerror(int code) {
     case 100 + HYB_STATUS_CAPACITY: return "device status: sequence outgrew its block table";
     case 100 + HYB_STATUS_SEQ_LEN: return "device status: seq_lens out of range for decode";
     case 100 + HYB_STATUS_TIMEOUT: return "device status: a bounded wait in a kernel ran out";
+    case 100 + HYB_STATUS_BAD_TIER:
+      return "device status: a migration target outside the block table or beyond max_delta";
     default: return "unknown code";
   }
 }
@@ -341,6 +343,47 @@ int hyb_combine(int32_t batch, int32_t num_q_heads, int32_t head_dim, int32_t n_
   hyb::CombineArgs c{o_partial, lse_partial, static_cast<__half *>(out), lse_out, n_splits};
   const cudaError_t e = hyb::launch_combine(c, static_cast<int>(rows), reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HYB_OK : cuda_fail(e);
+}
+
+int hyb_kv_migrate(const hyb_cache_desc *d, const int32_t *target_n_int4, int32_t max_delta,
+                   hyb_stream_t stream) {
+  const int rc = hyb_check_desc(d);
+  if (rc != HYB_OK) return rc;
+  if (d->quant_bits != 8) return HYB_ERR_UNSUPPORTED;
+  if (!d->n_int4_blocks || !aligned(d->n_int4_blocks, 4) || !target_n_int4 || !aligned(target_n_int4, 4) ||
+      max_delta < 0 || max_delta > d->max_blocks_per_seq)
+    return HYB_ERR_INVALID_VALUE;
+  hyb::MigrateArgs a;
+  a.cold = static_cast<uint8_t *>(d->cold);
+  a.scales = d->scales;
+  a.block_table = d->block_table;
+  a.seq_lens = d->seq_lens;
+  a.n_int4 = const_cast<int32_t *>(d->n_int4_blocks);
+  a.target = target_n_int4;
+  a.status = d->status;
+  a.hkv = d->num_kv_heads;
+  a.num_phys = d->num_phys_blocks;
+  a.max_blocks = d->max_blocks_per_seq;
+  a.max_delta = max_delta;
+  const cudaError_t e = hyb::launch_migrate(a, d->batch, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HYB_OK : cuda_fail(e);
+}
+
+double hyb_migration_threshold_ms(const int32_t *seq_lens, int32_t n) {
+  double log_sum = 0.0;
+  int used = 0;
+  for (int32_t i = 0; seq_lens && i < n; i++)
+    if (seq_lens[i] > 0) {
+      log_sum += std::log(static_cast<double>(seq_lens[i]));
+      used++;
+    }
+  const double load_factor = used > 0 ? std::exp(log_sum / used) / 512.0 : 0.0;
+  return 3000.0 * (1.0 + 0.2 * load_factor);
+}
+
+int hyb_migration_decision(double avg_interval_ms, double threshold_ms, int32_t block_is_int4) {
+  if (block_is_int4) return avg_interval_ms < threshold_ms ? 1 : 0;
+  return avg_interval_ms > 1.5 * threshold_ms ? -1 : 0;
 }
 
 int hyb_read_status(const hyb_cache_desc *d, int32_t *host_status, int32_t clear, hyb_stream_t stream) {

@@ -54,6 +54,17 @@ struct DecodeArgs {
   int32_t *seq_cnt;
 };
 
+struct MigrateArgs {
+  uint8_t *cold;              // [num_phys][Hkv][2][8192]
+  float *scales;              // [num_phys][Hkv][2]
+  const int32_t *block_table; // [batch][max_blocks]
+  const int32_t *seq_lens;    // [batch]
+  int32_t *n_int4;            // [batch]: INT4 blocks per sequence, moved to target
+  const int32_t *target;      // [batch]
+  int32_t *status;
+  int hkv, num_phys, max_blocks, max_delta;
+};
+
 struct CombineArgs {
   const float *o_part;        // [rows][n_splits][128]
   const float *lse_part;      // [rows][n_splits]
@@ -67,6 +78,7 @@ constexpr int kMergeFan = 16;
 
 cudaError_t launch_append(const AppendArgs &a, int batch, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream);
+cudaError_t launch_migrate(const MigrateArgs &a, int batch, cudaStream_t stream);
 cudaError_t launch_combine(const CombineArgs &a, int rows, cudaStream_t stream);
 int decode_max_split_blocks();
 int decode_ctas_per_sm(int group);

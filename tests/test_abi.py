@@ -133,3 +133,42 @@ def test_workload_shapes():
         used = w.block_table[w.block_table >= 0]
         assert len(np.unique(used)) == len(used) and used.max() < w.num_phys_blocks
         assert sum(int(s.sum()) for s in w.schedule) == int(w.lens.sum())
+
+
+def test_migration_policy_matches_fixture_and_oracle():
+    """hyb_migration_threshold_ms / hyb_migration_decision (host functions)
+    against the page's worked example (tests/golden/migration_threshold.txt)
+    and the oracle's restatement on random batches."""
+    import oracle
+    for line in open(os.path.join(GOLDEN, "migration_threshold.txt"), encoding="utf-8"):
+        f = line.split("#", 1)[0].split()
+        if f:
+            want, lens = float(f[0]), [int(x) for x in f[1:]]
+            assert abs(hk.hyb_migration_threshold_ms(lens) - want) <= 1e-9 * want, lens
+    rng = np.random.default_rng(5)
+    for _ in range(50):
+        lens = rng.integers(0, 200000, size=int(rng.integers(1, 64))).tolist()
+        t = hk.hyb_migration_threshold_ms(lens)
+        assert abs(t - oracle.migration_threshold_ms(lens)) <= 1e-9 * t
+        for iai in (0.5 * t, t, 1.2 * t, 1.5 * t, 2.0 * t):
+            for int4 in (True, False):
+                assert hk.hyb_migration_decision(iai, t, int4) == oracle.migration_decision(iai, t, int4)
+
+
+def test_migrate_argument_checks():
+    """hyb_kv_migrate rejects bad arguments on the host, before any launch."""
+    lib = hk.load()
+    d = _desc(batch=4, maxb=16, phys=64)
+    tgt = ctypes.c_void_p(0x7f0000400000)
+    # no per-sequence INT4 counts to move
+    assert lib.hyb_kv_migrate(ctypes.byref(d), tgt, 1, None) == _lib.HYB_ERR_INVALID_VALUE
+    d.n_int4_blocks = 0x7f0000330000
+    assert lib.hyb_kv_migrate(ctypes.byref(d), None, 1, None) == _lib.HYB_ERR_INVALID_VALUE
+    assert lib.hyb_kv_migrate(ctypes.byref(d), ctypes.c_void_p(0x7f0000400002), 1, None) == \
+        _lib.HYB_ERR_INVALID_VALUE  # misaligned target
+    for bad in (-1, 17):
+        assert lib.hyb_kv_migrate(ctypes.byref(d), tgt, bad, None) == _lib.HYB_ERR_INVALID_VALUE
+    d4 = _desc(batch=4, maxb=16, phys=64, qbits=4)
+    d4.n_int4_blocks = 0x7f0000330000
+    assert lib.hyb_kv_migrate(ctypes.byref(d4), tgt, 1, None) == _lib.HYB_ERR_UNSUPPORTED
+    assert "migration" in hk.strerror(100 + _lib.HYB_STATUS_BAD_TIER)
