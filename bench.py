@@ -47,6 +47,9 @@ def parse():
     p.add_argument("--workload", type=int, default=WORKLOAD,
                    help="1..5: the measured shapes (2, the default, is the headline workload)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--migrate", action="store_true",
+                   help="time hyb_kv_migrate instead of the decode step: demote a quarter of every "
+                        "sequence's cold blocks to INT4 and promote them back (workload default 3)")
     p.add_argument("--lean", action="store_true",
                    help="profiling run: no state restore, L2 flush, e2e or CPU baseline")
     return p.parse_args()
@@ -354,6 +357,70 @@ def run_native(args, rank, world, local_rank):
     return res, w
 
 
+def run_migrate(args):
+    """Tier migration on one GPU: per timed step, one hyb_kv_migrate call that
+    demotes the next quarter of every sequence's cold blocks (INT8 -> INT4),
+    and one that promotes them back, alternating; L2 flushed before each."""
+    import numpy as np
+    import torch
+    from int8_paged_kv_hybrid_b200 import synth
+    wl = args.workload if args.workload != WORKLOAD else 3
+    w = synth.make_workload(wl)
+    cache, n_last, k_last, v_last, q = build_gpu_state(w, torch)
+    cache.append(torch.from_numpy(n_last).cuda(), torch.from_numpy(k_last).cuda(), torch.from_numpy(v_last).cuda())
+    nb = w.cold_blocks()
+    n0 = np.zeros(w.batch, np.int32) if w.n_int4 is None else w.n_int4.astype(np.int32)
+    n1 = np.minimum(nb, n0 + nb // 4).astype(np.int32)
+    moved = int((n1 - n0).sum()) * w.num_kv_heads  # (block, kv head) tile pairs per call
+    delta = int((n1 - n0).max())
+    t_down = torch.from_numpy(n1).cuda()
+    t_up = torch.from_numpy(n0).cuda()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    clocks = ClockSampler(0)
+    times = {"demote": [], "promote": []}
+    for i in range(2 * (args.warmup + args.steps)):
+        kind = "demote" if i % 2 == 0 else "promote"
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        cache.migrate(t_down if kind == "demote" else t_up, delta)
+        e1.record()
+        if i == 2 * args.warmup:
+            torch.cuda.synchronize()
+            clocks.mark()
+        if i >= 2 * args.warmup:
+            times[kind].append((e0, e1))
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    assert cache.status() == 0
+    ms = {k: sum(a.elapsed_time(b) for a, b in v) / len(v) for k, v in times.items()}
+    peak, peak_kind = measured_peaks()
+    tile = 2 * 8192
+    # algorithmic bytes: the old tiles read and the new codes written (plus the
+    # 8-byte scale pair read and written); a demotion also zeroes the unused
+    # half of each tile (8 KB), counted in "bytes_written" but not here
+    alg = {"demote": moved * (tile + tile // 2 + 16), "promote": moved * (tile // 2 + tile + 16)}
+    gbs = {k: alg[k] / (ms[k] * 1e-3) / 1e9 for k in ms}
+    return {
+        "metric": "hyb_kv_migrate GB/s of tiles re-quantized (INT8 -> INT4 demotion; promotion in 'promote')",
+        "value": round(gbs["demote"], 1), "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms["demote"], 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": dict(workload_config(w, 0, 0), migration="quarter of every sequence's cold blocks: "
+                       "%d tile pairs per call, max_delta %d" % (moved, delta)),
+        "promote": {"value": round(gbs["promote"], 1), "unit": "GB/s", "ms_per_step": round(ms["promote"], 5)},
+        "roofline": {"bound": "hbm", "achieved": round(gbs["demote"], 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(gbs["demote"] / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                     "kernel": "hyb::migrate_kernel",
+                     "achieved_bytes": "per call: %d tile pairs x (16384 read + 8192 written + 16 scale bytes)"
+                                       % moved,
+                     "promote_frac": round(gbs["promote"] / peak, 4)},
+        "bytes_written_demote": moved * (tile // 2 + tile // 2 + 8),
+        "gpu_launches": 2 * args.steps * 2,
+        "clocks": clk,
+    }
+
+
 def oracle_step_rate(w, steps, warmup, budget_s=None):
     """Time the CPU oracle (as it stands) on the same workload: per step the
     1-token append plus FP64 attention of every (sequence, head).  The state
@@ -416,6 +483,10 @@ def main():
         return 0
 
     import torch
+    if args.migrate:
+        if rank == 0:
+            print(json.dumps(run_migrate(args)))
+        return 0
     if world > 1:
         import datetime
         import torch.distributed as dist

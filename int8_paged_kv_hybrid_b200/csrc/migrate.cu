@@ -14,11 +14,11 @@
 // -- the arithmetic of a tail block's re-quantization in hyb_kv_append, so the
 // result is bit-exact with the oracle.
 //
-// One CTA per (block to move, kv head, sequence): the K and V tiles are
-// unpacked into shared memory (codes of slots not yet sealed are taken as 0),
-// the new scale and a 255-entry code table are computed, and the tiles are
-// written back in the new packing (a demoted tile's unused upper 4 KB is
-// zeroed).  A second launch then commits the new counts, after every CTA of
+// One CTA per (block to move, kv head, sequence): each thread holds its part
+// of the K and V tiles in registers (codes of slots not yet sealed are taken
+// as 0), the new scale and a 256-entry code table are computed, and the
+// tiles are written back in the new packing (a demoted tile's unused upper
+// 4 KB is zeroed).  A second launch then commits the new counts, after every CTA of
 // the first has read the old ones.
 #include "kernels.cuh"
 
@@ -38,6 +38,21 @@ __device__ __forceinline__ bool tier_move(const MigrateArgs &a, int b, int &lo, 
   lo = min(cur, tgt);
   hi = max(cur, tgt);
   return true;
+}
+
+// Four table entries for the four INT8 codes of x, as bytes of one word.
+// Entry u of the table holds the new code of the INT8 code whose byte is
+// (u - 127) mod 256 (the -128 byte, never produced, reads as -127).
+__device__ __forceinline__ uint32_t tbl4(const uint8_t *tbl, uint32_t x) {
+  const uint32_t u = __vadd4(x, 0x7f7f7f7fu);  // per-byte index
+  return static_cast<uint32_t>(tbl[u & 0xff]) | (static_cast<uint32_t>(tbl[(u >> 8) & 0xff]) << 8) |
+         (static_cast<uint32_t>(tbl[(u >> 16) & 0xff]) << 16) | (static_cast<uint32_t>(tbl[u >> 24]) << 24);
+}
+
+// Largest |code| of the four INT8 codes of x (-128 read as 127).
+__device__ __forceinline__ uint32_t absmax4(uint32_t x) {
+  const uint32_t a = __vabsss4(x);  // per-byte |code|, saturating
+  return max(max(a & 0xff, (a >> 8) & 0xff), max((a >> 16) & 0xff, a >> 24));
 }
 
 __global__ void __launch_bounds__(kMigThreads) migrate_kernel(const MigrateArgs a) {
@@ -61,138 +76,133 @@ __global__ void __launch_bounds__(kMigThreads) migrate_kernel(const MigrateArgs 
   const bool demote = i < tgt;  // INT8 -> INT4
   const int qn = demote ? 7 : 127;
 
-  __shared__ __align__(16) int8_t cs[2][kBlock][kDim];  // codes, logical [kv][slot][channel]
   __shared__ int red[2][kMigWarps];
   __shared__ float s_new[2];
-  __shared__ int8_t tbl[2][256];
+  __shared__ uint8_t tbl[2][256];
   uint8_t *tile = a.cold + ((size_t)phys * a.hkv + h) * kTilePairBytes;
 
-  // ---- unpack the old tiles; slots not yet sealed count as code 0 ----
-  int amax[2] = {0, 0};
-  if (demote) {
-    // INT8: 512 16-byte vectors per tile
-    for (int kv = 0; kv < 2; kv++) {
-      const uint4 *src = reinterpret_cast<const uint4 *>(tile + kv * kTileBytes);
-      for (int v = tid; v < kTileBytes / 16; v += kMigThreads) {
-        const uint4 x = src[v];
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-        const int o = 16 * v;
+  // Every packed word maps onto a local piece of the other packing, so each
+  // thread keeps its part of both tiles in registers, as INT8 bytes:
+  //   INT8 K vector v (16 B): token v/8, channels 16(v%8)..+15
+  //        <-> INT4 K words 2v, 2v+1 (8 channels each, same token);
+  //   INT8 V vector v (16 B): channel v/4, the 16 slots of chunk position v%4
+  //        <-> the INT4 V unit (2 words) of those 16 slots.
+  // Thread tid takes INT8 vectors tid and tid + 256 of each tile.
+  uint32_t x[2][2][4];  // [kv][vector][word]
 #pragma unroll
-        for (int e = 0; e < 16; e++) {
-          // -128 is never produced; a corrupt byte is clamped so the table index stays in range
-          int code = max(-127, static_cast<int>(static_cast<int8_t>((w[e >> 2] >> (8 * (e & 3))) & 0xff)));
-          int t, c;
-          if (kv == 0) {
-            t = o / kDim;
-            c = o % kDim + e;
-          } else {
-            c = o / kBlock;
-            const int j = ((o % kBlock) / 16) ^ ((c >> 1) & 3);
-            t = 16 * j + e;
-          }
-          if (t >= sealed) code = 0;
-          cs[kv][t][c] = static_cast<int8_t>(code);
-          amax[kv] = max(amax[kv], abs(code));
+  for (int kv = 0; kv < 2; kv++) {
+#pragma unroll
+    for (int r = 0; r < 2; r++) {
+      const int v = tid + kMigThreads * r;
+      if (demote) {
+        const uint4 q = reinterpret_cast<const uint4 *>(tile + kv * kTileBytes)[v];
+        x[kv][r][0] = q.x; x[kv][r][1] = q.y; x[kv][r][2] = q.z; x[kv][r][3] = q.w;
+      } else {
+        // INT4 source: the two words that hold the same 16 codes
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(tile + kv * kTileBytes);
+        int wi;
+        if (kv == 0) {
+          wi = 2 * v;
+        } else {
+          const int c = v / 4;
+          const int j = (v % 4) ^ ((c >> 1) & 3);  // slots 16j..16j+15
+          wi = c * 8 + 2 * (j ^ ((c >> 2) & 3));
         }
+        const uint2 p = *reinterpret_cast<const uint2 *>(src + wi);
+        // sign-extend the nibbles to bytes: low nibbles are codes 0..3 of a
+        // word, high nibbles codes 4..7
+        x[kv][r][0] = sext_nibbles(p.x & 0x0f0f0f0fu);
+        x[kv][r][1] = sext_nibbles((p.x >> 4) & 0x0f0f0f0fu);
+        x[kv][r][2] = sext_nibbles(p.y & 0x0f0f0f0fu);
+        x[kv][r][3] = sext_nibbles((p.y >> 4) & 0x0f0f0f0fu);
       }
     }
-  } else {
-    // INT4: 1024 32-bit words per tile, 8 codes each
-    for (int kv = 0; kv < 2; kv++) {
-      const uint32_t *src = reinterpret_cast<const uint32_t *>(tile + kv * kTileBytes);
-      for (int w = tid; w < kTileBytes / 8; w += kMigThreads) {
-        const uint32_t x = src[w];
+  }
+  if (sealed < kBlock) {
+    // a partial tail block: slots not yet sealed count as code 0
 #pragma unroll
-        for (int e = 0; e < 8; e++) {
-          int code = nib_get(x, e);
-          int t, c;
-          if (kv == 0) {
-            t = w / 16;
-            c = 8 * (w % 16) + e;
-          } else {
-            c = w / 8;
-            const int wi = w % 8;
-            const int j = (wi >> 1) ^ ((c >> 2) & 3);
-            t = 16 * j + 8 * (wi & 1) + e;
+    for (int kv = 0; kv < 2; kv++)
+#pragma unroll
+      for (int r = 0; r < 2; r++) {
+        const int v = tid + kMigThreads * r;
+#pragma unroll
+        for (int q = 0; q < 4; q++)
+#pragma unroll
+          for (int e = 0; e < 4; e++) {
+            int t;
+            if (kv == 0) {
+              t = v / 8;
+            } else {
+              const int c = v / 4;
+              t = 16 * ((v % 4) ^ ((c >> 1) & 3)) + 4 * q + e;
+            }
+            if (t >= sealed) x[kv][r][q] &= ~(0xffu << (8 * e));
           }
-          if (t >= sealed) code = 0;
-          cs[kv][t][c] = static_cast<int8_t>(code);
-          amax[kv] = max(amax[kv], abs(code));
-        }
       }
-    }
   }
   // ---- largest |code| per tile, new scale, code table ----
 #pragma unroll
   for (int kv = 0; kv < 2; kv++) {
-    int m = amax[kv];
+    uint32_t m = 0;
+#pragma unroll
+    for (int r = 0; r < 2; r++)
+#pragma unroll
+      for (int q = 0; q < 4; q++) m = max(m, absmax4(x[kv][r][q]));
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, d));
-    if (lane == 0) red[kv][warp] = m;
+    if (lane == 0) red[kv][warp] = static_cast<int>(m);
   }
   __syncthreads();
   if (tid < 2) {
     int m = 0;
 #pragma unroll
     for (int w = 0; w < kMigWarps; w++) m = max(m, red[tid][w]);
+    m = min(m, 127);
     const float s_old = a.scales[((size_t)phys * a.hkv + h) * 2 + tid];
     s_new[tid] = __fdiv_rn(__fmul_rn(static_cast<float>(m), s_old), static_cast<float>(qn));
   }
   __syncthreads();
-  for (int e = tid; e < 2 * 255; e += kMigThreads) {
-    const int kv = e / 255, c = e % 255 - 127;
+  for (int e = tid; e < 2 * 256; e += kMigThreads) {
+    const int kv = e >> 8, u = e & 255;
+    const int c = u == 255 ? -127 : u - 127;
     const float s_old = a.scales[((size_t)phys * a.hkv + h) * 2 + kv];
-    tbl[kv][c + 127] = static_cast<int8_t>(s_new[kv] == 0.f ? 0 : requantize(c, s_old, s_new[kv], qn));
+    const int cn = s_new[kv] == 0.f ? 0 : requantize(c, s_old, s_new[kv], qn);
+    // INT4: the nibble; INT8: the byte
+    tbl[kv][u] = static_cast<uint8_t>(demote ? (cn & 0xf) : (cn & 0xff));
   }
-  __syncthreads();  // every thread has read the old scales and tiles
+  __syncthreads();  // every thread has read the old scales and its tile words
 
   // ---- write the tiles in the new packing, then the scales ----
+#pragma unroll
+  for (int kv = 0; kv < 2; kv++) {
+    const uint8_t *tb = tbl[kv];
+#pragma unroll
+    for (int r = 0; r < 2; r++) {
+      const int v = tid + kMigThreads * r;
+      const uint32_t *w = x[kv][r];
+      if (demote) {
+        // codes 0..3 in the low nibbles, 4..7 in the high nibbles of a word
+        const uint32_t o0 = tbl4(tb, w[0]) | (tbl4(tb, w[1]) << 4);
+        const uint32_t o1 = tbl4(tb, w[2]) | (tbl4(tb, w[3]) << 4);
+        uint2 *dst = reinterpret_cast<uint2 *>(tile + kv * kTileBytes);
+        if (kv == 0) {
+          dst[v] = make_uint2(o0, o1);
+        } else {
+          const int c = v / 4;
+          const int j = (v % 4) ^ ((c >> 1) & 3);
+          dst[c * 4 + (j ^ ((c >> 2) & 3))] = make_uint2(o0, o1);
+        }
+      } else {
+        reinterpret_cast<uint4 *>(tile + kv * kTileBytes)[v] =
+            make_uint4(tbl4(tb, w[0]), tbl4(tb, w[1]), tbl4(tb, w[2]), tbl4(tb, w[3]));
+      }
+    }
+  }
   if (demote) {
-    for (int kv = 0; kv < 2; kv++) {
-      uint32_t *dst = reinterpret_cast<uint32_t *>(tile + kv * kTileBytes);
-      for (int w = tid; w < kTileBytes / 8; w += kMigThreads) {
-        uint32_t x = 0;
+    // the unused upper half of each INT4 tile is zeroed
 #pragma unroll
-        for (int e = 0; e < 8; e++) {
-          int t, c;
-          if (kv == 0) {
-            t = w / 16;
-            c = 8 * (w % 16) + e;
-          } else {
-            c = w / 8;
-            const int wi = w % 8;
-            const int j = (wi >> 1) ^ ((c >> 2) & 3);
-            t = 16 * j + 8 * (wi & 1) + e;
-          }
-          x = nib_put(x, e, tbl[kv][cs[kv][t][c] + 127]);
-        }
-        dst[w] = x;
-      }
-      uint4 *hi4 = reinterpret_cast<uint4 *>(tile + kv * kTileBytes + kTileBytes / 2);
-      for (int v = tid; v < kTileBytes / 2 / 16; v += kMigThreads) hi4[v] = make_uint4(0u, 0u, 0u, 0u);
-    }
-  } else {
-    for (int kv = 0; kv < 2; kv++) {
-      uint32_t *dst = reinterpret_cast<uint32_t *>(tile + kv * kTileBytes);
-      for (int w = tid; w < kTileBytes / 4; w += kMigThreads) {
-        const int o = 4 * w;
-        uint32_t x = 0;
-#pragma unroll
-        for (int e = 0; e < 4; e++) {
-          int t, c;
-          if (kv == 0) {
-            t = o / kDim;
-            c = o % kDim + e;
-          } else {
-            c = o / kBlock;
-            const int j = ((o % kBlock) / 16) ^ ((c >> 1) & 3);
-            t = 16 * j + (o % 16) + e;
-          }
-          x |= static_cast<uint32_t>(static_cast<uint8_t>(tbl[kv][cs[kv][t][c] + 127])) << (8 * e);
-        }
-        dst[w] = x;
-      }
-    }
+    for (int kv = 0; kv < 2; kv++)
+      reinterpret_cast<uint4 *>(tile + kv * kTileBytes + kTileBytes / 2)[tid] = make_uint4(0u, 0u, 0u, 0u);
   }
   if (tid < 2) a.scales[((size_t)phys * a.hkv + h) * 2 + tid] = s_new[tid];
 }
