@@ -169,6 +169,31 @@ class ClockSampler:
                 "samples_timed": len(timed), "samples": len(rows)}
 
 
+def room_for_growth(w, extra_tokens):
+    """Give every sequence physical blocks for `extra_tokens` more tokens:
+    spare pool blocks (or new ones past the pool) go into the block table,
+    widened when needed.  For runs that let the cache grow."""
+    import numpy as np
+    from int8_paged_kv_hybrid_b200 import synth
+    need = [synth.cold_blocks_for(int(L) + extra_tokens) for L in w.lens]
+    width = max(w.max_blocks, max(need))
+    bt = np.full((w.batch, width), -1, np.int32)
+    bt[:, :w.max_blocks] = w.block_table
+    used = set(int(x) for x in w.block_table[w.block_table >= 0])
+    spare = [p for p in range(w.num_phys_blocks) if p not in used]
+    nxt = w.num_phys_blocks
+    for b in range(w.batch):
+        for j in range(synth.cold_blocks_for(int(w.lens[b])), need[b]):
+            if bt[b, j] < 0:
+                if spare:
+                    bt[b, j] = spare.pop(0)
+                else:
+                    bt[b, j] = nxt
+                    nxt += 1
+    w.block_table = bt
+    w.num_phys_blocks = nxt
+
+
 def build_gpu_state(w, torch):
     from int8_paged_kv_hybrid_b200 import HybridKVCache, synth
     cache = HybridKVCache(w.batch, w.num_kv_heads, w.num_q_heads, w.num_phys_blocks, w.max_blocks,
@@ -211,6 +236,8 @@ def run_native(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     clocks = ClockSampler(local_rank) if rank == 0 and not args.lean else None
     w = synth.make_workload(args.workload, seed_offset=1000 * rank)
+    if args.lean:
+        room_for_growth(w, args.warmup + args.steps + 2)  # the lean run lets the cache grow
     L = int(w.lens.max())
     cache, n_last, k_last, v_last, q = build_gpu_state(w, torch)
     if args.lean:

@@ -95,6 +95,11 @@ struct SealScratch {
 __device__ __forceinline__ void fused_append(SealScratch &ss, uint8_t *hot_st, uint8_t *tile_st, float2 *scl_tail,
                                              int tile_tail, bool int4_tail, const DecodeArgs &a, int b, int h,
                                              int L_old, bool do_seal, __half2 new_kv, int tid, int warp, int lane) {
+  // A tail block the block table does not give (entry < 0 or past the pool;
+  // HYB_STATUS_BAD_BLOCK is set when the entry is read): the evicted token is
+  // not sealed and nothing is written through the tile, as hyb_kv_append
+  // skips such a block; the new token still goes to the ring.
+  do_seal = do_seal && tile_tail >= 0;
   const int rs = L_old % kHot;  // ring slot of the evicted and of the new token
   const int e = L_old - kHot;   // position sealed (when do_seal)
   const int slot = do_seal ? e % kBlock : 0;

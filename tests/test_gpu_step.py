@@ -103,3 +103,41 @@ def test_mixed_and_invalid_n_new():
     torch.cuda.synchronize()
     assert cache.status(clear=True) == _lib.HYB_STATUS_BAD_N_NEW
     assert list(cache.seq_lens.cpu().numpy()) == [before[0], before[1] + 1, before[2]]
+
+
+def test_step_into_unallocated_block():
+    """The token that leaves the hot ring belongs to a block the table does
+    not give (-1): HYB_STATUS_BAD_BLOCK, nothing written to the cold pool for
+    that sequence (as hyb_kv_append skips such a block), the new token still
+    in the ring and seq_lens advanced; the other sequence is unaffected."""
+    import torch
+    from int8_paged_kv_hybrid_b200 import _lib
+    lens = [96, 200]  # sequence 0: its next sealed token opens block 1, not allocated
+    w = synth.custom_workload("unalloc", lens, 8, 2, seed=13, schedule="chunk")
+    assert w.block_table[0, 1] == -1
+    cache, ora = make_pair(w)
+    replay(w, cache, ora)
+    cold0 = cache.cold.clone()
+    rng = np.random.default_rng(2)
+    n = np.ones(2, np.int32)
+    k = rng.standard_normal((2, 1, 2, 128)).astype(np.float16)
+    v = rng.standard_normal((2, 1, 2, 128)).astype(np.float16)
+    q = rng.standard_normal((2, 8, 128)).astype(np.float16)
+    lse = torch.empty((2, 8), dtype=torch.float32, device="cuda")
+    out = cache.step(torch.from_numpy(n).cuda(), torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda(),
+                     torch.from_numpy(q).cuda(), w.softmax_scale, 201, 0, lse=lse)
+    torch.cuda.synchronize()
+    assert cache.status(clear=True) == _lib.HYB_STATUS_BAD_BLOCK
+    assert cache.seq_lens.tolist() == [97, 201]
+    assert torch.isfinite(out.float()).all()
+    # sequence 0: ring slot 96 % 32 = 0 holds the new token; its blocks are untouched
+    hot = cache.hot.cpu().numpy()
+    assert np.array_equal(hot[0, :, 0, 0], k[0, 0]) and np.array_equal(hot[0, :, 0, 1], v[0, 0])
+    phys0 = [int(p) for p in w.block_table[0] if p >= 0]
+    assert torch.equal(cache.cold[phys0], cold0[phys0])
+    # sequence 1 matches the oracle
+    ora.append(n, k, v)
+    ref, ref_lse = ora.decode(q, w.softmax_scale, pairs=[(1, hh) for hh in range(8)])
+    w.lens = ora.lens()
+    assert_decode_close(w, out.float().cpu().numpy().astype(np.float64), lse.cpu().numpy(), ref, ref_lse,
+                        pairs=[(1, hh) for hh in range(8)], what="sequence 1")
