@@ -60,6 +60,7 @@ def _load():
     lib.ora_decode.argtypes = [P, P, ctypes.c_double, P, i32, P, P, i32]
     lib.ora_combine.argtypes = [i32, i32, i32, P, P, P, P]
     lib.ora_get_block.argtypes = [P, i32, i32, P, P]
+    lib.ora_get_block_fp16.argtypes = [P, i32, i32, P]
     lib.ora_get_ring.argtypes = [P, i32, P]
     lib.ora_export.argtypes = [P, P, i32, P, P, P, P]
     lib.ora_migrate.argtypes = [P, P]
@@ -161,6 +162,12 @@ class OracleCache:
         q = self._lib.ora_get_block(self._h, b, i, _ptr(codes), _ptr(sc))
         return q, codes, sc
 
+    def get_block_fp16(self, b, i):
+        """FP16 cold block (quant_bits 0): (sealed?, float16 [hkv][2][block][d])."""
+        vals = np.zeros((self.hkv, 2, self.block, self.d), np.uint16)
+        ok = self._lib.ora_get_block_fp16(self._h, b, i, _ptr(vals))
+        return bool(ok), vals.view(np.float16)
+
     def ring(self, b):
         r = np.zeros((self.hkv, self.hot, 2, self.d), np.uint16)
         self._lib.ora_get_ring(self._h, b, _ptr(r))
@@ -168,11 +175,13 @@ class OracleCache:
 
     def export(self, block_table, num_phys):
         """Device memory format of the whole cache (see hyb_oracle.c):
-        returns dict(cold uint8 [num_phys][hkv][2][8192], scales float32
+        returns dict(cold uint8 [num_phys][hkv][2][8192] ([4][8192] for FP16
+        blocks), scales float32
         [num_phys][hkv][2], hot float16 [batch][hkv][hot][2][d], seq_lens int32)."""
         bt = _c(block_table, np.int32)
         assert bt.shape == (self.batch, self.max_blocks)
-        cold = np.zeros((num_phys, self.hkv, 2, self.block * self.d), np.uint8)
+        parts = 4 if self.quant_bits == 0 else 2  # FP16 blocks take twice the bytes
+        cold = np.zeros((num_phys, self.hkv, parts, self.block * self.d), np.uint8)
         sc = np.zeros((num_phys, self.hkv, 2), np.float32)
         hot = np.zeros((self.batch, self.hkv, self.hot, 2, self.d), np.uint16)
         sl = np.zeros(self.batch, np.int32)

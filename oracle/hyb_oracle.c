@@ -23,6 +23,8 @@
  *     block gets a new INT8 scale assigned in the kernel; the page is silent on
  *     partial blocks -- this is the plainest reading that keeps the block
  *     layout fixed).
+ *   - quantization_bits 0 (section 5.2: quantization switched off, the cold
+ *     zone kept in FP16): sealed tokens keep their FP16 values in the block.
  *   - Attention (section 4.2, steps 3-5): one softmax over hot and cold keys
  *     together, on the dequantized cold values (code * scale) and the FP16 hot
  *     values, evaluated here in FP64.  The page's torch.cat of two separately
@@ -84,8 +86,9 @@ typedef struct {
   uint16_t *ring;   /* [batch][hkv][hot][2][d] FP16 bits, slot = pos % hot */
   /* per (batch, logical block): NULL until the first token is sealed */
   int8_t **codes;   /* each [hkv][2][block][d], unpacked codes          */
+  uint16_t **half;  /* quant_bits 0: each [hkv][2][block][d] FP16 bits  */
   float **scale;    /* each [hkv][2]                                    */
-  int *qmax;        /* [batch*max_blocks] 127 or 7 once sealed, else 0  */
+  int *qmax;        /* [batch*max_blocks] 127 or 7 once sealed (-1: FP16), else 0 */
 } ora_cache;
 
 void ora_free(ora_cache *c);
@@ -93,7 +96,7 @@ void ora_free(ora_cache *c);
 ora_cache *ora_new(int batch, int hkv, int hq, int d, int hot, int block,
                    int max_blocks, int quant_bits) {
   if (batch <= 0 || hkv <= 0 || hq <= 0 || hq % hkv || d <= 0 || hot <= 0 ||
-      block <= 0 || max_blocks < 0 || (quant_bits != 8 && quant_bits != 4))
+      block <= 0 || max_blocks < 0 || (quant_bits != 8 && quant_bits != 4 && quant_bits != 0))
     return NULL;
   build_half_table();
   ora_cache *c = (ora_cache *)calloc(1, sizeof(ora_cache));
@@ -107,7 +110,8 @@ ora_cache *ora_new(int batch, int hkv, int hq, int d, int hot, int block,
   c->codes = (int8_t **)calloc(nb, sizeof(int8_t *));
   c->scale = (float **)calloc(nb, sizeof(float *));
   c->qmax = (int *)calloc(nb, sizeof(int));
-  if (!c->len || !c->n_int4 || !c->ring || !c->codes || !c->scale || !c->qmax) {
+  c->half = (uint16_t **)calloc(nb, sizeof(uint16_t *));
+  if (!c->len || !c->n_int4 || !c->ring || !c->codes || !c->scale || !c->qmax || !c->half) {
     ora_free(c);
     return NULL;
   }
@@ -121,7 +125,9 @@ void ora_free(ora_cache *c) {
     for (size_t i = 0; i < nb; i++) free(c->codes[i]);
   if (c->scale)
     for (size_t i = 0; i < nb; i++) free(c->scale[i]);
-  free(c->codes); free(c->scale); free(c->qmax);
+  if (c->half)
+    for (size_t i = 0; i < nb; i++) free(c->half[i]);
+  free(c->codes); free(c->scale); free(c->qmax); free(c->half);
   free(c->len); free(c->n_int4); free(c->ring);
   free(c);
 }
@@ -176,6 +182,21 @@ int ora_append(ora_cache *c, const int32_t *n_new, int max_new,
       const int p1 = (i + 1) * blk < e1 ? (i + 1) * blk : e1;
       const size_t bi = (size_t)b * c->max_blocks + i;
       const int first_slot = p0 - i * blk;
+      if (c->quant_bits == 0) {
+        /* FP16 cold block: the tokens keep their FP16 values */
+        if (!c->half[bi]) {
+          c->half[bi] = (uint16_t *)calloc((size_t)hkv * 2 * blk * d, sizeof(uint16_t));
+          if (!c->half[bi]) return ORA_ERR_NOMEM;
+          c->qmax[bi] = -1;
+        }
+        for (int h = 0; h < hkv; h++)
+          for (int kv = 0; kv < 2; kv++)
+            for (int p = p0; p < p1; p++)
+              for (int ch = 0; ch < d; ch++)
+                c->half[bi][(((size_t)h * 2 + kv) * blk + (p - i * blk)) * d + ch] = SRC(p, h, kv, ch);
+        p0 = p1;
+        continue;
+      }
       const int q = (c->quant_bits == 4 || i < c->n_int4[b]) ? 7 : 127;
       if (!c->codes[bi]) {
         c->codes[bi] = (int8_t *)calloc((size_t)hkv * 2 * blk * d, 1);
@@ -331,6 +352,8 @@ static double kv_value(const ora_cache *c, int b, int h, int kv, int p, int ch) 
         c->ring[((((size_t)b * c->hkv + h) * c->hot + p % c->hot) * 2 + kv) * c->d + ch]);
   const int i = p / c->block;
   const size_t bi = (size_t)b * c->max_blocks + i;
+  if (c->quant_bits == 0)
+    return (double)half_to_float(c->half[bi][(((size_t)h * 2 + kv) * c->block + (p - i * c->block)) * c->d + ch]);
   const int8_t code = c->codes[bi][(((size_t)h * 2 + kv) * c->block + (p - i * c->block)) * c->d + ch];
   return (double)code * (double)c->scale[bi][h * 2 + kv];
 }
@@ -428,9 +451,20 @@ int ora_combine(int rows, int n_splits, int d, const double *o_part,
 int ora_get_block(const ora_cache *c, int b, int i, int8_t *codes, float *scales) {
   const size_t bi = (size_t)b * c->max_blocks + i;
   if (b < 0 || b >= c->batch || i < 0 || i >= c->max_blocks || !c->codes[bi]) return 0;
+  if (c->quant_bits == 0) return 0;
   memcpy(codes, c->codes[bi], (size_t)c->hkv * 2 * c->block * c->d);
   memcpy(scales, c->scale[bi], (size_t)c->hkv * 2 * sizeof(float));
   return c->qmax[bi];
+}
+
+/* FP16 cold block i of sequence b (quant_bits 0): FP16 bits [hkv][2][block][d]
+ * (slots not yet sealed are 0).  Returns 1, or 0 if the block holds no sealed
+ * token. */
+int ora_get_block_fp16(const ora_cache *c, int b, int i, uint16_t *vals) {
+  const size_t bi = (size_t)b * c->max_blocks + i;
+  if (c->quant_bits != 0 || b < 0 || b >= c->batch || i < 0 || i >= c->max_blocks || !c->half[bi]) return 0;
+  memcpy(vals, c->half[bi], (size_t)c->hkv * 2 * c->block * c->d * sizeof(uint16_t));
+  return 1;
 }
 
 /* Hot ring of sequence b: FP16 bits [hkv][hot][2][d]. */
@@ -459,7 +493,10 @@ int ora_get_ring(const ora_cache *c, int b, uint16_t *ring) {
 /*     8-byte units of 16 tokens, unit u stored at u XOR ((ch/4) % 4); */
 /*     within a unit, tokens 0..7 in its first word, 8..15 in the      */
 /*     second.                                                         */
-/*   scales: float [num_phys][hkv][2].                                 */
+/*   FP16 cold blocks (quant_bits 0): cold pool bytes                  */
+/*   [num_phys][hkv][block][2][d] FP16, per token the K row then the V  */
+/*   row (the hot ring's layout), 32 KB per block and kv head.          */
+/*   scales: float [num_phys][hkv][2] (not used by FP16 blocks).        */
 /*   hot ring: FP16 [batch][hkv][hot][2][d] (K row, then V row).       */
 /* Only sealed slots are written; other bytes are left as they are.    */
 /* ------------------------------------------------------------------ */
@@ -475,6 +512,29 @@ int ora_export(const ora_cache *c, const int32_t *block_table, int num_phys,
   const int d = c->d, blk = c->block, hkv = c->hkv;
   const size_t tile = (size_t)blk * d;
   if (d != 128 || blk != 64) return ORA_ERR_INVALID; /* format defined for 64 x 128 */
+  if (c->quant_bits == 0) {
+    uint16_t *cold16 = (uint16_t *)cold;
+    for (int b = 0; b < c->batch; b++) {
+      const int L = c->len[b];
+      const int cold_len = L > c->hot ? L - c->hot : 0;
+      const int nblk = (cold_len + blk - 1) / blk;
+      for (int i = 0; i < nblk; i++) {
+        const size_t bi = (size_t)b * c->max_blocks + i;
+        const int phys = block_table[(size_t)b * c->max_blocks + i];
+        if (phys < 0 || phys >= num_phys) return ORA_ERR_INVALID;
+        const int sealed = cold_len - i * blk < blk ? cold_len - i * blk : blk;
+        for (int h = 0; h < hkv; h++)
+          for (int t = 0; t < sealed; t++)
+            for (int kv = 0; kv < 2; kv++)
+              for (int ch = 0; ch < d; ch++)
+                cold16[((((size_t)phys * hkv + h) * blk + t) * 2 + kv) * d + ch] =
+                    c->half[bi][(((size_t)h * 2 + kv) * blk + t) * d + ch];
+      }
+      seq_lens[b] = L;
+    }
+    memcpy(hot, c->ring, (size_t)c->batch * hkv * c->hot * 2 * d * sizeof(uint16_t));
+    return ORA_OK;
+  }
   for (int b = 0; b < c->batch; b++) {
     const int L = c->len[b];
     const int cold_len = L > c->hot ? L - c->hot : 0;
