@@ -50,25 +50,34 @@ def parse():
     p.add_argument("--migrate", action="store_true",
                    help="time hyb_kv_migrate instead of the decode step: demote a quarter of every "
                         "sequence's cold blocks to INT4 and promote them back (workload default 3)")
+    p.add_argument("--quant-bits", type=int, default=8, choices=[8, 4, 0],
+                   help="cold blocks: 8 (INT8, the default), 4 (all INT4) or 0 (FP16, quantization off)")
     p.add_argument("--lean", action="store_true",
                    help="profiling run: no state restore, L2 flush, e2e or CPU baseline")
     return p.parse_args()
 
 
-def workload_config(w, split, ns):
+COLD_KIND = {8: "INT8", 4: "INT4", 0: "FP16"}
+
+
+def workload_config(w, split, ns, qbits=8):
     lens = w.lens
+    cold = COLD_KIND[qbits]
+    if qbits == 8 and w.n_int4 is not None:
+        cold = "INT8 (oldest quarter INT4)"
     if w.name == "config2":
         what = ("llama3-8b decode attention, 1 layer: batch %d, Hq %d, Hkv %d, d 128, L %d (32 FP16 hot + "
-                "%d INT8 cold in 64-token blocks), %d-block pool"
-                % (w.batch, w.num_q_heads, w.num_kv_heads, int(lens[0]), int(lens[0]) - 32, w.num_phys_blocks))
+                "%d %s cold in 64-token blocks), %d-block pool"
+                % (w.batch, w.num_q_heads, w.num_kv_heads, int(lens[0]), int(lens[0]) - 32, cold,
+                   w.num_phys_blocks))
     else:
         what = ("decode attention, 1 layer: batch %d, Hq %d, Hkv %d, d 128, L %d..%d (mean %.0f), 32 FP16 hot "
                 "+ %s cold in 64-token blocks, %d-block pool"
                 % (w.batch, w.num_q_heads, w.num_kv_heads, int(lens.min()), int(lens.max()), float(lens.mean()),
-                   "INT8 (oldest quarter INT4)" if w.n_int4 is not None else "INT8", w.num_phys_blocks))
+                   cold, w.num_phys_blocks))
     return {"workload": what, "batch": int(w.batch), "seq_len": int(lens.max()),
             "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads, "head_dim": 128, "hot_tokens": 32,
-            "block_size": 64, "quant_bits": 8, "split_tokens": split, "n_splits": ns,
+            "block_size": 64, "quant_bits": qbits, "split_tokens": split, "n_splits": ns,
             "step": "hyb_decode_step: append 1 token/seq + split-KV attention, one launch",
             "l2": "flushed between timed steps (512 MB write)",
             "parallelism": "replicas (independent batch per GPU)"}
@@ -194,10 +203,11 @@ def room_for_growth(w, extra_tokens):
     w.num_phys_blocks = nxt
 
 
-def build_gpu_state(w, torch):
+def build_gpu_state(w, torch, qbits=8):
     from int8_paged_kv_hybrid_b200 import HybridKVCache, synth
     cache = HybridKVCache(w.batch, w.num_kv_heads, w.num_q_heads, w.num_phys_blocks, w.max_blocks,
-                          block_table=w.block_table, n_int4=w.n_int4)
+                          quant_bits=qbits, block_table=w.block_table,
+                          n_int4=w.n_int4 if qbits == 8 else None)
     # prefill to L-1 in 64-token appends; the benchmarked step appends the last token
     sched = synth._chunk_schedule(w.lens, 64)
     for si, n in enumerate(sched[:-1]):
@@ -239,7 +249,8 @@ def run_native(args, rank, world, local_rank):
     if args.lean:
         room_for_growth(w, args.warmup + args.steps + 2)  # the lean run lets the cache grow
     L = int(w.lens.max())
-    cache, n_last, k_last, v_last, q = build_gpu_state(w, torch)
+    qb = args.quant_bits
+    cache, n_last, k_last, v_last, q = build_gpu_state(w, torch, qb)
     if args.lean:
         L += args.warmup + args.steps  # the lean run lets the cache grow one token per step
     split, ns = cache.plan(L, args.split or w.split_tokens)
@@ -359,8 +370,8 @@ def run_native(args, rank, world, local_rank):
         ms_e2e = t.item()
     del g_step
 
-    kvb = synth.kv_bytes(w)
-    stepb = kvb + synth.append_bytes(w, n_last)
+    kvb = synth.kv_bytes(w, quant_bits=qb)
+    stepb = kvb + synth.append_bytes(w, n_last, qb)
     peak, peak_kind = measured_peaks()
     total_bytes = kvb * world
     value = total_bytes / (ms_step * 1e-3) / 1e9
@@ -371,17 +382,21 @@ def run_native(args, rank, world, local_rank):
         res = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": {8: "int8", 4: "int4", 0: "f16"}[qb],
             "data": "synthetic (seeded N(0,1) FP16 K/V/q; caches built by the library's own appends)",
-            "config": workload_config(w, split, ns),
+            "config": workload_config(w, split, ns, qb),
             "tokens_per_s": round(tokens_s, 1),
             "tokens_per_s_model_equiv": round(tokens_s / 32, 1),
             "kv_bytes_per_step": kvb,
             "frac_of_hbm_peak_step": round(value / world / peak, 4),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": profiled_traffic(),
-                         "kernel": "hyb::decode_kernel<4,true> (fused append + attention, the step's "
-                                   "only launch)", "peak_kind": peak_kind,
+                         "frac": round(achieved / peak, 4),
+                         # the committed ncu figure covers the default workload and cold format only
+                         "traffic": profiled_traffic() if (args.workload == WORKLOAD and qb == 8
+                                                           and not args.split) else None,
+                         "kernel": "hyb::decode_kernel (fused append + attention, the step's only launch)",
+                         "peak_kind": peak_kind,
                          "achieved_bytes": "algorithmic bytes per launch: attention %d + append %d"
                                            % (kvb, stepb - kvb)},
             "e2e": {"value": round(total_bytes / (ms_e2e * 1e-3) / 1e9, 1), "unit": UNIT,
@@ -457,7 +472,7 @@ def run_migrate(args):
     }
 
 
-def oracle_step_rate(w, steps, warmup, budget_s=None):
+def oracle_step_rate(w, steps, warmup, budget_s=None, qbits=8):
     """Time the CPU oracle (as it stands) on the same workload: per step the
     1-token append plus FP64 attention of every (sequence, head).  The state
     grows by one token per step (bounded sample)."""
@@ -465,7 +480,9 @@ def oracle_step_rate(w, steps, warmup, budget_s=None):
     import oracle
     from int8_paged_kv_hybrid_b200 import synth
     threads = os.cpu_count() or 1
-    ora = oracle.OracleCache(w.batch, w.num_kv_heads, w.num_q_heads, w.max_blocks + 16)
+    ora = oracle.OracleCache(w.batch, w.num_kv_heads, w.num_q_heads, w.max_blocks + 16, qbits)
+    if qbits == 8 and w.n_int4 is not None:
+        ora.set_n_int4(w.n_int4)
     sched = synth._chunk_schedule(w.lens, 64)
     for si, n in enumerate(sched[:-1]):
         k, v = synth.step_tokens(w, si, n, max_new=64)
@@ -502,14 +519,14 @@ def main():
         if rank != 0:
             return 0
         w = synth.make_workload(args.workload)
-        sec, n, threads = oracle_step_rate(w, args.steps, args.warmup, budget_s=150.0)
-        kvb = synth.kv_bytes(w)
+        sec, n, threads = oracle_step_rate(w, args.steps, args.warmup, budget_s=150.0, qbits=args.quant_bits)
+        kvb = synth.kv_bytes(w, quant_bits=args.quant_bits)
         val = kvb / sec / 1e9
         print(json.dumps({
             "impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": UNIT, "n_gpus": world,
             "steps": n, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(w, 0, 0),
+            "data": "synthetic", "config": workload_config(w, 0, 0, args.quant_bits),
             "tokens_per_s": round(w.batch / sec, 3),
             "cpu_baseline": {"value": round(val, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": "%d full steps of the workload (append 1 token/seq + FP64 attention "
@@ -531,8 +548,9 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     res, w = run_native(args, rank, world, local_rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.lean:
-        sec, n, threads = oracle_step_rate(w, 3, 0, budget_s=30.0)
-        res["cpu_baseline"] = {"value": round(synth.kv_bytes(w) / sec / 1e9, 4), "unit": UNIT,
+        sec, n, threads = oracle_step_rate(w, 3, 0, budget_s=30.0, qbits=args.quant_bits)
+        res["cpu_baseline"] = {"value": round(synth.kv_bytes(w, quant_bits=args.quant_bits) / sec / 1e9, 4),
+                               "unit": UNIT,
                                "cores": threads, "kind": "oracle",
                                "sample": "%d full steps of the same workload (1-token append + FP64 "
                                          "attention of all rows) on the host, OpenMP over rows" % n}

@@ -9,9 +9,11 @@
  *     INT8 with a block-wise scale, INT4 for the "L2" cold blocks (sections
  *     2.1, 2.2, 3.1), reached through a block table (section 3.2, block header).
  * The three fields of the hybrid_v2 contract are hot_tokens (power of two),
- * quantization_bits (4 or 8) and block_size (a multiple of 8); the example
- * set 32 / 8 / 64 is the only one this library implements (section 3.1;
- * section 5.1 for the invalid-value error).
+ * quantization_bits (4 or 8) and block_size (a multiple of 8); this library
+ * implements hot_tokens 32 and block_size 64 with quantization_bits 8 or 4
+ * (section 3.1; section 5.1 for the invalid-value error), and
+ * quantization_bits 0, which the page's section 5.2 gives as the switch that
+ * keeps the cold zone in FP16.
  *
  * Calls:
  *   hyb_kv_append      seal tokens leaving the hot zone into cold blocks
@@ -86,7 +88,9 @@ typedef struct CUstream_st *hyb_stream_t; /* same type as cudaStream_t */
  * Geometry: hot_tokens HOT = 32, block_size BLK = 64, head_dim D = 128,
  * num_kv_heads Hkv >= 1, num_q_heads Hq a multiple of Hkv with Hq/Hkv <= 8
  * (query head h reads kv head h / (Hq/Hkv)), quant_bits 8 (INT8 cold blocks;
- * logical blocks below n_int4_blocks[b] are INT4) or 4 (every cold block INT4).
+ * logical blocks below n_int4_blocks[b] are INT4), 4 (every cold block INT4)
+ * or 0 (FP16 cold blocks, nothing quantized; n_int4_blocks and scales are not
+ * read).
  *
  * Token positions 0..L-1 of sequence b (L = seq_lens[b]): positions >= L-32
  * are hot, the others cold; cold position p lives in logical block p/64,
@@ -117,6 +121,10 @@ typedef struct CUstream_st *hyb_stream_t; /* same type as cudaStream_t */
  *          never produced.  Bytes of slots not yet sealed are never written.
  *   scales FP32 [num_phys_blocks][Hkv][2]: K scale, V scale of each tile;
  *          the value of a cold element is code * scale.
+ *   cold, quant_bits 0: FP16 [num_phys_blocks][Hkv][BLK][2][D]: per physical
+ *          block and kv head 64 token slots in the hot ring's row layout (K
+ *          row then V row, 512 B per token), 32 KB per (block, kv head);
+ *          slot t at byte t*512.  Base 16-byte aligned.
  *   block_table int32 [batch][max_blocks_per_seq]; entries for blocks a
  *          sequence does not reach are ignored.  A block that appends write
  *          into must belong to one sequence only.
@@ -133,7 +141,7 @@ typedef struct hyb_cache_desc {
   int32_t hot_tokens;         /* must be 32 */
   int32_t block_size;         /* must be 64 */
   int32_t head_dim;           /* must be 128 */
-  int32_t quant_bits;         /* 8 or 4 */
+  int32_t quant_bits;         /* 8, 4 or 0 (FP16 cold blocks) */
   int32_t num_kv_heads;       /* Hkv >= 1 */
   int32_t num_q_heads;        /* Hq, multiple of Hkv, Hq/Hkv <= 8 */
   int32_t num_phys_blocks;    /* physical blocks in `cold` / `scales` */
@@ -152,7 +160,7 @@ typedef struct hyb_cache_desc {
 /*
  * Host-only check of a descriptor (no GPU needed, nothing enqueued).
  * Returns HYB_OK, HYB_ERR_INVALID_VALUE (hot_tokens not a power of two in
- * {16, 32, 64, 128}, block_size not a multiple of 8, quant_bits not 4 or 8,
+ * {16, 32, 64, 128}, block_size not a multiple of 8, quant_bits not 8, 4 or 0,
  * non-positive sizes, Hq not a multiple of Hkv, null or misaligned pointers)
  * or HYB_ERR_UNSUPPORTED (a valid configuration other than 32 / 64 / D=128,
  * or Hq/Hkv > 8).  The contract is the page's section 3.1 and 5.1.
@@ -342,7 +350,8 @@ int hyb_combine(int32_t batch, int32_t num_q_heads, int32_t head_dim, int32_t n_
  *                  over the batch (it sizes the grid), 0..max_blocks_per_seq.
  * Returns HYB_OK, HYB_ERR_INVALID_VALUE (bad descriptor, NULL n_int4_blocks,
  * NULL or misaligned target, max_delta out of range), HYB_ERR_UNSUPPORTED
- * (quant_bits 4: every block is INT4 already) or HYB_ERR_CUDA.  Device
+ * (quant_bits 4: every block is INT4 already; quant_bits 0: FP16 blocks have
+ * no tiers) or HYB_ERR_CUDA.  Device
  * errors: HYB_STATUS_BAD_TIER (that sequence left unchanged) and
  * HYB_STATUS_BAD_BLOCK (that block skipped).  Asynchronous on `stream`; it
  * must not overlap on the GPU with any other call on the same cache.

@@ -24,7 +24,9 @@ class HybridKVCache:
         dev = torch.device(device)
         self.device = dev
         self.hot = torch.zeros((self.batch, self.hkv, HOT, 2, HEAD_DIM), dtype=torch.float16, device=dev)
-        self.cold = torch.zeros((self.num_phys, self.hkv, 2, TILE_BYTES), dtype=torch.uint8, device=dev)
+        # quant_bits 0: FP16 blocks, 64 rows of K then V (twice the bytes)
+        parts = 4 if self.quant_bits == 0 else 2
+        self.cold = torch.zeros((self.num_phys, self.hkv, parts, TILE_BYTES), dtype=torch.uint8, device=dev)
         self.scales = torch.zeros((self.num_phys, self.hkv, 2), dtype=torch.float32, device=dev)
         if block_table is None:
             self.block_table = torch.full((self.batch, self.max_blocks), -1, dtype=torch.int32, device=dev)

@@ -4,7 +4,9 @@
 // Method: web page "DeepSeek V4混合式KV Cache推理优化实战解析", section 4.2
 // (quantize_int8 of the cold part), sections 2.1 / 3.1 (INT8, INT4 for L2
 // blocks, block size 64, hot zone = most recent 32 tokens in FP16) and 3.2
-// (per-block scale held in the block header, re-assigned inside the kernel).
+// (per-block scale held in the block header, re-assigned inside the kernel);
+// section 5.2 (quantization_bits 0: the cold zone stays FP16 -- sealed rows
+// are copied unchanged).
 //
 // One CTA per sequence; warp w handles (kv head, K|V) pairs w, w+nwarps, ...
 // A warp owns everything it writes (its tiles' bytes, its scale words and its
@@ -93,6 +95,21 @@ __global__ void __launch_bounds__(512) append_kernel(AppendArgs a) {
       const int phys = a.block_table[(size_t)b * a.max_blocks + i];
       if (phys < 0 || phys >= a.num_phys) {
         if (lane == 0) set_status(a.status, HYB_STATUS_BAD_BLOCK);
+        p0 = p1;
+        continue;
+      }
+      if (a.quant_bits == 0) {
+        // FP16 cold block: the rows move unchanged (K row then V row per slot)
+        __half *blk = reinterpret_cast<__half *>(a.cold + ((size_t)phys * a.hkv + h) * kFp16BlockBytes);
+        for (int t = p0; t < p1; t++) {
+          const __half *src;
+          if (t < L_old)
+            src = a.hot + ((((size_t)b * a.hkv + h) * kHot + (t % kHot)) * 2 + kv) * kDim;
+          else
+            src = (kv ? a.v_new : a.k_new) + (((size_t)b * a.max_new + (t - L_old)) * a.hkv + h) * kDim;
+          __half *dst = blk + ((t - i * kBlock) * 2 + kv) * kDim;
+          *reinterpret_cast<uint2 *>(dst + 4 * lane) = *reinterpret_cast<const uint2 *>(src + 4 * lane);
+        }
         p0 = p1;
         continue;
       }

@@ -15,6 +15,9 @@ constexpr int kTileBytes = kBlock * kDim;        // one K or V tile, INT8
 constexpr int kTilePairBytes = 2 * kTileBytes;   // K tile + V tile of one (block, kv head)
 constexpr int kHotTokenBytes = 2 * kDim * 2;     // K row + V row, FP16
 constexpr int kHotBytes = kHot * kHotTokenBytes; // 16 KB per (sequence, kv head)
+// quantization_bits 0: an FP16 cold block keeps the hot ring's row layout
+// (K row then V row per token), 32 KB per (block, kv head)
+constexpr int kFp16BlockBytes = kBlock * kHotTokenBytes;
 
 // First error wins; later errors leave the word unchanged.
 __device__ __forceinline__ void set_status(int32_t *status, int code) {

@@ -68,8 +68,9 @@ struct DecodeSmem {
 
 // kCluster: the grid is launched in clusters of n_splits CTAs (the splits of
 // one (sequence, kv head)); splits are merged through distributed shared
-// memory instead of the workspace.
-template <int G, bool kCluster>
+// memory instead of the workspace.  kF16: FP16 cold blocks (quantization_bits
+// 0), each attended as two items of 32 rows with the hot ring's arithmetic.
+template <int G, bool kCluster, bool kF16>
 __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(const DecodeArgs a) {
   constexpr int P = pow2_heads<G>();
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -120,13 +121,18 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
   if (!kCluster && s >= Sb) return;
   const int ncold = max(0, min(nblk, i0 + a.split_blocks) - i0);
   const int nhot = (s == Sb - 1) ? min(L, kHot) : 0;
-  const int nitems = ncold + (nhot > 0 ? 1 : 0);
+  // FP16 cold blocks (quantization_bits 0) are two items of 32 rows each
+  constexpr bool fp16 = kF16;
+  const int ncold_it = fp16 ? 2 * ncold : ncold;
+  const int kh = ncold_it;  // the hot item
+  const int nitems = ncold_it + (nhot > 0 ? 1 : 0);
   // fused step, in the split that holds the tail block and the hot ring: the
   // new token goes to ring slot L_old % 32 (whose old occupant, position
   // L_old - 32, is sealed into the tail block first)
   const bool do_ring = n_app == 1 && nhot > 0;
   const bool do_seal = do_ring && L_old >= kHot;
-  const int k_fused = do_seal ? ncold - 1 : ncold;  // item at which the append is done
+  // item at which the append is done: the one that receives the sealed token
+  const int k_fused = !do_seal ? kh : fp16 ? 2 * (ncold - 1) + ((L_old - kHot) % kBlock) / kHot : ncold - 1;
   __half2 new_kv = __halves2half2(__float2half_rn(0.f), __float2half_rn(0.f));
   if (do_ring) {
     const size_t o = ((size_t)b * a.hkv + h) * kDim + tid;
@@ -159,10 +165,20 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
   auto issue = [&](int k) {
     const int st = k % kStages;
     uint8_t *dst = sm.ring[st];
-    if (k < ncold) {
-      const int phys = sm.phys[k];
-      if (phys < 0) {
+    if (k < ncold_it) {
+      const int kb = fp16 ? k >> 1 : k;
+      const int phys = sm.phys[kb];
+      const int nrow = fp16 ? min(kHot, Lc - (i0 + kb) * kBlock - (k & 1) * kHot) : 1;
+      if (phys < 0 || nrow <= 0) {
         mbar_arrive(&sm.full[st]);
+        return;
+      }
+      if (fp16) {
+        // the half block's sealed rows
+        const uint8_t *src = a.cold + ((size_t)phys * a.hkv + h) * kFp16BlockBytes + (k & 1) * kHotBytes;
+        const uint32_t bytes = static_cast<uint32_t>(nrow) * kHotTokenBytes;
+        mbar_arrive_expect_tx(&sm.full[st], bytes);
+        bulk_g2s(dst, src, bytes, &sm.full[st], pol);
         return;
       }
       const uint8_t *src = a.cold + ((size_t)phys * a.hkv + h) * kTilePairBytes;
@@ -184,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
   // block scales: requested before the bulk copies so that they do not queue
   // behind them; stored once they arrive (overlapping the copies)
   float2 sc_ld = make_float2(0.f, 0.f);
-  if (tid < ncold && sm.phys[tid] >= 0)
+  if (!fp16 && tid < ncold && sm.phys[tid] >= 0)
     sc_ld = __ldg(reinterpret_cast<const float2 *>(a.scales + ((size_t)sm.phys[tid] * a.hkv + h) * 2));
   int issued = 0;
   if (tid == 0) {
@@ -232,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
     if (tid == 0) {
       for (; next_issue < min(nitems, k + kStages); next_issue++) {
         const int j = next_issue - kStages;  // previous item of that stage
-        if (next_issue <= k + ((do_ring && k == k_fused) ? 1 : 0)) {
+        if (next_issue <= ((do_ring && k == k_fused) ? kh : k)) {
           if (!mbar_wait_bounded(&sm.empty[j % kStages], (j / kStages) & 1, kWaitCycles)) {
             set_status(a.status, HYB_STATUS_TIMEOUT);
             sm.abort_flag = 1;
@@ -249,10 +265,13 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
     if (!ok && lane == 0) set_status(a.status, HYB_STATUS_TIMEOUT);
     if (do_ring && k == k_fused) {
       // ---------------- fused append (whole CTA, in the staged copies) ----------------
-      const int kh = ncold;  // the hot item
       if (k != kh) ok = ok && mbar_wait_bounded(&sm.full[kh % kStages], (kh / kStages) & 1, kWaitCycles);
       ok = __syncthreads_and(ok) != 0;
-      if (ok) {
+      if (ok && fp16) {
+        const int tb = do_seal ? ncold - 1 : 0;  // the tail block
+        fused_append_fp16(sm.ring[kh % kStages], sm.ring[k_fused % kStages], sm.phys[tb] * a.hkv + h, a, b, h,
+                          L_old, do_seal, new_kv, tid);
+      } else if (ok) {
         const int ti = do_seal ? ncold - 1 : 0;  // the tail block's item
         fused_append(sm.seal, sm.ring[ncold % kStages], sm.ring[ti % kStages], &sm.scl[ti],
                      sm.phys[ti] * a.hkv + h, (i0 + ti) < n_int4_b, a, b, h, L_old, do_seal, new_kv, tid, warp,
@@ -261,7 +280,11 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
     }
     ok = ok && *reinterpret_cast<volatile int *>(&sm.abort_flag) == 0;
     const uint8_t *stage = sm.ring[st];
-    if (ok && k < ncold) {
+    // rows of an FP16 item: the hot ring, or half of an FP16 cold block
+    int nrow = nhot;
+    if (k < ncold_it)
+      nrow = !fp16 || sm.phys[k >> 1] < 0 ? 0 : min(kHot, Lc - (i0 + (k >> 1)) * kBlock - (k & 1) * kHot);
+    if (ok && !fp16 && k < ncold) {
       // ---------------- cold block ----------------
       const int i = i0 + k;
       const int nvalid = sm.phys[k] < 0 ? 0 : min(kBlock, Lc - i * kBlock);
@@ -276,9 +299,9 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
         cold_block_general<G, P>(stage, nv, int4, warp, lane, tg, cs, qp, coef, sc.y * (1.f / 32767.f),
                                  sm.pcode[warp], hx, owner, m_run, acc, m_hx, l_lane, psum_lane);
       }
-    } else if (ok) {
-      // ---------------- hot ring (FP16, FP32 math) ----------------
-      hot_item<G, P>(stage, nhot, warp, lane, tg, cs, sm.qf, a.qk_scale, sm.phot[warp], hx, owner, m_run, acc, m_hx,
+    } else if (ok && nrow > 0) {
+      // ---------------- FP16 rows (FP32 math): hot ring or FP16 cold half block ----------------
+      hot_item<G, P>(stage, nrow, warp, lane, tg, cs, sm.qf, a.qk_scale, sm.phot[warp], hx, owner, m_run, acc, m_hx,
                      l_lane, psum_lane);
     }
     __syncwarp();
@@ -412,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
 // Largest cluster the decode kernel is launched with (portable size).
 constexpr int kMaxCluster = 8;
 
-template <int G>
+template <int G, bool kF16>
 static cudaError_t launch_decode_g(const DecodeArgs &a, int batch, bool cluster, cudaStream_t stream) {
   const size_t smem = sizeof(DecodeSmem<G>);
   static int configured_dev_mask = 0;  // one bit per device
@@ -420,10 +443,10 @@ static cudaError_t launch_decode_g(const DecodeArgs &a, int batch, bool cluster,
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 31 && !(configured_dev_mask & (1 << dev))) {
-    e = cudaFuncSetAttribute(decode_kernel<G, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(decode_kernel<G, false, kF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(decode_kernel<G, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = cudaFuncSetAttribute(decode_kernel<G, true, kF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     configured_dev_mask |= 1 << dev;
@@ -442,26 +465,32 @@ static cudaError_t launch_decode_g(const DecodeArgs &a, int batch, bool cluster,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_kernel<G, true>, a);
+    e = cudaLaunchKernelEx(&cfg, decode_kernel<G, true, kF16>, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
-  decode_kernel<G, false><<<grid, kThreads, smem, stream>>>(a);
+  decode_kernel<G, false, kF16><<<grid, kThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream) {
+template <bool kF16>
+static cudaError_t launch_decode_f(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream) {
   switch (group) {
-    case 1: return launch_decode_g<1>(a, batch, cluster, stream);
-    case 2: return launch_decode_g<2>(a, batch, cluster, stream);
-    case 3: return launch_decode_g<3>(a, batch, cluster, stream);
-    case 4: return launch_decode_g<4>(a, batch, cluster, stream);
-    case 5: return launch_decode_g<5>(a, batch, cluster, stream);
-    case 6: return launch_decode_g<6>(a, batch, cluster, stream);
-    case 7: return launch_decode_g<7>(a, batch, cluster, stream);
-    case 8: return launch_decode_g<8>(a, batch, cluster, stream);
+    case 1: return launch_decode_g<1, kF16>(a, batch, cluster, stream);
+    case 2: return launch_decode_g<2, kF16>(a, batch, cluster, stream);
+    case 3: return launch_decode_g<3, kF16>(a, batch, cluster, stream);
+    case 4: return launch_decode_g<4, kF16>(a, batch, cluster, stream);
+    case 5: return launch_decode_g<5, kF16>(a, batch, cluster, stream);
+    case 6: return launch_decode_g<6, kF16>(a, batch, cluster, stream);
+    case 7: return launch_decode_g<7, kF16>(a, batch, cluster, stream);
+    case 8: return launch_decode_g<8, kF16>(a, batch, cluster, stream);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream) {
+  return a.quant_bits == 0 ? launch_decode_f<true>(a, group, batch, cluster, stream)
+                           : launch_decode_f<false>(a, group, batch, cluster, stream);
 }
 
 int decode_max_cluster() { return kMaxCluster; }
@@ -484,10 +513,10 @@ int decode_ctas_per_sm(int group) {
   switch (group) {
 #define HYB_OCC(g)                                                                          \
   case g:                                                                                   \
-    e = cudaFuncSetAttribute(decode_kernel<g, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+    e = cudaFuncSetAttribute(decode_kernel<g, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              static_cast<int>(sizeof(DecodeSmem<g>)));                      \
     if (e == cudaSuccess)                                                                   \
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<g, false>, kThreads, \
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<g, false, false>, kThreads, \
                                                         sizeof(DecodeSmem<g>));             \
     break;
     HYB_OCC(1) HYB_OCC(2) HYB_OCC(3) HYB_OCC(4) HYB_OCC(5) HYB_OCC(6) HYB_OCC(7) HYB_OCC(8)

@@ -204,6 +204,38 @@ __device__ __forceinline__ void fused_append(SealScratch &ss, uint8_t *hot_st, u
   __syncthreads();
 }
 
+// Fused append for FP16 cold blocks (quantization_bits 0): the evicted token's
+// K and V rows move unchanged from its ring slot to slot e % 64 of the tail
+// block -- in the staged half-block item (row_st, when that item is staged)
+// and in the cache -- and the new token takes the ring slot, staged and in
+// the cache.  Thread tid moves channel tid of both rows.  tile_tail: (phys *
+// Hkv + kv head) of the tail block, < 0 when the block table gives none (the
+// evicted token is then not sealed, as hyb_kv_append skips such a block).
+__device__ __forceinline__ void fused_append_fp16(uint8_t *hot_st, uint8_t *row_st, int tile_tail,
+                                                  const DecodeArgs &a, int b, int h, int L_old, bool do_seal,
+                                                  __half2 new_kv, int tid) {
+  do_seal = do_seal && tile_tail >= 0;
+  const int rs = L_old % kHot;
+  __half *srow = reinterpret_cast<__half *>(hot_st + rs * kHotTokenBytes);
+  const int c = tid;
+  if (do_seal) {
+    const int slot = (L_old - kHot) % kBlock;
+    const __half k_old = srow[c], v_old = srow[kDim + c];
+    __half *trow = reinterpret_cast<__half *>(row_st + (slot % kHot) * kHotTokenBytes);
+    trow[c] = k_old;
+    trow[kDim + c] = v_old;
+    __half *grow = reinterpret_cast<__half *>(a.cold + (size_t)tile_tail * kFp16BlockBytes + slot * kHotTokenBytes);
+    grow[c] = k_old;
+    grow[kDim + c] = v_old;
+  }
+  srow[c] = __low2half(new_kv);
+  srow[kDim + c] = __high2half(new_kv);
+  __half *grow = reinterpret_cast<__half *>(a.hot) + ((((size_t)b * a.hkv + h) * kHot + rs) * 2) * kDim;
+  grow[c] = __low2half(new_kv);
+  grow[kDim + c] = __high2half(new_kv);
+  __syncthreads();
+}
+
 // Raise a warp's running max to cover an item's logits, whose maximum over a
 // lane's tokens is zmax (lane's head hx): m_run per head, the accumulators
 // and the lane's denominator (l_lane + psum_lane / 32767) are rescaled.

@@ -69,7 +69,8 @@ int hyb_check_desc(const hyb_cache_desc *d) {
   const int h = d->hot_tokens;
   if (!(h == 16 || h == 32 || h == 64 || h == 128)) return HYB_ERR_INVALID_VALUE;
   if (d->block_size <= 0 || d->block_size % 8 != 0) return HYB_ERR_INVALID_VALUE;
-  if (d->quant_bits != 8 && d->quant_bits != 4) return HYB_ERR_INVALID_VALUE;
+  // 8 or 4 (section 3.1); 0 keeps the cold zone in FP16 (section 5.2)
+  if (d->quant_bits != 8 && d->quant_bits != 4 && d->quant_bits != 0) return HYB_ERR_INVALID_VALUE;
   if (d->head_dim <= 0 || d->num_kv_heads <= 0 || d->num_q_heads <= 0 || d->batch <= 0 ||
       d->num_phys_blocks < 0 || d->max_blocks_per_seq <= 0)
     return HYB_ERR_INVALID_VALUE;

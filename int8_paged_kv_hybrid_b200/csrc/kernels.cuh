@@ -10,7 +10,7 @@ namespace hyb {
 
 struct AppendArgs {
   __half *hot;                // FP16 [batch][Hkv][32][2][128]
-  uint8_t *cold;              // [num_phys][Hkv][2][8192]
+  uint8_t *cold;              // [num_phys][Hkv][2][8192] (quant_bits 0: FP16 [num_phys][Hkv][64][2][128])
   float *scales;              // [num_phys][Hkv][2]
   const int32_t *block_table; // [batch][max_blocks]
   int32_t *seq_lens;          // [batch]

@@ -201,11 +201,13 @@ def query(w: Workload, step: int = 0) -> np.ndarray:
     return (q * w.q_std).astype(np.float16)
 
 
-def kv_bytes(w: Workload, lens: Optional[np.ndarray] = None) -> int:
+def kv_bytes(w: Workload, lens: Optional[np.ndarray] = None, quant_bits: int = 8) -> int:
     """Algorithmic bytes one decode pass must move: cold codes (256 B per
     token and kv head at INT8, 128 B at INT4), two FP32 scales per block and
     kv head, FP16 hot tokens (512 B per token and kv head), the block table
-    (4 B per block), q and the FP16 output."""
+    (4 B per block), q and the FP16 output.  quant_bits 4: every cold block
+    INT4; quant_bits 0: FP16 cold tokens (512 B per token and kv head) and no
+    scales."""
     lens = w.lens if lens is None else lens
     hkv, d = w.num_kv_heads, w.head_dim
     total = 0
@@ -215,13 +217,18 @@ def kv_bytes(w: Workload, lens: Optional[np.ndarray] = None) -> int:
         hot = L - cold
         nblk = (cold + BLOCK - 1) // BLOCK
         n4 = 0
-        if w.n_int4 is not None:
+        if quant_bits == 4:
+            n4 = nblk
+        elif w.n_int4 is not None and quant_bits == 8:
             n4 = min(int(w.n_int4[b]), nblk)
         # tokens in INT4 blocks (the oldest n4 blocks are always full)
         t4 = min(cold, n4 * BLOCK)
         t8 = cold - t4
-        total += hkv * (t8 * 2 * d + t4 * d)       # K + V codes
-        total += hkv * nblk * 2 * 4                # scales
+        if quant_bits == 0:
+            total += hkv * cold * 2 * d * 2        # K + V, FP16
+        else:
+            total += hkv * (t8 * 2 * d + t4 * d)   # K + V codes
+            total += hkv * nblk * 2 * 4            # scales
         total += hkv * hot * 2 * d * 2             # hot K + V FP16
         total += nblk * 4                          # block table entries
     total += w.batch * w.num_q_heads * d * 2 * 2   # q in, out
@@ -261,17 +268,20 @@ def custom_workload(name, lens, num_q_heads, num_kv_heads, seed, softmax_scale=N
                     split_tokens=split_tokens)
 
 
-def append_bytes(w: Workload, n_new: np.ndarray) -> int:
+def append_bytes(w: Workload, n_new: np.ndarray, quant_bits: int = 8) -> int:
     """Algorithmic bytes of appending n_new[b] in {0, 1} tokens beyond what the
     attention pass reads anyway (the evicted token and the tail block are in
     the attention bytes): the new token's FP16 K and V read (512 B per kv
     head) and written to the hot ring (512 B), the sealed token's codes
-    written (256 B at INT8) and the two scales (8 B), per kv head."""
+    written (256 B at INT8, 128 B at INT4, its 512 B FP16 rows at
+    quant_bits 0) and the two scales (8 B, none at quant_bits 0), per kv
+    head."""
+    seal = {8: 256 + 8, 4: 128 + 8, 0: 512}[quant_bits]
     total = 0
     for b, n in enumerate(np.asarray(n_new)):
         if int(n) == 0:
             continue
         L_old = int(w.lens[b]) - int(n)
-        per_head = 512 + 512 + ((256 + 8) if L_old >= HOT else 0)
+        per_head = 512 + 512 + (seal if L_old >= HOT else 0)
         total += w.num_kv_heads * per_head
     return total

@@ -111,13 +111,20 @@ def test_strerror_covers_codes():
 
 
 def test_kv_bytes_formula():
-    """Algorithmic bytes of config 2: 8 x 8 heads x (2016 cold tokens x 256 B +
-    32 hot x 512 B + 32 blocks x 8 B) + 8 x 32 block-table entries x 4 B +
-    q and out (8 x 32 x 128 x 2 B each)."""
+    """Algorithmic bytes of the Llama-3-8B batch-8 L-2048 workload: 8 x 8
+    heads x (2016 cold tokens x 256 B + 32 hot x 512 B + 32 blocks x 8 B) +
+    8 x 32 block-table entries x 4 B + q and out (8 x 32 x 128 x 2 B each);
+    all-INT4 cold blocks halve the codes, FP16 ones double them and drop the
+    scales."""
     w = synth.make_workload(2)
     want = 8 * 8 * (2016 * 256 + 32 * 512 + 32 * 8) + 8 * 32 * 4 + 2 * 8 * 32 * 128 * 2
     assert synth.kv_bytes(w) == want
     assert abs(want / 1e6 - 34.2) < 0.5   # "34.2 MB"
+    assert synth.kv_bytes(w, quant_bits=4) == want - 8 * 8 * 2016 * 128
+    assert synth.kv_bytes(w, quant_bits=0) == want + 8 * 8 * (2016 * 256 - 32 * 8)
+    n = np.ones(8, np.int32)
+    assert synth.append_bytes(w, n) == 8 * 8 * (1024 + 264)
+    assert synth.append_bytes(w, n, quant_bits=0) == 8 * 8 * (1024 + 512)
 
 
 def test_workload_shapes():
@@ -171,4 +178,7 @@ def test_migrate_argument_checks():
     d4 = _desc(batch=4, maxb=16, phys=64, qbits=4)
     d4.n_int4_blocks = 0x7f0000330000
     assert lib.hyb_kv_migrate(ctypes.byref(d4), tgt, 1, None) == _lib.HYB_ERR_UNSUPPORTED
+    d0 = _desc(batch=4, maxb=16, phys=64, qbits=0)  # FP16 cold blocks have no tiers
+    d0.n_int4_blocks = 0x7f0000330000
+    assert lib.hyb_kv_migrate(ctypes.byref(d0), tgt, 1, None) == _lib.HYB_ERR_UNSUPPORTED
     assert "migration" in hk.strerror(100 + _lib.HYB_STATUS_BAD_TIER)

@@ -65,7 +65,7 @@ def test_golden_values_on_gpu(fname, name):
 
 
 @pytest.mark.parametrize("hkv,hq,qbits,int4", [(1, 1, 8, False), (2, 8, 8, True), (2, 2, 4, False),
-                                               (4, 28, 8, True)])
+                                               (4, 28, 8, True), (2, 8, 0, False)])
 def test_random_schedule_bit_exact(hkv, hq, qbits, int4):
     """Random 1..70-token appends; the whole cache is compared after every call."""
     lens = [0, 1, 31, 32, 33, 97, 200, 333]

@@ -38,6 +38,20 @@ def test_int4_parity(qbits, int4):
         assert_decode_close(w, got, lse, ref, ref_lse, what="int4 split=%d" % split)
 
 
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (32, 8), (28, 4)])
+@pytest.mark.parametrize("split", [0, 64, 192])
+def test_fp16_cold_parity(hq, hkv, split):
+    """quantization_bits 0: FP16 cold blocks, attended as half-block items of
+    32 rows; cache bit-exact, output within the bar."""
+    w = synth.custom_workload("fp16", SMALL_LENS, hq, hkv, seed=hq * 17 + hkv, max_step=64)
+    cache, ora = make_pair(w, quant_bits=0)
+    replay(w, cache, ora)
+    assert_cache_equal(w, cache, ora)
+    got, lse, ref, ref_lse = decode_both(w, cache, ora, split_tokens=split)
+    assert_decode_close(w, got, lse, ref, ref_lse, what="fp16 G=%d split=%d" % (hq // hkv, split))
+    assert cache.status() == 0
+
+
 def test_softmax_scale_one_with_scaled_q():
     """Config-2 convention: q ~ N(0,1)/sqrt(d) and softmax_scale = 1."""
     w = synth.custom_workload("s1", [300, 2048], 32, 8, seed=9, softmax_scale=1.0, schedule="chunk")

@@ -57,6 +57,27 @@ def test_steps_bit_exact_and_close(hq, hkv, split):
     _run_steps(w, cache, ora, 70, split, seed=11)
 
 
+@pytest.mark.parametrize("hq,hkv,split", [(8, 2, 0), (32, 8, 128)])
+def test_steps_fp16_cold(hq, hkv, split):
+    """quantization_bits 0: the sealed token's FP16 rows move into the staged
+    half block and the cache; 70 steps cross both halves of a block."""
+    lens = [0, 1, 31, 32, 33, 63, 64, 65, 95, 96, 97, 500, 1200]
+    w = synth.custom_workload("step16", lens, hq, hkv, seed=hq + hkv, max_step=64, pool_extra=0)
+    nb = [synth.cold_blocks_for(L + 70) for L in lens]
+    bt = np.full((w.batch, max(nb)), -1, np.int32)
+    bt[:, :w.max_blocks] = w.block_table
+    nxt = w.num_phys_blocks
+    for b in range(w.batch):
+        for j in range(synth.cold_blocks_for(int(w.lens[b])), nb[b]):
+            bt[b, j] = nxt
+            nxt += 1
+    w.block_table = bt
+    w.num_phys_blocks = nxt
+    cache, ora = make_pair(w, quant_bits=0)
+    replay(w, cache, ora)
+    _run_steps(w, cache, ora, 70, split, seed=17, qbits=0)
+
+
 @pytest.mark.parametrize("qbits,int4", [(4, False), (8, True)])
 def test_steps_int4(qbits, int4):
     lens = [40, 130, 600]
