@@ -3,14 +3,16 @@
  *
  * The method: web page "DeepSeek V4混合式KV Cache推理优化实战解析" (cited as
  * [hybrid_v2 page] below).  A sequence's KV cache has two tiers:
- *   - a hot zone holding the most recent 32 tokens in FP16, never quantized,
+ *   - a hot zone holding the most recent hot_tokens (32 in the page's example
+ *     set; 16, 64 or 128 also built) tokens in FP16, never quantized,
  *     K and V interleaved per token, 512-byte aligned (sections 2.1, 3.1, 3.2);
  *   - a cold zone holding all earlier tokens in 64-token blocks of symmetric
  *     INT8 with a block-wise scale, INT4 for the "L2" cold blocks (sections
  *     2.1, 2.2, 3.1), reached through a block table (section 3.2, block header).
  * The three fields of the hybrid_v2 contract are hot_tokens (power of two),
  * quantization_bits (4 or 8) and block_size (a multiple of 8); this library
- * implements hot_tokens 32 and block_size 64 with quantization_bits 8 or 4
+ * implements block_size 64 with hot_tokens 16, 32, 64 or 128 and
+ * quantization_bits 8 or 4
  * (section 3.1; section 5.1 for the invalid-value error), and
  * quantization_bits 0, which the page's section 5.2 gives as the switch that
  * keeps the cold zone in FP16.
@@ -63,8 +65,8 @@ typedef struct CUstream_st *hyb_stream_t; /* same type as cudaStream_t */
 #define HYB_OK 0
 #define HYB_ERR_INVALID_VALUE (-1) /* bad config value, shape, null or misaligned pointer;
                                       named after the page's CUDA_ERROR_INVALID_VALUE (3.1) */
-#define HYB_ERR_UNSUPPORTED (-2)   /* valid per the page but not built: hot_tokens != 32,
-                                      block_size != 64, head_dim != 128, Hq/Hkv > 8 */
+#define HYB_ERR_UNSUPPORTED (-2)   /* valid per the page but not built: block_size != 64,
+                                      head_dim != 128, Hq/Hkv > 8 */
 #define HYB_ERR_WORKSPACE (-3)     /* workspace missing or smaller than required */
 #define HYB_ERR_CUDA (-4)          /* a CUDA runtime call or launch failed */
 #define HYB_ERR_SCRATCH_LIMIT (-5) /* hyb_decode_attn_noalloc: the call needs more scratch
@@ -85,22 +87,24 @@ typedef struct CUstream_st *hyb_stream_t; /* same type as cudaStream_t */
 /*
  * The cache descriptor (host struct; the pointers inside are device memory).
  *
- * Geometry: hot_tokens HOT = 32, block_size BLK = 64, head_dim D = 128,
+ * Geometry: hot_tokens HOT in {16, 32, 64, 128} (32 is the page's value),
+ * block_size BLK = 64, head_dim D = 128,
  * num_kv_heads Hkv >= 1, num_q_heads Hq a multiple of Hkv with Hq/Hkv <= 8
  * (query head h reads kv head h / (Hq/Hkv)), quant_bits 8 (INT8 cold blocks;
  * logical blocks below n_int4_blocks[b] are INT4), 4 (every cold block INT4)
  * or 0 (FP16 cold blocks, nothing quantized; n_int4_blocks and scales are not
  * read).
  *
- * Token positions 0..L-1 of sequence b (L = seq_lens[b]): positions >= L-32
+ * Token positions 0..L-1 of sequence b (L = seq_lens[b]): positions >= L-HOT
  * are hot, the others cold; cold position p lives in logical block p/64,
  * slot p%64, of physical block block_table[b][p/64].
  *
  * Memory layouts (all little-endian, all device memory):
- *   hot    FP16 [batch][Hkv][HOT][2][D]: per (sequence, kv head) a ring of 32
- *          token slots, slot = position % 32, each slot the K row (D halves)
- *          followed by the V row (D halves) -- 512 B per token, 16 KB per
- *          (sequence, kv head).  Base 512-byte aligned ([hybrid_v2 page] 3.2).
+ *   hot    FP16 [batch][Hkv][HOT][2][D]: per (sequence, kv head) a ring of HOT
+ *          token slots, slot = position % HOT, each slot the K row (D halves)
+ *          followed by the V row (D halves) -- 512 B per token, HOT * 512 B
+ *          per (sequence, kv head).  Base 512-byte aligned ([hybrid_v2 page]
+ *          3.2).
  *   cold   bytes [num_phys_blocks][Hkv][2][8192]: per physical block and kv
  *          head a K tile then a V tile of 64 tokens x 128 channels.  Base
  *          16-byte aligned.
@@ -162,8 +166,9 @@ typedef struct hyb_cache_desc {
  * Returns HYB_OK, HYB_ERR_INVALID_VALUE (hot_tokens not a power of two in
  * {16, 32, 64, 128}, block_size not a multiple of 8, quant_bits not 8, 4 or 0,
  * non-positive sizes, Hq not a multiple of Hkv, null or misaligned pointers)
- * or HYB_ERR_UNSUPPORTED (a valid configuration other than 32 / 64 / D=128,
- * or Hq/Hkv > 8).  The contract is the page's section 3.1 and 5.1.
+ * or HYB_ERR_UNSUPPORTED (a valid configuration with block_size != 64 or
+ * head_dim != 128, or Hq/Hkv > 8).  The contract is the page's section 3.1
+ * and 5.1 (quant_bits 0: section 5.2).
  */
 int hyb_check_desc(const hyb_cache_desc *desc);
 
@@ -175,7 +180,7 @@ int hyb_check_desc(const hyb_cache_desc *desc);
  *          is position seq_lens[b] + j.  Rows j >= n_new[b] are not read.
  *          16-byte aligned.
  * For L_old = seq_lens[b] and L_new = L_old + n_new[b], the positions
- * max(0, L_old-32) .. max(0, L_new-32)-1 leave the hot zone in ascending
+ * max(0, L_old-HOT) .. max(0, L_new-HOT)-1 leave the hot zone in ascending
  * order (their FP16 values come from the hot ring, or straight from k_new /
  * v_new for new tokens that never become hot).  They are grouped by logical
  * block; per group, kv head and K|V:
@@ -186,8 +191,9 @@ int hyb_check_desc(const hyb_cache_desc *desc);
  *        clamp(rint((c * s_old) / s_c), -Q, Q) and s = s_c;
  *   else s = s_old;
  *   new codes = (s == 0) ? 0 : clamp(rint(x / s), -Q, Q)   (rint: half to even).
- * Then the newest min(n_new[b], 32) tokens are written to hot slots
- * position % 32 and seq_lens[b] = L_new.  The result is bit-exact and does
+ * (quant_bits 0: the rows are copied unchanged, no scale.)  Then the newest
+ * min(n_new[b], HOT) tokens are written to hot slots position % HOT and
+ * seq_lens[b] = L_new.  The result is bit-exact and does
  * not depend on the launch configuration.
  * Device errors: HYB_STATUS_BAD_N_NEW or HYB_STATUS_CAPACITY (sequence
  * untouched), HYB_STATUS_BAD_BLOCK (that block skipped, seq_lens still
@@ -201,7 +207,7 @@ int hyb_kv_append(const hyb_cache_desc *desc, const int32_t *n_new, int32_t max_
  * upper bound of seq_lens[b]; split_tokens is a multiple of 64 (tokens per
  * split of the cold range) or 0 for automatic.  Writes the split size used
  * and the number of splits per sequence, n_splits = max(1,
- * ceil(max(0, max_seq_len - 32) / split_tokens)).  Returns HYB_OK or
+ * ceil(max(0, max_seq_len - HOT) / split_tokens)).  Returns HYB_OK or
  * HYB_ERR_INVALID_VALUE.  The automatic choice depends on the GPU's SM count
  * (device 0 of the current context when none is current).
  */

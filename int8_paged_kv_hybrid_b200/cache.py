@@ -16,14 +16,16 @@ TILE_BYTES = BLOCK * HEAD_DIM
 
 class HybridKVCache:
     def __init__(self, batch, num_kv_heads, num_q_heads, num_phys_blocks, max_blocks_per_seq,
-                 quant_bits=8, block_table=None, n_int4=None, device="cuda"):
+                 quant_bits=8, block_table=None, n_int4=None, device="cuda", hot_tokens=HOT):
         import torch
         self.batch, self.hkv, self.hq = int(batch), int(num_kv_heads), int(num_q_heads)
         self.num_phys, self.max_blocks = int(num_phys_blocks), int(max_blocks_per_seq)
         self.quant_bits = int(quant_bits)
+        self.hot_tokens = int(hot_tokens)
         dev = torch.device(device)
         self.device = dev
-        self.hot = torch.zeros((self.batch, self.hkv, HOT, 2, HEAD_DIM), dtype=torch.float16, device=dev)
+        self.hot = torch.zeros((self.batch, self.hkv, self.hot_tokens, 2, HEAD_DIM), dtype=torch.float16,
+                               device=dev)
         # quant_bits 0: FP16 blocks, 64 rows of K then V (twice the bytes)
         parts = 4 if self.quant_bits == 0 else 2
         self.cold = torch.zeros((self.num_phys, self.hkv, parts, TILE_BYTES), dtype=torch.uint8, device=dev)
@@ -45,7 +47,7 @@ class HybridKVCache:
 
     def _make_desc(self):
         d = _lib.CacheDesc()
-        d.hot_tokens, d.block_size, d.head_dim = HOT, BLOCK, HEAD_DIM
+        d.hot_tokens, d.block_size, d.head_dim = self.hot_tokens, BLOCK, HEAD_DIM
         d.quant_bits = self.quant_bits
         d.num_kv_heads, d.num_q_heads = self.hkv, self.hq
         d.num_phys_blocks, d.max_blocks_per_seq, d.batch = self.num_phys, self.max_blocks, self.batch

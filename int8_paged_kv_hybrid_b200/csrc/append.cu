@@ -54,7 +54,7 @@ __device__ __forceinline__ void load4(const AppendArgs &a, int b, int h, int kv,
                                       int lane, float x[4]) {
   const __half *src;
   if (t < L_old)
-    src = a.hot + ((((size_t)b * a.hkv + h) * kHot + (t % kHot)) * 2 + kv) * kDim;
+    src = a.hot + ((((size_t)b * a.hkv + h) * a.hot_tokens + (t & (a.hot_tokens - 1))) * 2 + kv) * kDim;
   else
     src = (kv ? a.v_new : a.k_new) + (((size_t)b * a.max_new + (t - L_old)) * a.hkv + h) * kDim;
   const uint2 raw = *reinterpret_cast<const uint2 *>(src + 4 * lane);
@@ -77,13 +77,13 @@ __global__ void __launch_bounds__(512) append_kernel(AppendArgs a) {
     return;
   }
   const long long L_new_ll = static_cast<long long>(L_old) + n;
-  if (L_new_ll - kHot > static_cast<long long>(a.max_blocks) * kBlock || L_new_ll > 0x7fffffffLL) {
+  if (L_new_ll - a.hot_tokens > static_cast<long long>(a.max_blocks) * kBlock || L_new_ll > 0x7fffffffLL) {
     if (threadIdx.x == 0) set_status(a.status, HYB_STATUS_CAPACITY);
     return;
   }
   if (n == 0) return;
   const int L_new = static_cast<int>(L_new_ll);
-  const int e0 = max(0, L_old - kHot), e1 = max(0, L_new - kHot);
+  const int e0 = max(0, L_old - a.hot_tokens), e1 = max(0, L_new - a.hot_tokens);
   __shared__ int8_t s_tbl[16][256];  // per-warp re-quantization tables
 
   for (int pair = warp; pair < 2 * a.hkv; pair += nwarps) {
@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(512) append_kernel(AppendArgs a) {
         for (int t = p0; t < p1; t++) {
           const __half *src;
           if (t < L_old)
-            src = a.hot + ((((size_t)b * a.hkv + h) * kHot + (t % kHot)) * 2 + kv) * kDim;
+            src = a.hot + ((((size_t)b * a.hkv + h) * a.hot_tokens + (t & (a.hot_tokens - 1))) * 2 + kv) * kDim;
           else
             src = (kv ? a.v_new : a.k_new) + (((size_t)b * a.max_new + (t - L_old)) * a.hkv + h) * kDim;
           __half *dst = blk + ((t - i * kBlock) * 2 + kv) * kDim;
@@ -185,13 +185,13 @@ __global__ void __launch_bounds__(512) append_kernel(AppendArgs a) {
       __syncwarp();
       p0 = p1;
     }
-    // newest min(n, 32) tokens into the hot ring (after their slots' old
+    // newest min(n, hot) tokens into the hot ring (after their slots' old
     // occupants were read above)
-    const int nh = min(n, kHot);
+    const int nh = min(n, a.hot_tokens);
     for (int t = L_new - nh; t < L_new; t++) {
       const __half *src =
           (kv ? a.v_new : a.k_new) + (((size_t)b * a.max_new + (t - L_old)) * a.hkv + h) * kDim;
-      __half *dst = a.hot + ((((size_t)b * a.hkv + h) * kHot + (t % kHot)) * 2 + kv) * kDim;
+      __half *dst = a.hot + ((((size_t)b * a.hkv + h) * a.hot_tokens + (t & (a.hot_tokens - 1))) * 2 + kv) * kDim;
       *reinterpret_cast<uint2 *>(dst + 4 * lane) = *reinterpret_cast<const uint2 *>(src + 4 * lane);
     }
   }

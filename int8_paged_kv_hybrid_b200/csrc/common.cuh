@@ -8,13 +8,17 @@
 
 namespace hyb {
 
-constexpr int kHot = 32;          // hot-zone tokens per sequence
+// hot-zone tokens per sequence: a run-time power of two in {16, 32, 64, 128}
+// (hot_tokens of the descriptor); kMaxHot bounds it
+constexpr int kMaxHot = 128;
 constexpr int kBlock = 64;        // tokens per cold block
 constexpr int kDim = 128;         // head dimension
 constexpr int kTileBytes = kBlock * kDim;        // one K or V tile, INT8
 constexpr int kTilePairBytes = 2 * kTileBytes;   // K tile + V tile of one (block, kv head)
 constexpr int kHotTokenBytes = 2 * kDim * 2;     // K row + V row, FP16
-constexpr int kHotBytes = kHot * kHotTokenBytes; // 16 KB per (sequence, kv head)
+// FP16 rows (hot ring, FP16 cold blocks) are staged 32 rows (16 KB) at a time
+constexpr int kItemRows = 32;
+constexpr int kItemBytes = kItemRows * kHotTokenBytes;
 // quantization_bits 0: an FP16 cold block keeps the hot ring's row layout
 // (K row then V row per token), 32 KB per (block, kv head)
 constexpr int kFp16BlockBytes = kBlock * kHotTokenBytes;

@@ -113,30 +113,39 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
       a.seq_cnt[b] = 0;
     }
   }
-  const int Lc = max(0, L - kHot);
+  const int H = a.hot_tokens;
+  const int Lc = max(0, L - H);
   const int nblk = (Lc + kBlock - 1) / kBlock;
   const int Sb = max(1, (nblk + a.split_blocks - 1) / a.split_blocks);
   // past this sequence's last split: no work and no partial (a cluster member
   // still takes part in the cluster's merge, with an empty state)
   if (!kCluster && s >= Sb) return;
   const int ncold = max(0, min(nblk, i0 + a.split_blocks) - i0);
-  const int nhot = (s == Sb - 1) ? min(L, kHot) : 0;
-  // FP16 cold blocks (quantization_bits 0) are two items of 32 rows each
+  // FP16 rows (the hot ring, FP16 cold blocks) are items of up to 32 rows;
+  // FP16 cold blocks (quantization_bits 0) are two items each
+  const int nhot = (s == Sb - 1) ? min(L, H) : 0;
   constexpr bool fp16 = kF16;
   const int ncold_it = fp16 ? 2 * ncold : ncold;
-  const int kh = ncold_it;  // the hot item
-  const int nitems = ncold_it + (nhot > 0 ? 1 : 0);
+  const int kh = ncold_it;  // the first hot item
+  const int nitems = ncold_it + (nhot + kItemRows - 1) / kItemRows;
   // fused step, in the split that holds the tail block and the hot ring: the
-  // new token goes to ring slot L_old % 32 (whose old occupant, position
-  // L_old - 32, is sealed into the tail block first)
+  // new token goes to ring slot rs = L_old % hot, whose old occupant
+  // (position L_old - hot, read in the prologue) is sealed into the tail
+  // block at that block's item; the ring slot is rewritten at its hot item
   const bool do_ring = n_app == 1 && nhot > 0;
-  const bool do_seal = do_ring && L_old >= kHot;
-  // item at which the append is done: the one that receives the sealed token
-  const int k_fused = !do_seal ? kh : fp16 ? 2 * (ncold - 1) + ((L_old - kHot) % kBlock) / kHot : ncold - 1;
+  const bool do_seal = do_ring && L_old >= H;
+  const int rs = L_old & (H - 1);
+  const int k_ring = kh + rs / kItemRows;
+  const int k_seal = !do_seal ? -1 : fp16 ? 2 * (ncold - 1) + ((L_old - H) % kBlock) / kItemRows : ncold - 1;
   __half2 new_kv = __halves2half2(__float2half_rn(0.f), __float2half_rn(0.f));
+  __half2 old_kv = new_kv;
   if (do_ring) {
     const size_t o = ((size_t)b * a.hkv + h) * kDim + tid;
     new_kv = __halves2half2(a.k_new[o], a.v_new[o]);
+    if (do_seal) {
+      const __half *er = reinterpret_cast<const __half *>(a.hot) + (((size_t)b * a.hkv + h) * H + rs) * 2 * kDim;
+      old_kv = __halves2half2(er[tid], er[kDim + tid]);
+    }
   }
   const int n_int4_b = a.quant_bits == 4 ? 0x7fffffff : (a.n_int4 ? a.n_int4[b] : 0);
 
@@ -148,6 +157,10 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
     }
     sm.abort_flag = 0;
     mbar_fence_init();
+  }
+  if (do_seal) {
+    sm.seal.erow[tid] = __low2half(old_kv);
+    sm.seal.erow[kDim + tid] = __high2half(old_kv);
   }
   if (tid < ncold) {
     int phys = phys_raw;
@@ -168,14 +181,14 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
     if (k < ncold_it) {
       const int kb = fp16 ? k >> 1 : k;
       const int phys = sm.phys[kb];
-      const int nrow = fp16 ? min(kHot, Lc - (i0 + kb) * kBlock - (k & 1) * kHot) : 1;
+      const int nrow = fp16 ? min(kItemRows, Lc - (i0 + kb) * kBlock - (k & 1) * kItemRows) : 1;
       if (phys < 0 || nrow <= 0) {
         mbar_arrive(&sm.full[st]);
         return;
       }
       if (fp16) {
         // the half block's sealed rows
-        const uint8_t *src = a.cold + ((size_t)phys * a.hkv + h) * kFp16BlockBytes + (k & 1) * kHotBytes;
+        const uint8_t *src = a.cold + ((size_t)phys * a.hkv + h) * kFp16BlockBytes + (k & 1) * kItemBytes;
         const uint32_t bytes = static_cast<uint32_t>(nrow) * kHotTokenBytes;
         mbar_arrive_expect_tx(&sm.full[st], bytes);
         bulk_g2s(dst, src, bytes, &sm.full[st], pol);
@@ -191,8 +204,10 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
         bulk_g2s(dst + kTileBytes, src + kTileBytes, kTileBytes / 2, &sm.full[st], pol);
       }
     } else {
-      const uint8_t *src = a.hot + ((size_t)b * a.hkv + h) * kHotBytes;
-      const uint32_t bytes = static_cast<uint32_t>(nhot) * kHotTokenBytes;
+      // hot item j: ring slots 32j .. min(32j + 32, nhot) - 1
+      const int j = k - kh;
+      const uint8_t *src = a.hot + (((size_t)b * a.hkv + h) * H + j * kItemRows) * kHotTokenBytes;
+      const uint32_t bytes = static_cast<uint32_t>(min(kItemRows, nhot - j * kItemRows)) * kHotTokenBytes;
       mbar_arrive_expect_tx(&sm.full[st], bytes);
       bulk_g2s(dst, src, bytes, &sm.full[st], pol);
     }
@@ -248,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
     if (tid == 0) {
       for (; next_issue < min(nitems, k + kStages); next_issue++) {
         const int j = next_issue - kStages;  // previous item of that stage
-        if (next_issue <= ((do_ring && k == k_fused) ? kh : k)) {
+        if (next_issue <= k) {
           if (!mbar_wait_bounded(&sm.empty[j % kStages], (j / kStages) & 1, kWaitCycles)) {
             set_status(a.status, HYB_STATUS_TIMEOUT);
             sm.abort_flag = 1;
@@ -263,27 +278,26 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
     }
     bool ok = mbar_wait_bounded(&sm.full[st], (k / kStages) & 1, kWaitCycles);
     if (!ok && lane == 0) set_status(a.status, HYB_STATUS_TIMEOUT);
-    if (do_ring && k == k_fused) {
+    if (k == k_seal || (do_ring && k == k_ring)) {
       // ---------------- fused append (whole CTA, in the staged copies) ----------------
-      if (k != kh) ok = ok && mbar_wait_bounded(&sm.full[kh % kStages], (kh / kStages) & 1, kWaitCycles);
       ok = __syncthreads_and(ok) != 0;
-      if (ok && fp16) {
-        const int tb = do_seal ? ncold - 1 : 0;  // the tail block
-        fused_append_fp16(sm.ring[kh % kStages], sm.ring[k_fused % kStages], sm.phys[tb] * a.hkv + h, a, b, h,
-                          L_old, do_seal, new_kv, tid);
+      if (ok && k == k_seal) {
+        const int tb = ncold - 1;  // the tail block
+        if (fp16)
+          fused_seal_fp16(sm.seal, sm.ring[st], sm.phys[tb] * a.hkv + h, a, L_old, true, tid);
+        else
+          fused_seal(sm.seal, sm.ring[st], &sm.scl[tb], sm.phys[tb] * a.hkv + h, (i0 + tb) < n_int4_b, a, L_old,
+                     true, tid, warp, lane);
       } else if (ok) {
-        const int ti = do_seal ? ncold - 1 : 0;  // the tail block's item
-        fused_append(sm.seal, sm.ring[ncold % kStages], sm.ring[ti % kStages], &sm.scl[ti],
-                     sm.phys[ti] * a.hkv + h, (i0 + ti) < n_int4_b, a, b, h, L_old, do_seal, new_kv, tid, warp,
-                     lane);
+        ring_put(sm.ring[st], rs, new_kv, a, b, h, tid);
       }
     }
     ok = ok && *reinterpret_cast<volatile int *>(&sm.abort_flag) == 0;
     const uint8_t *stage = sm.ring[st];
     // rows of an FP16 item: the hot ring, or half of an FP16 cold block
-    int nrow = nhot;
+    int nrow = min(kItemRows, nhot - (k - kh) * kItemRows);
     if (k < ncold_it)
-      nrow = !fp16 || sm.phys[k >> 1] < 0 ? 0 : min(kHot, Lc - (i0 + (k >> 1)) * kBlock - (k & 1) * kHot);
+      nrow = !fp16 || sm.phys[k >> 1] < 0 ? 0 : min(kItemRows, Lc - (i0 + (k >> 1)) * kBlock - (k & 1) * kItemRows);
     if (ok && !fp16 && k < ncold) {
       // ---------------- cold block ----------------
       const int i = i0 + k;

@@ -85,30 +85,33 @@ struct SealScratch {
   int8_t rqt[2][256];  // re-quantization tables of the tail block (K, V)
   float seal_s[2];     // the tail block's scales after sealing
   int seal_rq[2];      // 1 if the tail block's codes were re-quantized
+  alignas(16) __half erow[2 * kDim];  // the evicted token: K row, V row (FP16)
 };
 
-// Fused decode step: append the sequence's new token inside the staged copies
-// of the tail block (tile_st, scales *scl_tail, tile index tile_tail = its
-// physical block * Hkv + h) and
-// of the hot ring (hot_st), with the arithmetic of hyb_kv_append
-// (bit-exact), and write back what changed.  All threads of the CTA call it.
-__device__ __forceinline__ void fused_append(SealScratch &ss, uint8_t *hot_st, uint8_t *tile_st, float2 *scl_tail,
-                                             int tile_tail, bool int4_tail, const DecodeArgs &a, int b, int h,
-                                             int L_old, bool do_seal, __half2 new_kv, int tid, int warp, int lane) {
+// Fused decode step, seal half: the token leaving the hot zone (position e =
+// L_old - hot, its FP16 rows in ss.erow) is quantized into slot e % 64 of the
+// tail block, inside the staged copy of that block (tile_st, scales
+// *scl_tail, so that this attention sees it) and in the cache (tile index
+// tile_tail = physical block * Hkv + kv head).  Same arithmetic as
+// hyb_kv_append: absmax scale, a grown scale re-quantizes the codes already
+// in the block, RNE codes.  Called by the whole CTA.
+__device__ __forceinline__ void fused_seal(SealScratch &ss, uint8_t *tile_st, float2 *scl_tail, int tile_tail,
+                                           bool int4_tail, const DecodeArgs &a, int L_old, bool do_seal, int tid,
+                                           int warp, int lane) {
   // A tail block the block table does not give (entry < 0 or past the pool;
   // HYB_STATUS_BAD_BLOCK is set when the entry is read): the evicted token is
   // not sealed and nothing is written through the tile, as hyb_kv_append
-  // skips such a block; the new token still goes to the ring.
+  // skips such a block.
   do_seal = do_seal && tile_tail >= 0;
-  const int rs = L_old % kHot;  // ring slot of the evicted and of the new token
-  const int e = L_old - kHot;   // position sealed (when do_seal)
-  const int slot = do_seal ? e % kBlock : 0;
-  const bool int4 = do_seal && int4_tail;
+  if (!do_seal) return;
+  const int e = L_old - a.hot_tokens;  // position sealed
+  const int slot = e % kBlock;
+  const bool int4 = int4_tail;
   const int Q = int4 ? 7 : 127;
-  if (do_seal && warp < 2) {
+  if (warp < 2) {
     // warp 0: K, warp 1: V -- absmax of the evicted token, new scale
     const int kv = warp;
-    const __half *row = reinterpret_cast<const __half *>(hot_st + rs * kHotTokenBytes) + kv * kDim;
+    const __half *row = ss.erow + kv * kDim;
     float amax = 0.f;
 #pragma unroll
     for (int j = 0; j < 4; j++) amax = fmaxf(amax, fabsf(__half2float(row[4 * lane + j])));
@@ -131,24 +134,21 @@ __device__ __forceinline__ void fused_append(SealScratch &ss, uint8_t *hot_st, u
     }
   }
   __syncthreads();
-  if (do_seal && tid == 0) *scl_tail = make_float2(ss.seal_s[0], ss.seal_s[1]);  // attention uses these
-  if (do_seal) {
-    // codes already in the tail block, under a grown scale
+  if (tid == 0) *scl_tail = make_float2(ss.seal_s[0], ss.seal_s[1]);  // attention uses these
+  // codes already in the tail block, under a grown scale
 #pragma unroll
-    for (int kv = 0; kv < 2; kv++) {
-      if (!ss.seal_rq[kv]) continue;
-      uint32_t *w32 = reinterpret_cast<uint32_t *>(tile_st + kv * kTileBytes);
-      const int nw = requant_nwords(kv, int4, slot);
-      for (int w = tid; w < nw; w += kThreads) w32[w] = requant_word(w32[w], w, kv, int4, slot, ss.rqt[kv]);
-    }
+  for (int kv = 0; kv < 2; kv++) {
+    if (!ss.seal_rq[kv]) continue;
+    uint32_t *w32 = reinterpret_cast<uint32_t *>(tile_st + kv * kTileBytes);
+    const int nw = requant_nwords(kv, int4, slot);
+    for (int w = tid; w < nw; w += kThreads) w32[w] = requant_word(w32[w], w, kv, int4, slot, ss.rqt[kv]);
   }
   __syncthreads();
   const int c = tid;  // channel
-  if (do_seal) {
+  {
     // the evicted token's codes into slot `slot`
-    const __half *krow = reinterpret_cast<const __half *>(hot_st + rs * kHotTokenBytes);
-    const int ck = quantize(__half2float(krow[c]), ss.seal_s[0], Q);
-    const int cv = quantize(__half2float(krow[kDim + c]), ss.seal_s[1], Q);
+    const int ck = quantize(__half2float(ss.erow[c]), ss.seal_s[0], Q);
+    const int cv = quantize(__half2float(ss.erow[kDim + c]), ss.seal_s[1], Q);
     if (!int4) {
       tile_st[slot * kDim + c] = static_cast<uint8_t>(ck);
       tile_st[kTileBytes + c * 64 + 16 * ((slot >> 4) ^ ((c >> 1) & 3)) + (slot & 15)] = static_cast<uint8_t>(cv);
@@ -168,16 +168,7 @@ __device__ __forceinline__ void fused_append(SealScratch &ss, uint8_t *hot_st, u
     }
   }
   __syncthreads();
-  // the new token into the ring slot: the staged copy (for this attention) and the cache
   {
-    __half *srow = reinterpret_cast<__half *>(hot_st + rs * kHotTokenBytes);
-    srow[c] = __low2half(new_kv);
-    srow[kDim + c] = __high2half(new_kv);
-    __half *grow = reinterpret_cast<__half *>(a.hot) + ((((size_t)b * a.hkv + h) * kHot + rs) * 2) * kDim;
-    grow[c] = __low2half(new_kv);
-    grow[kDim + c] = __high2half(new_kv);
-  }
-  if (do_seal) {
     // write back what changed in the tail block: scales, then the whole tile
     // if its codes were re-quantized, else the sealed token's codes
     uint8_t *gtile = a.cold + (size_t)tile_tail * kTilePairBytes;
@@ -204,33 +195,35 @@ __device__ __forceinline__ void fused_append(SealScratch &ss, uint8_t *hot_st, u
   __syncthreads();
 }
 
-// Fused append for FP16 cold blocks (quantization_bits 0): the evicted token's
-// K and V rows move unchanged from its ring slot to slot e % 64 of the tail
-// block -- in the staged half-block item (row_st, when that item is staged)
-// and in the cache -- and the new token takes the ring slot, staged and in
-// the cache.  Thread tid moves channel tid of both rows.  tile_tail: (phys *
-// Hkv + kv head) of the tail block, < 0 when the block table gives none (the
-// evicted token is then not sealed, as hyb_kv_append skips such a block).
-__device__ __forceinline__ void fused_append_fp16(uint8_t *hot_st, uint8_t *row_st, int tile_tail,
-                                                  const DecodeArgs &a, int b, int h, int L_old, bool do_seal,
-                                                  __half2 new_kv, int tid) {
-  do_seal = do_seal && tile_tail >= 0;
-  const int rs = L_old % kHot;
-  __half *srow = reinterpret_cast<__half *>(hot_st + rs * kHotTokenBytes);
+// Fused decode step, seal half for FP16 cold blocks (quantization_bits 0):
+// the evicted token's rows (ss.erow) move unchanged to slot e % 64 of the
+// tail block -- in its staged half-block item (row_st, rows slot % 32) and in
+// the cache.  Thread tid moves channel tid of both rows.
+__device__ __forceinline__ void fused_seal_fp16(const SealScratch &ss, uint8_t *row_st, int tile_tail,
+                                                const DecodeArgs &a, int L_old, bool do_seal, int tid) {
+  if (!do_seal || tile_tail < 0) return;
+  const int slot = (L_old - a.hot_tokens) % kBlock;
   const int c = tid;
-  if (do_seal) {
-    const int slot = (L_old - kHot) % kBlock;
-    const __half k_old = srow[c], v_old = srow[kDim + c];
-    __half *trow = reinterpret_cast<__half *>(row_st + (slot % kHot) * kHotTokenBytes);
-    trow[c] = k_old;
-    trow[kDim + c] = v_old;
-    __half *grow = reinterpret_cast<__half *>(a.cold + (size_t)tile_tail * kFp16BlockBytes + slot * kHotTokenBytes);
-    grow[c] = k_old;
-    grow[kDim + c] = v_old;
-  }
+  const __half k_old = ss.erow[c], v_old = ss.erow[kDim + c];
+  __half *trow = reinterpret_cast<__half *>(row_st + (slot % kItemRows) * kHotTokenBytes);
+  trow[c] = k_old;
+  trow[kDim + c] = v_old;
+  __half *grow = reinterpret_cast<__half *>(a.cold + (size_t)tile_tail * kFp16BlockBytes + slot * kHotTokenBytes);
+  grow[c] = k_old;
+  grow[kDim + c] = v_old;
+  __syncthreads();
+}
+
+// Fused decode step, ring half: the new token goes to ring slot rs = L_old %
+// hot -- row rs % 32 of its staged hot item (item_st, for this attention) and
+// the cache.  Thread tid writes channel tid of both rows.
+__device__ __forceinline__ void ring_put(uint8_t *item_st, int rs, __half2 new_kv, const DecodeArgs &a, int b,
+                                         int h, int tid) {
+  const int c = tid;
+  __half *srow = reinterpret_cast<__half *>(item_st + (rs % kItemRows) * kHotTokenBytes);
   srow[c] = __low2half(new_kv);
   srow[kDim + c] = __high2half(new_kv);
-  __half *grow = reinterpret_cast<__half *>(a.hot) + ((((size_t)b * a.hkv + h) * kHot + rs) * 2) * kDim;
+  __half *grow = reinterpret_cast<__half *>(a.hot) + ((((size_t)b * a.hkv + h) * a.hot_tokens + rs) * 2) * kDim;
   grow[c] = __low2half(new_kv);
   grow[kDim + c] = __high2half(new_kv);
   __syncthreads();

@@ -83,7 +83,7 @@ int hyb_check_desc(const hyb_cache_desc *d) {
       (d->n_int4_blocks && !aligned(d->n_int4_blocks, 4)))
     return HYB_ERR_INVALID_VALUE;
   // what this library builds
-  if (h != hyb::kHot || d->block_size != hyb::kBlock || d->head_dim != hyb::kDim)
+  if (d->block_size != hyb::kBlock || d->head_dim != hyb::kDim)
     return HYB_ERR_UNSUPPORTED;
   if (d->num_q_heads / d->num_kv_heads > 8) return HYB_ERR_UNSUPPORTED;
   return HYB_OK;
@@ -112,6 +112,7 @@ int hyb_kv_append(const hyb_cache_desc *d, const int32_t *n_new, int32_t max_new
   a.max_blocks = d->max_blocks_per_seq;
   a.quant_bits = d->quant_bits;
   a.max_new = max_new;
+  a.hot_tokens = d->hot_tokens;
   const cudaError_t e = hyb::launch_append(a, d->batch, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HYB_OK : cuda_fail(e);
 }
@@ -138,8 +139,8 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
   const int rc = hyb_check_desc(d);
   if (rc != HYB_OK) return rc;
   if (max_seq_len < 0) return HYB_ERR_INVALID_VALUE;
-  const long long nblk = (static_cast<long long>(max_seq_len) - hyb::kHot > 0)
-                             ? (max_seq_len - hyb::kHot + hyb::kBlock - 1) / hyb::kBlock
+  const long long nblk = (static_cast<long long>(max_seq_len) - d->hot_tokens > 0)
+                             ? (max_seq_len - d->hot_tokens + hyb::kBlock - 1) / hyb::kBlock
                              : 0;
   if (nblk > d->max_blocks_per_seq) return HYB_ERR_INVALID_VALUE;
   const int group = d->num_q_heads / d->num_kv_heads;
@@ -295,6 +296,7 @@ static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_s
   a.num_phys = d->num_phys_blocks;
   a.max_blocks = d->max_blocks_per_seq;
   a.quant_bits = d->quant_bits;
+  a.hot_tokens = d->hot_tokens;
   a.n_splits = pl.ns;
   a.split_blocks = pl.tb;
   a.max_seq_len = max_seq_len;
@@ -366,6 +368,7 @@ int hyb_kv_migrate(const hyb_cache_desc *d, const int32_t *target_n_int4, int32_
   a.num_phys = d->num_phys_blocks;
   a.max_blocks = d->max_blocks_per_seq;
   a.max_delta = max_delta;
+  a.hot_tokens = d->hot_tokens;
   const cudaError_t e = hyb::launch_migrate(a, d->batch, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HYB_OK : cuda_fail(e);
 }

@@ -9,7 +9,7 @@
 namespace hyb {
 
 struct AppendArgs {
-  __half *hot;                // FP16 [batch][Hkv][32][2][128]
+  __half *hot;                // FP16 [batch][Hkv][hot][2][128]
   uint8_t *cold;              // [num_phys][Hkv][2][8192] (quant_bits 0: FP16 [num_phys][Hkv][64][2][128])
   float *scales;              // [num_phys][Hkv][2]
   const int32_t *block_table; // [batch][max_blocks]
@@ -20,6 +20,7 @@ struct AppendArgs {
   const __half *k_new;        // FP16 [batch][max_new][Hkv][128]
   const __half *v_new;
   int hkv, num_phys, max_blocks, quant_bits, max_new;
+  int hot_tokens;             // hot-zone tokens (power of two, 16..128)
 };
 
 struct DecodeArgs {
@@ -44,6 +45,7 @@ struct DecodeArgs {
   int32_t *g_counters;
   int n_groups;
   int hkv, hq, num_phys, max_blocks, quant_bits, n_splits, split_blocks, max_seq_len;
+  int hot_tokens;             // hot-zone tokens (power of two, 16..128)
   float qk_scale;             // softmax_scale * log2(e)
   // fused decode step (null for attention only): append n_new[b] in {0, 1}
   // tokens first; k_new / v_new FP16 [batch][Hkv][128]; seq_cnt [batch]
@@ -63,6 +65,7 @@ struct MigrateArgs {
   const int32_t *target;      // [batch]
   int32_t *status;
   int hkv, num_phys, max_blocks, max_delta;
+  int hot_tokens;             // hot-zone tokens
 };
 
 struct CombineArgs {

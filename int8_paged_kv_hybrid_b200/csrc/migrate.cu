@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(kMigThreads) migrate_kernel(const MigrateArgs 
   }
   const int i = lo + k;
   if (i >= hi) return;
-  const int Lc = max(0, a.seq_lens[b] - kHot);
+  const int Lc = max(0, a.seq_lens[b] - a.hot_tokens);
   if (i * kBlock >= Lc) return;  // nothing sealed in this block yet: only its tier changes
   const int sealed = min(kBlock, Lc - i * kBlock);
   const int phys = a.block_table[(size_t)b * a.max_blocks + i];

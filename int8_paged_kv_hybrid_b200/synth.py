@@ -38,18 +38,19 @@ class Workload:
     outlier_channels: Optional[np.ndarray] = None  # int [hkv][4] scaled x10 in K
     split_tokens: int = 0
     head_dim: int = HEAD_DIM
+    hot_tokens: int = HOT
 
     @property
     def max_blocks(self) -> int:
         return self.block_table.shape[1]
 
     def cold_blocks(self) -> np.ndarray:
-        return np.array([cold_blocks_for(int(L)) for L in self.lens], np.int64)
+        return np.array([cold_blocks_for(int(L), self.hot_tokens) for L in self.lens], np.int64)
 
 
-def cold_blocks_for(L: int) -> int:
-    """Cold blocks a sequence of L tokens occupies (the newest HOT stay hot)."""
-    return (max(0, L - HOT) + BLOCK - 1) // BLOCK
+def cold_blocks_for(L: int, hot: int = HOT) -> int:
+    """Cold blocks a sequence of L tokens occupies (the newest `hot` stay hot)."""
+    return (max(0, L - hot) + BLOCK - 1) // BLOCK
 
 
 def _block_table(rng, nblk: np.ndarray, pool: int) -> np.ndarray:
@@ -213,7 +214,7 @@ def kv_bytes(w: Workload, lens: Optional[np.ndarray] = None, quant_bits: int = 8
     total = 0
     for b, L in enumerate(lens):
         L = int(L)
-        cold = max(0, L - HOT)
+        cold = max(0, L - w.hot_tokens)
         hot = L - cold
         nblk = (cold + BLOCK - 1) // BLOCK
         n4 = 0
@@ -237,14 +238,14 @@ def kv_bytes(w: Workload, lens: Optional[np.ndarray] = None, quant_bits: int = 8
 
 def custom_workload(name, lens, num_q_heads, num_kv_heads, seed, softmax_scale=None,
                     schedule="random", chunk=64, max_step=64, pool_extra=3, n_int4=None,
-                    outliers=False, split_tokens=0) -> Workload:
+                    outliers=False, split_tokens=0, hot=HOT) -> Workload:
     """A small workload with the given final lengths (for parity tests).
     schedule: "random" (U[1, max_step] tokens per call), "chunk" (prefill in
     `chunk`-token calls then one 1-token call) or "one" (a single call)."""
     rng = np.random.default_rng([seed, 0])
     lens = np.asarray(lens, np.int64)
     B = len(lens)
-    nblk = np.array([cold_blocks_for(int(L)) for L in lens])
+    nblk = np.array([cold_blocks_for(int(L), hot) for L in lens])
     pool = int(nblk.sum()) + pool_extra
     bt = _block_table(rng, nblk, pool)
     if schedule == "random":
@@ -265,7 +266,7 @@ def custom_workload(name, lens, num_q_heads, num_kv_heads, seed, softmax_scale=N
                     num_phys_blocks=pool, block_table=bt,
                     n_int4=None if n_int4 is None else np.asarray(n_int4, np.int32),
                     schedule=sched, max_new=mx, seed=seed, outlier_channels=outl,
-                    split_tokens=split_tokens)
+                    split_tokens=split_tokens, hot_tokens=hot)
 
 
 def append_bytes(w: Workload, n_new: np.ndarray, quant_bits: int = 8) -> int:
@@ -282,6 +283,6 @@ def append_bytes(w: Workload, n_new: np.ndarray, quant_bits: int = 8) -> int:
         if int(n) == 0:
             continue
         L_old = int(w.lens[b]) - int(n)
-        per_head = 512 + 512 + (seal if L_old >= HOT else 0)
+        per_head = 512 + 512 + (seal if L_old >= w.hot_tokens else 0)
         total += w.num_kv_heads * per_head
     return total

@@ -77,6 +77,16 @@ def test_random_schedule_bit_exact(hkv, hq, qbits, int4):
     assert_cache_equal(w, cache, ora, "final")
 
 
+@pytest.mark.parametrize("hot,qbits", [(16, 8), (64, 8), (128, 4), (64, 0)])
+def test_hot_sizes_bit_exact(hot, qbits):
+    """hot_tokens 16 / 64 / 128: ring of that many slots, sealing at L - hot."""
+    lens = [0, 1, hot - 1, hot, hot + 1, hot + 63, hot + 64, 400]
+    w = synth.custom_workload("hot%d" % hot, lens, 8, 2, seed=hot + qbits, max_step=70, hot=hot)
+    cache, ora = make_pair(w, quant_bits=qbits)
+    replay(w, cache, ora, check_every=1)
+    assert_cache_equal(w, cache, ora, "final")
+
+
 def test_outliers_and_big_appends_bit_exact():
     """Outlier K channels (x10) and single calls sealing many blocks at once."""
     lens = [1000, 90, 5000]

@@ -52,6 +52,20 @@ def test_fp16_cold_parity(hq, hkv, split):
     assert cache.status() == 0
 
 
+@pytest.mark.parametrize("hot", [16, 64, 128])
+@pytest.mark.parametrize("split", [0, 64])
+def test_hot_sizes_parity(hot, split):
+    """hot_tokens 16 / 64 / 128: up to four 32-row hot items per sequence."""
+    lens = [0, 1, 5, hot - 1, hot, hot + 1, hot + 64, 700, 2100]
+    w = synth.custom_workload("hot%d" % hot, lens, 32, 8, seed=hot * 3 + split, max_step=64, hot=hot)
+    cache, ora = make_pair(w)
+    replay(w, cache, ora)
+    assert_cache_equal(w, cache, ora)
+    got, lse, ref, ref_lse = decode_both(w, cache, ora, split_tokens=split)
+    assert_decode_close(w, got, lse, ref, ref_lse, what="hot=%d split=%d" % (hot, split))
+    assert cache.status() == 0
+
+
 def test_softmax_scale_one_with_scaled_q():
     """Config-2 convention: q ~ N(0,1)/sqrt(d) and softmax_scale = 1."""
     w = synth.custom_workload("s1", [300, 2048], 32, 8, seed=9, softmax_scale=1.0, schedule="chunk")

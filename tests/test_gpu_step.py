@@ -78,6 +78,30 @@ def test_steps_fp16_cold(hq, hkv, split):
     _run_steps(w, cache, ora, 70, split, seed=17, qbits=0)
 
 
+@pytest.mark.parametrize("hot,qbits,hq,hkv,split", [(16, 8, 8, 2, 0), (64, 8, 32, 8, 0), (128, 8, 8, 2, 64),
+                                                    (64, 0, 8, 2, 0), (128, 4, 28, 4, 0)])
+def test_steps_hot_sizes(hot, qbits, hq, hkv, split):
+    """hot_tokens 16 / 64 / 128: the evicted token (position L - hot, read in
+    the prologue) is sealed at the tail block's item, the new token written
+    at the hot item holding ring slot L % hot."""
+    lens = [0, 1, hot - 1, hot, hot + 1, hot + 63, hot + 64, 500]
+    w = synth.custom_workload("steph%d" % hot, lens, hq, hkv, seed=hot + qbits, max_step=64, pool_extra=0,
+                              hot=hot)
+    nb = [synth.cold_blocks_for(L + 70, hot) for L in lens]
+    bt = np.full((w.batch, max(max(nb), w.max_blocks)), -1, np.int32)
+    bt[:, :w.max_blocks] = w.block_table
+    nxt = w.num_phys_blocks
+    for b in range(w.batch):
+        for j in range(synth.cold_blocks_for(int(w.lens[b]), hot), nb[b]):
+            bt[b, j] = nxt
+            nxt += 1
+    w.block_table = bt
+    w.num_phys_blocks = nxt
+    cache, ora = make_pair(w, quant_bits=qbits)
+    replay(w, cache, ora)
+    _run_steps(w, cache, ora, 70, split, seed=hot, qbits=qbits)
+
+
 @pytest.mark.parametrize("qbits,int4", [(4, False), (8, True)])
 def test_steps_int4(qbits, int4):
     lens = [40, 130, 600]

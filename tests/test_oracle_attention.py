@@ -33,18 +33,19 @@ def _fill(oc, rng, total, hkv, max_step=70, kscale=1.0, vscale=1.0):
 
 
 def _dense_kv(oc, b, L):
-    """Rebuild K, V [L][hkv][D] (float64) position by position: the newest 32
-    from the hot ring (slot p % 32), older ones as code * scale of block p//64,
-    slot p%64."""
+    """Rebuild K, V [L][hkv][D] (float64) position by position: the newest
+    oc.hot from the hot ring (slot p % hot), older ones as code * scale of
+    block p//64, slot p%64."""
     K = np.zeros((L, oc.hkv, D))
     V = np.zeros((L, oc.hkv, D))
     ring = oc.ring(b).astype(np.float64)
-    cold = max(0, L - HOT)
+    H = oc.hot
+    cold = max(0, L - H)
     blocks = {}
     for p in range(L):
         if p >= cold:
-            K[p] = ring[:, p % HOT, 0]
-            V[p] = ring[:, p % HOT, 1]
+            K[p] = ring[:, p % H, 0]
+            V[p] = ring[:, p % H, 1]
         else:
             i = p // 64
             if i not in blocks:
@@ -83,6 +84,38 @@ def test_brute_force_tiny(hkv, g, qbits):
             assert np.all(out[b] == 0) and np.all(np.isneginf(lse[b]))
             continue
         K, V = _dense_kv(oc, b, L)
+        o2, l2 = _brute(q[b], K, V, scale, g)
+        assert np.abs(out[b] - o2).max() < 1e-12
+        assert np.abs(lse[b] - l2).max() < 1e-12
+
+
+@pytest.mark.parametrize("hot", [16, 64, 128])
+def test_brute_force_other_hot_sizes(hot):
+    """hot_tokens 16 / 64 / 128 (the contract's other powers of two): the
+    newest `hot` tokens stay FP16, the rest is sealed into blocks."""
+    rng = np.random.default_rng(200 + hot)
+    total = np.array([300, 1, hot - 1, hot, hot + 1, hot + 64, 0])
+    B, hkv, g = len(total), 2, 4
+    oc = oracle.OracleCache(B, hkv, hkv * g, max_blocks_per_seq=5, hot=hot)
+    ks, vs = _fill(oc, rng, total, hkv)
+    q = rng.standard_normal((B, hkv * g, D)).astype(np.float16)
+    scale = 1.0 / np.sqrt(D)
+    out, lse = oc.decode(q, scale, nthreads=2)
+    for b in range(B):
+        L = int(total[b])
+        if L == 0:
+            assert np.all(out[b] == 0) and np.all(np.isneginf(lse[b]))
+            continue
+        # the hot ring holds exactly the newest min(L, hot) inputs
+        ring = oc.ring(b)
+        for p in range(max(0, L - hot), L):
+            assert np.array_equal(ring[:, p % hot, 0], ks[b][p]) and np.array_equal(ring[:, p % hot, 1], vs[b][p])
+        # sealed blocks: one per started 64 tokens of the cold range
+        nb = (max(0, L - hot) + 63) // 64
+        assert [oc.get_block(b, i)[0] != 0 for i in range(5)] == [i < nb for i in range(5)]
+        K, V = _dense_kv(oc, b, L)
+        if L <= hot:  # nothing quantized: plain attention on the inputs
+            assert np.array_equal(K, ks[b].astype(np.float64)) and np.array_equal(V, vs[b].astype(np.float64))
         o2, l2 = _brute(q[b], K, V, scale, g)
         assert np.abs(out[b] - o2).max() < 1e-12
         assert np.abs(lse[b] - l2).max() < 1e-12
