@@ -58,6 +58,10 @@ def _load():
     lib.ora_len.restype = ctypes.c_int32
     lib.ora_append.argtypes = [P, P, i32, P, P]
     lib.ora_decode.argtypes = [P, P, ctypes.c_double, P, i32, P, P, i32]
+    lib.ora_decode_topk.argtypes = [P, P, ctypes.c_double, i32, P, i32, P, P, i32]
+    lib.ora_decode_topk.restype = ctypes.c_int32
+    lib.ora_sparse_top_k.argtypes = [ctypes.c_long]
+    lib.ora_sparse_top_k.restype = ctypes.c_int32
     lib.ora_combine.argtypes = [i32, i32, i32, P, P, P, P]
     lib.ora_get_block.argtypes = [P, i32, i32, P, P]
     lib.ora_get_block_fp16.argtypes = [P, i32, i32, P]
@@ -137,10 +141,12 @@ class OracleCache:
     def lens(self):
         return np.array([self._lib.ora_len(self._h, b) for b in range(self.batch)], np.int32)
 
-    def decode(self, q, softmax_scale, pairs=None, nthreads=None):
+    def decode(self, q, softmax_scale, pairs=None, nthreads=None, top_k=None):
         """q: float16 [batch][hq][d].  Returns (out float64 [batch][hq][d],
         lse float64 [batch][hq]); with `pairs` ([(b, h), ...]) only those rows
-        are computed and the others are NaN."""
+        are computed and the others are NaN.  top_k: sparse L2 blocks (each
+        head attends only the top_k of its INT4-block tokens, see
+        ora_decode_topk); None = dense."""
         qq = _c(q, np.float16)
         out = np.full((self.batch, self.hq, self.d), np.nan)
         lse = np.full((self.batch, self.hq), np.nan)
@@ -150,9 +156,11 @@ class OracleCache:
             pp = _c(np.asarray(pairs, np.int32).reshape(-1, 2), np.int32)
             npairs = pp.shape[0]
         nt = nthreads or os.cpu_count() or 1
-        self._lib.ora_decode(self._h, _ptr(qq.view(np.uint16)), float(softmax_scale),
-                             None if pp is None else _ptr(pp), npairs,
-                             _ptr(out), _ptr(lse), nt)
+        rc = self._lib.ora_decode_topk(self._h, _ptr(qq.view(np.uint16)), float(softmax_scale),
+                                       -1 if top_k is None else int(top_k),
+                                       None if pp is None else _ptr(pp), npairs, _ptr(out), _ptr(lse), nt)
+        if rc != 0:
+            raise MemoryError("oracle decode failed (rc=%d)" % rc)
         return out, lse
 
     def get_block(self, b, i):
@@ -190,6 +198,11 @@ class OracleCache:
         if rc != 0:
             raise ValueError("oracle export failed (rc=%d)" % rc)
         return dict(cold=cold, scales=sc, hot=hot.view(np.float16), seq_lens=sl)
+
+
+def sparse_top_k(context_length):
+    """The page's sparse_top_k rule (see ora_sparse_top_k)."""
+    return int(_load().ora_sparse_top_k(int(context_length)))
 
 
 def migration_threshold_ms(lens):

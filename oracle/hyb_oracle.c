@@ -25,6 +25,17 @@
  *     layout fixed).
  *   - quantization_bits 0 (section 5.2: quantization switched off, the cold
  *     zone kept in FP16): sealed tokens keep their FP16 values in the block.
+ *   - Sparse "L2" blocks (section 2.2: the L2 cold blocks keep only the KV of
+ *     the top-k attention scores; section 5.3: sparse_top_k, default 32, and
+ *     the rule min(128, context_length / 256)): in ora_decode_topk each query
+ *     head attends, of the tokens in its sequence's INT4 blocks, only the
+ *     top_k with the largest scores (ties: the older position first), plus
+ *     every other token.  The score that decides the selection is taken in
+ *     the same FP32 / integer arithmetic as the GPU kernel (a decision that
+ *     picks a discrete set must be made in one precision on both sides):
+ *     q in 16-bit fixed point per head, qi = clamp(rint(q * (32767 / max|q|))),
+ *     key = (float)(sum_c qi_c * code_c) * K-scale.  The attention over the
+ *     selected set is exact FP64 as below.
  *   - Attention (section 4.2, steps 3-5): one softmax over hot and cold keys
  *     together, on the dequantized cold values (code * scale) and the FP16 hot
  *     values, evaluated here in FP64.  The page's torch.cat of two separately
@@ -365,13 +376,67 @@ static double kv_value(const ora_cache *c, int b, int h, int kv, int p, int ch) 
  * out: [batch][hq][d], lse: [batch][hq] (natural log); entries of pairs not
  * listed are left untouched.  An empty sequence gives out = 0, lse = -inf.
  */
-int ora_decode(const ora_cache *c, const uint16_t *q, double softmax_scale,
-               const int32_t *pairs, int npairs, double *out, double *lse,
-               int nthreads) {
+/* Tokens of sequence b held in its INT4 ("L2") blocks: the oldest ones, in
+ * logical blocks below n_int4[b] (every cold block when quant_bits is 4; none
+ * with FP16 blocks). */
+static int l2_tokens(const ora_cache *c, int b) {
+  const int L = c->len[b];
+  const int cold = L > c->hot ? L - c->hot : 0;
+  long n4 = c->quant_bits == 4 ? c->max_blocks : c->quant_bits == 8 ? c->n_int4[b] : 0;
+  const long cap = n4 * c->block;
+  return cold < cap ? cold : (int)cap;
+}
+
+/* Selection key of L2 position p for a query head (see the header):
+ * qi: the head's q in 16-bit fixed point. */
+static float l2_key(const ora_cache *c, int b, int hk, int p, const int32_t *qi) {
+  const int i = p / c->block;
+  const size_t bi = (size_t)b * c->max_blocks + i;
+  const int8_t *codes = c->codes[bi] + (((size_t)hk * 2 + 0) * c->block + (p - i * c->block)) * c->d;
+  int64_t dot = 0;
+  for (int ch = 0; ch < c->d; ch++) dot += (int64_t)qi[ch] * codes[ch];
+  const float sk = c->scale[bi][(size_t)hk * 2 + 0];
+  return (float)dot * sk;
+}
+
+static void q_fixed16(const uint16_t *qh, int d, int32_t *qi) {
+  float amax = 0.0f;
+  for (int ch = 0; ch < d; ch++) {
+    const float a = fabsf(half_to_float(qh[ch]));
+    if (a > amax) amax = a;
+  }
+  const float inv = amax > 0.0f ? 32767.0f / amax : 0.0f;
+  for (int ch = 0; ch < d; ch++) {
+    const float t = half_to_float(qh[ch]) * inv;
+    long v = lrintf(t);
+    if (v > 32767) v = 32767;
+    if (v < -32767) v = -32767;
+    qi[ch] = (int32_t)v;
+  }
+}
+
+typedef struct { float key; int pos; } l2_cand;
+
+/* Order: larger key first, then the older position. */
+static int cand_cmp(const void *x, const void *y) {
+  const l2_cand *a = (const l2_cand *)x, *b = (const l2_cand *)y;
+  if (a->key != b->key) return a->key > b->key ? -1 : 1;
+  return a->pos - b->pos;
+}
+
+/*
+ * Decode attention: out[b][h][:] and lse[b][h] (natural log) for every
+ * (sequence, query head), or only the npairs (b, h) pairs given.  top_k < 0:
+ * dense (every token).  top_k >= 0: of the L2 tokens only the top_k
+ * selected as the header describes (all of them when there are no more).
+ */
+int ora_decode_topk(const ora_cache *c, const uint16_t *q, double softmax_scale, int top_k,
+                    const int32_t *pairs, int npairs, double *out, double *lse, int nthreads) {
   const int d = c->d, g = c->hq / c->hkv;
   const int total = pairs ? npairs : c->batch * c->hq;
   if (nthreads < 1) nthreads = 1;
-#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads) reduction(| : bad)
   for (int w = 0; w < total; w++) {
     const int b = pairs ? pairs[2 * w] : w / c->hq;
     const int hh = pairs ? pairs[2 * w + 1] : w % c->hq;
@@ -383,30 +448,67 @@ int ora_decode(const ora_cache *c, const uint16_t *q, double softmax_scale,
       lse[(size_t)b * c->hq + hh] = -INFINITY;
       continue;
     }
-    double *z = (double *)malloc(sizeof(double) * L);
     const uint16_t *qh = q + ((size_t)b * c->hq + hh) * d;
+    /* the positions attended */
+    int *pos = (int *)malloc(sizeof(int) * L);
+    int n = 0;
+    const int n2 = top_k < 0 ? 0 : l2_tokens(c, b);
+    if (n2 > 0) {
+      int32_t *qi = (int32_t *)malloc(sizeof(int32_t) * d);
+      l2_cand *cand = (l2_cand *)malloc(sizeof(l2_cand) * n2);
+      if (!qi || !cand || !pos) {
+        bad = 1;
+        free(qi); free(cand); free(pos);
+        continue;
+      }
+      q_fixed16(qh, d, qi);
+      for (int p = 0; p < n2; p++) {
+        cand[p].key = l2_key(c, b, hk, p, qi);
+        cand[p].pos = p;
+      }
+      qsort(cand, n2, sizeof(l2_cand), cand_cmp);
+      const int keep = top_k < n2 ? top_k : n2;
+      for (int t = 0; t < keep; t++) pos[n++] = cand[t].pos;
+      free(qi);
+      free(cand);
+    }
+    for (int p = n2; p < L; p++) pos[n++] = p;
+    double *z = (double *)malloc(sizeof(double) * (n > 0 ? n : 1));
     double m = -INFINITY;
-    for (int j = 0; j < L; j++) {
+    for (int j = 0; j < n; j++) {
       double acc = 0.0;
       for (int ch = 0; ch < d; ch++)
-        acc += (double)half_to_float(qh[ch]) * kv_value(c, b, hk, 0, j, ch);
+        acc += (double)half_to_float(qh[ch]) * kv_value(c, b, hk, 0, pos[j], ch);
       z[j] = softmax_scale * acc;
       if (z[j] > m) m = z[j];
     }
     double l = 0.0;
-    for (int j = 0; j < L; j++) {
+    for (int j = 0; j < n; j++) {
       z[j] = exp(z[j] - m);
       l += z[j];
     }
     for (int ch = 0; ch < d; ch++) {
       double acc = 0.0;
-      for (int j = 0; j < L; j++) acc += z[j] * kv_value(c, b, hk, 1, j, ch);
-      o[ch] = acc / l;
+      for (int j = 0; j < n; j++) acc += z[j] * kv_value(c, b, hk, 1, pos[j], ch);
+      o[ch] = n > 0 ? acc / l : 0.0;
     }
-    lse[(size_t)b * c->hq + hh] = m + log(l);
+    lse[(size_t)b * c->hq + hh] = n > 0 ? m + log(l) : -INFINITY;
     free(z);
+    free(pos);
   }
-  return ORA_OK;
+  return bad ? ORA_ERR_NOMEM : ORA_OK;
+}
+
+int ora_decode(const ora_cache *c, const uint16_t *q, double softmax_scale,
+               const int32_t *pairs, int npairs, double *out, double *lse,
+               int nthreads) {
+  return ora_decode_topk(c, q, softmax_scale, -1, pairs, npairs, out, lse, nthreads);
+}
+
+/* The page's rule for sparse_top_k (section 5.3): min(128, context_length / 256). */
+int ora_sparse_top_k(long context_length) {
+  const long k = context_length / 256;
+  return k < 128 ? (int)k : 128;
 }
 
 /*
