@@ -54,6 +54,10 @@ def parse():
                    help="cold blocks: 8 (INT8, the default), 4 (all INT4) or 0 (FP16, quantization off)")
     p.add_argument("--hot-tokens", type=int, default=32, choices=[16, 32, 64, 128],
                    help="hot-zone tokens (32, the default, is the page's value)")
+    p.add_argument("--sparse-top-k", type=int, default=None,
+                   help="time hyb_decode_attn_sparse with this top_k (-1: the page's rule min(128, L // 256)) "
+                        "against the dense hyb_decode_attn on the same cache (workload default 4, the older "
+                        "half of every sequence's cold blocks INT4)")
     p.add_argument("--lean", action="store_true",
                    help="profiling run: no state restore, L2 flush, e2e or CPU baseline")
     return p.parse_args()
@@ -479,6 +483,76 @@ def run_migrate(args):
     }
 
 
+def run_sparse(args):
+    """Sparse L2 attention on one GPU: hyb_decode_attn_sparse and the dense
+    hyb_decode_attn on the same cache, alternating, L2 flushed before each."""
+    import numpy as np
+    import torch
+    from int8_paged_kv_hybrid_b200 import hyb_sparse_top_k, synth
+    wl = args.workload if args.workload != WORKLOAD else 4
+    w = synth.make_workload(wl)
+    if w.n_int4 is None:
+        w.n_int4 = (w.cold_blocks() // 2).astype(np.int32)
+    cache, n_last, k_last, v_last, q = build_gpu_state(w, torch)
+    cache.append(torch.from_numpy(n_last).cuda(), torch.from_numpy(k_last).cuda(), torch.from_numpy(v_last).cuda())
+    L = int(w.lens.max())
+    top_k = hyb_sparse_top_k(L) if args.sparse_top_k < 0 else args.sparse_top_k
+    split = args.split or w.split_tokens
+    qd = torch.from_numpy(q).cuda()
+    out = torch.empty((w.batch, w.num_q_heads, 128), dtype=torch.float16, device="cuda")
+    lse = torch.empty((w.batch, w.num_q_heads), dtype=torch.float32, device="cuda")
+    ws_s = cache.sparse_workspace(L, split)
+    ws_d = cache.workspace(L, split)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    clocks = ClockSampler(0)
+    times = {"sparse": [], "dense": []}
+    for i in range(2 * (args.warmup + args.steps)):
+        kind = "sparse" if i % 2 == 0 else "dense"
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        if kind == "sparse":
+            cache.decode_sparse(qd, w.softmax_scale, L, top_k, split, out=out, lse=lse, workspace=ws_s)
+        else:
+            cache.decode(qd, w.softmax_scale, L, split, out=out, lse=lse, workspace=ws_d)
+        e1.record()
+        if i == 2 * args.warmup:
+            torch.cuda.synchronize()
+            clocks.mark()
+        if i >= 2 * args.warmup:
+            times[kind].append((e0, e1))
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    assert cache.status() == 0 and torch.isfinite(out.float()).all()
+    ms = {k: sum(a.elapsed_time(b) for a, b in v) / len(v) for k, v in times.items()}
+    # L2 tokens per sequence and the bytes the sparse call must move: the
+    # dense bytes minus the L2 V codes (64 B per token and kv head), plus the
+    # selected tokens' V codes (64 B per token and query head)
+    nb = w.cold_blocks()
+    l2 = np.minimum(np.maximum(w.lens - w.hot_tokens, 0), w.n_int4 * 64)
+    dense_b = synth.kv_bytes(w)
+    sel = np.minimum(l2, top_k)
+    sparse_b = dense_b - int(l2.sum()) * w.num_kv_heads * 64 + int(sel.sum()) * w.num_q_heads * 64
+    peak, peak_kind = measured_peaks()
+    gbs = sparse_b / (ms["sparse"] * 1e-3) / 1e9
+    return {
+        "metric": "hyb_decode_attn_sparse (top-k of the INT4 L2 tokens) GB/s of the bytes the sparse pass must move",
+        "value": round(gbs, 1), "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms["sparse"], 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4", "data": "synthetic",
+        "config": dict(workload_config(w, split, 0), top_k=top_k,
+                       l2="older half of every sequence's cold blocks INT4: %d L2 tokens in all" % int(l2.sum())),
+        "dense": {"ms_per_step": round(ms["dense"], 5), "kv_bytes": dense_b,
+                  "GB/s": round(dense_b / (ms["dense"] * 1e-3) / 1e9, 1)},
+        "sparse_bytes": sparse_b,
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(gbs / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                     "kernel": "decode_kernel (l2_skip) + l2_score_kernel + l2_topk_kernel"},
+        "gpu_launches": 3 * args.steps + args.steps,
+        "clocks": clk,
+    }
+
+
 def oracle_step_rate(w, steps, warmup, budget_s=None, qbits=8):
     """Time the CPU oracle (as it stands) on the same workload: per step the
     1-token append plus FP64 attention of every (sequence, head).  The state
@@ -547,6 +621,10 @@ def main():
     if args.migrate:
         if rank == 0:
             print(json.dumps(run_migrate(args)))
+        return 0
+    if args.sparse_top_k is not None:
+        if rank == 0:
+            print(json.dumps(run_sparse(args)))
         return 0
     if world > 1:
         import datetime

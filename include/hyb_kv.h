@@ -258,6 +258,43 @@ int hyb_decode_attn(const hyb_cache_desc *desc, const void *q, float softmax_sca
                     size_t workspace_bytes, void *out, float *lse_out, hyb_stream_t stream);
 
 /*
+ * Sparse L2 decode attention ([hybrid_v2 page] 2.2: the L2 cold blocks keep
+ * only the KV of the top-k attention scores; 5.3: sparse_top_k).  As
+ * hyb_decode_attn, except that of the tokens a sequence holds in its INT4
+ * ("L2") blocks -- logical blocks below n_int4_blocks[b] (quant_bits 8), every
+ * cold block (quant_bits 4) -- each query head attends only the top_k with
+ * the largest selection keys, plus every other token:
+ *   key_j = (float)(sum_c qi_c * Kcode_j,c) * Kscale_j   (FP32, one rounding
+ *           per operation; -0 counts as +0),
+ *   qi_c  = clamp(rint(q_c * (32767 / max_c |q_c|)), -32767, 32767),
+ * the head's q in 16-bit fixed point; equal keys keep the older position.
+ * All L2 tokens are attended when there are at most top_k of them; top_k 0
+ * attends none.  Accuracy as hyb_decode_attn.
+ *   top_k      0 .. 1024 (the page's default is 32; see hyb_sparse_top_k).
+ *   workspace  at least hyb_decode_sparse_workspace_bytes() bytes, 16-byte
+ *              aligned, zero-filled before its first use (its leading part is
+ *              the dense pass's workspace); holds the keys of every L2 token.
+ * Launches: the decode kernel over everything but the L2 blocks, a scoring
+ * kernel over the L2 blocks' INT4 K tiles, and a top-k kernel per (sequence,
+ * query head) that selects, attends the selected tokens' V and merges with
+ * the dense result by log-sum-exp.
+ * Returns as hyb_decode_attn, plus HYB_ERR_UNSUPPORTED for quant_bits 0 (FP16
+ * cold blocks have no L2 tier) and HYB_ERR_INVALID_VALUE for top_k outside
+ * 0..1024.
+ */
+int hyb_decode_attn_sparse(const hyb_cache_desc *desc, const void *q, float softmax_scale,
+                           int32_t max_seq_len, int32_t split_tokens, int32_t top_k, void *workspace,
+                           size_t workspace_bytes, void *out, float *lse_out, hyb_stream_t stream);
+
+/* Bytes of workspace hyb_decode_attn_sparse needs (0 with an invalid descriptor). */
+size_t hyb_decode_sparse_workspace_bytes(const hyb_cache_desc *desc, int32_t max_seq_len,
+                                         int32_t split_tokens);
+
+/* The page's sparse_top_k rule ([hybrid_v2 page] 5.3): min(128,
+ * context_length / 256) (0 for a negative length).  Host only. */
+int hyb_sparse_top_k(int64_t context_length);
+
+/*
  * hyb_decode_attn without a caller-provided workspace (the pages have no
  * counterpart: this is an integration convenience).  For callers that cannot
  * allocate device memory when they run attention -- code handed a fixed

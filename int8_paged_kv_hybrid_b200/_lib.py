@@ -34,6 +34,7 @@ EXPORTED = (
     "hyb_read_status", "hyb_strerror",
     "hyb_last_cuda_error", "hyb_version", "hyb_decode_attn_noalloc", "hyb_noalloc_scratch_limit",
     "hyb_kv_migrate", "hyb_migration_threshold_ms", "hyb_migration_decision",
+    "hyb_decode_attn_sparse", "hyb_decode_sparse_workspace_bytes", "hyb_sparse_top_k",
 )
 
 
@@ -86,6 +87,11 @@ def load(path: str = LIB_PATH):
     lib.hyb_decode_workspace_bytes.argtypes = [D, i32, i32]
     lib.hyb_decode_workspace_bytes.restype = sz
     lib.hyb_decode_attn.argtypes = [D, P, ctypes.c_float, i32, i32, P, sz, P, P, P]
+    lib.hyb_decode_attn_sparse.argtypes = [D, P, ctypes.c_float, i32, i32, i32, P, sz, P, P, P]
+    lib.hyb_decode_sparse_workspace_bytes.argtypes = [D, i32, i32]
+    lib.hyb_decode_sparse_workspace_bytes.restype = sz
+    lib.hyb_sparse_top_k.argtypes = [ctypes.c_int64]
+    lib.hyb_sparse_top_k.restype = i32
     lib.hyb_decode_step.argtypes = [D, P, P, P, P, ctypes.c_float, i32, i32, P, sz, P, P, P]
     lib.hyb_decode_step_workspace_bytes.argtypes = [D, i32, i32]
     lib.hyb_decode_step_workspace_bytes.restype = sz
@@ -155,6 +161,22 @@ def hyb_decode_attn(desc, q, softmax_scale, max_seq_len, split_tokens, workspace
     _check(load().hyb_decode_attn(ctypes.byref(desc), _ptr(q), float(softmax_scale), int(max_seq_len),
                                   int(split_tokens), _ptr(workspace), ws_bytes, _ptr(out),
                                   _ptr(lse_out), _stream(stream)), "hyb_decode_attn")
+
+
+def hyb_decode_sparse_workspace_bytes(desc, max_seq_len, split_tokens=0) -> int:
+    return int(load().hyb_decode_sparse_workspace_bytes(ctypes.byref(desc), int(max_seq_len), int(split_tokens)))
+
+
+def hyb_decode_attn_sparse(desc, q, softmax_scale, max_seq_len, split_tokens, top_k, workspace, out,
+                           lse_out=None, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().hyb_decode_attn_sparse(ctypes.byref(desc), _ptr(q), float(softmax_scale), int(max_seq_len),
+                                         int(split_tokens), int(top_k), _ptr(workspace), ws_bytes, _ptr(out),
+                                         _ptr(lse_out), _stream(stream)), "hyb_decode_attn_sparse")
+
+
+def hyb_sparse_top_k(context_length) -> int:
+    return int(load().hyb_sparse_top_k(int(context_length)))
 
 
 def hyb_decode_step_workspace_bytes(desc, max_seq_len, split_tokens=0) -> int:

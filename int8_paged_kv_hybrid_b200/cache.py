@@ -100,6 +100,25 @@ class HybridKVCache:
                              out, lse, stream)
         return out
 
+    def sparse_workspace(self, max_seq_len, split_tokens=0):
+        import torch
+        n = _lib.hyb_decode_sparse_workspace_bytes(self.desc, max_seq_len, split_tokens)
+        return torch.zeros(max(n, 16), dtype=torch.uint8, device=self.device)
+
+    def decode_sparse(self, q, softmax_scale, max_seq_len, top_k, split_tokens=0, out=None, lse=None,
+                      workspace=None, stream=None):
+        """As decode, but each query head attends only the top_k of the tokens
+        in its sequence's INT4 (L2) blocks (hyb_decode_attn_sparse)."""
+        import torch
+        assert q.is_contiguous()
+        if out is None:
+            out = torch.empty((self.batch, self.hq, HEAD_DIM), dtype=torch.float16, device=self.device)
+        if workspace is None:
+            workspace = self.sparse_workspace(max_seq_len, split_tokens)
+        _lib.hyb_decode_attn_sparse(self.desc, q, softmax_scale, max_seq_len, split_tokens, top_k, workspace,
+                                    out, lse, stream)
+        return out
+
     def step_workspace(self, max_seq_len, split_tokens=0):
         import torch
         n = _lib.hyb_decode_step_workspace_bytes(self.desc, max_seq_len, split_tokens)

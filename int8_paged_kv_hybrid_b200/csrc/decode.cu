@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
       const int kb = fp16 ? k >> 1 : k;
       const int phys = sm.phys[kb];
       const int nrow = fp16 ? min(kItemRows, Lc - (i0 + kb) * kBlock - (k & 1) * kItemRows) : 1;
-      if (phys < 0 || nrow <= 0) {
+      if (phys < 0 || nrow <= 0 || (!fp16 && a.l2_skip && i0 + kb < n_int4_b)) {
         mbar_arrive(&sm.full[st]);
         return;
       }
@@ -301,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
     if (ok && !fp16 && k < ncold) {
       // ---------------- cold block ----------------
       const int i = i0 + k;
-      const int nvalid = sm.phys[k] < 0 ? 0 : min(kBlock, Lc - i * kBlock);
+      const int nvalid = (sm.phys[k] < 0 || (a.l2_skip && i < n_int4_b)) ? 0 : min(kBlock, Lc - i * kBlock);
       const int nv = nvalid - 16 * warp;
       const bool int4 = i < n_int4_b;
       const float2 sc = sm.scl[k];

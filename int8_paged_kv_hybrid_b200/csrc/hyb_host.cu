@@ -258,7 +258,7 @@ size_t hyb_decode_workspace_bytes(const hyb_cache_desc *d, int32_t max_seq_len, 
 static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_scale, int32_t max_seq_len,
                          int32_t split_tokens, void *workspace, size_t workspace_bytes, void *out,
                          float *lse_out, hyb_stream_t stream, const int32_t *n_new, const void *k_new,
-                         const void *v_new) {
+                         const void *v_new, bool l2_skip = false) {
   Plan pl;
   const int rc = make_plan(d, max_seq_len, split_tokens, &pl);
   if (rc != HYB_OK) return rc;
@@ -305,6 +305,7 @@ static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_s
   a.k_new = static_cast<const __half *>(k_new);
   a.v_new = static_cast<const __half *>(v_new);
   a.seq_cnt = step ? reinterpret_cast<int32_t *>(ws + wl.seq_cnt) : nullptr;
+  a.l2_skip = l2_skip ? 1 : 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int group = d->num_q_heads / d->num_kv_heads;
   const cudaError_t e = hyb::launch_decode(a, group, d->batch, pl.cluster, s);
@@ -317,6 +318,79 @@ int hyb_decode_attn(const hyb_cache_desc *d, const void *q, float softmax_scale,
                     float *lse_out, hyb_stream_t stream) {
   return decode_launch(d, q, softmax_scale, max_seq_len, split_tokens, workspace, workspace_bytes, out,
                        lse_out, stream, nullptr, nullptr, nullptr);
+}
+
+// Workspace of hyb_decode_attn_sparse: the dense pass's workspace, then a
+// log-sum-exp row per (sequence, query head), then the selection keys
+// [batch][Hq][max_l2], max_l2 = the cold tokens of a max_seq_len sequence.
+struct SparseWs {
+  size_t dense, lse, keys, total;
+  int max_l2;
+};
+
+static int sparse_ws(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens, SparseWs *w) {
+  Plan pl;
+  const int rc = make_plan(d, max_seq_len, split_tokens, &pl);
+  if (rc != HYB_OK) return rc;
+  const size_t rows = static_cast<size_t>(d->batch) * d->num_q_heads;
+  const long long cold = static_cast<long long>(max_seq_len) - d->hot_tokens;
+  w->max_l2 = cold > 0 ? static_cast<int>((cold + hyb::kBlock - 1) / hyb::kBlock * hyb::kBlock) : 0;
+  w->dense = ws_layout(d, pl, false).total;
+  w->lse = round_up(w->dense, kWsAlign);
+  w->keys = w->lse + round_up(rows * sizeof(float), kWsAlign);
+  w->total = w->keys + round_up(rows * static_cast<size_t>(w->max_l2) * sizeof(float), kWsAlign);
+  return HYB_OK;
+}
+
+size_t hyb_decode_sparse_workspace_bytes(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens) {
+  SparseWs w;
+  if (sparse_ws(d, max_seq_len, split_tokens, &w) != HYB_OK) return 0;
+  return w.total;
+}
+
+int hyb_decode_attn_sparse(const hyb_cache_desc *d, const void *q, float softmax_scale, int32_t max_seq_len,
+                           int32_t split_tokens, int32_t top_k, void *workspace, size_t workspace_bytes,
+                           void *out, float *lse_out, hyb_stream_t stream) {
+  SparseWs w;
+  const int rc = sparse_ws(d, max_seq_len, split_tokens, &w);
+  if (rc != HYB_OK) return rc;
+  if (d->quant_bits == 0) return HYB_ERR_UNSUPPORTED;  // FP16 blocks: no L2 tier
+  if (top_k < 0 || top_k > hyb::kMaxTopK) return HYB_ERR_INVALID_VALUE;
+  if (!workspace || workspace_bytes < w.total || !aligned(workspace, 16)) return HYB_ERR_WORKSPACE;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  float *lse = lse_out ? lse_out : reinterpret_cast<float *>(ws + w.lse);
+  const int r = decode_launch(d, q, softmax_scale, max_seq_len, split_tokens, workspace, w.dense, out, lse, stream,
+                              nullptr, nullptr, nullptr, true);
+  if (r != HYB_OK) return r;
+  hyb::SparseArgs a;
+  a.cold = static_cast<const uint8_t *>(d->cold);
+  a.scales = d->scales;
+  a.block_table = d->block_table;
+  a.seq_lens = d->seq_lens;
+  a.n_int4 = d->quant_bits == 8 ? d->n_int4_blocks : nullptr;
+  a.status = d->status;
+  a.q = static_cast<const __half *>(q);
+  a.keys = reinterpret_cast<float *>(ws + w.keys);
+  a.out = static_cast<__half *>(out);
+  a.lse = lse;
+  a.hkv = d->num_kv_heads;
+  a.hq = d->num_q_heads;
+  a.num_phys = d->num_phys_blocks;
+  a.max_blocks = d->max_blocks_per_seq;
+  a.quant_bits = d->quant_bits;
+  a.hot_tokens = d->hot_tokens;
+  a.max_l2 = w.max_l2;
+  a.top_k = top_k;
+  a.blocks_per_cta = 4;
+  a.qk_scale = softmax_scale * 1.4426950408889634f;
+  const cudaError_t e = hyb::launch_sparse_l2(a, d->batch, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HYB_OK : cuda_fail(e);
+}
+
+int hyb_sparse_top_k(int64_t context_length) {
+  if (context_length < 0) return 0;
+  const int64_t k = context_length / 256;
+  return k < 128 ? static_cast<int>(k) : 128;
 }
 
 size_t hyb_decode_step_workspace_bytes(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens) {

@@ -54,6 +54,9 @@ struct DecodeArgs {
   const __half *k_new;
   const __half *v_new;
   int32_t *seq_cnt;
+  // sparse L2 mode: the INT4 ("L2") blocks are left out of this pass (they
+  // are attended by the top-k kernels of sparse.cu)
+  int l2_skip;
 };
 
 struct MigrateArgs {
@@ -67,6 +70,25 @@ struct MigrateArgs {
   int hkv, num_phys, max_blocks, max_delta;
   int hot_tokens;             // hot-zone tokens
 };
+
+// Sparse L2 attention (top-k of the INT4-block tokens per query head).
+struct SparseArgs {
+  const uint8_t *cold;        // [num_phys][Hkv][2][8192]
+  const float *scales;        // [num_phys][Hkv][2]
+  const int32_t *block_table; // [batch][max_blocks]
+  const int32_t *seq_lens;    // [batch]
+  const int32_t *n_int4;      // [batch] or null
+  int32_t *status;
+  const __half *q;            // FP16 [batch][Hq][128]
+  float *keys;                // [batch][Hq][max_l2] selection keys (workspace)
+  __half *out;                // FP16 [batch][Hq][128]: the dense pass's result in, the merged result out
+  float *lse;                 // [batch][Hq]: the dense pass's log-sum-exp in, merged out (natural log)
+  int hkv, hq, num_phys, max_blocks, quant_bits, hot_tokens, max_l2, top_k, blocks_per_cta;
+  float qk_scale;             // softmax_scale * log2(e)
+};
+
+// Largest top_k of the sparse L2 mode (the selected positions live in shared memory).
+constexpr int kMaxTopK = 1024;
 
 struct CombineArgs {
   const float *o_part;        // [rows][n_splits][128]
@@ -83,6 +105,7 @@ cudaError_t launch_append(const AppendArgs &a, int batch, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream);
 cudaError_t launch_migrate(const MigrateArgs &a, int batch, cudaStream_t stream);
 cudaError_t launch_combine(const CombineArgs &a, int rows, cudaStream_t stream);
+cudaError_t launch_sparse_l2(const SparseArgs &a, int batch, cudaStream_t stream);
 int decode_max_split_blocks();
 int decode_ctas_per_sm(int group);
 int decode_max_cluster();

@@ -1,0 +1,307 @@
+// sparse.cu -- sparse L2 attention: of the tokens a sequence holds in its INT4
+// ("L2") cold blocks, each query head attends only the top_k with the
+// largest scores; the rest of the cache is attended densely by the decode
+// kernel (run with l2_skip), and the two softmax pieces are merged here.
+//
+// Method: web page "DeepSeek V4混合式KV Cache推理优化实战解析", section 2.2 (L2
+// cold blocks keep only the KV of the top-k attention scores) and section 5.3
+// (sparse_top_k: default 32, min(128, context_length / 256) for long
+// contexts).  Selection key of an L2 token for a query head: the exact
+// integer dot product of the head's q in 16-bit fixed point (the decode
+// kernel's quantize_q) with the token's INT4 K codes, times the block's K
+// scale, in FP32; equal keys keep the older position.
+//
+//  l2_score_kernel   grid (chunks of L2 blocks, Hkv, batch): the keys of every
+//                    L2 token for the G query heads of a kv head, from the
+//                    INT4 K tiles only (4 KB per block).
+//  l2_topk_kernel    grid (Hq, batch): radix select of the top_k keys (four
+//                    8-bit passes over histograms in shared memory), ordered
+//                    compaction of the selected positions, softmax over them
+//                    in FP32 with their INT4 V codes, and the log-sum-exp
+//                    merge with the dense pass's output and log-sum-exp.
+#include "kernels.cuh"
+
+namespace hyb {
+
+constexpr int kScoreThreads = 128;
+constexpr int kTopkThreads = 256;
+constexpr float kLn2f = 0.6931471805599453f;
+
+// Tokens of sequence b held in its INT4 blocks (the oldest ones), or 0 when
+// its length is out of range (the dense pass reports that).
+__device__ __forceinline__ int l2_count(const SparseArgs &a, int b) {
+  const int L = a.seq_lens[b];
+  if (L < 0) return 0;
+  const int Lc = max(0, L - a.hot_tokens);
+  const long long n4 = a.quant_bits == 4 ? a.max_blocks : (a.n_int4 ? a.n_int4[b] : 0);
+  const long long n = min(static_cast<long long>(Lc), max(0LL, n4) * kBlock);
+  return n > a.max_l2 ? -1 : static_cast<int>(n);
+}
+
+// Monotone map of a finite float to uint32 (larger float, larger word).
+__device__ __forceinline__ uint32_t key_order(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ int sext4(uint32_t nib) { return static_cast<int>(nib << 28) >> 28; }
+
+__global__ void __launch_bounds__(kScoreThreads) l2_score_kernel(const SparseArgs a) {
+  const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = a.hq / a.hkv;
+  const int n = l2_count(a, b);
+  if (n <= 0) return;
+  const int nb = (n + kBlock - 1) / kBlock;
+  const int blk0 = chunk * a.blocks_per_cta;
+  if (blk0 >= nb) return;
+
+  // q of the G heads in 16-bit fixed point, as the decode kernel makes it
+  __shared__ alignas(16) int16_t qi[8][kDim];
+  for (int j = warp; j < G; j += kScoreThreads / 32) {
+    const __half *qh = a.q + ((size_t)b * a.hq + h * G + j) * kDim;
+    float qv[4];
+    float amax = 0.f;
+#pragma unroll
+    for (int t = 0; t < 4; t++) {
+      qv[t] = __half2float(qh[lane + 32 * t]);
+      amax = fmaxf(amax, fabsf(qv[t]));
+    }
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+    const float inv = amax > 0.f ? 32767.f / amax : 0.f;
+#pragma unroll
+    for (int t = 0; t < 4; t++) {
+      const int v = __float2int_rn(qv[t] * inv);
+      qi[j][lane + 32 * t] = static_cast<int16_t>(max(-32767, min(32767, v)));
+    }
+  }
+  __syncthreads();
+
+  // thread: token tok of the block, channels 64*half .. 64*half + 63
+  const int tok = tid >> 1, half = tid & 1;
+  const int blk1 = min(nb, blk0 + a.blocks_per_cta);
+  for (int blk = blk0; blk < blk1; blk++) {
+    const int phys = a.block_table[(size_t)b * a.max_blocks + blk];
+    const bool okp = phys >= 0 && phys < a.num_phys;
+    if (!okp && tid == 0) set_status(a.status, HYB_STATUS_BAD_BLOCK);
+    int dot[8];
+#pragma unroll
+    for (int g = 0; g < 8; g++) dot[g] = 0;
+    if (okp) {
+      // INT4 K: 64 bytes per token, word w holds channels 8w..8w+7 (byte i:
+      // channel 8w+i in the low nibble, 8w+4+i in the high nibble)
+      const uint8_t *ktile = a.cold + ((size_t)phys * a.hkv + h) * kTilePairBytes;
+      const uint32_t *kp = reinterpret_cast<const uint32_t *>(ktile + tok * 64 + half * 32);
+#pragma unroll 1
+      for (int w = 0; w < 8; w++) {
+        const uint32_t word = kp[w];
+        const int cb = 64 * half + 8 * w;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+          const int lo = sext4((word >> (8 * i)) & 0xfu);
+          const int hi = sext4((word >> (8 * i + 4)) & 0xfu);
+#pragma unroll
+          for (int g = 0; g < 8; g++)
+            if (g < G) dot[g] += static_cast<int>(qi[g][cb + i]) * lo + static_cast<int>(qi[g][cb + 4 + i]) * hi;
+        }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < 8; g++) dot[g] += __shfl_xor_sync(0xffffffffu, dot[g], 1);
+    const int pos = blk * kBlock + tok;
+    if (half == 0 && pos < n) {
+      const float sk = okp ? a.scales[((size_t)phys * a.hkv + h) * 2] : 0.f;
+#pragma unroll
+      for (int g = 0; g < 8; g++) {
+        if (g < G) {
+          float key = okp ? __fmul_rn(__int2float_rn(dot[g]), sk) : -INFINITY;
+          if (key == 0.f) key = 0.f;  // -0 and +0 are one key
+          a.keys[((size_t)b * a.hq + h * G + g) * a.max_l2 + pos] = key;
+        }
+      }
+    }
+  }
+}
+
+// Exclusive prefix count of `flag` over the CTA's threads in thread order;
+// *total gets the CTA's count.  Every thread calls it.
+__device__ __forceinline__ int cta_prefix(bool flag, int *s_warp, int tid, int *total) {
+  const int lane = tid & 31, warp = tid >> 5;
+  const unsigned bal = __ballot_sync(0xffffffffu, flag);
+  if (lane == 0) s_warp[warp] = __popc(bal);
+  __syncthreads();
+  int before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < kTopkThreads / 32; w++) {
+    const int c = s_warp[w];
+    before += w < warp ? c : 0;
+    all += c;
+  }
+  __syncthreads();
+  *total = all;
+  return before + __popc(bal & ((1u << lane) - 1u));
+}
+
+__device__ __forceinline__ float cta_reduce(float v, float *s_red, int tid, bool is_max) {
+  const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, v, m);
+    v = is_max ? fmaxf(v, o) : v + o;
+  }
+  if (lane == 0) s_red[warp] = v;
+  __syncthreads();
+  float r = s_red[0];
+#pragma unroll
+  for (int w = 1; w < kTopkThreads / 32; w++) r = is_max ? fmaxf(r, s_red[w]) : r + s_red[w];
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kTopkThreads) l2_topk_kernel(const SparseArgs a) {
+  const int hh = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x;
+  const int G = a.hq / a.hkv;
+  const int h = hh / G;
+  const int n = l2_count(a, b);
+  const int k = min(a.top_k, max(n, 0));
+  if (k <= 0) return;  // no L2 token attended: the dense result stands
+  const float *keys = a.keys + ((size_t)b * a.hq + hh) * a.max_l2;
+
+  __shared__ int hist[256];
+  __shared__ int s_warp[kTopkThreads / 32];
+  __shared__ float s_red[kTopkThreads / 32];
+  __shared__ int s_digit, s_need;
+  __shared__ int s_pos[kMaxTopK];
+  __shared__ float s_p[kMaxTopK];
+  __shared__ float s_sv[kMaxTopK];
+  __shared__ int s_vt[kMaxTopK];
+  __shared__ float s_acc[kDim];
+
+  // ---- the k-th largest key (exact), by four 8-bit radix passes ----
+  uint32_t thr = 0;
+  int need_eq = k;
+  if (k < n) {
+    uint32_t prefix = 0, mask = 0;
+    int need = k;
+    for (int pass = 0; pass < 4; pass++) {
+      const int shift = 24 - 8 * pass;
+      hist[tid] = 0;
+      __syncthreads();
+      for (int i = tid; i < n; i += kTopkThreads) {
+        const uint32_t u = key_order(keys[i]);
+        if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int above = 0, d = 255;
+        for (; d > 0; d--) {
+          if (above + hist[d] >= need) break;
+          above += hist[d];
+        }
+        s_digit = d;
+        s_need = need - above;
+      }
+      __syncthreads();
+      prefix |= static_cast<uint32_t>(s_digit) << shift;
+      mask |= 255u << shift;
+      need = s_need;
+      __syncthreads();
+    }
+    thr = prefix;
+    need_eq = need;
+  }
+
+  // ---- the selected positions, in position order ----
+  int base = 0, eq_seen = 0;
+  for (int c0 = 0; c0 < n; c0 += kTopkThreads) {
+    const int i = c0 + tid;
+    bool sel;
+    if (k < n) {
+      const uint32_t u = i < n ? key_order(keys[i]) : 0u;
+      const bool gt = i < n && u > thr;
+      const bool eq = i < n && u == thr;
+      int eq_tot;
+      const int eq_rank = cta_prefix(eq, s_warp, tid, &eq_tot);
+      sel = gt || (eq && eq_seen + eq_rank < need_eq);
+      eq_seen += eq_tot;
+    } else {
+      sel = i < n;
+    }
+    int sel_tot;
+    const int r = cta_prefix(sel, s_warp, tid, &sel_tot);
+    if (sel && base + r < kMaxTopK) s_pos[base + r] = i;
+    base += sel_tot;
+  }
+  const int ns = min(base, k);  // == k
+
+  // ---- softmax over the selected tokens (log2 domain, FP32) ----
+  const __half *qh = a.q + ((size_t)b * a.hq + hh) * kDim;
+  float qa = tid < kDim ? fabsf(__half2float(qh[tid])) : 0.f;
+  const float amax = cta_reduce(qa, s_red, tid, true);
+  const float coef = (amax / 32767.f) * a.qk_scale;
+  float zmax = -INFINITY;
+  for (int j = tid; j < ns; j += kTopkThreads) {
+    const int pos = s_pos[j];
+    const int phys = a.block_table[(size_t)b * a.max_blocks + pos / kBlock];
+    const bool okp = phys >= 0 && phys < a.num_phys;
+    const float z = keys[pos] * coef;
+    s_p[j] = z;
+    s_vt[j] = okp ? (phys * a.hkv + h) : -1;
+    s_sv[j] = okp ? a.scales[((size_t)phys * a.hkv + h) * 2 + 1] : 0.f;
+    zmax = fmaxf(zmax, z);
+  }
+  const float m = cta_reduce(zmax, s_red, tid, true);
+  float lsum = 0.f;
+  for (int j = tid; j < ns; j += kTopkThreads) {
+    const float p = exp2f(s_p[j] - m);
+    s_p[j] = p;
+    lsum += p;
+  }
+  const float l = cta_reduce(lsum, s_red, tid, false);
+
+  // ---- P.V over the selected tokens' INT4 V codes (channel c, two halves of the list) ----
+  const int c = tid & (kDim - 1), part = tid >> 7;
+  float acc = 0.f;
+  for (int j = part; j < ns; j += 2) {
+    const int vt = s_vt[j];
+    if (vt < 0) continue;
+    const int slot = s_pos[j] & (kBlock - 1);
+    const uint8_t *vtile = a.cold + (size_t)vt * kTilePairBytes + kTileBytes;
+    const uint8_t byte =
+        vtile[c * 32 + 8 * ((slot >> 4) ^ ((c >> 2) & 3)) + ((slot & 15) >> 3) * 4 + (slot & 3)];
+    const int code = sext4((slot & 4) ? (byte >> 4) : (byte & 0xfu));
+    acc = fmaf(s_p[j] * s_sv[j], static_cast<float>(code), acc);
+  }
+  if (part == 1) s_acc[c] = acc;
+  __syncthreads();
+  if (part == 0) {
+    acc += s_acc[c];
+    // merge with the dense pass (its output and natural-log log-sum-exp)
+    const size_t row = (size_t)b * a.hq + hh;
+    const float o_s = acc / l;
+    const float lse_s = (m + log2f(l)) * kLn2f;
+    const float lse_d = a.lse[row];
+    const float o_d = __half2float(a.out[row * kDim + c]);
+    const float M = fmaxf(lse_d, lse_s);
+    const float wd = lse_d == -INFINITY ? 0.f : expf(lse_d - M);
+    const float ws = expf(lse_s - M);
+    a.out[row * kDim + c] = __float2half_rn((wd * o_d + ws * o_s) / (wd + ws));
+    if (c == 0) a.lse[row] = M + logf(wd + ws);
+  }
+}
+
+cudaError_t launch_sparse_l2(const SparseArgs &a, int batch, cudaStream_t stream) {
+  if (a.max_l2 <= 0 || a.top_k <= 0) return cudaSuccess;
+  const int max_nb = (a.max_l2 + kBlock - 1) / kBlock;
+  dim3 g1((max_nb + a.blocks_per_cta - 1) / a.blocks_per_cta, a.hkv, batch);
+  l2_score_kernel<<<g1, kScoreThreads, 0, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dim3 g2(a.hq, batch);
+  l2_topk_kernel<<<g2, kTopkThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace hyb

@@ -162,6 +162,27 @@ def test_migration_policy_matches_fixture_and_oracle():
                 assert hk.hyb_migration_decision(iai, t, int4) == oracle.migration_decision(iai, t, int4)
 
 
+def test_sparse_argument_checks():
+    """hyb_decode_attn_sparse rejects bad arguments on the host, before any launch."""
+    lib = hk.load()
+    d = _desc(batch=4, maxb=16, phys=64)
+    q = ctypes.c_void_p(0x7f0000400000)
+    out = ctypes.c_void_p(0x7f0000500000)
+    ws = ctypes.c_void_p(0x7f0000600000)
+    need = lib.hyb_decode_sparse_workspace_bytes(ctypes.byref(d), 1000, 0)
+    assert need >= 4 * 8 * 4 + 4 * 8 * 1024 * 4  # lse rows + keys [4][8][max_l2 = 1024]
+    for top_k in (-1, 1025):
+        assert lib.hyb_decode_attn_sparse(ctypes.byref(d), q, ctypes.c_float(0.1), 1000, 0, top_k, ws, need,
+                                          out, None, None) == _lib.HYB_ERR_INVALID_VALUE
+    assert lib.hyb_decode_attn_sparse(ctypes.byref(d), q, ctypes.c_float(0.1), 1000, 0, 32, ws, need - 1,
+                                      out, None, None) == _lib.HYB_ERR_WORKSPACE
+    d0 = _desc(batch=4, maxb=16, phys=64, qbits=0)
+    assert lib.hyb_decode_attn_sparse(ctypes.byref(d0), q, ctypes.c_float(0.1), 1000, 0, 32, ws, need,
+                                      out, None, None) == _lib.HYB_ERR_UNSUPPORTED
+    # the page's rule, section 5.3
+    assert [hk.hyb_sparse_top_k(x) for x in (32768, 8192, 255, -5, 10 ** 9)] == [128, 32, 0, 0, 128]
+
+
 def test_migrate_argument_checks():
     """hyb_kv_migrate rejects bad arguments on the host, before any launch."""
     lib = hk.load()
