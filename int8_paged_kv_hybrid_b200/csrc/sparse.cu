@@ -24,7 +24,6 @@
 namespace hyb {
 
 constexpr int kScoreThreads = 128;
-constexpr int kTopkThreads = 256;
 constexpr float kLn2f = 0.6931471805599453f;
 
 // Tokens of sequence b held in its INT4 blocks (the oldest ones), or 0 when
@@ -124,8 +123,9 @@ __global__ void __launch_bounds__(kScoreThreads) l2_score_kernel(const SparseArg
   }
 }
 
-// Exclusive prefix count of `flag` over the CTA's threads in thread order;
+// Exclusive prefix count of `flag` over the CTA's kT threads in thread order;
 // *total gets the CTA's count.  Every thread calls it.
+template <int kT>
 __device__ __forceinline__ int cta_prefix(bool flag, int *s_warp, int tid, int *total) {
   const int lane = tid & 31, warp = tid >> 5;
   const unsigned bal = __ballot_sync(0xffffffffu, flag);
@@ -133,7 +133,7 @@ __device__ __forceinline__ int cta_prefix(bool flag, int *s_warp, int tid, int *
   __syncthreads();
   int before = 0, all = 0;
 #pragma unroll
-  for (int w = 0; w < kTopkThreads / 32; w++) {
+  for (int w = 0; w < kT / 32; w++) {
     const int c = s_warp[w];
     before += w < warp ? c : 0;
     all += c;
@@ -143,6 +143,7 @@ __device__ __forceinline__ int cta_prefix(bool flag, int *s_warp, int tid, int *
   return before + __popc(bal & ((1u << lane) - 1u));
 }
 
+template <int kT>
 __device__ __forceinline__ float cta_reduce(float v, float *s_red, int tid, bool is_max) {
   const int lane = tid & 31, warp = tid >> 5;
 #pragma unroll
@@ -154,12 +155,16 @@ __device__ __forceinline__ float cta_reduce(float v, float *s_red, int tid, bool
   __syncthreads();
   float r = s_red[0];
 #pragma unroll
-  for (int w = 1; w < kTopkThreads / 32; w++) r = is_max ? fmaxf(r, s_red[w]) : r + s_red[w];
+  for (int w = 1; w < kT / 32; w++) r = is_max ? fmaxf(r, s_red[w]) : r + s_red[w];
   __syncthreads();
   return r;
 }
 
-__global__ void __launch_bounds__(kTopkThreads) l2_topk_kernel(const SparseArgs a) {
+// kT threads per CTA: 1024 for long L2 ranges, 256 for short ones.
+template <int kT>
+__global__ void __launch_bounds__(kT) l2_topk_kernel(const SparseArgs a) {
+  constexpr int kTopkThreads = kT;
+  constexpr int kWarpsT = kT / 32;
   const int hh = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x;
   const int G = a.hq / a.hkv;
@@ -169,77 +174,144 @@ __global__ void __launch_bounds__(kTopkThreads) l2_topk_kernel(const SparseArgs 
   if (k <= 0) return;  // no L2 token attended: the dense result stands
   const float *keys = a.keys + ((size_t)b * a.hq + hh) * a.max_l2;
 
-  __shared__ int hist[256];
+  constexpr int kParts = kTopkThreads / kDim;
+  constexpr int kHists = kWarpsT / 4;
+  __shared__ int hist[kHists][256];  // one histogram per 4 warps (fewer colliding atomics)
   __shared__ int s_warp[kTopkThreads / 32];
   __shared__ float s_red[kTopkThreads / 32];
-  __shared__ int s_digit, s_need;
+  __shared__ int s_digit, s_need, s_eq, s_cnt;
   __shared__ int s_pos[kMaxTopK];
   __shared__ float s_p[kMaxTopK];
   __shared__ float s_sv[kMaxTopK];
   __shared__ int s_vt[kMaxTopK];
-  __shared__ float s_acc[kDim];
+  __shared__ float s_acc[kParts][kDim];
+  const float4 *keys4 = reinterpret_cast<const float4 *>(keys);  // rows are 256-byte aligned
+  const int n4 = (n + 3) / 4;
 
   // ---- the k-th largest key (exact), by four 8-bit radix passes ----
   uint32_t thr = 0;
-  int need_eq = k;
+  int need_eq = k, n_eq = 0;
   if (k < n) {
     uint32_t prefix = 0, mask = 0;
     int need = k;
     for (int pass = 0; pass < 4; pass++) {
       const int shift = 24 - 8 * pass;
-      hist[tid] = 0;
+      for (int i = tid; i < kHists * 256; i += kT) hist[i >> 8][i & 255] = 0;
       __syncthreads();
-      for (int i = tid; i < n; i += kTopkThreads) {
-        const uint32_t u = key_order(keys[i]);
-        if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
+      const int warp = tid >> 5, lane = tid & 31;
+      // the same trip count for every lane, so that whole warps match bins
+      for (int i4b = 0; i4b < n4; i4b += kT) {
+        const int i4 = i4b + tid;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i4 < n4) v = keys4[i4];
+        const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int t = 0; t < 4; t++) {
+          const uint32_t u = key_order(e[t]);
+          const bool in = i4 < n4 && 4 * i4 + t < n && (u & mask) == prefix;
+          const int bin = in ? static_cast<int>((u >> shift) & 255u) : 256;
+          // lanes with the same bin add once, by their lowest lane
+          const unsigned peers = __match_any_sync(0xffffffffu, bin);
+          if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[warp >> 2][bin], __popc(peers));
+        }
+      }
+      __syncthreads();
+      // fold the warps' histograms into the first
+      for (int d = tid; d < 256; d += kT) {
+        int sum = 0;
+#pragma unroll
+        for (int w = 0; w < kHists; w++) sum += hist[w][d];
+        hist[0][d] = sum;
       }
       __syncthreads();
       if (tid == 0) {
         int above = 0, d = 255;
         for (; d > 0; d--) {
-          if (above + hist[d] >= need) break;
-          above += hist[d];
+          if (above + hist[0][d] >= need) break;
+          above += hist[0][d];
         }
         s_digit = d;
         s_need = need - above;
+        s_eq = hist[0][d];  // after the last pass: the keys equal to the threshold
       }
       __syncthreads();
       prefix |= static_cast<uint32_t>(s_digit) << shift;
       mask |= 255u << shift;
       need = s_need;
+      n_eq = s_eq;
       __syncthreads();
     }
     thr = prefix;
     need_eq = need;
   }
 
-  // ---- the selected positions, in position order ----
-  int base = 0, eq_seen = 0;
-  for (int c0 = 0; c0 < n; c0 += kTopkThreads) {
-    const int i = c0 + tid;
-    bool sel;
-    if (k < n) {
+  // ---- the selected positions ----
+  if (k >= n) {
+    for (int i = tid; i < n; i += kTopkThreads) s_pos[i] = i;
+  } else if (need_eq == n_eq) {
+    // every key >= the threshold is taken: gather in any order, then sort
+    if (tid == 0) s_cnt = 0;
+    __syncthreads();
+    for (int i4 = tid; i4 < n4; i4 += kTopkThreads) {
+      const float4 v = keys4[i4];
+      const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int t = 0; t < 4; t++) {
+        const int i = 4 * i4 + t;
+        if (i < n && key_order(e[t]) >= thr) {
+          const int slot = atomicAdd(&s_cnt, 1);
+          if (slot < kMaxTopK) s_pos[slot] = i;
+        }
+      }
+    }
+    __syncthreads();
+    // bitonic sort of the k positions (ascending), padded to a power of two
+    int p2 = 1;
+    while (p2 < k) p2 <<= 1;
+    for (int i = k + tid; i < p2; i += kTopkThreads) s_pos[i] = 0x7fffffff;
+    __syncthreads();
+    for (int size = 2; size <= p2; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int i = tid; i < p2; i += kTopkThreads) {
+          const int j = i ^ stride;
+          if (j > i) {
+            const int x = s_pos[i], y = s_pos[j];
+            const bool up = (i & size) == 0;
+            if ((x > y) == up) {
+              s_pos[i] = y;
+              s_pos[j] = x;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+  } else {
+    // only some of the keys equal to the threshold are taken (the older
+    // ones): ordered compaction in position order
+    int base = 0, eq_seen = 0;
+    for (int c0 = 0; c0 < n; c0 += kTopkThreads) {
+      const int i = c0 + tid;
       const uint32_t u = i < n ? key_order(keys[i]) : 0u;
       const bool gt = i < n && u > thr;
       const bool eq = i < n && u == thr;
       int eq_tot;
-      const int eq_rank = cta_prefix(eq, s_warp, tid, &eq_tot);
-      sel = gt || (eq && eq_seen + eq_rank < need_eq);
+      const int eq_rank = cta_prefix<kT>(eq, s_warp, tid, &eq_tot);
+      const bool sel = gt || (eq && eq_seen + eq_rank < need_eq);
       eq_seen += eq_tot;
-    } else {
-      sel = i < n;
+      int sel_tot;
+      const int r = cta_prefix<kT>(sel, s_warp, tid, &sel_tot);
+      if (sel && base + r < kMaxTopK) s_pos[base + r] = i;
+      base += sel_tot;
     }
-    int sel_tot;
-    const int r = cta_prefix(sel, s_warp, tid, &sel_tot);
-    if (sel && base + r < kMaxTopK) s_pos[base + r] = i;
-    base += sel_tot;
   }
-  const int ns = min(base, k);  // == k
+  __syncthreads();
+  const int ns = k;
 
   // ---- softmax over the selected tokens (log2 domain, FP32) ----
   const __half *qh = a.q + ((size_t)b * a.hq + hh) * kDim;
   float qa = tid < kDim ? fabsf(__half2float(qh[tid])) : 0.f;
-  const float amax = cta_reduce(qa, s_red, tid, true);
+  const float amax = cta_reduce<kT>(qa, s_red, tid, true);
   const float coef = (amax / 32767.f) * a.qk_scale;
   float zmax = -INFINITY;
   for (int j = tid; j < ns; j += kTopkThreads) {
@@ -252,19 +324,19 @@ __global__ void __launch_bounds__(kTopkThreads) l2_topk_kernel(const SparseArgs 
     s_sv[j] = okp ? a.scales[((size_t)phys * a.hkv + h) * 2 + 1] : 0.f;
     zmax = fmaxf(zmax, z);
   }
-  const float m = cta_reduce(zmax, s_red, tid, true);
+  const float m = cta_reduce<kT>(zmax, s_red, tid, true);
   float lsum = 0.f;
   for (int j = tid; j < ns; j += kTopkThreads) {
     const float p = exp2f(s_p[j] - m);
     s_p[j] = p;
     lsum += p;
   }
-  const float l = cta_reduce(lsum, s_red, tid, false);
+  const float l = cta_reduce<kT>(lsum, s_red, tid, false);
 
-  // ---- P.V over the selected tokens' INT4 V codes (channel c, two halves of the list) ----
+  // ---- P.V over the selected tokens' INT4 V codes (channel c, kParts slices of the list) ----
   const int c = tid & (kDim - 1), part = tid >> 7;
   float acc = 0.f;
-  for (int j = part; j < ns; j += 2) {
+  for (int j = part; j < ns; j += kParts) {
     const int vt = s_vt[j];
     if (vt < 0) continue;
     const int slot = s_pos[j] & (kBlock - 1);
@@ -274,10 +346,11 @@ __global__ void __launch_bounds__(kTopkThreads) l2_topk_kernel(const SparseArgs 
     const int code = sext4((slot & 4) ? (byte >> 4) : (byte & 0xfu));
     acc = fmaf(s_p[j] * s_sv[j], static_cast<float>(code), acc);
   }
-  if (part == 1) s_acc[c] = acc;
+  s_acc[part][c] = acc;
   __syncthreads();
   if (part == 0) {
-    acc += s_acc[c];
+#pragma unroll
+    for (int t = 1; t < kParts; t++) acc += s_acc[t][c];
     // merge with the dense pass (its output and natural-log log-sum-exp)
     const size_t row = (size_t)b * a.hq + hh;
     const float o_s = acc / l;
@@ -300,7 +373,10 @@ cudaError_t launch_sparse_l2(const SparseArgs &a, int batch, cudaStream_t stream
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 g2(a.hq, batch);
-  l2_topk_kernel<<<g2, kTopkThreads, 0, stream>>>(a);
+  if (a.max_l2 >= 32768)
+    l2_topk_kernel<1024><<<g2, 1024, 0, stream>>>(a);
+  else
+    l2_topk_kernel<256><<<g2, 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
