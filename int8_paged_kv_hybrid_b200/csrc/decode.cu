@@ -70,7 +70,9 @@ struct DecodeSmem {
 // one (sequence, kv head)); splits are merged through distributed shared
 // memory instead of the workspace.  kF16: FP16 cold blocks (quantization_bits
 // 0), each attended as two items of 32 rows with the hot ring's arithmetic.
-template <int G, bool kCluster, bool kF16>
+// kSkip: sparse L2 mode -- the sequence's INT4 ("L2") blocks are left to the
+// top-k kernels, and the splits cover the blocks from its INT4 count on.
+template <int G, bool kCluster, bool kF16, bool kSkip>
 __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(const DecodeArgs a) {
   constexpr int P = pow2_heads<G>();
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -80,7 +82,12 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int S = a.n_splits;
   const int hq0 = h * G;
-  const int i0 = s * a.split_blocks;
+  int ib = 0;  // first block of the splits
+  if constexpr (kSkip) {
+    const int n4 = a.quant_bits == 4 ? a.max_blocks : (a.n_int4 ? a.n_int4[b] : 0);
+    ib = min(max(n4, 0), a.max_blocks);
+  }
+  const int i0 = ib + s * a.split_blocks;
 
   // independent loads first: the sequence length, this split's block-table
   // entries (one per thread, clamped to the row) and q
@@ -116,7 +123,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
   const int H = a.hot_tokens;
   const int Lc = max(0, L - H);
   const int nblk = (Lc + kBlock - 1) / kBlock;
-  const int Sb = max(1, (nblk + a.split_blocks - 1) / a.split_blocks);
+  const int Sb = max(1, (max(0, nblk - ib) + a.split_blocks - 1) / a.split_blocks);
   // past this sequence's last split: no work and no partial (a cluster member
   // still takes part in the cluster's merge, with an empty state)
   if (!kCluster && s >= Sb) return;
@@ -182,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
       const int kb = fp16 ? k >> 1 : k;
       const int phys = sm.phys[kb];
       const int nrow = fp16 ? min(kItemRows, Lc - (i0 + kb) * kBlock - (k & 1) * kItemRows) : 1;
-      if (phys < 0 || nrow <= 0 || (!fp16 && a.l2_skip && i0 + kb < n_int4_b)) {
+      if (phys < 0 || nrow <= 0) {
         mbar_arrive(&sm.full[st]);
         return;
       }
@@ -301,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
     if (ok && !fp16 && k < ncold) {
       // ---------------- cold block ----------------
       const int i = i0 + k;
-      const int nvalid = (sm.phys[k] < 0 || (a.l2_skip && i < n_int4_b)) ? 0 : min(kBlock, Lc - i * kBlock);
+      const int nvalid = sm.phys[k] < 0 ? 0 : min(kBlock, Lc - i * kBlock);
       const int nv = nvalid - 16 * warp;
       const bool int4 = i < n_int4_b;
       const float2 sc = sm.scl[k];
@@ -449,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
 // Largest cluster the decode kernel is launched with (portable size).
 constexpr int kMaxCluster = 8;
 
-template <int G, bool kF16>
+template <int G, bool kF16, bool kSkip>
 static cudaError_t launch_decode_g(const DecodeArgs &a, int batch, bool cluster, cudaStream_t stream) {
   const size_t smem = sizeof(DecodeSmem<G>);
   static int configured_dev_mask = 0;  // one bit per device
@@ -457,10 +464,10 @@ static cudaError_t launch_decode_g(const DecodeArgs &a, int batch, bool cluster,
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 31 && !(configured_dev_mask & (1 << dev))) {
-    e = cudaFuncSetAttribute(decode_kernel<G, false, kF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(decode_kernel<G, false, kF16, kSkip>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(decode_kernel<G, true, kF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = cudaFuncSetAttribute(decode_kernel<G, true, kF16, kSkip>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     configured_dev_mask |= 1 << dev;
@@ -479,32 +486,33 @@ static cudaError_t launch_decode_g(const DecodeArgs &a, int batch, bool cluster,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_kernel<G, true, kF16>, a);
+    e = cudaLaunchKernelEx(&cfg, decode_kernel<G, true, kF16, kSkip>, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
-  decode_kernel<G, false, kF16><<<grid, kThreads, smem, stream>>>(a);
+  decode_kernel<G, false, kF16, kSkip><<<grid, kThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
-template <bool kF16>
+template <bool kF16, bool kSkip>
 static cudaError_t launch_decode_f(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream) {
   switch (group) {
-    case 1: return launch_decode_g<1, kF16>(a, batch, cluster, stream);
-    case 2: return launch_decode_g<2, kF16>(a, batch, cluster, stream);
-    case 3: return launch_decode_g<3, kF16>(a, batch, cluster, stream);
-    case 4: return launch_decode_g<4, kF16>(a, batch, cluster, stream);
-    case 5: return launch_decode_g<5, kF16>(a, batch, cluster, stream);
-    case 6: return launch_decode_g<6, kF16>(a, batch, cluster, stream);
-    case 7: return launch_decode_g<7, kF16>(a, batch, cluster, stream);
-    case 8: return launch_decode_g<8, kF16>(a, batch, cluster, stream);
+    case 1: return launch_decode_g<1, kF16, kSkip>(a, batch, cluster, stream);
+    case 2: return launch_decode_g<2, kF16, kSkip>(a, batch, cluster, stream);
+    case 3: return launch_decode_g<3, kF16, kSkip>(a, batch, cluster, stream);
+    case 4: return launch_decode_g<4, kF16, kSkip>(a, batch, cluster, stream);
+    case 5: return launch_decode_g<5, kF16, kSkip>(a, batch, cluster, stream);
+    case 6: return launch_decode_g<6, kF16, kSkip>(a, batch, cluster, stream);
+    case 7: return launch_decode_g<7, kF16, kSkip>(a, batch, cluster, stream);
+    case 8: return launch_decode_g<8, kF16, kSkip>(a, batch, cluster, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream) {
-  return a.quant_bits == 0 ? launch_decode_f<true>(a, group, batch, cluster, stream)
-                           : launch_decode_f<false>(a, group, batch, cluster, stream);
+  if (a.quant_bits == 0) return launch_decode_f<true, false>(a, group, batch, cluster, stream);
+  if (a.l2_skip) return launch_decode_f<false, true>(a, group, batch, cluster, stream);
+  return launch_decode_f<false, false>(a, group, batch, cluster, stream);
 }
 
 int decode_max_cluster() { return kMaxCluster; }
@@ -527,10 +535,10 @@ int decode_ctas_per_sm(int group) {
   switch (group) {
 #define HYB_OCC(g)                                                                          \
   case g:                                                                                   \
-    e = cudaFuncSetAttribute(decode_kernel<g, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+    e = cudaFuncSetAttribute(decode_kernel<g, false, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              static_cast<int>(sizeof(DecodeSmem<g>)));                      \
     if (e == cudaSuccess)                                                                   \
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<g, false, false>, kThreads, \
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<g, false, false, false>, kThreads, \
                                                         sizeof(DecodeSmem<g>));             \
     break;
     HYB_OCC(1) HYB_OCC(2) HYB_OCC(3) HYB_OCC(4) HYB_OCC(5) HYB_OCC(6) HYB_OCC(7) HYB_OCC(8)

@@ -77,32 +77,70 @@ __global__ void __launch_bounds__(kScoreThreads) l2_score_kernel(const SparseArg
   }
   __syncthreads();
 
-  // thread: token tok of the block, channels 64*half .. 64*half + 63
+  // the chunk's INT4 K tiles (4 KB each) staged in shared memory, every
+  // thread's loads issued together
+  constexpr int kMaxChunk = 4;
+  __shared__ alignas(16) uint32_t tiles[kMaxChunk][1024];
+  __shared__ int s_phys[kMaxChunk];
+  const int nblk = min(nb - blk0, min(a.blocks_per_cta, kMaxChunk));
+  uint4 stage[kMaxChunk][2];
+#pragma unroll
+  for (int t = 0; t < kMaxChunk; t++) {
+    stage[t][0] = make_uint4(0u, 0u, 0u, 0u);
+    stage[t][1] = stage[t][0];
+    if (t < nblk) {
+      const int phys = a.block_table[(size_t)b * a.max_blocks + blk0 + t];
+      const bool okp = phys >= 0 && phys < a.num_phys;
+      if (tid == 0) s_phys[t] = okp ? phys : -1;
+      if (!okp && tid == 0) set_status(a.status, HYB_STATUS_BAD_BLOCK);
+      if (okp) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.cold + ((size_t)phys * a.hkv + h) * kTilePairBytes);
+        stage[t][0] = src[tid];
+        stage[t][1] = src[kScoreThreads + tid];
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < kMaxChunk; t++) {
+    if (t < nblk) {
+      reinterpret_cast<uint4 *>(tiles[t])[tid] = stage[t][0];
+      reinterpret_cast<uint4 *>(tiles[t])[kScoreThreads + tid] = stage[t][1];
+    }
+  }
+  __syncthreads();
+
+  // thread: token tok of a block, channels 64*half .. 64*half + 63
   const int tok = tid >> 1, half = tid & 1;
-  const int blk1 = min(nb, blk0 + a.blocks_per_cta);
-  for (int blk = blk0; blk < blk1; blk++) {
-    const int phys = a.block_table[(size_t)b * a.max_blocks + blk];
-    const bool okp = phys >= 0 && phys < a.num_phys;
-    if (!okp && tid == 0) set_status(a.status, HYB_STATUS_BAD_BLOCK);
+  for (int t = 0; t < nblk; t++) {
+    const int blk = blk0 + t;
+    const int phys = s_phys[t];
+    const bool okp = phys >= 0;
     int dot[8];
 #pragma unroll
     for (int g = 0; g < 8; g++) dot[g] = 0;
     if (okp) {
       // INT4 K: 64 bytes per token, word w holds channels 8w..8w+7 (byte i:
       // channel 8w+i in the low nibble, 8w+4+i in the high nibble)
-      const uint8_t *ktile = a.cold + ((size_t)phys * a.hkv + h) * kTilePairBytes;
-      const uint32_t *kp = reinterpret_cast<const uint32_t *>(ktile + tok * 64 + half * 32);
-#pragma unroll 1
+      // per word: the codes as bytes (channels 8w..8w+3, then 8w+4..8w+7)
+      // against q pairs, two 16x8-bit products per dp2a, exact in int32
+      const uint32_t *kp = tiles[t] + tok * 16 + half * 8;
+#pragma unroll 2
       for (int w = 0; w < 8; w++) {
         const uint32_t word = kp[w];
+        const int lo4 = static_cast<int>(sext_nibbles(word & 0x0f0f0f0fu));
+        const int hi4 = static_cast<int>(sext_nibbles((word >> 4) & 0x0f0f0f0fu));
         const int cb = 64 * half + 8 * w;
 #pragma unroll
-        for (int i = 0; i < 4; i++) {
-          const int lo = sext4((word >> (8 * i)) & 0xfu);
-          const int hi = sext4((word >> (8 * i + 4)) & 0xfu);
-#pragma unroll
-          for (int g = 0; g < 8; g++)
-            if (g < G) dot[g] += static_cast<int>(qi[g][cb + i]) * lo + static_cast<int>(qi[g][cb + 4 + i]) * hi;
+        for (int g = 0; g < 8; g++) {
+          if (g < G) {
+            const uint4 qp = *reinterpret_cast<const uint4 *>(&qi[g][cb]);  // channels cb..cb+7
+            int d = dot[g];
+            d = __dp2a_lo(static_cast<int>(qp.x), lo4, d);
+            d = __dp2a_hi(static_cast<int>(qp.y), lo4, d);
+            d = __dp2a_lo(static_cast<int>(qp.z), hi4, d);
+            d = __dp2a_hi(static_cast<int>(qp.w), hi4, d);
+            dot[g] = d;
+          }
         }
       }
     }
