@@ -578,8 +578,9 @@ int ora_get_ring(const ora_cache *c, int b, uint16_t *ring) {
 
 /* ------------------------------------------------------------------ */
 /* The device memory format, written out from its definition:          */
-/*   cold pool bytes [num_phys][hkv][2][tile] with tile = block*d bytes */
-/*   (K tile, then V tile, per physical block and kv head).            */
+/*   cold pool bytes [num_phys][hkv][2][tile] with tile = 64*d bytes   */
+/*   (K tile, then V tile, per physical block of 64 tokens and kv      */
+/*   head).                                                            */
 /*   K tile, INT8: token-major, byte (t, ch) at t*d + ch.              */
 /*   V tile, INT8: channel-major, 64 token bytes per channel row, the  */
 /*     four 16-byte chunks of row ch stored at chunk index             */
@@ -595,9 +596,12 @@ int ora_get_ring(const ora_cache *c, int b, uint16_t *ring) {
 /*     8-byte units of 16 tokens, unit u stored at u XOR ((ch/4) % 4); */
 /*     within a unit, tokens 0..7 in its first word, 8..15 in the      */
 /*     second.                                                         */
+/*   Blocks of 128 tokens are stored as two such 64-slot sub-blocks:   */
+/*   [num_phys][hkv][2 sub-blocks][2][8192], slot t of the block in    */
+/*   slot t%64 of sub-block t/64; the block keeps one scale per K|V.   */
 /*   FP16 cold blocks (quant_bits 0): cold pool bytes                  */
 /*   [num_phys][hkv][block][2][d] FP16, per token the K row then the V  */
-/*   row (the hot ring's layout), 32 KB per block and kv head.          */
+/*   row (the hot ring's layout), 512 B per token and kv head.          */
 /*   scales: float [num_phys][hkv][2] (not used by FP16 blocks).        */
 /*   hot ring: FP16 [batch][hkv][hot][2][d] (K row, then V row).       */
 /* Only sealed slots are written; other bytes are left as they are.    */
@@ -612,8 +616,10 @@ static void put_nibble(uint8_t *word4, int e, int code) {
 int ora_export(const ora_cache *c, const int32_t *block_table, int num_phys,
                uint8_t *cold, float *scales, uint16_t *hot, int32_t *seq_lens) {
   const int d = c->d, blk = c->block, hkv = c->hkv;
-  const size_t tile = (size_t)blk * d;
-  if (d != 128 || blk != 64) return ORA_ERR_INVALID; /* format defined for 64 x 128 */
+  const size_t tile = (size_t)64 * d; /* one K or V tile of a 64-slot sub-block */
+  const int nsub = blk / 64;          /* sub-blocks per block */
+  /* format defined for d = 128 and blocks of 64 or 128 tokens */
+  if (d != 128 || (blk != 64 && blk != 128)) return ORA_ERR_INVALID;
   if (c->quant_bits == 0) {
     uint16_t *cold16 = (uint16_t *)cold;
     for (int b = 0; b < c->batch; b++) {
@@ -649,11 +655,13 @@ int ora_export(const ora_cache *c, const int32_t *block_table, int num_phys,
       for (int h = 0; h < hkv; h++) {
         for (int kv = 0; kv < 2; kv++) {
           const int8_t *cd = c->codes[bi] + ((size_t)h * 2 + kv) * blk * d;
-          uint8_t *t8 = cold + (((size_t)phys * hkv + h) * 2 + kv) * tile;
           scales[((size_t)phys * hkv + h) * 2 + kv] = c->scale[bi][h * 2 + kv];
-          for (int t = 0; t < sealed; t++)
+          for (int tb = 0; tb < sealed; tb++)
             for (int ch = 0; ch < d; ch++) {
-              const int code = cd[t * d + ch];
+              /* slot tb of the block: slot t = tb % 64 of sub-block tb / 64 */
+              const int t = tb % 64;
+              uint8_t *t8 = cold + (((((size_t)phys * hkv + h) * nsub + tb / 64) * 2) + kv) * tile;
+              const int code = cd[tb * d + ch];
               if (c->qmax[bi] == 127) {
                 if (kv == 0) t8[t * d + ch] = (uint8_t)code;
                 else t8[ch * 64 + (((t / 16) ^ ((ch / 2) % 4)) * 16) + t % 16] = (uint8_t)code;

@@ -47,12 +47,12 @@ def _dense_kv(oc, b, L):
             K[p] = ring[:, p % H, 0]
             V[p] = ring[:, p % H, 1]
         else:
-            i = p // 64
+            i = p // oc.block
             if i not in blocks:
                 blocks[i] = oc.get_block(b, i)
             _, codes, sc = blocks[i]
-            K[p] = codes[:, 0, p % 64].astype(np.float64) * sc[:, 0:1].astype(np.float64)
-            V[p] = codes[:, 1, p % 64].astype(np.float64) * sc[:, 1:2].astype(np.float64)
+            K[p] = codes[:, 0, p % oc.block].astype(np.float64) * sc[:, 0:1].astype(np.float64)
+            V[p] = codes[:, 1, p % oc.block].astype(np.float64) * sc[:, 1:2].astype(np.float64)
     return K, V
 
 
@@ -119,6 +119,39 @@ def test_brute_force_other_hot_sizes(hot):
         o2, l2 = _brute(q[b], K, V, scale, g)
         assert np.abs(out[b] - o2).max() < 1e-12
         assert np.abs(lse[b] - l2).max() < 1e-12
+
+
+@pytest.mark.parametrize("qbits", [8, 4])
+def test_brute_force_128_token_blocks(qbits):
+    """block_size 128: one scale per 128 sealed tokens (the textbook absmax
+    quantizer over the whole group when it is sealed in one call), attention
+    equal to dense brute force."""
+    rng = np.random.default_rng(300 + qbits)
+    total = np.array([32 + 128, 32 + 300, 5, 0])
+    B, hkv, g = len(total), 2, 4
+    oc = oracle.OracleCache(B, hkv, hkv * g, max_blocks_per_seq=3, quant_bits=qbits, block=128)
+    k = rng.standard_normal((B, 332, hkv, D)).astype(np.float16)
+    v = rng.standard_normal((B, 332, hkv, D)).astype(np.float16)
+    oc.append(total.astype(np.int32), k, v)
+    Q = 127 if qbits == 8 else 7
+    # sequence 0: exactly one full block, sealed in one call
+    _, codes, sc = oc.get_block(0, 0)
+    for h in range(hkv):
+        for kv, x in ((0, k), (1, v)):
+            grp = x[0, :128, h].astype(np.float32)
+            s = np.float32(np.abs(grp).max()) / np.float32(Q)
+            assert sc[h, kv] == s
+            want = np.clip(np.rint(grp / s), -Q, Q)
+            assert np.array_equal(codes[h, kv, :128], want)
+    q = rng.standard_normal((B, hkv * g, D)).astype(np.float16)
+    out, lse = oc.decode(q, 0.088, nthreads=2)
+    for b in range(B):
+        L = int(total[b])
+        if L == 0:
+            continue
+        K, V = _dense_kv(oc, b, L)
+        o2, l2 = _brute(q[b], K, V, 0.088, g)
+        assert np.abs(out[b] - o2).max() < 1e-12 and np.abs(lse[b] - l2).max() < 1e-12
 
 
 def test_pairs_subset_matches_full():

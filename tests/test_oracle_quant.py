@@ -206,3 +206,30 @@ def test_metadata_block_counts():
         assert -(-ctx // bs) == nblk and nblk * 16 == hdr
         if bs == 64:
             assert synth.cold_blocks_for(ctx) == nblk
+
+
+def test_export_128_token_blocks_as_two_sub_blocks():
+    """block_size 128 in the device format: slot t of a block is slot t % 64
+    of sub-block t // 64 (each sub-block a 64-slot K tile + V tile of the
+    64-token format); one scale pair per block."""
+    rng = np.random.default_rng(12)
+    L = 32 + 200
+    oc = oracle.OracleCache(1, 2, 2, max_blocks_per_seq=2, quant_bits=8, block=128)
+    k = rng.standard_normal((1, L, 2, D)).astype(np.float16)
+    v = rng.standard_normal((1, L, 2, D)).astype(np.float16)
+    oc.append(np.array([L], np.int32), k, v)
+    table = np.array([[3, 1]], np.int32)
+    ex = oc.export(table, 4)
+    cold = ex["cold"].reshape(4, 2, 2, 2, 64 * D)  # [phys][h][sub-block][K|V][8192]
+    for i, phys in enumerate(table[0]):
+        _, codes, sc = oc.get_block(0, i)
+        assert np.array_equal(ex["scales"][phys], sc)
+        n = min(128, L - 32 - 128 * i)
+        for t in range(n):
+            sb, s = divmod(t, 64)
+            kt = cold[phys, :, sb, 0].view(np.int8)
+            vt = cold[phys, :, sb, 1].view(np.int8)
+            assert np.array_equal(kt[:, s * D:(s + 1) * D], codes[:, 0, t])
+            for ch in (0, 5, 77, 127):
+                off = ch * 64 + (((s // 16) ^ ((ch // 2) % 4)) * 16) + s % 16
+                assert np.array_equal(vt[:, off], codes[:, 1, t, ch])
