@@ -54,6 +54,8 @@ def parse():
                    help="cold blocks: 8 (INT8, the default), 4 (all INT4) or 0 (FP16, quantization off)")
     p.add_argument("--hot-tokens", type=int, default=32, choices=[16, 32, 64, 128],
                    help="hot-zone tokens (32, the default, is the page's value)")
+    p.add_argument("--block-size", type=int, default=64, choices=[64, 128],
+                   help="tokens per cold block (64, the default, is the page's value)")
     p.add_argument("--sparse-top-k", type=int, default=None,
                    help="time hyb_decode_attn_sparse with this top_k (-1: the page's rule min(128, L // 256)) "
                         "against the dense hyb_decode_attn on the same cache (workload default 4, the older "
@@ -74,17 +76,17 @@ def workload_config(w, split, ns, qbits=8):
     H = w.hot_tokens
     if w.name == "config2":
         what = ("llama3-8b decode attention, 1 layer: batch %d, Hq %d, Hkv %d, d 128, L %d (%d FP16 hot + "
-                "%d %s cold in 64-token blocks), %d-block pool"
+                "%d %s cold in %d-token blocks), %d-block pool"
                 % (w.batch, w.num_q_heads, w.num_kv_heads, int(lens[0]), H, int(lens[0]) - H, cold,
-                   w.num_phys_blocks))
+                   w.block_size, w.num_phys_blocks))
     else:
         what = ("decode attention, 1 layer: batch %d, Hq %d, Hkv %d, d 128, L %d..%d (mean %.0f), %d FP16 hot "
-                "+ %s cold in 64-token blocks, %d-block pool"
+                "+ %s cold in %d-token blocks, %d-block pool"
                 % (w.batch, w.num_q_heads, w.num_kv_heads, int(lens.min()), int(lens.max()), float(lens.mean()),
-                   H, cold, w.num_phys_blocks))
+                   H, cold, w.block_size, w.num_phys_blocks))
     return {"workload": what, "batch": int(w.batch), "seq_len": int(lens.max()),
             "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads, "head_dim": 128, "hot_tokens": H,
-            "block_size": 64, "quant_bits": qbits, "split_tokens": split, "n_splits": ns,
+            "block_size": w.block_size, "quant_bits": qbits, "split_tokens": split, "n_splits": ns,
             "step": "hyb_decode_step: append 1 token/seq + split-KV attention, one launch",
             "l2": "flushed between timed steps (512 MB write)",
             "parallelism": "replicas (independent batch per GPU)"}
@@ -191,7 +193,7 @@ def room_for_growth(w, extra_tokens):
     widened when needed.  For runs that let the cache grow."""
     import numpy as np
     from int8_paged_kv_hybrid_b200 import synth
-    need = [synth.cold_blocks_for(int(L) + extra_tokens, w.hot_tokens) for L in w.lens]
+    need = [synth.cold_blocks_for(int(L) + extra_tokens, w.hot_tokens, w.block_size) for L in w.lens]
     width = max(w.max_blocks, max(need))
     bt = np.full((w.batch, width), -1, np.int32)
     bt[:, :w.max_blocks] = w.block_table
@@ -199,7 +201,7 @@ def room_for_growth(w, extra_tokens):
     spare = [p for p in range(w.num_phys_blocks) if p not in used]
     nxt = w.num_phys_blocks
     for b in range(w.batch):
-        for j in range(synth.cold_blocks_for(int(w.lens[b]), w.hot_tokens), need[b]):
+        for j in range(synth.cold_blocks_for(int(w.lens[b]), w.hot_tokens, w.block_size), need[b]):
             if bt[b, j] < 0:
                 if spare:
                     bt[b, j] = spare.pop(0)
@@ -214,7 +216,8 @@ def build_gpu_state(w, torch, qbits=8):
     from int8_paged_kv_hybrid_b200 import HybridKVCache, synth
     cache = HybridKVCache(w.batch, w.num_kv_heads, w.num_q_heads, w.num_phys_blocks, w.max_blocks,
                           quant_bits=qbits, block_table=w.block_table,
-                          n_int4=w.n_int4 if qbits == 8 else None, hot_tokens=w.hot_tokens)
+                          n_int4=w.n_int4 if qbits == 8 else None, hot_tokens=w.hot_tokens,
+                          block_size=w.block_size)
     # prefill to L-1 in 64-token appends; the benchmarked step appends the last token
     sched = synth._chunk_schedule(w.lens, 64)
     for si, n in enumerate(sched[:-1]):
@@ -237,7 +240,7 @@ def _touched_blocks(w, n_last):
         L_new = int(w.lens[b])
         L_old = L_new - int(n_last[b])
         e0, e1 = max(0, L_old - w.hot_tokens), max(0, L_new - w.hot_tokens)
-        for i in range(e0 // 64, (e1 + 63) // 64):
+        for i in range(e0 // w.block_size, (e1 + w.block_size - 1) // w.block_size):
             if e1 > e0:
                 phys.append(int(w.block_table[b, i]))
     return np.array(sorted(set(phys)), np.int64)
@@ -253,9 +256,11 @@ def run_native(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     clocks = ClockSampler(local_rank) if rank == 0 and not args.lean else None
     w = synth.make_workload(args.workload, seed_offset=1000 * rank)
-    if args.hot_tokens != w.hot_tokens:
-        w.hot_tokens = args.hot_tokens
-        room_for_growth(w, 0)  # a smaller hot zone seals more blocks
+    if args.hot_tokens != w.hot_tokens or args.block_size != w.block_size:
+        # a smaller hot zone seals more blocks; larger blocks use the first
+        # entries of the same table
+        w.hot_tokens, w.block_size = args.hot_tokens, args.block_size
+        room_for_growth(w, 0)
     if args.lean:
         room_for_growth(w, args.warmup + args.steps + 2)  # the lean run lets the cache grow
     L = int(w.lens.max())
@@ -404,7 +409,8 @@ def run_native(args, rank, world, local_rank):
                          "frac": round(achieved / peak, 4),
                          # the committed ncu figure covers the default workload and cold format only
                          "traffic": profiled_traffic() if (args.workload == WORKLOAD and qb == 8
-                                                           and args.hot_tokens == 32 and not args.split)
+                                                           and args.hot_tokens == 32 and args.block_size == 64
+                                                           and not args.split)
                                     else None,
                          "kernel": "hyb::decode_kernel (fused append + attention, the step's only launch)",
                          "peak_kind": peak_kind,
@@ -561,7 +567,8 @@ def oracle_step_rate(w, steps, warmup, budget_s=None, qbits=8):
     import oracle
     from int8_paged_kv_hybrid_b200 import synth
     threads = os.cpu_count() or 1
-    ora = oracle.OracleCache(w.batch, w.num_kv_heads, w.num_q_heads, w.max_blocks + 16, qbits, hot=w.hot_tokens)
+    ora = oracle.OracleCache(w.batch, w.num_kv_heads, w.num_q_heads, w.max_blocks + 16, qbits, hot=w.hot_tokens,
+                             block=w.block_size)
     if qbits == 8 and w.n_int4 is not None:
         ora.set_n_int4(w.n_int4)
     sched = synth._chunk_schedule(w.lens, 64)
@@ -600,7 +607,7 @@ def main():
         if rank != 0:
             return 0
         w = synth.make_workload(args.workload)
-        w.hot_tokens = args.hot_tokens
+        w.hot_tokens, w.block_size = args.hot_tokens, args.block_size
         sec, n, threads = oracle_step_rate(w, args.steps, args.warmup, budget_s=150.0, qbits=args.quant_bits)
         kvb = synth.kv_bytes(w, quant_bits=args.quant_bits)
         val = kvb / sec / 1e9

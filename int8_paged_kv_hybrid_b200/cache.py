@@ -16,18 +16,21 @@ TILE_BYTES = BLOCK * HEAD_DIM
 
 class HybridKVCache:
     def __init__(self, batch, num_kv_heads, num_q_heads, num_phys_blocks, max_blocks_per_seq,
-                 quant_bits=8, block_table=None, n_int4=None, device="cuda", hot_tokens=HOT):
+                 quant_bits=8, block_table=None, n_int4=None, device="cuda", hot_tokens=HOT,
+                 block_size=BLOCK):
         import torch
         self.batch, self.hkv, self.hq = int(batch), int(num_kv_heads), int(num_q_heads)
         self.num_phys, self.max_blocks = int(num_phys_blocks), int(max_blocks_per_seq)
         self.quant_bits = int(quant_bits)
         self.hot_tokens = int(hot_tokens)
+        self.block_size = int(block_size)
         dev = torch.device(device)
         self.device = dev
         self.hot = torch.zeros((self.batch, self.hkv, self.hot_tokens, 2, HEAD_DIM), dtype=torch.float16,
                                device=dev)
-        # quant_bits 0: FP16 blocks, 64 rows of K then V (twice the bytes)
-        parts = 4 if self.quant_bits == 0 else 2
+        # 8 KB parts per block and kv head: K and V tiles of each 64-token
+        # sub-block; FP16 blocks (quant_bits 0) hold rows of K then V, twice the bytes
+        parts = (4 if self.quant_bits == 0 else 2) * max(1, self.block_size // BLOCK)
         self.cold = torch.zeros((self.num_phys, self.hkv, parts, TILE_BYTES), dtype=torch.uint8, device=dev)
         self.scales = torch.zeros((self.num_phys, self.hkv, 2), dtype=torch.float32, device=dev)
         if block_table is None:
@@ -47,7 +50,7 @@ class HybridKVCache:
 
     def _make_desc(self):
         d = _lib.CacheDesc()
-        d.hot_tokens, d.block_size, d.head_dim = self.hot_tokens, BLOCK, HEAD_DIM
+        d.hot_tokens, d.block_size, d.head_dim = self.hot_tokens, self.block_size, HEAD_DIM
         d.quant_bits = self.quant_bits
         d.num_kv_heads, d.num_q_heads = self.hkv, self.hq
         d.num_phys_blocks, d.max_blocks_per_seq, d.batch = self.num_phys, self.max_blocks, self.batch

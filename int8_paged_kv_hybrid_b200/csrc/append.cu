@@ -77,7 +77,8 @@ __global__ void __launch_bounds__(512) append_kernel(AppendArgs a) {
     return;
   }
   const long long L_new_ll = static_cast<long long>(L_old) + n;
-  if (L_new_ll - a.hot_tokens > static_cast<long long>(a.max_blocks) * kBlock || L_new_ll > 0x7fffffffLL) {
+  const int B = kBlock << a.lsub;  // tokens per block
+  if (L_new_ll - a.hot_tokens > static_cast<long long>(a.max_blocks) * B || L_new_ll > 0x7fffffffLL) {
     if (threadIdx.x == 0) set_status(a.status, HYB_STATUS_CAPACITY);
     return;
   }
@@ -89,9 +90,9 @@ __global__ void __launch_bounds__(512) append_kernel(AppendArgs a) {
   for (int pair = warp; pair < 2 * a.hkv; pair += nwarps) {
     const int h = pair >> 1, kv = pair & 1;
     for (int p0 = e0; p0 < e1;) {
-      const int i = p0 / kBlock;
-      const int p1 = min((i + 1) * kBlock, e1);
-      const int first = p0 - i * kBlock;
+      const int i = p0 / B;
+      const int p1 = min((i + 1) * B, e1);
+      const int first = p0 - i * B;
       const int phys = a.block_table[(size_t)b * a.max_blocks + i];
       if (phys < 0 || phys >= a.num_phys) {
         if (lane == 0) set_status(a.status, HYB_STATUS_BAD_BLOCK);
@@ -100,14 +101,14 @@ __global__ void __launch_bounds__(512) append_kernel(AppendArgs a) {
       }
       if (a.quant_bits == 0) {
         // FP16 cold block: the rows move unchanged (K row then V row per slot)
-        __half *blk = reinterpret_cast<__half *>(a.cold + ((size_t)phys * a.hkv + h) * kFp16BlockBytes);
+        __half *blk = reinterpret_cast<__half *>(a.cold + ((size_t)phys * a.hkv + h) * (kFp16BlockBytes << a.lsub));
         for (int t = p0; t < p1; t++) {
           const __half *src;
           if (t < L_old)
             src = a.hot + ((((size_t)b * a.hkv + h) * a.hot_tokens + (t & (a.hot_tokens - 1))) * 2 + kv) * kDim;
           else
             src = (kv ? a.v_new : a.k_new) + (((size_t)b * a.max_new + (t - L_old)) * a.hkv + h) * kDim;
-          __half *dst = blk + ((t - i * kBlock) * 2 + kv) * kDim;
+          __half *dst = blk + ((t - i * B) * 2 + kv) * kDim;
           *reinterpret_cast<uint2 *>(dst + 4 * lane) = *reinterpret_cast<const uint2 *>(src + 4 * lane);
         }
         p0 = p1;
@@ -129,15 +130,21 @@ __global__ void __launch_bounds__(512) append_kernel(AppendArgs a) {
       }
       for (int m = 16; m > 0; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
       const float s_c = __fdiv_rn(amax, static_cast<float>(q));
-      uint8_t *tile = a.cold + (((size_t)phys * a.hkv + h) * 2 + kv) * kTileBytes;
+      // the block's 64-slot sub-blocks: K tile + V tile each
+      uint8_t *tile0 = a.cold + ((((size_t)phys * a.hkv + h) << a.lsub) * 2 + kv) * kTileBytes;
       float *sp = a.scales + ((size_t)phys * a.hkv + h) * 2 + kv;
       float s = s_c;
       if (first != 0) {
         const float s_old = *sp;
-        if (s_c > s_old)
-          requant_tile(tile, kv, int4, first, s_old, s_c, q, lane, s_tbl[warp]);
-        else
+        if (s_c > s_old) {
+          for (int u = 0; u <= a.lsub; u++) {
+            const int first_u = min(max(first - kBlock * u, 0), kBlock);
+            if (first_u > 0)
+              requant_tile(tile0 + (size_t)u * kTilePairBytes, kv, int4, first_u, s_old, s_c, q, lane, s_tbl[warp]);
+          }
+        } else {
           s = s_old;
+        }
       }
       __syncwarp();
       for (int t0 = p0; t0 < p1; t0 += 8) {
@@ -149,7 +156,9 @@ __global__ void __launch_bounds__(512) append_kernel(AppendArgs a) {
         for (int u = 0; u < 8; u++) {
         const int t = t0 + u;
         if (t >= p1) break;
-        const int slot = t - i * kBlock;
+        const int slot_b = t - i * B;  // slot in the block: slot_b % 64 of sub-block slot_b / 64
+        const int slot = slot_b & (kBlock - 1);
+        uint8_t *tile = tile0 + (size_t)(slot_b >> 6) * kTilePairBytes;
         int c[4];
         for (int j = 0; j < 4; j++) c[j] = quantize(xb[u][j], s, q);
         if (!int4 && kv == 0) {

@@ -72,7 +72,8 @@ struct DecodeSmem {
 // 0), each attended as two items of 32 rows with the hot ring's arithmetic.
 // kSkip: sparse L2 mode -- the sequence's INT4 ("L2") blocks are left to the
 // top-k kernels, and the splits cover the blocks from its INT4 count on.
-template <int G, bool kCluster, bool kF16, bool kSkip>
+// kLsub: log2 of the 64-token sub-blocks per block (block_size 64: 0, 128: 1).
+template <int G, bool kCluster, bool kF16, bool kSkip, int kLsub>
 __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(const DecodeArgs a) {
   constexpr int P = pow2_heads<G>();
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -122,17 +123,20 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
   }
   const int H = a.hot_tokens;
   const int Lc = max(0, L - H);
-  const int nblk = (Lc + kBlock - 1) / kBlock;
+  constexpr int lsub = kLsub;        // a block is 1 << lsub sub-blocks of 64 tokens
+  const int Bt = kBlock << lsub;      // tokens per block
+  const int nblk = (Lc + Bt - 1) / Bt;
   const int Sb = max(1, (max(0, nblk - ib) + a.split_blocks - 1) / a.split_blocks);
   // past this sequence's last split: no work and no partial (a cluster member
   // still takes part in the cluster's merge, with an empty state)
   if (!kCluster && s >= Sb) return;
   const int ncold = max(0, min(nblk, i0 + a.split_blocks) - i0);
-  // FP16 rows (the hot ring, FP16 cold blocks) are items of up to 32 rows;
-  // FP16 cold blocks (quantization_bits 0) are two items each
+  // Items: one per 64-token sub-block (16 KB K + V tiles), or per 32 rows of
+  // FP16 (the hot ring, FP16 cold blocks: 2 << lsub items per block)
   const int nhot = (s == Sb - 1) ? min(L, H) : 0;
   constexpr bool fp16 = kF16;
-  const int ncold_it = fp16 ? 2 * ncold : ncold;
+  const int ish = (fp16 ? 1 : 0) + lsub;  // log2 of the items per block
+  const int ncold_it = ncold << ish;
   const int kh = ncold_it;  // the first hot item
   const int nitems = ncold_it + (nhot + kItemRows - 1) / kItemRows;
   // fused step, in the split that holds the tail block and the hot ring: the
@@ -143,7 +147,21 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
   const bool do_seal = do_ring && L_old >= H;
   const int rs = L_old & (H - 1);
   const int k_ring = kh + rs / kItemRows;
-  const int k_seal = !do_seal ? -1 : fp16 ? 2 * (ncold - 1) + ((L_old - H) % kBlock) / kItemRows : ncold - 1;
+  // slot of the sealed token in the tail block; in the split that seals, the
+  // tail block's sub-blocks run last-first, so that a scale the seal grows
+  // reaches the earlier sub-block before that one is attended (k_rq)
+  const int slot_e = do_seal ? (L_old - H) % Bt : 0;
+  const int nsub1 = (1 << lsub) - 1;
+  const int k_seal = !do_seal ? -1
+                     : fp16   ? ((ncold - 1) << ish) + slot_e / kItemRows
+                              : ((ncold - 1) << lsub) + nsub1 - (slot_e >> 6);
+  const int k_rq = (!fp16 && do_seal && (slot_e >> 6) > 0) ? ((ncold - 1) << lsub) + nsub1 : -1;
+  // item k: its block, and (cold INT8/INT4 items) its sub-block
+  auto item_block = [&](int k) { return k >> ish; };
+  auto item_sub = [&](int k) {
+    const int part = k & ((1 << ish) - 1);
+    return (do_seal && (k >> ish) == ncold - 1) ? nsub1 - part : part;
+  };
   __half2 new_kv = __halves2half2(__float2half_rn(0.f), __float2half_rn(0.f));
   __half2 old_kv = new_kv;
   if (do_ring) {
@@ -186,23 +204,26 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
     const int st = k % kStages;
     uint8_t *dst = sm.ring[st];
     if (k < ncold_it) {
-      const int kb = fp16 ? k >> 1 : k;
+      const int kb = item_block(k);
       const int phys = sm.phys[kb];
-      const int nrow = fp16 ? min(kItemRows, Lc - (i0 + kb) * kBlock - (k & 1) * kItemRows) : 1;
+      const int part = k & ((1 << ish) - 1);
+      const int u = fp16 ? 0 : item_sub(k);
+      const int nrow = fp16 ? min(kItemRows, Lc - (i0 + kb) * Bt - part * kItemRows)
+                            : Lc - (i0 + kb) * Bt - u * kBlock;
       if (phys < 0 || nrow <= 0) {
         mbar_arrive(&sm.full[st]);
         return;
       }
       if (fp16) {
-        // the half block's sealed rows
-        const uint8_t *src = a.cold + ((size_t)phys * a.hkv + h) * kFp16BlockBytes + (k & 1) * kItemBytes;
+        // 32 of the block's sealed rows
+        const uint8_t *src = a.cold + ((size_t)phys * a.hkv + h) * (kFp16BlockBytes << lsub) + part * kItemBytes;
         const uint32_t bytes = static_cast<uint32_t>(nrow) * kHotTokenBytes;
         mbar_arrive_expect_tx(&sm.full[st], bytes);
         bulk_g2s(dst, src, bytes, &sm.full[st], pol);
         return;
       }
-      const uint8_t *src = a.cold + ((size_t)phys * a.hkv + h) * kTilePairBytes;
-      if (i0 + k >= n_int4_b) {
+      const uint8_t *src = a.cold + ((((size_t)phys * a.hkv + h) << lsub) + u) * kTilePairBytes;
+      if (i0 + kb >= n_int4_b) {
         mbar_arrive_expect_tx(&sm.full[st], kTilePairBytes);
         bulk_g2s(dst, src, kTilePairBytes, &sm.full[st], pol);
       } else {
@@ -285,16 +306,19 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
     }
     bool ok = mbar_wait_bounded(&sm.full[st], (k / kStages) & 1, kWaitCycles);
     if (!ok && lane == 0) set_status(a.status, HYB_STATUS_TIMEOUT);
-    if (k == k_seal || (do_ring && k == k_ring)) {
+    if (k == k_seal || k == k_rq || (do_ring && k == k_ring)) {
       // ---------------- fused append (whole CTA, in the staged copies) ----------------
       ok = __syncthreads_and(ok) != 0;
+      const int tb = ncold - 1;  // the tail block
       if (ok && k == k_seal) {
-        const int tb = ncold - 1;  // the tail block
         if (fp16)
           fused_seal_fp16(sm.seal, sm.ring[st], sm.phys[tb] * a.hkv + h, a, L_old, true, tid);
         else
           fused_seal(sm.seal, sm.ring[st], &sm.scl[tb], sm.phys[tb] * a.hkv + h, (i0 + tb) < n_int4_b, a, L_old,
                      true, tid, warp, lane);
+      } else if (ok && k == k_rq) {
+        if (sm.phys[tb] >= 0)
+          requant_staged(sm.seal, sm.ring[st], (sm.phys[tb] * a.hkv + h) << lsub, (i0 + tb) < n_int4_b, a, tid);
       } else if (ok) {
         ring_put(sm.ring[st], rs, new_kv, a, b, h, tid);
       }
@@ -304,14 +328,17 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
     // rows of an FP16 item: the hot ring, or half of an FP16 cold block
     int nrow = min(kItemRows, nhot - (k - kh) * kItemRows);
     if (k < ncold_it)
-      nrow = !fp16 || sm.phys[k >> 1] < 0 ? 0 : min(kItemRows, Lc - (i0 + (k >> 1)) * kBlock - (k & 1) * kItemRows);
-    if (ok && !fp16 && k < ncold) {
-      // ---------------- cold block ----------------
-      const int i = i0 + k;
-      const int nvalid = sm.phys[k] < 0 ? 0 : min(kBlock, Lc - i * kBlock);
+      nrow = !fp16 || sm.phys[item_block(k)] < 0
+                 ? 0
+                 : min(kItemRows, Lc - (i0 + item_block(k)) * Bt - (k & ((1 << ish) - 1)) * kItemRows);
+    if (ok && !fp16 && k < ncold_it) {
+      // ---------------- cold sub-block (64 tokens) ----------------
+      const int kb = item_block(k);
+      const int i = i0 + kb;
+      const int nvalid = sm.phys[kb] < 0 ? 0 : min(kBlock, Lc - i * Bt - item_sub(k) * kBlock);
       const int nv = nvalid - 16 * warp;
       const bool int4 = i < n_int4_b;
-      const float2 sc = sm.scl[k];
+      const float2 sc = sm.scl[kb];
       const float coef = sq_hd * sc.x * a.qk_scale;
       if (nvalid == kBlock && !int4) {
         cold_block_full<G, P>(stage, k_lane, v_lane, qp, coef, sc.y * (1.f / 32767.f), sm.pcode[warp], hx, tg,
@@ -456,19 +483,19 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
 // Largest cluster the decode kernel is launched with (portable size).
 constexpr int kMaxCluster = 8;
 
-template <int G, bool kF16, bool kSkip>
+template <int G, bool kF16, bool kSkip, int kLsub>
 static cudaError_t launch_decode_g(const DecodeArgs &a, int batch, bool cluster, cudaStream_t stream) {
   const size_t smem = sizeof(DecodeSmem<G>);
-  static int configured_dev_mask = 0;  // one bit per device
+  static int configured_dev_mask = 0;  // one bit per device (per instantiation)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 31 && !(configured_dev_mask & (1 << dev))) {
-    e = cudaFuncSetAttribute(decode_kernel<G, false, kF16, kSkip>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
+    e = cudaFuncSetAttribute(decode_kernel<G, false, kF16, kSkip, kLsub>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(decode_kernel<G, true, kF16, kSkip>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
+      e = cudaFuncSetAttribute(decode_kernel<G, true, kF16, kSkip, kLsub>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     configured_dev_mask |= 1 << dev;
   }
@@ -486,33 +513,39 @@ static cudaError_t launch_decode_g(const DecodeArgs &a, int batch, bool cluster,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_kernel<G, true, kF16, kSkip>, a);
+    e = cudaLaunchKernelEx(&cfg, decode_kernel<G, true, kF16, kSkip, kLsub>, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
-  decode_kernel<G, false, kF16, kSkip><<<grid, kThreads, smem, stream>>>(a);
+  decode_kernel<G, false, kF16, kSkip, kLsub><<<grid, kThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
-template <bool kF16, bool kSkip>
+template <bool kF16, bool kSkip, int kLsub>
 static cudaError_t launch_decode_f(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream) {
   switch (group) {
-    case 1: return launch_decode_g<1, kF16, kSkip>(a, batch, cluster, stream);
-    case 2: return launch_decode_g<2, kF16, kSkip>(a, batch, cluster, stream);
-    case 3: return launch_decode_g<3, kF16, kSkip>(a, batch, cluster, stream);
-    case 4: return launch_decode_g<4, kF16, kSkip>(a, batch, cluster, stream);
-    case 5: return launch_decode_g<5, kF16, kSkip>(a, batch, cluster, stream);
-    case 6: return launch_decode_g<6, kF16, kSkip>(a, batch, cluster, stream);
-    case 7: return launch_decode_g<7, kF16, kSkip>(a, batch, cluster, stream);
-    case 8: return launch_decode_g<8, kF16, kSkip>(a, batch, cluster, stream);
+    case 1: return launch_decode_g<1, kF16, kSkip, kLsub>(a, batch, cluster, stream);
+    case 2: return launch_decode_g<2, kF16, kSkip, kLsub>(a, batch, cluster, stream);
+    case 3: return launch_decode_g<3, kF16, kSkip, kLsub>(a, batch, cluster, stream);
+    case 4: return launch_decode_g<4, kF16, kSkip, kLsub>(a, batch, cluster, stream);
+    case 5: return launch_decode_g<5, kF16, kSkip, kLsub>(a, batch, cluster, stream);
+    case 6: return launch_decode_g<6, kF16, kSkip, kLsub>(a, batch, cluster, stream);
+    case 7: return launch_decode_g<7, kF16, kSkip, kLsub>(a, batch, cluster, stream);
+    case 8: return launch_decode_g<8, kF16, kSkip, kLsub>(a, batch, cluster, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
+template <int kLsub>
+static cudaError_t launch_decode_l(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream) {
+  if (a.quant_bits == 0) return launch_decode_f<true, false, kLsub>(a, group, batch, cluster, stream);
+  if (a.l2_skip) return launch_decode_f<false, true, kLsub>(a, group, batch, cluster, stream);
+  return launch_decode_f<false, false, kLsub>(a, group, batch, cluster, stream);
+}
+
 cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream) {
-  if (a.quant_bits == 0) return launch_decode_f<true, false>(a, group, batch, cluster, stream);
-  if (a.l2_skip) return launch_decode_f<false, true>(a, group, batch, cluster, stream);
-  return launch_decode_f<false, false>(a, group, batch, cluster, stream);
+  return a.lsub ? launch_decode_l<1>(a, group, batch, cluster, stream)
+                : launch_decode_l<0>(a, group, batch, cluster, stream);
 }
 
 int decode_max_cluster() { return kMaxCluster; }
@@ -535,10 +568,10 @@ int decode_ctas_per_sm(int group) {
   switch (group) {
 #define HYB_OCC(g)                                                                          \
   case g:                                                                                   \
-    e = cudaFuncSetAttribute(decode_kernel<g, false, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+    e = cudaFuncSetAttribute(decode_kernel<g, false, false, false, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              static_cast<int>(sizeof(DecodeSmem<g>)));                      \
     if (e == cudaSuccess)                                                                   \
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<g, false, false, false>, kThreads, \
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<g, false, false, false, 0>, kThreads, \
                                                         sizeof(DecodeSmem<g>));             \
     break;
     HYB_OCC(1) HYB_OCC(2) HYB_OCC(3) HYB_OCC(4) HYB_OCC(5) HYB_OCC(6) HYB_OCC(7) HYB_OCC(8)

@@ -89,10 +89,13 @@ struct SealScratch {
 };
 
 // Fused decode step, seal half: the token leaving the hot zone (position e =
-// L_old - hot, its FP16 rows in ss.erow) is quantized into slot e % 64 of the
-// tail block, inside the staged copy of that block (tile_st, scales
-// *scl_tail, so that this attention sees it) and in the cache (tile index
-// tile_tail = physical block * Hkv + kv head).  Same arithmetic as
+// L_old - hot, its FP16 rows in ss.erow) is quantized into its slot of the
+// tail block (slot e % block of the block: slot e % 64 of sub-block
+// (e % block) / 64), inside the staged copy of that sub-block (tile_st,
+// scales *scl_tail, so that this attention sees it) and in the cache
+// (tile_tail = physical block * Hkv + kv head).  A grown scale re-quantizes
+// the staged sub-block here and an earlier sub-block of the block in
+// requant_staged.  Same arithmetic as
 // hyb_kv_append: absmax scale, a grown scale re-quantizes the codes already
 // in the block, RNE codes.  Called by the whole CTA.
 __device__ __forceinline__ void fused_seal(SealScratch &ss, uint8_t *tile_st, float2 *scl_tail, int tile_tail,
@@ -105,7 +108,8 @@ __device__ __forceinline__ void fused_seal(SealScratch &ss, uint8_t *tile_st, fl
   do_seal = do_seal && tile_tail >= 0;
   if (!do_seal) return;
   const int e = L_old - a.hot_tokens;  // position sealed
-  const int slot = e % kBlock;
+  const int slot_b = e % (kBlock << a.lsub);  // its slot in the block
+  const int slot = slot_b & (kBlock - 1);     // ... and in its sub-block
   const bool int4 = int4_tail;
   const int Q = int4 ? 7 : 127;
   if (warp < 2) {
@@ -121,7 +125,7 @@ __device__ __forceinline__ void fused_seal(SealScratch &ss, uint8_t *tile_st, fl
     const float s_old = kv ? scl_tail->y : scl_tail->x;
     float s_new = s_c;
     int rq = 0;
-    if (slot != 0) {
+    if (slot_b != 0) {
       if (s_c > s_old) rq = 1;
       else s_new = s_old;
     }
@@ -171,7 +175,7 @@ __device__ __forceinline__ void fused_seal(SealScratch &ss, uint8_t *tile_st, fl
   {
     // write back what changed in the tail block: scales, then the whole tile
     // if its codes were re-quantized, else the sealed token's codes
-    uint8_t *gtile = a.cold + (size_t)tile_tail * kTilePairBytes;
+    uint8_t *gtile = a.cold + ((static_cast<size_t>(tile_tail) << a.lsub) + (slot_b >> 6)) * kTilePairBytes;
     if (tid < 2) a.scales[(size_t)tile_tail * 2 + tid] = ss.seal_s[tid];
 #pragma unroll
     for (int kv = 0; kv < 2; kv++) {
@@ -202,15 +206,42 @@ __device__ __forceinline__ void fused_seal(SealScratch &ss, uint8_t *tile_st, fl
 __device__ __forceinline__ void fused_seal_fp16(const SealScratch &ss, uint8_t *row_st, int tile_tail,
                                                 const DecodeArgs &a, int L_old, bool do_seal, int tid) {
   if (!do_seal || tile_tail < 0) return;
-  const int slot = (L_old - a.hot_tokens) % kBlock;
+  const int slot = (L_old - a.hot_tokens) % (kBlock << a.lsub);
   const int c = tid;
   const __half k_old = ss.erow[c], v_old = ss.erow[kDim + c];
   __half *trow = reinterpret_cast<__half *>(row_st + (slot % kItemRows) * kHotTokenBytes);
   trow[c] = k_old;
   trow[kDim + c] = v_old;
-  __half *grow = reinterpret_cast<__half *>(a.cold + (size_t)tile_tail * kFp16BlockBytes + slot * kHotTokenBytes);
+  __half *grow = reinterpret_cast<__half *>(a.cold + (size_t)tile_tail * (kFp16BlockBytes << a.lsub) +
+                                            slot * kHotTokenBytes);
   grow[c] = k_old;
   grow[kDim + c] = v_old;
+  __syncthreads();
+}
+
+// Fused decode step, 128-token blocks: the seal landed in the block's second
+// sub-block and grew the block's scale -- the first sub-block's codes (all 64
+// slots, staged in tile_st) are re-quantized with the seal's tables, for this
+// attention and in the cache (sub-block pair index pair0 = (physical block *
+// Hkv + kv head) * 2).  Called by the whole CTA after fused_seal.
+__device__ __forceinline__ void requant_staged(const SealScratch &ss, uint8_t *tile_st, int pair0, bool int4,
+                                               const DecodeArgs &a, int tid) {
+#pragma unroll
+  for (int kv = 0; kv < 2; kv++) {
+    if (!ss.seal_rq[kv]) continue;
+    uint32_t *w32 = reinterpret_cast<uint32_t *>(tile_st + kv * kTileBytes);
+    const int nw = requant_nwords(kv, int4, kBlock);
+    for (int w = tid; w < nw; w += kThreads) w32[w] = requant_word(w32[w], w, kv, int4, kBlock, ss.rqt[kv]);
+  }
+  __syncthreads();
+  uint8_t *g = a.cold + (size_t)pair0 * kTilePairBytes;
+#pragma unroll
+  for (int kv = 0; kv < 2; kv++) {
+    if (!ss.seal_rq[kv]) continue;
+    const int nvec = (int4 ? kTileBytes / 2 : kTileBytes) / 16;
+    for (int v = tid; v < nvec; v += kThreads)
+      reinterpret_cast<uint4 *>(g + kv * kTileBytes)[v] = reinterpret_cast<const uint4 *>(tile_st + kv * kTileBytes)[v];
+  }
   __syncthreads();
 }
 

@@ -63,6 +63,9 @@ const char *hyb_strerror(int code) {
   }
 }
 
+// log2 of the 64-token sub-blocks per block (block_size 64: 0, 128: 1)
+static int lsub_of(const hyb_cache_desc *d) { return d->block_size == 2 * hyb::kBlock ? 1 : 0; }
+
 int hyb_check_desc(const hyb_cache_desc *d) {
   if (!d) return HYB_ERR_INVALID_VALUE;
   // hybrid_v2 contract (page sections 3.1 / 5.1)
@@ -83,7 +86,7 @@ int hyb_check_desc(const hyb_cache_desc *d) {
       (d->n_int4_blocks && !aligned(d->n_int4_blocks, 4)))
     return HYB_ERR_INVALID_VALUE;
   // what this library builds
-  if (d->block_size != hyb::kBlock || d->head_dim != hyb::kDim)
+  if ((d->block_size != hyb::kBlock && d->block_size != 2 * hyb::kBlock) || d->head_dim != hyb::kDim)
     return HYB_ERR_UNSUPPORTED;
   if (d->num_q_heads / d->num_kv_heads > 8) return HYB_ERR_UNSUPPORTED;
   return HYB_OK;
@@ -113,6 +116,7 @@ int hyb_kv_append(const hyb_cache_desc *d, const int32_t *n_new, int32_t max_new
   a.quant_bits = d->quant_bits;
   a.max_new = max_new;
   a.hot_tokens = d->hot_tokens;
+  a.lsub = lsub_of(d);
   const cudaError_t e = hyb::launch_append(a, d->batch, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HYB_OK : cuda_fail(e);
 }
@@ -140,7 +144,7 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
   if (rc != HYB_OK) return rc;
   if (max_seq_len < 0) return HYB_ERR_INVALID_VALUE;
   const long long nblk = (static_cast<long long>(max_seq_len) - d->hot_tokens > 0)
-                             ? (max_seq_len - d->hot_tokens + hyb::kBlock - 1) / hyb::kBlock
+                             ? (max_seq_len - d->hot_tokens + d->block_size - 1) / d->block_size
                              : 0;
   if (nblk > d->max_blocks_per_seq) return HYB_ERR_INVALID_VALUE;
   const int group = d->num_q_heads / d->num_kv_heads;
@@ -167,8 +171,8 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
       if (tb > nblk) tb = nblk > 0 ? nblk : 1;
     }
   } else {
-    if (split_tokens < 0 || split_tokens % hyb::kBlock != 0) return HYB_ERR_INVALID_VALUE;
-    tb = split_tokens / hyb::kBlock;
+    if (split_tokens < 0 || split_tokens % d->block_size != 0) return HYB_ERR_INVALID_VALUE;
+    tb = split_tokens / d->block_size;
     if (tb < 1) return HYB_ERR_INVALID_VALUE;
   }
   long long ns = (nblk + tb - 1) / tb;
@@ -244,7 +248,7 @@ int hyb_decode_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_
   Plan pl;
   const int rc = make_plan(d, max_seq_len, split_tokens, &pl);
   if (rc != HYB_OK) return rc;
-  if (split_tokens_out) *split_tokens_out = pl.tb * hyb::kBlock;
+  if (split_tokens_out) *split_tokens_out = pl.tb * d->block_size;
   if (n_splits_out) *n_splits_out = pl.ns;
   return HYB_OK;
 }
@@ -297,6 +301,7 @@ static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_s
   a.max_blocks = d->max_blocks_per_seq;
   a.quant_bits = d->quant_bits;
   a.hot_tokens = d->hot_tokens;
+  a.lsub = lsub_of(d);
   a.n_splits = pl.ns;
   a.split_blocks = pl.tb;
   a.max_seq_len = max_seq_len;
@@ -379,6 +384,7 @@ int hyb_decode_attn_sparse(const hyb_cache_desc *d, const void *q, float softmax
   a.max_blocks = d->max_blocks_per_seq;
   a.quant_bits = d->quant_bits;
   a.hot_tokens = d->hot_tokens;
+  a.lsub = lsub_of(d);
   a.max_l2 = w.max_l2;
   a.top_k = top_k;
   a.blocks_per_cta = 4;
@@ -443,6 +449,7 @@ int hyb_kv_migrate(const hyb_cache_desc *d, const int32_t *target_n_int4, int32_
   a.max_blocks = d->max_blocks_per_seq;
   a.max_delta = max_delta;
   a.hot_tokens = d->hot_tokens;
+  a.lsub = lsub_of(d);
   const cudaError_t e = hyb::launch_migrate(a, d->batch, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HYB_OK : cuda_fail(e);
 }

@@ -10,7 +10,7 @@ namespace hyb {
 
 struct AppendArgs {
   __half *hot;                // FP16 [batch][Hkv][hot][2][128]
-  uint8_t *cold;              // [num_phys][Hkv][2][8192] (quant_bits 0: FP16 [num_phys][Hkv][64][2][128])
+  uint8_t *cold;              // [num_phys][Hkv][sub][2][8192] (quant_bits 0: FP16 [num_phys][Hkv][block][2][128])
   float *scales;              // [num_phys][Hkv][2]
   const int32_t *block_table; // [batch][max_blocks]
   int32_t *seq_lens;          // [batch]
@@ -21,6 +21,7 @@ struct AppendArgs {
   const __half *v_new;
   int hkv, num_phys, max_blocks, quant_bits, max_new;
   int hot_tokens;             // hot-zone tokens (power of two, 16..128)
+  int lsub;                   // log2 of the 64-token sub-blocks per block (block_size 64: 0, 128: 1)
 };
 
 struct DecodeArgs {
@@ -46,6 +47,7 @@ struct DecodeArgs {
   int n_groups;
   int hkv, hq, num_phys, max_blocks, quant_bits, n_splits, split_blocks, max_seq_len;
   int hot_tokens;             // hot-zone tokens (power of two, 16..128)
+  int lsub;                   // log2 of the 64-token sub-blocks per block
   float qk_scale;             // softmax_scale * log2(e)
   // fused decode step (null for attention only): append n_new[b] in {0, 1}
   // tokens first; k_new / v_new FP16 [batch][Hkv][128]; seq_cnt [batch]
@@ -69,6 +71,7 @@ struct MigrateArgs {
   int32_t *status;
   int hkv, num_phys, max_blocks, max_delta;
   int hot_tokens;             // hot-zone tokens
+  int lsub;                   // log2 of the 64-token sub-blocks per block
 };
 
 // Sparse L2 attention (top-k of the INT4-block tokens per query head).
@@ -84,6 +87,7 @@ struct SparseArgs {
   __half *out;                // FP16 [batch][Hq][128]: the dense pass's result in, the merged result out
   float *lse;                 // [batch][Hq]: the dense pass's log-sum-exp in, merged out (natural log)
   int hkv, hq, num_phys, max_blocks, quant_bits, hot_tokens, max_l2, top_k, blocks_per_cta;
+  int lsub;                   // log2 of the 64-token sub-blocks per block
   float qk_scale;             // softmax_scale * log2(e)
 };
 

@@ -14,18 +14,19 @@
 // -- the arithmetic of a tail block's re-quantization in hyb_kv_append, so the
 // result is bit-exact with the oracle.
 //
-// One CTA per (block to move, kv head, sequence): each thread holds its part
-// of the K and V tiles in registers (codes of slots not yet sealed are taken
-// as 0), the new scale and a 256-entry code table are computed, and the
-// tiles are written back in the new packing (a demoted tile's unused upper
-// 4 KB is zeroed).  A second launch then commits the new counts, after every CTA of
+// One CTA per (block to move, kv head, sequence), 256 threads per 64-token
+// sub-block of the block (512 for 128-token blocks, whose two sub-blocks
+// share the scale): each thread holds its part of the K and V tiles in
+// registers (codes of slots not yet sealed are taken as 0), the new scale
+// and a 256-entry code table are computed, and the tiles are written back in
+// the new packing (a demoted tile's unused upper 4 KB is zeroed).  A second launch then commits the new counts, after every CTA of
 // the first has read the old ones.
 #include "kernels.cuh"
 
 namespace hyb {
 
-constexpr int kMigThreads = 256;
-constexpr int kMigWarps = kMigThreads / 32;
+constexpr int kMigThreads = 256;               // per 64-token sub-block
+constexpr int kMigWarpsMax = 2 * kMigThreads / 32;  // 128-token blocks
 
 // The sequence's move, or false (sequence left as it is) when the target is
 // outside [0, max_blocks] or farther than max_delta from the current count.
@@ -55,31 +56,35 @@ __device__ __forceinline__ uint32_t absmax4(uint32_t x) {
   return max(max(a & 0xff, (a >> 8) & 0xff), max((a >> 16) & 0xff, a >> 24));
 }
 
-__global__ void __launch_bounds__(kMigThreads) migrate_kernel(const MigrateArgs a) {
+__global__ void __launch_bounds__(2 * kMigThreads) migrate_kernel(const MigrateArgs a) {
   const int k = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid_all = threadIdx.x, lane = tid_all & 31, warp = tid_all >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const int u = tid_all / kMigThreads;    // this thread's sub-block
+  const int tid = tid_all % kMigThreads;  // ... and its index there
+  const int Bt = kBlock << a.lsub;
   int lo, hi, tgt;
   if (!tier_move(a, b, lo, hi, tgt)) {
-    if (k == 0 && h == 0 && tid == 0) set_status(a.status, HYB_STATUS_BAD_TIER);
+    if (k == 0 && h == 0 && tid_all == 0) set_status(a.status, HYB_STATUS_BAD_TIER);
     return;
   }
   const int i = lo + k;
   if (i >= hi) return;
   const int Lc = max(0, a.seq_lens[b] - a.hot_tokens);
-  if (i * kBlock >= Lc) return;  // nothing sealed in this block yet: only its tier changes
-  const int sealed = min(kBlock, Lc - i * kBlock);
+  if (i * Bt >= Lc) return;  // nothing sealed in this block yet: only its tier changes
+  const int sealed = max(0, min(kBlock, Lc - i * Bt - u * kBlock));  // in this sub-block
   const int phys = a.block_table[(size_t)b * a.max_blocks + i];
   if (phys < 0 || phys >= a.num_phys) {
-    if (tid == 0) set_status(a.status, HYB_STATUS_BAD_BLOCK);
+    if (tid_all == 0) set_status(a.status, HYB_STATUS_BAD_BLOCK);
     return;
   }
   const bool demote = i < tgt;  // INT8 -> INT4
   const int qn = demote ? 7 : 127;
 
-  __shared__ int red[2][kMigWarps];
+  __shared__ int red[2][kMigWarpsMax];
   __shared__ float s_new[2];
   __shared__ uint8_t tbl[2][256];
-  uint8_t *tile = a.cold + ((size_t)phys * a.hkv + h) * kTilePairBytes;
+  uint8_t *tile = a.cold + ((((size_t)phys * a.hkv + h) << a.lsub) + u) * kTilePairBytes;
 
   // Every packed word maps onto a local piece of the other packing, so each
   // thread keeps its part of both tiles in registers, as INT8 bytes:
@@ -153,22 +158,22 @@ __global__ void __launch_bounds__(kMigThreads) migrate_kernel(const MigrateArgs 
     if (lane == 0) red[kv][warp] = static_cast<int>(m);
   }
   __syncthreads();
-  if (tid < 2) {
+  if (tid_all < 2) {
+    const int kvr = tid_all;
     int m = 0;
-#pragma unroll
-    for (int w = 0; w < kMigWarps; w++) m = max(m, red[tid][w]);
+    for (int w = 0; w < nwarps; w++) m = max(m, red[kvr][w]);
     m = min(m, 127);
-    const float s_old = a.scales[((size_t)phys * a.hkv + h) * 2 + tid];
-    s_new[tid] = __fdiv_rn(__fmul_rn(static_cast<float>(m), s_old), static_cast<float>(qn));
+    const float s_old = a.scales[((size_t)phys * a.hkv + h) * 2 + kvr];
+    s_new[kvr] = __fdiv_rn(__fmul_rn(static_cast<float>(m), s_old), static_cast<float>(qn));
   }
   __syncthreads();
-  for (int e = tid; e < 2 * 256; e += kMigThreads) {
-    const int kv = e >> 8, u = e & 255;
-    const int c = u == 255 ? -127 : u - 127;
+  for (int e = tid_all; e < 2 * 256; e += blockDim.x) {
+    const int kv = e >> 8, ue = e & 255;
+    const int c = ue == 255 ? -127 : ue - 127;
     const float s_old = a.scales[((size_t)phys * a.hkv + h) * 2 + kv];
     const int cn = s_new[kv] == 0.f ? 0 : requantize(c, s_old, s_new[kv], qn);
     // INT4: the nibble; INT8: the byte
-    tbl[kv][u] = static_cast<uint8_t>(demote ? (cn & 0xf) : (cn & 0xff));
+    tbl[kv][ue] = static_cast<uint8_t>(demote ? (cn & 0xf) : (cn & 0xff));
   }
   __syncthreads();  // every thread has read the old scales and its tile words
 
@@ -204,7 +209,7 @@ __global__ void __launch_bounds__(kMigThreads) migrate_kernel(const MigrateArgs 
     for (int kv = 0; kv < 2; kv++)
       reinterpret_cast<uint4 *>(tile + kv * kTileBytes + kTileBytes / 2)[tid] = make_uint4(0u, 0u, 0u, 0u);
   }
-  if (tid < 2) a.scales[((size_t)phys * a.hkv + h) * 2 + tid] = s_new[tid];
+  if (tid_all < 2) a.scales[((size_t)phys * a.hkv + h) * 2 + tid_all] = s_new[tid_all];
 }
 
 // The new counts, once every CTA of migrate_kernel has read the old ones.
@@ -218,7 +223,7 @@ __global__ void migrate_commit_kernel(const MigrateArgs a, int batch) {
 cudaError_t launch_migrate(const MigrateArgs &a, int batch, cudaStream_t stream) {
   if (a.max_delta > 0) {
     dim3 grid(a.max_delta, a.hkv, batch);
-    migrate_kernel<<<grid, kMigThreads, 0, stream>>>(a);
+    migrate_kernel<<<grid, kMigThreads << a.lsub, 0, stream>>>(a);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

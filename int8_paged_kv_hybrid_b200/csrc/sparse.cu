@@ -33,7 +33,7 @@ __device__ __forceinline__ int l2_count(const SparseArgs &a, int b) {
   if (L < 0) return 0;
   const int Lc = max(0, L - a.hot_tokens);
   const long long n4 = a.quant_bits == 4 ? a.max_blocks : (a.n_int4 ? a.n_int4[b] : 0);
-  const long long n = min(static_cast<long long>(Lc), max(0LL, n4) * kBlock);
+  const long long n = min(static_cast<long long>(Lc), max(0LL, n4) * (kBlock << a.lsub));
   return n > a.max_l2 ? -1 : static_cast<int>(n);
 }
 
@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(kScoreThreads) l2_score_kernel(const SparseArg
   const int G = a.hq / a.hkv;
   const int n = l2_count(a, b);
   if (n <= 0) return;
+  // units of 64 tokens (sub-blocks; a block is 1 << lsub of them)
   const int nb = (n + kBlock - 1) / kBlock;
   const int blk0 = chunk * a.blocks_per_cta;
   if (blk0 >= nb) return;
@@ -89,12 +90,14 @@ __global__ void __launch_bounds__(kScoreThreads) l2_score_kernel(const SparseArg
     stage[t][0] = make_uint4(0u, 0u, 0u, 0u);
     stage[t][1] = stage[t][0];
     if (t < nblk) {
-      const int phys = a.block_table[(size_t)b * a.max_blocks + blk0 + t];
+      const int unit = blk0 + t;
+      const int phys = a.block_table[(size_t)b * a.max_blocks + (unit >> a.lsub)];
       const bool okp = phys >= 0 && phys < a.num_phys;
       if (tid == 0) s_phys[t] = okp ? phys : -1;
       if (!okp && tid == 0) set_status(a.status, HYB_STATUS_BAD_BLOCK);
       if (okp) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.cold + ((size_t)phys * a.hkv + h) * kTilePairBytes);
+        const size_t pair = (((size_t)phys * a.hkv + h) << a.lsub) + (unit & ((1 << a.lsub) - 1));
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.cold + pair * kTilePairBytes);
         stage[t][0] = src[tid];
         stage[t][1] = src[kScoreThreads + tid];
       }
@@ -354,11 +357,12 @@ __global__ void __launch_bounds__(kT) l2_topk_kernel(const SparseArgs a) {
   float zmax = -INFINITY;
   for (int j = tid; j < ns; j += kTopkThreads) {
     const int pos = s_pos[j];
-    const int phys = a.block_table[(size_t)b * a.max_blocks + pos / kBlock];
+    const int phys = a.block_table[(size_t)b * a.max_blocks + (pos / (kBlock << a.lsub))];
     const bool okp = phys >= 0 && phys < a.num_phys;
     const float z = keys[pos] * coef;
     s_p[j] = z;
-    s_vt[j] = okp ? (phys * a.hkv + h) : -1;
+    // the sub-block pair holding pos
+    s_vt[j] = okp ? (((phys * a.hkv + h) << a.lsub) + ((pos / kBlock) & ((1 << a.lsub) - 1))) : -1;
     s_sv[j] = okp ? a.scales[((size_t)phys * a.hkv + h) * 2 + 1] : 0.f;
     zmax = fmaxf(zmax, z);
   }

@@ -39,18 +39,19 @@ class Workload:
     split_tokens: int = 0
     head_dim: int = HEAD_DIM
     hot_tokens: int = HOT
+    block_size: int = BLOCK
 
     @property
     def max_blocks(self) -> int:
         return self.block_table.shape[1]
 
     def cold_blocks(self) -> np.ndarray:
-        return np.array([cold_blocks_for(int(L), self.hot_tokens) for L in self.lens], np.int64)
+        return np.array([cold_blocks_for(int(L), self.hot_tokens, self.block_size) for L in self.lens], np.int64)
 
 
-def cold_blocks_for(L: int, hot: int = HOT) -> int:
+def cold_blocks_for(L: int, hot: int = HOT, block: int = BLOCK) -> int:
     """Cold blocks a sequence of L tokens occupies (the newest `hot` stay hot)."""
-    return (max(0, L - hot) + BLOCK - 1) // BLOCK
+    return (max(0, L - hot) + block - 1) // block
 
 
 def _block_table(rng, nblk: np.ndarray, pool: int) -> np.ndarray:
@@ -216,14 +217,14 @@ def kv_bytes(w: Workload, lens: Optional[np.ndarray] = None, quant_bits: int = 8
         L = int(L)
         cold = max(0, L - w.hot_tokens)
         hot = L - cold
-        nblk = (cold + BLOCK - 1) // BLOCK
+        nblk = (cold + w.block_size - 1) // w.block_size
         n4 = 0
         if quant_bits == 4:
             n4 = nblk
         elif w.n_int4 is not None and quant_bits == 8:
             n4 = min(int(w.n_int4[b]), nblk)
         # tokens in INT4 blocks (the oldest n4 blocks are always full)
-        t4 = min(cold, n4 * BLOCK)
+        t4 = min(cold, n4 * w.block_size)
         t8 = cold - t4
         if quant_bits == 0:
             total += hkv * cold * 2 * d * 2        # K + V, FP16
@@ -238,14 +239,14 @@ def kv_bytes(w: Workload, lens: Optional[np.ndarray] = None, quant_bits: int = 8
 
 def custom_workload(name, lens, num_q_heads, num_kv_heads, seed, softmax_scale=None,
                     schedule="random", chunk=64, max_step=64, pool_extra=3, n_int4=None,
-                    outliers=False, split_tokens=0, hot=HOT) -> Workload:
+                    outliers=False, split_tokens=0, hot=HOT, block=BLOCK) -> Workload:
     """A small workload with the given final lengths (for parity tests).
     schedule: "random" (U[1, max_step] tokens per call), "chunk" (prefill in
     `chunk`-token calls then one 1-token call) or "one" (a single call)."""
     rng = np.random.default_rng([seed, 0])
     lens = np.asarray(lens, np.int64)
     B = len(lens)
-    nblk = np.array([cold_blocks_for(int(L), hot) for L in lens])
+    nblk = np.array([cold_blocks_for(int(L), hot, block) for L in lens])
     pool = int(nblk.sum()) + pool_extra
     bt = _block_table(rng, nblk, pool)
     if schedule == "random":
@@ -266,7 +267,7 @@ def custom_workload(name, lens, num_q_heads, num_kv_heads, seed, softmax_scale=N
                     num_phys_blocks=pool, block_table=bt,
                     n_int4=None if n_int4 is None else np.asarray(n_int4, np.int32),
                     schedule=sched, max_new=mx, seed=seed, outlier_channels=outl,
-                    split_tokens=split_tokens, hot_tokens=hot)
+                    split_tokens=split_tokens, hot_tokens=hot, block_size=block)
 
 
 def append_bytes(w: Workload, n_new: np.ndarray, quant_bits: int = 8) -> int:

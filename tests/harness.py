@@ -11,7 +11,7 @@ MAX_REL_L2 = 1e-3
 
 def make_pair(w, quant_bits=8, gpu=True):
     ora = oracle.OracleCache(w.batch, w.num_kv_heads, w.num_q_heads, w.max_blocks, quant_bits,
-                             hot=w.hot_tokens)
+                             hot=w.hot_tokens, block=w.block_size)
     if w.n_int4 is not None:
         ora.set_n_int4(w.n_int4)
     cache = None
@@ -19,7 +19,7 @@ def make_pair(w, quant_bits=8, gpu=True):
         from int8_paged_kv_hybrid_b200 import HybridKVCache
         cache = HybridKVCache(w.batch, w.num_kv_heads, w.num_q_heads, w.num_phys_blocks, w.max_blocks,
                               quant_bits=quant_bits, block_table=w.block_table, n_int4=w.n_int4,
-                              hot_tokens=w.hot_tokens)
+                              hot_tokens=w.hot_tokens, block_size=w.block_size)
     return cache, ora
 
 
