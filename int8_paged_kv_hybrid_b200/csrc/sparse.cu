@@ -106,13 +106,18 @@ __global__ void __launch_bounds__(kScoreThreads) l2_score_kernel(const SparseArg
 #pragma unroll
   for (int t = 0; t < kMaxChunk; t++) {
     if (t < nblk) {
-      reinterpret_cast<uint4 *>(tiles[t])[tid] = stage[t][0];
-      reinterpret_cast<uint4 *>(tiles[t])[kScoreThreads + tid] = stage[t][1];
+      // 16-byte chunk c of token row r stored at chunk c ^ ((r / 2) % 4), so
+      // that the reads below spread over the banks
+#pragma unroll
+      for (int r2 = 0; r2 < 2; r2++) {
+        const int v = r2 * kScoreThreads + tid, row = v >> 2;
+        reinterpret_cast<uint4 *>(tiles[t])[row * 4 + ((v & 3) ^ ((row >> 1) & 3))] = stage[t][r2];
+      }
     }
   }
   __syncthreads();
 
-  // thread: token tok of a block, channels 64*half .. 64*half + 63
+  // thread: token tok of a block, half of its 16 words (channels 8wi..8wi+7)
   const int tok = tid >> 1, half = tid & 1;
   for (int t = 0; t < nblk; t++) {
     const int blk = blk0 + t;
@@ -126,13 +131,17 @@ __global__ void __launch_bounds__(kScoreThreads) l2_score_kernel(const SparseArg
       // channel 8w+i in the low nibble, 8w+4+i in the high nibble)
       // per word: the codes as bytes (channels 8w..8w+3, then 8w+4..8w+7)
       // against q pairs, two 16x8-bit products per dp2a, exact in int32
-      const uint32_t *kp = tiles[t] + tok * 16 + half * 8;
+      // the two threads of a token take alternate words (wi = 2w + half), so
+      // their q chunks are adjacent
+      const uint32_t *kp = tiles[t] + tok * 16;
+      const int sw = (tok >> 1) & 3;
 #pragma unroll 2
       for (int w = 0; w < 8; w++) {
-        const uint32_t word = kp[w];
+        const int wi = 2 * w + half;
+        const uint32_t word = kp[(((wi >> 2) ^ sw) << 2) + (wi & 3)];
         const int lo4 = static_cast<int>(sext_nibbles(word & 0x0f0f0f0fu));
         const int hi4 = static_cast<int>(sext_nibbles((word >> 4) & 0x0f0f0f0fu));
-        const int cb = 64 * half + 8 * w;
+        const int cb = 8 * wi;
 #pragma unroll
         for (int g = 0; g < 8; g++) {
           if (g < G) {
