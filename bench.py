@@ -92,6 +92,23 @@ def workload_config(w, split, ns, qbits=8):
             "parallelism": "replicas (independent batch per GPU)"}
 
 
+def max_over_ranks(x, world, device=None):
+    """The largest x over all ranks (each rank passes its own); x itself with
+    one rank.  A collective: every rank must call it, in the same order."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def job_throughput(bytes_per_rank, world, ms):
+    """Whole-job GB/s: what every rank processed over the slowest rank's ms."""
+    return bytes_per_rank * world / (ms * 1e-3) / 1e9
+
+
 def kernel_sha():
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
@@ -344,11 +361,7 @@ def run_native(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop() if clocks else None
-    ms_step = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
-    if world > 1:
-        t = torch.tensor([ms_step], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = t.item()
+    ms_step = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / len(evs), world, dev)
     assert torch.isfinite(out.float()).all() and cache.status() == 0
     if args.lean:
         return {"lean": True, "ms_per_step": ms_step}, w
@@ -378,18 +391,14 @@ def run_native(args, rank, world, local_rank):
     torch.cuda.synchronize()
     assert torch.equal(h_out, out.cpu())
     del g_e2e
-    ms_e2e = sum(a.elapsed_time(b) for a, b in e2e) / len(e2e)
-    if world > 1:
-        t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = t.item()
+    ms_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e) / len(e2e), world, dev)
     del g_step
 
     kvb = synth.kv_bytes(w, quant_bits=qb)
     stepb = kvb + synth.append_bytes(w, n_last, qb)
     peak, peak_kind = measured_peaks()
     total_bytes = kvb * world
-    value = total_bytes / (ms_step * 1e-3) / 1e9
+    value = job_throughput(kvb, world, ms_step)
     tokens_s = w.batch * world / (ms_step * 1e-3)
     achieved = stepb / (ms_step * 1e-3) / 1e9
     res = None
@@ -416,7 +425,7 @@ def run_native(args, rank, world, local_rank):
                          "peak_kind": peak_kind,
                          "achieved_bytes": "algorithmic bytes per launch: attention %d + append %d"
                                            % (kvb, stepb - kvb)},
-            "e2e": {"value": round(total_bytes / (ms_e2e * 1e-3) / 1e9, 1), "unit": UNIT,
+            "e2e": {"value": round(job_throughput(kvb, world, ms_e2e), 1), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(ms_e2e, 5)},
             "gpu_launches": args.steps,
