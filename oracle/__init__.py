@@ -188,8 +188,9 @@ class OracleCache:
         [num_phys][hkv][2], hot float16 [batch][hkv][hot][2][d], seq_lens int32)."""
         bt = _c(block_table, np.int32)
         assert bt.shape == (self.batch, self.max_blocks)
-        # 8 KB parts: K and V tiles per 64-slot sub-block, twice that for FP16
-        parts = (4 if self.quant_bits == 0 else 2) * (self.block // 64)
+        # 8 KB parts: K and V tiles per 64-slot sub-block (a 32-token block
+        # uses half of one); FP16 blocks: 512 B per token row
+        parts = self.block // 16 if self.quant_bits == 0 else 2 * max(1, self.block // 64)
         cold = np.zeros((num_phys, self.hkv, parts, 64 * self.d), np.uint8)
         sc = np.zeros((num_phys, self.hkv, 2), np.float32)
         hot = np.zeros((self.batch, self.hkv, self.hot, 2, self.d), np.uint16)

@@ -599,6 +599,7 @@ int ora_get_ring(const ora_cache *c, int b, uint16_t *ring) {
 /*   Blocks of 128 tokens are stored as two such 64-slot sub-blocks:   */
 /*   [num_phys][hkv][2 sub-blocks][2][8192], slot t of the block in    */
 /*   slot t%64 of sub-block t/64; the block keeps one scale per K|V.   */
+/*   Blocks of 32 tokens use slots 0..31 of one 64-slot tile pair.     */
 /*   FP16 cold blocks (quant_bits 0): cold pool bytes                  */
 /*   [num_phys][hkv][block][2][d] FP16, per token the K row then the V  */
 /*   row (the hot ring's layout), 512 B per token and kv head.          */
@@ -616,10 +617,10 @@ static void put_nibble(uint8_t *word4, int e, int code) {
 int ora_export(const ora_cache *c, const int32_t *block_table, int num_phys,
                uint8_t *cold, float *scales, uint16_t *hot, int32_t *seq_lens) {
   const int d = c->d, blk = c->block, hkv = c->hkv;
-  const size_t tile = (size_t)64 * d; /* one K or V tile of a 64-slot sub-block */
-  const int nsub = blk / 64;          /* sub-blocks per block */
-  /* format defined for d = 128 and blocks of 64 or 128 tokens */
-  if (d != 128 || (blk != 64 && blk != 128)) return ORA_ERR_INVALID;
+  const size_t tile = (size_t)64 * d;   /* one K or V tile of a 64-slot sub-block */
+  const int nsub = blk > 64 ? blk / 64 : 1; /* sub-blocks per block */
+  /* format defined for d = 128 and blocks of 32, 64 or 128 tokens */
+  if (d != 128 || (blk != 32 && blk != 64 && blk != 128)) return ORA_ERR_INVALID;
   if (c->quant_bits == 0) {
     uint16_t *cold16 = (uint16_t *)cold;
     for (int b = 0; b < c->batch; b++) {

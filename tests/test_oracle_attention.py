@@ -121,15 +121,15 @@ def test_brute_force_other_hot_sizes(hot):
         assert np.abs(lse[b] - l2).max() < 1e-12
 
 
-@pytest.mark.parametrize("qbits", [8, 4])
-def test_brute_force_128_token_blocks(qbits):
-    """block_size 128: one scale per 128 sealed tokens (the textbook absmax
-    quantizer over the whole group when it is sealed in one call), attention
-    equal to dense brute force."""
-    rng = np.random.default_rng(300 + qbits)
-    total = np.array([32 + 128, 32 + 300, 5, 0])
+@pytest.mark.parametrize("qbits,blk", [(8, 128), (4, 128), (8, 32), (4, 32)])
+def test_brute_force_other_block_sizes(qbits, blk):
+    """block_size 128 / 32: one scale per block of sealed tokens (the textbook
+    absmax quantizer over the whole group when it is sealed in one call),
+    attention equal to dense brute force."""
+    rng = np.random.default_rng(300 + qbits + blk)
+    total = np.array([32 + blk, 32 + 300, 5, 0])
     B, hkv, g = len(total), 2, 4
-    oc = oracle.OracleCache(B, hkv, hkv * g, max_blocks_per_seq=3, quant_bits=qbits, block=128)
+    oc = oracle.OracleCache(B, hkv, hkv * g, max_blocks_per_seq=300 // blk + 1, quant_bits=qbits, block=blk)
     k = rng.standard_normal((B, 332, hkv, D)).astype(np.float16)
     v = rng.standard_normal((B, 332, hkv, D)).astype(np.float16)
     oc.append(total.astype(np.int32), k, v)
@@ -138,11 +138,11 @@ def test_brute_force_128_token_blocks(qbits):
     _, codes, sc = oc.get_block(0, 0)
     for h in range(hkv):
         for kv, x in ((0, k), (1, v)):
-            grp = x[0, :128, h].astype(np.float32)
+            grp = x[0, :blk, h].astype(np.float32)
             s = np.float32(np.abs(grp).max()) / np.float32(Q)
             assert sc[h, kv] == s
             want = np.clip(np.rint(grp / s), -Q, Q)
-            assert np.array_equal(codes[h, kv, :128], want)
+            assert np.array_equal(codes[h, kv, :blk], want)
     q = rng.standard_normal((B, hkv * g, D)).astype(np.float16)
     out, lse = oc.decode(q, 0.088, nthreads=2)
     for b in range(B):

@@ -233,3 +233,33 @@ def test_export_128_token_blocks_as_two_sub_blocks():
             for ch in (0, 5, 77, 127):
                 off = ch * 64 + (((s // 16) ^ ((ch // 2) % 4)) * 16) + s % 16
                 assert np.array_equal(vt[:, off], codes[:, 1, t, ch])
+
+
+def test_export_32_token_blocks_in_half_a_tile():
+    """block_size 32 in the device format: a block uses slots 0..31 of one
+    64-slot K/V tile pair (16 KB per block and kv head); one scale pair per
+    32 tokens; slots 32..63 stay untouched."""
+    rng = np.random.default_rng(13)
+    L = 32 + 80
+    oc = oracle.OracleCache(1, 1, 1, max_blocks_per_seq=3, quant_bits=8, block=32)
+    k = rng.standard_normal((1, L, 1, D)).astype(np.float16)
+    v = rng.standard_normal((1, L, 1, D)).astype(np.float16)
+    oc.append(np.array([L], np.int32), k, v)
+    # one scale per 32 sealed tokens: the textbook absmax quantizer per block
+    for i in range(2):
+        _, codes, sc = oc.get_block(0, i)
+        grp = k[0, 32 * i:32 * i + 32, 0].astype(np.float32)
+        assert sc[0, 0] == np.float32(np.abs(grp).max()) / np.float32(127)
+    table = np.array([[2, 0, 1]], np.int32)
+    ex = oc.export(table, 3)
+    cold = ex["cold"].reshape(3, 1, 2, 64 * D)
+    for i, phys in enumerate(table[0][:3]):
+        _, codes, sc = oc.get_block(0, i)
+        n = min(32, L - 32 - 32 * i)
+        kt = cold[phys, 0, 0].view(np.int8)
+        vt = cold[phys, 0, 1].view(np.int8)
+        for t in range(n):
+            assert np.array_equal(kt[t * D:(t + 1) * D], codes[0, 0, t])
+            for ch in (0, 9, 127):
+                assert vt[ch * 64 + (((t // 16) ^ ((ch // 2) % 4)) * 16) + t % 16] == codes[0, 1, t, ch]
+        assert not kt[32 * D:].any()  # the tile's upper 32 slots are never written
