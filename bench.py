@@ -54,7 +54,7 @@ def parse():
                    help="cold blocks: 8 (INT8, the default), 4 (all INT4) or 0 (FP16, quantization off)")
     p.add_argument("--hot-tokens", type=int, default=32, choices=[16, 32, 64, 128],
                    help="hot-zone tokens (32, the default, is the page's value)")
-    p.add_argument("--block-size", type=int, default=64, choices=[64, 128],
+    p.add_argument("--block-size", type=int, default=64, choices=[32, 64, 128],
                    help="tokens per cold block (64, the default, is the page's value)")
     p.add_argument("--sparse-top-k", type=int, default=None,
                    help="time hyb_decode_attn_sparse with this top_k (-1: the page's rule min(128, L // 256)) "

@@ -6,12 +6,12 @@
  *   - a hot zone holding the most recent hot_tokens (32 in the page's example
  *     set; 16, 64 or 128 also built) tokens in FP16, never quantized,
  *     K and V interleaved per token, 512-byte aligned (sections 2.1, 3.1, 3.2);
- *   - a cold zone holding all earlier tokens in 64-token (or 128-token) blocks of symmetric
+ *   - a cold zone holding all earlier tokens in 64-token (or 32- or 128-token) blocks of symmetric
  *     INT8 with a block-wise scale, INT4 for the "L2" cold blocks (sections
  *     2.1, 2.2, 3.1), reached through a block table (section 3.2, block header).
  * The three fields of the hybrid_v2 contract are hot_tokens (power of two),
  * quantization_bits (4 or 8) and block_size (a multiple of 8); this library
- * implements block_size 64 or 128 with hot_tokens 16, 32, 64 or 128 and
+ * implements block_size 32, 64 or 128 with hot_tokens 16, 32, 64 or 128 and
  * quantization_bits 8 or 4
  * (section 3.1; section 5.1 for the invalid-value error), and
  * quantization_bits 0, which the page's section 5.2 gives as the switch that
@@ -65,7 +65,7 @@ typedef struct CUstream_st *hyb_stream_t; /* same type as cudaStream_t */
 #define HYB_OK 0
 #define HYB_ERR_INVALID_VALUE (-1) /* bad config value, shape, null or misaligned pointer;
                                       named after the page's CUDA_ERROR_INVALID_VALUE (3.1) */
-#define HYB_ERR_UNSUPPORTED (-2)   /* valid per the page but not built: block_size not 64 or 128,
+#define HYB_ERR_UNSUPPORTED (-2)   /* valid per the page but not built: block_size not 32, 64 or 128,
                                       head_dim != 128, Hq/Hkv > 8 */
 #define HYB_ERR_WORKSPACE (-3)     /* workspace missing or smaller than required */
 #define HYB_ERR_CUDA (-4)          /* a CUDA runtime call or launch failed */
@@ -88,7 +88,7 @@ typedef struct CUstream_st *hyb_stream_t; /* same type as cudaStream_t */
  * The cache descriptor (host struct; the pointers inside are device memory).
  *
  * Geometry: hot_tokens HOT in {16, 32, 64, 128} (32 is the page's value),
- * block_size BLK = 64 or 128 (64 is the page's value), head_dim D = 128,
+ * block_size BLK = 32, 64 or 128 (64 is the page's value), head_dim D = 128,
  * num_kv_heads Hkv >= 1, num_q_heads Hq a multiple of Hkv with Hq/Hkv <= 8
  * (query head h reads kv head h / (Hq/Hkv)), quant_bits 8 (INT8 cold blocks;
  * logical blocks below n_int4_blocks[b] are INT4), 4 (every cold block INT4)
@@ -109,7 +109,9 @@ typedef struct CUstream_st *hyb_stream_t; /* same type as cudaStream_t */
  *          and kv head, per 64-token sub-block (slot t of a block is slot
  *          t % 64 of sub-block t / 64), a K tile then a V tile of 64 tokens
  *          x 128 channels; the tiles below use the sub-block's slot t.  A
- *          block's sub-blocks share its scales.  Base 16-byte aligned.
+ *          block's sub-blocks share its scales.  A 32-token block takes
+ *          slots 0..31 of one such tile pair (BLK/64 read as 1).  Base
+ *          16-byte aligned.
  *            K, INT8: token-major, code of (slot t, channel c) at t*128 + c.
  *            V, INT8: channel-major rows of 64 bytes; the 16-byte chunk
  *              holding slots 16j..16j+15 of channel c is stored at chunk
@@ -145,7 +147,7 @@ typedef struct CUstream_st *hyb_stream_t; /* same type as cudaStream_t */
  */
 typedef struct hyb_cache_desc {
   int32_t hot_tokens;         /* 16, 32, 64 or 128 */
-  int32_t block_size;         /* 64 or 128 */
+  int32_t block_size;         /* 32, 64 or 128 */
   int32_t head_dim;           /* must be 128 */
   int32_t quant_bits;         /* 8, 4 or 0 (FP16 cold blocks) */
   int32_t num_kv_heads;       /* Hkv >= 1 */
@@ -168,7 +170,7 @@ typedef struct hyb_cache_desc {
  * Returns HYB_OK, HYB_ERR_INVALID_VALUE (hot_tokens not a power of two in
  * {16, 32, 64, 128}, block_size not a multiple of 8, quant_bits not 8, 4 or 0,
  * non-positive sizes, Hq not a multiple of Hkv, null or misaligned pointers)
- * or HYB_ERR_UNSUPPORTED (a valid configuration with block_size not 64 or 128, or
+ * or HYB_ERR_UNSUPPORTED (a valid configuration with block_size not 32, 64 or 128, or
  * head_dim != 128, or Hq/Hkv > 8).  The contract is the page's section 3.1
  * and 5.1 (quant_bits 0: section 5.2).
  */

@@ -29,8 +29,9 @@ class HybridKVCache:
         self.hot = torch.zeros((self.batch, self.hkv, self.hot_tokens, 2, HEAD_DIM), dtype=torch.float16,
                                device=dev)
         # 8 KB parts per block and kv head: K and V tiles of each 64-token
-        # sub-block; FP16 blocks (quant_bits 0) hold rows of K then V, twice the bytes
-        parts = (4 if self.quant_bits == 0 else 2) * max(1, self.block_size // BLOCK)
+        # sub-block (a 32-token block uses half of one); FP16 blocks
+        # (quant_bits 0) hold 512-byte rows of K then V
+        parts = self.block_size // 16 if self.quant_bits == 0 else 2 * max(1, self.block_size // BLOCK)
         self.cold = torch.zeros((self.num_phys, self.hkv, parts, TILE_BYTES), dtype=torch.uint8, device=dev)
         self.scales = torch.zeros((self.num_phys, self.hkv, 2), dtype=torch.float32, device=dev)
         if block_table is None:

@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(512) append_kernel(AppendArgs a) {
     return;
   }
   const long long L_new_ll = static_cast<long long>(L_old) + n;
-  const int B = kBlock << a.lsub;  // tokens per block
+  const int B = 1 << a.bshift;  // tokens per block
   if (L_new_ll - a.hot_tokens > static_cast<long long>(a.max_blocks) * B || L_new_ll > 0x7fffffffLL) {
     if (threadIdx.x == 0) set_status(a.status, HYB_STATUS_CAPACITY);
     return;
@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(512) append_kernel(AppendArgs a) {
       }
       if (a.quant_bits == 0) {
         // FP16 cold block: the rows move unchanged (K row then V row per slot)
-        __half *blk = reinterpret_cast<__half *>(a.cold + ((size_t)phys * a.hkv + h) * (kFp16BlockBytes << a.lsub));
+        __half *blk = reinterpret_cast<__half *>(a.cold + ((size_t)phys * a.hkv + h) * B * kHotTokenBytes);
         for (int t = p0; t < p1; t++) {
           const __half *src;
           if (t < L_old)

@@ -72,8 +72,10 @@ struct DecodeSmem {
 // 0), each attended as two items of 32 rows with the hot ring's arithmetic.
 // kSkip: sparse L2 mode -- the sequence's INT4 ("L2") blocks are left to the
 // top-k kernels, and the splits cover the blocks from its INT4 count on.
-// kLsub: log2 of the 64-token sub-blocks per block (block_size 64: 0, 128: 1).
-template <int G, bool kCluster, bool kF16, bool kSkip, int kLsub>
+// kBshift: log2 of the tokens per block (block_size 32: 5, 64: 6, 128: 7); a
+// 128-token block is two 64-token sub-blocks, a 32-token block the first half
+// of one.
+template <int G, bool kCluster, bool kF16, bool kSkip, int kBshift>
 __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(const DecodeArgs a) {
   constexpr int P = pow2_heads<G>();
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -123,8 +125,9 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
   }
   const int H = a.hot_tokens;
   const int Lc = max(0, L - H);
-  constexpr int lsub = kLsub;        // a block is 1 << lsub sub-blocks of 64 tokens
-  const int Bt = kBlock << lsub;      // tokens per block
+  constexpr int lsub = kBshift > 6 ? kBshift - 6 : 0;  // a block is 1 << lsub sub-blocks
+  constexpr int Bt = 1 << kBshift;                      // tokens per block
+  constexpr int St = Bt < kBlock ? Bt : kBlock;         // tokens per sub-block
   const int nblk = (Lc + Bt - 1) / Bt;
   const int Sb = max(1, (max(0, nblk - ib) + a.split_blocks - 1) / a.split_blocks);
   // past this sequence's last split: no work and no partial (a cluster member
@@ -135,7 +138,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
   // FP16 (the hot ring, FP16 cold blocks: 2 << lsub items per block)
   const int nhot = (s == Sb - 1) ? min(L, H) : 0;
   constexpr bool fp16 = kF16;
-  const int ish = (fp16 ? 1 : 0) + lsub;  // log2 of the items per block
+  constexpr int ish = fp16 ? kBshift - 5 : lsub;  // log2 of the items per block
   const int ncold_it = ncold << ish;
   const int kh = ncold_it;  // the first hot item
   const int nitems = ncold_it + (nhot + kItemRows - 1) / kItemRows;
@@ -216,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
       }
       if (fp16) {
         // 32 of the block's sealed rows
-        const uint8_t *src = a.cold + ((size_t)phys * a.hkv + h) * (kFp16BlockBytes << lsub) + part * kItemBytes;
+        const uint8_t *src = a.cold + ((size_t)phys * a.hkv + h) * Bt * kHotTokenBytes + part * kItemBytes;
         const uint32_t bytes = static_cast<uint32_t>(nrow) * kHotTokenBytes;
         mbar_arrive_expect_tx(&sm.full[st], bytes);
         bulk_g2s(dst, src, bytes, &sm.full[st], pol);
@@ -224,11 +227,19 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
       }
       const uint8_t *src = a.cold + ((((size_t)phys * a.hkv + h) << lsub) + u) * kTilePairBytes;
       if (i0 + kb >= n_int4_b) {
-        mbar_arrive_expect_tx(&sm.full[st], kTilePairBytes);
-        bulk_g2s(dst, src, kTilePairBytes, &sm.full[st], pol);
+        if constexpr (St == kBlock) {
+          mbar_arrive_expect_tx(&sm.full[st], kTilePairBytes);
+          bulk_g2s(dst, src, kTilePairBytes, &sm.full[st], pol);
+        } else {
+          // a 32-token block: the K rows it holds, and its V tile (whose
+          // rows interleave its slots with the unused ones)
+          mbar_arrive_expect_tx(&sm.full[st], St * kDim + kTileBytes);
+          bulk_g2s(dst, src, St * kDim, &sm.full[st], pol);
+          bulk_g2s(dst + kTileBytes, src + kTileBytes, kTileBytes, &sm.full[st], pol);
+        }
       } else {
-        mbar_arrive_expect_tx(&sm.full[st], kTileBytes);
-        bulk_g2s(dst, src, kTileBytes / 2, &sm.full[st], pol);
+        mbar_arrive_expect_tx(&sm.full[st], St * kDim / 2 + kTileBytes / 2);
+        bulk_g2s(dst, src, St * kDim / 2, &sm.full[st], pol);
         bulk_g2s(dst + kTileBytes, src + kTileBytes, kTileBytes / 2, &sm.full[st], pol);
       }
     } else {
@@ -335,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
       // ---------------- cold sub-block (64 tokens) ----------------
       const int kb = item_block(k);
       const int i = i0 + kb;
-      const int nvalid = sm.phys[kb] < 0 ? 0 : min(kBlock, Lc - i * Bt - item_sub(k) * kBlock);
+      const int nvalid = sm.phys[kb] < 0 ? 0 : min(St, Lc - i * Bt - item_sub(k) * kBlock);
       const int nv = nvalid - 16 * warp;
       const bool int4 = i < n_int4_b;
       const float2 sc = sm.scl[kb];
@@ -483,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(cons
 // Largest cluster the decode kernel is launched with (portable size).
 constexpr int kMaxCluster = 8;
 
-template <int G, bool kF16, bool kSkip, int kLsub>
+template <int G, bool kF16, bool kSkip, int kBshift>
 static cudaError_t launch_decode_g(const DecodeArgs &a, int batch, bool cluster, cudaStream_t stream) {
   const size_t smem = sizeof(DecodeSmem<G>);
   static int configured_dev_mask = 0;  // one bit per device (per instantiation)
@@ -491,10 +502,10 @@ static cudaError_t launch_decode_g(const DecodeArgs &a, int batch, bool cluster,
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 31 && !(configured_dev_mask & (1 << dev))) {
-    e = cudaFuncSetAttribute(decode_kernel<G, false, kF16, kSkip, kLsub>,
+    e = cudaFuncSetAttribute(decode_kernel<G, false, kF16, kSkip, kBshift>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(decode_kernel<G, true, kF16, kSkip, kLsub>,
+      e = cudaFuncSetAttribute(decode_kernel<G, true, kF16, kSkip, kBshift>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     configured_dev_mask |= 1 << dev;
@@ -513,39 +524,43 @@ static cudaError_t launch_decode_g(const DecodeArgs &a, int batch, bool cluster,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_kernel<G, true, kF16, kSkip, kLsub>, a);
+    e = cudaLaunchKernelEx(&cfg, decode_kernel<G, true, kF16, kSkip, kBshift>, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
-  decode_kernel<G, false, kF16, kSkip, kLsub><<<grid, kThreads, smem, stream>>>(a);
+  decode_kernel<G, false, kF16, kSkip, kBshift><<<grid, kThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
-template <bool kF16, bool kSkip, int kLsub>
+template <bool kF16, bool kSkip, int kBshift>
 static cudaError_t launch_decode_f(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream) {
   switch (group) {
-    case 1: return launch_decode_g<1, kF16, kSkip, kLsub>(a, batch, cluster, stream);
-    case 2: return launch_decode_g<2, kF16, kSkip, kLsub>(a, batch, cluster, stream);
-    case 3: return launch_decode_g<3, kF16, kSkip, kLsub>(a, batch, cluster, stream);
-    case 4: return launch_decode_g<4, kF16, kSkip, kLsub>(a, batch, cluster, stream);
-    case 5: return launch_decode_g<5, kF16, kSkip, kLsub>(a, batch, cluster, stream);
-    case 6: return launch_decode_g<6, kF16, kSkip, kLsub>(a, batch, cluster, stream);
-    case 7: return launch_decode_g<7, kF16, kSkip, kLsub>(a, batch, cluster, stream);
-    case 8: return launch_decode_g<8, kF16, kSkip, kLsub>(a, batch, cluster, stream);
+    case 1: return launch_decode_g<1, kF16, kSkip, kBshift>(a, batch, cluster, stream);
+    case 2: return launch_decode_g<2, kF16, kSkip, kBshift>(a, batch, cluster, stream);
+    case 3: return launch_decode_g<3, kF16, kSkip, kBshift>(a, batch, cluster, stream);
+    case 4: return launch_decode_g<4, kF16, kSkip, kBshift>(a, batch, cluster, stream);
+    case 5: return launch_decode_g<5, kF16, kSkip, kBshift>(a, batch, cluster, stream);
+    case 6: return launch_decode_g<6, kF16, kSkip, kBshift>(a, batch, cluster, stream);
+    case 7: return launch_decode_g<7, kF16, kSkip, kBshift>(a, batch, cluster, stream);
+    case 8: return launch_decode_g<8, kF16, kSkip, kBshift>(a, batch, cluster, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int kLsub>
+template <int kBshift>
 static cudaError_t launch_decode_l(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream) {
-  if (a.quant_bits == 0) return launch_decode_f<true, false, kLsub>(a, group, batch, cluster, stream);
-  if (a.l2_skip) return launch_decode_f<false, true, kLsub>(a, group, batch, cluster, stream);
-  return launch_decode_f<false, false, kLsub>(a, group, batch, cluster, stream);
+  if (a.quant_bits == 0) return launch_decode_f<true, false, kBshift>(a, group, batch, cluster, stream);
+  if (a.l2_skip) return launch_decode_f<false, true, kBshift>(a, group, batch, cluster, stream);
+  return launch_decode_f<false, false, kBshift>(a, group, batch, cluster, stream);
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream) {
-  return a.lsub ? launch_decode_l<1>(a, group, batch, cluster, stream)
-                : launch_decode_l<0>(a, group, batch, cluster, stream);
+  switch (a.bshift) {
+    case 5: return launch_decode_l<5>(a, group, batch, cluster, stream);
+    case 6: return launch_decode_l<6>(a, group, batch, cluster, stream);
+    case 7: return launch_decode_l<7>(a, group, batch, cluster, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 int decode_max_cluster() { return kMaxCluster; }
@@ -568,10 +583,10 @@ int decode_ctas_per_sm(int group) {
   switch (group) {
 #define HYB_OCC(g)                                                                          \
   case g:                                                                                   \
-    e = cudaFuncSetAttribute(decode_kernel<g, false, false, false, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+    e = cudaFuncSetAttribute(decode_kernel<g, false, false, false, 6>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              static_cast<int>(sizeof(DecodeSmem<g>)));                      \
     if (e == cudaSuccess)                                                                   \
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<g, false, false, false, 0>, kThreads, \
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<g, false, false, false, 6>, kThreads, \
                                                         sizeof(DecodeSmem<g>));             \
     break;
     HYB_OCC(1) HYB_OCC(2) HYB_OCC(3) HYB_OCC(4) HYB_OCC(5) HYB_OCC(6) HYB_OCC(7) HYB_OCC(8)

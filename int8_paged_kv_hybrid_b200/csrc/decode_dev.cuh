@@ -108,7 +108,7 @@ __device__ __forceinline__ void fused_seal(SealScratch &ss, uint8_t *tile_st, fl
   do_seal = do_seal && tile_tail >= 0;
   if (!do_seal) return;
   const int e = L_old - a.hot_tokens;  // position sealed
-  const int slot_b = e % (kBlock << a.lsub);  // its slot in the block
+  const int slot_b = e & ((1 << a.bshift) - 1);  // its slot in the block
   const int slot = slot_b & (kBlock - 1);     // ... and in its sub-block
   const bool int4 = int4_tail;
   const int Q = int4 ? 7 : 127;
@@ -182,7 +182,12 @@ __device__ __forceinline__ void fused_seal(SealScratch &ss, uint8_t *tile_st, fl
       uint8_t *g = gtile + kv * kTileBytes;
       const uint8_t *t = tile_st + kv * kTileBytes;
       if (ss.seal_rq[kv]) {
-        const int nvec = (int4 ? kTileBytes / 2 : kTileBytes) / 16;
+        // the bytes the block's codes occupy: K rows of its slots only (a
+        // 32-token block stages and owns the first half of a K tile), the
+        // whole V tile
+        const int st_tok = min(kBlock, 1 << a.bshift);
+        const int kbytes = (int4 ? 64 : kDim) * st_tok;
+        const int nvec = (kv == 0 ? kbytes : (int4 ? kTileBytes / 2 : kTileBytes)) / 16;
         for (int v = tid; v < nvec; v += kThreads)
           reinterpret_cast<uint4 *>(g)[v] = reinterpret_cast<const uint4 *>(t)[v];
       } else if (kv == 0) {
@@ -206,13 +211,13 @@ __device__ __forceinline__ void fused_seal(SealScratch &ss, uint8_t *tile_st, fl
 __device__ __forceinline__ void fused_seal_fp16(const SealScratch &ss, uint8_t *row_st, int tile_tail,
                                                 const DecodeArgs &a, int L_old, bool do_seal, int tid) {
   if (!do_seal || tile_tail < 0) return;
-  const int slot = (L_old - a.hot_tokens) % (kBlock << a.lsub);
+  const int slot = (L_old - a.hot_tokens) & ((1 << a.bshift) - 1);
   const int c = tid;
   const __half k_old = ss.erow[c], v_old = ss.erow[kDim + c];
   __half *trow = reinterpret_cast<__half *>(row_st + (slot % kItemRows) * kHotTokenBytes);
   trow[c] = k_old;
   trow[kDim + c] = v_old;
-  __half *grow = reinterpret_cast<__half *>(a.cold + (size_t)tile_tail * (kFp16BlockBytes << a.lsub) +
+  __half *grow = reinterpret_cast<__half *>(a.cold + ((size_t)tile_tail << a.bshift) * kHotTokenBytes +
                                             slot * kHotTokenBytes);
   grow[c] = k_old;
   grow[kDim + c] = v_old;

@@ -63,8 +63,10 @@ const char *hyb_strerror(int code) {
   }
 }
 
-// log2 of the 64-token sub-blocks per block (block_size 64: 0, 128: 1)
+// log2 of the 64-token sub-blocks per block (block_size 32, 64: 0; 128: 1)
 static int lsub_of(const hyb_cache_desc *d) { return d->block_size == 2 * hyb::kBlock ? 1 : 0; }
+// log2 of the tokens per block (32: 5, 64: 6, 128: 7)
+static int bshift_of(const hyb_cache_desc *d) { return d->block_size == 32 ? 5 : d->block_size == 64 ? 6 : 7; }
 
 int hyb_check_desc(const hyb_cache_desc *d) {
   if (!d) return HYB_ERR_INVALID_VALUE;
@@ -86,7 +88,8 @@ int hyb_check_desc(const hyb_cache_desc *d) {
       (d->n_int4_blocks && !aligned(d->n_int4_blocks, 4)))
     return HYB_ERR_INVALID_VALUE;
   // what this library builds
-  if ((d->block_size != hyb::kBlock && d->block_size != 2 * hyb::kBlock) || d->head_dim != hyb::kDim)
+  if ((d->block_size != 32 && d->block_size != hyb::kBlock && d->block_size != 2 * hyb::kBlock) ||
+      d->head_dim != hyb::kDim)
     return HYB_ERR_UNSUPPORTED;
   if (d->num_q_heads / d->num_kv_heads > 8) return HYB_ERR_UNSUPPORTED;
   return HYB_OK;
@@ -117,6 +120,7 @@ int hyb_kv_append(const hyb_cache_desc *d, const int32_t *n_new, int32_t max_new
   a.max_new = max_new;
   a.hot_tokens = d->hot_tokens;
   a.lsub = lsub_of(d);
+  a.bshift = bshift_of(d);
   const cudaError_t e = hyb::launch_append(a, d->batch, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HYB_OK : cuda_fail(e);
 }
@@ -302,6 +306,7 @@ static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_s
   a.quant_bits = d->quant_bits;
   a.hot_tokens = d->hot_tokens;
   a.lsub = lsub_of(d);
+  a.bshift = bshift_of(d);
   a.n_splits = pl.ns;
   a.split_blocks = pl.tb;
   a.max_seq_len = max_seq_len;
@@ -385,6 +390,7 @@ int hyb_decode_attn_sparse(const hyb_cache_desc *d, const void *q, float softmax
   a.quant_bits = d->quant_bits;
   a.hot_tokens = d->hot_tokens;
   a.lsub = lsub_of(d);
+  a.bshift = bshift_of(d);
   a.max_l2 = w.max_l2;
   a.top_k = top_k;
   a.blocks_per_cta = 4;
@@ -450,6 +456,7 @@ int hyb_kv_migrate(const hyb_cache_desc *d, const int32_t *target_n_int4, int32_
   a.max_delta = max_delta;
   a.hot_tokens = d->hot_tokens;
   a.lsub = lsub_of(d);
+  a.bshift = bshift_of(d);
   const cudaError_t e = hyb::launch_migrate(a, d->batch, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HYB_OK : cuda_fail(e);
 }

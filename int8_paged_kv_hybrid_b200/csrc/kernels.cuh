@@ -21,7 +21,8 @@ struct AppendArgs {
   const __half *v_new;
   int hkv, num_phys, max_blocks, quant_bits, max_new;
   int hot_tokens;             // hot-zone tokens (power of two, 16..128)
-  int lsub;                   // log2 of the 64-token sub-blocks per block (block_size 64: 0, 128: 1)
+  int lsub;                   // log2 of the 64-token sub-blocks per block (block_size 32, 64: 0; 128: 1)
+  int bshift;                 // log2 of the tokens per block (block_size 32: 5, 64: 6, 128: 7)
 };
 
 struct DecodeArgs {
@@ -48,6 +49,7 @@ struct DecodeArgs {
   int hkv, hq, num_phys, max_blocks, quant_bits, n_splits, split_blocks, max_seq_len;
   int hot_tokens;             // hot-zone tokens (power of two, 16..128)
   int lsub;                   // log2 of the 64-token sub-blocks per block
+  int bshift;                 // log2 of the tokens per block
   float qk_scale;             // softmax_scale * log2(e)
   // fused decode step (null for attention only): append n_new[b] in {0, 1}
   // tokens first; k_new / v_new FP16 [batch][Hkv][128]; seq_cnt [batch]
@@ -72,6 +74,7 @@ struct MigrateArgs {
   int hkv, num_phys, max_blocks, max_delta;
   int hot_tokens;             // hot-zone tokens
   int lsub;                   // log2 of the 64-token sub-blocks per block
+  int bshift;                 // log2 of the tokens per block
 };
 
 // Sparse L2 attention (top-k of the INT4-block tokens per query head).
@@ -88,6 +91,7 @@ struct SparseArgs {
   float *lse;                 // [batch][Hq]: the dense pass's log-sum-exp in, merged out (natural log)
   int hkv, hq, num_phys, max_blocks, quant_bits, hot_tokens, max_l2, top_k, blocks_per_cta;
   int lsub;                   // log2 of the 64-token sub-blocks per block
+  int bshift;                 // log2 of the tokens per block
   float qk_scale;             // softmax_scale * log2(e)
 };
 

@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(2 * kMigThreads) migrate_kernel(const MigrateA
   const int nwarps = blockDim.x >> 5;
   const int u = tid_all / kMigThreads;    // this thread's sub-block
   const int tid = tid_all % kMigThreads;  // ... and its index there
-  const int Bt = kBlock << a.lsub;
+  const int Bt = 1 << a.bshift;
   int lo, hi, tgt;
   if (!tier_move(a, b, lo, hi, tgt)) {
     if (k == 0 && h == 0 && tid_all == 0) set_status(a.status, HYB_STATUS_BAD_TIER);
@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(2 * kMigThreads) migrate_kernel(const MigrateA
   if (i >= hi) return;
   const int Lc = max(0, a.seq_lens[b] - a.hot_tokens);
   if (i * Bt >= Lc) return;  // nothing sealed in this block yet: only its tier changes
-  const int sealed = max(0, min(kBlock, Lc - i * Bt - u * kBlock));  // in this sub-block
+  const int sealed = max(0, min(min(kBlock, Bt), Lc - i * Bt - u * kBlock));  // in this sub-block
   const int phys = a.block_table[(size_t)b * a.max_blocks + i];
   if (phys < 0 || phys >= a.num_phys) {
     if (tid_all == 0) set_status(a.status, HYB_STATUS_BAD_BLOCK);

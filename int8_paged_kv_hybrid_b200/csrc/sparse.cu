@@ -33,7 +33,7 @@ __device__ __forceinline__ int l2_count(const SparseArgs &a, int b) {
   if (L < 0) return 0;
   const int Lc = max(0, L - a.hot_tokens);
   const long long n4 = a.quant_bits == 4 ? a.max_blocks : (a.n_int4 ? a.n_int4[b] : 0);
-  const long long n = min(static_cast<long long>(Lc), max(0LL, n4) * (kBlock << a.lsub));
+  const long long n = min(static_cast<long long>(Lc), max(0LL, n4) << a.bshift);
   return n > a.max_l2 ? -1 : static_cast<int>(n);
 }
 
@@ -51,8 +51,10 @@ __global__ void __launch_bounds__(kScoreThreads) l2_score_kernel(const SparseArg
   const int G = a.hq / a.hkv;
   const int n = l2_count(a, b);
   if (n <= 0) return;
-  // units of 64 tokens (sub-blocks; a block is 1 << lsub of them)
-  const int nb = (n + kBlock - 1) / kBlock;
+  // units of St tokens: 64-token sub-blocks (a block is 1 << lsub of them),
+  // or whole 32-token blocks
+  const int St = min(kBlock, 1 << a.bshift);
+  const int nb = (n + St - 1) / St;
   const int blk0 = chunk * a.blocks_per_cta;
   if (blk0 >= nb) return;
 
@@ -158,8 +160,8 @@ __global__ void __launch_bounds__(kScoreThreads) l2_score_kernel(const SparseArg
     }
 #pragma unroll
     for (int g = 0; g < 8; g++) dot[g] += __shfl_xor_sync(0xffffffffu, dot[g], 1);
-    const int pos = blk * kBlock + tok;
-    if (half == 0 && pos < n) {
+    const int pos = blk * St + tok;
+    if (half == 0 && tok < St && pos < n) {
       const float sk = okp ? a.scales[((size_t)phys * a.hkv + h) * 2] : 0.f;
 #pragma unroll
       for (int g = 0; g < 8; g++) {
@@ -366,12 +368,12 @@ __global__ void __launch_bounds__(kT) l2_topk_kernel(const SparseArgs a) {
   float zmax = -INFINITY;
   for (int j = tid; j < ns; j += kTopkThreads) {
     const int pos = s_pos[j];
-    const int phys = a.block_table[(size_t)b * a.max_blocks + (pos / (kBlock << a.lsub))];
+    const int phys = a.block_table[(size_t)b * a.max_blocks + (pos >> a.bshift)];
     const bool okp = phys >= 0 && phys < a.num_phys;
     const float z = keys[pos] * coef;
     s_p[j] = z;
     // the sub-block pair holding pos
-    s_vt[j] = okp ? (((phys * a.hkv + h) << a.lsub) + ((pos / kBlock) & ((1 << a.lsub) - 1))) : -1;
+    s_vt[j] = okp ? (((phys * a.hkv + h) << a.lsub) + ((pos & ((1 << a.bshift) - 1)) >> 6)) : -1;
     s_sv[j] = okp ? a.scales[((size_t)phys * a.hkv + h) * 2 + 1] : 0.f;
     zmax = fmaxf(zmax, z);
   }
@@ -390,7 +392,7 @@ __global__ void __launch_bounds__(kT) l2_topk_kernel(const SparseArgs a) {
   for (int j = part; j < ns; j += kParts) {
     const int vt = s_vt[j];
     if (vt < 0) continue;
-    const int slot = s_pos[j] & (kBlock - 1);
+    const int slot = s_pos[j] & ((1 << a.bshift) - 1) & (kBlock - 1);
     const uint8_t *vtile = a.cold + (size_t)vt * kTilePairBytes + kTileBytes;
     const uint8_t byte =
         vtile[c * 32 + 8 * ((slot >> 4) ^ ((c >> 2) & 3)) + ((slot & 15) >> 3) * 4 + (slot & 3)];
@@ -418,7 +420,8 @@ __global__ void __launch_bounds__(kT) l2_topk_kernel(const SparseArgs a) {
 
 cudaError_t launch_sparse_l2(const SparseArgs &a, int batch, cudaStream_t stream) {
   if (a.max_l2 <= 0 || a.top_k <= 0) return cudaSuccess;
-  const int max_nb = (a.max_l2 + kBlock - 1) / kBlock;
+  const int St = min(kBlock, 1 << a.bshift);
+  const int max_nb = (a.max_l2 + St - 1) / St;
   dim3 g1((max_nb + a.blocks_per_cta - 1) / a.blocks_per_cta, a.hkv, batch);
   l2_score_kernel<<<g1, kScoreThreads, 0, stream>>>(a);
   cudaError_t e = cudaGetLastError();

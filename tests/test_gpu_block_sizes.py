@@ -1,8 +1,9 @@
-"""block_size 128 on the GPU against the oracle: a block is two 64-token
-sub-blocks sharing one scale pair.  Appends bit-exact (including a grown
+"""block_size 128 and 32 on the GPU against the oracle.  A 128-token block is
+two 64-token sub-blocks sharing one scale pair; a 32-token block uses the
+first half of one 64-slot tile pair.  Appends bit-exact (including a grown
 scale re-quantizing the first sub-block), decode within the accuracy bar,
-fused steps whose seal lands in the second sub-block and grows the scale,
-tier migration of both sub-blocks together, sparse L2 decode."""
+fused steps whose seals grow the block's scale, tier migration, sparse L2
+decode."""
 import numpy as np
 import pytest
 
@@ -26,36 +27,42 @@ def _widen(w, extra_tokens):
     w.block_table, w.num_phys_blocks = bt, nxt
 
 
+BLOCKS = [128, 32]
+
+
+@pytest.mark.parametrize("blk", BLOCKS)
 @pytest.mark.parametrize("qbits,int4", [(8, False), (8, True), (4, False), (0, False)])
-def test_appends_bit_exact(qbits, int4):
-    nb = [synth.cold_blocks_for(L, 32, 128) for L in LENS]
-    w = synth.custom_workload("b128", LENS, 8, 2, seed=qbits + 10 * int4, max_step=70, block=128,
+def test_appends_bit_exact(qbits, int4, blk):
+    nb = [synth.cold_blocks_for(L, 32, blk) for L in LENS]
+    w = synth.custom_workload("b%d" % blk, LENS, 8, 2, seed=qbits + 10 * int4, max_step=70, block=blk,
                               n_int4=[n // 2 for n in nb] if int4 else None)
     cache, ora = make_pair(w, quant_bits=qbits)
     replay(w, cache, ora, check_every=1)
     assert_cache_equal(w, cache, ora, "final")
 
 
+@pytest.mark.parametrize("blk", BLOCKS)
 @pytest.mark.parametrize("qbits,hq,hkv", [(8, 32, 8), (4, 28, 4), (0, 8, 2)])
 @pytest.mark.parametrize("split", [0, 128, 256])
-def test_decode_parity(qbits, hq, hkv, split):
-    nb = [synth.cold_blocks_for(L, 32, 128) for L in LENS]
-    w = synth.custom_workload("b128d", LENS, hq, hkv, seed=hq + split, max_step=64, block=128,
+def test_decode_parity(qbits, hq, hkv, split, blk):
+    nb = [synth.cold_blocks_for(L, 32, blk) for L in LENS]
+    w = synth.custom_workload("b%dd" % blk, LENS, hq, hkv, seed=hq + split, max_step=64, block=blk,
                               n_int4=[n // 3 for n in nb] if qbits == 8 else None)
     cache, ora = make_pair(w, quant_bits=qbits)
     replay(w, cache, ora)
     got, lse, ref, ref_lse = decode_both(w, cache, ora, split_tokens=split)
-    assert_decode_close(w, got, lse, ref, ref_lse, what="block 128 qbits=%d split=%d" % (qbits, split))
+    assert_decode_close(w, got, lse, ref, ref_lse, what="block %d qbits=%d split=%d" % (blk, qbits, split))
     assert cache.status() == 0
 
 
+@pytest.mark.parametrize("blk", BLOCKS)
 @pytest.mark.parametrize("qbits,split", [(8, 0), (8, 128), (4, 0), (0, 0)])
-def test_fused_steps(qbits, split):
+def test_fused_steps(qbits, split, blk):
     """90 one-token steps; some tokens carry a K four times larger or a V
     outlier channel, so that seals into the second sub-block grow the block's
     K or V scale (outputs stay of unit size, so the absolute bar applies)."""
     import torch
-    w = synth.custom_workload("b128s", LENS, 8, 2, seed=5 + qbits, max_step=64, pool_extra=0, block=128)
+    w = synth.custom_workload("b%ds" % blk, LENS, 8, 2, seed=5 + qbits, max_step=64, pool_extra=0, block=blk)
     _widen(w, 100)
     cache, ora = make_pair(w, quant_bits=qbits)
     replay(w, cache, ora)
@@ -82,11 +89,12 @@ def test_fused_steps(qbits, split):
                             what="step %d" % st)
 
 
-def test_migration_moves_both_sub_blocks():
+@pytest.mark.parametrize("blk", BLOCKS)
+def test_migration(blk):
     import torch
     lens = [97, 300, 700, 1300]
-    nb = [synth.cold_blocks_for(L, 32, 128) for L in lens]
-    w = synth.custom_workload("b128m", lens, 32, 8, seed=8, max_step=64, block=128, n_int4=[1, 0, 2, 3])
+    nb = [synth.cold_blocks_for(L, 32, blk) for L in lens]
+    w = synth.custom_workload("b%dm" % blk, lens, 32, 8, seed=8, max_step=64, block=blk, n_int4=[1, 0, 2, 3])
     cache, ora = make_pair(w)
     replay(w, cache, ora)
     for tgt in ([n for n in nb], [0, 1, 1, 2], [min(n + 1, w.max_blocks) for n in nb]):
@@ -98,12 +106,13 @@ def test_migration_moves_both_sub_blocks():
         assert_decode_close(w, got, lse, ref, ref_lse, what="after move to %s" % tgt)
 
 
+@pytest.mark.parametrize("blk", BLOCKS)
 @pytest.mark.parametrize("k", [0, 5, 64, 1024])
-def test_sparse_l2(k):
+def test_sparse_l2(k, blk):
     import torch
     lens = [300, 1300, 2100]
-    nb = [synth.cold_blocks_for(L, 32, 128) for L in lens]
-    w = synth.custom_workload("b128p", lens, 28, 4, seed=k, max_step=64, block=128,
+    nb = [synth.cold_blocks_for(L, 32, blk) for L in lens]
+    w = synth.custom_workload("b%dp" % blk, lens, 28, 4, seed=k, max_step=64, block=blk,
                               n_int4=[(2 * n) // 3 for n in nb])
     cache, ora = make_pair(w)
     replay(w, cache, ora)
@@ -113,4 +122,4 @@ def test_sparse_l2(k):
     torch.cuda.synchronize()
     ref, ref_lse = ora.decode(q, w.softmax_scale, top_k=k)
     assert_decode_close(w, out.float().cpu().numpy().astype(np.float64), lse.cpu().numpy(), ref, ref_lse,
-                        what="block 128 sparse k=%d" % k)
+                        what="block %d sparse k=%d" % (blk, k))
