@@ -74,7 +74,7 @@ def workload_config(w, split, ns, qbits=8):
     if qbits == 8 and w.n_int4 is not None:
         cold = "INT8 (oldest quarter INT4)"
     H = w.hot_tokens
-    if w.name == "config2":
+    if w.name == synth_name(2):
         what = ("llama3-8b decode attention, 1 layer: batch %d, Hq %d, Hkv %d, d 128, L %d (%d FP16 hot + "
                 "%d %s cold in %d-token blocks), %d-block pool"
                 % (w.batch, w.num_q_heads, w.num_kv_heads, int(lens[0]), H, int(lens[0]) - H, cold,
@@ -107,6 +107,11 @@ def max_over_ranks(x, world, device=None):
 def job_throughput(bytes_per_rank, world, ms):
     """Whole-job GB/s: what every rank processed over the slowest rank's ms."""
     return bytes_per_rank * world / (ms * 1e-3) / 1e9
+
+
+def synth_name(idx):
+    from int8_paged_kv_hybrid_b200 import synth
+    return synth.WORKLOAD_NAMES[idx]
 
 
 def kernel_sha():

@@ -49,6 +49,16 @@ class Workload:
         return np.array([cold_blocks_for(int(L), self.hot_tokens, self.block_size) for L in self.lens], np.int64)
 
 
+# The measured workloads, by what they are.
+WORKLOAD_NAMES = {
+    1: "one_seq_mha8_L1024",
+    2: "llama3_8b_b8_L2048",
+    3: "var64_gqa4_L256_8192",
+    4: "long_b4_L32k_128k",
+    5: "qwen2_7b_b128_mixed_int4",
+}
+
+
 def cold_blocks_for(L: int, hot: int = HOT, block: int = BLOCK) -> int:
     """Cold blocks a sequence of L tokens occupies (the newest `hot` stay hot)."""
     return (max(0, L - hot) + block - 1) // block
@@ -166,7 +176,7 @@ def make_workload(idx: int, scale_down: int = 1, seed_offset: int = 0) -> Worklo
     else:
         sched = _random_step_schedule(rng, lens, 1, 64)
         max_new = 64
-    return Workload(name="config%d" % idx, batch=B, num_q_heads=hq, num_kv_heads=hkv,
+    return Workload(name=WORKLOAD_NAMES[idx], batch=B, num_q_heads=hq, num_kv_heads=hkv,
                     lens=lens.astype(np.int32), softmax_scale=sm, q_std=qstd,
                     num_phys_blocks=pool, block_table=bt, n_int4=n_int4,
                     schedule=sched, max_new=max_new, seed=seed,
