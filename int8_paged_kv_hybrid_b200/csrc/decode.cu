@@ -9,10 +9,12 @@
 //
 // Work decomposition: one CTA (4 warps) per (split, kv head, sequence).  A
 // split is a run of up to `split_blocks` cold blocks; the split that holds
-// the sequence's last cold block also attends the hot ring.  Each cold block
-// (K tile 8 KB + V tile 8 KB, or 4 + 4 KB for INT4) and the hot ring (16 KB)
-// is one pipeline item, brought into a 3-stage shared-memory ring by the TMA
-// engine with one 1-D bulk copy (no cluster multicast) completing on an
+// the sequence's last cold block also attends the hot ring.  Pipeline items:
+// a 64-token sub-block of a cold block (K tile 8 KB + V tile 8 KB, or 4 + 4
+// KB for INT4; a 128-token block is two, a 32-token block the first half of
+// one), 32 FP16 rows (16 KB) of an FP16 cold block, and 32 rows of the hot
+// ring.  Each item is brought into a 3-stage shared-memory ring by the TMA
+// engine with 1-D bulk copies (no cluster multicast) completing on an
 // mbarrier; every wait is bounded.  Three CTAs fit on an SM for up to 4 query
 // heads per kv head (two above that).  When all splits are resident at once
 // (one wave) 2..8 splits of a (sequence, kv head) run as one thread-block
@@ -38,7 +40,8 @@
 //    CTA of a (sequence, kv head) to finish merges the splits (log-sum-exp)
 //    and writes the FP16 output.
 // Tensor cores are not used: per byte of KV the work is a few integer
-// multiply-adds, and the kernel is bound by HBM bandwidth.
+// multiply-adds (a GEMV per kv head), so the roof is HBM bandwidth; the
+// measured loop is bound by the latency of that integer work.
 #include "decode_dev.cuh"
 
 namespace hyb {
