@@ -210,9 +210,10 @@ class ClockSampler:
 
 
 def room_for_growth(w, extra_tokens):
-    """Give every sequence physical blocks for `extra_tokens` more tokens:
-    spare pool blocks (or new ones past the pool) go into the block table,
-    widened when needed.  For runs that let the cache grow."""
+    """Give every sequence physical blocks for its tokens plus `extra_tokens`
+    more: every missing table entry gets a spare pool block (or a new one past
+    the pool), the table widened when needed.  For runs that let the cache
+    grow, or whose hot or block size needs more blocks than the table has."""
     import numpy as np
     from int8_paged_kv_hybrid_b200 import synth
     need = [synth.cold_blocks_for(int(L) + extra_tokens, w.hot_tokens, w.block_size) for L in w.lens]
@@ -223,7 +224,7 @@ def room_for_growth(w, extra_tokens):
     spare = [p for p in range(w.num_phys_blocks) if p not in used]
     nxt = w.num_phys_blocks
     for b in range(w.batch):
-        for j in range(synth.cold_blocks_for(int(w.lens[b]), w.hot_tokens, w.block_size), need[b]):
+        for j in range(need[b]):
             if bt[b, j] < 0:
                 if spare:
                     bt[b, j] = spare.pop(0)

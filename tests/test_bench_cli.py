@@ -1,0 +1,39 @@
+"""bench.py's command line and the JSON fields it derives on the host (no GPU):
+every cold-format, hot-size and block-size variant parses, and its
+configuration object names the workload by what it is."""
+import json
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from int8_paged_kv_hybrid_b200 import synth  # noqa: E402
+
+
+@pytest.mark.parametrize("argv", [
+    [], ["--quant-bits", "0"], ["--quant-bits", "4"], ["--hot-tokens", "16"], ["--hot-tokens", "128"],
+    ["--block-size", "32"], ["--block-size", "128"], ["--sparse-top-k", "-1"], ["--migrate"],
+    ["--lean", "--steps", "3", "--warmup", "1"], ["--impl", "reference", "--gpus", "2"],
+])
+def test_arguments_parse(argv, monkeypatch):
+    monkeypatch.setattr(sys, "argv", ["bench.py"] + argv)
+    a = bench.parse()
+    assert a.steps > 0 and a.warmup >= 0
+
+
+@pytest.mark.parametrize("qb,hot,blk", [(8, 32, 64), (0, 64, 64), (4, 16, 32), (8, 128, 128)])
+def test_config_object(qb, hot, blk):
+    w = synth.make_workload(2)
+    w.hot_tokens, w.block_size = hot, blk
+    bench.room_for_growth(w, 0)
+    cfg = bench.workload_config(w, 0, 6, qb)
+    json.dumps(cfg)
+    assert cfg["hot_tokens"] == hot and cfg["block_size"] == blk and cfg["quant_bits"] == qb
+    assert "llama3-8b" in cfg["workload"] and "%d-token blocks" % blk in cfg["workload"]
+    # every sequence has a physical block for each of its cold blocks
+    need = w.cold_blocks()
+    assert all((w.block_table[b, :need[b]] >= 0).all() for b in range(w.batch))
