@@ -104,6 +104,24 @@ def test_plan_and_workspace():
     assert hk.hyb_decode_plan(d, 2048, 0)[1] >= 8
 
 
+@pytest.mark.parametrize("block,hot", [(32, 16), (128, 64), (64, 128)])
+def test_plan_other_block_and_hot_sizes(block, hot):
+    """Splits count blocks of the descriptor's size; the cold range is the
+    length minus the hot zone."""
+    d = _desc(hot=hot, block=block, batch=4, maxb=4096, phys=8192)
+    for L in (hot + 1, 1000, 40000):
+        st, ns = hk.hyb_decode_plan(d, L, 0)
+        assert st % block == 0 and st >= block and ns == max(1, -(-max(0, L - hot) // st))
+    st, ns = hk.hyb_decode_plan(d, 40000, 4 * block)
+    assert st == 4 * block and ns == -(-(40000 - hot) // st)
+    for bad in (block // 2, 3 * block + 8):
+        with pytest.raises(hk.HybError):
+            hk.hyb_decode_plan(d, 4096, bad)
+    # the block table bounds the length in blocks of this size
+    with pytest.raises(hk.HybError):
+        hk.hyb_decode_plan(d, block * 4096 + hot + 1, 0)
+
+
 def test_strerror_covers_codes():
     for c in (0, -1, -2, -3, -4, 100, 101, 102, 103, 104, 105):
         assert hk.strerror(c) and hk.strerror(c) != "unknown code"
