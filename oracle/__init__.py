@@ -60,6 +60,10 @@ def _load():
     lib.ora_decode.argtypes = [P, P, ctypes.c_double, P, i32, P, P, i32]
     lib.ora_decode_topk.argtypes = [P, P, ctypes.c_double, i32, P, i32, P, P, i32]
     lib.ora_decode_topk.restype = ctypes.c_int32
+    lib.ora_decode_sel.argtypes = [P, P, ctypes.c_double, P, i32, P, P, i32, P, P, i32]
+    lib.ora_decode_sel.restype = ctypes.c_int32
+    lib.ora_l2_scores.argtypes = [P, P, ctypes.c_double, i32, i32, P]
+    lib.ora_l2_scores.restype = ctypes.c_int32
     lib.ora_sparse_top_k.argtypes = [ctypes.c_long]
     lib.ora_sparse_top_k.restype = ctypes.c_int32
     lib.ora_combine.argtypes = [i32, i32, i32, P, P, P, P]
@@ -141,12 +145,14 @@ class OracleCache:
     def lens(self):
         return np.array([self._lib.ora_len(self._h, b) for b in range(self.batch)], np.int32)
 
-    def decode(self, q, softmax_scale, pairs=None, nthreads=None, top_k=None):
+    def decode(self, q, softmax_scale, pairs=None, nthreads=None, top_k=None, sel=None):
         """q: float16 [batch][hq][d].  Returns (out float64 [batch][hq][d],
         lse float64 [batch][hq]); with `pairs` ([(b, h), ...]) only those rows
         are computed and the others are NaN.  top_k: sparse L2 blocks (each
-        head attends only the top_k of its INT4-block tokens, see
-        ora_decode_topk); None = dense."""
+        head attends only the top_k of its INT4-block tokens by attention
+        logit, see ora_decode_topk); None = dense.  sel: a given selection
+        instead, a list over rows r = b * hq + h of the L2 positions that row
+        attends (see ora_decode_sel)."""
         qq = _c(q, np.float16)
         out = np.full((self.batch, self.hq, self.d), np.nan)
         lse = np.full((self.batch, self.hq), np.nan)
@@ -156,12 +162,38 @@ class OracleCache:
             pp = _c(np.asarray(pairs, np.int32).reshape(-1, 2), np.int32)
             npairs = pp.shape[0]
         nt = nthreads or os.cpu_count() or 1
+        if sel is not None:
+            rows = self.batch * self.hq
+            assert len(sel) == rows
+            stride = max(1, max(len(x) for x in sel))
+            sa = np.zeros((rows, stride), np.int32)
+            cnt = np.zeros(rows, np.int32)
+            for r, x in enumerate(sel):
+                sa[r, :len(x)] = x
+                cnt[r] = len(x)
+            rc = self._lib.ora_decode_sel(self._h, _ptr(qq.view(np.uint16)), float(softmax_scale), _ptr(sa),
+                                          stride, _ptr(cnt), None if pp is None else _ptr(pp), npairs,
+                                          _ptr(out), _ptr(lse), nt)
+            if rc != 0:
+                raise ValueError("oracle decode_sel rejected the selection (rc=%d)" % rc)
+            return out, lse
         rc = self._lib.ora_decode_topk(self._h, _ptr(qq.view(np.uint16)), float(softmax_scale),
                                        -1 if top_k is None else int(top_k),
                                        None if pp is None else _ptr(pp), npairs, _ptr(out), _ptr(lse), nt)
         if rc != 0:
             raise MemoryError("oracle decode failed (rc=%d)" % rc)
         return out, lse
+
+    def l2_scores(self, q, softmax_scale, b, h):
+        """FP64 attention logits of the L2 tokens of sequence b for query head
+        h (the scores the top-k selection ranks), positions 0.. in order."""
+        qq = _c(q, np.float16)
+        buf = np.zeros(max(1, int(self.lens()[b])), np.float64)
+        n = self._lib.ora_l2_scores(self._h, _ptr(qq.view(np.uint16)), float(softmax_scale), int(b), int(h),
+                                    _ptr(buf))
+        if n < 0:
+            raise ValueError("oracle l2_scores rejected (b, h)")
+        return buf[:n].copy()
 
     def get_block(self, b, i):
         """(Q, codes int8 [hkv][2][block][d], scales float32 [hkv][2]); Q = 0 if unsealed."""

@@ -29,13 +29,13 @@
  *     the top-k attention scores; section 5.3: sparse_top_k, default 32, and
  *     the rule min(128, context_length / 256)): in ora_decode_topk each query
  *     head attends, of the tokens in its sequence's INT4 blocks, only the
- *     top_k with the largest scores (ties: the older position first), plus
- *     every other token.  The score that decides the selection is taken in
- *     the same FP32 / integer arithmetic as the GPU kernel (a decision that
- *     picks a discrete set must be made in one precision on both sides):
- *     q in 16-bit fixed point per head, qi = clamp(rint(q * (32767 / max|q|))),
- *     key = (float)(sum_c qi_c * code_c) * K-scale.  The attention over the
- *     selected set is exact FP64 as below.
+ *     top_k with the largest attention scores, plus every other token.  The
+ *     score of a token is its attention logit, softmax_scale * sum_c q_c *
+ *     (code_c * scale), in FP64 -- the same number the softmax below uses.
+ *     Equal scores keep the older position first.  ora_decode_sel attends a
+ *     given selection instead (any valid top-k set, for a caller whose
+ *     selection may resolve near-ties differently), and ora_l2_scores returns
+ *     the scores themselves.
  *   - Attention (section 4.2, steps 3-5): one softmax over hot and cold keys
  *     together, on the dequantized cold values (code * scale) and the FP16 hot
  *     values, evaluated here in FP64.  The page's torch.cat of two separately
@@ -369,13 +369,6 @@ static double kv_value(const ora_cache *c, int b, int h, int kv, int p, int ch) 
   return (double)code * (double)c->scale[bi][h * 2 + kv];
 }
 
-/*
- * Single-query decode attention, FP64, for the (b, query head) pairs listed in
- * `pairs` (2*npairs ints) or for all pairs when pairs == NULL.
- * q: FP16 [batch][hq][d].  Query head h reads kv head h / (hq/hkv).
- * out: [batch][hq][d], lse: [batch][hq] (natural log); entries of pairs not
- * listed are left untouched.  An empty sequence gives out = 0, lse = -inf.
- */
 /* Tokens of sequence b held in its INT4 ("L2") blocks: the oldest ones, in
  * logical blocks below n_int4[b] (every cold block when quant_bits is 4; none
  * with FP16 blocks). */
@@ -387,51 +380,69 @@ static int l2_tokens(const ora_cache *c, int b) {
   return cold < cap ? cold : (int)cap;
 }
 
-/* Selection key of L2 position p for a query head (see the header):
- * qi: the head's q in 16-bit fixed point. */
-static float l2_key(const ora_cache *c, int b, int hk, int p, const int32_t *qi) {
-  const int i = p / c->block;
-  const size_t bi = (size_t)b * c->max_blocks + i;
-  const int8_t *codes = c->codes[bi] + (((size_t)hk * 2 + 0) * c->block + (p - i * c->block)) * c->d;
-  int64_t dot = 0;
-  for (int ch = 0; ch < c->d; ch++) dot += (int64_t)qi[ch] * codes[ch];
-  const float sk = c->scale[bi][(size_t)hk * 2 + 0];
-  return (float)dot * sk;
+/* Attention logit of position p for query head qh (kv head hk), FP64:
+ * softmax_scale * sum_c q_c * K_{p,c}, K from kv_value. */
+static double logit(const ora_cache *c, int b, int hk, const uint16_t *qh, double softmax_scale, int p) {
+  double acc = 0.0;
+  for (int ch = 0; ch < c->d; ch++) acc += (double)half_to_float(qh[ch]) * kv_value(c, b, hk, 0, p, ch);
+  return softmax_scale * acc;
 }
 
-static void q_fixed16(const uint16_t *qh, int d, int32_t *qi) {
-  float amax = 0.0f;
-  for (int ch = 0; ch < d; ch++) {
-    const float a = fabsf(half_to_float(qh[ch]));
-    if (a > amax) amax = a;
-  }
-  const float inv = amax > 0.0f ? 32767.0f / amax : 0.0f;
-  for (int ch = 0; ch < d; ch++) {
-    const float t = half_to_float(qh[ch]) * inv;
-    long v = lrintf(t);
-    if (v > 32767) v = 32767;
-    if (v < -32767) v = -32767;
-    qi[ch] = (int32_t)v;
-  }
-}
+typedef struct { double key; int pos; } l2_cand;
 
-typedef struct { float key; int pos; } l2_cand;
-
-/* Order: larger key first, then the older position. */
+/* Order: larger score first, then the older position. */
 static int cand_cmp(const void *x, const void *y) {
   const l2_cand *a = (const l2_cand *)x, *b = (const l2_cand *)y;
   if (a->key != b->key) return a->key > b->key ? -1 : 1;
   return a->pos - b->pos;
 }
 
+static int cmp_int(const void *x, const void *y) {
+  const int a = *(const int *)x, b = *(const int *)y;
+  return a < b ? -1 : (a > b);
+}
+
+/* Softmax attention of query head hh (kv head hk) over the n positions pos[]
+ * of sequence b, FP64: o[d], *lse (natural log); no position: o = 0, -inf. */
+static void attend(const ora_cache *c, int b, int hk, const uint16_t *qh, double softmax_scale,
+                   const int *pos, int n, double *z, double *o, double *lse) {
+  double m = -INFINITY;
+  for (int j = 0; j < n; j++) {
+    z[j] = logit(c, b, hk, qh, softmax_scale, pos[j]);
+    if (z[j] > m) m = z[j];
+  }
+  double l = 0.0;
+  for (int j = 0; j < n; j++) {
+    z[j] = exp(z[j] - m);
+    l += z[j];
+  }
+  for (int ch = 0; ch < c->d; ch++) {
+    double acc = 0.0;
+    for (int j = 0; j < n; j++) acc += z[j] * kv_value(c, b, hk, 1, pos[j], ch);
+    o[ch] = n > 0 ? acc / l : 0.0;
+  }
+  *lse = n > 0 ? m + log(l) : -INFINITY;
+}
+
 /*
- * Decode attention: out[b][h][:] and lse[b][h] (natural log) for every
- * (sequence, query head), or only the npairs (b, h) pairs given.  top_k < 0:
- * dense (every token).  top_k >= 0: of the L2 tokens only the top_k
- * selected as the header describes (all of them when there are no more).
+ * Single-query decode attention, FP64, for the (b, query head) pairs listed in
+ * `pairs` (2*npairs ints) or for all pairs when pairs == NULL.
+ * q: FP16 [batch][hq][d].  Query head h reads kv head h / (hq/hkv).
+ * out: [batch][hq][d], lse: [batch][hq] (natural log); entries of pairs not
+ * listed are left untouched.  An empty sequence gives out = 0, lse = -inf.
+ * The L2 tokens a row attends:
+ *   sel == NULL, top_k < 0:  all of them (dense);
+ *   sel == NULL, top_k >= 0: the top_k with the largest logits (ties: the
+ *                            older position), all of them when there are no
+ *                            more;
+ *   sel != NULL:             the sel_count[r] positions sel[r * sel_stride
+ *                            ...] of row r = b * hq + h (each must be an L2
+ *                            position of b, no repeats), for any top_k.
+ * Every token that is not in an L2 block is attended.
  */
-int ora_decode_topk(const ora_cache *c, const uint16_t *q, double softmax_scale, int top_k,
-                    const int32_t *pairs, int npairs, double *out, double *lse, int nthreads) {
+static int decode_rows(const ora_cache *c, const uint16_t *q, double softmax_scale, int top_k,
+                       const int32_t *sel, int sel_stride, const int32_t *sel_count, const int32_t *pairs,
+                       int npairs, double *out, double *lse, int nthreads) {
   const int d = c->d, g = c->hq / c->hkv;
   const int total = pairs ? npairs : c->batch * c->hq;
   if (nthreads < 1) nthreads = 1;
@@ -440,63 +451,78 @@ int ora_decode_topk(const ora_cache *c, const uint16_t *q, double softmax_scale,
   for (int w = 0; w < total; w++) {
     const int b = pairs ? pairs[2 * w] : w / c->hq;
     const int hh = pairs ? pairs[2 * w + 1] : w % c->hq;
+    const size_t row = (size_t)b * c->hq + hh;
     const int hk = hh / g;
     const int L = c->len[b];
-    double *o = out + ((size_t)b * c->hq + hh) * d;
-    if (L == 0) {
-      for (int ch = 0; ch < d; ch++) o[ch] = 0.0;
-      lse[(size_t)b * c->hq + hh] = -INFINITY;
+    const uint16_t *qh = q + row * d;
+    int *pos = (int *)malloc(sizeof(int) * (L > 0 ? L : 1));
+    double *z = (double *)malloc(sizeof(double) * (L > 0 ? L : 1));
+    if (!pos || !z) {
+      bad = 1;
+      free(pos); free(z);
       continue;
     }
-    const uint16_t *qh = q + ((size_t)b * c->hq + hh) * d;
-    /* the positions attended */
-    int *pos = (int *)malloc(sizeof(int) * L);
     int n = 0;
-    const int n2 = top_k < 0 ? 0 : l2_tokens(c, b);
-    if (n2 > 0) {
-      int32_t *qi = (int32_t *)malloc(sizeof(int32_t) * d);
+    const int n2 = (top_k < 0 && !sel) ? 0 : l2_tokens(c, b);
+    if (sel) {
+      const int cnt = sel_count[row];
+      if (cnt < 0 || cnt > n2) bad = 1;
+      for (int t = 0; t < cnt && t < n2; t++) {
+        const int p = sel[row * (size_t)sel_stride + t];
+        if (p < 0 || p >= n2) {
+          bad = 1;
+          continue;
+        }
+        pos[n++] = p;
+      }
+      qsort(pos, n, sizeof(int), cmp_int);
+      for (int t = 1; t < n; t++)
+        if (pos[t] == pos[t - 1]) bad = 1;
+    } else if (n2 > 0) {
       l2_cand *cand = (l2_cand *)malloc(sizeof(l2_cand) * n2);
-      if (!qi || !cand || !pos) {
+      if (!cand) {
         bad = 1;
-        free(qi); free(cand); free(pos);
+        free(pos); free(z);
         continue;
       }
-      q_fixed16(qh, d, qi);
       for (int p = 0; p < n2; p++) {
-        cand[p].key = l2_key(c, b, hk, p, qi);
+        cand[p].key = logit(c, b, hk, qh, softmax_scale, p);
         cand[p].pos = p;
       }
       qsort(cand, n2, sizeof(l2_cand), cand_cmp);
       const int keep = top_k < n2 ? top_k : n2;
       for (int t = 0; t < keep; t++) pos[n++] = cand[t].pos;
-      free(qi);
+      qsort(pos, n, sizeof(int), cmp_int);
       free(cand);
     }
     for (int p = n2; p < L; p++) pos[n++] = p;
-    double *z = (double *)malloc(sizeof(double) * (n > 0 ? n : 1));
-    double m = -INFINITY;
-    for (int j = 0; j < n; j++) {
-      double acc = 0.0;
-      for (int ch = 0; ch < d; ch++)
-        acc += (double)half_to_float(qh[ch]) * kv_value(c, b, hk, 0, pos[j], ch);
-      z[j] = softmax_scale * acc;
-      if (z[j] > m) m = z[j];
-    }
-    double l = 0.0;
-    for (int j = 0; j < n; j++) {
-      z[j] = exp(z[j] - m);
-      l += z[j];
-    }
-    for (int ch = 0; ch < d; ch++) {
-      double acc = 0.0;
-      for (int j = 0; j < n; j++) acc += z[j] * kv_value(c, b, hk, 1, pos[j], ch);
-      o[ch] = n > 0 ? acc / l : 0.0;
-    }
-    lse[(size_t)b * c->hq + hh] = n > 0 ? m + log(l) : -INFINITY;
+    attend(c, b, hk, qh, softmax_scale, pos, n, z, out + row * d, &lse[row]);
     free(z);
     free(pos);
   }
-  return bad ? ORA_ERR_NOMEM : ORA_OK;
+  return bad ? ORA_ERR_INVALID : ORA_OK;
+}
+
+int ora_decode_topk(const ora_cache *c, const uint16_t *q, double softmax_scale, int top_k,
+                    const int32_t *pairs, int npairs, double *out, double *lse, int nthreads) {
+  return decode_rows(c, q, softmax_scale, top_k, NULL, 0, NULL, pairs, npairs, out, lse, nthreads);
+}
+
+int ora_decode_sel(const ora_cache *c, const uint16_t *q, double softmax_scale, const int32_t *sel,
+                   int sel_stride, const int32_t *sel_count, const int32_t *pairs, int npairs, double *out,
+                   double *lse, int nthreads) {
+  if (!sel || !sel_count || sel_stride < 0) return ORA_ERR_INVALID;
+  return decode_rows(c, q, softmax_scale, 0, sel, sel_stride, sel_count, pairs, npairs, out, lse, nthreads);
+}
+
+/* The attention logits of the L2 tokens of sequence b for query head hh (the
+ * scores the top-k selection ranks): scores[p] for p < the returned count. */
+int ora_l2_scores(const ora_cache *c, const uint16_t *q, double softmax_scale, int b, int hh, double *scores) {
+  if (b < 0 || b >= c->batch || hh < 0 || hh >= c->hq) return ORA_ERR_INVALID;
+  const int n2 = l2_tokens(c, b);
+  const uint16_t *qh = q + ((size_t)b * c->hq + hh) * c->d;
+  for (int p = 0; p < n2; p++) scores[p] = logit(c, b, hh / (c->hq / c->hkv), qh, softmax_scale, p);
+  return n2;
 }
 
 int ora_decode(const ora_cache *c, const uint16_t *q, double softmax_scale,

@@ -2,8 +2,13 @@
 
 Source: web page "DeepSeek V4混合式KV Cache推理优化实战解析", section 2.2 (the
 L2 cold blocks keep only the KV of the top-k attention scores) and section
-5.3 (sparse_top_k, default 32; rule min(128, context_length // 256)).  Pins:
-the dense result when k covers every L2 token or there is no L2 block;
+5.3 (sparse_top_k, default 32; rule min(128, context_length // 256)).  The
+score of a token is its FP64 attention logit.  Pins: a hand-worked selection
+whose scores are exact in FP64, with a near-tie that 16-bit fixed-point q
+would resolve differently (tests/golden/sparse_select.txt); brute force on
+small random caches (numpy logits on K rebuilt from the stored codes, ranked
+by numpy); the dense result when k covers every L2 token or there is no L2
+block;
 planted tokens whose scores stand far above the rest are exactly the ones
 kept (checked against dense brute force over that set, rebuilt from the
 stored codes); equal scores keep the oldest positions; k = 0 drops the L2
@@ -14,7 +19,7 @@ import pytest
 from scipy.special import logsumexp, softmax
 
 import oracle
-from golden_cases import D
+from golden_cases import D, GOLDEN
 
 BLOCK = 64
 
@@ -125,3 +130,94 @@ def test_sparse_top_k_rule():
     assert oracle.sparse_top_k(8192) == 32
     assert oracle.sparse_top_k(255) == 0
     assert oracle.sparse_top_k(10 ** 7) == 128
+
+
+def _fixture():
+    cfg, q, ktok, scores, sel = {}, {}, {}, {}, {}
+    with open(GOLDEN + "/sparse_select.txt", encoding="utf-8") as f:
+        for raw in f:
+            line = raw.split("#", 1)[0].split()
+            if not line:
+                continue
+            if line[0] == "config":
+                cfg = {k: int(v) for k, v in (x.split("=") for x in line[1:])}
+            elif line[0] == "q":
+                q = {int(a): float(b) for a, b in (x.split("=") for x in line[1:])}
+            elif line[0] == "ktok":
+                ktok[int(line[1])] = {int(a): float(b) for a, b in (x.split("=") for x in line[2:])}
+            elif line[0] == "score":
+                scores[int(line[1])] = float(line[2])
+            elif line[0] == "select":
+                sel[int(line[1])] = [int(x) for x in line[2:]]
+    return cfg, q, ktok, scores, sel
+
+
+def test_golden_selection():
+    """The hand-worked fixture: exact FP64 scores, the kept sets for every
+    listed top_k (near-ties decided by the 2^-20 term, exact ties by age)."""
+    cfg, qd, ktok, scores, sel = _fixture()
+    L, n4 = cfg["L"], cfg["n_int4"]
+    oc = oracle.OracleCache(1, 1, 1, max_blocks_per_seq=2, quant_bits=8)
+    oc.set_n_int4(np.array([n4], np.int32))
+    k = np.zeros((1, L, 1, D), np.float32)
+    for p, vals in ktok.items():
+        for ch, val in vals.items():
+            k[0, p, 0, ch] = val
+    v = np.random.default_rng(21).standard_normal((1, L, 1, D)).astype(np.float16)
+    oc.append(np.array([L], np.int32), k.astype(np.float16), v)
+    q = np.zeros((1, 1, D), np.float32)
+    for ch, val in qd.items():
+        q[0, 0, ch] = val
+    q = q.astype(np.float16)
+    assert float(q[0, 0, 1]) == 2.0 ** -20  # exact in FP16
+    got = oc.l2_scores(q, 1.0, 0, 0)
+    assert got.shape == (64,)
+    for p in range(64):
+        assert got[p] == scores.get(p, 0.0), (p, got[p])
+    K, V = _dense_kv(oc, 0, L)
+    for kk, want in sel.items():
+        keep = want + list(range(64, L))
+        ref, ref_l = _attend(q[0, 0], K, V, keep, 1.0, 0)
+        out, lse = oc.decode(q, 1.0, top_k=kk)
+        assert np.abs(out[0, 0] - ref).max() < 1e-12 and abs(lse[0, 0] - ref_l) < 1e-12, kk
+        # the same rows through an explicit selection
+        out2, lse2 = oc.decode(q, 1.0, sel=[want])
+        assert np.array_equal(out2, out) and np.array_equal(lse2, lse), kk
+    # a wrong set (the fixed-point answer for top_k = 2) gives another output
+    wrong, _ = _attend(q[0, 0], K, V, [5, 9] + list(range(64, L)), 1.0, 0)
+    out, _ = oc.decode(q, 1.0, top_k=2)
+    assert np.abs(out[0, 0] - wrong).max() > 1e-3
+
+
+@pytest.mark.parametrize("seed,qbits,hkv,hq,scale", [(0, 8, 1, 2, 0.088), (1, 8, 2, 8, 1.0), (2, 4, 1, 4, 0.3),
+                                                     (3, 8, 1, 1, -0.5)])
+def test_selection_matches_brute_force(seed, qbits, hkv, hq, scale):
+    """Random caches: the kept set is numpy's top_k of numpy logits on K
+    rebuilt position by position (ties, which random data does not produce,
+    would go to the older position), for several top_k; the output is dense
+    softmax attention over that set."""
+    L = 350
+    n4 = 3
+    oc = _cache(L, n4, hkv=hkv, hq=hq, qbits=qbits, seed=10 + seed)
+    q = np.random.default_rng(40 + seed).standard_normal((1, hq, D)).astype(np.float16)
+    K, V = _dense_kv(oc, 0, L)
+    n2 = min(L - 32, (n4 if qbits == 8 else 99) * BLOCK)
+    g = hq // hkv
+    for kk in (0, 1, 5, 40, n2 - 1):
+        out, lse = oc.decode(q, scale, top_k=kk)
+        for h in range(hq):
+            z = scale * (K[:n2, h // g, :] @ q[0, h].astype(np.float64))
+            order = np.lexsort((np.arange(n2), -z))
+            keep = sorted(order[:kk].tolist()) + list(range(n2, L))
+            want, wl = _attend(q[0, h], K, V, keep, scale, h // g)
+            assert np.abs(out[0, h] - want).max() < 1e-12 and abs(lse[0, h] - wl) < 1e-12, (kk, h)
+            sc = oc.l2_scores(q, scale, 0, h)
+            assert np.allclose(sc, z, rtol=0, atol=1e-12)
+
+
+def test_selection_rejects_bad_sets():
+    oc = _cache(300, 2, seed=9)
+    q = np.random.default_rng(3).standard_normal((1, 1, D)).astype(np.float16)
+    for bad in ([200], [3, 3], [-1]):
+        with pytest.raises(ValueError):
+            oc.decode(q, 0.1, sel=[bad])
