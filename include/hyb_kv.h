@@ -294,6 +294,23 @@ int hyb_decode_attn_sparse(const hyb_cache_desc *desc, const void *q, float soft
 size_t hyb_decode_sparse_workspace_bytes(const hyb_cache_desc *desc, int32_t max_seq_len,
                                          int32_t split_tokens);
 
+/*
+ * Where hyb_decode_attn_sparse leaves its selection ([hybrid_v2 page] 2.2:
+ * which L2 tokens each query head kept).  Returns the byte offset, inside a
+ * workspace sized by hyb_decode_sparse_workspace_bytes() for the same
+ * (desc, max_seq_len, split_tokens), of an int32 array [batch][Hq][stride]
+ * (*row_stride = stride, at most 1024): after a call with top_k > 0, row
+ * (b, h) holds in its first min(top_k, L2 tokens of b) entries the positions
+ * attended, ascending (a position p < L2 tokens of b is token p of the
+ * sequence); other entries, and every entry of a row whose sequence has no
+ * L2 token or of a call with top_k 0, are left as they were.  The offset is
+ * never 0 for a valid descriptor; 0 means invalid arguments.  Host only;
+ * reading the array is the caller's (device memory, after the stream
+ * completes).
+ */
+size_t hyb_decode_sparse_selection(const hyb_cache_desc *desc, int32_t max_seq_len, int32_t split_tokens,
+                                   int32_t *row_stride);
+
 /* The page's sparse_top_k rule ([hybrid_v2 page] 5.3): min(128,
  * context_length / 256) (0 for a negative length).  Host only. */
 int hyb_sparse_top_k(int64_t context_length);
@@ -426,6 +443,22 @@ int hyb_migration_decision(double avg_interval_ms, double threshold_ms, int32_t 
  * reset it to 0 when `clear` is nonzero. */
 int hyb_read_status(const hyb_cache_desc *desc, int32_t *host_status, int32_t clear,
                     hyb_stream_t stream);
+
+/*
+ * Limit, in SM clock cycles, of each bounded wait of the decode kernel's
+ * copy pipeline (a stage's data landing, a stage being released), for every
+ * later hyb_decode_attn / hyb_decode_step / hyb_decode_attn_sparse /
+ * hyb_decode_attn_noalloc launch of this process.  cycles <= 0 restores the
+ * default, 2^31 cycles (about 1 s at B200 clocks).  No counterpart in the
+ * pages: it exists so that the timeout path can be exercised -- with a limit
+ * of a few cycles the first wait gives up, the kernel records
+ * HYB_STATUS_TIMEOUT, lets every bulk copy it issued land (that drain wait
+ * always keeps the default limit), and returns with its rows' output zero
+ * and log-sum-exp -inf.  A timed-out hyb_decode_step may have appended its
+ * token to some kv heads and not others; the status word says the step
+ * failed.  Host only; takes effect at the next launch.  Returns HYB_OK.
+ */
+int hyb_set_wait_limit(int64_t cycles);
 
 /* Text of a HYB_ERR_* return code or HYB_STATUS_* code (status codes are
  * passed as 100 + code). Never NULL. */

@@ -34,7 +34,8 @@ EXPORTED = (
     "hyb_read_status", "hyb_strerror",
     "hyb_last_cuda_error", "hyb_version", "hyb_decode_attn_noalloc", "hyb_noalloc_scratch_limit",
     "hyb_kv_migrate", "hyb_migration_threshold_ms", "hyb_migration_decision",
-    "hyb_decode_attn_sparse", "hyb_decode_sparse_workspace_bytes", "hyb_sparse_top_k",
+    "hyb_decode_attn_sparse", "hyb_decode_sparse_workspace_bytes", "hyb_decode_sparse_selection",
+    "hyb_sparse_top_k", "hyb_set_wait_limit",
 )
 
 
@@ -90,6 +91,9 @@ def load(path: str = LIB_PATH):
     lib.hyb_decode_attn_sparse.argtypes = [D, P, ctypes.c_float, i32, i32, i32, P, sz, P, P, P]
     lib.hyb_decode_sparse_workspace_bytes.argtypes = [D, i32, i32]
     lib.hyb_decode_sparse_workspace_bytes.restype = sz
+    lib.hyb_decode_sparse_selection.argtypes = [D, i32, i32, ctypes.POINTER(ctypes.c_int32)]
+    lib.hyb_decode_sparse_selection.restype = sz
+    lib.hyb_set_wait_limit.argtypes = [ctypes.c_int64]
     lib.hyb_sparse_top_k.argtypes = [ctypes.c_int64]
     lib.hyb_sparse_top_k.restype = i32
     lib.hyb_decode_step.argtypes = [D, P, P, P, P, ctypes.c_float, i32, i32, P, sz, P, P, P]
@@ -167,6 +171,17 @@ def hyb_decode_sparse_workspace_bytes(desc, max_seq_len, split_tokens=0) -> int:
     return int(load().hyb_decode_sparse_workspace_bytes(ctypes.byref(desc), int(max_seq_len), int(split_tokens)))
 
 
+def hyb_decode_sparse_selection(desc, max_seq_len, split_tokens=0):
+    """(byte offset in the sparse workspace, row stride) of the selected L2
+    positions; raises on invalid arguments."""
+    stride = ctypes.c_int32(0)
+    off = int(load().hyb_decode_sparse_selection(ctypes.byref(desc), int(max_seq_len), int(split_tokens),
+                                                  ctypes.byref(stride)))
+    if off == 0:
+        raise HybError(HYB_ERR_INVALID_VALUE, "hyb_decode_sparse_selection")
+    return off, stride.value
+
+
 def hyb_decode_attn_sparse(desc, q, softmax_scale, max_seq_len, split_tokens, top_k, workspace, out,
                            lse_out=None, stream=None):
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -235,6 +250,11 @@ def hyb_read_status(desc, clear=False, stream=None) -> int:
     _check(load().hyb_read_status(ctypes.byref(desc), ctypes.byref(v), 1 if clear else 0,
                                   _stream(stream)), "hyb_read_status")
     return v.value
+
+
+def hyb_set_wait_limit(cycles: int) -> None:
+    """Limit (SM cycles) of the decode pipeline's bounded waits; <= 0 restores the default."""
+    _check(load().hyb_set_wait_limit(int(cycles)), "hyb_set_wait_limit")
 
 
 def hyb_last_cuda_error() -> int:

@@ -123,6 +123,15 @@ class HybridKVCache:
                                     out, lse, stream)
         return out
 
+    def sparse_selection(self, workspace, max_seq_len, split_tokens=0):
+        """The selected L2 positions the last decode_sparse call with this
+        workspace left: int32 CUDA view [batch][Hq][stride] (row (b, h): the
+        first min(top_k, L2 tokens of b) entries, ascending)."""
+        import torch
+        off, stride = _lib.hyb_decode_sparse_selection(self.desc, max_seq_len, split_tokens)
+        n = self.batch * self.hq * stride * 4
+        return workspace[off:off + n].view(torch.int32).view(self.batch, self.hq, stride)
+
     def step_workspace(self, max_seq_len, split_tokens=0):
         import torch
         n = _lib.hyb_decode_step_workspace_bytes(self.desc, max_seq_len, split_tokens)

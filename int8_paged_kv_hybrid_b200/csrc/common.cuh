@@ -89,6 +89,12 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       : "memory");
 }
 
+// Order this thread's generic-proxy writes to shared memory before later
+// async-proxy (bulk copy) writes to the same bytes.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // L2 policy for data read once per decode step (KV tiles): evict first.
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t pol;

@@ -1,554 +1,17 @@
-// decode.cu -- hyb_decode_attn: split-KV single-query attention over the
-// hybrid_v2 cache (FP16 hot ring + INT8/INT4 cold blocks behind a block
-// table) on sm_100a CUDA cores.
-//
-// Method: web page "DeepSeek V4混合式KV Cache推理优化实战解析", section 4.2
-// (attention over the FP16 hot zone plus the dequantized cold zone; one
-// softmax over both, merged by log-sum-exp instead of the page's torch.cat),
-// section 3.2 (hot zone: K and V interleaved per token, 512-byte aligned).
-//
-// Work decomposition: one CTA (4 warps) per (split, kv head, sequence).  A
-// split is a run of up to `split_blocks` cold blocks; the split that holds
-// the sequence's last cold block also attends the hot ring.  Pipeline items:
-// a 64-token sub-block of a cold block (K tile 8 KB + V tile 8 KB, or 4 + 4
-// KB for INT4; a 128-token block is two, a 32-token block the first half of
-// one), 32 FP16 rows (16 KB) of an FP16 cold block, and 32 rows of the hot
-// ring.  Each item is brought into a 3-stage shared-memory ring by the TMA
-// engine with 1-D bulk copies (no cluster multicast) completing on an
-// mbarrier; every wait is bounded.  Three CTAs fit on an SM for up to 4 query
-// heads per kv head (two above that).  When all splits are resident at once
-// (one wave) 2..8 splits of a (sequence, kv head) run as one thread-block
-// cluster and merge through distributed shared memory; otherwise the last
-// split to finish merges them from the workspace.
-//
-// Arithmetic (per kv head, for its G = Hq/Hkv query heads):
-//  * q is turned into 16-bit fixed point per query head (q_i = rint(q * 32767
-//    / max|q|)); a cold logit is the exact int32 dot product of q_i with the
-//    K codes (dp2a: two 16x8-bit products per instruction), times
-//    max|q|/32767 * K-scale * softmax_scale * log2(e).  Eight lanes share a
-//    token (16 channels each); each lane keeps its heads in a lane-dependent
-//    order (head = k XOR x(lane)) so the cross-lane reduction that leaves one
-//    head's total in each lane needs no selects.
-//  * Warp w owns tokens 16w..16w+15 of every block and keeps its own online
-//    softmax state (running max, sum, FP32 output accumulator) per head,
-//    rescaling only when the running max grows.  Its softmax weights relative
-//    to the running maximum are 16-bit fixed point (p_i = rint(32767 *
-//    2^(z - max))); P.V is again an exact int32 dp2a sum over the V codes,
-//    folded into the FP32 state with the V scale.
-//  * Hot tokens are attended in FP32 from the FP16 values (never quantized).
-//  * The 4 warp states are merged in FP32 at the end of the split; the last
-//    CTA of a (sequence, kv head) to finish merges the splits (log-sum-exp)
-//    and writes the FP16 output.
-// Tensor cores are not used: per byte of KV the work is a few integer
-// multiply-adds (a GEMV per kv head), so the roof is HBM bandwidth; the
-// measured loop is bound by the latency of that integer work.
-#include "decode_dev.cuh"
+// decode.cu -- dispatch of hyb_decode_attn / hyb_decode_step launches to the
+// decode kernel's instantiations (decode_kernel.cuh; one translation unit per
+// block size and variant, decode_b*_*.cu), and the kernel's launch limits.
+#include "kernels.cuh"
 
 namespace hyb {
 
-constexpr int kMaxSplitBlocks = 128;  // == kThreads: one block-table entry per thread
-
-template <int G>
-struct DecodeSmem {
-  static constexpr int P = pow2_heads<G>();
-  alignas(128) uint8_t ring[kStages][kTilePairBytes];
-  uint64_t full[kStages];   // data of the stage landed (TMA transaction count)
-  uint64_t empty[kStages];  // every warp is done with the stage
-  int32_t phys[kMaxSplitBlocks];
-  float2 scl[kMaxSplitBlocks];  // (K scale, V scale) of each block of the split
-  alignas(16) float qf[P][kDim];     // q in FP32 (rows >= G are zero)
-  alignas(16) int16_t qi[P][kDim];   // q in 16-bit fixed point (rows >= G are zero)
-  float sq[P];                       // fixed-point step of each head's q
-  alignas(16) uint16_t pcode[kWarps][G][16];
-  alignas(16) float phot[kWarps][G][8];
-  float mrun[kWarps][G];
-  float lrun[kWarps][G];
-  SealScratch seal;  // fused step
-  float cl_l[G];   // this split's log2-sum-exp per head, read by the cluster's merge
-  int last;
-  int abort_flag;
-};
-
-// kCluster: the grid is launched in clusters of n_splits CTAs (the splits of
-// one (sequence, kv head)); splits are merged through distributed shared
-// memory instead of the workspace.  kF16: FP16 cold blocks (quantization_bits
-// 0), each attended as two items of 32 rows with the hot ring's arithmetic.
-// kSkip: sparse L2 mode -- the sequence's INT4 ("L2") blocks are left to the
-// top-k kernels, and the splits cover the blocks from its INT4 count on.
-// kBshift: log2 of the tokens per block (block_size 32: 5, 64: 6, 128: 7); a
-// 128-token block is two 64-token sub-blocks, a 32-token block the first half
-// of one.
-template <int G, bool kCluster, bool kF16, bool kSkip, int kBshift>
-__global__ void __launch_bounds__(kThreads, (G <= 4 ? 3 : 2)) decode_kernel(const DecodeArgs a) {
-  constexpr int P = pow2_heads<G>();
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  DecodeSmem<G> &sm = *reinterpret_cast<DecodeSmem<G> *>(smem_raw);
-
-  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int S = a.n_splits;
-  const int hq0 = h * G;
-  int ib = 0;  // first block of the splits
-  if constexpr (kSkip) {
-    const int n4 = a.quant_bits == 4 ? a.max_blocks : (a.n_int4 ? a.n_int4[b] : 0);
-    ib = min(max(n4, 0), a.max_blocks);
-  }
-  const int i0 = ib + s * a.split_blocks;
-
-  // independent loads first: the sequence length, this split's block-table
-  // entries (one per thread, clamped to the row) and q
-  const int L_old = a.seq_lens[b];
-  int n_app = a.n_new ? a.n_new[b] : 0;  // fused step: tokens appended to this sequence
-  const int i_tid = i0 + tid;
-  const int phys_raw =
-      (tid < a.split_blocks && i_tid < a.max_blocks) ? a.block_table[(size_t)b * a.max_blocks + i_tid] : -1;
-  float qv[G];
-#pragma unroll
-  for (int j = 0; j < G; j++) qv[j] = __half2float(a.q[((size_t)b * a.hq + hq0) * kDim + j * kDim + tid]);
-
-  if (n_app < 0 || n_app > 1) {
-    if (tid == 0 && s == 0 && h == 0) set_status(a.status, HYB_STATUS_BAD_N_NEW);
-    n_app = 0;
-  }
-  int L = L_old + n_app;
-  if (L_old < 0 || L > a.max_seq_len) {
-    // sequence skipped: treated as empty (zero output, lse -inf), not appended to
-    if (tid == 0 && s == 0 && h == 0) set_status(a.status, HYB_STATUS_SEQ_LEN);
-    L = 0;
-    n_app = 0;
-  }
-  if (a.n_new && tid == 32) {
-    // every CTA of the grid has read seq_lens[b] once this count is complete;
-    // the last one advances it
-    const int ticket = atomicAdd(&a.seq_cnt[b], 1);
-    if (ticket == static_cast<int>(gridDim.x * gridDim.y) - 1) {
-      a.seq_lens[b] = L_old + n_app;
-      a.seq_cnt[b] = 0;
-    }
-  }
-  const int H = a.hot_tokens;
-  const int Lc = max(0, L - H);
-  constexpr int lsub = kBshift > 6 ? kBshift - 6 : 0;  // a block is 1 << lsub sub-blocks
-  constexpr int Bt = 1 << kBshift;                      // tokens per block
-  constexpr int St = Bt < kBlock ? Bt : kBlock;         // tokens per sub-block
-  const int nblk = (Lc + Bt - 1) / Bt;
-  const int Sb = max(1, (max(0, nblk - ib) + a.split_blocks - 1) / a.split_blocks);
-  // past this sequence's last split: no work and no partial (a cluster member
-  // still takes part in the cluster's merge, with an empty state)
-  if (!kCluster && s >= Sb) return;
-  const int ncold = max(0, min(nblk, i0 + a.split_blocks) - i0);
-  // Items: one per 64-token sub-block (16 KB K + V tiles), or per 32 rows of
-  // FP16 (the hot ring, FP16 cold blocks: 2 << lsub items per block)
-  const int nhot = (s == Sb - 1) ? min(L, H) : 0;
-  constexpr bool fp16 = kF16;
-  constexpr int ish = fp16 ? kBshift - 5 : lsub;  // log2 of the items per block
-  const int ncold_it = ncold << ish;
-  const int kh = ncold_it;  // the first hot item
-  const int nitems = ncold_it + (nhot + kItemRows - 1) / kItemRows;
-  // fused step, in the split that holds the tail block and the hot ring: the
-  // new token goes to ring slot rs = L_old % hot, whose old occupant
-  // (position L_old - hot, read in the prologue) is sealed into the tail
-  // block at that block's item; the ring slot is rewritten at its hot item
-  const bool do_ring = n_app == 1 && nhot > 0;
-  const bool do_seal = do_ring && L_old >= H;
-  const int rs = L_old & (H - 1);
-  const int k_ring = kh + rs / kItemRows;
-  // slot of the sealed token in the tail block; in the split that seals, the
-  // tail block's sub-blocks run last-first, so that a scale the seal grows
-  // reaches the earlier sub-block before that one is attended (k_rq)
-  const int slot_e = do_seal ? (L_old - H) % Bt : 0;
-  const int nsub1 = (1 << lsub) - 1;
-  const int k_seal = !do_seal ? -1
-                     : fp16   ? ((ncold - 1) << ish) + slot_e / kItemRows
-                              : ((ncold - 1) << lsub) + nsub1 - (slot_e >> 6);
-  const int k_rq = (!fp16 && do_seal && (slot_e >> 6) > 0) ? ((ncold - 1) << lsub) + nsub1 : -1;
-  // item k: its block, and (cold INT8/INT4 items) its sub-block
-  auto item_block = [&](int k) { return k >> ish; };
-  auto item_sub = [&](int k) {
-    const int part = k & ((1 << ish) - 1);
-    return (do_seal && (k >> ish) == ncold - 1) ? nsub1 - part : part;
-  };
-  __half2 new_kv = __halves2half2(__float2half_rn(0.f), __float2half_rn(0.f));
-  __half2 old_kv = new_kv;
-  if (do_ring) {
-    const size_t o = ((size_t)b * a.hkv + h) * kDim + tid;
-    new_kv = __halves2half2(a.k_new[o], a.v_new[o]);
-    if (do_seal) {
-      const __half *er = reinterpret_cast<const __half *>(a.hot) + (((size_t)b * a.hkv + h) * H + rs) * 2 * kDim;
-      old_kv = __halves2half2(er[tid], er[kDim + tid]);
-    }
-  }
-  const int n_int4_b = a.quant_bits == 4 ? 0x7fffffff : (a.n_int4 ? a.n_int4[b] : 0);
-
-  if (tid == 0) {
-#pragma unroll
-    for (int st = 0; st < kStages; st++) {
-      mbar_init(&sm.full[st], 1);
-      mbar_init(&sm.empty[st], kWarps);
-    }
-    sm.abort_flag = 0;
-    mbar_fence_init();
-  }
-  if (do_seal) {
-    sm.seal.erow[tid] = __low2half(old_kv);
-    sm.seal.erow[kDim + tid] = __high2half(old_kv);
-  }
-  if (tid < ncold) {
-    int phys = phys_raw;
-    if (phys < 0 || phys >= a.num_phys) {
-      set_status(a.status, HYB_STATUS_BAD_BLOCK);
-      phys = -1;
-    }
-    sm.phys[tid] = phys;
-  }
-#pragma unroll
-  for (int j = 0; j < P; j++) sm.qf[j][tid] = j < G ? qv[j] : 0.f;
-  __syncthreads();
-
-  const uint64_t pol = l2_policy_evict_first();
-  auto issue = [&](int k) {
-    const int st = k % kStages;
-    uint8_t *dst = sm.ring[st];
-    if (k < ncold_it) {
-      const int kb = item_block(k);
-      const int phys = sm.phys[kb];
-      const int part = k & ((1 << ish) - 1);
-      const int u = fp16 ? 0 : item_sub(k);
-      const int nrow = fp16 ? min(kItemRows, Lc - (i0 + kb) * Bt - part * kItemRows)
-                            : Lc - (i0 + kb) * Bt - u * kBlock;
-      if (phys < 0 || nrow <= 0) {
-        mbar_arrive(&sm.full[st]);
-        return;
-      }
-      if (fp16) {
-        // 32 of the block's sealed rows
-        const uint8_t *src = a.cold + ((size_t)phys * a.hkv + h) * Bt * kHotTokenBytes + part * kItemBytes;
-        const uint32_t bytes = static_cast<uint32_t>(nrow) * kHotTokenBytes;
-        mbar_arrive_expect_tx(&sm.full[st], bytes);
-        bulk_g2s(dst, src, bytes, &sm.full[st], pol);
-        return;
-      }
-      const uint8_t *src = a.cold + ((((size_t)phys * a.hkv + h) << lsub) + u) * kTilePairBytes;
-      if (i0 + kb >= n_int4_b) {
-        if constexpr (St == kBlock) {
-          mbar_arrive_expect_tx(&sm.full[st], kTilePairBytes);
-          bulk_g2s(dst, src, kTilePairBytes, &sm.full[st], pol);
-        } else {
-          // a 32-token block: the K rows it holds, and its V tile (whose
-          // rows interleave its slots with the unused ones)
-          mbar_arrive_expect_tx(&sm.full[st], St * kDim + kTileBytes);
-          bulk_g2s(dst, src, St * kDim, &sm.full[st], pol);
-          bulk_g2s(dst + kTileBytes, src + kTileBytes, kTileBytes, &sm.full[st], pol);
-        }
-      } else {
-        mbar_arrive_expect_tx(&sm.full[st], St * kDim / 2 + kTileBytes / 2);
-        bulk_g2s(dst, src, St * kDim / 2, &sm.full[st], pol);
-        bulk_g2s(dst + kTileBytes, src + kTileBytes, kTileBytes / 2, &sm.full[st], pol);
-      }
-    } else {
-      // hot item j: ring slots 32j .. min(32j + 32, nhot) - 1
-      const int j = k - kh;
-      const uint8_t *src = a.hot + (((size_t)b * a.hkv + h) * H + j * kItemRows) * kHotTokenBytes;
-      const uint32_t bytes = static_cast<uint32_t>(min(kItemRows, nhot - j * kItemRows)) * kHotTokenBytes;
-      mbar_arrive_expect_tx(&sm.full[st], bytes);
-      bulk_g2s(dst, src, bytes, &sm.full[st], pol);
-    }
-  };
-  // block scales: requested before the bulk copies so that they do not queue
-  // behind them; stored once they arrive (overlapping the copies)
-  float2 sc_ld = make_float2(0.f, 0.f);
-  if (!fp16 && tid < ncold && sm.phys[tid] >= 0)
-    sc_ld = __ldg(reinterpret_cast<const float2 *>(a.scales + ((size_t)sm.phys[tid] * a.hkv + h) * 2));
-  int issued = 0;
-  if (tid == 0) {
-    issued = min(nitems, kStages);
-    for (int k = 0; k < issued; k++) issue(k);
-  }
-  if (tid < ncold) sm.scl[tid] = sc_ld;
-  // q in 16-bit fixed point per head (padding heads stay zero)
-  quantize_q<P>(sm.qf, sm.qi, sm.sq, warp, lane);
-  __syncthreads();
-
-  const int tg = lane >> 3, cs = lane & 7;
-  const int hx = head_xor<P>(lane);   // this lane's value k is head k ^ hx; its final head is hx
-  const bool owner = (lane & (8 / P - 1)) == 0 && hx < G;
-  const float sq_hd = sm.sq[hx];
-  // full-block path: the lane's K row (tokens 16w + 4tg + step) and V words
-  const int k_lane = (16 * warp + 4 * tg) * kDim + 16 * cs;
-  const int v_lane = kTileBytes + lane * kBlock + 16 * (warp ^ ((lane >> 1) & 3));
-
-  uint32_t qp[P][8];  // q pairs of this lane's 16 channels, in the lane's head order
-  load_qp<P>(sm.qi, hx, cs, qp);
-
-  // Online-softmax state of this warp.  m_run: running max per head (the
-  // same in every lane); acc: unnormalised output of the lane's channels;
-  // weights are taken relative to m_run, so the denominator can be summed
-  // per lane (head hx, its own tokens) and reduced across lanes only at the
-  // end: l_lane (FP32) plus psum_lane (integer sum of 16-bit weight codes).
-  float m_run[G], acc[G][4];
-#pragma unroll
-  for (int hh = 0; hh < G; hh++) {
-    m_run[hh] = -INFINITY;
-#pragma unroll
-    for (int kk = 0; kk < 4; kk++) acc[hh][kk] = 0.f;
-  }
-  float m_hx = hx < G ? -INFINITY : INFINITY;  // m_run of this lane's head (+inf: padding head)
-  float l_lane = 0.f;
-  int psum_lane = 0;
-
-  bool aborted = false;
-  int next_issue = issued;  // thread 0: next item to bring in
-  for (int k = 0; k < nitems; k++) {
-    const int st = k % kStages;
-    // thread 0 refills stages the warps have released: item k must be in
-    // flight before anyone waits for it, later ones only if already free
-    if (tid == 0) {
-      for (; next_issue < min(nitems, k + kStages); next_issue++) {
-        const int j = next_issue - kStages;  // previous item of that stage
-        if (next_issue <= k) {
-          if (!mbar_wait_bounded(&sm.empty[j % kStages], (j / kStages) & 1, kWaitCycles)) {
-            set_status(a.status, HYB_STATUS_TIMEOUT);
-            sm.abort_flag = 1;
-            break;
-          }
-        } else if (!mbar_try_wait(&sm.empty[j % kStages], (j / kStages) & 1)) {
-          break;
-        }
-        issue(next_issue);
-      }
-      issued = next_issue;
-    }
-    bool ok = mbar_wait_bounded(&sm.full[st], (k / kStages) & 1, kWaitCycles);
-    if (!ok && lane == 0) set_status(a.status, HYB_STATUS_TIMEOUT);
-    if (k == k_seal || k == k_rq || (do_ring && k == k_ring)) {
-      // ---------------- fused append (whole CTA, in the staged copies) ----------------
-      ok = __syncthreads_and(ok) != 0;
-      const int tb = ncold - 1;  // the tail block
-      if (ok && k == k_seal) {
-        if (fp16)
-          fused_seal_fp16(sm.seal, sm.ring[st], sm.phys[tb] * a.hkv + h, a, L_old, true, tid);
-        else
-          fused_seal(sm.seal, sm.ring[st], &sm.scl[tb], sm.phys[tb] * a.hkv + h, (i0 + tb) < n_int4_b, a, L_old,
-                     true, tid, warp, lane);
-      } else if (ok && k == k_rq) {
-        if (sm.phys[tb] >= 0)
-          requant_staged(sm.seal, sm.ring[st], (sm.phys[tb] * a.hkv + h) << lsub, (i0 + tb) < n_int4_b, a, tid);
-      } else if (ok) {
-        ring_put(sm.ring[st], rs, new_kv, a, b, h, tid);
-      }
-    }
-    ok = ok && *reinterpret_cast<volatile int *>(&sm.abort_flag) == 0;
-    const uint8_t *stage = sm.ring[st];
-    // rows of an FP16 item: the hot ring, or half of an FP16 cold block
-    int nrow = min(kItemRows, nhot - (k - kh) * kItemRows);
-    if (k < ncold_it)
-      nrow = !fp16 || sm.phys[item_block(k)] < 0
-                 ? 0
-                 : min(kItemRows, Lc - (i0 + item_block(k)) * Bt - (k & ((1 << ish) - 1)) * kItemRows);
-    if (ok && !fp16 && k < ncold_it) {
-      // ---------------- cold sub-block (64 tokens) ----------------
-      const int kb = item_block(k);
-      const int i = i0 + kb;
-      const int nvalid = sm.phys[kb] < 0 ? 0 : min(St, Lc - i * Bt - item_sub(k) * kBlock);
-      const int nv = nvalid - 16 * warp;
-      const bool int4 = i < n_int4_b;
-      const float2 sc = sm.scl[kb];
-      const float coef = sq_hd * sc.x * a.qk_scale;
-      if (nvalid == kBlock && !int4) {
-        cold_block_full<G, P>(stage, k_lane, v_lane, qp, coef, sc.y * (1.f / 32767.f), sm.pcode[warp], hx, tg,
-                              owner, m_run, acc, m_hx, l_lane, psum_lane);
-      } else if (nv > 0) {
-        cold_block_general<G, P>(stage, nv, int4, warp, lane, tg, cs, qp, coef, sc.y * (1.f / 32767.f),
-                                 sm.pcode[warp], hx, owner, m_run, acc, m_hx, l_lane, psum_lane);
-      }
-    } else if (ok && nrow > 0) {
-      // ---------------- FP16 rows (FP32 math): hot ring or FP16 cold half block ----------------
-      hot_item<G, P>(stage, nrow, warp, lane, tg, cs, sm.qf, a.qk_scale, sm.phot[warp], hx, owner, m_run, acc, m_hx,
-                     l_lane, psum_lane);
-    }
-    __syncwarp();
-    if (!ok) {
-      sm.abort_flag = 1;
-      aborted = true;
-      break;
-    }
-    if (lane == 0) mbar_arrive(&sm.empty[st]);
-  }
-  aborted = __syncthreads_or(aborted) != 0;
-  // this split's normalised output (channel tid) and log2-sum-exp per head
-  float o_s[G], lse2_s[G];
-  if (aborted) {
-    // let every copy still in flight land before the CTA's shared memory is
-    // released: the last item issued into each stage
-    if (tid == 0) {
-      for (int j = max(0, issued - kStages); j < issued; j++)
-        (void)mbar_wait_bounded(&sm.full[j % kStages], (j / kStages) & 1, kWaitCycles);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int hh = 0; hh < G; hh++) {
-      o_s[hh] = 0.f;
-      lse2_s[hh] = -INFINITY;
-    }
-  } else {
-    merge_warps<G, P>(reinterpret_cast<float *>(&sm.ring[0][0]), sm.mrun, sm.lrun, m_run, acc, l_lane, psum_lane,
-                      warp, lane, tid, o_s, lse2_s);
-  }
-  if constexpr (kCluster) {
-    // ---------------- split merge across the cluster (distributed shared memory) ----------------
-    float *cl_o = reinterpret_cast<float *>(&sm.ring[0][0]);  // [G][kDim], this split's output
-#pragma unroll
-    for (int hh = 0; hh < G; hh++) cl_o[hh * kDim + tid] = o_s[hh];
-    if (tid == 0) {
-#pragma unroll
-      for (int hh = 0; hh < G; hh++) sm.cl_l[hh] = lse2_s[hh];
-    }
-    cluster_sync_all();
-    // CTA s of the cluster merges output elements [s*per, (s+1)*per)
-    const int per = (G * kDim + S - 1) / S;
-    for (int e = s * per + tid; e < min((s + 1) * per, G * kDim); e += kThreads) {
-      const int hh = e / kDim, c = e - hh * kDim;
-      float lj[16];
-      float m = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < 16; j++) {
-        lj[j] = j < S ? ld_cluster_f32(&sm.cl_l[hh], j) : -INFINITY;
-        m = fmaxf(m, lj[j]);
-      }
-      float num = 0.f, den = 0.f;
-      if (m != -INFINITY) {
-#pragma unroll
-        for (int j = 0; j < 16; j++) {
-          if (j < S) {
-            const float wgt = ex2(lj[j] - m);
-            num = fmaf(wgt, ld_cluster_f32(&cl_o[hh * kDim + c], j), num);
-            den += wgt;
-          }
-        }
-      }
-      const size_t row = (size_t)b * a.hq + hq0 + hh;
-      a.out[row * kDim + c] = __float2half_rn(den > 0.f ? num / den : 0.f);
-      if (c == 0 && a.lse_out) a.lse_out[row] = den > 0.f ? (m + log2f(den)) * kLn2 : -INFINITY;
-    }
-    cluster_sync_all();  // no CTA leaves while its shared memory may still be read
-    return;
-  }
-  if (Sb == 1) {
-#pragma unroll
-    for (int hh = 0; hh < G; hh++) {
-      const size_t row = (size_t)b * a.hq + hq0 + hh;
-      a.out[row * kDim + tid] = __float2half_rn(o_s[hh]);
-      if (tid == 0 && a.lse_out) a.lse_out[row] = lse2_s[hh] * kLn2;
-    }
-    return;
-  }
-  // ---------------- split merge in global memory ----------------
-  // The last CTA of (sequence, kv head) to finish merges the splits; with
-  // more than kMergeFan splits, the last CTA of each group of kMergeFan
-  // splits merges the group first and the last group merges the groups.
-  const size_t row0 = (size_t)b * a.hq + hq0;
-#pragma unroll
-  for (int hh = 0; hh < G; hh++) {
-    a.o_part[((row0 + hh) * S + s) * kDim + tid] = o_s[hh];
-    if (tid == 0) a.lse_part[(row0 + hh) * S + s] = lse2_s[hh];
-  }
-  const int unit = b * a.hkv + h;
-  const bool grouped = Sb > kMergeFan;
-  const int grp = s / kMergeFan;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    int32_t *cnt = grouped ? &a.g_counters[(size_t)unit * a.n_groups + grp] : &a.counters[unit];
-    const int need = grouped ? min(kMergeFan, Sb - grp * kMergeFan) : Sb;
-    const int last = atomicAdd(cnt, 1) == need - 1;
-    if (last) *cnt = 0;  // ready for the next call
-    sm.last = last;
-  }
-  __syncthreads();
-  if (!sm.last) return;
-  __threadfence();
-  if (!grouped) {
-    merge_splits<G>(a.o_part + row0 * S * kDim, kDim, (size_t)S * kDim, a.lse_part + row0 * S, 1, S, Sb,
-                    [](int j) { return j; }, warp, lane, a.out + row0 * kDim, a.lse_out ? a.lse_out + row0 : nullptr,
-                    nullptr, 0, nullptr, 0);
-    return;
-  }
-  const int NG = a.n_groups;
-  const int j0 = grp * kMergeFan;
-  merge_splits<G>(a.o_part + (row0 * S + j0) * kDim, kDim, (size_t)S * kDim, a.lse_part + row0 * S + j0, 1, S,
-                  min(kMergeFan, Sb - j0), [](int j) { return j; }, warp, lane, nullptr, nullptr,
-                  a.g_part + (row0 * NG + grp) * kDim, (size_t)NG * kDim, a.g_lse + row0 * NG + grp, NG);
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const int ngb = (Sb + kMergeFan - 1) / kMergeFan;
-    const int last = atomicAdd(&a.counters[unit], 1) == ngb - 1;
-    if (last) a.counters[unit] = 0;
-    sm.last = last;
-  }
-  __syncthreads();
-  if (!sm.last) return;
-  __threadfence();
-  merge_splits<G>(a.g_part + row0 * NG * kDim, kDim, (size_t)NG * kDim, a.g_lse + row0 * NG, 1, NG,
-                  (Sb + kMergeFan - 1) / kMergeFan, [](int j) { return j; }, warp, lane, a.out + row0 * kDim,
-                  a.lse_out ? a.lse_out + row0 : nullptr, nullptr, 0, nullptr, 0);
-}
-
-// Largest cluster the decode kernel is launched with (portable size).
-constexpr int kMaxCluster = 8;
-
-template <int G, bool kF16, bool kSkip, int kBshift>
-static cudaError_t launch_decode_g(const DecodeArgs &a, int batch, bool cluster, cudaStream_t stream) {
-  const size_t smem = sizeof(DecodeSmem<G>);
-  static int configured_dev_mask = 0;  // one bit per device (per instantiation)
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 31 && !(configured_dev_mask & (1 << dev))) {
-    e = cudaFuncSetAttribute(decode_kernel<G, false, kF16, kSkip, kBshift>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(decode_kernel<G, true, kF16, kSkip, kBshift>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    configured_dev_mask |= 1 << dev;
-  }
-  dim3 grid(a.n_splits, a.hkv, batch);
-  if (cluster && a.n_splits >= 2 && a.n_splits <= kMaxCluster) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = a.n_splits;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_kernel<G, true, kF16, kSkip, kBshift>, a);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
-  }
-  decode_kernel<G, false, kF16, kSkip, kBshift><<<grid, kThreads, smem, stream>>>(a);
-  return cudaGetLastError();
-}
+constexpr int kMaxSplitBlocksD = 128;  // == the kernel's threads: one block-table entry per thread
+constexpr int kMaxClusterD = 8;        // largest cluster the kernel is launched with (portable size)
 
 template <bool kF16, bool kSkip, int kBshift>
-static cudaError_t launch_decode_f(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream) {
-  switch (group) {
-    case 1: return launch_decode_g<1, kF16, kSkip, kBshift>(a, batch, cluster, stream);
-    case 2: return launch_decode_g<2, kF16, kSkip, kBshift>(a, batch, cluster, stream);
-    case 3: return launch_decode_g<3, kF16, kSkip, kBshift>(a, batch, cluster, stream);
-    case 4: return launch_decode_g<4, kF16, kSkip, kBshift>(a, batch, cluster, stream);
-    case 5: return launch_decode_g<5, kF16, kSkip, kBshift>(a, batch, cluster, stream);
-    case 6: return launch_decode_g<6, kF16, kSkip, kBshift>(a, batch, cluster, stream);
-    case 7: return launch_decode_g<7, kF16, kSkip, kBshift>(a, batch, cluster, stream);
-    case 8: return launch_decode_g<8, kF16, kSkip, kBshift>(a, batch, cluster, stream);
-    default: return cudaErrorInvalidValue;
-  }
-}
+cudaError_t launch_decode_f(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream);
+template <bool kF16, bool kSkip, int kBshift>
+int decode_occupancy(int group);
 
 template <int kBshift>
 static cudaError_t launch_decode_l(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream) {
@@ -566,12 +29,12 @@ cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, bool cluste
   }
 }
 
-int decode_max_cluster() { return kMaxCluster; }
+int decode_max_cluster() { return kMaxClusterD; }
 
-int decode_max_split_blocks() { return kMaxSplitBlocks; }
+int decode_max_split_blocks() { return kMaxSplitBlocksD; }
 
 // CTAs of the decode kernel one SM holds at once for this head group (0 if
-// the device cannot be queried).
+// the device cannot be queried); cached per device.
 int decode_ctas_per_sm(int group) {
   static int cached[32][9];  // [device][group], 0 = not yet known
   int dev = 0;
@@ -579,28 +42,9 @@ int decode_ctas_per_sm(int group) {
     cudaGetLastError();
     return 0;
   }
-  if (dev >= 0 && dev < 32 && group >= 1 && group <= 8 && cached[dev][group] > 0)
-    return cached[dev][group];
-  int n = 0;
-  cudaError_t e = cudaErrorInvalidValue;
-  switch (group) {
-#define HYB_OCC(g)                                                                          \
-  case g:                                                                                   \
-    e = cudaFuncSetAttribute(decode_kernel<g, false, false, false, 6>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             static_cast<int>(sizeof(DecodeSmem<g>)));                      \
-    if (e == cudaSuccess)                                                                   \
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<g, false, false, false, 6>, kThreads, \
-                                                        sizeof(DecodeSmem<g>));             \
-    break;
-    HYB_OCC(1) HYB_OCC(2) HYB_OCC(3) HYB_OCC(4) HYB_OCC(5) HYB_OCC(6) HYB_OCC(7) HYB_OCC(8)
-#undef HYB_OCC
-    default: break;
-  }
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return 0;
-  }
-  if (dev >= 0 && dev < 32 && group >= 1 && group <= 8) cached[dev][group] = n;
+  if (dev >= 0 && dev < 32 && group >= 1 && group <= 8 && cached[dev][group] > 0) return cached[dev][group];
+  const int n = decode_occupancy<false, false, 6>(group);
+  if (n > 0 && dev >= 0 && dev < 32 && group >= 1 && group <= 8) cached[dev][group] = n;
   return n;
 }
 

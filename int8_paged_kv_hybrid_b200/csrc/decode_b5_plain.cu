@@ -1,0 +1,8 @@
+// decode_b5_plain.cu -- instantiation of the decode kernel for 32-token
+// blocks, dense variant (one translation unit per block size and variant so that
+// the build compiles them in parallel).
+#include "decode_kernel.cuh"
+
+namespace hyb {
+template cudaError_t launch_decode_f<false, false, 5>(const DecodeArgs &, int, int, bool, cudaStream_t);
+}  // namespace hyb

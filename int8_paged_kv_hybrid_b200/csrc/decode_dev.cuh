@@ -1,25 +1,41 @@
 // decode_dev.cuh -- device building blocks of the decode kernel
-// (decode.cu): the per-item arithmetic on a staged cold block or hot ring, the fused
-// append of the decode step, the merge of the four warps' softmax states and
-// the log-sum-exp merge of partial results.  The arithmetic is described at
-// the top of decode.cu.
+// (decode.cu): the per-item arithmetic on a staged cold block or FP16 rows
+// (tensor-core mma.sync), the fused append of the decode step, the merge of
+// the four warps' softmax states and the log-sum-exp merge of partial
+// results.  The arithmetic is described at the top of decode.cu.
 #pragma once
 
 #include <cfloat>
 
 #include "kernels.cuh"
+#include "mma.cuh"
 
 namespace hyb {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kStages = 3;
-constexpr long long kWaitCycles = 1ll << 31;  // ~1 s at B200 clocks
+constexpr long long kWaitCycles = kDefaultWaitCycles;  // drain waits (never shortened)
 constexpr float kLn2 = 0.69314718055994531f;
+// FP16 rows (hot ring, FP16 cold blocks) are staged one 512-byte row per bulk
+// copy at this pitch, so that the 8 rows an ldmatrix reads start 16 bytes
+// apart modulo 128 (distinct banks).
+constexpr int kRowStride = kHotTokenBytes + 16;
+constexpr int kStageBytes = kItemRows * kRowStride;  // >= kTilePairBytes
+static_assert(kStageBytes >= kTilePairBytes, "a stage holds a K + V tile pair");
+// Merge buffer pitch (floats per head row): 136 puts the 32 lanes' stores of
+// merge_warps in distinct banks.
+constexpr int kMbufPitch = kDim + 8;
+// q as a 24-bit fixed-point integer per head: |q_int| <= 127 * 65536, three
+// signed base-256 digits (hi, mid, lo), each in [-128, 127].
+constexpr float kQFix = 8323072.f;  // 127 * 65536
+// softmax weights in 16-bit fixed point relative to their group's maximum
+constexpr float kPFix = 65535.f;
 
+// Query-head slots per kv head: one quad of 4 (G <= 4) or two (G <= 8).
 template <int G>
-__host__ __device__ constexpr int pow2_heads() {
-  return G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : 8));
+__host__ __device__ constexpr int head_quads() {
+  return G <= 4 ? 1 : 2;
 }
 
 // 2^x on the SFU (max relative error ~2^-22); 2^-inf = +0.
@@ -27,35 +43,6 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// Sum P per-lane values over the 8 lanes of a lane octet.  Lane l holds its
-// values in the order head = k ^ x(l) (see head_xor); at each level a lane
-// keeps its lower half and adds the partner's upper half, which (because the
-// partner's order differs in exactly that bit) holds the same heads.  On
-// return v[0] is the octet total for head x(l).
-template <int P, typename T>
-__device__ __forceinline__ void transpose_reduce(T (&v)[P]) {
-  int c = P;
-#pragma unroll
-  for (int m = 4; m >= 1; m >>= 1) {
-    if (c > 1) {
-#pragma unroll
-      for (int k = 0; k < c / 2; k++) v[k] += __shfl_xor_sync(0xffffffffu, v[k + c / 2], m);
-      c /= 2;
-    } else {
-      v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
-    }
-  }
-}
-
-// Head order of a lane: value k of the lane is head k ^ head_xor(lane).
-template <int P>
-__device__ __forceinline__ int head_xor(int lane) {
-  if constexpr (P == 8) return lane & 7;
-  if constexpr (P == 4) return (lane >> 1) & 3;
-  if constexpr (P == 2) return (lane >> 2) & 1;
-  return 0;
 }
 
 // Barrier over all threads of all CTAs of the cluster (release / acquire).
@@ -201,26 +188,28 @@ __device__ __forceinline__ void fused_seal(SealScratch &ss, uint8_t *tile_st, fl
       }
     }
   }
+  fence_proxy_async_smem();  // the staged tile is refilled by bulk copies later
   __syncthreads();
 }
 
 // Fused decode step, seal half for FP16 cold blocks (quantization_bits 0):
 // the evicted token's rows (ss.erow) move unchanged to slot e % 64 of the
-// tail block -- in its staged half-block item (row_st, rows slot % 32) and in
-// the cache.  Thread tid moves channel tid of both rows.
+// tail block -- in its staged half-block item (row_st, rows slot % 32 at the
+// staging pitch kRowStride) and in the cache.  Thread tid moves channel tid of both rows.
 __device__ __forceinline__ void fused_seal_fp16(const SealScratch &ss, uint8_t *row_st, int tile_tail,
                                                 const DecodeArgs &a, int L_old, bool do_seal, int tid) {
   if (!do_seal || tile_tail < 0) return;
   const int slot = (L_old - a.hot_tokens) & ((1 << a.bshift) - 1);
   const int c = tid;
   const __half k_old = ss.erow[c], v_old = ss.erow[kDim + c];
-  __half *trow = reinterpret_cast<__half *>(row_st + (slot % kItemRows) * kHotTokenBytes);
+  __half *trow = reinterpret_cast<__half *>(row_st + (slot % kItemRows) * kRowStride);
   trow[c] = k_old;
   trow[kDim + c] = v_old;
   __half *grow = reinterpret_cast<__half *>(a.cold + ((size_t)tile_tail << a.bshift) * kHotTokenBytes +
                                             slot * kHotTokenBytes);
   grow[c] = k_old;
   grow[kDim + c] = v_old;
+  fence_proxy_async_smem();
   __syncthreads();
 }
 
@@ -247,51 +236,24 @@ __device__ __forceinline__ void requant_staged(const SealScratch &ss, uint8_t *t
     for (int v = tid; v < nvec; v += kThreads)
       reinterpret_cast<uint4 *>(g + kv * kTileBytes)[v] = reinterpret_cast<const uint4 *>(tile_st + kv * kTileBytes)[v];
   }
+  fence_proxy_async_smem();
   __syncthreads();
 }
 
 // Fused decode step, ring half: the new token goes to ring slot rs = L_old %
-// hot -- row rs % 32 of its staged hot item (item_st, for this attention) and
-// the cache.  Thread tid writes channel tid of both rows.
+// hot -- row rs % 32 of its staged hot item (item_st, pitch kRowStride, for
+// this attention) and the cache.  Thread tid writes channel tid of both rows.
 __device__ __forceinline__ void ring_put(uint8_t *item_st, int rs, __half2 new_kv, const DecodeArgs &a, int b,
                                          int h, int tid) {
   const int c = tid;
-  __half *srow = reinterpret_cast<__half *>(item_st + (rs % kItemRows) * kHotTokenBytes);
+  __half *srow = reinterpret_cast<__half *>(item_st + (rs % kItemRows) * kRowStride);
   srow[c] = __low2half(new_kv);
   srow[kDim + c] = __high2half(new_kv);
   __half *grow = reinterpret_cast<__half *>(a.hot) + ((((size_t)b * a.hkv + h) * a.hot_tokens + rs) * 2) * kDim;
   grow[c] = __low2half(new_kv);
   grow[kDim + c] = __high2half(new_kv);
+  fence_proxy_async_smem();
   __syncthreads();
-}
-
-// Raise a warp's running max to cover an item's logits, whose maximum over a
-// lane's tokens is zmax (lane's head hx): m_run per head, the accumulators
-// and the lane's denominator (l_lane + psum_lane / 32767) are rescaled.
-// Warp-uniform call; rare once the first blocks are seen.
-template <int G, int P>
-__device__ __forceinline__ void raise_max(float zmax, float (&m_run)[G], float (&acc)[G][4], float &m_hx,
-                                          float &l_lane, int &psum_lane, int hx) {
-  float mb = zmax;
-  mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 8));
-  mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 16));
-  float alpha_hx = 1.f;
-#pragma unroll
-  for (int hh = 0; hh < G; hh++) {
-    const float mbh = __shfl_sync(0xffffffffu, mb, hh * (8 / P));  // a lane holding head hh
-    if (mbh > m_run[hh]) {
-      const float alpha = ex2(m_run[hh] - mbh);
-#pragma unroll
-      for (int kk = 0; kk < 4; kk++) acc[hh][kk] *= alpha;
-      if (hh == hx) alpha_hx = alpha;
-      m_run[hh] = mbh;
-    }
-    if (hh == hx) m_hx = m_run[hh];
-  }
-  if (alpha_hx != 1.f) {
-    l_lane = (l_lane + static_cast<float>(psum_lane) * (1.f / 32767.f)) * alpha_hx;
-    psum_lane = 0;
-  }
 }
 
 // Log-sum-exp merge of n partial results of the G query heads of one kv head
@@ -362,315 +324,351 @@ __device__ __forceinline__ void merge_splits(const float *o, size_t o_js, size_t
   }
 }
 
-// q of one kv head's G query heads in 16-bit fixed point per head: warp w
-// quantizes heads w, w + 4, ... of qf (FP32 [P][128], rows >= G zero) into qi
-// and the step max|q| / 32767 into sq.  Callers synchronise around it.
-template <int P>
-__device__ __forceinline__ void quantize_q(const float (*qf)[kDim], int16_t (*qi)[kDim], float *sq, int warp,
-                                           int lane) {
-  for (int j = warp; j < P; j += kWarps) {
-    float amax = 0.f;
-    for (int c = lane; c < kDim; c += 32) amax = fmaxf(amax, fabsf(qf[j][c]));
+
+// ---------------------------------------------------------------------------
+// Per-item arithmetic on the tensor cores (mma.sync).  A lane is (g, t) =
+// (lane / 4, lane % 4).  Two layouts meet here:
+//  * score layout -- the C fragment of the QK product: lane (g, t) holds the
+//    logits of head 4 * nt + g / 2 (head quad nt) for its tokens;
+//  * value layout -- the C fragment of the P.V product: lane (g, t) holds the
+//    output of head 4 * nt + t for channels 16 * mt + g and 16 * mt + g + 8
+//    (mt = 0..7); a warp's online-softmax state lives in this layout.
+// ---------------------------------------------------------------------------
+
+// Online-softmax state of one warp (value layout).
+template <int NT>
+struct WarpState {
+  float acc[NT][8][2];  // unnormalised output, head 4nt + t, channels 16mt + g (+ 8)
+  float m_run[NT];      // running maximum logit (log2 domain) of head 4nt + t
+  float l_run[NT];      // sum of the weights relative to m_run
+};
+
+template <int NT>
+__device__ __forceinline__ void state_init(WarpState<NT> &st) {
 #pragma unroll
-    for (int m = 16; m > 0; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
-    const float inv = amax > 0.f ? 32767.f / amax : 0.f;
-    for (int c = lane; c < kDim; c += 32) {
-      const int v = __float2int_rn(qf[j][c] * inv);
-      qi[j][c] = static_cast<int16_t>(max(-32767, min(32767, v)));
-    }
-    if (lane == 0) sq[j] = amax > 0.f ? amax / 32767.f : 0.f;
+  for (int nt = 0; nt < NT; nt++) {
+    st.m_run[nt] = -INFINITY;
+    st.l_run[nt] = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < 8; mt++) st.acc[nt][mt][0] = st.acc[nt][mt][1] = 0.f;
   }
 }
 
-// The lane's q pairs: its 16 channels (16cs..16cs+15) of every head, in the
-// lane's head order (value k is head k ^ hx).
-template <int P>
-__device__ __forceinline__ void load_qp(const int16_t (*qi)[kDim], int hx, int cs, uint32_t (&qp)[P][8]) {
+// A group of tokens (its maximum logit mx, its weights' sum S relative to mx)
+// joins the state of one head: the running maximum is raised to cover mx
+// (rescaling what was accumulated), the sum grows by 2^(mx - m_run) * S, and
+// the factor 2^(mx - m_run) that the group's P.V result takes is returned.
+// An empty group (mx = -inf) changes nothing and gets factor 0.
+__device__ __forceinline__ float group_update(float mx, float S, float &m_run, float &l_run, float (&acc)[8][2]) {
+  if (mx > m_run) {
+    const float alpha = ex2(m_run - mx);  // 0 for the first group
 #pragma unroll
-  for (int k = 0; k < P; k++) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(&qi[k ^ hx][16 * cs]);
-    const uint4 x0 = src[0], x1 = src[1];
-    qp[k][0] = x0.x; qp[k][1] = x0.y; qp[k][2] = x0.z; qp[k][3] = x0.w;
-    qp[k][4] = x1.x; qp[k][5] = x1.y; qp[k][6] = x1.z; qp[k][7] = x1.w;
+    for (int mt = 0; mt < 8; mt++) {
+      acc[mt][0] *= alpha;
+      acc[mt][1] *= alpha;
+    }
+    l_run *= alpha;
+    m_run = mx;
+  }
+  const float e = mx == -INFINITY ? 0.f : ex2(mx - m_run);
+  l_run = fmaf(e, S, l_run);
+  return e;
+}
+
+// q of one kv head's query heads, prepared once per CTA: every thread holds
+// channel tid of each head (qv, FP32 from FP16).  Writes the head's 24-bit
+// fixed-point digits qd[h][0..2][c] (hi, mid, lo), its FP16 copy qh[h][c] and
+// the fixed-point step sq[h] = max|q_h| / kQFix; heads >= G are zero.
+// qmax_w [kWarps][NH] is scratch.  Two CTA barriers.
+template <int G, int NH>
+__device__ __forceinline__ void prepare_q(const float (&qv)[G], int8_t (*qd)[3][kDim], __half (*qh)[kDim],
+                                          float *sq, float (*qmax_w)[NH], int warp, int lane, int tid) {
+#pragma unroll
+  for (int j = 0; j < G; j++) {
+    float m = fabsf(qv[j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) qmax_w[warp][j] = m;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < NH; j++) {
+    int8_t d0 = 0, d1 = 0, d2 = 0;
+    __half hv = __float2half_rn(0.f);
+    if (j < G) {
+      const float M = fmaxf(fmaxf(qmax_w[0][j], qmax_w[1][j]), fmaxf(qmax_w[2][j], qmax_w[3][j]));
+      const float inv = M > 0.f ? kQFix / M : 0.f;
+      int qi = __float2int_rn(qv[j] * inv);
+      qi = max(-8323072, min(8323072, qi));
+      const int lo = ((qi + 128) & 255) - 128;
+      const int r = (qi - lo) >> 8;
+      const int mid = ((r + 128) & 255) - 128;
+      const int hi = (r - mid) >> 8;
+      d0 = static_cast<int8_t>(hi);
+      d1 = static_cast<int8_t>(mid);
+      d2 = static_cast<int8_t>(lo);
+      hv = __float2half_rn(qv[j]);
+      if (tid == 0) sq[j] = M / kQFix;
+    } else if (tid == 0) {
+      sq[j] = 0.f;
+    }
+    qd[j][0][tid] = d0;
+    qd[j][1][tid] = d1;
+    qd[j][2][tid] = d2;
+    qh[j][tid] = hv;
+  }
+  __syncthreads();
+}
+
+// The QK A fragments of this lane (score layout).  Rows of the 16 x 32 A
+// operand per head quad nt: row 2i = hi digits of head 4nt + i, row 2i + 8 =
+// its mid digits, row 2i + 1 = its lo digits, row 2i + 9 = 0.  The k index of
+// k-step ks maps to channel d as k = 4t' + i -> d = 32t' + 8ks + i and
+// k = 16 + 4t' + i -> d = 32t' + 8ks + 4 + i, so lane (g, t) needs channels
+// 32t .. 32t + 31 only (the K loads below follow the same map).
+template <int NT>
+__device__ __forceinline__ void load_qfrag(const int8_t (*qd)[3][kDim], int g, int t, uint32_t (&qa)[NT][4][4]) {
+  const bool even = (g & 1) == 0;
+#pragma unroll
+  for (int nt = 0; nt < NT; nt++) {
+    const int h = 4 * nt + (g >> 1);
+    const int8_t *dig = qd[h][even ? 0 : 2];
+    const int8_t *mid = qd[h][1];
+#pragma unroll
+    for (int ks = 0; ks < 4; ks++) {
+      const int c = 32 * t + 8 * ks;
+      qa[nt][ks][0] = *reinterpret_cast<const uint32_t *>(dig + c);
+      qa[nt][ks][2] = *reinterpret_cast<const uint32_t *>(dig + c + 4);
+      qa[nt][ks][1] = even ? *reinterpret_cast<const uint32_t *>(mid + c) : 0u;
+      qa[nt][ks][3] = even ? *reinterpret_cast<const uint32_t *>(mid + c + 4) : 0u;
+    }
   }
 }
 
-// One full INT8 cold block (all 64 tokens valid), for one warp.  The warp's
-// tokens are 16w..16w+15; lane (tg, cs) takes tokens 16w + 4tg + step, step
-// 0..3 (channels 16cs..16cs+15), so the four weight codes an owner lane
-// produces for its head are adjacent and leave in one 8-byte store.  k_lane
-// and v_lane are the lane's byte offsets of its K row (step 0) and of its V
-// words inside a stage; pc is this warp's weight-code rows.  Same arithmetic
-// as the general path; no masks, no INT4 branches, offsets fixed per lane.
-template <int G, int P>
-__device__ __forceinline__ void cold_block_full(const uint8_t *stage, int k_lane, int v_lane,
-                                                const uint32_t (&qp)[P][8], float coef, float cv,
-                                                uint16_t (*pc_rows)[16], int hx, int tg, bool owner,
-                                                float (&m_run)[G], float (&acc)[G][4], float &m_hx,
-                                                float &l_lane, int &psum_lane) {
-  float z[4];
+// One 64-token INT8 or INT4 sub-block staged at `stage` (K tile, then V tile
+// at +8 KB), for one warp: its 16 tokens 16w .. 16w + 15 (tokens >= nvalid
+// are masked when kMasked).
+//  QK: mma m16n8k32 s8 per (head quad, 8-token column tile j, k-step): the
+//      digits of q against the K codes, exact in int32; the lane pair (g,
+//      g ^ 1) joins hi/mid and lo into the logit.  Column n of tile j is
+//      token 16w + 4(n / 2) + 2j + n % 2, so lane (g, t) ends up with the
+//      logits of tokens 16w + 4t + u, u = 0..3, in C order.
+//  Softmax weights: p = rint(65535 * 2^(z - mx)), mx = the 16-token group's
+//      maximum for the head (16-bit fixed point relative to the group's own
+//      maximum), split into a high and a low byte.
+//  P.V: mma m16n8k16 s8 x u8 per (channel tile, head quad): A = V codes of 16
+//      channels x the warp's 16 tokens (ldmatrix on the channel-major tile),
+//      B columns 2i / 2i + 1 = the high / low bytes of head i's weights, so
+//      lane (g, t) gets head t's two partial sums per channel and joins them
+//      exactly (256 * hi + lo) before the FP32 fold with the V scale.
+// coef[nt]: K scale * q step of head 4nt + g/2 * softmax scale * log2(e);
+// sv: V scale; psel: prmt selector of the lane's weight byte (g odd: low);
+// v_lane: shared address of this lane's V row for the ldmatrix of channel
+// tile pair 0 (INT8).
+template <int NT, bool kInt4, bool kMasked>
+__device__ __forceinline__ void cold_item(const uint8_t *stage, int nvalid, int warp, int g, int t,
+                                          const uint32_t (&qa)[NT][4][4], const float (&coef)[NT], float sv,
+                                          uint32_t psel, uint32_t v_lane, WarpState<NT> &st) {
+  const bool even = (g & 1) == 0;
+  int c[NT][2][4];
 #pragma unroll
-  for (int step = 0; step < 4; step++) {
-    const uint4 v = *reinterpret_cast<const uint4 *>(stage + k_lane + step * kDim);
-    const uint32_t kw[4] = {v.x, v.y, v.z, v.w};
-    int dot[P];
+  for (int nt = 0; nt < NT; nt++)
 #pragma unroll
-    for (int kk = 0; kk < P; kk++) dot[kk] = 0;
+    for (int j = 0; j < 2; j++) c[nt][j][0] = c[nt][j][1] = c[nt][j][2] = c[nt][j][3] = 0;
 #pragma unroll
-    for (int j = 0; j < 4; j++) {
+  for (int j = 0; j < 2; j++) {
+    const int tok = 16 * warp + 4 * (g >> 1) + 2 * j + (g & 1);
+    uint32_t kw[8];
+    if constexpr (!kInt4) {
+      const uint4 x0 = *reinterpret_cast<const uint4 *>(stage + tok * kDim + 32 * t);
+      const uint4 x1 = *reinterpret_cast<const uint4 *>(stage + tok * kDim + 32 * t + 16);
+      kw[0] = x0.x; kw[1] = x0.y; kw[2] = x0.z; kw[3] = x0.w;
+      kw[4] = x1.x; kw[5] = x1.y; kw[6] = x1.z; kw[7] = x1.w;
+    } else {
+      // INT4 word ks of the lane's 16 bytes holds channels 32t + 8ks + 0..7:
+      // low nibbles 0..3, high nibbles 4..7 -- exactly the two B registers
+      const uint4 x = *reinterpret_cast<const uint4 *>(stage + tok * 64 + 16 * t);
+      const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-      for (int kk = 0; kk < P; kk++)
-        dot[kk] = __dp2a_lo(static_cast<int>(qp[kk][2 * j]), static_cast<int>(kw[j]), dot[kk]);
-#pragma unroll
-      for (int kk = 0; kk < P; kk++)
-        dot[kk] = __dp2a_hi(static_cast<int>(qp[kk][2 * j + 1]), static_cast<int>(kw[j]), dot[kk]);
+      for (int ks = 0; ks < 4; ks++) unpack_int4(w4[ks], kw[2 * ks], kw[2 * ks + 1]);
     }
-    transpose_reduce<P>(dot);
-    z[step] = static_cast<float>(dot[0]) * coef;
+#pragma unroll
+    for (int ks = 0; ks < 4; ks++)
+#pragma unroll
+      for (int nt = 0; nt < NT; nt++)
+        mma_s8s8_k32(c[nt][j], qa[nt][ks][0], qa[nt][ks][1], qa[nt][ks][2], qa[nt][ks][3], kw[2 * ks],
+                     kw[2 * ks + 1]);
   }
-  {
-    const float zmax = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
-    if (__any_sync(0xffffffffu, zmax > m_hx)) raise_max<G, P>(zmax, m_run, acc, m_hx, l_lane, psum_lane, hx);
+  const int m1 = even ? 256 : 1;
+  const float w_self = even ? 256.f : 1.f, w_other = even ? 1.f : 256.f;
+  uint32_t pb[NT];
+  float f[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; nt++) {
+    float z[4];
+#pragma unroll
+    for (int j = 0; j < 2; j++)
+#pragma unroll
+      for (int e = 0; e < 2; e++) {
+        const int x = c[nt][j][e] * m1 + c[nt][j][2 + e];  // even: 256 hi + mid; odd: lo
+        const int y = __shfl_xor_sync(0xffffffffu, x, 4);
+        const float zz = fmaf(static_cast<float>(x), w_self, static_cast<float>(y) * w_other) * coef[nt];
+        z[2 * j + e] = (kMasked && 16 * warp + 4 * t + 2 * j + e >= nvalid) ? -INFINITY : zz;
+      }
+    float mx = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float mref = mx == -INFINITY ? 0.f : mx;
+    uint32_t p[4];
+    int S = 0;
+#pragma unroll
+    for (int u = 0; u < 4; u++) {
+      // rint(65535 * 2^(z - mx)) by the 1.5 * 2^23 magic add (exact for [0, 2^22))
+      p[u] = __float_as_uint(fmaf(ex2(z[u] - mref), kPFix, 12582912.f)) - 0x4B400000u;
+      S += static_cast<int>(p[u]);
+    }
+    S += __shfl_xor_sync(0xffffffffu, S, 1);
+    S += __shfl_xor_sync(0xffffffffu, S, 2);
+    pb[nt] = prmt(prmt(p[0], p[1], 0x5410u), prmt(p[2], p[3], 0x5410u), psel);
+    // the group's statistics for head 4nt + t (from lane 8t, which has g = 2t)
+    const float mx_t = __shfl_sync(0xffffffffu, mx, 8 * t);
+    const int S_t = __shfl_sync(0xffffffffu, S, 8 * t);
+    const float e = group_update(mx_t, static_cast<float>(S_t) * (1.f / kPFix), st.m_run[nt], st.l_run[nt],
+                                 st.acc[nt]);
+    f[nt] = e * sv * (1.f / kPFix);
   }
-  uint32_t pc[4];
-#pragma unroll
-  for (int step = 0; step < 4; step++) {
-    const float pq = fmaf(ex2(z[step] - m_hx), 32767.f, 12582912.f);
-    pc[step] = __float_as_uint(pq) - 0x4B400000u;
-    psum_lane += static_cast<int>(pc[step]);
-  }
-  if (owner)
-    *reinterpret_cast<uint2 *>(&pc_rows[hx][4 * tg]) = make_uint2(pc[0] | (pc[1] << 16), pc[2] | (pc[3] << 16));
-  __syncwarp();
-  uint32_t vw[4][4];
-#pragma unroll
-  for (int kk = 0; kk < 4; kk++) {
-    const uint4 v = *reinterpret_cast<const uint4 *>(stage + v_lane + 32 * kBlock * kk);
-    vw[kk][0] = v.x; vw[kk][1] = v.y; vw[kk][2] = v.z; vw[kk][3] = v.w;
+  // V codes of channel tiles 2mp, 2mp + 1 and the P.V products
+  uint32_t v_off0 = 0, v_off1 = 0;
+  if constexpr (kInt4) {
+    // INT4 V: channel row c at 32c bytes, the 8-byte unit of tokens 16w..16w+15
+    // at (w ^ ((c / 4) % 4)) * 8, tokens 8i..8i+7 in its word i (low nibbles
+    // first); lane (g, t) needs channel 16mt + g (+ 8), tokens 16w + 4t + 0..3
+    v_off0 = kTileBytes + g * 32 + 8 * (warp ^ (g >> 2)) + 4 * (t >> 1);
+    v_off1 = kTileBytes + (g + 8) * 32 + 8 * (warp ^ (2 + (g >> 2))) + 4 * (t >> 1);
   }
 #pragma unroll
-  for (int hh = 0; hh < G; hh++) {
-    const uint4 pa = *reinterpret_cast<const uint4 *>(&pc_rows[hh][0]);
-    const uint4 pb = *reinterpret_cast<const uint4 *>(&pc_rows[hh][8]);
-    const uint32_t pp[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
-    int ai[4] = {0, 0, 0, 0};
+  for (int mp = 0; mp < 4; mp++) {
+    uint32_t va[4];
+    if constexpr (!kInt4) {
+      ldmatrix_x4(va, v_lane + mp * 32 * kBlock);
+    } else {
+      const int sh = 4 * (t & 1);
 #pragma unroll
-    for (int j = 0; j < 4; j++) {
-#pragma unroll
-      for (int kk = 0; kk < 4; kk++) {
-        ai[kk] = __dp2a_lo(static_cast<int>(pp[2 * j]), static_cast<int>(vw[kk][j]), ai[kk]);
-        ai[kk] = __dp2a_hi(static_cast<int>(pp[2 * j + 1]), static_cast<int>(vw[kk][j]), ai[kk]);
+      for (int h2 = 0; h2 < 2; h2++) {
+        const int mt = 2 * mp + h2;
+        const uint32_t x0 = *reinterpret_cast<const uint32_t *>(stage + v_off0 + mt * 16 * 32);
+        const uint32_t x1 = *reinterpret_cast<const uint32_t *>(stage + v_off1 + mt * 16 * 32);
+        va[2 * h2] = sext_nibbles((x0 >> sh) & 0x0f0f0f0fu);
+        va[2 * h2 + 1] = sext_nibbles((x1 >> sh) & 0x0f0f0f0fu);
       }
     }
 #pragma unroll
-    for (int kk = 0; kk < 4; kk++) acc[hh][kk] = fmaf(cv, static_cast<float>(ai[kk]), acc[hh][kk]);
-  }
-}
-
-// A cold block that is INT4 or not full (nv = valid tokens from this warp's
-// first one), for one warp: lane (tg, cs) takes tokens 16w + 4step + tg.
-// Same arithmetic as cold_block_full.
-template <int G, int P>
-__device__ __forceinline__ void cold_block_general(const uint8_t *stage, int nv, bool int4, int warp, int lane,
-                                                   int tg, int cs, const uint32_t (&qp)[P][8], float coef,
-                                                   float cv, uint16_t (*pc_rows)[16], int hx, bool owner,
-                                                   float (&m_run)[G], float (&acc)[G][4], float &m_hx,
-                                                   float &l_lane, int &psum_lane) {
-  float z[4];
+    for (int h2 = 0; h2 < 2; h2++) {
+      const int mt = 2 * mp + h2;
 #pragma unroll
-  for (int step = 0; step < 4; step++) {
-    const int t = 16 * warp + 4 * step + tg;
-    uint32_t kw[4];
-    if (!int4) {
-      const uint4 v = *reinterpret_cast<const uint4 *>(stage + t * kDim + 16 * cs);
-      kw[0] = v.x; kw[1] = v.y; kw[2] = v.z; kw[3] = v.w;
-    } else {
-      const uint2 v = *reinterpret_cast<const uint2 *>(stage + t * 64 + 8 * cs);
-      unpack_int4(v.x, kw[0], kw[1]);
-      unpack_int4(v.y, kw[2], kw[3]);
-    }
-    int dot[P];
-#pragma unroll
-    for (int kk = 0; kk < P; kk++) dot[kk] = 0;
-#pragma unroll
-    for (int j = 0; j < 4; j++) {
-#pragma unroll
-      for (int kk = 0; kk < P; kk++)
-        dot[kk] = __dp2a_lo(static_cast<int>(qp[kk][2 * j]), static_cast<int>(kw[j]), dot[kk]);
-#pragma unroll
-      for (int kk = 0; kk < P; kk++)
-        dot[kk] = __dp2a_hi(static_cast<int>(qp[kk][2 * j + 1]), static_cast<int>(kw[j]), dot[kk]);
-    }
-    transpose_reduce<P>(dot);
-    z[step] = (4 * step + tg < nv) ? static_cast<float>(dot[0]) * coef : -INFINITY;
-  }
-  // the running max must cover these logits (rare after the first blocks)
-  {
-    const float zmax = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
-    if (__any_sync(0xffffffffu, zmax > m_hx)) raise_max<G, P>(zmax, m_run, acc, m_hx, l_lane, psum_lane, hx);
-  }
-  // 16-bit weights relative to the running max: round(32767 * 2^(z - m))
-  // via the 1.5*2^23 magic add
-  uint32_t pc[4];
-#pragma unroll
-  for (int step = 0; step < 4; step++) {
-    const float pq = fmaf(ex2(z[step] - m_hx), 32767.f, 12582912.f);
-    pc[step] = __float_as_uint(pq) - 0x4B400000u;
-    psum_lane += static_cast<int>(pc[step]);
-  }
-  if (owner) {
-#pragma unroll
-    for (int step = 0; step < 4; step++)
-      pc_rows[hx][4 * step + tg] = static_cast<uint16_t>(pc[step]);
-  }
-  __syncwarp();
-  // P.V over this warp's 16 tokens; lane owns channels lane + 32*kk
-  uint32_t vw[4][4];
-#pragma unroll
-  for (int kk = 0; kk < 4; kk++) {
-    const int c = lane + 32 * kk;
-    if (!int4) {
-      const uint4 v = *reinterpret_cast<const uint4 *>(
-          stage + kTileBytes + c * 64 + 16 * (warp ^ ((c >> 1) & 3)));
-      vw[kk][0] = v.x; vw[kk][1] = v.y; vw[kk][2] = v.z; vw[kk][3] = v.w;
-    } else {
-      const uint2 v = *reinterpret_cast<const uint2 *>(
-          stage + kTileBytes + c * 32 + 8 * (warp ^ ((c >> 2) & 3)));
-      unpack_int4(v.x, vw[kk][0], vw[kk][1]);
-      unpack_int4(v.y, vw[kk][2], vw[kk][3]);
-    }
-  }
-#pragma unroll
-  for (int hh = 0; hh < G; hh++) {
-    // p codes of this warp's 16 tokens, as 16-bit pairs (tokens 2i, 2i+1)
-    const uint4 pa = *reinterpret_cast<const uint4 *>(&pc_rows[hh][0]);
-    const uint4 pb = *reinterpret_cast<const uint4 *>(&pc_rows[hh][8]);
-    const uint32_t pp[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
-    int ai[4] = {0, 0, 0, 0};
-#pragma unroll
-    for (int j = 0; j < 4; j++) {
-#pragma unroll
-      for (int kk = 0; kk < 4; kk++) {
-        ai[kk] = __dp2a_lo(static_cast<int>(pp[2 * j]), static_cast<int>(vw[kk][j]), ai[kk]);
-        ai[kk] = __dp2a_hi(static_cast<int>(pp[2 * j + 1]), static_cast<int>(vw[kk][j]), ai[kk]);
+      for (int nt = 0; nt < NT; nt++) {
+        int d[4];
+        mma_s8u8_k16_z(d, va[2 * h2], va[2 * h2 + 1], pb[nt]);
+        st.acc[nt][mt][0] = fmaf(f[nt], static_cast<float>(d[0] * 256 + d[1]), st.acc[nt][mt][0]);
+        st.acc[nt][mt][1] = fmaf(f[nt], static_cast<float>(d[2] * 256 + d[3]), st.acc[nt][mt][1]);
       }
     }
-#pragma unroll
-    for (int kk = 0; kk < 4; kk++) acc[hh][kk] = fmaf(cv, static_cast<float>(ai[kk]), acc[hh][kk]);
   }
 }
 
-// The hot ring (nhot FP16 tokens, K and V interleaved per token), for one
-// warp: tokens 8w..8w+7, FP32 arithmetic on the FP16 values with q in FP32
-// (qf [P][128]); weights go through ph_rows ([G][8], this warp's).
-template <int G, int P>
-__device__ __forceinline__ void hot_item(const uint8_t *stage, int nhot, int warp, int lane, int tg, int cs,
-                                         const float (*qf)[kDim], float qk_scale, float (*ph_rows)[8], int hx,
-                                         bool owner, float (&m_run)[G], float (&acc)[G][4], float &m_hx,
-                                         float &l_lane, int &psum_lane) {
-  const int nv = nhot - 8 * warp;
-  if (nv > 0) {
+// nrow FP16 rows (K row, V row) staged at `stage` with pitch kRowStride --
+// the hot ring, or half of an FP16 cold block -- for one warp: rows 8w ..
+// 8w + 7 (rows >= nrow masked; their V is read from the zero row at
+// zero_addr).  QK: mma m16n8k16 f16 (FP32 accumulation) of the FP16 q (A
+// rows g: head g/2, rows g + 8: head 4 + g/2) with the K rows (ldmatrix);
+// weights 2^(z - mx) relative to the 8-row group's maximum, in FP16; P.V: mma
+// m16n8k8 f16 of the V rows (ldmatrix.trans) with B columns 2i = head i's
+// weights, 2i + 1 = 0, so lane (g, t) gets head t's sums.
+template <int NT>
+__device__ __forceinline__ void hot_item(const uint8_t *stage, int nrow, int warp, int lane, int g, int t,
+                                         const __half (*qh)[kDim], float qk_scale, uint32_t zero_addr,
+                                         WarpState<NT> &st) {
+  const int nv = nrow - 8 * warp;
+  if (nv <= 0) return;
+  const uint32_t row0 = smem_addr(stage) + (8 * warp + (lane & 7)) * kRowStride;
+  float c[4] = {0.f, 0.f, 0.f, 0.f};
+  const __half *q0 = qh[g >> 1];
+  const __half *q1 = qh[NT > 1 ? 4 + (g >> 1) : 0];
+#pragma unroll
+  for (int xq = 0; xq < 4; xq++) {
+    uint32_t kb[4];
+    ldmatrix_x4(kb, row0 + 16 * (lane >> 3) + 64 * xq);
+#pragma unroll
+    for (int kk = 0; kk < 2; kk++) {
+      const int d0 = 16 * (2 * xq + kk) + 2 * t;
+      const uint32_t a0 = *reinterpret_cast<const uint32_t *>(q0 + d0);
+      const uint32_t a2 = *reinterpret_cast<const uint32_t *>(q0 + d0 + 8);
+      const uint32_t a1 = NT > 1 ? *reinterpret_cast<const uint32_t *>(q1 + d0) : 0u;
+      const uint32_t a3 = NT > 1 ? *reinterpret_cast<const uint32_t *>(q1 + d0 + 8) : 0u;
+      mma_f16_k16(c, a0, a1, a2, a3, kb[2 * kk], kb[2 * kk + 1]);
+    }
+  }
+  uint32_t pb[NT];
+  float f[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; nt++) {
     float z[2];
 #pragma unroll
-    for (int step = 0; step < 2; step++) {
-      const int t = 8 * warp + 4 * step + tg;
-      const uint4 *kp = reinterpret_cast<const uint4 *>(stage + t * kHotTokenBytes + 32 * cs);
-      const uint4 k0 = kp[0], k1 = kp[1];
-      const uint32_t kr[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-      float kf[16];
+    for (int e = 0; e < 2; e++) z[e] = (2 * t + e < nv) ? c[2 * nt + e] * qk_scale : -INFINITY;
+    float mx = fmaxf(z[0], z[1]);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float mref = mx == -INFINITY ? 0.f : mx;
+    const __half2 hp = __floats2half2_rn(ex2(z[0] - mref), ex2(z[1] - mref));
+    const float2 pr = __half22float2(hp);  // the weights as the tensor cores see them
+    float S = pr.x + pr.y;
+    S += __shfl_xor_sync(0xffffffffu, S, 1);
+    S += __shfl_xor_sync(0xffffffffu, S, 2);
+    pb[nt] = (g & 1) ? 0u : *reinterpret_cast<const uint32_t *>(&hp);
+    const float mx_t = __shfl_sync(0xffffffffu, mx, 8 * t);
+    const float S_t = __shfl_sync(0xffffffffu, S, 8 * t);
+    f[nt] = group_update(mx_t, S_t, st.m_run[nt], st.l_run[nt], st.acc[nt]);
+  }
+  const bool row_ok = (lane & 7) < nv;
 #pragma unroll
-      for (int j = 0; j < 8; j++) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&kr[j]));
-        kf[2 * j] = f.x;
-        kf[2 * j + 1] = f.y;
-      }
-      float dot[P];
+  for (int xp = 0; xp < 4; xp++) {
+    uint32_t va[4];
+    ldmatrix_x4_trans(va, row_ok ? row0 + kHotTokenBytes / 2 + 16 * (lane >> 3) + 64 * xp : zero_addr);
 #pragma unroll
-      for (int kk = 0; kk < P; kk++) {
-        const float4 *qv4 = reinterpret_cast<const float4 *>(&qf[kk ^ hx][16 * cs]);
-        float d = 0.f;
+    for (int h2 = 0; h2 < 2; h2++) {
+      const int mt = 2 * xp + h2;
 #pragma unroll
-        for (int j = 0; j < 4; j++) {
-          const float4 qq = qv4[j];
-          d = fmaf(qq.x, kf[4 * j], d);
-          d = fmaf(qq.y, kf[4 * j + 1], d);
-          d = fmaf(qq.z, kf[4 * j + 2], d);
-          d = fmaf(qq.w, kf[4 * j + 3], d);
-        }
-        dot[kk] = d;
-      }
-      transpose_reduce<P>(dot);
-      z[step] = (4 * step + tg < nv) ? dot[0] * qk_scale : -INFINITY;
-    }
-    {
-      const float zmax = fmaxf(z[0], z[1]);
-      if (__any_sync(0xffffffffu, zmax > m_hx)) raise_max<G, P>(zmax, m_run, acc, m_hx, l_lane, psum_lane, hx);
-    }
-    float pv[2];
-#pragma unroll
-    for (int step = 0; step < 2; step++) {
-      pv[step] = ex2(z[step] - m_hx);
-      l_lane += pv[step];
-    }
-    if (owner) {
-      ph_rows[hx][tg] = pv[0];
-      ph_rows[hx][4 + tg] = pv[1];
-    }
-    __syncwarp();
-    float ah[G][4];
-#pragma unroll
-    for (int hh = 0; hh < G; hh++)
-#pragma unroll
-      for (int kk = 0; kk < 4; kk++) ah[hh][kk] = 0.f;
-    const int ntok = min(nv, 8);
-    for (int tt = 0; tt < ntok; tt++) {
-      const __half *vrow =
-          reinterpret_cast<const __half *>(stage + (8 * warp + tt) * kHotTokenBytes) + kDim;
-      float v[4];
-#pragma unroll
-      for (int kk = 0; kk < 4; kk++) v[kk] = __half2float(vrow[lane + 32 * kk]);
-#pragma unroll
-      for (int hh = 0; hh < G; hh++) {
-        const float p = ph_rows[hh][tt];
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++) ah[hh][kk] = fmaf(p, v[kk], ah[hh][kk]);
+      for (int nt = 0; nt < NT; nt++) {
+        float d[4];
+        mma_f16_k8_z(d, va[2 * h2], va[2 * h2 + 1], pb[nt]);
+        st.acc[nt][mt][0] = fmaf(f[nt], d[0], st.acc[nt][mt][0]);
+        st.acc[nt][mt][1] = fmaf(f[nt], d[2], st.acc[nt][mt][1]);
       }
     }
-#pragma unroll
-    for (int hh = 0; hh < G; hh++)
-#pragma unroll
-      for (int kk = 0; kk < 4; kk++) acc[hh][kk] += ah[hh][kk];
   }
 }
 
-// End of a split: the four warps' online-softmax states merged into the
-// split's normalised output for channel tid (o_s per head) and its
-// log2-sum-exp per head (-inf and 0 when empty).  mbuf: FP32 [kWarps][G][128]
-// and mrun / lrun [kWarps][G] in shared memory.  Two CTA barriers; on return
-// mbuf may be reused.
-template <int G, int P>
-__device__ __forceinline__ void merge_warps(float *mbuf, float (*mrun)[G], float (*lrun)[G], const float (&m_run)[G],
-                                            const float (&acc)[G][4], float l_lane, int psum_lane, int warp,
-                                            int lane, int tid, float (&o_s)[G], float (&lse2_s)[G]) {
-  // denominators: this lane's partial for head hx, summed over the 4 token
-  // groups, then gathered per head from a lane that holds it
-  float l_run[G];
-  {
-    float lt = l_lane + static_cast<float>(psum_lane) * (1.f / 32767.f);
-    lt += __shfl_xor_sync(0xffffffffu, lt, 8);
-    lt += __shfl_xor_sync(0xffffffffu, lt, 16);
+// End of a split: the four warps' states merged into the split's normalised
+// output for channel tid (o_s per head) and its log2-sum-exp per head (-inf
+// and 0 when empty).  mbuf: FP32 [kWarps][4 * NT][kMbufPitch], mrun / lrun
+// [kWarps][4 * NT] in shared memory.  Two CTA barriers; on return mbuf may be
+// reused.
+template <int G, int NT>
+__device__ __forceinline__ void merge_warps(float *mbuf, float (*mrun)[4 * NT], float (*lrun)[4 * NT],
+                                            const WarpState<NT> &st, int warp, int lane, int tid, float (&o_s)[G],
+                                            float (&lse2_s)[G]) {
+  const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-    for (int hh = 0; hh < G; hh++) l_run[hh] = __shfl_sync(0xffffffffu, lt, hh * (8 / P));
-  }
+  for (int nt = 0; nt < NT; nt++) {
+    float *row = mbuf + (warp * 4 * NT + 4 * nt + t) * kMbufPitch;
 #pragma unroll
-  for (int hh = 0; hh < G; hh++)
-#pragma unroll
-    for (int kk = 0; kk < 4; kk++) mbuf[(warp * G + hh) * kDim + lane + 32 * kk] = acc[hh][kk];
-  if (lane == 0) {
-#pragma unroll
-    for (int hh = 0; hh < G; hh++) {
-      mrun[warp][hh] = m_run[hh];
-      lrun[warp][hh] = l_run[hh];
+    for (int mt = 0; mt < 8; mt++) {
+      row[16 * mt + g] = st.acc[nt][mt][0];
+      row[16 * mt + g + 8] = st.acc[nt][mt][1];
+    }
+    if (g == 0) {
+      mrun[warp][4 * nt + t] = st.m_run[nt];
+      lrun[warp][4 * nt + t] = st.l_run[nt];
     }
   }
   __syncthreads();
@@ -685,9 +683,9 @@ __device__ __forceinline__ void merge_warps(float *mbuf, float (*mrun)[G], float
     if (mm != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < kWarps; w++) {
-        const float f = ex2(mrun[w][hh] - mm);
-        num = fmaf(f, mbuf[(w * G + hh) * kDim + tid], num);
-        den = fmaf(f, lrun[w][hh], den);
+        const float fw = ex2(mrun[w][hh] - mm);
+        num = fmaf(fw, mbuf[(w * 4 * NT + hh) * kMbufPitch + tid], num);
+        den = fmaf(fw, lrun[w][hh], den);
       }
     }
     if (den > 0.f) {

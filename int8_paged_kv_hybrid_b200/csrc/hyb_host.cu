@@ -5,6 +5,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <atomic>
 #include <cstring>
 
 #include "kernels.cuh"
@@ -12,6 +13,9 @@
 namespace {
 
 thread_local int g_last_cuda_error = 0;
+
+// limit of the decode pipeline's bounded waits (hyb_set_wait_limit); 0 = default
+std::atomic<long long> g_wait_cycles{0};
 
 int cuda_fail(cudaError_t e) {
   g_last_cuda_error = static_cast<int>(e);
@@ -40,6 +44,11 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 extern "C" {
 
 int hyb_version(void) { return 10000; }
+
+int hyb_set_wait_limit(int64_t cycles) {
+  g_wait_cycles.store(cycles > 0 ? static_cast<long long>(cycles) : 0, std::memory_order_relaxed);
+  return HYB_OK;
+}
 
 int hyb_last_cuda_error(void) { return g_last_cuda_error; }
 
@@ -316,6 +325,8 @@ static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_s
   a.v_new = static_cast<const __half *>(v_new);
   a.seq_cnt = step ? reinterpret_cast<int32_t *>(ws + wl.seq_cnt) : nullptr;
   a.l2_skip = l2_skip ? 1 : 0;
+  const long long wait = g_wait_cycles.load(std::memory_order_relaxed);
+  a.wait_cycles = wait > 0 ? wait : hyb::kDefaultWaitCycles;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int group = d->num_q_heads / d->num_kv_heads;
   const cudaError_t e = hyb::launch_decode(a, group, d->batch, pl.cluster, s);
@@ -332,10 +343,11 @@ int hyb_decode_attn(const hyb_cache_desc *d, const void *q, float softmax_scale,
 
 // Workspace of hyb_decode_attn_sparse: the dense pass's workspace, then a
 // log-sum-exp row per (sequence, query head), then the selection keys
-// [batch][Hq][max_l2], max_l2 = the cold tokens of a max_seq_len sequence.
+// [batch][Hq][max_l2], max_l2 = the cold tokens of a max_seq_len sequence,
+// then the selected positions int32 [batch][Hq][sel_stride].
 struct SparseWs {
-  size_t dense, lse, keys, total;
-  int max_l2;
+  size_t dense, lse, keys, sel, total;
+  int max_l2, sel_stride;
 };
 
 static int sparse_ws(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens, SparseWs *w) {
@@ -348,7 +360,9 @@ static int sparse_ws(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split
   w->dense = ws_layout(d, pl, false).total;
   w->lse = round_up(w->dense, kWsAlign);
   w->keys = w->lse + round_up(rows * sizeof(float), kWsAlign);
-  w->total = w->keys + round_up(rows * static_cast<size_t>(w->max_l2) * sizeof(float), kWsAlign);
+  w->sel = w->keys + round_up(rows * static_cast<size_t>(w->max_l2) * sizeof(float), kWsAlign);
+  w->sel_stride = w->max_l2 < hyb::kMaxTopK ? (w->max_l2 > 0 ? w->max_l2 : 1) : hyb::kMaxTopK;
+  w->total = w->sel + round_up(rows * static_cast<size_t>(w->sel_stride) * sizeof(int32_t), kWsAlign);
   return HYB_OK;
 }
 
@@ -356,6 +370,14 @@ size_t hyb_decode_sparse_workspace_bytes(const hyb_cache_desc *d, int32_t max_se
   SparseWs w;
   if (sparse_ws(d, max_seq_len, split_tokens, &w) != HYB_OK) return 0;
   return w.total;
+}
+
+size_t hyb_decode_sparse_selection(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens,
+                                   int32_t *row_stride) {
+  SparseWs w;
+  if (sparse_ws(d, max_seq_len, split_tokens, &w) != HYB_OK) return 0;
+  if (row_stride) *row_stride = w.sel_stride;
+  return w.sel;
 }
 
 int hyb_decode_attn_sparse(const hyb_cache_desc *d, const void *q, float softmax_scale, int32_t max_seq_len,
@@ -381,6 +403,8 @@ int hyb_decode_attn_sparse(const hyb_cache_desc *d, const void *q, float softmax
   a.status = d->status;
   a.q = static_cast<const __half *>(q);
   a.keys = reinterpret_cast<float *>(ws + w.keys);
+  a.sel = reinterpret_cast<int32_t *>(ws + w.sel);
+  a.sel_stride = w.sel_stride;
   a.out = static_cast<__half *>(out);
   a.lse = lse;
   a.hkv = d->num_kv_heads;

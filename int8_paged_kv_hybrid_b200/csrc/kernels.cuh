@@ -61,6 +61,8 @@ struct DecodeArgs {
   // sparse L2 mode: the INT4 ("L2") blocks are left out of this pass (they
   // are attended by the top-k kernels of sparse.cu)
   int l2_skip;
+  // limit (SM cycles) of the copy pipeline's bounded waits
+  long long wait_cycles;
 };
 
 struct MigrateArgs {
@@ -89,6 +91,8 @@ struct SparseArgs {
   float *keys;                // [batch][Hq][max_l2] selection keys (workspace)
   __half *out;                // FP16 [batch][Hq][128]: the dense pass's result in, the merged result out
   float *lse;                 // [batch][Hq]: the dense pass's log-sum-exp in, merged out (natural log)
+  int32_t *sel;               // [batch][Hq][sel_stride]: the selected L2 positions, ascending (workspace)
+  int sel_stride;
   int hkv, hq, num_phys, max_blocks, quant_bits, hot_tokens, max_l2, top_k, blocks_per_cta;
   int lsub;                   // log2 of the 64-token sub-blocks per block
   int bshift;                 // log2 of the tokens per block
@@ -108,6 +112,9 @@ struct CombineArgs {
 
 // Partial results merged per round (and per group when there are more).
 constexpr int kMergeFan = 16;
+
+// Default limit of a bounded wait: 2^31 SM cycles, about 1 s at B200 clocks.
+constexpr long long kDefaultWaitCycles = 1ll << 31;
 
 cudaError_t launch_append(const AppendArgs &a, int batch, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream);

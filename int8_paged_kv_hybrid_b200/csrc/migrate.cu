@@ -19,8 +19,10 @@
 // share the scale): each thread holds its part of the K and V tiles in
 // registers (codes of slots not yet sealed are taken as 0), the new scale
 // and a 256-entry code table are computed, and the tiles are written back in
-// the new packing (a demoted tile's unused upper 4 KB is zeroed).  A second launch then commits the new counts, after every CTA of
-// the first has read the old ones.
+// the new packing.  A demoted tile's upper 4 KB (unused by INT4 codes) is
+// left as it was: no reader of an INT4 tile looks at it.  A second launch
+// then commits the new counts, after every CTA of the first has read the old
+// ones.
 #include "kernels.cuh"
 
 namespace hyb {
@@ -202,12 +204,6 @@ __global__ void __launch_bounds__(2 * kMigThreads) migrate_kernel(const MigrateA
             make_uint4(tbl4(tb, w[0]), tbl4(tb, w[1]), tbl4(tb, w[2]), tbl4(tb, w[3]));
       }
     }
-  }
-  if (demote) {
-    // the unused upper half of each INT4 tile is zeroed
-#pragma unroll
-    for (int kv = 0; kv < 2; kv++)
-      reinterpret_cast<uint4 *>(tile + kv * kTileBytes + kTileBytes / 2)[tid] = make_uint4(0u, 0u, 0u, 0u);
   }
   if (tid_all < 2) a.scales[((size_t)phys * a.hkv + h) * 2 + tid_all] = s_new[tid_all];
 }

@@ -22,9 +22,13 @@
 
 namespace {
 
-// Largest scratch a call may use: enough for, e.g., batch 16 x 32 query heads
-// x 120 splits.  Problems that need more are rejected with
-// HYB_ERR_SCRATCH_LIMIT.
+// Largest scratch a call may use.  A call whose splits are merged through the
+// scratch needs about rows x (splits + groups) x 516 bytes plus its arrival
+// counters (rows = batch x query heads, groups = ceil(splits / 16) above 16
+// splits, 512 bytes of partial output and 4 of log-sum-exp per row and
+// split or group): e.g. 512 rows (batch 16 x 32 heads) x 15 splits, or 128
+// rows x 59 splits.  Plans whose splits merge inside a thread-block cluster
+// use none.  Problems that need more are rejected with HYB_ERR_SCRATCH_LIMIT.
 constexpr size_t kScratchBytes = 4u << 20;
 
 static __device__ __align__(256) unsigned char g_hyb_scratch[kScratchBytes];

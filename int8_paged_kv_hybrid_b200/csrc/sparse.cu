@@ -166,7 +166,10 @@ __global__ void __launch_bounds__(kScoreThreads) l2_score_kernel(const SparseArg
 #pragma unroll
       for (int g = 0; g < 8; g++) {
         if (g < G) {
+          // the key orders tokens as their logits do: negated for a negative
+          // softmax scale
           float key = okp ? __fmul_rn(__int2float_rn(dot[g]), sk) : -INFINITY;
+          if (okp && a.qk_scale < 0.f) key = -key;
           if (key == 0.f) key = 0.f;  // -0 and +0 are one key
           a.keys[((size_t)b * a.hq + h * G + g) * a.max_l2 + pos] = key;
         }
@@ -359,12 +362,14 @@ __global__ void __launch_bounds__(kT) l2_topk_kernel(const SparseArgs a) {
   }
   __syncthreads();
   const int ns = k;
+  // the selection, left in the workspace for the caller
+  for (int j = tid; j < ns; j += kTopkThreads) a.sel[((size_t)b * a.hq + hh) * a.sel_stride + j] = s_pos[j];
 
   // ---- softmax over the selected tokens (log2 domain, FP32) ----
   const __half *qh = a.q + ((size_t)b * a.hq + hh) * kDim;
   float qa = tid < kDim ? fabsf(__half2float(qh[tid])) : 0.f;
   const float amax = cta_reduce<kT>(qa, s_red, tid, true);
-  const float coef = (amax / 32767.f) * a.qk_scale;
+  const float coef = (amax / 32767.f) * fabsf(a.qk_scale);  // keys carry the sign of the scale
   float zmax = -INFINITY;
   for (int j = tid; j < ns; j += kTopkThreads) {
     const int pos = s_pos[j];

@@ -247,6 +247,31 @@ def kv_bytes(w: Workload, lens: Optional[np.ndarray] = None, quant_bits: int = 8
     return total
 
 
+def append_call_bytes(w: Workload, lens_old: np.ndarray, n_new: np.ndarray, quant_bits: int = 8) -> int:
+    """Algorithmic bytes of one hyb_kv_append call that adds n_new[b] tokens
+    to sequences of lens_old[b] tokens: per kv head, the new tokens' FP16 K
+    and V read (512 B each), the ring rows written (512 B per new token kept
+    hot), the evicted tokens' FP16 rows read from the ring (512 B each, for
+    those that were in the cache before the call), their codes written (256 B
+    per token at INT8, 128 B at INT4; their 512 B FP16 rows at quant_bits 0)
+    and the scale pair of every block they land in read and written (16 B)."""
+    H, Bs = w.hot_tokens, w.block_size
+    total = 0
+    for L0, n in zip(lens_old, n_new):
+        L0, n = int(L0), int(n)
+        L1 = L0 + n
+        e0, e1 = max(0, L0 - H), max(0, L1 - H)
+        evicted = e1 - e0
+        from_ring = max(0, min(e1, L0) - e0)
+        blocks = ((e1 - 1) // Bs - e0 // Bs + 1) if evicted > 0 else 0
+        per_token_code = 512 if quant_bits == 0 else (256 if quant_bits == 8 else 128)
+        b = n * 512 + min(n, H) * 512 + from_ring * 512 + evicted * per_token_code
+        if quant_bits != 0:
+            b += blocks * 16
+        total += b * w.num_kv_heads
+    return total
+
+
 def custom_workload(name, lens, num_q_heads, num_kv_heads, seed, softmax_scale=None,
                     schedule="random", chunk=64, max_step=64, pool_extra=3, n_int4=None,
                     outliers=False, split_tokens=0, hot=HOT, block=BLOCK) -> Workload:

@@ -70,6 +70,8 @@ def _load():
     lib.ora_get_block.argtypes = [P, i32, i32, P, P]
     lib.ora_get_block_fp16.argtypes = [P, i32, i32, P]
     lib.ora_get_ring.argtypes = [P, i32, P]
+    lib.ora_block_q.argtypes = [P, i32, i32]
+    lib.ora_block_q.restype = ctypes.c_int32
     lib.ora_export.argtypes = [P, P, i32, P, P, P, P]
     lib.ora_migrate.argtypes = [P, P]
     lib.ora_n_int4.argtypes = [P, i32]
@@ -207,6 +209,11 @@ class OracleCache:
         vals = np.zeros((self.hkv, 2, self.block, self.d), np.uint16)
         ok = self._lib.ora_get_block_fp16(self._h, b, i, _ptr(vals))
         return bool(ok), vals.view(np.float16)
+
+    def block_q(self, b, i):
+        """127 (INT8), 7 (INT4), -1 (FP16) once block i of sequence b holds a
+        sealed token, else 0."""
+        return int(self._lib.ora_block_q(self._h, int(b), int(i)))
 
     def ring(self, b):
         r = np.zeros((self.hkv, self.hot, 2, self.d), np.uint16)

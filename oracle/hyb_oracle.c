@@ -595,6 +595,13 @@ int ora_get_block_fp16(const ora_cache *c, int b, int i, uint16_t *vals) {
   return 1;
 }
 
+/* Width of logical block i of sequence b: 127 (INT8), 7 (INT4), -1 (FP16)
+ * once a token is sealed in it, else 0. */
+int ora_block_q(const ora_cache *c, int b, int i) {
+  if (b < 0 || b >= c->batch || i < 0 || i >= c->max_blocks) return 0;
+  return c->qmax[(size_t)b * c->max_blocks + i];
+}
+
 /* Hot ring of sequence b: FP16 bits [hkv][hot][2][d]. */
 int ora_get_ring(const ora_cache *c, int b, uint16_t *ring) {
   memcpy(ring, c->ring + (size_t)b * c->hkv * c->hot * 2 * c->d,
@@ -632,6 +639,9 @@ int ora_get_ring(const ora_cache *c, int b, uint16_t *ring) {
 /*   scales: float [num_phys][hkv][2] (not used by FP16 blocks).        */
 /*   hot ring: FP16 [batch][hkv][hot][2][d] (K row, then V row).       */
 /* Only sealed slots are written; other bytes are left as they are.    */
+/* The upper half of an INT4 block's tiles holds no code: its content  */
+/* on the device is unspecified (a block demoted from INT8 keeps its   */
+/* old bytes there), and comparisons leave it out.                     */
 /* ------------------------------------------------------------------ */
 static void put_nibble(uint8_t *word4, int e, int code) {
   uint8_t *byte = word4 + (e & 3);

@@ -47,10 +47,21 @@ def assert_cache_equal(w, cache, ora, where=""):
     hot = cache.hot.cpu().numpy()
     sl = cache.seq_lens.cpu().numpy()
     assert np.array_equal(sl, ex["seq_lens"]), (where, sl, ex["seq_lens"])
-    if not np.array_equal(cold, ex["cold"]):
-        bad = np.argwhere(cold != ex["cold"])
+    want = ex["cold"]
+    if ora.quant_bits != 0:
+        # the upper half of an INT4 block's tiles holds no code (unspecified)
+        cold = cold.copy()
+        want = want.copy()
+        bt = np.asarray(w.block_table)
+        for b in range(w.batch):
+            for i in range(bt.shape[1]):
+                if bt[b, i] >= 0 and ora.block_q(b, i) == 7:
+                    cold[bt[b, i], :, :, 4096:] = 0
+                    want[bt[b, i], :, :, 4096:] = 0
+    if not np.array_equal(cold, want):
+        bad = np.argwhere(cold != want)
         raise AssertionError("%s: %d cold bytes differ, first at %s (gpu %d, oracle %d)" % (
-            where, len(bad), tuple(bad[0]), cold[tuple(bad[0])], ex["cold"][tuple(bad[0])]))
+            where, len(bad), tuple(bad[0]), cold[tuple(bad[0])], want[tuple(bad[0])]))
     if not np.array_equal(sc.view(np.uint32), ex["scales"].view(np.uint32)):
         bad = np.argwhere(sc.view(np.uint32) != ex["scales"].view(np.uint32))
         raise AssertionError("%s: %d scales differ, first at %s (gpu %r, oracle %r)" % (

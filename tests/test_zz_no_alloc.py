@@ -10,7 +10,7 @@ also passes alone in a fresh process."""
 import numpy as np
 import pytest
 
-from harness import MAX_ABS, make_pair, replay
+from harness import MAX_ABS, assert_decode_close, make_pair, replay
 from int8_paged_kv_hybrid_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -38,6 +38,37 @@ def test_noalloc_matches_workspace_entry_point_twice():
         err = float((out.float() - ref).abs().max())
         assert err <= MAX_ABS, (call, err)
         assert torch.isfinite(lse[:3]).all() and torch.isneginf(lse[3]).all()
+    assert cache.status() == 0
+
+
+def test_noalloc_matches_oracle_and_alternates_merge_paths():
+    """Against the FP64 oracle within the accuracy bar, and call after call
+    with plans that alternate between a split merge inside a thread-block
+    cluster (the scratch is not used) and merges through the scratch buffer
+    (one level, and two levels above 16 splits), so that each call finds the
+    buffer as the previous, different call left it."""
+    import torch
+    from int8_paged_kv_hybrid_b200 import _lib
+    w = synth.custom_workload("noalloc_ora", [3100, 700, 1, 64, 2300], 32, 8, seed=8, max_step=64)
+    cache, ora = make_pair(w)
+    replay(w, cache, ora)
+    L = int(w.lens.max())
+    qn = synth.query(w)
+    q = torch.from_numpy(qn).cuda()
+    ref, ref_lse = ora.decode(qn, w.softmax_scale)
+    uses = {}
+    for split in (0, 64, 1024, 128, 0, 64, 3072, 64):
+        need = _lib.hyb_decode_workspace_bytes(cache.desc, L, split)
+        assert need <= _lib.hyb_noalloc_scratch_limit()
+        _, ns = _lib.hyb_decode_plan(cache.desc, L, split)
+        uses[need > 0] = True
+        out = torch.empty((w.batch, w.num_q_heads, 128), dtype=torch.float16, device="cuda")
+        lse = torch.empty((w.batch, w.num_q_heads), dtype=torch.float32, device="cuda")
+        _lib.hyb_decode_attn_noalloc(cache.desc, q, w.softmax_scale, L, split, out, lse)
+        torch.cuda.synchronize()
+        assert_decode_close(w, out.float().cpu().numpy().astype(np.float64), lse.cpu().numpy(), ref, ref_lse,
+                            what="noalloc split=%d (%d splits)" % (split, ns))
+    assert uses.get(True) and uses.get(False), "both merge paths must be exercised"
     assert cache.status() == 0
 
 
