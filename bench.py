@@ -1,15 +1,24 @@
 #!/usr/bin/env python
 """Benchmark of the hybrid_v2 decode path on B200.
 
-One step = one pass of the whole hot path over one batch: hyb_kv_append of
-the step's token (hot-ring write + sealing of the token that leaves the hot
-zone, with quantization) followed by hyb_decode_attn (split-KV attention over
-the hot ring and the INT8 cold blocks, with the log-sum-exp merge of its
-splits).  Workload: Llama-3-8B attention shapes, one layer, batch 8, Hq 32,
-Hkv 8, d 128, every sequence 2048 tokens (32 FP16 hot + 2016 INT8 cold in a
-4096-block pool), seeded synthetic N(0,1) data.
+One step = one pass of the whole hot path over one batch: hyb_decode_step,
+i.e. the append of the step's token (hot-ring write + sealing of the token
+that leaves the hot zone, with quantization) fused with split-KV attention
+over the hot ring and the INT8 cold blocks and the log-sum-exp merge of its
+splits, in one launch.
+
+Default run (the line the driver reads): the headline is the long-context
+workload (batch 4, L = 32K, 32K, 128K, 128K, Llama-3-8B attention shapes,
+512-token splits), the largest single-GPU configuration; the same run
+reports sub-records for the Llama-3-8B batch-8 L=2048 workload, the
+variable-length batch of 64 and the Qwen2-7B mixed batch of 128 (each with
+its own e2e and CPU baseline), an append-only record (one hyb_kv_append of
+U[1,64] tokens per sequence on the variable-length batch) and the oracle's
+one-thread time on the single-sequence workload.  Seeded synthetic N(0,1)
+data throughout.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload 1..5] [--lean] [--migrate] [--sparse-top-k K] ...
 
 Prints one JSON line (rank 0).  With N > 1 (torchrun), every rank runs its
 own batch (weak scaling, no data-path collective); times are the max over
@@ -31,9 +40,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode-attn KV GB/s (frac of HBM peak) and tokens/s at 1 B200 vs CPU oracle"
 UNIT = "GB/s"
-WORKLOAD = 2
-PROFILE = os.path.join(ROOT, "profiles", "decode_splitkv_llama8b_b8_L2048.md")
-KERNEL_SOURCES = ["decode.cu", "decode_dev.cuh", "common.cuh", "kernels.cuh"]  # the profiled kernel's sources
+HEADLINE = 4              # the largest single-GPU configuration
+SUB_WORKLOADS = (2, 3, 5)  # reported in the same run
+APPEND_WORKLOAD = 3
+PROFILE_JSON = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
+# the profiled kernel's sources (their hash tells whether a capture is current)
+KERNEL_SOURCES = ["decode_kernel.cuh", "decode_dev.cuh", "mma.cuh", "common.cuh", "kernels.cuh"]
 FLUSH_BYTES = 512 << 20   # > 126 MB L2
 
 
@@ -44,8 +56,9 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--split", type=int, default=0, help="split_tokens (0 = automatic)")
-    p.add_argument("--workload", type=int, default=WORKLOAD,
-                   help="1..5: the measured shapes (2, the default, is the headline workload)")
+    p.add_argument("--workload", type=int, default=None,
+                   help="1..5: measure this workload alone (default: the headline workload 4 plus the "
+                        "sub-records of workloads 2, 3 and 5, the append record and the 1-thread oracle)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--migrate", action="store_true",
                    help="time hyb_kv_migrate instead of the decode step: demote a quarter of every "
@@ -122,24 +135,33 @@ def kernel_sha():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
-    """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current kernel source."""
+def profiled_traffic(workload_name):
+    """(DRAM bytes per decode launch, how it was obtained) for this workload
+    from the committed ncu figures (profiles/decode_kernel_traffic.json), if
+    they were taken on the current kernel source; else (None, reason)."""
     try:
-        text = open(PROFILE, encoding="utf-8").read()
+        with open(PROFILE_JSON, encoding="utf-8") as fh:
+            d = json.load(fh)
+    except (OSError, ValueError):
+        return None, "no committed ncu figures"
+    if d.get("kernel_source_sha") != kernel_sha():
+        return None, "committed ncu figures predate the current kernel source"
+    rec = d.get("workloads", {}).get(workload_name)
+    if not rec:
+        return None, "no ncu figure for this workload"
+    return float(rec["dram_bytes_per_launch"]), rec.get("how", "ncu")
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo", encoding="utf-8") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
     except OSError:
-        return None
-    vals = {}
-    for line in text.splitlines():
-        if ":" in line and line.strip().startswith("- "):
-            k, v = line.strip()[2:].split(":", 1)
-            vals[k.strip()] = v.strip().strip("`")
-    if vals.get("kernel_source_sha") != kernel_sha():
-        return None
-    try:
-        return float(vals["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 def measured_peaks():
@@ -235,17 +257,21 @@ def room_for_growth(w, extra_tokens):
     w.num_phys_blocks = nxt
 
 
-def build_gpu_state(w, torch, qbits=8):
+def build_gpu_state(w, torch, qbits=8, ora=None):
+    """The library's cache for workload w, prefilled by the library's own
+    appends (64-token calls) to one token short of w.lens; the oracle `ora`,
+    if given, replays the very same calls.  Returns (cache, n_last, k_last, v_last, q): the step's inputs."""
     from int8_paged_kv_hybrid_b200 import HybridKVCache, synth
     cache = HybridKVCache(w.batch, w.num_kv_heads, w.num_q_heads, w.num_phys_blocks, w.max_blocks,
                           quant_bits=qbits, block_table=w.block_table,
                           n_int4=w.n_int4 if qbits == 8 else None, hot_tokens=w.hot_tokens,
                           block_size=w.block_size)
-    # prefill to L-1 in 64-token appends; the benchmarked step appends the last token
     sched = synth._chunk_schedule(w.lens, 64)
     for si, n in enumerate(sched[:-1]):
         k, v = synth.step_tokens(w, si, n, max_new=64)
         cache.append(torch.from_numpy(n).cuda(), torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
+        if ora is not None:
+            ora.append(n, k, v)
     last = len(sched) - 1
     n_last = sched[-1]
     k_last, v_last = synth.step_tokens(w, last, n_last, max_new=1)
@@ -254,14 +280,25 @@ def build_gpu_state(w, torch, qbits=8):
     return cache, n_last, k_last, v_last, q
 
 
-def _touched_blocks(w, n_last):
-    """Physical blocks the step's append can write (the blocks holding the
-    positions that leave the hot zone)."""
+def new_oracle(w, qbits=8):
+    import oracle
+    ora = oracle.OracleCache(w.batch, w.num_kv_heads, w.num_q_heads, w.max_blocks + 16, qbits, hot=w.hot_tokens,
+                             block=w.block_size)
+    if qbits == 8 and w.n_int4 is not None:
+        ora.set_n_int4(w.n_int4)
+    return ora
+
+
+def _touched_blocks(w, n_new, lens_new=None):
+    """Physical blocks an append of n_new[b] tokens (reaching lens_new[b],
+    default w.lens) can write: the blocks holding the positions that leave
+    the hot zone."""
     import numpy as np
+    lens_new = w.lens if lens_new is None else lens_new
     phys = []
     for b in range(w.batch):
-        L_new = int(w.lens[b])
-        L_old = L_new - int(n_last[b])
+        L_new = int(lens_new[b])
+        L_old = L_new - int(n_new[b])
         e0, e1 = max(0, L_old - w.hot_tokens), max(0, L_new - w.hot_tokens)
         for i in range(e0 // w.block_size, (e1 + w.block_size - 1) // w.block_size):
             if e1 > e0:
@@ -269,7 +306,48 @@ def _touched_blocks(w, n_last):
     return np.array(sorted(set(phys)), np.int64)
 
 
-def run_native(args, rank, world, local_rank):
+class StateSnapshot:
+    """What a step changes (hot ring, scales, lengths, the blocks it seals
+    into), copied once and restored before every timed step, untimed."""
+
+    def __init__(self, cache, touched, torch, dev):
+        self.cache = cache
+        self.touched = torch.from_numpy(touched).to(dev)
+        self.snap = {"hot": cache.hot.clone(), "scales": cache.scales.clone(),
+                     "seq_lens": cache.seq_lens.clone(), "cold": cache.cold.index_select(0, self.touched)}
+
+    def restore(self):
+        c, sn = self.cache, self.snap
+        c.hot.copy_(sn["hot"])
+        c.scales.copy_(sn["scales"])
+        c.seq_lens.copy_(sn["seq_lens"])
+        c.cold.index_copy_(0, self.touched, sn["cold"])
+
+
+def time_events(n, stream, before, body):
+    """n iterations of before() (untimed) then body() between two CUDA events
+    on `stream`; returns the event pairs."""
+    import torch
+    evs = []
+    for _ in range(n):
+        before()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        body()
+        e1.record(stream)
+        evs.append((e0, e1))
+    return evs
+
+
+def mean_ms(evs):
+    return sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+
+
+def run_config(args, wl, rank, world, local_rank, clocks=None, cpu=True):
+    """One workload: the fused decode step timed on the device (a CUDA graph
+    of the hyb_decode_step launch, replayed per step), end to end through the
+    C ABI with host buffers, and the oracle on the host cores (rank 0, N=1).
+    Returns (record, workload)."""
     import numpy as np
     import torch
     import torch.distributed as dist
@@ -277,8 +355,7 @@ def run_native(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    clocks = ClockSampler(local_rank) if rank == 0 and not args.lean else None
-    w = synth.make_workload(args.workload, seed_offset=1000 * rank)
+    w = synth.make_workload(wl, seed_offset=1000 * rank)
     if args.hot_tokens != w.hot_tokens or args.block_size != w.block_size:
         # a smaller hot zone seals more blocks; larger blocks use the first
         # entries of the same table
@@ -288,12 +365,14 @@ def run_native(args, rank, world, local_rank):
         room_for_growth(w, args.warmup + args.steps + 2)  # the lean run lets the cache grow
     L = int(w.lens.max())
     qb = args.quant_bits
-    cache, n_last, k_last, v_last, q = build_gpu_state(w, torch, qb)
+    want_cpu = cpu and rank == 0 and world == 1 and not args.no_cpu_baseline and not args.lean
+    ora = new_oracle(w, qb) if want_cpu else None
+    cache, n_last, k_last, v_last, q = build_gpu_state(w, torch, qb, ora)
     if args.lean:
         L += args.warmup + args.steps  # the lean run lets the cache grow one token per step
     split, ns = cache.plan(L, args.split or w.split_tokens)
-    # the step's inputs packed in one buffer (each part 256-byte aligned), so
-    # that the end-to-end run moves them from the host in one copy
+    # the step's inputs packed in one pinned host buffer (each part 256-byte
+    # aligned), moved in one copy per step
     parts = [np.ascontiguousarray(a) for a in (n_last, k_last, v_last, q)]
     offs, off = [], 0
     for a in parts:
@@ -309,21 +388,13 @@ def run_native(args, rank, world, local_rank):
     lse = torch.empty((w.batch, w.num_q_heads), dtype=torch.float32, device=dev)
     ws = cache.step_workspace(L, split)
 
-    # state the step changes, restored before every step (untimed)
-    touched = torch.from_numpy(_touched_blocks(w, n_last)).to(dev)
-    snap = None
-    if not args.lean:
-        snap = {"hot": cache.hot.clone(), "scales": cache.scales.clone(),
-                "seq_lens": cache.seq_lens.clone(), "cold": cache.cold.index_select(0, touched)}
+    snap = None if args.lean else StateSnapshot(cache, _touched_blocks(w, n_last), torch, dev)
     flush = torch.empty(0 if args.lean else FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def restore():
-        if snap is None:
-            return
-        cache.hot.copy_(snap["hot"])
-        cache.scales.copy_(snap["scales"])
-        cache.seq_lens.copy_(snap["seq_lens"])
-        cache.cold.index_copy_(0, touched, snap["cold"])
+    def before():
+        if snap is not None:
+            snap.restore()
+        flush.zero_()
 
     # one eager run (sets kernel attributes, checks the path), then capture the
     # step -- hyb_decode_step: append of the step's token + attention, one
@@ -331,9 +402,9 @@ def run_native(args, rank, world, local_rank):
     side = torch.cuda.Stream(device=dev)
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
-        restore()
+        before()
         cache.step(n_d, k_d, v_d, q_d, w.softmax_scale, L, split, out=out, lse=lse, workspace=ws)
-        restore()
+        before()
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
     g_step = torch.cuda.CUDAGraph()
@@ -342,102 +413,160 @@ def run_native(args, rank, world, local_rank):
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
-    def timed_steps(n):
-        evs = []
-        for _ in range(n):
-            restore()
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            g_step.replay()
-            e1.record(stream)
-            evs.append((e0, e1))
-        return evs
-
-    timed_steps(args.warmup)
+    time_events(args.warmup, stream, before, g_step.replay)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     if clocks:
         clocks.mark()
-    evs = timed_steps(args.steps)
+    evs = time_events(args.steps, stream, before, g_step.replay)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop() if clocks else None
-    ms_step = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / len(evs), world, dev)
+    ms_step = max_over_ranks(mean_ms(evs), world, dev)
     assert torch.isfinite(out.float()).all() and cache.status() == 0
     if args.lean:
         return {"lean": True, "ms_per_step": ms_step}, w
+    del g_step
 
-    # end to end with host buffers: the step's inputs copied from pinned host
-    # memory (one packed copy), the library's fused step, the output copied
-    # back -- all inside the timed span, captured as one CUDA graph
+    # end to end through the C ABI with host buffers: every step copies its
+    # inputs (n_new, k_new, v_new, q) from pinned host memory in one
+    # cudaMemcpyAsync, calls hyb_decode_step (host checks, planning and the
+    # launch, from Python through ctypes) and copies the output back into
+    # pinned host memory -- all between the two events
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     h2d = int(h_in.numel())
     d2h = h_out.numel() * h_out.element_size()
-    g_e2e = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_e2e, stream=side):
+
+    def e2e_body():
         d_in.copy_(h_in, non_blocking=True)
         cache.step(n_d, k_d, v_d, q_d, w.softmax_scale, L, split, out=out, lse=lse, workspace=ws)
         h_out.copy_(out, non_blocking=True)
+
+    time_events(args.warmup, stream, before, e2e_body)
     torch.cuda.synchronize()
-    e2e = []
-    for i in range(args.warmup + args.steps):
-        restore()
-        flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        g_e2e.replay()
-        e1.record(stream)
-        if i >= args.warmup:
-            e2e.append((e0, e1))
+    if world > 1:
+        dist.barrier()
+    e2e = time_events(args.steps, stream, before, e2e_body)
     torch.cuda.synchronize()
     assert torch.equal(h_out, out.cpu())
+    ms_e2e = max_over_ranks(mean_ms(e2e), world, dev)
+
+    # the same, with the three operations captured once as a CUDA graph
+    g_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_e2e, stream=side):
+        e2e_body()
+    torch.cuda.synchronize()
+    time_events(args.warmup, stream, before, g_e2e.replay)
+    e2e_g = time_events(args.steps, stream, before, g_e2e.replay)
+    torch.cuda.synchronize()
     del g_e2e
-    ms_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e) / len(e2e), world, dev)
-    del g_step
+    ms_e2e_g = max_over_ranks(mean_ms(e2e_g), world, dev)
 
     kvb = synth.kv_bytes(w, quant_bits=qb)
     stepb = kvb + synth.append_bytes(w, n_last, qb)
     peak, peak_kind = measured_peaks()
-    total_bytes = kvb * world
     value = job_throughput(kvb, world, ms_step)
     tokens_s = w.batch * world / (ms_step * 1e-3)
     achieved = stepb / (ms_step * 1e-3) / 1e9
-    res = None
-    if rank == 0:
-        res = {
-            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": {8: "int8", 4: "int4", 0: "f16"}[qb],
-            "data": "synthetic (seeded N(0,1) FP16 K/V/q; caches built by the library's own appends)",
-            "config": workload_config(w, split, ns, qb),
-            "tokens_per_s": round(tokens_s, 1),
-            "tokens_per_s_model_equiv": round(tokens_s / 32, 1),
-            "kv_bytes_per_step": kvb,
-            "frac_of_hbm_peak_step": round(value / world / peak, 4),
-            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4),
-                         # the committed ncu figure covers the default workload and cold format only
-                         "traffic": profiled_traffic() if (args.workload == WORKLOAD and qb == 8
-                                                           and args.hot_tokens == 32 and args.block_size == 64
-                                                           and not args.split)
-                                    else None,
-                         "kernel": "hyb::decode_kernel (fused append + attention, the step's only launch)",
-                         "peak_kind": peak_kind,
-                         "achieved_bytes": "algorithmic bytes per launch: attention %d + append %d"
-                                           % (kvb, stepb - kvb)},
-            "e2e": {"value": round(job_throughput(kvb, world, ms_e2e), 1), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": round(ms_e2e, 5)},
-            "gpu_launches": args.steps,
-            "clocks": clk,
-        }
-    return res, w
+    default_shape = (qb == 8 and args.hot_tokens == 32 and args.block_size == 64 and not args.split)
+    traffic, traffic_how = profiled_traffic(w.name) if default_shape else (None, "non-default shape")
+    layers = 28 if w.num_q_heads == 28 else 32
+    rec = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": {8: "int8", 4: "int4", 0: "f16"}[qb],
+        "data": "synthetic (seeded N(0,1) FP16 K/V/q; caches built by the library's own appends)",
+        "config": workload_config(w, split, ns, qb),
+        "tokens_per_s": round(tokens_s, 1),
+        "tokens_per_s_model_equiv": round(tokens_s / layers, 1),
+        "kv_bytes_per_step": kvb,
+        "frac_of_hbm_peak_step": round(value / world / peak, 4),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4),
+                     "traffic": None if traffic is None else int(traffic),
+                     "traffic_source": traffic_how,
+                     "kernel": "hyb::decode_kernel (fused append + attention, the step's only launch)",
+                     "peak_kind": peak_kind,
+                     "achieved_bytes": "algorithmic bytes per launch: attention %d + append %d"
+                                       % (kvb, stepb - kvb)},
+        "e2e": {"value": round(job_throughput(kvb, world, ms_e2e), 1), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 5),
+                "path": "per step: cudaMemcpyAsync of the packed inputs from pinned host memory, "
+                        "hyb_decode_step through the C ABI (ctypes), cudaMemcpyAsync of the output to "
+                        "pinned host memory"},
+        "e2e_graph": {"value": round(job_throughput(kvb, world, ms_e2e_g), 1), "unit": UNIT,
+                      "ms_per_step": round(ms_e2e_g, 5),
+                      "path": "the same three operations captured once as a CUDA graph and replayed"},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+    }
+    if want_cpu:
+        sec, n, threads = oracle_step_rate(ora, w, n_last, k_last, v_last, q, 3, 0, budget_s=25.0, qbits=qb)
+        rec["cpu_baseline"] = {"value": round(kvb / sec / 1e9, 4), "unit": UNIT, "cores": threads,
+                               "kind": "oracle", "cpu_model": cpu_model(),
+                               "sample": "%d full steps of the same workload (1-token append + FP64 attention "
+                                         "of all rows) on the host, OpenMP over rows" % n}
+    del ora
+    return rec, w
+
+
+def run_append(args, rank, world, local_rank):
+    """hyb_kv_append alone on the variable-length batch: the cache is built
+    to L - n, then one timed call appends n[b] ~ U[1, 64] tokens to every
+    sequence (sealing the tokens that leave the hot zone, quantizing them
+    into their blocks, and writing the newest tokens into the ring).  The
+    state the call changes is restored before every call (untimed) and L2 is
+    flushed."""
+    import numpy as np
+    import torch
+    from int8_paged_kv_hybrid_b200 import HybridKVCache, synth
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.make_workload(APPEND_WORKLOAD, seed_offset=1000 * rank)
+    rng = np.random.default_rng([w.seed, 7])
+    n_step = np.minimum(rng.integers(1, 65, size=w.batch), w.lens).astype(np.int32)
+    start = (w.lens - n_step).astype(np.int64)
+    cache = HybridKVCache(w.batch, w.num_kv_heads, w.num_q_heads, w.num_phys_blocks, w.max_blocks,
+                          block_table=w.block_table, hot_tokens=w.hot_tokens, block_size=w.block_size)
+    sched = synth._chunk_schedule(start, 64)  # prefill to exactly `start` tokens
+    for si, n in enumerate(sched):
+        k, v = synth.step_tokens(w, si, n, max_new=64)
+        cache.append(torch.from_numpy(n).to(dev), torch.from_numpy(k).to(dev), torch.from_numpy(v).to(dev))
+    torch.cuda.synchronize()
+    assert np.array_equal(cache.seq_lens.cpu().numpy(), start.astype(np.int32))
+    k, v = synth.step_tokens(w, 10_000, n_step, max_new=64)
+    n_d, k_d, v_d = (torch.from_numpy(x).to(dev) for x in (n_step, k, v))
+    snap = StateSnapshot(cache, _touched_blocks(w, n_step), torch, dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def before():
+        snap.restore()
+        flush.zero_()
+
+    def body():
+        cache.append(n_d, k_d, v_d)
+
+    stream = torch.cuda.current_stream()
+    time_events(args.warmup, stream, before, body)
+    evs = time_events(args.steps, stream, before, body)
+    torch.cuda.synchronize()
+    assert cache.status() == 0
+    ms = max_over_ranks(mean_ms(evs), world, dev)
+    ab = synth.append_call_bytes(w, start, n_step)
+    return {"workload": "hyb_kv_append on the variable-length batch: 64 sequences, L in [256, 8192], one call of "
+                        "U[1,64] new tokens per sequence (%d in all), INT8 cold blocks" % int(n_step.sum()),
+            "ms_per_call": round(ms, 5), "us_per_call": round(ms * 1e3, 2),
+            "GB/s": round(ab / (ms * 1e-3) / 1e9, 1), "algorithmic_bytes": ab,
+            "tokens_per_s": round(float(n_step.sum()) / (ms * 1e-3), 1),
+            "bytes": "per kv head: new K/V read (512 B/token), ring rows written (512 B each), evicted FP16 rows "
+                     "read from the ring (512 B each), sealed codes written (256 B/token), the touched blocks' "
+                     "scale pairs read and written (16 B/block)",
+            "gpu_launches": args.steps}
 
 
 def run_migrate(args):
@@ -447,7 +576,7 @@ def run_migrate(args):
     import numpy as np
     import torch
     from int8_paged_kv_hybrid_b200 import synth
-    wl = args.workload if args.workload != WORKLOAD else 3
+    wl = args.workload if args.workload is not None else 3
     w = synth.make_workload(wl)
     cache, n_last, k_last, v_last, q = build_gpu_state(w, torch)
     cache.append(torch.from_numpy(n_last).cuda(), torch.from_numpy(k_last).cuda(), torch.from_numpy(v_last).cuda())
@@ -480,8 +609,7 @@ def run_migrate(args):
     peak, peak_kind = measured_peaks()
     tile = 2 * 8192
     # algorithmic bytes: the old tiles read and the new codes written (plus the
-    # 8-byte scale pair read and written); a demotion also zeroes the unused
-    # half of each tile (8 KB), counted in "bytes_written" but not here
+    # 8-byte scale pair read and written)
     alg = {"demote": moved * (tile + tile // 2 + 16), "promote": moved * (tile // 2 + tile + 16)}
     gbs = {k: alg[k] / (ms[k] * 1e-3) / 1e9 for k in ms}
     return {
@@ -498,7 +626,7 @@ def run_migrate(args):
                      "achieved_bytes": "per call: %d tile pairs x (16384 read + 8192 written + 16 scale bytes)"
                                        % moved,
                      "promote_frac": round(gbs["promote"] / peak, 4)},
-        "bytes_written_demote": moved * (tile // 2 + tile // 2 + 8),
+        "bytes_written_demote": moved * (tile // 2 + 8),
         "gpu_launches": 2 * args.steps * 2,
         "clocks": clk,
     }
@@ -510,7 +638,7 @@ def run_sparse(args):
     import numpy as np
     import torch
     from int8_paged_kv_hybrid_b200 import hyb_sparse_top_k, synth
-    wl = args.workload if args.workload != WORKLOAD else 4
+    wl = args.workload if args.workload is not None else 4
     w = synth.make_workload(wl)
     if w.n_int4 is None:
         w.n_int4 = (w.cold_blocks() // 2).astype(np.int32)
@@ -574,26 +702,11 @@ def run_sparse(args):
     }
 
 
-def oracle_step_rate(w, steps, warmup, budget_s=None, qbits=8):
-    """Time the CPU oracle (as it stands) on the same workload: per step the
-    1-token append plus FP64 attention of every (sequence, head).  The state
-    grows by one token per step (bounded sample)."""
-    import numpy as np
-    import oracle
-    from int8_paged_kv_hybrid_b200 import synth
-    threads = os.cpu_count() or 1
-    ora = oracle.OracleCache(w.batch, w.num_kv_heads, w.num_q_heads, w.max_blocks + 16, qbits, hot=w.hot_tokens,
-                             block=w.block_size)
-    if qbits == 8 and w.n_int4 is not None:
-        ora.set_n_int4(w.n_int4)
-    sched = synth._chunk_schedule(w.lens, 64)
-    for si, n in enumerate(sched[:-1]):
-        k, v = synth.step_tokens(w, si, n, max_new=64)
-        ora.append(n, k, v)
-    last = len(sched) - 1
-    n_last = sched[-1]
-    k_last, v_last = synth.step_tokens(w, last, n_last, max_new=1)
-    q = synth.query(w)
+def oracle_step_rate(ora, w, n_last, k_last, v_last, q, steps, warmup, budget_s=None, qbits=8, nthreads=None):
+    """Time the CPU oracle (as it stands) on a prefilled copy of the workload:
+    per step the 1-token append plus FP64 attention of every (sequence,
+    head).  The state grows by one token per step (bounded sample)."""
+    threads = nthreads or os.cpu_count() or 1
     times = []
     for i in range(warmup + steps):
         t0 = time.perf_counter()
@@ -607,6 +720,37 @@ def oracle_step_rate(w, steps, warmup, budget_s=None, qbits=8):
     return sum(times) / len(times), len(times), threads
 
 
+def oracle_prefilled(w, qbits=8):
+    """The oracle with the workload's prefill replayed (the same arrays the
+    library gets) and the step's inputs."""
+    from int8_paged_kv_hybrid_b200 import synth
+    ora = new_oracle(w, qbits)
+    sched = synth._chunk_schedule(w.lens, 64)
+    for si, n in enumerate(sched[:-1]):
+        k, v = synth.step_tokens(w, si, n, max_new=64)
+        ora.append(n, k, v)
+    last = len(sched) - 1
+    n_last = sched[-1]
+    k_last, v_last = synth.step_tokens(w, last, n_last, max_new=1)
+    return ora, n_last, k_last, v_last, synth.query(w)
+
+
+def oracle_one_thread_config1():
+    """The oracle on the single-sequence workload (L = 1024, 8 heads) with one
+    thread: FP64 attention of all rows, per step."""
+    from int8_paged_kv_hybrid_b200 import synth
+    w = synth.make_workload(1)
+    ora, n_last, k_last, v_last, q = oracle_prefilled(w)
+    sec, n, _ = oracle_step_rate(ora, w, n_last, k_last, v_last, q, 20, 2, budget_s=10.0, nthreads=1)
+    kvb = synth.kv_bytes(w)
+    return {"workload": w.name, "threads": 1, "ms_per_step": round(sec * 1e3, 3),
+            "value": round(kvb / sec / 1e9, 4), "unit": UNIT, "steps": n, "cpu_model": cpu_model()}
+
+
+SUB_KEYS = ("value", "unit", "ms_per_step", "tokens_per_s", "tokens_per_s_model_equiv", "kv_bytes_per_step",
+            "frac_of_hbm_peak_step", "e2e", "e2e_graph", "cpu_baseline", "config")
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -616,25 +760,30 @@ def main():
         print(json.dumps({"error": "run N > 1 under torchrun"}))
         return 2
     from int8_paged_kv_hybrid_b200 import synth
+    wl_main = HEADLINE if args.workload is None else args.workload
 
     if args.impl == "reference":
         # the CPU oracle on the host cores: rank 0 alone
         if rank != 0:
             return 0
-        w = synth.make_workload(args.workload)
+        w = synth.make_workload(wl_main)
         w.hot_tokens, w.block_size = args.hot_tokens, args.block_size
-        sec, n, threads = oracle_step_rate(w, args.steps, args.warmup, budget_s=150.0, qbits=args.quant_bits)
+        ora, n_last, k_last, v_last, q = oracle_prefilled(w, args.quant_bits)
+        sec, n, threads = oracle_step_rate(ora, w, n_last, k_last, v_last, q, args.steps, args.warmup,
+                                           budget_s=120.0, qbits=args.quant_bits)
         kvb = synth.kv_bytes(w, quant_bits=args.quant_bits)
         val = kvb / sec / 1e9
         print(json.dumps({
             "impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": UNIT, "n_gpus": world,
             "steps": n, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(w, 0, 0, args.quant_bits),
+            "data": "synthetic", "config": workload_config(w, w.split_tokens, 0, args.quant_bits),
             "tokens_per_s": round(w.batch / sec, 3),
             "cpu_baseline": {"value": round(val, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "cpu_model": cpu_model(),
                              "sample": "%d full steps of the workload (append 1 token/seq + FP64 attention "
-                                       "of all 256 rows), state growing 1 token per step" % n},
+                                       "of all %d rows), state growing 1 token per step (at most ~120 s)"
+                                       % (n, w.batch * w.num_q_heads)},
             "e2e": {"value": round(val, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }))
         return 0
@@ -654,14 +803,22 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
                                 device_id=torch.device("cuda", local_rank))
-    res, w = run_native(args, rank, world, local_rank)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.lean:
-        sec, n, threads = oracle_step_rate(w, 3, 0, budget_s=30.0, qbits=args.quant_bits)
-        res["cpu_baseline"] = {"value": round(synth.kv_bytes(w, quant_bits=args.quant_bits) / sec / 1e9, 4),
-                               "unit": UNIT,
-                               "cores": threads, "kind": "oracle",
-                               "sample": "%d full steps of the same workload (1-token append + FP64 "
-                                         "attention of all rows) on the host, OpenMP over rows" % n}
+    clocks = ClockSampler(local_rank) if rank == 0 and not args.lean else None
+    res, w = run_config(args, wl_main, rank, world, local_rank, clocks=clocks)
+    if args.workload is None and not args.lean:
+        # every other measured configuration in the same run, then the
+        # append-only record and the oracle's one-thread time
+        res["configs"] = {}
+        for wl in SUB_WORKLOADS:
+            sub, ws = run_config(args, wl, rank, world, local_rank)
+            res["configs"][ws.name] = {k: sub[k] for k in SUB_KEYS if k in sub}
+            res["configs"][ws.name]["roofline_frac"] = sub["roofline"]["frac"]
+            res["configs"][ws.name]["traffic"] = sub["roofline"]["traffic"]
+            res["gpu_launches"] += sub["gpu_launches"]
+        res["append"] = run_append(args, rank, world, local_rank)
+        res["gpu_launches"] += res["append"]["gpu_launches"]
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            res["oracle_one_thread"] = oracle_one_thread_config1()
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
