@@ -250,12 +250,16 @@ size_t hyb_decode_workspace_bytes(const hyb_cache_desc *desc, int32_t max_seq_le
  * are merged by log-sum-exp (the same merge as hyb_combine) through
  * distributed shared memory; with more, the last CTA of a (sequence, kv head)
  * to finish merges them through the workspace.
- * Arithmetic: cold dot products run exactly in integers (16-bit fixed-point q
- * per head, 16-bit fixed-point softmax weights per 16-token group); hot
- * tokens in FP32; the online softmax, the per-block scale products and all
- * merges in FP32.  Accuracy versus exact FP64 attention on the same cache:
- * max-abs error <= 2e-3 and per-row relative L2 <= 1e-3 on the measured
- * workloads.
+ * Arithmetic (tensor cores, warp-level mma): cold dot products run exactly
+ * in integers -- q in 24-bit fixed point per head (relative to its largest
+ * channel) against the codes, and softmax weights in 16-bit fixed point
+ * relative to the maximum of their 16-token group against the V codes; FP16
+ * rows (hot ring, FP16 cold blocks) with FP16 weights relative to their
+ * 8-row group's maximum and FP32 accumulation; the online softmax, the
+ * per-block scale products and all merges in FP32.  Accuracy versus exact
+ * FP64 attention on the same cache: max-abs error <= 2e-3 and per-row
+ * relative L2 <= 1e-3 on the measured workloads, an attention sink 12 nats
+ * above a 32K-token tail and a q with one channel 100x the others.
  */
 int hyb_decode_attn(const hyb_cache_desc *desc, const void *q, float softmax_scale,
                     int32_t max_seq_len, int32_t split_tokens, void *workspace,
@@ -267,13 +271,20 @@ int hyb_decode_attn(const hyb_cache_desc *desc, const void *q, float softmax_sca
  * hyb_decode_attn, except that of the tokens a sequence holds in its INT4
  * ("L2") blocks -- logical blocks below n_int4_blocks[b] (quant_bits 8), every
  * cold block (quant_bits 4) -- each query head attends only the top_k with
- * the largest selection keys, plus every other token:
+ * the largest attention scores (logits), plus every other token.  The
+ * selection ranks by a key that approximates the logit:
  *   key_j = (float)(sum_c qi_c * Kcode_j,c) * Kscale_j   (FP32, one rounding
- *           per operation; -0 counts as +0),
+ *           per operation; -0 counts as +0; negated for a negative
+ *           softmax_scale),
  *   qi_c  = clamp(rint(q_c * (32767 / max_c |q_c|)), -32767, 32767),
  * the head's q in 16-bit fixed point; equal keys keep the older position.
- * All L2 tokens are attended when there are at most top_k of them; top_k 0
- * attends none.  Accuracy as hyb_decode_attn.
+ * So a kept token's logit is never below an unselected token's by more than
+ * their two key errors, |softmax_scale| * max|q| / 32767 * 0.502 * Kscale_j
+ * * sum_c |Kcode_j,c| + 2^-22 * |logit_j| each (where two logits are closer
+ * than that, either choice is a correct top-k).  All L2 tokens are attended
+ * when there are at most top_k of them; top_k 0 attends none.  The selection
+ * is left in the workspace (hyb_decode_sparse_selection).  Accuracy as
+ * hyb_decode_attn over the selected set.
  *   top_k      0 .. 1024 (the page's default is 32; see hyb_sparse_top_k).
  *   workspace  at least hyb_decode_sparse_workspace_bytes() bytes, 16-byte
  *              aligned, zero-filled before its first use (its leading part is

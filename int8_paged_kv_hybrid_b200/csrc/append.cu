@@ -71,6 +71,24 @@ __device__ __forceinline__ void word_elem(int w, int e, int kv, bool int4, int &
   }
 }
 
+// Code matrix of one block's new slots, one byte per code.  K: token-major
+// rows of 128 channels, so that the 4 (8) codes of an INT8 (INT4) K word are
+// consecutive bytes; V: channel-major rows of the block's slots (pitch 132,
+// which spreads the per-channel stores over the banks), so that the codes of
+// a V word are consecutive bytes too.
+constexpr int kCmPitchV = 2 * kBlock + 4;
+union CodeMatrix {
+  int8_t k[2 * kBlock][kDim];   // [block slot - first][channel]
+  int8_t v[kDim][kCmPitchV];    // [channel][block slot - first]
+};
+
+struct AppendSmem {
+  __half xs[2 * kBlock][kDim];  // the block's new values [block slot - first][channel]
+  CodeMatrix cm;
+  int8_t tbl[256];              // re-quantization table
+  float s_max[kAppendThreads / 32];
+};
+
 __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendArgs a) {
   const int pair = blockIdx.x, b = blockIdx.y;
   const int h = pair >> 1, kv = pair & 1;
@@ -87,34 +105,51 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendArgs a) {
   const int H = a.hot_tokens;
   const int B = 1 << a.bshift;  // tokens per block
   const int e0 = max(0, L_old - H), e1 = max(0, L_new - H);
-  __shared__ int8_t cm[2 * kBlock][kDim];  // codes of the block's new slots [block slot - first][ch]
-  __shared__ int8_t tbl[256];                         // re-quantization table
-  __shared__ float s_max[kAppendThreads / 32];
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  AppendSmem &sm = *reinterpret_cast<AppendSmem *>(smem_raw);
+  auto &xs = sm.xs;
+  auto &cm = sm.cm;
+  auto &tbl = sm.tbl;
+  auto &s_max = sm.s_max;
   const int c = tid;  // channel
 
   for (int p0 = e0; p0 < e1;) {
     const int i = p0 / B;
     const int p1 = min((i + 1) * B, e1);
     const int first = p0 - i * B, last = p1 - i * B;  // new slots [first, last) of the block
+    const int nn = p1 - p0;
     const int phys = a.block_table[(size_t)b * a.max_blocks + i];
     if (phys < 0 || phys >= a.num_phys) {
       if (tid == 0) set_status(a.status, HYB_STATUS_BAD_BLOCK);
       p0 = p1;
       continue;
     }
+    // the new values of channel c, 16 loads in flight at a time, into xs;
+    // their absmax (FP32, exact)
+    float amax = 0.f;
+    for (int t0 = 0; t0 < nn; t0 += 16) {
+      __half x[16];
+#pragma unroll
+      for (int u = 0; u < 16; u++)
+        x[u] = t0 + u < nn ? src_row(a, b, h, kv, L_old, p0 + t0 + u)[c] : __float2half_rn(0.f);
+#pragma unroll
+      for (int u = 0; u < 16; u++) {
+        if (t0 + u < nn) {
+          xs[t0 + u][c] = x[u];
+          amax = fmaxf(amax, fabsf(__half2float(x[u])));
+        }
+      }
+    }
     if (a.quant_bits == 0) {
       // FP16 cold block: the rows move unchanged (K row then V row per slot)
       __half *blk = reinterpret_cast<__half *>(a.cold + ((size_t)phys * a.hkv + h) * B * kHotTokenBytes);
-      for (int t = p0; t < p1; t++) blk[((t - i * B) * 2 + kv) * kDim + c] = src_row(a, b, h, kv, L_old, t)[c];
+      for (int t = 0; t < nn; t++) blk[((first + t) * 2 + kv) * kDim + c] = xs[t][c];
+      __syncthreads();  // xs reused by the next block
       p0 = p1;
       continue;
     }
     const bool int4 = a.quant_bits == 4 || (a.n_int4 != nullptr && i < a.n_int4[b]);
     const int q = int4 ? 7 : 127;
-    // absmax of the new values (exact in FP32), thread = channel
-    float amax = 0.f;
-#pragma unroll 8
-    for (int t = p0; t < p1; t++) amax = fmaxf(amax, fabsf(__half2float(src_row(a, b, h, kv, L_old, t)[c])));
 #pragma unroll
     for (int m = 16; m > 0; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
     if (lane == 0) s_max[warp] = amax;
@@ -132,53 +167,68 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendArgs a) {
     }
     if (rq)
       for (int cc = tid - 127; cc <= 127; cc += kAppendThreads) tbl[cc + 127] = static_cast<int8_t>(requantize(cc, s_old, s, q));
-    // the new slots' codes
-#pragma unroll 8
-    for (int t = p0; t < p1; t++) cm[t - p0][c] = static_cast<int8_t>(quantize(__half2float(src_row(a, b, h, kv, L_old, t)[c]), s, q));
+    // the new slots' codes, in the layout of this CTA's half (K or V)
+    for (int t = 0; t < nn; t++) {
+      const int8_t code = static_cast<int8_t>(quantize(__half2float(xs[t][c]), s, q));
+      if (kv == 0) cm.k[t][c] = code;
+      else cm.v[c][t] = code;
+    }
     __syncthreads();
     // rewrite the tiles of the block's 64-slot sub-blocks: only words holding
     // a new slot, or an existing one when the scale grew
     const int St = min(B, kBlock);
     const int lo = rq ? 0 : first;  // slots [lo, last) change
+    const int ne = int4 ? 8 : 4;    // codes per 32-bit word
     for (int u = (lo / kBlock); u <= (last - 1) / kBlock; u++) {
       uint32_t *tile = reinterpret_cast<uint32_t *>(
           a.cold + ((((size_t)phys * a.hkv + h) << a.lsub) + u) * kTilePairBytes + kv * kTileBytes);
       const int s0 = max(lo - kBlock * u, 0), s1 = min(last - kBlock * u, St);  // slots of this sub-block
       const int fu = first - kBlock * u;  // new slots of this sub-block start at fu (may be < 0 or > s1)
-      // words to visit: K rows [s0, s1); V every channel row (its chunks are filtered per word)
+      // words to visit: K rows [s0, s1); V every channel row (its words are
+      // filtered by slot range)
       const int wpr = int4 ? (kv == 0 ? 16 : 8) : (kv == 0 ? 32 : 16);  // words per row
       const int w_begin = kv == 0 ? s0 * wpr : 0;
       const int w_end = kv == 0 ? s1 * wpr : kDim * wpr;
-      const int ne = int4 ? 8 : 4;
       for (int w = w_begin + tid; w < w_end; w += kAppendThreads) {
+        // element e of the word: K -> (slot0, ch0 + e), V -> (slot0 + e, ch0)
         int slot0, ch0;
         word_elem(w, 0, kv, int4, slot0, ch0);
-        // a word covers 4 (INT8) or 8 (INT4) consecutive slots of one channel
-        // row (V) or one slot (K); skip V words entirely outside [s0, s1)
-        if (kv != 0 && (slot0 + ne <= s0 || slot0 >= s1)) continue;
-        const bool need_old = (kv != 0 && (slot0 < fu || slot0 + ne > s1)) || (kv == 0 && slot0 < fu);
-        uint32_t x = need_old ? tile[w] : 0u;
-        uint32_t y = x;
+        if (kv != 0 && (slot0 + ne <= s0 || slot0 >= s1)) continue;  // no slot of the word changes
+        const bool all_new = slot0 >= fu && (kv == 0 || slot0 + ne <= s1);
+        uint32_t y;
+        if (all_new && !int4) {
+          // four new INT8 codes: consecutive bytes of the code matrix
+          const int8_t *src = kv == 0 ? &cm.k[slot0 - fu][ch0] : &cm.v[ch0][slot0 - fu];
+          y = kv == 0 ? *reinterpret_cast<const uint32_t *>(src)
+                      : static_cast<uint32_t>(static_cast<uint8_t>(src[0])) |
+                            (static_cast<uint32_t>(static_cast<uint8_t>(src[1])) << 8) |
+                            (static_cast<uint32_t>(static_cast<uint8_t>(src[2])) << 16) |
+                            (static_cast<uint32_t>(static_cast<uint8_t>(src[3])) << 24);
+        } else {
+          const uint32_t x = all_new ? 0u : tile[w];
+          y = x;
 #pragma unroll
-        for (int e = 0; e < 8; e++) {
-          if (e >= ne) break;
-          int sl, ch;
-          word_elem(w, e, kv, int4, sl, ch);
-          if (sl < s0 || sl >= s1) continue;          // unchanged
-          int code;
-          if (sl >= fu) code = cm[sl - fu][ch];       // new slot (block slot 64u + sl)
-          else {                                      // existing slot under a grown scale
-            const int old = int4 ? nib_get(x, e) : static_cast<int8_t>((x >> (8 * e)) & 0xff);
-            code = tbl[old + 127];
+          for (int e = 0; e < 8; e++) {
+            if (e >= ne) break;
+            const int sl = kv == 0 ? slot0 : slot0 + e;
+            const int ch = kv == 0 ? ch0 + e : ch0;
+            if (sl < s0 || sl >= s1) continue;  // unchanged
+            int code;
+            if (sl >= fu) {
+              code = kv == 0 ? cm.k[sl - fu][ch] : cm.v[ch][sl - fu];  // new slot
+            } else {  // existing slot under a grown scale
+              const int old = int4 ? nib_get(x, e) : static_cast<int8_t>((x >> (8 * e)) & 0xff);
+              code = tbl[old + 127];
+            }
+            if (int4) y = nib_put(y, e, code);
+            else y = (y & ~(0xffu << (8 * e))) | (static_cast<uint32_t>(code & 0xff) << (8 * e));
           }
-          if (int4) y = nib_put(y, e, code);
-          else y = (y & ~(0xffu << (8 * e))) | (static_cast<uint32_t>(code & 0xff) << (8 * e));
         }
         tile[w] = y;
       }
     }
     if (tid == 0) *sp = s;
-    __syncthreads();  // cm / tbl reused by the next block
+    __syncthreads();  // xs, cm and tbl are reused by the next block
     p0 = p1;
   }
   // newest min(n, hot) tokens into the hot ring (their slots' old occupants
@@ -202,7 +252,17 @@ __global__ void append_lens_kernel(AppendArgs a, int batch) {
 }
 
 cudaError_t launch_append(const AppendArgs &a, int batch, cudaStream_t stream) {
-  append_kernel<<<dim3(2 * a.hkv, batch), kAppendThreads, 0, stream>>>(a);
+  static int configured_dev_mask = 0;  // one bit per device
+  int dev = 0;
+  cudaError_t e0 = cudaGetDevice(&dev);
+  if (e0 != cudaSuccess) return e0;
+  if (dev < 31 && !(configured_dev_mask & (1 << dev))) {
+    e0 = cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(sizeof(AppendSmem)));
+    if (e0 != cudaSuccess) return e0;
+    configured_dev_mask |= 1 << dev;
+  }
+  append_kernel<<<dim3(2 * a.hkv, batch), kAppendThreads, sizeof(AppendSmem), stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   append_lens_kernel<<<(batch + 127) / 128, 128, 0, stream>>>(a, batch);

@@ -68,6 +68,8 @@ struct DecodeSmem {
   SealScratch seal;  // fused step
   float cl_l[G];     // this split's log2-sum-exp per head, read by the cluster's merge
   alignas(16) uint32_t zero16[4];  // a zero 16-byte row for masked FP16 rows
+  int rel_cnt[kStages];  // warps done with the stage's current item
+  int issued;            // items issued so far (in order)
   int last;
   int abort_flag;
 };
@@ -200,6 +202,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 3)) decode_kernel(cons
     for (int st = 0; st < kStages; st++) {
       mbar_init(&sm.full[st], 1);
       mbar_init(&sm.empty[st], kWarps);
+      sm.rel_cnt[st] = 0;
     }
     sm.abort_flag = 0;
     mbar_fence_init();
@@ -276,10 +279,9 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 3)) decode_kernel(cons
   float2 sc_ld = make_float2(0.f, 0.f);
   if (!fp16 && tid < ncold && sm.phys[tid] >= 0)
     sc_ld = __ldg(reinterpret_cast<const float2 *>(a.scales + ((size_t)sm.phys[tid] * a.hkv + h) * 2));
-  int issued = 0;
   if (tid == 0) {
-    issued = min(nitems, kStages);
-    for (int k = 0; k < issued; k++) issue(k);
+    sm.issued = min(nitems, kStages);
+    for (int k = 0; k < sm.issued; k++) issue(k);
   }
   if (tid < ncold) sm.scl[tid] = sc_ld;
   // q of the head group in 24-bit fixed point and FP16 (padding heads zero)
@@ -301,31 +303,19 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 3)) decode_kernel(cons
   WarpState<NT> ws;
   state_init<NT>(ws);
 
-  // Once a wait runs out, this warp stops waiting and computing but still
-  // goes through the remaining items, so that every warp passes the same CTA
-  // barriers (those of the fused append); thread 0 stops issuing copies.
+  // Pipeline: item k sits in stage k % kStages.  Each warp releases a stage
+  // when it is done with it (mbarrier `empty`, release semantics); the last
+  // warp to release it -- elected by a shared counter -- waits on that
+  // barrier (already complete, acquire semantics) and issues item k +
+  // kStages into the stage at once, whichever warp that is, so that a
+  // released stage never waits for one particular warp.  Items are issued in
+  // order (the last release of item k precedes that of item k + 1).
+  // Once a wait runs out, a warp stops waiting, computing and releasing but
+  // still goes through the remaining items, so that every warp passes the
+  // same CTA barriers (those of the fused append); no later item is issued.
   bool aborted = false;
-  int next_issue = issued;  // thread 0: next item to bring in
   for (int k = 0; k < nitems; k++) {
     const int st = k % kStages;
-    // thread 0 refills stages the warps have released: item k must be in
-    // flight before anyone waits for it, later ones only if already free
-    if (tid == 0 && !aborted) {
-      for (; next_issue < min(nitems, k + kStages); next_issue++) {
-        const int j = next_issue - kStages;  // previous item of that stage
-        if (next_issue <= k) {
-          if (!mbar_wait_bounded(&sm.empty[j % kStages], (j / kStages) & 1, a.wait_cycles)) {
-            set_status(a.status, HYB_STATUS_TIMEOUT);
-            sm.abort_flag = 1;
-            break;
-          }
-        } else if (!mbar_try_wait(&sm.empty[j % kStages], (j / kStages) & 1)) {
-          break;
-        }
-        issue(next_issue);
-      }
-      issued = next_issue;
-    }
     aborted = aborted || *reinterpret_cast<volatile int *>(&sm.abort_flag) != 0;
     bool ok = !aborted && mbar_wait_bounded(&sm.full[st], (k / kStages) & 1, a.wait_cycles);
     if (!ok && !aborted && lane == 0) set_status(a.status, HYB_STATUS_TIMEOUT);
@@ -385,7 +375,22 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 3)) decode_kernel(cons
       aborted = true;
       continue;
     }
-    if (lane == 0) mbar_arrive(&sm.empty[st]);
+    if (lane == 0) {
+      mbar_arrive(&sm.empty[st]);
+      if (atomicAdd(&sm.rel_cnt[st], 1) == kWarps - 1) {
+        sm.rel_cnt[st] = 0;  // no warp touches it again before item k + kStages lands
+        const int nk = k + kStages;
+        if (nk < nitems && *reinterpret_cast<volatile int *>(&sm.abort_flag) == 0) {
+          if (!mbar_wait_bounded(&sm.empty[st], (k / kStages) & 1, a.wait_cycles)) {
+            set_status(a.status, HYB_STATUS_TIMEOUT);
+            sm.abort_flag = 1;
+          } else {
+            issue(nk);
+            sm.issued = nk + 1;
+          }
+        }
+      }
+    }
   }
   aborted = __syncthreads_or(aborted) != 0;
   // this split's normalised output (channel tid) and log2-sum-exp per head
@@ -394,6 +399,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 3)) decode_kernel(cons
     // let every copy still in flight land before the CTA's shared memory is
     // released: the last item issued into each stage
     if (tid == 0) {
+      const int issued = *reinterpret_cast<volatile int *>(&sm.issued);
       for (int j = max(0, issued - kStages); j < issued; j++)
         (void)mbar_wait_bounded(&sm.full[j % kStages], (j / kStages) & 1, kWaitCycles);
     }

@@ -176,10 +176,14 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
       if (tb < 1) tb = 1;
       if (tb > max_tb) tb = max_tb;
     }
-    if (tb == 0 || units * ((nblk + tb - 1) / tb) > slots) {
+    if (tb == 0 || tb > kMultiWaveSplit || units * ((nblk + tb - 1) / tb) > slots) {
       // several waves: short splits, so that the CTA scheduler evens out
       // sequences of different lengths and CTAs that run at different speeds
-      // (the last CTA placed on an SM gets the fewest issue slots)
+      // (the last CTA placed on an SM gets the fewest issue slots).  Also
+      // when one wave would need splits longer than that: a batch of
+      // (sequence, kv head) rows nearly as large as the GPU's CTA slots would
+      // otherwise give each row one long split, and rows of different
+      // lengths would leave SMs idle.
       tb = kMultiWaveSplit;
       if (tb > nblk) tb = nblk > 0 ? nblk : 1;
     }

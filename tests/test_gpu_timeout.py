@@ -15,7 +15,9 @@ from int8_paged_kv_hybrid_b200 import synth
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("split", [0, 64])
+# splits far longer than the 3-stage copy ring, so that most items are
+# issued during the loop and waited for shortly after
+@pytest.mark.parametrize("split", [64 * 40, 64 * 128])
 def test_wait_limit_times_out_then_recovers(split):
     import torch
     from int8_paged_kv_hybrid_b200 import _lib
@@ -56,6 +58,7 @@ def test_wait_limit_in_fused_step():
     cache, ora = make_pair(w)
     replay(w, cache, ora)
     L = int(w.lens.max()) + 1
+    split = 64 * 40
     rng = np.random.default_rng(3)
     n = torch.ones(w.batch, dtype=torch.int32, device="cuda")
     k = torch.from_numpy(rng.standard_normal((w.batch, 1, 8, 128)).astype(np.float16)).cuda()
@@ -63,12 +66,12 @@ def test_wait_limit_in_fused_step():
     q = torch.from_numpy(synth.query(w)).cuda()
     try:
         _lib.hyb_set_wait_limit(4)
-        cache.step(n, k, v, q, w.softmax_scale, L, 64)
+        cache.step(n, k, v, q, w.softmax_scale, L, split)
         torch.cuda.synchronize()
     finally:
         _lib.hyb_set_wait_limit(0)
     assert cache.status(clear=True) == _lib.HYB_STATUS_TIMEOUT
-    out = cache.decode(q, w.softmax_scale, L, 64)
+    out = cache.decode(q, w.softmax_scale, L, split)
     torch.cuda.synchronize()
     assert torch.isfinite(out.float()).all()
     assert cache.status() == 0

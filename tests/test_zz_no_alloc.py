@@ -49,7 +49,7 @@ def test_noalloc_matches_oracle_and_alternates_merge_paths():
     buffer as the previous, different call left it."""
     import torch
     from int8_paged_kv_hybrid_b200 import _lib
-    w = synth.custom_workload("noalloc_ora", [3100, 700, 1, 64, 2300], 32, 8, seed=8, max_step=64)
+    w = synth.custom_workload("noalloc_ora", [3100, 700, 1, 2300], 32, 8, seed=8, max_step=64)
     cache, ora = make_pair(w)
     replay(w, cache, ora)
     L = int(w.lens.max())
