@@ -209,19 +209,26 @@ int hyb_kv_append(const hyb_cache_desc *desc, const int32_t *n_new, int32_t max_
 /*
  * Split planning for hyb_decode_attn (host only).  max_seq_len is a host
  * upper bound of seq_lens[b]; split_tokens is a multiple of BLK (tokens per
- * split of the cold range) or 0 for automatic.  Writes the split size used
- * and the number of splits per sequence, n_splits = max(1,
- * ceil(max(0, max_seq_len - HOT) / split_tokens)).  Returns HYB_OK or
- * HYB_ERR_INVALID_VALUE.  The automatic choice depends on the GPU's SM count
- * (device 0 of the current context when none is current).
+ * split of the cold range) or 0 for automatic.  A sequence's cold blocks are
+ * cut into runs of tb = split_tokens / BLK blocks; the last split also
+ * attends the hot ring, whose ceil(min(L, HOT) / 32) items of 32 FP16 rows
+ * count as h = min(tb, ceil(items / I)) blocks (I = items per block: 1 for
+ * INT8/INT4 blocks of 32 or 64 tokens, 2 for 128-token blocks, BLK / 32 for
+ * FP16 blocks), so that no split holds more than tb blocks' worth of items.
+ * Writes the split size used and the number of splits per sequence,
+ * n_splits = max(1, ceil((nblk + h) / tb)), nblk = ceil(max(0, max_seq_len -
+ * HOT) / BLK).  Returns HYB_OK or HYB_ERR_INVALID_VALUE.  The automatic
+ * choice depends on the GPU's SM count (device 0 of the current context
+ * when none is current).
  */
 int hyb_decode_plan(const hyb_cache_desc *desc, int32_t max_seq_len, int32_t split_tokens,
                     int32_t *split_tokens_out, int32_t *n_splits_out);
 
 /* Bytes of workspace hyb_decode_attn needs for these arguments, or 0 with an
- * invalid descriptor.  It is 0 when each sequence takes at most 8 splits:
- * the splits of a (sequence, kv head) then run as one thread-block cluster
- * and are merged through distributed shared memory. */
+ * invalid descriptor.  It is 0 when each sequence takes one split, or when
+ * the splits of every (sequence, kv head) run as one thread-block cluster
+ * (2..16 splits, all clusters resident on the GPU at once) and are merged
+ * through distributed shared memory. */
 size_t hyb_decode_workspace_bytes(const hyb_cache_desc *desc, int32_t max_seq_len,
                                   int32_t split_tokens);
 
@@ -245,11 +252,12 @@ size_t hyb_decode_workspace_bytes(const hyb_cache_desc *desc, int32_t max_seq_le
  *   out      device FP16 [batch][Hq][D] (round to nearest even), 16-byte aligned.
  *   lse_out  device FP32 [batch][Hq] natural-log log-sum-exp of the logits, or NULL.
  * An empty sequence (L = 0) gives out = 0 and lse = -inf.
- * One kernel launch: one CTA per (split, kv head, sequence).  With at most 8
- * splits the splits of a (sequence, kv head) form a thread-block cluster and
- * are merged by log-sum-exp (the same merge as hyb_combine) through
- * distributed shared memory; with more, the last CTA of a (sequence, kv head)
- * to finish merges them through the workspace.
+ * One kernel launch: one CTA per (split, kv head, sequence).  When every
+ * split fits on the GPU at once and a (sequence, kv head) has 2..16 splits
+ * whose clusters can all be resident, its splits form a thread-block
+ * cluster and are merged by log-sum-exp (the same merge as hyb_combine)
+ * through distributed shared memory; otherwise the last CTA of a (sequence,
+ * kv head) to finish merges them through the workspace.
  * Arithmetic (tensor cores, warp-level mma): cold dot products run exactly
  * in integers -- q in 24-bit fixed point per head (relative to its largest
  * channel) against the codes, and softmax weights in 16-bit fixed point

@@ -2,16 +2,18 @@
 
     python -m int8_paged_kv_hybrid_b200.build [--force] [--verbose]
 
-Each .cu file is compiled to an object in parallel (objects under _build/,
-git-ignored), then linked into one shared library.  No fast-math: the append
+Each .cu file is compiled to an object in parallel (in a temporary
+directory, removed afterwards), then linked into one shared library.  No fast-math: the append
 kernel must reproduce IEEE division and round-half-even exactly.
 """
 from __future__ import annotations
 
 import glob
 import os
+import shutil
 import subprocess
 import sys
+import tempfile
 from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
@@ -19,7 +21,6 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libhybkv.so")
-OBJ_DIR = os.path.join(PKG, "_build")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -49,29 +50,30 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in _deps())
 
 
-def _compile(src: str, verbose: bool) -> str:
-    obj = os.path.join(OBJ_DIR, os.path.basename(src)[:-3] + ".o")
-    tmp = obj + ".tmp%d" % os.getpid()
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-c", "-o", tmp, src]
+def _compile(src: str, obj_dir: str, verbose: bool) -> str:
+    obj = os.path.join(obj_dir, os.path.basename(src)[:-3] + ".o")
+    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-c", "-o", obj, src]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)
-    os.replace(tmp, obj)
     return obj
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not _stale():
         return LIB
-    os.makedirs(OBJ_DIR, exist_ok=True)
     srcs = sources()
-    with ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
-    tmp = LIB + ".tmp%d" % os.getpid()
-    subprocess.check_call([nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs,
-                           "-lcudart"])
-    os.replace(tmp, LIB)
+    obj_dir = tempfile.mkdtemp(prefix="hybkv_build_")
+    try:
+        with ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
+            objs = list(ex.map(lambda s: _compile(s, obj_dir, verbose), srcs))
+        tmp = LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call([nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs,
+                               "-lcudart"])
+        os.replace(tmp, LIB)
+    finally:
+        shutil.rmtree(obj_dir, ignore_errors=True)
     return LIB
 
 

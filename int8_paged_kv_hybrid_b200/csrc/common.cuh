@@ -126,6 +126,16 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   return pol;
 }
 
+// Arrival counter increment with acquire-release semantics at GPU scope.
+// Used after a CTA barrier by one thread: it publishes the writes the CTA
+// made before the barrier (release), and the thread that sees the final
+// count observes every other CTA's published writes (acquire).
+__device__ __forceinline__ int atomic_add_acq_rel_gpu(int32_t *p, int v) {
+  int old;
+  asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 // ---- integer helpers ----
 // Sign-extend the four 4-bit values held in the low nibbles of the bytes of
 // u (high nibbles zero) to four int8 bytes.

@@ -6,12 +6,14 @@
 namespace hyb {
 
 constexpr int kMaxSplitBlocksD = 128;  // == the kernel's threads: one block-table entry per thread
-constexpr int kMaxClusterD = 8;        // largest cluster the kernel is launched with (portable size)
+constexpr int kMaxClusterD = 16;       // largest cluster the kernel is launched with (non-portable above 8)
 
 template <bool kF16, bool kSkip, int kBshift>
 cudaError_t launch_decode_f(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream);
 template <bool kF16, bool kSkip, int kBshift>
 int decode_occupancy(int group);
+template <bool kF16, bool kSkip, int kBshift>
+int decode_active_clusters(int group, int csize);
 
 template <int kBshift>
 static cudaError_t launch_decode_l(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream) {
@@ -30,6 +32,22 @@ cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, bool cluste
 }
 
 int decode_max_cluster() { return kMaxClusterD; }
+
+// Clusters of csize CTAs (2..16) that can be resident at once for this head
+// group (0 if none, or the device cannot be queried); cached per device.
+int decode_resident_clusters(int group, int csize) {
+  static int cached[32][9][kMaxClusterD + 1];  // [device][group][size], 0 = not yet known, -1 = none
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (group < 1 || group > 8 || csize < 2 || csize > kMaxClusterD) return 0;
+  if (dev >= 0 && dev < 32 && cached[dev][group][csize] != 0) return cached[dev][group][csize] > 0 ? cached[dev][group][csize] : 0;
+  const int n = decode_active_clusters<false, false, 6>(group, csize);
+  if (dev >= 0 && dev < 32) cached[dev][group][csize] = n > 0 ? n : -1;
+  return n;
+}
 
 int decode_max_split_blocks() { return kMaxSplitBlocksD; }
 

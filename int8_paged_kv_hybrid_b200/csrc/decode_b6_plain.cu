@@ -6,4 +6,5 @@
 namespace hyb {
 template cudaError_t launch_decode_f<false, false, 6>(const DecodeArgs &, int, int, bool, cudaStream_t);
 template int decode_occupancy<false, false, 6>(int);
+template int decode_active_clusters<false, false, 6>(int, int);
 }  // namespace hyb

@@ -241,17 +241,14 @@ __device__ __forceinline__ void requant_staged(const SealScratch &ss, uint8_t *t
 }
 
 // Fused decode step, ring half: the new token goes to ring slot rs = L_old %
-// hot -- row rs % 32 of its staged hot item (item_st, pitch kRowStride, for
-// this attention) and the cache.  Thread tid writes channel tid of both rows.
-__device__ __forceinline__ void ring_put(uint8_t *item_st, int rs, __half2 new_kv, const DecodeArgs &a, int b,
-                                         int h, int tid) {
+// hot -- row rs % 32 of its staged hot item (item_st, pitch kRowStride), for
+// this attention (the kernel writes it into the ring in HBM separately).
+// Thread tid writes channel tid of both rows.
+__device__ __forceinline__ void ring_put(uint8_t *item_st, int rs, __half2 new_kv, int tid) {
   const int c = tid;
   __half *srow = reinterpret_cast<__half *>(item_st + (rs % kItemRows) * kRowStride);
   srow[c] = __low2half(new_kv);
   srow[kDim + c] = __high2half(new_kv);
-  __half *grow = reinterpret_cast<__half *>(a.hot) + ((((size_t)b * a.hkv + h) * a.hot_tokens + rs) * 2) * kDim;
-  grow[c] = __low2half(new_kv);
-  grow[kDim + c] = __high2half(new_kv);
   fence_proxy_async_smem();
   __syncthreads();
 }

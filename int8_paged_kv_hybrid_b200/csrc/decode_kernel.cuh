@@ -129,7 +129,17 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 3)) decode_kernel(cons
   constexpr int Bt = 1 << kBshift;                      // tokens per block
   constexpr int St = Bt < kBlock ? Bt : kBlock;         // tokens per sub-block
   const int nblk = (Lc + Bt - 1) / Bt;
-  const int Sb = max(1, (max(0, nblk - ib) + a.split_blocks - 1) / a.split_blocks);
+  constexpr bool fp16 = kF16;
+  constexpr int ish = fp16 ? kBshift - 5 : lsub;  // log2 of the items per block
+  // Splits of this sequence: runs of split_blocks cold blocks from block ib
+  // on; the last split also attends the hot ring, whose items count as
+  // (up to split_blocks) blocks when the sequence is cut, so that no split
+  // has more than split_blocks blocks' worth of items (the hot ring may then
+  // be alone in its split)
+  const int nrem = max(0, nblk - ib);
+  const int dh = (min(L, H) + kItemRows - 1) / kItemRows;  // hot items
+  const int dhb = min((dh + (1 << ish) - 1) >> ish, a.split_blocks);
+  const int Sb = max(1, (nrem + dhb + a.split_blocks - 1) / a.split_blocks);
   // Fused step: the last CTA of the sequence advances seq_lens[b].  A CTA
   // takes its ticket only after a barrier that follows every one of its
   // threads' reads of seq_lens[b], so the CTA holding the last ticket writes
@@ -156,18 +166,25 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 3)) decode_kernel(cons
   const int ncold = max(0, min(nblk, i0 + a.split_blocks) - i0);
   // Items: one per 64-token sub-block (16 KB K + V tiles), or per 32 rows of
   // FP16 (the hot ring, FP16 cold blocks: 2 << lsub items per block)
-  const int nhot = (s == Sb - 1) ? min(L, H) : 0;
-  constexpr bool fp16 = kF16;
-  constexpr int ish = fp16 ? kBshift - 5 : lsub;  // log2 of the items per block
+  const bool holds_hot = s == Sb - 1;
+  const bool holds_tail = ncold > 0 && i0 + ncold == nblk;  // the sequence's last cold block
+  const int nhot = holds_hot ? min(L, H) : 0;
   const int ncold_it = ncold << ish;
   const int kh = ncold_it;  // the first hot item
   const int nitems = ncold_it + (nhot + kItemRows - 1) / kItemRows;
-  // fused step, in the split that holds the tail block and the hot ring: the
-  // new token goes to ring slot rs = L_old % hot, whose old occupant
-  // (position L_old - hot, read in the prologue) is sealed into the tail
-  // block at that block's item; the ring slot is rewritten at its hot item
-  const bool do_ring = n_app == 1 && nhot > 0;
-  const bool do_seal = do_ring && L_old >= H;
+  // Fused step: the new token goes to ring slot rs = L_old % hot, whose old
+  // occupant (position L_old - hot) is sealed into the tail block.  The CTA
+  // holding the tail block reads that occupant in its prologue, seals it at
+  // the tail block's item, and writes the new token into the ring in HBM
+  // (after its own read of the slot); the CTA holding the hot ring puts the
+  // new token into its staged copy of the slot -- which, if the tail block is
+  // in another CTA, may have been copied before or after that write, so the
+  // staged put makes both cases the same.  With nothing to seal (L_old <
+  // hot), the hot-ring CTA writes the ring in HBM itself.
+  const bool do_seal_seq = n_app == 1 && L_old >= H;  // a token leaves the hot zone
+  const bool do_seal = do_seal_seq && holds_tail;
+  const bool do_ring = n_app == 1 && holds_hot;       // staged put
+  const bool ring_hbm = n_app == 1 && (do_seal_seq ? holds_tail : holds_hot);
   const int rs = L_old & (H - 1);
   const int k_ring = kh + rs / kItemRows;
   // slot of the sealed token in the tail block; in the split that seals, the
@@ -187,13 +204,20 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 3)) decode_kernel(cons
   };
   __half2 new_kv = __halves2half2(__float2half_rn(0.f), __float2half_rn(0.f));
   __half2 old_kv = new_kv;
-  if (do_ring) {
+  if (do_ring || ring_hbm) {
     const size_t o = ((size_t)b * a.hkv + h) * kDim + tid;
     new_kv = __halves2half2(a.k_new[o], a.v_new[o]);
-    if (do_seal) {
-      const __half *er = reinterpret_cast<const __half *>(a.hot) + (((size_t)b * a.hkv + h) * H + rs) * 2 * kDim;
-      old_kv = __halves2half2(er[tid], er[kDim + tid]);
-    }
+  }
+  if (do_seal) {
+    const __half *er = reinterpret_cast<const __half *>(a.hot) + (((size_t)b * a.hkv + h) * H + rs) * 2 * kDim;
+    old_kv = __halves2half2(er[tid], er[kDim + tid]);
+  }
+  if (ring_hbm) {
+    // the new token into the ring in HBM; thread tid writes channel tid of
+    // both rows, after (in program order) its own read of the old occupant
+    __half *grow = reinterpret_cast<__half *>(a.hot) + (((size_t)b * a.hkv + h) * H + rs) * 2 * kDim;
+    grow[tid] = __low2half(new_kv);
+    grow[kDim + tid] = __high2half(new_kv);
   }
   const int n_int4_b = a.quant_bits == 4 ? 0x7fffffff : (a.n_int4 ? a.n_int4[b] : 0);
 
@@ -333,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 3)) decode_kernel(cons
         if (sm.phys[tb] >= 0)
           requant_staged(sm.seal, sm.ring[st], (sm.phys[tb] * a.hkv + h) << lsub, (i0 + tb) < n_int4_b, a, tid);
       } else if (ok) {
-        ring_put(sm.ring[st], rs, new_kv, a, b, h, tid);
+        ring_put(sm.ring[st], rs, new_kv, tid);
       }
     }
     ok = ok && *reinterpret_cast<volatile int *>(&sm.abort_flag) == 0;
@@ -474,18 +498,20 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 3)) decode_kernel(cons
   const int unit = b * a.hkv + h;
   const bool grouped = Sb > kMergeFan;
   const int grp = s / kMergeFan;
-  __threadfence();
+  // arrival: the CTA barrier orders every thread's partial stores before
+  // thread 0's acquire-release increment, which publishes them; the CTA that
+  // completes the count acquires every other CTA's (the merge then reads the
+  // partials through L2, __ldcg)
   __syncthreads();
   if (tid == 0) {
     int32_t *cnt = grouped ? &a.g_counters[(size_t)unit * a.n_groups + grp] : &a.counters[unit];
     const int need = grouped ? min(kMergeFan, Sb - grp * kMergeFan) : Sb;
-    const int last = atomicAdd(cnt, 1) == need - 1;
+    const int last = atomic_add_acq_rel_gpu(cnt, 1) == need - 1;
     if (last) *cnt = 0;  // ready for the next call
     sm.last = last;
   }
   __syncthreads();
   if (!sm.last) return;
-  __threadfence();
   if (!grouped) {
     merge_splits<G>(a.o_part + row0 * S * kDim, kDim, (size_t)S * kDim, a.lse_part + row0 * S, 1, S, Sb,
                     [](int j) { return j; }, warp, lane, a.out + row0 * kDim, a.lse_out ? a.lse_out + row0 : nullptr,
@@ -497,24 +523,23 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 3)) decode_kernel(cons
   merge_splits<G>(a.o_part + (row0 * S + j0) * kDim, kDim, (size_t)S * kDim, a.lse_part + row0 * S + j0, 1, S,
                   min(kMergeFan, Sb - j0), [](int j) { return j; }, warp, lane, nullptr, nullptr,
                   a.g_part + (row0 * NG + grp) * kDim, (size_t)NG * kDim, a.g_lse + row0 * NG + grp, NG);
-  __threadfence();
   __syncthreads();
   if (tid == 0) {
     const int ngb = (Sb + kMergeFan - 1) / kMergeFan;
-    const int last = atomicAdd(&a.counters[unit], 1) == ngb - 1;
+    const int last = atomic_add_acq_rel_gpu(&a.counters[unit], 1) == ngb - 1;
     if (last) a.counters[unit] = 0;
     sm.last = last;
   }
   __syncthreads();
   if (!sm.last) return;
-  __threadfence();
   merge_splits<G>(a.g_part + row0 * NG * kDim, kDim, (size_t)NG * kDim, a.g_lse + row0 * NG, 1, NG,
                   (Sb + kMergeFan - 1) / kMergeFan, [](int j) { return j; }, warp, lane, a.out + row0 * kDim,
                   a.lse_out ? a.lse_out + row0 : nullptr, nullptr, 0, nullptr, 0);
 }
 
-// Largest cluster the decode kernel is launched with (portable size).
-constexpr int kMaxCluster = 8;
+// Largest cluster the decode kernel is launched with (sizes above 8 are
+// non-portable; B200 allows 16).  The split merge reads up to 16 partners.
+constexpr int kMaxCluster = 16;
 
 template <int G, bool kF16, bool kSkip, int kBshift>
 cudaError_t launch_decode_g(const DecodeArgs &a, int batch, bool cluster, cudaStream_t stream) {
@@ -529,6 +554,9 @@ cudaError_t launch_decode_g(const DecodeArgs &a, int batch, bool cluster, cudaSt
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(decode_kernel<G, true, kF16, kSkip, kBshift>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(decode_kernel<G, true, kF16, kSkip, kBshift>,
+                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
     configured_dev_mask |= 1 << dev;
   }
@@ -595,6 +623,52 @@ int decode_occupancy(int group) {
     return 0;
   }
   return n;
+}
+
+// How many clusters of `csize` CTAs of the cluster-merge kernel (plain
+// variant) can be resident on the device at once, for head group `group`
+// (0 on error or when such clusters cannot run).
+template <int G, bool kF16, bool kSkip, int kBshift>
+int decode_active_clusters_g(int csize) {
+  auto kern = decode_kernel<G, true, kF16, kSkip, kBshift>;
+  const size_t smem = sizeof(DecodeSmem<G>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  int n = 0;
+  if (e == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(csize, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+template <bool kF16, bool kSkip, int kBshift>
+int decode_active_clusters(int group, int csize) {
+  switch (group) {
+    case 1: return decode_active_clusters_g<1, kF16, kSkip, kBshift>(csize);
+    case 2: return decode_active_clusters_g<2, kF16, kSkip, kBshift>(csize);
+    case 3: return decode_active_clusters_g<3, kF16, kSkip, kBshift>(csize);
+    case 4: return decode_active_clusters_g<4, kF16, kSkip, kBshift>(csize);
+    case 5: return decode_active_clusters_g<5, kF16, kSkip, kBshift>(csize);
+    case 6: return decode_active_clusters_g<6, kF16, kSkip, kBshift>(csize);
+    case 7: return decode_active_clusters_g<7, kF16, kSkip, kBshift>(csize);
+    case 8: return decode_active_clusters_g<8, kF16, kSkip, kBshift>(csize);
+    default: return 0;
+  }
 }
 
 }  // namespace hyb

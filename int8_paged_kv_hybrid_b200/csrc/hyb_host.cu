@@ -167,16 +167,26 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
   const long long slots = static_cast<long long>(sms) * occ;
   const long long units = static_cast<long long>(d->batch) * d->num_kv_heads;
   const int max_tb = hyb::decode_max_split_blocks();
+  // the hot ring's items, counted in blocks when a sequence is cut into
+  // splits (the kernel uses the same rule, capped at one split's blocks)
+  const long long hot_n = max_seq_len < d->hot_tokens ? max_seq_len : d->hot_tokens;
+  const long long dh = (hot_n + 31) / 32;
+  const long long ipb = d->quant_bits == 0 ? d->block_size / 32 : (d->block_size > hyb::kBlock ? 2 : 1);
+  const long long dhb = (dh + ipb - 1) / ipb;
+  auto n_splits = [&](long long t) {
+    const long long v = (nblk + (dhb < t ? dhb : t) + t - 1) / t;
+    return v < 1 ? 1 : v;
+  };
   long long tb = 0;
   if (split_tokens == 0) {
     // one wave: enough splits of the longest sequence to fill the GPU, no more
     const long long s_wave = slots / units;
     if (s_wave >= 1) {
-      tb = (nblk + s_wave - 1) / s_wave;
+      tb = (nblk + dhb + s_wave - 1) / s_wave;
       if (tb < 1) tb = 1;
       if (tb > max_tb) tb = max_tb;
     }
-    if (tb == 0 || tb > kMultiWaveSplit || units * ((nblk + tb - 1) / tb) > slots) {
+    if (tb == 0 || tb > kMultiWaveSplit || units * n_splits(tb) > slots) {
       // several waves: short splits, so that the CTA scheduler evens out
       // sequences of different lengths and CTAs that run at different speeds
       // (the last CTA placed on an SM gets the fewest issue slots).  Also
@@ -192,12 +202,13 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
     tb = split_tokens / d->block_size;
     if (tb < 1) return HYB_ERR_INVALID_VALUE;
   }
-  long long ns = (nblk + tb - 1) / tb;
-  if (ns < 1) ns = 1;
+  const long long ns = n_splits(tb);
   if (tb > max_tb || ns > 65535) return HYB_ERR_INVALID_VALUE;
-  // clusters only when every split is resident at once: a cluster holds its
-  // CTAs until its slowest split is done
-  p->cluster = units * ns <= slots && ns >= 2 && ns <= hyb::decode_max_cluster();
+  // clusters only when every split is resident at once (a cluster holds its
+  // CTAs until its slowest split is done): every (sequence, kv head)'s
+  // cluster must fit on the GPU together
+  p->cluster = units * ns <= slots && ns >= 2 && ns <= hyb::decode_max_cluster() &&
+               units <= hyb::decode_resident_clusters(group, static_cast<int>(ns));
   p->tb = static_cast<int>(tb);
   p->ns = static_cast<int>(ns);
   return HYB_OK;

@@ -124,6 +124,7 @@ cudaError_t launch_sparse_l2(const SparseArgs &a, int batch, cudaStream_t stream
 int decode_max_split_blocks();
 int decode_ctas_per_sm(int group);
 int decode_max_cluster();
+int decode_resident_clusters(int group, int csize);
 size_t decode_ws_zero_prefix(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens);
 
 }  // namespace hyb

@@ -79,17 +79,28 @@ def test_descriptor_rejections():
     assert hk.load().hyb_check_desc(None) == _lib.HYB_ERR_INVALID_VALUE
 
 
+def _splits(L, st, hot=32, block=64, qbits=8):
+    """Splits of a sequence of L tokens at st tokens per split: the cold
+    blocks plus the hot ring's items counted as blocks (capped at a split)."""
+    tb = st // block
+    nblk = -(-max(0, L - hot) // block)
+    ipb = block // 32 if qbits == 0 else (2 if block == 128 else 1)
+    dh = -(-min(L, hot) // 32)
+    dhb = min(-(-dh // ipb), tb)
+    return max(1, -(-(nblk + dhb) // tb))
+
+
 def test_plan_and_workspace():
     d = _desc(batch=4, maxb=2048, phys=8192)
     st, ns = hk.hyb_decode_plan(d, 131072, 512)
-    assert st == 512 and ns == 256      # ceil((131072 - 32) / 512)
+    assert st == 512 and ns == 257      # ceil((2048 cold blocks + 1 hot item) / 8)
     st, ns = hk.hyb_decode_plan(d, 32768, 512)
-    assert ns == 64                     # the page's 32K context: >= 64 splits at 512 tokens
+    assert ns == 65                     # the page's 32K context: >= 64 splits at 512 tokens
     st, ns = hk.hyb_decode_plan(d, 32, 512)
     assert ns == 1 and hk.hyb_decode_workspace_bytes(d, 32, 512) == 0
     ws = hk.hyb_decode_workspace_bytes(d, 131072, 512)
     rows = 4 * 32
-    assert ws >= rows * 256 * 128 * 4 + rows * 256 * 4
+    assert ws >= rows * 257 * 128 * 4 + rows * 257 * 4
     for bad in (100, -64, 64 * 129):
         with pytest.raises(hk.HybError):
             hk.hyb_decode_plan(d, 4096, bad)
@@ -99,7 +110,7 @@ def test_plan_and_workspace():
     for L in (33, 1000, 2048, 131072):
         st, ns = hk.hyb_decode_plan(d, L, 0)
         assert st % 64 == 0 and 64 <= st <= 8192 and ns >= 1
-        assert ns == max(1, -(-max(0, L - 32) // st))
+        assert ns == _splits(L, st)
     # one wave when every split fits on the GPU at once (4 x 8 units x 16 <= 444)
     assert hk.hyb_decode_plan(d, 2048, 0)[1] >= 8
 
@@ -111,9 +122,9 @@ def test_plan_other_block_and_hot_sizes(block, hot):
     d = _desc(hot=hot, block=block, batch=4, maxb=4096, phys=8192)
     for L in (hot + 1, 1000, 40000):
         st, ns = hk.hyb_decode_plan(d, L, 0)
-        assert st % block == 0 and st >= block and ns == max(1, -(-max(0, L - hot) // st))
+        assert st % block == 0 and st >= block and ns == _splits(L, st, hot, block)
     st, ns = hk.hyb_decode_plan(d, 40000, 4 * block)
-    assert st == 4 * block and ns == -(-(40000 - hot) // st)
+    assert st == 4 * block and ns == _splits(40000, st, hot, block)
     for bad in (block // 2, 3 * block + 8):
         with pytest.raises(hk.HybError):
             hk.hyb_decode_plan(d, 4096, bad)
