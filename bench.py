@@ -45,8 +45,11 @@ SUB_WORKLOADS = (2, 3, 5)  # reported in the same run
 APPEND_WORKLOAD = 3
 PROFILE_JSON = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
 # the profiled kernel's sources (their hash tells whether a capture is current)
-KERNEL_SOURCES = ["decode_kernel.cuh", "decode_dev.cuh", "mma.cuh", "common.cuh", "kernels.cuh"]
+KERNEL_SOURCES = ["decode_kernel.cuh", "decode_persist.cuh", "decode_dev.cuh", "mma.cuh", "common.cuh",
+                  "kernels.cuh"]
 FLUSH_BYTES = 512 << 20   # > 126 MB L2
+DECODE_KERNELS = {"persistent": "hyb::decode_persist_kernel", "split_cta": "hyb::decode_kernel",
+                  "cluster": "hyb::decode_kernel (clusters)"}
 
 
 def parse():
@@ -81,7 +84,16 @@ def parse():
 COLD_KIND = {8: "INT8", 4: "INT4", 0: "FP16"}
 
 
-def workload_config(w, split, ns, qbits=8):
+def split_desc(split, split_len, ns):
+    if split < 0:
+        return ("per sequence: at least %d near-equal splits of <= 32 blocks (the longest sequence: %d splits "
+                "of <= %d tokens)" % (-split, ns, split_len))
+    if split == 0:
+        return "automatic: %d splits of %d tokens" % (ns, split_len)
+    return "%d splits of %d tokens" % (ns, split)
+
+
+def workload_config(w, split, ns, qbits=8, split_len=None):
     lens = w.lens
     cold = COLD_KIND[qbits]
     if qbits == 8 and w.n_int4 is not None:
@@ -100,6 +112,7 @@ def workload_config(w, split, ns, qbits=8):
     return {"workload": what, "batch": int(w.batch), "seq_len": int(lens.max()),
             "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads, "head_dim": 128, "hot_tokens": H,
             "block_size": w.block_size, "quant_bits": qbits, "split_tokens": split, "n_splits": ns,
+            "splits": split_desc(split, split if split_len is None else split_len, ns),
             "step": "hyb_decode_step: append 1 token/seq + split-KV attention, one launch",
             "l2": "flushed between timed steps (512 MB write)",
             "parallelism": "replicas (independent batch per GPU)"}
@@ -370,7 +383,11 @@ def run_config(args, wl, rank, world, local_rank, clocks=None, cpu=True):
     cache, n_last, k_last, v_last, q = build_gpu_state(w, torch, qb, ora)
     if args.lean:
         L += args.warmup + args.steps  # the lean run lets the cache grow one token per step
-    split, ns = cache.plan(L, args.split or w.split_tokens)
+    # split_tokens as asked (negative: at least that many splits per sequence)
+    # and the plan it gives: the longest sequence's split length, its splits
+    split = args.split or w.split_tokens
+    split_len, ns = cache.plan(L, split)
+    launch_kind, launch_ctas, launch_occ = cache.launch_info(L, split)
     # the step's inputs packed in one pinned host buffer (each part 256-byte
     # aligned), moved in one copy per step
     parts = [np.ascontiguousarray(a) for a in (n_last, k_last, v_last, q)]
@@ -481,7 +498,7 @@ def run_config(args, wl, rank, world, local_rank, clocks=None, cpu=True):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": {8: "int8", 4: "int4", 0: "f16"}[qb],
         "data": "synthetic (seeded N(0,1) FP16 K/V/q; caches built by the library's own appends)",
-        "config": workload_config(w, split, ns, qb),
+        "config": workload_config(w, split, ns, qb, split_len),
         "tokens_per_s": round(tokens_s, 1),
         "tokens_per_s_model_equiv": round(tokens_s / layers, 1),
         "kv_bytes_per_step": kvb,
@@ -490,7 +507,8 @@ def run_config(args, wl, rank, world, local_rank, clocks=None, cpu=True):
                      "frac": round(achieved / peak, 4),
                      "traffic": None if traffic is None else int(traffic),
                      "traffic_source": traffic_how,
-                     "kernel": "hyb::decode_kernel (fused append + attention, the step's only launch)",
+                     "kernel": "%s (fused append + attention, the step's only launch; %d CTAs, %d per SM)"
+                               % (DECODE_KERNELS[launch_kind], launch_ctas, launch_occ),
                      "peak_kind": peak_kind,
                      "achieved_bytes": "algorithmic bytes per launch: attention %d + append %d"
                                        % (kvb, stepb - kvb)},
@@ -667,7 +685,9 @@ def run_sparse(args):
     cache.append(torch.from_numpy(n_last).cuda(), torch.from_numpy(k_last).cuda(), torch.from_numpy(v_last).cuda())
     L = int(w.lens.max())
     top_k = hyb_sparse_top_k(L) if args.sparse_top_k < 0 else args.sparse_top_k
-    split = args.split or w.split_tokens
+    # the sparse path takes a fixed split length (512 tokens: >= 64 splits
+    # for every sequence of the long-context workload)
+    split = args.split or (w.split_tokens if w.split_tokens >= 0 else 512)
     qd = torch.from_numpy(q).cuda()
     out = torch.empty((w.batch, w.num_q_heads, 128), dtype=torch.float16, device="cuda")
     lse = torch.empty((w.batch, w.num_q_heads), dtype=torch.float32, device="cuda")

@@ -220,9 +220,45 @@ int hyb_kv_append(const hyb_cache_desc *desc, const int32_t *n_new, int32_t max_
  * HOT) / BLK).  Returns HYB_OK or HYB_ERR_INVALID_VALUE.  The automatic
  * choice depends on the GPU's SM count (device 0 of the current context
  * when none is current).
+ * split_tokens = -n (1 <= n <= 65535) asks for per-sequence splits: a
+ * sequence with nblk_b cold blocks counts c_b = nblk_b + 1 items (the hot
+ * ring as one; c_b = 0 when it is empty) and is cut into
+ * S_b = min(c_b, max(n, ceil(c_b / 32))) splits of near-equal length --
+ * split s takes items [floor(s c_b / S_b), floor((s + 1) c_b / S_b)), the
+ * ring being the last -- so every sequence with at least n blocks gets at
+ * least n splits of at most 32 blocks, as long as the longest allows.  Then
+ * n_splits = S for c = nblk + 1 of max_seq_len, and split_tokens_out is the
+ * longest sequence's split length (ceil(c / n_splits) blocks).  This needs
+ * 64-token INT8/INT4 blocks and batch <= 256 (the persistent kernel); other
+ * caches take the longest sequence's split length for every sequence
+ * (n_splits and split_tokens_out as for split_tokens = that length).
+ * hyb_decode_attn_sparse does not take it (HYB_ERR_INVALID_VALUE).
  */
 int hyb_decode_plan(const hyb_cache_desc *desc, int32_t max_seq_len, int32_t split_tokens,
                     int32_t *split_tokens_out, int32_t *n_splits_out);
+
+/*
+ * Which decode kernel hyb_decode_attn / hyb_decode_step launch for these
+ * arguments (host only; the same plan as hyb_decode_plan):
+ *   HYB_KERNEL_SPLIT_CTA   one CTA per (split, kv head, sequence), splits
+ *                          merged through the workspace by the last to finish;
+ *   HYB_KERNEL_CLUSTER     the same CTAs, the splits of a (sequence, kv head)
+ *                          one thread-block cluster merged in distributed
+ *                          shared memory;
+ *   HYB_KERNEL_PERSISTENT  `ctas` resident CTAs that take the splits as work
+ *                          units from a counter (64-token INT8/INT4 blocks,
+ *                          batch <= 256, splits of at most 32 blocks).
+ * Writes the kernel, the CTAs of the launch and the CTAs one SM holds (the
+ * device's occupancy for that kernel; 0 when no device can be queried).  Any
+ * output pointer may be NULL.  Returns HYB_OK or HYB_ERR_INVALID_VALUE (the
+ * cases hyb_decode_plan rejects).  A benchmark or a scheduler reads it; the
+ * attention calls do not need it.
+ */
+#define HYB_KERNEL_SPLIT_CTA 0
+#define HYB_KERNEL_CLUSTER 1
+#define HYB_KERNEL_PERSISTENT 2
+int hyb_decode_launch_info(const hyb_cache_desc *desc, int32_t max_seq_len, int32_t split_tokens,
+                           int32_t *kernel, int32_t *ctas, int32_t *ctas_per_sm);
 
 /* Bytes of workspace hyb_decode_attn needs for these arguments, or 0 with an
  * invalid descriptor.  It is 0 when each sequence takes one split, or when
@@ -242,7 +278,8 @@ size_t hyb_decode_workspace_bytes(const hyb_cache_desc *desc, int32_t max_seq_le
  *   softmax_scale  finite, usually 1/sqrt(D).
  *   max_seq_len    host upper bound of seq_lens (a larger device value sets
  *            HYB_STATUS_SEQ_LEN and that sequence is skipped).
- *   split_tokens   multiple of BLK, or 0 = automatic (hyb_decode_plan).
+ *   split_tokens   multiple of BLK, 0 = automatic, or -n = at least n splits
+ *            per sequence (hyb_decode_plan).
  *   workspace, workspace_bytes  device scratch of at least
  *            hyb_decode_workspace_bytes() bytes (may be NULL when that is 0),
  *            16-byte aligned.  It must be zero-filled before its first use;

@@ -9,7 +9,7 @@ blocks), the log-sum-exp combine and the INT8 <-> INT4 tier migration.  This
 package is its thin Python binding.
 """
 from ._lib import (  # noqa: F401
-    CacheDesc, HybError, hyb_check_desc, hyb_combine, hyb_decode_attn, hyb_decode_plan,
+    CacheDesc, HybError, hyb_check_desc, hyb_combine, hyb_decode_attn, hyb_decode_plan, hyb_decode_launch_info,
     hyb_decode_attn_sparse, hyb_decode_sparse_workspace_bytes, hyb_decode_step,
     hyb_decode_step_workspace_bytes, hyb_sparse_top_k,
     hyb_decode_workspace_bytes, hyb_kv_append, hyb_kv_migrate, hyb_last_cuda_error,

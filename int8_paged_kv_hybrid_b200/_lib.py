@@ -35,7 +35,7 @@ EXPORTED = (
     "hyb_last_cuda_error", "hyb_version", "hyb_decode_attn_noalloc", "hyb_noalloc_scratch_limit",
     "hyb_kv_migrate", "hyb_migration_threshold_ms", "hyb_migration_decision",
     "hyb_decode_attn_sparse", "hyb_decode_sparse_workspace_bytes", "hyb_decode_sparse_selection",
-    "hyb_sparse_top_k", "hyb_set_wait_limit",
+    "hyb_sparse_top_k", "hyb_set_wait_limit", "hyb_decode_launch_info",
 )
 
 
@@ -87,6 +87,9 @@ def load(path: str = LIB_PATH):
     lib.hyb_decode_plan.argtypes = [D, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
     lib.hyb_decode_workspace_bytes.argtypes = [D, i32, i32]
     lib.hyb_decode_workspace_bytes.restype = sz
+    lib.hyb_decode_launch_info.argtypes = [D, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32),
+                                           ctypes.POINTER(i32)]
+    lib.hyb_decode_launch_info.restype = ctypes.c_int
     lib.hyb_decode_attn.argtypes = [D, P, ctypes.c_float, i32, i32, P, sz, P, P, P]
     lib.hyb_decode_attn_sparse.argtypes = [D, P, ctypes.c_float, i32, i32, i32, P, sz, P, P, P]
     lib.hyb_decode_sparse_workspace_bytes.argtypes = [D, i32, i32]
@@ -153,6 +156,17 @@ def hyb_decode_plan(desc, max_seq_len, split_tokens=0):
     _check(load().hyb_decode_plan(ctypes.byref(desc), int(max_seq_len), int(split_tokens),
                                   ctypes.byref(st), ctypes.byref(ns)), "hyb_decode_plan")
     return st.value, ns.value
+
+
+KERNEL_NAMES = {0: "split_cta", 1: "cluster", 2: "persistent"}
+
+
+def hyb_decode_launch_info(desc, max_seq_len, split_tokens=0):
+    """(kernel name, CTAs of the launch, CTAs per SM) of the decode launch."""
+    k, c, o = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check(load().hyb_decode_launch_info(ctypes.byref(desc), int(max_seq_len), int(split_tokens), ctypes.byref(k),
+                                         ctypes.byref(c), ctypes.byref(o)), "hyb_decode_launch_info")
+    return KERNEL_NAMES[k.value], c.value, o.value
 
 
 def hyb_decode_workspace_bytes(desc, max_seq_len, split_tokens=0) -> int:

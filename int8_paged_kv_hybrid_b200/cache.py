@@ -86,6 +86,10 @@ class HybridKVCache:
     def plan(self, max_seq_len, split_tokens=0):
         return _lib.hyb_decode_plan(self.desc, max_seq_len, split_tokens)
 
+    def launch_info(self, max_seq_len, split_tokens=0):
+        """(kernel, CTAs, CTAs per SM) of the decode launch for these arguments."""
+        return _lib.hyb_decode_launch_info(self.desc, max_seq_len, split_tokens)
+
     def workspace(self, max_seq_len, split_tokens=0):
         import torch
         n = _lib.hyb_decode_workspace_bytes(self.desc, max_seq_len, split_tokens)

@@ -45,6 +45,15 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Barrier of the threads that run the per-item arithmetic: the whole CTA
+// (kNamed false), or the 128 consumer threads of a warp-specialized CTA
+// (named barrier 1; the producer warp never takes part).
+template <bool kNamed>
+__device__ __forceinline__ void work_sync() {
+  if constexpr (kNamed) asm volatile("bar.sync 1, 128;" ::: "memory");
+  else __syncthreads();
+}
+
 // Barrier over all threads of all CTAs of the cluster (release / acquire).
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile(
@@ -85,6 +94,7 @@ struct SealScratch {
 // requant_staged.  Same arithmetic as
 // hyb_kv_append: absmax scale, a grown scale re-quantizes the codes already
 // in the block, RNE codes.  Called by the whole CTA.
+template <bool kNamed = false>
 __device__ __forceinline__ void fused_seal(SealScratch &ss, uint8_t *tile_st, float2 *scl_tail, int tile_tail,
                                            bool int4_tail, const DecodeArgs &a, int L_old, bool do_seal, int tid,
                                            int warp, int lane) {
@@ -124,7 +134,7 @@ __device__ __forceinline__ void fused_seal(SealScratch &ss, uint8_t *tile_st, fl
       ss.seal_rq[kv] = rq;
     }
   }
-  __syncthreads();
+  work_sync<kNamed>();
   if (tid == 0) *scl_tail = make_float2(ss.seal_s[0], ss.seal_s[1]);  // attention uses these
   // codes already in the tail block, under a grown scale
 #pragma unroll
@@ -134,7 +144,7 @@ __device__ __forceinline__ void fused_seal(SealScratch &ss, uint8_t *tile_st, fl
     const int nw = requant_nwords(kv, int4, slot);
     for (int w = tid; w < nw; w += kThreads) w32[w] = requant_word(w32[w], w, kv, int4, slot, ss.rqt[kv]);
   }
-  __syncthreads();
+  work_sync<kNamed>();
   const int c = tid;  // channel
   {
     // the evicted token's codes into slot `slot`
@@ -158,7 +168,7 @@ __device__ __forceinline__ void fused_seal(SealScratch &ss, uint8_t *tile_st, fl
                        : static_cast<uint8_t>((*byte & 0xf0) | (cv & 0xf));
     }
   }
-  __syncthreads();
+  work_sync<kNamed>();
   {
     // write back what changed in the tail block: scales, then the whole tile
     // if its codes were re-quantized, else the sealed token's codes
@@ -189,13 +199,14 @@ __device__ __forceinline__ void fused_seal(SealScratch &ss, uint8_t *tile_st, fl
     }
   }
   fence_proxy_async_smem();  // the staged tile is refilled by bulk copies later
-  __syncthreads();
+  work_sync<kNamed>();
 }
 
 // Fused decode step, seal half for FP16 cold blocks (quantization_bits 0):
 // the evicted token's rows (ss.erow) move unchanged to slot e % 64 of the
 // tail block -- in its staged half-block item (row_st, rows slot % 32 at the
 // staging pitch kRowStride) and in the cache.  Thread tid moves channel tid of both rows.
+template <bool kNamed = false>
 __device__ __forceinline__ void fused_seal_fp16(const SealScratch &ss, uint8_t *row_st, int tile_tail,
                                                 const DecodeArgs &a, int L_old, bool do_seal, int tid) {
   if (!do_seal || tile_tail < 0) return;
@@ -210,7 +221,7 @@ __device__ __forceinline__ void fused_seal_fp16(const SealScratch &ss, uint8_t *
   grow[c] = k_old;
   grow[kDim + c] = v_old;
   fence_proxy_async_smem();
-  __syncthreads();
+  work_sync<kNamed>();
 }
 
 // Fused decode step, 128-token blocks: the seal landed in the block's second
@@ -218,6 +229,7 @@ __device__ __forceinline__ void fused_seal_fp16(const SealScratch &ss, uint8_t *
 // slots, staged in tile_st) are re-quantized with the seal's tables, for this
 // attention and in the cache (sub-block pair index pair0 = (physical block *
 // Hkv + kv head) * 2).  Called by the whole CTA after fused_seal.
+template <bool kNamed = false>
 __device__ __forceinline__ void requant_staged(const SealScratch &ss, uint8_t *tile_st, int pair0, bool int4,
                                                const DecodeArgs &a, int tid) {
 #pragma unroll
@@ -227,7 +239,7 @@ __device__ __forceinline__ void requant_staged(const SealScratch &ss, uint8_t *t
     const int nw = requant_nwords(kv, int4, kBlock);
     for (int w = tid; w < nw; w += kThreads) w32[w] = requant_word(w32[w], w, kv, int4, kBlock, ss.rqt[kv]);
   }
-  __syncthreads();
+  work_sync<kNamed>();
   uint8_t *g = a.cold + (size_t)pair0 * kTilePairBytes;
 #pragma unroll
   for (int kv = 0; kv < 2; kv++) {
@@ -237,20 +249,21 @@ __device__ __forceinline__ void requant_staged(const SealScratch &ss, uint8_t *t
       reinterpret_cast<uint4 *>(g + kv * kTileBytes)[v] = reinterpret_cast<const uint4 *>(tile_st + kv * kTileBytes)[v];
   }
   fence_proxy_async_smem();
-  __syncthreads();
+  work_sync<kNamed>();
 }
 
 // Fused decode step, ring half: the new token goes to ring slot rs = L_old %
-// hot -- row rs % 32 of its staged hot item (item_st, pitch kRowStride), for
+// hot -- row rs % 32 of its staged hot item (item_st, row pitch kPitch), for
 // this attention (the kernel writes it into the ring in HBM separately).
 // Thread tid writes channel tid of both rows.
+template <bool kNamed = false, int kPitch = kRowStride>
 __device__ __forceinline__ void ring_put(uint8_t *item_st, int rs, __half2 new_kv, int tid) {
   const int c = tid;
-  __half *srow = reinterpret_cast<__half *>(item_st + (rs % kItemRows) * kRowStride);
+  __half *srow = reinterpret_cast<__half *>(item_st + (rs % kItemRows) * kPitch);
   srow[c] = __low2half(new_kv);
   srow[kDim + c] = __high2half(new_kv);
   fence_proxy_async_smem();
-  __syncthreads();
+  work_sync<kNamed>();
 }
 
 // Log-sum-exp merge of n partial results of the G query heads of one kv head
@@ -258,23 +271,23 @@ __device__ __forceinline__ void ring_put(uint8_t *item_st, int rs, __half2 new_k
 // array of partials: head hh's 128 FP32 at o + slot * o_js + hh * o_hs, its
 // log2-sum-exp at lse + slot * l_js + hh * l_hs (-inf: empty, output 0).
 // Warp w merges heads w, w + 4, ...; lane l channels 4l..4l+3; the loads of
-// kMergeFan partials are issued together.  Writes the FP16 output rows
+// kFan partials are issued together.  Writes the FP16 output rows
 // [G][128] at out (and the natural-log lse at lse_out), or, when out is null,
 // the merged FP32 rows at p_o (head stride p_hs floats) with their
 // log2-sum-exp at p_lse (head stride p_lhs).
-template <int G, typename SlotOf>
+template <int G, typename SlotOf, int kFan = kMergeFan>
 __device__ __forceinline__ void merge_splits(const float *o, size_t o_js, size_t o_hs, const float *lse, size_t l_js,
                                              size_t l_hs, int n, SlotOf slot_of, int warp, int lane, __half *out,
                                              float *lse_out, float *p_o, size_t p_hs, float *p_lse, size_t p_lhs) {
   for (int hh = warp; hh < G; hh += kWarps) {
     float m = -INFINITY, den = 0.f;
     float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = 0; j0 < n; j0 += kMergeFan) {
-      const int nj = min(kMergeFan, n - j0);
+    for (int j0 = 0; j0 < n; j0 += kFan) {
+      const int nj = min(kFan, n - j0);
       const long long my_slot = lane < nj ? static_cast<long long>(slot_of(j0 + lane)) : 0;
-      float4 ov[kMergeFan];
+      float4 ov[kFan];
 #pragma unroll
-      for (int j = 0; j < kMergeFan; j++) {
+      for (int j = 0; j < kFan; j++) {
         const long long sj = __shfl_sync(0xffffffffu, my_slot, j);
         ov[j] = j < nj ? __ldcg(reinterpret_cast<const float4 *>(o + sj * o_js + hh * o_hs + 4 * lane))
                        : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -295,7 +308,7 @@ __device__ __forceinline__ void merge_splits(const float *o, size_t o_js, size_t
       for (int d = 16; d > 0; d >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, d);
       den += ws;
 #pragma unroll
-      for (int j = 0; j < kMergeFan; j++) {
+      for (int j = 0; j < kFan; j++) {
         const float wj = __shfl_sync(0xffffffffu, wl, j);
         num.x = fmaf(wj, ov[j].x, num.x);
         num.y = fmaf(wj, ov[j].y, num.y);
@@ -377,7 +390,7 @@ __device__ __forceinline__ float group_update(float mx, float S, float &m_run, f
 // fixed-point digits qd[h][0..2][c] (hi, mid, lo), its FP16 copy qh[h][c] and
 // the fixed-point step sq[h] = max|q_h| / kQFix; heads >= G are zero.
 // qmax_w [kWarps][NH] is scratch.  Two CTA barriers.
-template <int G, int NH>
+template <int G, int NH, bool kNamed = false>
 __device__ __forceinline__ void prepare_q(const float (&qv)[G], int8_t (*qd)[3][kDim], __half (*qh)[kDim],
                                           float *sq, float (*qmax_w)[NH], int warp, int lane, int tid) {
 #pragma unroll
@@ -387,7 +400,7 @@ __device__ __forceinline__ void prepare_q(const float (&qv)[G], int8_t (*qd)[3][
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (lane == 0) qmax_w[warp][j] = m;
   }
-  __syncthreads();
+  work_sync<kNamed>();
 #pragma unroll
   for (int j = 0; j < NH; j++) {
     int8_t d0 = 0, d1 = 0, d2 = 0;
@@ -414,7 +427,7 @@ __device__ __forceinline__ void prepare_q(const float (&qv)[G], int8_t (*qd)[3][
     qd[j][2][tid] = d2;
     qh[j][tid] = hv;
   }
-  __syncthreads();
+  work_sync<kNamed>();
 }
 
 // The QK A fragments of this lane (score layout).  Rows of the 16 x 32 A
@@ -573,21 +586,22 @@ __device__ __forceinline__ void cold_item(const uint8_t *stage, int nvalid, int 
   }
 }
 
-// nrow FP16 rows (K row, V row) staged at `stage` with pitch kRowStride --
-// the hot ring, or half of an FP16 cold block -- for one warp: rows 8w ..
+// nrow FP16 rows (K row, V row) staged at `stage` with pitch kPitch (kRowStride,
+// 16 bytes of padding, spreads ldmatrix rows over the banks) -- the hot ring, or
+// half of an FP16 cold block -- for one warp: rows 8w ..
 // 8w + 7 (rows >= nrow masked; their V is read from the zero row at
 // zero_addr).  QK: mma m16n8k16 f16 (FP32 accumulation) of the FP16 q (A
 // rows g: head g/2, rows g + 8: head 4 + g/2) with the K rows (ldmatrix);
 // weights 2^(z - mx) relative to the 8-row group's maximum, in FP16; P.V: mma
 // m16n8k8 f16 of the V rows (ldmatrix.trans) with B columns 2i = head i's
 // weights, 2i + 1 = 0, so lane (g, t) gets head t's sums.
-template <int NT>
+template <int NT, int kPitch = kRowStride>
 __device__ __forceinline__ void hot_item(const uint8_t *stage, int nrow, int warp, int lane, int g, int t,
                                          const __half (*qh)[kDim], float qk_scale, uint32_t zero_addr,
                                          WarpState<NT> &st) {
   const int nv = nrow - 8 * warp;
   if (nv <= 0) return;
-  const uint32_t row0 = smem_addr(stage) + (8 * warp + (lane & 7)) * kRowStride;
+  const uint32_t row0 = smem_addr(stage) + (8 * warp + (lane & 7)) * kPitch;
   float c[4] = {0.f, 0.f, 0.f, 0.f};
   const __half *q0 = qh[g >> 1];
   const __half *q1 = qh[NT > 1 ? 4 + (g >> 1) : 0];
@@ -650,7 +664,7 @@ __device__ __forceinline__ void hot_item(const uint8_t *stage, int nrow, int war
 // and 0 when empty).  mbuf: FP32 [kWarps][4 * NT][kMbufPitch], mrun / lrun
 // [kWarps][4 * NT] in shared memory.  Two CTA barriers; on return mbuf may be
 // reused.
-template <int G, int NT>
+template <int G, int NT, bool kNamed = false>
 __device__ __forceinline__ void merge_warps(float *mbuf, float (*mrun)[4 * NT], float (*lrun)[4 * NT],
                                             const WarpState<NT> &st, int warp, int lane, int tid, float (&o_s)[G],
                                             float (&lse2_s)[G]) {
@@ -668,7 +682,7 @@ __device__ __forceinline__ void merge_warps(float *mbuf, float (*mrun)[4 * NT], 
       lrun[warp][4 * nt + t] = st.l_run[nt];
     }
   }
-  __syncthreads();
+  work_sync<kNamed>();
 #pragma unroll
   for (int hh = 0; hh < G; hh++) {
     o_s[hh] = 0.f;
@@ -690,7 +704,7 @@ __device__ __forceinline__ void merge_warps(float *mbuf, float (*mrun)[4 * NT], 
       lse2_s[hh] = mm + __log2f(den);
     }
   }
-  __syncthreads();
+  work_sync<kNamed>();
 }
 
 }  // namespace hyb

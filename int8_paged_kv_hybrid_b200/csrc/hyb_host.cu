@@ -148,7 +148,10 @@ constexpr int kMultiWaveSplit = 16;
 // run in several waves, merged through the workspace.
 struct Plan {
   bool cluster;  // clusters of ns CTAs (split merge in distributed shared memory)
-  int tb;        // cold blocks per split
+  bool persist;  // the persistent kernel: `ctas` CTAs take the splits as work units
+  int ctas;
+  int tb;        // cold blocks per split (per-sequence splits: the longest sequence's)
+  int per_seq;   // > 0: per-sequence splits, at least this many per sequence
   int ns;        // splits per (sequence, kv head), at most
 };
 
@@ -177,6 +180,30 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
     const long long v = (nblk + (dhb < t ? dhb : t) + t - 1) / t;
     return v < 1 ? 1 : v;
   };
+  p->per_seq = 0;
+  if (split_tokens < 0) {
+    // per-sequence splits (per_seq_splits): the persistent kernel only; where
+    // it cannot run, every sequence takes the longest one's split length
+    const long long n = -static_cast<long long>(split_tokens);
+    if (n > 65535) return HYB_ERR_INVALID_VALUE;
+    const long long c = nblk + (max_seq_len > 0 ? 1 : 0);
+    const long long ns = hyb::per_seq_splits(c, n);
+    const long long tb = c > 0 ? (c + ns - 1) / ns : 1;
+    if (d->block_size == hyb::kBlock && d->quant_bits != 0 && d->batch <= hyb::kPMaxBatch) {
+      int pocc = hyb::decode_persist_ctas_per_sm(group);
+      if (pocc <= 0) pocc = group <= 4 ? 3 : 2;  // no GPU to ask: the compiled kernel's occupancy
+      long long ctas = static_cast<long long>(sms) * pocc;
+      if (ctas > units * ns) ctas = units * ns;
+      p->cluster = false;
+      p->persist = true;
+      p->ctas = static_cast<int>(ctas);
+      p->per_seq = static_cast<int>(n);
+      p->tb = static_cast<int>(tb);
+      p->ns = static_cast<int>(ns);
+      return HYB_OK;
+    }
+    split_tokens = static_cast<int32_t>(tb * d->block_size);
+  }
   long long tb = 0;
   if (split_tokens == 0) {
     // one wave: enough splits of the longest sequence to fill the GPU, no more
@@ -198,7 +225,7 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
       if (tb > nblk) tb = nblk > 0 ? nblk : 1;
     }
   } else {
-    if (split_tokens < 0 || split_tokens % d->block_size != 0) return HYB_ERR_INVALID_VALUE;
+    if (split_tokens % d->block_size != 0) return HYB_ERR_INVALID_VALUE;
     tb = split_tokens / d->block_size;
     if (tb < 1) return HYB_ERR_INVALID_VALUE;
   }
@@ -209,6 +236,20 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
   // cluster must fit on the GPU together
   p->cluster = units * ns <= slots && ns >= 2 && ns <= hyb::decode_max_cluster() &&
                units <= hyb::decode_resident_clusters(group, static_cast<int>(ns));
+  // several waves of splits: the persistent kernel, whose CTAs stay resident
+  // and stream the splits back to back (64-token INT8/INT4 blocks, splits of
+  // up to kPMaxSplitBlocks blocks, batches of up to kPMaxBatch sequences)
+  p->persist = false;
+  p->ctas = 0;
+  if (!p->cluster && units * ns > slots && d->block_size == hyb::kBlock && d->quant_bits != 0 &&
+      tb <= hyb::kPMaxSplitBlocks && d->batch <= hyb::kPMaxBatch) {
+    int pocc = hyb::decode_persist_ctas_per_sm(group);
+    if (pocc <= 0) pocc = group <= 4 ? 3 : 2;  // no GPU to ask: the compiled kernel's occupancy
+    long long c = static_cast<long long>(sms) * pocc;
+    if (c > units * ns) c = units * ns;
+    p->persist = true;
+    p->ctas = static_cast<int>(c);
+  }
   p->tb = static_cast<int>(tb);
   p->ns = static_cast<int>(ns);
   return HYB_OK;
@@ -223,16 +264,20 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
 // [batch][Hq][ng].  Each part starts on a 256-byte boundary; the counters
 // come first.
 struct WsLayout {
-  size_t seq_cnt, counters, g_counters, o_part, lse_part, g_part, g_lse, total;
+  size_t seq_cnt, unit_ctr, counters, g_counters, o_part, lse_part, g_part, g_lse, total;
   int n_groups;
 };
 
 WsLayout ws_layout(const hyb_cache_desc *d, const Plan &pl, bool step) {
-  WsLayout w{0, 0, 0, 0, 0, 0, 0, 0, 0};
+  WsLayout w{0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
   size_t off = 0;
   if (step) {
     w.seq_cnt = 0;
     off = round_up(static_cast<size_t>(d->batch) * sizeof(int32_t), kWsAlign);
+  }
+  if (pl.persist) {
+    w.unit_ctr = off;
+    off += kWsAlign;
   }
   const size_t rows = static_cast<size_t>(d->batch) * d->num_q_heads;
   const size_t units = static_cast<size_t>(d->batch) * d->num_kv_heads;
@@ -265,7 +310,7 @@ size_t decode_ws_zero_prefix(const hyb_cache_desc *d, int32_t max_seq_len, int32
   Plan pl;
   if (make_plan(d, max_seq_len, split_tokens, &pl) != HYB_OK) return 0;
   const WsLayout w = ws_layout(d, pl, false);
-  return w.total > 0 ? w.o_part : 0;
+  return w.o_part > 0 ? w.o_part : w.total;  // the counters come first
 }
 }  // namespace hyb
 
@@ -278,6 +323,20 @@ int hyb_decode_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_
   if (rc != HYB_OK) return rc;
   if (split_tokens_out) *split_tokens_out = pl.tb * d->block_size;
   if (n_splits_out) *n_splits_out = pl.ns;
+  return HYB_OK;
+}
+
+int hyb_decode_launch_info(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens, int32_t *kernel,
+                           int32_t *ctas, int32_t *ctas_per_sm) {
+  Plan pl;
+  const int rc = make_plan(d, max_seq_len, split_tokens, &pl);
+  if (rc != HYB_OK) return rc;
+  const int group = d->num_q_heads / d->num_kv_heads;
+  const int units = d->batch * d->num_kv_heads;
+  if (kernel) *kernel = pl.persist ? HYB_KERNEL_PERSISTENT : (pl.cluster ? HYB_KERNEL_CLUSTER : HYB_KERNEL_SPLIT_CTA);
+  if (ctas) *ctas = pl.persist ? pl.ctas : units * pl.ns;
+  if (ctas_per_sm)
+    *ctas_per_sm = pl.persist ? hyb::decode_persist_ctas_per_sm(group) : hyb::decode_ctas_per_sm(group);
   return HYB_OK;
 }
 
@@ -342,9 +401,14 @@ static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_s
   a.l2_skip = l2_skip ? 1 : 0;
   const long long wait = g_wait_cycles.load(std::memory_order_relaxed);
   a.wait_cycles = wait > 0 ? wait : hyb::kDefaultWaitCycles;
+  a.batch = d->batch;
+  const bool persist = pl.persist && !l2_skip;
+  a.unit_ctr = pl.persist ? reinterpret_cast<int32_t *>(ws + wl.unit_ctr) : nullptr;
+  a.min_splits = pl.per_seq;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int group = d->num_q_heads / d->num_kv_heads;
-  const cudaError_t e = hyb::launch_decode(a, group, d->batch, pl.cluster, s);
+  const cudaError_t e = persist ? hyb::launch_decode_persist(a, group, d->batch, pl.ctas, s)
+                                : hyb::launch_decode(a, group, d->batch, pl.cluster, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return HYB_OK;
 }
@@ -366,6 +430,7 @@ struct SparseWs {
 };
 
 static int sparse_ws(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens, SparseWs *w) {
+  if (split_tokens < 0) return HYB_ERR_INVALID_VALUE;  // per-sequence splits: dense calls only
   Plan pl;
   const int rc = make_plan(d, max_seq_len, split_tokens, &pl);
   if (rc != HYB_OK) return rc;

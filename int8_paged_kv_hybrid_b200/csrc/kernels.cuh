@@ -63,7 +63,34 @@ struct DecodeArgs {
   int l2_skip;
   // limit (SM cycles) of the copy pipeline's bounded waits
   long long wait_cycles;
+  // persistent kernel: [0] work-unit counter, [1] exit counter of the CTAs
+  // (zero between calls; the last CTA to exit resets both) and the batch
+  int32_t *unit_ctr;
+  int batch;
+  // persistent kernel: > 0 = per-sequence splits (per_seq_splits), at least
+  // this many per sequence; 0 = runs of split_blocks blocks
+  int min_splits;
 };
+
+// Persistent decode kernel limits: blocks per split (one block-table entry
+// per producer lane) and sequences per call (their lengths are staged in
+// shared memory).
+constexpr int kPMaxSplitBlocks = 32;
+
+// Per-sequence splits: a sequence of nblk cold blocks and a non-empty hot
+// ring counts c = nblk + 1 items (the ring as one), and is cut into
+// per_seq_splits(c, n) splits of near-equal length -- split s covers items
+// [s * c / S, (s + 1) * c / S) (floor), the ring being the last item -- at
+// least n of them (one per item when c < n), at most kPMaxSplitBlocks items
+// each.  Non-decreasing in c.
+__host__ __device__ inline int per_seq_splits(long long c, long long n) {
+  if (c <= 0) return 1;
+  long long s = (c + kPMaxSplitBlocks - 1) / kPMaxSplitBlocks;
+  if (s < n) s = n;
+  if (s > c) s = c;
+  return static_cast<int>(s);
+}
+constexpr int kPMaxBatch = 256;
 
 struct MigrateArgs {
   uint8_t *cold;              // [num_phys][Hkv][2][8192]
@@ -118,6 +145,8 @@ constexpr long long kDefaultWaitCycles = 1ll << 31;
 
 cudaError_t launch_append(const AppendArgs &a, int batch, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream);
+cudaError_t launch_decode_persist(const DecodeArgs &a, int group, int batch, int ctas, cudaStream_t stream);
+int decode_persist_ctas_per_sm(int group);
 cudaError_t launch_migrate(const MigrateArgs &a, int batch, cudaStream_t stream);
 cudaError_t launch_combine(const CombineArgs &a, int rows, cudaStream_t stream);
 cudaError_t launch_sparse_l2(const SparseArgs &a, int batch, cudaStream_t stream);

@@ -148,7 +148,7 @@ def make_workload(idx: int, scale_down: int = 1, seed_offset: int = 0) -> Worklo
         sm, qstd = 1.0 / math.sqrt(d), 1.0
         nblk = np.array([cold_blocks_for(int(L)) for L in lens])
         pool = int(nblk.sum())
-        split = max(64, (512 // scale_down) // 64 * 64)
+        split = -64  # per-sequence splits: at least 64 for every sequence
         sched_kind = "chunk"
     elif idx == 5:
         # Qwen2-7B mixed serving load, batch 128: 50% L in [64,512],

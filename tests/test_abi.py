@@ -101,7 +101,7 @@ def test_plan_and_workspace():
     ws = hk.hyb_decode_workspace_bytes(d, 131072, 512)
     rows = 4 * 32
     assert ws >= rows * 257 * 128 * 4 + rows * 257 * 4
-    for bad in (100, -64, 64 * 129):
+    for bad in (100, -65536, 64 * 129):
         with pytest.raises(hk.HybError):
             hk.hyb_decode_plan(d, 4096, bad)
     with pytest.raises(hk.HybError):
@@ -113,6 +113,70 @@ def test_plan_and_workspace():
         assert ns == _splits(L, st)
     # one wave when every split fits on the GPU at once (4 x 8 units x 16 <= 444)
     assert hk.hyb_decode_plan(d, 2048, 0)[1] >= 8
+
+
+def _per_seq_splits(c, n):
+    """Splits of a sequence of c items (cold blocks + 1 for the hot ring) when
+    at least n per sequence are asked for: near-equal runs of <= 32 items."""
+    if c <= 0:
+        return 1
+    return min(c, max(n, -(-c // 32)))
+
+
+def test_plan_per_sequence_splits():
+    """split_tokens = -n: every sequence cut into at least n near-equal splits
+    (one per item when it has fewer), none longer than 32 blocks."""
+    d = _desc(batch=4, maxb=2048, phys=8192)
+    st, ns = hk.hyb_decode_plan(d, 131072, -64)
+    assert (st, ns) == (32 * 64, 65)    # 2048 cold blocks + the ring = 2049 items
+    st, ns = hk.hyb_decode_plan(d, 32768, -64)
+    assert (st, ns) == (9 * 64, 64)     # 513 items: runs of 8 or 9
+    assert hk.hyb_decode_plan(d, 20, -64) == (64, 1)
+    assert hk.hyb_decode_plan(d, 0, -3) == (64, 1)
+    for L in (33, 100, 1000, 5000, 131072):
+        nblk = -(-max(0, L - 32) // 64)
+        assert hk.hyb_decode_plan(d, L, -5)[1] == _per_seq_splits(nblk + 1, 5)
+    # the split ranges the kernel uses: every item once, runs of 1..32, at
+    # least min(n, c) of them, and never more splits for a shorter sequence
+    for n in (1, 3, 64, 200):
+        prev = 1
+        for c in range(0, 7000, 3):
+            S = _per_seq_splits(c, n)
+            assert S >= prev
+            prev = S
+            if c == 0:
+                assert S == 1
+                continue
+            edges = [s * c // S for s in range(S + 1)]
+            assert edges[0] == 0 and edges[-1] == c
+            assert all(1 <= edges[i + 1] - edges[i] <= 32 for i in range(S))
+            assert S >= min(n, c)
+    ws = hk.hyb_decode_workspace_bytes(d, 131072, -64)
+    assert ws >= 4 * 32 * 65 * 128 * 4
+    # caches the persistent kernel does not take (FP16 cold blocks): every
+    # sequence takes the longest one's split length
+    d0 = _desc(batch=4, maxb=2048, phys=8192, qbits=0)
+    st, ns = hk.hyb_decode_plan(d0, 32768, -64)
+    assert st == 9 * 64 and ns == _splits(32768, st, qbits=0)
+    # the sparse path takes no per-sequence splits
+    assert hk.hyb_decode_sparse_workspace_bytes(d, 32768, -64) == 0
+
+
+def test_launch_info():
+    """The kernel a plan launches: per-sequence splits and several waves of
+    splits take the persistent kernel, one wave of a few splits the
+    one-CTA-per-split kernel; FP16 cold blocks never the persistent one."""
+    d = _desc(batch=4, maxb=2048, phys=8192)
+    kern, ctas, occ = hk.hyb_decode_launch_info(d, 131072, -64)
+    assert kern == "persistent" and 1 <= ctas <= 4 * 8 * 65 and occ >= 0
+    kern, ctas, _ = hk.hyb_decode_launch_info(d, 131072, 512)
+    assert kern == "persistent" and ctas <= 4 * 8 * 257
+    kern, ctas, _ = hk.hyb_decode_launch_info(d, 100, 64)
+    assert kern == "split_cta" and ctas == 4 * 8 * hk.hyb_decode_plan(d, 100, 64)[1]
+    d0 = _desc(batch=4, maxb=2048, phys=8192, qbits=0)
+    assert hk.hyb_decode_launch_info(d0, 131072, -64)[0] != "persistent"
+    with pytest.raises(hk.HybError):
+        hk.hyb_decode_launch_info(d, 4096, 100)
 
 
 @pytest.mark.parametrize("block,hot", [(32, 16), (128, 64), (64, 128)])
@@ -158,7 +222,7 @@ def test_kv_bytes_formula():
 
 def test_workload_shapes():
     w = synth.make_workload(4)
-    assert list(w.lens) == [32768, 32768, 131072, 131072] and w.split_tokens == 512
+    assert list(w.lens) == [32768, 32768, 131072, 131072] and w.split_tokens == -64
     w5 = synth.make_workload(5)
     assert w5.num_q_heads == 28 and w5.num_kv_heads == 4 and w5.batch == 128
     nb = w5.cold_blocks()

@@ -14,7 +14,7 @@ SMALL_LENS = [0, 1, 5, 31, 32, 33, 64, 95, 96, 97, 130, 255, 1000, 2047, 3001]
 
 
 @pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 4), (32, 8), (28, 4), (16, 2)])
-@pytest.mark.parametrize("split", [0, 64, 192])
+@pytest.mark.parametrize("split", [0, 64, 192, -3, -16])
 def test_small_parity(hq, hkv, split):
     w = synth.custom_workload("small", SMALL_LENS, hq, hkv, seed=hq * 31 + hkv, max_step=64)
     cache, ora = make_pair(w)
@@ -33,7 +33,7 @@ def test_int4_parity(qbits, int4):
     cache, ora = make_pair(w, quant_bits=qbits)
     replay(w, cache, ora)
     assert_cache_equal(w, cache, ora)
-    for split in (0, 128):
+    for split in (0, 128, -5):
         got, lse, ref, ref_lse = decode_both(w, cache, ora, split_tokens=split)
         assert_decode_close(w, got, lse, ref, ref_lse, what="int4 split=%d" % split)
 
@@ -53,7 +53,7 @@ def test_fp16_cold_parity(hq, hkv, split):
 
 
 @pytest.mark.parametrize("hot", [16, 64, 128])
-@pytest.mark.parametrize("split", [0, 64])
+@pytest.mark.parametrize("split", [0, 64, -7])
 def test_hot_sizes_parity(hot, split):
     """hot_tokens 16 / 64 / 128: up to four 32-row hot items per sequence."""
     lens = [0, 1, 5, hot - 1, hot, hot + 1, hot + 64, 700, 2100]
