@@ -20,10 +20,13 @@
 //    point, the items (cold_item / hot_item), the fused append where the
 //    unit has it, then the unit's epilogue -- the warp merge and the split
 //    merge through the workspace -- while the producer keeps the ring full.
-// The ring has 4 stages of 16 KB for G <= 4 (3 CTAs per SM), 5 above (2 per
-// SM): with a copy latency of ~1.5 us under load and ~0.5 us of arithmetic
-// per item and CTA, 3 stages left the consumers waiting on most items.  A
-// stage holds one tile pair, or 32 hot rows at a 512-byte pitch.
+// The ring has 4 stages of 16 KB for G <= 4: with copies landing ~2.5 us
+// after issue under load and ~0.6 us of arithmetic per item and CTA, 3
+// stages left the consumers waiting on most items.  Above G = 4 an item
+// takes twice the arithmetic and 3 stages cover the latency; 3 CTAs per SM
+// either way (128 registers: 3 CTAs of 5 warps put 4 warps on some SM
+// sub-partitions, whose register file holds 16 K).  A stage holds one tile
+// pair, or 32 hot rows at a 512-byte pitch.
 // The consumers synchronise among themselves with named barriers 1 (all
 // four) and 2..4 (pairs, for the warp merge); the producer takes part in no
 // CTA barrier after the start.  Every wait is bounded; after a timeout the
@@ -45,8 +48,8 @@ template <int G>
 struct PersistCfg {
   static constexpr int NT = head_quads<G>();
   static constexpr int NH = 4 * NT;
-  static constexpr int kStages = G <= 4 ? 4 : 5;
-  static constexpr int kCtasPerSm = G <= 4 ? 3 : 2;
+  static constexpr int kStages = G <= 4 ? 4 : 3;
+  static constexpr int kCtasPerSm = 3;
 };
 
 // One work unit as the producer hands it to the consumers.

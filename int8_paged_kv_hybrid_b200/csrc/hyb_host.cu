@@ -180,6 +180,9 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
     const long long v = (nblk + (dhb < t ? dhb : t) + t - 1) / t;
     return v < 1 ? 1 : v;
   };
+  // caches the persistent kernel takes (64-token INT8/INT4 blocks, batch
+  // <= 256 sequences)
+  const bool persist_ok = d->block_size == hyb::kBlock && d->quant_bits != 0 && d->batch <= hyb::kPMaxBatch;
   p->per_seq = 0;
   if (split_tokens < 0) {
     // per-sequence splits (per_seq_splits): the persistent kernel only; where
@@ -189,9 +192,9 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
     const long long c = nblk + (max_seq_len > 0 ? 1 : 0);
     const long long ns = hyb::per_seq_splits(c, n);
     const long long tb = c > 0 ? (c + ns - 1) / ns : 1;
-    if (d->block_size == hyb::kBlock && d->quant_bits != 0 && d->batch <= hyb::kPMaxBatch) {
+    if (persist_ok) {
       int pocc = hyb::decode_persist_ctas_per_sm(group);
-      if (pocc <= 0) pocc = group <= 4 ? 3 : 2;  // no GPU to ask: the compiled kernel's occupancy
+      if (pocc <= 0) pocc = 3;  // no GPU to ask: the compiled kernel's occupancy
       long long ctas = static_cast<long long>(sms) * pocc;
       if (ctas > units * ns) ctas = units * ns;
       p->cluster = false;
@@ -205,6 +208,7 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
     split_tokens = static_cast<int32_t>(tb * d->block_size);
   }
   long long tb = 0;
+  bool multi_wave = false;  // the automatic choice found no one-wave plan
   if (split_tokens == 0) {
     // one wave: enough splits of the longest sequence to fill the GPU, no more
     const long long s_wave = slots / units;
@@ -214,14 +218,16 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
       if (tb > max_tb) tb = max_tb;
     }
     if (tb == 0 || tb > kMultiWaveSplit || units * n_splits(tb) > slots) {
-      // several waves: short splits, so that the CTA scheduler evens out
-      // sequences of different lengths and CTAs that run at different speeds
-      // (the last CTA placed on an SM gets the fewest issue slots).  Also
-      // when one wave would need splits longer than that: a batch of
-      // (sequence, kv head) rows nearly as large as the GPU's CTA slots would
-      // otherwise give each row one long split, and rows of different
-      // lengths would leave SMs idle.
-      tb = kMultiWaveSplit;
+      // several waves (also when one wave would need splits longer than
+      // kMultiWaveSplit: a batch of (sequence, kv head) rows nearly as large
+      // as the GPU's CTA slots would otherwise give each row one long split).
+      // The persistent kernel takes these plans where it can: it hands out
+      // the longest splits first and claims units late, so long splits
+      // (fewer per-unit prologues and merges) cost no tail; the split-per-CTA
+      // kernel gets short splits, so that the CTA scheduler evens out rows of
+      // different lengths.
+      tb = persist_ok ? hyb::kPMaxSplitBlocks : kMultiWaveSplit;
+      multi_wave = true;
       if (tb > nblk) tb = nblk > 0 ? nblk : 1;
     }
   } else {
@@ -241,10 +247,9 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
   // up to kPMaxSplitBlocks blocks, batches of up to kPMaxBatch sequences)
   p->persist = false;
   p->ctas = 0;
-  if (!p->cluster && units * ns > slots && d->block_size == hyb::kBlock && d->quant_bits != 0 &&
-      tb <= hyb::kPMaxSplitBlocks && d->batch <= hyb::kPMaxBatch) {
+  if (!p->cluster && (units * ns > slots || multi_wave) && persist_ok && tb <= hyb::kPMaxSplitBlocks) {
     int pocc = hyb::decode_persist_ctas_per_sm(group);
-    if (pocc <= 0) pocc = group <= 4 ? 3 : 2;  // no GPU to ask: the compiled kernel's occupancy
+    if (pocc <= 0) pocc = 3;  // no GPU to ask: the compiled kernel's occupancy
     long long c = static_cast<long long>(sms) * pocc;
     if (c > units * ns) c = units * ns;
     p->persist = true;
