@@ -48,6 +48,28 @@ PROFILE_JSON = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
 KERNEL_SOURCES = ["decode_kernel.cuh", "decode_persist.cuh", "decode_dev.cuh", "mma.cuh", "common.cuh",
                   "kernels.cuh"]
 FLUSH_BYTES = 512 << 20   # > 126 MB L2
+CLEAN_BYTES = 256 << 20   # read after the flush write: L2 holds no dirty line when the timed step starts
+L2_NOTE = ("flushed between timed steps: a 512 MB write, then a read of another 256 MB buffer, so that the "
+           "flush's dirty lines are written back before the timed step, not inside it")
+
+
+class L2Flush:
+    """Evicts everything from L2 between timed steps: writes a buffer larger
+    than L2, then reads another one (the write-backs of the written lines
+    happen during that read, outside the timed region)."""
+
+    def __init__(self, torch, dev, enabled=True):
+        self.sum = torch.sum
+        self.w = torch.empty(FLUSH_BYTES if enabled else 0, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros((CLEAN_BYTES // 4) if enabled else 0, dtype=torch.int32, device=dev)
+        self.acc = torch.zeros((), dtype=torch.int64, device=dev)
+
+    def __call__(self):
+        if self.w.numel():
+            self.w.zero_()
+            self.sum(self.r, 0, out=self.acc)
+
+
 DECODE_KERNELS = {"persistent": "hyb::decode_persist_kernel", "split_cta": "hyb::decode_kernel",
                   "cluster": "hyb::decode_kernel (clusters)"}
 
@@ -114,7 +136,7 @@ def workload_config(w, split, ns, qbits=8, split_len=None):
             "block_size": w.block_size, "quant_bits": qbits, "split_tokens": split, "n_splits": ns,
             "splits": split_desc(split, split if split_len is None else split_len, ns),
             "step": "hyb_decode_step: append 1 token/seq + split-KV attention, one launch",
-            "l2": "flushed between timed steps (512 MB write)",
+            "l2": L2_NOTE,
             "parallelism": "replicas (independent batch per GPU)"}
 
 
@@ -406,12 +428,12 @@ def run_config(args, wl, rank, world, local_rank, clocks=None, cpu=True):
     ws = cache.step_workspace(L, split)
 
     snap = None if args.lean else StateSnapshot(cache, _touched_blocks(w, n_last), torch, dev)
-    flush = torch.empty(0 if args.lean else FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(torch, dev, enabled=not args.lean)
 
     def before():
         if snap is not None:
             snap.restore()
-        flush.zero_()
+        flush()
 
     # one eager run (sets kernel attributes, checks the path), then capture the
     # step -- hyb_decode_step: append of the step's token + attention, one
@@ -560,11 +582,11 @@ def run_append(args, rank, world, local_rank):
     k, v = synth.step_tokens(w, 10_000, n_step, max_new=64)
     n_d, k_d, v_d = (torch.from_numpy(x).to(dev) for x in (n_step, k, v))
     snap = StateSnapshot(cache, _touched_blocks(w, n_step), torch, dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(torch, dev)
 
     def before():
         snap.restore()
-        flush.zero_()
+        flush()
 
     def body():
         cache.append(n_d, k_d, v_d)
@@ -626,12 +648,12 @@ def run_migrate(args):
     delta = int((n1 - n0).max())
     t_down = torch.from_numpy(n1).cuda()
     t_up = torch.from_numpy(n0).cuda()
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = L2Flush(torch, "cuda")
     clocks = ClockSampler(0)
     times = {"demote": [], "promote": []}
     for i in range(2 * (args.warmup + args.steps)):
         kind = "demote" if i % 2 == 0 else "promote"
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         cache.migrate(t_down if kind == "demote" else t_up, delta)
@@ -693,12 +715,12 @@ def run_sparse(args):
     lse = torch.empty((w.batch, w.num_q_heads), dtype=torch.float32, device="cuda")
     ws_s = cache.sparse_workspace(L, split)
     ws_d = cache.workspace(L, split)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = L2Flush(torch, "cuda")
     clocks = ClockSampler(0)
     times = {"sparse": [], "dense": []}
     for i in range(2 * (args.warmup + args.steps)):
         kind = "sparse" if i % 2 == 0 else "dense"
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         if kind == "sparse":

@@ -140,12 +140,19 @@ namespace {
 
 // Cold blocks per split when the splits take several waves.
 constexpr int kMultiWaveSplit = 16;
+// Fewest blocks per split of a one-wave plan: a CTA's fixed cost (the
+// metadata round trip before its first copy, the epilogue and the split
+// merge, ~3 us) wants a few items of work.  On the Llama-3-8B batch of 8 at
+// L = 2048 (33 items per sequence and kv head), 6-block splits measured
+// 22.7 us per step, 4-block splits (the most the GPU holds at once) 28.5 us.
+constexpr int kMinWaveSplit = 6;
 
 // How a decode call runs: grid (ns, Hkv, batch) of the decode kernel.  When
 // every split fits on the GPU at once (one wave), automatic plans cut the
-// longest sequence into as many splits as fill the GPU, and 2..8 splits are
-// merged inside a thread-block cluster.  Otherwise the splits are short and
-// run in several waves, merged through the workspace.
+// longest sequence into as many splits as fill the GPU (of at least
+// kMinWaveSplit blocks), and 2..16 splits are merged inside a thread-block
+// cluster when all clusters fit.  Otherwise the splits run in several waves,
+// merged through the workspace (the persistent kernel where it applies).
 struct Plan {
   bool cluster;  // clusters of ns CTAs (split merge in distributed shared memory)
   bool persist;  // the persistent kernel: `ctas` CTAs take the splits as work units
@@ -214,7 +221,7 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
     const long long s_wave = slots / units;
     if (s_wave >= 1) {
       tb = (nblk + dhb + s_wave - 1) / s_wave;
-      if (tb < 1) tb = 1;
+      if (tb < kMinWaveSplit) tb = kMinWaveSplit;
       if (tb > max_tb) tb = max_tb;
     }
     if (tb == 0 || tb > kMultiWaveSplit || units * n_splits(tb) > slots) {

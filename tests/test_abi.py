@@ -111,8 +111,9 @@ def test_plan_and_workspace():
         st, ns = hk.hyb_decode_plan(d, L, 0)
         assert st % 64 == 0 and 64 <= st <= 8192 and ns >= 1
         assert ns == _splits(L, st)
-    # one wave when every split fits on the GPU at once (4 x 8 units x 16 <= 444)
-    assert hk.hyb_decode_plan(d, 2048, 0)[1] >= 8
+    # one wave when every split fits on the GPU at once: 4 x 8 rows, splits of
+    # at least 6 blocks (33 items -> 6 splits)
+    assert hk.hyb_decode_plan(d, 2048, 0) == (384, 6)
 
 
 def _per_seq_splits(c, n):
