@@ -9,7 +9,7 @@ splits, in one launch.
 
 Default run (the line the driver reads): the headline is the long-context
 workload (batch 4, L = 32K, 32K, 128K, 128K, Llama-3-8B attention shapes,
-512-token splits), the largest single-GPU configuration; the same run
+at least 64 splits per sequence), the largest single-GPU configuration; the same run
 reports sub-records for the Llama-3-8B batch-8 L=2048 workload, the
 variable-length batch of 64 and the Qwen2-7B mixed batch of 128 (each with
 its own e2e and CPU baseline), an append-only record (one hyb_kv_append of
