@@ -76,6 +76,25 @@ def test_softmax_scale_one_with_scaled_q():
     assert_decode_close(w, got, lse, ref, ref_lse, what="scale 1")
 
 
+@pytest.mark.parametrize("batch", [256, 257])
+def test_persistent_batch_limit(batch):
+    """256 sequences (the persistent kernel's limit: their lengths are staged
+    in shared memory) take the persistent kernel with per-sequence splits and
+    longest-first ordering; 257 fall back to the one-CTA-per-split kernel.
+    Both within the bar against the oracle."""
+    rng = np.random.default_rng(batch)
+    lens = [int(x) for x in rng.integers(0, 400, size=batch)]
+    lens[0], lens[1] = 0, 33  # an empty sequence and one just past the hot zone
+    w = synth.custom_workload("batch%d" % batch, lens, 8, 2, seed=batch, max_step=64)
+    cache, ora = make_pair(w)
+    replay(w, cache, ora)
+    kern = cache.launch_info(int(w.lens.max()), -3)[0]
+    assert kern == ("persistent" if batch <= 256 else "split_cta")
+    got, lse, ref, ref_lse = decode_both(w, cache, ora, split_tokens=-3)
+    assert_decode_close(w, got, lse, ref, ref_lse, what="batch %d" % batch)
+    assert cache.status() == 0
+
+
 def test_split_invariance():
     """One split per sequence vs 64-token splits: same result within FP32 merges."""
     w = synth.custom_workload("inv", [5000, 700, 33], 32, 8, seed=21)

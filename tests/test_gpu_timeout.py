@@ -16,8 +16,10 @@ pytestmark = pytest.mark.gpu
 
 
 # splits far longer than the 3-stage copy ring, so that most items are
-# issued during the loop and waited for shortly after
-@pytest.mark.parametrize("split", [64 * 40, 64 * 128])
+# issued during the loop and waited for shortly after (one CTA per split);
+# split_tokens -4: per-sequence splits on the persistent kernel, whose
+# producer then hands out the remaining units with no items
+@pytest.mark.parametrize("split", [64 * 40, 64 * 128, -4])
 def test_wait_limit_times_out_then_recovers(split):
     import torch
     from int8_paged_kv_hybrid_b200 import _lib
@@ -48,7 +50,8 @@ def test_wait_limit_times_out_then_recovers(split):
     assert cache.status() == 0
 
 
-def test_wait_limit_in_fused_step():
+@pytest.mark.parametrize("split", [64 * 40, -4])
+def test_wait_limit_in_fused_step(split):
     """The fused step with the short limit: the status reports the timeout and
     every barrier of the fused append is still passed by all warps (the call
     returns); after restoring the limit the library keeps working."""
@@ -58,7 +61,6 @@ def test_wait_limit_in_fused_step():
     cache, ora = make_pair(w)
     replay(w, cache, ora)
     L = int(w.lens.max()) + 1
-    split = 64 * 40
     rng = np.random.default_rng(3)
     n = torch.ones(w.batch, dtype=torch.int32, device="cuda")
     k = torch.from_numpy(rng.standard_normal((w.batch, 1, 8, 128)).astype(np.float16)).cuda()
