@@ -71,7 +71,9 @@ class L2Flush:
 
 
 DECODE_KERNELS = {"persistent": "hyb::decode_persist_kernel", "split_cta": "hyb::decode_kernel",
-                  "cluster": "hyb::decode_kernel (clusters)"}
+                  "cluster": "hyb::decode_kernel (clusters)",
+                  "persistent+combine": "hyb::decode_persist_kernel, then hyb::persist_combine_kernel"}
+DECODE_LAUNCHES = {"persistent": 1, "split_cta": 1, "cluster": 1, "persistent+combine": 2}
 
 
 def parse():
@@ -529,8 +531,9 @@ def run_config(args, wl, rank, world, local_rank, clocks=None, cpu=True):
                      "frac": round(achieved / peak, 4),
                      "traffic": None if traffic is None else int(traffic),
                      "traffic_source": traffic_how,
-                     "kernel": "%s (fused append + attention, the step's only launch; %d CTAs, %d per SM)"
-                               % (DECODE_KERNELS[launch_kind], launch_ctas, launch_occ),
+                     "kernel": "%s (fused append + attention; %d CTAs, %d per SM; %d launch(es) per step, "
+                               "all inside the timed span)"
+                               % (DECODE_KERNELS[launch_kind], launch_ctas, launch_occ, DECODE_LAUNCHES[launch_kind]),
                      "peak_kind": peak_kind,
                      "achieved_bytes": "algorithmic bytes per launch: attention %d + append %d"
                                        % (kvb, stepb - kvb)},
@@ -542,7 +545,7 @@ def run_config(args, wl, rank, world, local_rank, clocks=None, cpu=True):
         "e2e_graph": {"value": round(job_throughput(kvb, world, ms_e2e_g), 1), "unit": UNIT,
                       "ms_per_step": round(ms_e2e_g, 5),
                       "path": "the same three operations captured once as a CUDA graph and replayed"},
-        "gpu_launches": args.steps,
+        "gpu_launches": DECODE_LAUNCHES[launch_kind] * args.steps,
         "clocks": clk,
     }
     if want_cpu:

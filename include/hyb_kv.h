@@ -247,7 +247,12 @@ int hyb_decode_plan(const hyb_cache_desc *desc, int32_t max_seq_len, int32_t spl
  *                          shared memory;
  *   HYB_KERNEL_PERSISTENT  `ctas` resident CTAs that take the splits as work
  *                          units from a counter (64-token INT8/INT4 blocks,
- *                          batch <= 256, splits of at most 32 blocks).
+ *                          batch <= 256, splits of at most 32 blocks), the
+ *                          splits merged inside the launch;
+ *   HYB_KERNEL_PERSISTENT_COMBINE  the same kernel when a sequence may have
+ *                          more than 16 splits: it writes every split's
+ *                          partial and a second launch (one CTA per sequence
+ *                          and kv head) merges them by log-sum-exp.
  * Writes the kernel, the CTAs of the launch and the CTAs one SM holds (the
  * device's occupancy for that kernel; 0 when no device can be queried).  Any
  * output pointer may be NULL.  Returns HYB_OK or HYB_ERR_INVALID_VALUE (the
@@ -257,6 +262,7 @@ int hyb_decode_plan(const hyb_cache_desc *desc, int32_t max_seq_len, int32_t spl
 #define HYB_KERNEL_SPLIT_CTA 0
 #define HYB_KERNEL_CLUSTER 1
 #define HYB_KERNEL_PERSISTENT 2
+#define HYB_KERNEL_PERSISTENT_COMBINE 3
 int hyb_decode_launch_info(const hyb_cache_desc *desc, int32_t max_seq_len, int32_t split_tokens,
                            int32_t *kernel, int32_t *ctas, int32_t *ctas_per_sm);
 
@@ -289,12 +295,16 @@ size_t hyb_decode_workspace_bytes(const hyb_cache_desc *desc, int32_t max_seq_le
  *   out      device FP16 [batch][Hq][D] (round to nearest even), 16-byte aligned.
  *   lse_out  device FP32 [batch][Hq] natural-log log-sum-exp of the logits, or NULL.
  * An empty sequence (L = 0) gives out = 0 and lse = -inf.
- * One kernel launch: one CTA per (split, kv head, sequence).  When every
- * split fits on the GPU at once and a (sequence, kv head) has 2..16 splits
- * whose clusters can all be resident, its splits form a thread-block
+ * Launches (hyb_decode_launch_info tells which): one wave of splits -- one
+ * CTA per (split, kv head, sequence); when a (sequence, kv head) has 2..16
+ * splits whose clusters can all be resident, its splits form a thread-block
  * cluster and are merged by log-sum-exp (the same merge as hyb_combine)
- * through distributed shared memory; otherwise the last CTA of a (sequence,
- * kv head) to finish merges them through the workspace.
+ * through distributed shared memory, otherwise the last CTA of a (sequence,
+ * kv head) to finish merges them through the workspace.  Several waves, or
+ * per-sequence splits -- the persistent kernel: resident CTAs take the splits
+ * as work units; up to 16 splits per sequence are merged inside the launch
+ * (by the unit that finishes last), more by a second launch (one CTA per
+ * sequence and kv head) after it.
  * Arithmetic (tensor cores, warp-level mma): cold dot products run exactly
  * in integers -- q in 24-bit fixed point per head (relative to its largest
  * channel) against the codes, and softmax weights in 16-bit fixed point
@@ -400,13 +410,16 @@ int hyb_decode_attn_noalloc(const hyb_cache_desc *desc, const void *q, float sof
 size_t hyb_noalloc_scratch_limit(void);
 
 /*
- * One decode step in one launch: hyb_kv_append of n_new[b] in {0, 1} tokens
+ * One decode step in one launch (two when the attention's splits are merged
+ * by a launch of their own, as hyb_decode_attn says): hyb_kv_append of
+ * n_new[b] in {0, 1} tokens
  * followed by hyb_decode_attn over the grown cache ([hybrid_v2 page] 4.2,
  * steps 2-5 fused).  The CTA that attends a sequence's tail block and hot ring
  * seals the token leaving the hot zone inside its staged copies (same
  * arithmetic as hyb_kv_append, bit-exact), writes the changed codes, scale
  * and ring slot back, and attends the updated copies; seq_lens[b] is
- * advanced by the last CTA of the sequence.
+ * advanced by the last CTA of the sequence (persistent kernel: by the last
+ * CTA of the launch).
  *   n_new    device int32 [batch], each 0 or 1 (other values: that sequence
  *            gets HYB_STATUS_BAD_N_NEW and is attended without appending).
  *   k_new, v_new  device FP16 [batch][1][Hkv][D] (the hyb_kv_append layout

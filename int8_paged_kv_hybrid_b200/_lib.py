@@ -158,7 +158,7 @@ def hyb_decode_plan(desc, max_seq_len, split_tokens=0):
     return st.value, ns.value
 
 
-KERNEL_NAMES = {0: "split_cta", 1: "cluster", 2: "persistent"}
+KERNEL_NAMES = {0: "split_cta", 1: "cluster", 2: "persistent", 3: "persistent+combine"}
 
 
 def hyb_decode_launch_info(desc, max_seq_len, split_tokens=0):

@@ -18,6 +18,20 @@ cudaError_t launch_decode_persist(const DecodeArgs &a, int group, int batch, int
   }
 }
 
+cudaError_t launch_persist_combine(const DecodeArgs &a, int group, int batch, cudaStream_t stream) {
+  switch (group) {
+    case 1: return launch_persist_combine_g<1>(a, batch, stream);
+    case 2: return launch_persist_combine_g<2>(a, batch, stream);
+    case 3: return launch_persist_combine_g<3>(a, batch, stream);
+    case 4: return launch_persist_combine_g<4>(a, batch, stream);
+    case 5: return launch_persist_combine_g<5>(a, batch, stream);
+    case 6: return launch_persist_combine_g<6>(a, batch, stream);
+    case 7: return launch_persist_combine_g<7>(a, batch, stream);
+    case 8: return launch_persist_combine_g<8>(a, batch, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 // CTAs of the persistent kernel one SM holds at once for this head group (0
 // if the device cannot be queried); cached per device.
 int decode_persist_ctas_per_sm(int group) {

@@ -744,7 +744,7 @@ __global__ void __launch_bounds__(kPThreads, PersistCfg<G>::kCtasPerSm) decode_p
           const float l = ws.l_run[nt];
           const float inv = l > 0.f ? __frcp_rn(l) : 0.f;
           const float lse2 = l > 0.f ? ws.m_run[nt] + __log2f(l) : -INFINITY;
-          if (Sb == 1) {
+          if (Sb == 1 && !a.defer_merge) {
             __half *o = a.out + (row0 + hh) * kDim;
 #pragma unroll
             for (int mt = 0; mt < 8; mt++) {
@@ -768,7 +768,10 @@ __global__ void __launch_bounds__(kPThreads, PersistCfg<G>::kCtasPerSm) decode_p
     // the registers
     if (run_pend) pend_run(pm);
     if (warp == 0) {
-      if (Sb > 1) {
+      if (a.defer_merge) {
+        // the merge comes after the launch: it needs the split count
+        if (s == 0 && lane == 0) a.counters[b * a.hkv + h] = Sb;
+      } else if (Sb > 1) {
         // arrival: the last unit of (sequence, kv head) -- or of its group of
         // kMergeFan splits -- merges; the answer is read at the next epilogue
         __syncwarp();
@@ -797,6 +800,107 @@ __global__ void __launch_bounds__(kPThreads, PersistCfg<G>::kCtasPerSm) decode_p
     const PendMerge pm = sm.pend;
     pend_run(pm);
   }
+}
+
+// After a persistent launch with defer_merge: the splits of (kv head h,
+// sequence b) -- counters[b][h] of them, written by the launch -- merged by
+// log-sum-exp for each of the G query heads.  Method: the same merge as
+// hyb_combine (web page "DeepSeek V4混合式KV Cache推理优化实战解析",
+// section 4.2, step 5).  One CTA of 16 warps per (kv head, sequence): warp w
+// takes head w % G and every P-th split from w / G (P = 16 / G subsets per
+// head), with all of its partials' loads in flight at once (lane l: channels
+// 4l .. 4l + 3); the subsets then join through shared memory, and the CTA
+// resets the counter for the next call.
+constexpr int kCombWarps = 16;
+constexpr int kCombBatch = 8;  // partials a warp loads at a time
+
+template <int G>
+__global__ void __launch_bounds__(32 * kCombWarps) persist_combine_kernel(const DecodeArgs a) {
+  constexpr int P = kCombWarps / G;  // subsets of the splits per head
+  __shared__ float4 s_num[G][P][32];
+  __shared__ float s_m[G][P], s_den[G][P];
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int NS = a.n_splits;
+  int32_t *cnt = &a.counters[b * a.hkv + h];
+  const int Sb = min(max(*cnt, 1), NS);
+  const size_t row0 = (size_t)b * a.hq + h * G;
+  if (warp < G * P) {
+    const int hh = warp % G, p = warp / G;
+    const float *o = a.o_part + (row0 + hh) * NS * kDim + 4 * lane;
+    const float *lse = a.lse_part + (row0 + hh) * NS;
+    float m = -INFINITY, den = 0.f;
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = p; j0 < Sb; j0 += P * kCombBatch) {
+      float4 ov[kCombBatch];
+      float lv[kCombBatch];
+#pragma unroll
+      for (int jj = 0; jj < kCombBatch; jj++) {
+        const int j = j0 + jj * P;
+        ov[jj] = j < Sb ? __ldcg(reinterpret_cast<const float4 *>(o + (size_t)j * kDim)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        lv[jj] = j < Sb ? __ldcg(lse + j) : -INFINITY;
+      }
+      float mr = m;
+#pragma unroll
+      for (int jj = 0; jj < kCombBatch; jj++) mr = fmaxf(mr, lv[jj]);
+      if (mr == -INFINITY) continue;  // nothing but empty partials so far
+      const float sc = ex2(m - mr);
+      num.x *= sc; num.y *= sc; num.z *= sc; num.w *= sc;
+      den *= sc;
+      m = mr;
+#pragma unroll
+      for (int jj = 0; jj < kCombBatch; jj++) {
+        const float wj = ex2(lv[jj] - m);  // 0 for an empty partial
+        den += wj;
+        num.x = fmaf(wj, ov[jj].x, num.x);
+        num.y = fmaf(wj, ov[jj].y, num.y);
+        num.z = fmaf(wj, ov[jj].z, num.z);
+        num.w = fmaf(wj, ov[jj].w, num.w);
+      }
+    }
+    s_num[hh][p][lane] = num;
+    if (lane == 0) {
+      s_m[hh][p] = m;
+      s_den[hh][p] = den;
+    }
+  }
+  __syncthreads();
+  if (warp < G) {
+    const int hh = warp;
+    float m = -INFINITY;
+#pragma unroll
+    for (int p = 0; p < P; p++) m = fmaxf(m, s_m[hh][p]);
+    float den = 0.f;
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (m != -INFINITY) {
+#pragma unroll
+      for (int p = 0; p < P; p++) {
+        const float wp = ex2(s_m[hh][p] - m);
+        const float4 v = s_num[hh][p][lane];
+        den = fmaf(wp, s_den[hh][p], den);
+        num.x = fmaf(wp, v.x, num.x);
+        num.y = fmaf(wp, v.y, num.y);
+        num.z = fmaf(wp, v.z, num.z);
+        num.w = fmaf(wp, v.w, num.w);
+      }
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    const __half2 h01 = __floats2half2_rn(num.x * inv, num.y * inv);
+    const __half2 h23 = __floats2half2_rn(num.z * inv, num.w * inv);
+    uint2 pk;
+    pk.x = *reinterpret_cast<const uint32_t *>(&h01);
+    pk.y = *reinterpret_cast<const uint32_t *>(&h23);
+    *reinterpret_cast<uint2 *>(a.out + (row0 + hh) * kDim + 4 * lane) = pk;
+    if (lane == 0 && a.lse_out) a.lse_out[row0 + hh] = den > 0.f ? (m + log2f(den)) * kLn2 : -INFINITY;
+  }
+  __syncthreads();
+  if (tid == 0) *cnt = 0;
+}
+
+template <int G>
+cudaError_t launch_persist_combine_g(const DecodeArgs &a, int batch, cudaStream_t stream) {
+  persist_combine_kernel<G><<<dim3(a.hkv, batch), 32 * kCombWarps, 0, stream>>>(a);
+  return cudaGetLastError();
 }
 
 template <int G>

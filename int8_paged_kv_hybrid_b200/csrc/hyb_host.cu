@@ -159,6 +159,7 @@ struct Plan {
   int ctas;
   int tb;        // cold blocks per split (per-sequence splits: the longest sequence's)
   int per_seq;   // > 0: per-sequence splits, at least this many per sequence
+  bool defer;    // persistent with more than kMergeFan splits: partials only, then persist_combine_kernel
   int ns;        // splits per (sequence, kv head), at most
 };
 
@@ -191,6 +192,7 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
   // <= 256 sequences)
   const bool persist_ok = d->block_size == hyb::kBlock && d->quant_bits != 0 && d->batch <= hyb::kPMaxBatch;
   p->per_seq = 0;
+  p->defer = false;
   if (split_tokens < 0) {
     // per-sequence splits (per_seq_splits): the persistent kernel only; where
     // it cannot run, every sequence takes the longest one's split length
@@ -210,6 +212,7 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
       p->per_seq = static_cast<int>(n);
       p->tb = static_cast<int>(tb);
       p->ns = static_cast<int>(ns);
+      p->defer = ns > hyb::kMergeFan;
       return HYB_OK;
     }
     split_tokens = static_cast<int32_t>(tb * d->block_size);
@@ -261,6 +264,7 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
     if (c > units * ns) c = units * ns;
     p->persist = true;
     p->ctas = static_cast<int>(c);
+    p->defer = ns > hyb::kMergeFan;
   }
   p->tb = static_cast<int>(tb);
   p->ns = static_cast<int>(ns);
@@ -345,7 +349,9 @@ int hyb_decode_launch_info(const hyb_cache_desc *d, int32_t max_seq_len, int32_t
   if (rc != HYB_OK) return rc;
   const int group = d->num_q_heads / d->num_kv_heads;
   const int units = d->batch * d->num_kv_heads;
-  if (kernel) *kernel = pl.persist ? HYB_KERNEL_PERSISTENT : (pl.cluster ? HYB_KERNEL_CLUSTER : HYB_KERNEL_SPLIT_CTA);
+  if (kernel)
+    *kernel = pl.persist ? (pl.defer ? HYB_KERNEL_PERSISTENT_COMBINE : HYB_KERNEL_PERSISTENT)
+                         : (pl.cluster ? HYB_KERNEL_CLUSTER : HYB_KERNEL_SPLIT_CTA);
   if (ctas) *ctas = pl.persist ? pl.ctas : units * pl.ns;
   if (ctas_per_sm)
     *ctas_per_sm = pl.persist ? hyb::decode_persist_ctas_per_sm(group) : hyb::decode_ctas_per_sm(group);
@@ -417,10 +423,14 @@ static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_s
   const bool persist = pl.persist && !l2_skip;
   a.unit_ctr = pl.persist ? reinterpret_cast<int32_t *>(ws + wl.unit_ctr) : nullptr;
   a.min_splits = pl.per_seq;
+  a.defer_merge = persist && pl.defer ? 1 : 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int group = d->num_q_heads / d->num_kv_heads;
-  const cudaError_t e = persist ? hyb::launch_decode_persist(a, group, d->batch, pl.ctas, s)
-                                : hyb::launch_decode(a, group, d->batch, pl.cluster, s);
+  cudaError_t e = persist ? hyb::launch_decode_persist(a, group, d->batch, pl.ctas, s)
+                          : hyb::launch_decode(a, group, d->batch, pl.cluster, s);
+  // many splits per sequence: their merge is a launch of its own, so that no
+  // CTA of the persistent kernel spends the end of the launch merging
+  if (e == cudaSuccess && a.defer_merge) e = hyb::launch_persist_combine(a, group, d->batch, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return HYB_OK;
 }

@@ -70,6 +70,10 @@ struct DecodeArgs {
   // persistent kernel: > 0 = per-sequence splits (per_seq_splits), at least
   // this many per sequence; 0 = runs of split_blocks blocks
   int min_splits;
+  // persistent kernel: every unit writes its partial, the unit of split 0
+  // writes the sequence's split count into counters[sequence][kv head], and
+  // persist_combine_kernel merges them after the launch (no arrivals)
+  int defer_merge;
 };
 
 // Persistent decode kernel limits: blocks per split (one block-table entry
@@ -147,6 +151,9 @@ cudaError_t launch_append(const AppendArgs &a, int batch, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, bool cluster, cudaStream_t stream);
 cudaError_t launch_decode_persist(const DecodeArgs &a, int group, int batch, int ctas, cudaStream_t stream);
 int decode_persist_ctas_per_sm(int group);
+// The log-sum-exp merge after a persistent launch with defer_merge: one CTA
+// per (kv head, sequence) merges its counters[] splits of every query head.
+cudaError_t launch_persist_combine(const DecodeArgs &a, int group, int batch, cudaStream_t stream);
 cudaError_t launch_migrate(const MigrateArgs &a, int batch, cudaStream_t stream);
 cudaError_t launch_combine(const CombineArgs &a, int rows, cudaStream_t stream);
 cudaError_t launch_sparse_l2(const SparseArgs &a, int batch, cudaStream_t stream);

@@ -168,10 +168,14 @@ def test_launch_info():
     splits take the persistent kernel, one wave of a few splits the
     one-CTA-per-split kernel; FP16 cold blocks never the persistent one."""
     d = _desc(batch=4, maxb=2048, phys=8192)
+    # more than 16 splits per sequence: partials, then a merge launch
     kern, ctas, occ = hk.hyb_decode_launch_info(d, 131072, -64)
-    assert kern == "persistent" and 1 <= ctas <= 4 * 8 * 65 and occ >= 0
+    assert kern == "persistent+combine" and 1 <= ctas <= 4 * 8 * 65 and occ >= 0
     kern, ctas, _ = hk.hyb_decode_launch_info(d, 131072, 512)
-    assert kern == "persistent" and ctas <= 4 * 8 * 257
+    assert kern == "persistent+combine" and ctas <= 4 * 8 * 257
+    # up to 16: merged inside the launch
+    kern, ctas, _ = hk.hyb_decode_launch_info(d, 8192, -8)
+    assert kern == "persistent" and hk.hyb_decode_plan(d, 8192, -8)[1] == 8
     kern, ctas, _ = hk.hyb_decode_launch_info(d, 100, 64)
     assert kern == "split_cta" and ctas == 4 * 8 * hk.hyb_decode_plan(d, 100, 64)[1]
     d0 = _desc(batch=4, maxb=2048, phys=8192, qbits=0)
