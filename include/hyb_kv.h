@@ -251,8 +251,8 @@ int hyb_decode_plan(const hyb_cache_desc *desc, int32_t max_seq_len, int32_t spl
  *                          splits merged inside the launch;
  *   HYB_KERNEL_PERSISTENT_COMBINE  the same kernel when a sequence may have
  *                          more than 16 splits: it writes every split's
- *                          partial and a second launch (one CTA per sequence
- *                          and kv head) merges them by log-sum-exp.
+ *                          partial and a second launch (one CTA per query
+ *                          head and sequence) merges them by log-sum-exp.
  * Writes the kernel, the CTAs of the launch and the CTAs one SM holds (the
  * device's occupancy for that kernel; 0 when no device can be queried).  Any
  * output pointer may be NULL.  Returns HYB_OK or HYB_ERR_INVALID_VALUE (the
@@ -304,7 +304,7 @@ size_t hyb_decode_workspace_bytes(const hyb_cache_desc *desc, int32_t max_seq_le
  * per-sequence splits -- the persistent kernel: resident CTAs take the splits
  * as work units; up to 16 splits per sequence are merged inside the launch
  * (by the unit that finishes last), more by a second launch (one CTA per
- * sequence and kv head) after it.
+ * query head and sequence) after it.
  * Arithmetic (tensor cores, warp-level mma): cold dot products run exactly
  * in integers -- q in 24-bit fixed point per head (relative to its largest
  * channel) against the codes, and softmax weights in 16-bit fixed point

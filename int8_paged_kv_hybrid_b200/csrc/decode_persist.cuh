@@ -203,6 +203,9 @@ __global__ void __launch_bounds__(kPThreads, PersistCfg<G>::kCtasPerSm) decode_p
     mbar_fence_init();
   }
   if (tid < 4) sm.zero16[tid] = 0u;
+  // a merge launch that follows (defer_merge) may be placed on the SMs as
+  // this launch's CTAs leave them; it waits for this grid's results itself
+  if (tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // lengths at launch and the work units of each sequence: its splits with
   // work (at least one, which writes the output of an empty sequence) times
   // the kv heads.  Units are numbered sequence by sequence, so the counter
@@ -770,7 +773,7 @@ __global__ void __launch_bounds__(kPThreads, PersistCfg<G>::kCtasPerSm) decode_p
     if (warp == 0) {
       if (a.defer_merge) {
         // the merge comes after the launch: it needs the split count
-        if (s == 0 && lane == 0) a.counters[b * a.hkv + h] = Sb;
+        if (s == 0 && lane == 0) a.split_count[b * a.hkv + h] = Sb;
       } else if (Sb > 1) {
         // arrival: the last unit of (sequence, kv head) -- or of its group of
         // kMergeFan splits -- merges; the answer is read at the next epilogue
@@ -802,104 +805,109 @@ __global__ void __launch_bounds__(kPThreads, PersistCfg<G>::kCtasPerSm) decode_p
   }
 }
 
-// After a persistent launch with defer_merge: the splits of (kv head h,
-// sequence b) -- counters[b][h] of them, written by the launch -- merged by
-// log-sum-exp for each of the G query heads.  Method: the same merge as
-// hyb_combine (web page "DeepSeek V4混合式KV Cache推理优化实战解析",
-// section 4.2, step 5).  One CTA of 16 warps per (kv head, sequence): warp w
-// takes head w % G and every P-th split from w / G (P = 16 / G subsets per
-// head), with all of its partials' loads in flight at once (lane l: channels
-// 4l .. 4l + 3); the subsets then join through shared memory, and the CTA
-// resets the counter for the next call.
+// After a persistent launch with defer_merge: the splits of query head hq of
+// sequence b -- split_count[b][hq / G] of them, written by the launch --
+// merged by log-sum-exp.  Method: the same merge as hyb_combine (web page
+// "DeepSeek V4混合式KV Cache推理优化实战解析", section 4.2, step 5).  One
+// CTA of 16 warps per (query head, sequence): warp w takes every 16th split
+// from w, with all of its partials' loads in flight at once (lane l:
+// channels 4l .. 4l + 3); the 16 subsets then join through shared memory.
 constexpr int kCombWarps = 16;
 constexpr int kCombBatch = 8;  // partials a warp loads at a time
 
 template <int G>
 __global__ void __launch_bounds__(32 * kCombWarps) persist_combine_kernel(const DecodeArgs a) {
-  constexpr int P = kCombWarps / G;  // subsets of the splits per head
-  __shared__ float4 s_num[G][P][32];
-  __shared__ float s_m[G][P], s_den[G][P];
-  const int h = blockIdx.x, b = blockIdx.y;
+  __shared__ float4 s_num[kCombWarps][32];
+  __shared__ float s_m[kCombWarps], s_den[kCombWarps];
+  const int hq = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int NS = a.n_splits;
-  int32_t *cnt = &a.counters[b * a.hkv + h];
-  const int Sb = min(max(*cnt, 1), NS);
-  const size_t row0 = (size_t)b * a.hq + h * G;
-  if (warp < G * P) {
-    const int hh = warp % G, p = warp / G;
-    const float *o = a.o_part + (row0 + hh) * NS * kDim + 4 * lane;
-    const float *lse = a.lse_part + (row0 + hh) * NS;
-    float m = -INFINITY, den = 0.f;
-    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = p; j0 < Sb; j0 += P * kCombBatch) {
-      float4 ov[kCombBatch];
-      float lv[kCombBatch];
+  // launched as a programmatic dependent of the persistent kernel: nothing
+  // of its results is read before that grid has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int Sb = min(max(a.split_count[b * a.hkv + hq / G], 1), NS);
+  const size_t row = (size_t)b * a.hq + hq;
+  const float *o = a.o_part + row * NS * kDim + 4 * lane;
+  const float *lse = a.lse_part + row * NS;
+  float m = -INFINITY, den = 0.f;
+  float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j0 = warp; j0 < Sb; j0 += kCombWarps * kCombBatch) {
+    float4 ov[kCombBatch];
+    float lv[kCombBatch];
 #pragma unroll
-      for (int jj = 0; jj < kCombBatch; jj++) {
-        const int j = j0 + jj * P;
-        ov[jj] = j < Sb ? __ldcg(reinterpret_cast<const float4 *>(o + (size_t)j * kDim)) : make_float4(0.f, 0.f, 0.f, 0.f);
-        lv[jj] = j < Sb ? __ldcg(lse + j) : -INFINITY;
-      }
-      float mr = m;
-#pragma unroll
-      for (int jj = 0; jj < kCombBatch; jj++) mr = fmaxf(mr, lv[jj]);
-      if (mr == -INFINITY) continue;  // nothing but empty partials so far
-      const float sc = ex2(m - mr);
-      num.x *= sc; num.y *= sc; num.z *= sc; num.w *= sc;
-      den *= sc;
-      m = mr;
-#pragma unroll
-      for (int jj = 0; jj < kCombBatch; jj++) {
-        const float wj = ex2(lv[jj] - m);  // 0 for an empty partial
-        den += wj;
-        num.x = fmaf(wj, ov[jj].x, num.x);
-        num.y = fmaf(wj, ov[jj].y, num.y);
-        num.z = fmaf(wj, ov[jj].z, num.z);
-        num.w = fmaf(wj, ov[jj].w, num.w);
-      }
+    for (int jj = 0; jj < kCombBatch; jj++) {
+      const int j = j0 + jj * kCombWarps;
+      ov[jj] = j < Sb ? __ldcg(reinterpret_cast<const float4 *>(o + (size_t)j * kDim)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      lv[jj] = j < Sb ? __ldcg(lse + j) : -INFINITY;
     }
-    s_num[hh][p][lane] = num;
-    if (lane == 0) {
-      s_m[hh][p] = m;
-      s_den[hh][p] = den;
+    float mr = m;
+#pragma unroll
+    for (int jj = 0; jj < kCombBatch; jj++) mr = fmaxf(mr, lv[jj]);
+    if (mr == -INFINITY) continue;  // nothing but empty partials so far
+    const float sc = ex2(m - mr);
+    num.x *= sc; num.y *= sc; num.z *= sc; num.w *= sc;
+    den *= sc;
+    m = mr;
+#pragma unroll
+    for (int jj = 0; jj < kCombBatch; jj++) {
+      const float wj = ex2(lv[jj] - m);  // 0 for an empty partial
+      den += wj;
+      num.x = fmaf(wj, ov[jj].x, num.x);
+      num.y = fmaf(wj, ov[jj].y, num.y);
+      num.z = fmaf(wj, ov[jj].z, num.z);
+      num.w = fmaf(wj, ov[jj].w, num.w);
     }
   }
+  s_num[warp][lane] = num;
+  if (lane == 0) {
+    s_m[warp] = m;
+    s_den[warp] = den;
+  }
   __syncthreads();
-  if (warp < G) {
-    const int hh = warp;
-    float m = -INFINITY;
+  if (warp == 0) {
+    float mm = -INFINITY;
 #pragma unroll
-    for (int p = 0; p < P; p++) m = fmaxf(m, s_m[hh][p]);
-    float den = 0.f;
-    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (m != -INFINITY) {
+    for (int p = 0; p < kCombWarps; p++) mm = fmaxf(mm, s_m[p]);
+    float dd = 0.f;
+    float4 nn = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (mm != -INFINITY) {
 #pragma unroll
-      for (int p = 0; p < P; p++) {
-        const float wp = ex2(s_m[hh][p] - m);
-        const float4 v = s_num[hh][p][lane];
-        den = fmaf(wp, s_den[hh][p], den);
-        num.x = fmaf(wp, v.x, num.x);
-        num.y = fmaf(wp, v.y, num.y);
-        num.z = fmaf(wp, v.z, num.z);
-        num.w = fmaf(wp, v.w, num.w);
+      for (int p = 0; p < kCombWarps; p++) {
+        const float wp = ex2(s_m[p] - mm);
+        const float4 v = s_num[p][lane];
+        dd = fmaf(wp, s_den[p], dd);
+        nn.x = fmaf(wp, v.x, nn.x);
+        nn.y = fmaf(wp, v.y, nn.y);
+        nn.z = fmaf(wp, v.z, nn.z);
+        nn.w = fmaf(wp, v.w, nn.w);
       }
     }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    const __half2 h01 = __floats2half2_rn(num.x * inv, num.y * inv);
-    const __half2 h23 = __floats2half2_rn(num.z * inv, num.w * inv);
+    const float inv = dd > 0.f ? 1.f / dd : 0.f;
+    const __half2 h01 = __floats2half2_rn(nn.x * inv, nn.y * inv);
+    const __half2 h23 = __floats2half2_rn(nn.z * inv, nn.w * inv);
     uint2 pk;
     pk.x = *reinterpret_cast<const uint32_t *>(&h01);
     pk.y = *reinterpret_cast<const uint32_t *>(&h23);
-    *reinterpret_cast<uint2 *>(a.out + (row0 + hh) * kDim + 4 * lane) = pk;
-    if (lane == 0 && a.lse_out) a.lse_out[row0 + hh] = den > 0.f ? (m + log2f(den)) * kLn2 : -INFINITY;
+    *reinterpret_cast<uint2 *>(a.out + row * kDim + 4 * lane) = pk;
+    if (lane == 0 && a.lse_out) a.lse_out[row] = dd > 0.f ? (mm + log2f(dd)) * kLn2 : -INFINITY;
   }
-  __syncthreads();
-  if (tid == 0) *cnt = 0;
 }
 
 template <int G>
 cudaError_t launch_persist_combine_g(const DecodeArgs &a, int batch, cudaStream_t stream) {
-  persist_combine_kernel<G><<<dim3(a.hkv, batch), 32 * kCombWarps, 0, stream>>>(a);
+  // a programmatic dependent launch of the persistent kernel before it
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.hq, batch);
+  cfg.blockDim = dim3(32 * kCombWarps, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, persist_combine_kernel<G>, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -280,12 +280,12 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
 // [batch][Hq][ng].  Each part starts on a 256-byte boundary; the counters
 // come first.
 struct WsLayout {
-  size_t seq_cnt, unit_ctr, counters, g_counters, o_part, lse_part, g_part, g_lse, total;
+  size_t seq_cnt, unit_ctr, counters, g_counters, o_part, lse_part, g_part, g_lse, split_count, total;
   int n_groups;
 };
 
 WsLayout ws_layout(const hyb_cache_desc *d, const Plan &pl, bool step) {
-  WsLayout w{0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
+  WsLayout w{0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
   size_t off = 0;
   if (step) {
     w.seq_cnt = 0;
@@ -312,6 +312,11 @@ WsLayout ws_layout(const hyb_cache_desc *d, const Plan &pl, bool step) {
     w.g_part = off;
     w.g_lse = w.g_part + round_up(rows * ng * hyb::kDim * sizeof(float), kWsAlign);
     off = w.g_lse + round_up(rows * ng * sizeof(float), kWsAlign);
+  }
+  if (pl.defer) {
+    // splits of each (sequence, kv head), written by every call before it is read
+    w.split_count = off;
+    off += round_up(units * sizeof(int32_t), kWsAlign);
   }
   w.total = off;
   return w;
@@ -424,6 +429,7 @@ static int decode_launch(const hyb_cache_desc *d, const void *q, float softmax_s
   a.unit_ctr = pl.persist ? reinterpret_cast<int32_t *>(ws + wl.unit_ctr) : nullptr;
   a.min_splits = pl.per_seq;
   a.defer_merge = persist && pl.defer ? 1 : 0;
+  a.split_count = a.defer_merge ? reinterpret_cast<int32_t *>(ws + wl.split_count) : nullptr;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int group = d->num_q_heads / d->num_kv_heads;
   cudaError_t e = persist ? hyb::launch_decode_persist(a, group, d->batch, pl.ctas, s)

@@ -71,9 +71,10 @@ struct DecodeArgs {
   // this many per sequence; 0 = runs of split_blocks blocks
   int min_splits;
   // persistent kernel: every unit writes its partial, the unit of split 0
-  // writes the sequence's split count into counters[sequence][kv head], and
-  // persist_combine_kernel merges them after the launch (no arrivals)
+  // writes the sequence's split count into split_count[sequence][kv head],
+  // and persist_combine_kernel merges them after the launch (no arrivals)
   int defer_merge;
+  int32_t *split_count;
 };
 
 // Persistent decode kernel limits: blocks per split (one block-table entry
@@ -152,7 +153,7 @@ cudaError_t launch_decode(const DecodeArgs &a, int group, int batch, bool cluste
 cudaError_t launch_decode_persist(const DecodeArgs &a, int group, int batch, int ctas, cudaStream_t stream);
 int decode_persist_ctas_per_sm(int group);
 // The log-sum-exp merge after a persistent launch with defer_merge: one CTA
-// per (kv head, sequence) merges its counters[] splits of every query head.
+// per (query head, sequence) merges its split_count[] splits.
 cudaError_t launch_persist_combine(const DecodeArgs &a, int group, int batch, cudaStream_t stream);
 cudaError_t launch_migrate(const MigrateArgs &a, int batch, cudaStream_t stream);
 cudaError_t launch_combine(const CombineArgs &a, int rows, cudaStream_t stream);

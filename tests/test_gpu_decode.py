@@ -14,7 +14,7 @@ SMALL_LENS = [0, 1, 5, 31, 32, 33, 64, 95, 96, 97, 130, 255, 1000, 2047, 3001]
 
 
 @pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 4), (32, 8), (28, 4), (16, 2)])
-@pytest.mark.parametrize("split", [0, 64, 192, -3, -16])
+@pytest.mark.parametrize("split", [0, 64, 192, -3, -16, -20])
 def test_small_parity(hq, hkv, split):
     w = synth.custom_workload("small", SMALL_LENS, hq, hkv, seed=hq * 31 + hkv, max_step=64)
     cache, ora = make_pair(w)

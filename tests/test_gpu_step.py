@@ -36,7 +36,7 @@ def _run_steps(w, cache, ora, n_steps, split, seed, n_pattern=None, qbits=8):
 
 
 @pytest.mark.parametrize("hq,hkv,split", [(8, 8, 0), (32, 8, 128), (28, 4, 64), (16, 2, 0), (32, 8, -4),
-                                           (16, 2, -9)])
+                                           (16, 2, -9), (32, 8, -20), (28, 4, -24)])
 def test_steps_bit_exact_and_close(hq, hkv, split):
     """Lengths around every edge: empty, below / at the hot size, first seal,
     block boundaries, several splits (cluster and workspace merges)."""
