@@ -25,13 +25,20 @@ int cuda_fail(cudaError_t e) {
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 int sm_count() {
+  // cached per device: the planner runs on every call
+  static int cached[32];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    dev = 0;
+  }
+  if (dev >= 0 && dev < 32 && cached[dev] > 0) return cached[dev];
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
     cudaGetLastError();  // clear the sticky-free error this query may leave
-    n = 148;             // B200
+    return 148;          // B200 (not cached: a later call on a device may answer)
   }
+  if (dev >= 0 && dev < 32) cached[dev] = n;
   return n;
 }
 
