@@ -380,6 +380,38 @@ def mean_ms(evs):
     return sum(a.elapsed_time(b) for a, b in evs) / len(evs)
 
 
+def read_floor(torch, dev, nbytes, stream, side, args, world):
+    """Time hyb_stream_read over `nbytes` (rounded up to 16) the way the step is
+    timed: a CUDA graph of the one launch, replayed between two events, L2
+    flushed before each replay.  The result is the attainable time of any
+    kernel that reads that many bytes once: no table lookup, no dependent load,
+    no arithmetic, only the launch, the ramp-up and the drain."""
+    from int8_paged_kv_hybrid_b200 import hyb_stream_read
+    nb = (nbytes + 15) // 16 * 16
+    buf = torch.empty(nb, dtype=torch.uint8, device=dev)
+    buf.fill_(0x5a)
+    sink = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = L2Flush(torch, dev)
+    with torch.cuda.stream(side):
+        hyb_stream_read(buf, sink)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        hyb_stream_read(buf, sink, stream=side)
+    torch.cuda.synchronize()
+    time_events(args.warmup, stream, flush, g.replay)
+    evs = time_events(args.steps, stream, flush, g.replay)
+    torch.cuda.synchronize()
+    del g, buf
+    ms = max_over_ranks(mean_ms(evs), world, dev)
+    return {"bytes": nb, "ms_per_call": round(ms, 5), "GB/s": round(nb / (ms * 1e-3) / 1e9, 1),
+            "what": "hyb_stream_read of the step's algorithmic bytes: one coalesced streaming read with no "
+                    "lookup, dependent load or arithmetic, timed like the step (CUDA-graph replay between "
+                    "events, L2 flushed before each); the attainable time of any kernel that reads these "
+                    "bytes once",
+            "gpu_launches": args.steps}
+
+
 def run_config(args, wl, rank, world, local_rank, clocks=None, cpu=True):
     """One workload: the fused decode step timed on the device (a CUDA graph
     of the hyb_decode_step launch, replayed per step), end to end through the
@@ -509,6 +541,7 @@ def run_config(args, wl, rank, world, local_rank, clocks=None, cpu=True):
 
     kvb = synth.kv_bytes(w, quant_bits=qb)
     stepb = kvb + synth.append_bytes(w, n_last, qb)
+    floor = read_floor(torch, dev, stepb, stream, side, args, world)
     peak, peak_kind = measured_peaks()
     value = job_throughput(kvb, world, ms_step)
     tokens_s = w.batch * world / (ms_step * 1e-3)
@@ -548,6 +581,9 @@ def run_config(args, wl, rank, world, local_rank, clocks=None, cpu=True):
         "gpu_launches": DECODE_LAUNCHES[launch_kind] * args.steps,
         "clocks": clk,
     }
+    floor["frac"] = round(floor["GB/s"] / peak, 4)
+    floor["step_over_floor"] = round(ms_step / floor["ms_per_call"], 3)
+    rec["read_floor"] = floor
     if want_cpu:
         sec, n, threads = oracle_step_rate(ora, w, n_last, k_last, v_last, q, 3, 0, budget_s=25.0, qbits=qb)
         rec["cpu_baseline"] = {"value": round(kvb / sec / 1e9, 4), "unit": UNIT, "cores": threads,
@@ -814,7 +850,7 @@ def oracle_one_thread_config1():
 
 
 SUB_KEYS = ("value", "unit", "ms_per_step", "tokens_per_s", "tokens_per_s_model_equiv", "kv_bytes_per_step",
-            "frac_of_hbm_peak_step", "e2e", "e2e_graph", "cpu_baseline", "config")
+            "frac_of_hbm_peak_step", "e2e", "e2e_graph", "cpu_baseline", "config", "read_floor")
 
 
 def main():

@@ -13,6 +13,7 @@ from ._lib import (  # noqa: F401
     hyb_decode_attn_sparse, hyb_decode_sparse_workspace_bytes, hyb_decode_step,
     hyb_decode_step_workspace_bytes, hyb_sparse_top_k,
     hyb_decode_workspace_bytes, hyb_kv_append, hyb_kv_migrate, hyb_last_cuda_error,
-    hyb_migration_decision, hyb_migration_threshold_ms, hyb_read_status, hyb_version, load, strerror,
+    hyb_migration_decision, hyb_migration_threshold_ms, hyb_read_status, hyb_stream_read, hyb_version, load,
+    strerror,
 )
 from .cache import HybridKVCache  # noqa: F401

@@ -35,7 +35,7 @@ EXPORTED = (
     "hyb_last_cuda_error", "hyb_version", "hyb_decode_attn_noalloc", "hyb_noalloc_scratch_limit",
     "hyb_kv_migrate", "hyb_migration_threshold_ms", "hyb_migration_decision",
     "hyb_decode_attn_sparse", "hyb_decode_sparse_workspace_bytes", "hyb_decode_sparse_selection",
-    "hyb_sparse_top_k", "hyb_set_wait_limit", "hyb_decode_launch_info",
+    "hyb_sparse_top_k", "hyb_set_wait_limit", "hyb_decode_launch_info", "hyb_stream_read",
 )
 
 
@@ -113,6 +113,8 @@ def load(path: str = LIB_PATH):
     lib.hyb_migration_decision.argtypes = [ctypes.c_double, ctypes.c_double, i32]
     lib.hyb_migration_decision.restype = ctypes.c_int
     lib.hyb_read_status.argtypes = [D, ctypes.POINTER(i32), i32, P]
+    lib.hyb_stream_read.argtypes = [P, sz, P, P]
+    lib.hyb_stream_read.restype = ctypes.c_int
     lib.hyb_strerror.argtypes = [ctypes.c_int]
     lib.hyb_strerror.restype = ctypes.c_char_p
     for name in ("hyb_check_desc", "hyb_kv_append", "hyb_decode_plan", "hyb_decode_attn", "hyb_decode_step",
@@ -273,6 +275,15 @@ def hyb_set_wait_limit(cycles: int) -> None:
 
 def hyb_last_cuda_error() -> int:
     return load().hyb_last_cuda_error()
+
+
+def hyb_stream_read(src, sink, stream=None) -> None:
+    """One streaming read of the CUDA tensor `src` (contiguous, 16-byte aligned, nbytes a
+    multiple of 16): XORs the XOR of its 32-bit words into the int32 CUDA tensor `sink`."""
+    if not src.is_contiguous():
+        raise HybError(HYB_ERR_INVALID_VALUE, "hyb_stream_read: src must be contiguous")
+    _check(load().hyb_stream_read(_ptr(src), src.numel() * src.element_size(), _ptr(sink),
+                                  _stream(stream)), "hyb_stream_read")
 
 
 def hyb_version() -> int:

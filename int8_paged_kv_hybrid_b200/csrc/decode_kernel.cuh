@@ -231,10 +231,6 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 3)) decode_kernel(cons
     sm.abort_flag = 0;
     mbar_fence_init();
   }
-  if (do_seal) {
-    sm.seal.erow[tid] = __low2half(old_kv);
-    sm.seal.erow[kDim + tid] = __high2half(old_kv);
-  }
   if (tid < ncold) {
     int phys = phys_raw;
     if (phys < 0 || phys >= a.num_phys) {
@@ -245,7 +241,6 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 3)) decode_kernel(cons
   }
   if (tid < 4) sm.zero16[tid] = 0u;
   __syncthreads();
-  if (a.n_new && tid == 32) take_ticket();  // every thread read seq_lens[b] before the barrier above
 
   const uint64_t pol = l2_policy_evict_first();
   auto issue = [&](int k) {
@@ -308,6 +303,13 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 3)) decode_kernel(cons
     for (int k = 0; k < sm.issued; k++) issue(k);
   }
   if (tid < ncold) sm.scl[tid] = sc_ld;
+  // the sealed token's rows: their load depends on seq_lens[b] (the ring
+  // slot), so they are stored only after the copies are on their way; the
+  // barriers of the q preparation below publish them before the seal's item
+  if (do_seal) {
+    sm.seal.erow[tid] = __low2half(old_kv);
+    sm.seal.erow[kDim + tid] = __high2half(old_kv);
+  }
   // q of the head group in 24-bit fixed point and FP16 (padding heads zero)
   prepare_q<G, NH>(qv, sm.qd, sm.qh, sm.sq, sm.qmax_w, warp, lane, tid);
 
@@ -322,6 +324,11 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 4 : 3)) decode_kernel(cons
   // the first channel-tile pair, chunk of tokens 16w..16w+15 (swizzled)
   const uint32_t v_lane0 = smem_addr(sm.ring[0]) + kTileBytes + lane * kBlock + 16 * (warp ^ ((lane >> 1) & 3));
   const uint32_t zero_addr = smem_addr(sm.zero16);
+
+  // The sequence-length ticket (every thread read seq_lens[b] before the
+  // barrier that follows the block-table loads); taken here so that its round
+  // trip overlaps the wait for the first stage
+  if (a.n_new && tid == 32) take_ticket();
 
   // Online-softmax state of this warp (value layout, see decode_dev.cuh)
   WarpState<NT> ws;

@@ -1,13 +1,15 @@
-// hyb_host.cu -- the C ABI declared in include/hyb_kv.h: argument checks,
+// hyb_host.cu -- the C ABI declared in include/hyb_kv.h and include/hyb_measure.h: argument checks,
 // split planning, workspace sizing and kernel launches.  No memory is
 // allocated here; every buffer belongs to the caller.
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdint>
+#include <algorithm>
 #include <atomic>
 #include <cstring>
 
+#include "hyb_measure.h"
 #include "kernels.cuh"
 
 namespace {
@@ -51,6 +53,17 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 extern "C" {
 
 int hyb_version(void) { return 10000; }
+
+int hyb_stream_read(const void *src, size_t bytes, uint32_t *sink, hyb_stream_t stream) {
+  if (bytes == 0) return HYB_OK;  // nothing to read: no launch, no pointer is touched
+  if (!src || !sink || !aligned(src, 16) || !aligned(sink, 4) || bytes % 16 != 0) return HYB_ERR_INVALID_VALUE;
+  const size_t n16 = bytes / 16;
+  const size_t per_cta = static_cast<size_t>(hyb::kStreamReadThreads);
+  const size_t want = (n16 + per_cta - 1) / per_cta;  // no CTA without a load
+  const int grid = static_cast<int>(std::min<size_t>(want, static_cast<size_t>(sm_count()) * hyb::kStreamReadCtasPerSm));
+  const cudaError_t e = hyb::launch_stream_read(src, bytes, sink, grid, stream);
+  return e == cudaSuccess ? HYB_OK : cuda_fail(e);
+}
 
 int hyb_set_wait_limit(int64_t cycles) {
   g_wait_cycles.store(cycles > 0 ? static_cast<long long>(cycles) : 0, std::memory_order_relaxed);

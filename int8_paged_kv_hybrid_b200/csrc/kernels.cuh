@@ -158,6 +158,11 @@ cudaError_t launch_persist_combine(const DecodeArgs &a, int group, int batch, cu
 cudaError_t launch_migrate(const MigrateArgs &a, int batch, cudaStream_t stream);
 cudaError_t launch_combine(const CombineArgs &a, int rows, cudaStream_t stream);
 cudaError_t launch_sparse_l2(const SparseArgs &a, int batch, cudaStream_t stream);
+// hyb_stream_read: one streaming read of `bytes` (a multiple of 16) at src,
+// grid CTAs of kStreamReadThreads threads
+constexpr int kStreamReadThreads = 256;
+constexpr int kStreamReadCtasPerSm = 8;
+cudaError_t launch_stream_read(const void *src, size_t bytes, uint32_t *sink, int grid, cudaStream_t stream);
 int decode_max_split_blocks();
 int decode_ctas_per_sm(int group);
 int decode_max_cluster();

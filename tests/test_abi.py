@@ -301,3 +301,17 @@ def test_migrate_argument_checks():
     d0.n_int4_blocks = 0x7f0000330000
     assert lib.hyb_kv_migrate(ctypes.byref(d0), tgt, 1, None) == _lib.HYB_ERR_UNSUPPORTED
     assert "migration" in hk.strerror(100 + _lib.HYB_STATUS_BAD_TIER)
+
+
+def test_stream_read_argument_checks():
+    """hyb_stream_read rejects null, misaligned and ragged arguments on the host; a
+    zero-byte read launches nothing."""
+    lib = hk.load()
+    src, sink = ctypes.c_void_p(0x7f0000400000), ctypes.c_void_p(0x7f0000500000)
+    bad = _lib.HYB_ERR_INVALID_VALUE
+    assert lib.hyb_stream_read(None, 16, sink, None) == bad
+    assert lib.hyb_stream_read(src, 16, None, None) == bad
+    assert lib.hyb_stream_read(ctypes.c_void_p(0x7f0000400008), 16, sink, None) == bad  # src not 16-aligned
+    assert lib.hyb_stream_read(src, 16, ctypes.c_void_p(0x7f0000500002), None) == bad  # sink not 4-aligned
+    assert lib.hyb_stream_read(src, 24, sink, None) == bad  # not a multiple of 16 bytes
+    assert lib.hyb_stream_read(src, 0, sink, None) == _lib.HYB_OK
