@@ -215,6 +215,12 @@ int hyb_kv_append(const hyb_cache_desc *desc, const int32_t *n_new, int32_t max_
  * count as h = min(tb, ceil(items / I)) blocks (I = items per block: 1 for
  * INT8/INT4 blocks of 32 or 64 tokens, 2 for 128-token blocks, BLK / 32 for
  * FP16 blocks), so that no split holds more than tb blocks' worth of items.
+ * A sequence's splits follow that rule in the kernels that take one CTA per
+ * split; the persistent kernel (several waves, 64-token INT8/INT4 blocks)
+ * cuts sequence b's c_b = nblk_b + h_b items into S_b = max(1, ceil(c_b /
+ * tb)) runs of near-equal length instead -- split s takes items
+ * [floor(s c_b / S_b), floor((s + 1) c_b / S_b)), the ring being the last --
+ * the same count of splits, none longer than tb blocks.
  * Writes the split size used and the number of splits per sequence,
  * n_splits = max(1, ceil((nblk + h) / tb)), nblk = ceil(max(0, max_seq_len -
  * HOT) / BLK).  Returns HYB_OK or HYB_ERR_INVALID_VALUE.  The automatic

@@ -65,6 +65,9 @@ struct PersistMeta {
   int do_seal, do_ring, ring_hbm, pad;
   int32_t phys[kPMaxSplitBlocks];
   float2 scl[kPMaxSplitBlocks];
+  // per query head h: kQFix / max|q_h| and its fixed-point step max|q_h| /
+  // kQFix (0 for rows >= G or an all-zero q)
+  float qinv[NH], qstep[NH];
   alignas(16) __half q[NH][kDim];  // FP16 q of the kv head's query heads, rows >= G zero
 };
 
@@ -97,7 +100,6 @@ struct PersistSmem {
     float mg[2][NH * kMbufPitch];  // warp merge, in the unit's epilogue: two warps' outputs (value layout)
   } u;
   float mg_m[2][NH], mg_l[2][NH];
-  float sq[NH];
   alignas(16) uint32_t zero16[4];
   PendMerge pend;
   int pend_last;  // the pending split merge is this CTA's to do
@@ -313,14 +315,13 @@ __global__ void __launch_bounds__(kPThreads, PersistCfg<G>::kCtasPerSm) decode_p
       const int L = n8 < 0 ? 0 : x.L_old + n_app;
       x.Lc = max(0, L - H);
       const int nblk = (x.Lc + kBlock - 1) / kBlock;
-      if (a.min_splits > 0) {
-        const long long c = nblk + (L > 0 ? 1 : 0);
-        x.i0 = static_cast<int>(x.s * c / x.Sb);
-        x.ncold = max(0, min(nblk, static_cast<int>((x.s + 1) * c / x.Sb)) - x.i0);
-      } else {
-        x.i0 = x.s * tb;
-        x.ncold = max(0, min(nblk, x.i0 + tb) - x.i0);
-      }
+      // the sequence's c items (cold blocks, then the hot ring) in Sb
+      // near-equal runs, so that all its units are the same size (the key of
+      // the longest-first order) and none exceeds split_blocks items
+      const long long c = a.min_splits > 0 ? nblk + (L > 0 ? 1 : 0)
+                                           : nblk + min((min(L, H) + kItemRows - 1) / kItemRows, tb);
+      x.i0 = static_cast<int>(x.s * c / x.Sb);
+      x.ncold = max(0, min(nblk, static_cast<int>((x.s + 1) * c / x.Sb)) - x.i0);
       const bool holds_hot = x.s == x.Sb - 1;
       const bool holds_tail = x.ncold > 0 && x.i0 + x.ncold == nblk;
       x.nhot = holds_hot ? min(L, H) : 0;
@@ -337,9 +338,11 @@ __global__ void __launch_bounds__(kPThreads, PersistCfg<G>::kCtasPerSm) decode_p
     // claimed only a few items before the current one's copies are all out,
     // not a whole unit ahead: a CTA that took a long unit late must not hold
     // another one while the others run out of work.
-    int pend = 0;
+    // The first unit of CTA c is unit c; the counter hands out the units
+    // from gridDim.x on.
+    int pend = blockIdx.x;
     auto claim = [&]() {
-      if (lane == 0) pend = atomicAdd(&a.unit_ctr[0], 1);
+      if (lane == 0) pend = static_cast<int>(gridDim.x) + atomicAdd(&a.unit_ctr[0], 1);
     };
     auto take = [&]() -> Unit {
       const int u = __shfl_sync(0xffffffffu, pend, 0);
@@ -366,13 +369,18 @@ __global__ void __launch_bounds__(kPThreads, PersistCfg<G>::kCtasPerSm) decode_p
       for (int j = 0; j < G; j++) l.q[j] = *reinterpret_cast<const uint2 *>(qb + j * kDim + 4 * lane);
       return l;
     };
-    // the block scales of a unit: a second round trip, issued once its
-    // block-table entries are in (the entry of an invalid block becomes -1)
-    auto load_scales = [&](const Unit &x, Loads &l) {
+    // the block-table entries once they are in: an invalid block's becomes
+    // -1 (no copy, no scale)
+    auto check_phys = [&](const Unit &x, Loads &l) {
       if (lane < x.ncold && (l.phys < 0 || l.phys >= a.num_phys)) {
         set_status(a.status, HYB_STATUS_BAD_BLOCK);
         l.phys = -1;
       }
+    };
+    // the block scales of a unit: a second round trip, issued once its
+    // block-table entries are in
+    auto load_scales = [&](const Unit &x, Loads &l) {
+      check_phys(x, l);
       if (lane < x.ncold && l.phys >= 0)
         l.sc = __ldg(reinterpret_cast<const float2 *>(a.scales + ((size_t)l.phys * a.hkv + x.h) * 2));
     };
@@ -388,10 +396,29 @@ __global__ void __launch_bounds__(kPThreads, PersistCfg<G>::kCtasPerSm) decode_p
       const bool ab = aborted_now(&sm.abort_flag);
       m.phys[lane] = l.phys;
       m.scl[lane] = l.sc;
+      // each head's largest |q| over the lanes' 4 channels, and from it the
+      // reciprocal and the step of the consumers' 24-bit fixed point
+      float qinv = 0.f, qstep = 0.f;  // head `lane`'s
 #pragma unroll
-      for (int j = 0; j < G; j++) *reinterpret_cast<uint2 *>(&m.q[j][4 * lane]) = l.q[j];
+      for (int j = 0; j < G; j++) {
+        *reinterpret_cast<uint2 *>(&m.q[j][4 * lane]) = l.q[j];
+        const __half2 p0 = *reinterpret_cast<const __half2 *>(&l.q[j].x);
+        const __half2 p1 = *reinterpret_cast<const __half2 *>(&l.q[j].y);
+        float mx = fmaxf(fmaxf(fabsf(__low2float(p0)), fabsf(__high2float(p0))),
+                         fmaxf(fabsf(__low2float(p1)), fabsf(__high2float(p1))));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == j) {
+          qinv = mx > 0.f ? kQFix / mx : 0.f;
+          qstep = mx / kQFix;
+        }
+      }
 #pragma unroll
       for (int j = G; j < NH; j++) *reinterpret_cast<uint2 *>(&m.q[j][4 * lane]) = make_uint2(0u, 0u);
+      if (lane < NH) {
+        m.qinv[lane] = qinv;
+        m.qstep[lane] = qstep;
+      }
       if (lane == 0) {
         m.unit = x.u;
         m.b = x.b;
@@ -458,9 +485,11 @@ __global__ void __launch_bounds__(kPThreads, PersistCfg<G>::kCtasPerSm) decode_p
       qi++;
     };
 
-    claim();
     Unit cur = take();
     Loads lcur;
+    // The first unit's copies go out only after its scales are in: issued
+    // earlier, the copies of all CTAs would fill the memory queues ahead of
+    // the scale loads, and the descriptor would come later than the data.
     if (cur.u >= 0) {
       lcur = load(cur);
       load_scales(cur, lcur);
@@ -602,45 +631,26 @@ __global__ void __launch_bounds__(kPThreads, PersistCfg<G>::kCtasPerSm) decode_p
     const bool do_seal = m.do_seal != 0, do_ring = m.do_ring != 0, ring_hbm = m.ring_hbm != 0;
     const int hq0 = h * G;
     const int rs = L_old & (H - 1);
-    // fused step: the evicted token (ring slot rs, read here before the new
-    // token is written there -- same thread, same bytes) into the seal
-    // scratch (seen by the other consumers after the barrier below); the
-    // new token is read again where it goes into the staged ring
-    const size_t kvo = ((size_t)b * a.hkv + h) * kDim + tid;  // channel tid of the new token
-    if (do_seal || ring_hbm) {
-      __half *grow = reinterpret_cast<__half *>(a.hot) + (((size_t)b * a.hkv + h) * H + rs) * 2 * kDim;
-      if (do_seal) {
-        sm.u.w.seal.erow[tid] = grow[tid];
-        sm.u.w.seal.erow[kDim + tid] = grow[kDim + tid];
-      }
-      if (ring_hbm) {
-        grow[tid] = a.k_new[kvo];
-        grow[kDim + tid] = a.v_new[kvo];
-      }
+    // fused step: channel tid of the evicted token (ring slot rs) and of the
+    // new token, loaded now and first used at the seal's item, the ring's
+    // item and after the items, so that no consumer waits for them here.
+    // The evicted token is read before the new one is written to the same
+    // bytes by the same thread.
+    __half *const grow = reinterpret_cast<__half *>(a.hot) + (((size_t)b * a.hkv + h) * H + rs) * 2 * kDim;
+    __half2 old_kv = __halves2half2(__float2half_rn(0.f), __float2half_rn(0.f)), new_kv = old_kv;
+    if (do_seal) old_kv = __halves2half2(grow[tid], grow[kDim + tid]);
+    if (do_ring || ring_hbm) {
+      const size_t kvo = ((size_t)b * a.hkv + h) * kDim + tid;
+      new_kv = __halves2half2(a.k_new[kvo], a.v_new[kvo]);
     }
-    // q of the unit's heads in 24-bit fixed point: every warp finds the
-    // heads' largest |q| itself, thread tid writes channel tid's digits
+    // q of the unit's heads in 24-bit fixed point (the producer found each
+    // head's largest |q|): thread tid writes channel tid's digits
     {
-      float qv[G], qm[G];
-#pragma unroll
-      for (int j = 0; j < G; j++) {
-        qv[j] = __half2float(m.q[j][tid]);
-        const uint2 w4 = *reinterpret_cast<const uint2 *>(&m.q[j][4 * lane]);
-        const __half2 p0 = *reinterpret_cast<const __half2 *>(&w4.x);
-        const __half2 p1 = *reinterpret_cast<const __half2 *>(&w4.y);
-        float mx = fmaxf(fmaxf(fabsf(__low2float(p0)), fabsf(__high2float(p0))),
-                         fmaxf(fabsf(__low2float(p1)), fabsf(__high2float(p1))));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        qm[j] = mx;
-      }
 #pragma unroll
       for (int j = 0; j < NH; j++) {
         int8_t d0 = 0, d1 = 0, d2 = 0;
         if (j < G) {
-          const float M = qm[j < G ? j : 0];
-          const float inv = M > 0.f ? kQFix / M : 0.f;
-          int qi = __float2int_rn(qv[j < G ? j : 0] * inv);
+          int qi = __float2int_rn(__half2float(m.q[j][tid]) * m.qinv[j]);
           qi = max(-8323072, min(8323072, qi));
           const int lo = ((qi + 128) & 255) - 128;
           const int r = (qi - lo) >> 8;
@@ -649,9 +659,6 @@ __global__ void __launch_bounds__(kPThreads, PersistCfg<G>::kCtasPerSm) decode_p
           d0 = static_cast<int8_t>(hi);
           d1 = static_cast<int8_t>(mid);
           d2 = static_cast<int8_t>(lo);
-          if (tid == 0) sm.sq[j] = M / kQFix;
-        } else if (tid == 0) {
-          sm.sq[j] = 0.f;
         }
         sm.u.w.qd[j][0][tid] = d0;
         sm.u.w.qd[j][1][tid] = d1;
@@ -663,7 +670,7 @@ __global__ void __launch_bounds__(kPThreads, PersistCfg<G>::kCtasPerSm) decode_p
     load_qfrag<NT>(sm.u.w.qd, g, t, qa);
     float sqh[NT];
 #pragma unroll
-    for (int nt = 0; nt < NT; nt++) sqh[nt] = sm.sq[4 * nt + (g >> 1)];
+    for (int nt = 0; nt < NT; nt++) sqh[nt] = m.qstep[4 * nt + (g >> 1)];
     const int k_seal = do_seal ? ncold - 1 : -1;
     const int k_ring = do_ring ? ncold + rs / kItemRows : -1;
 
@@ -674,13 +681,18 @@ __global__ void __launch_bounds__(kPThreads, PersistCfg<G>::kCtasPerSm) decode_p
       bool ok = !aborted_now(&sm.abort_flag) && mbar_wait_bounded(&sm.full[st], (qc / S) & 1, a.wait_cycles);
       if (!ok && lane == 0 && !aborted_now(&sm.abort_flag)) set_status(a.status, HYB_STATUS_TIMEOUT);
       if (k == k_seal || k == k_ring) {
+        if (k == k_seal) {
+          // published to the other consumers by the barrier below
+          sm.u.w.seal.erow[tid] = __low2half(old_kv);
+          sm.u.w.seal.erow[kDim + tid] = __high2half(old_kv);
+        }
         ok = consumers_and(ok);
         if (ok && k == k_seal)
           fused_seal<true>(sm.u.w.seal, sm.ring[st], &sm.meta[slot].scl[ncold - 1],
                            m.phys[ncold - 1] * a.hkv + h, (i0 + ncold - 1) < n_int4_b, a, L_old, true, tid, warp,
                            lane);
         else if (ok)
-          ring_put<true, kPRowPitch>(sm.ring[st], rs, __halves2half2(a.k_new[kvo], a.v_new[kvo]), tid);
+          ring_put<true, kPRowPitch>(sm.ring[st], rs, new_kv, tid);
       }
       if (!ok) sm.abort_flag = 1;
       const uint8_t *stage = sm.ring[st];
@@ -710,6 +722,12 @@ __global__ void __launch_bounds__(kPThreads, PersistCfg<G>::kCtasPerSm) decode_p
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[st]);
       qc++;
+    }
+    if (ring_hbm) {
+      // the new token into the ring in HBM (after this thread's read of the
+      // evicted token from the same bytes)
+      grow[tid] = __low2half(new_kv);
+      grow[kDim + tid] = __high2half(new_kv);
     }
     // the slot is not read after this point (the epilogue works from
     // registers and the merge buffer)

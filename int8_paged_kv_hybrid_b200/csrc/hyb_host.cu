@@ -160,6 +160,13 @@ namespace {
 
 // Cold blocks per split when the splits take several waves.
 constexpr int kMultiWaveSplit = 16;
+// Longest automatic split of the persistent kernel for head groups above 4
+// (two 4-head MMA row tiles): their blocks cost about twice the arithmetic
+// of a group of up to 4, so a split of kPMaxSplitBlocks blocks runs twice as
+// long and the last units handed out leave that much of a tail.  Measured on
+// the Qwen2-7B mixed batch (group 7): 24-block splits 121.4 us per step, 32:
+// 125.7, 16: 125.2, 12: 136.3.
+constexpr int kPWideSplit = 24;
 // Fewest blocks per split of a one-wave plan: a CTA's fixed cost (the
 // metadata round trip before its first copy, the epilogue and the split
 // merge, ~3 us) wants a few items of work.  On the Llama-3-8B batch of 8 at
@@ -253,10 +260,11 @@ int make_plan(const hyb_cache_desc *d, int32_t max_seq_len, int32_t split_tokens
       // as the GPU's CTA slots would otherwise give each row one long split).
       // The persistent kernel takes these plans where it can: it hands out
       // the longest splits first and claims units late, so long splits
-      // (fewer per-unit prologues and merges) cost no tail; the split-per-CTA
+      // (fewer per-unit prologues and merges) cost little tail -- shorter
+      // ones for wide head groups, whose blocks take longer; the split-per-CTA
       // kernel gets short splits, so that the CTA scheduler evens out rows of
       // different lengths.
-      tb = persist_ok ? hyb::kPMaxSplitBlocks : kMultiWaveSplit;
+      tb = !persist_ok ? kMultiWaveSplit : group > 4 ? kPWideSplit : hyb::kPMaxSplitBlocks;
       multi_wave = true;
       if (tb > nblk) tb = nblk > 0 ? nblk : 1;
     }

@@ -40,10 +40,16 @@ def test_wait_limit_times_out_then_recovers(split):
     o = out.float()
     assert torch.isfinite(o).all()
     # rows whose splits all gave up are exactly zero with lse -inf; a split
-    # whose copies had already landed may still contribute to its row
+    # whose copies had already landed may still contribute to its row.  In
+    # the one-CTA-per-split kernel some rows always give up whole; in the
+    # persistent kernel (split < 0) the producer issues a unit's first copies
+    # before its consumers reach it, so whether every unit of a row finds
+    # data missing within the limit depends on timing
     gave_up = torch.isneginf(lse)
-    assert gave_up.any()
-    assert float(o[gave_up].abs().max()) == 0.0
+    if split > 0:
+        assert gave_up.any()
+    if gave_up.any():
+        assert float(o[gave_up].abs().max()) == 0.0
     # the cache is untouched and the next call, with the default limit, is right
     got, lse2, ref, ref_lse = decode_both(w, cache, ora, split_tokens=split)
     assert_decode_close(w, got, lse2, ref, ref_lse, what="after timeout split=%d" % split)
