@@ -141,8 +141,22 @@ __device__ __forceinline__ void fused_seal(SealScratch &ss, uint8_t *tile_st, fl
   for (int kv = 0; kv < 2; kv++) {
     if (!ss.seal_rq[kv]) continue;
     uint32_t *w32 = reinterpret_cast<uint32_t *>(tile_st + kv * kTileBytes);
-    const int nw = requant_nwords(kv, int4, slot);
-    for (int w = tid; w < nw; w += kThreads) w32[w] = requant_word(w32[w], w, kv, int4, slot, ss.rqt[kv]);
+    if (kv == 0) {
+      // K, token-major: the words of slots < slot lead the tile
+      const int nw = requant_nwords(0, int4, slot);
+      for (int w = tid; w < nw; w += kThreads) w32[w] = requant_word(w32[w], w, 0, int4, slot, ss.rqt[0]);
+    } else {
+      // V, channel-major: per channel row only the words of tokens < slot
+      // (4 INT8 or 8 INT4 tokens a word, at their swizzled places)
+      const int tw = int4 ? 8 : 4;  // tokens per word
+      const int per_row = (slot + tw - 1) / tw;
+      for (int i = tid; i < kDim * per_row; i += kThreads) {
+        const int r = i / per_row, tj = i - r * per_row;
+        const int w = int4 ? r * 8 + 2 * ((tj >> 1) ^ ((r >> 2) & 3)) + (tj & 1)
+                           : r * 16 + 4 * ((tj >> 2) ^ ((r >> 1) & 3)) + (tj & 3);
+        w32[w] = requant_word(w32[w], w, 1, int4, slot, ss.rqt[1]);
+      }
+    }
   }
   work_sync<kNamed>();
   const int c = tid;  // channel
