@@ -108,16 +108,18 @@ def parse():
 COLD_KIND = {8: "INT8", 4: "INT4", 0: "FP16"}
 
 
-def split_desc(split, split_len, ns):
+def split_desc(split, split_len, ns, persistent=False):
     if split < 0:
         return ("per sequence: at least %d near-equal splits of <= 32 blocks (the longest sequence: %d splits "
                 "of <= %d tokens)" % (-split, ns, split_len))
-    if split == 0:
-        return "automatic: %d splits of %d tokens" % (ns, split_len)
-    return "%d splits of %d tokens" % (ns, split)
+    head = "automatic: " if split == 0 else ""
+    if persistent:
+        # the persistent kernel cuts each sequence into near-equal splits of at most split_len tokens
+        return "%seach sequence in near-equal splits of <= %d tokens (the longest: %d)" % (head, split_len, ns)
+    return "%s%d splits of %d tokens" % (head, ns, split_len)
 
 
-def workload_config(w, split, ns, qbits=8, split_len=None):
+def workload_config(w, split, ns, qbits=8, split_len=None, persistent=False):
     lens = w.lens
     cold = COLD_KIND[qbits]
     if qbits == 8 and w.n_int4 is not None:
@@ -136,7 +138,7 @@ def workload_config(w, split, ns, qbits=8, split_len=None):
     return {"workload": what, "batch": int(w.batch), "seq_len": int(lens.max()),
             "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads, "head_dim": 128, "hot_tokens": H,
             "block_size": w.block_size, "quant_bits": qbits, "split_tokens": split, "n_splits": ns,
-            "splits": split_desc(split, split if split_len is None else split_len, ns),
+            "splits": split_desc(split, split if split_len is None else split_len, ns, persistent),
             "step": "hyb_decode_step: append 1 token/seq + split-KV attention, one launch",
             "l2": L2_NOTE,
             "parallelism": "replicas (independent batch per GPU)"}
@@ -555,7 +557,7 @@ def run_config(args, wl, rank, world, local_rank, clocks=None, cpu=True):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": {8: "int8", 4: "int4", 0: "f16"}[qb],
         "data": "synthetic (seeded N(0,1) FP16 K/V/q; caches built by the library's own appends)",
-        "config": workload_config(w, split, ns, qb, split_len),
+        "config": workload_config(w, split, ns, qb, split_len, persistent=launch_kind >= 2),
         "tokens_per_s": round(tokens_s, 1),
         "tokens_per_s_model_equiv": round(tokens_s / layers, 1),
         "kv_bytes_per_step": kvb,
