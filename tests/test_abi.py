@@ -184,6 +184,22 @@ def test_launch_info():
         hk.hyb_decode_launch_info(d, 4096, 100)
 
 
+def test_automatic_multiwave_split_length_by_head_group():
+    """Several waves of splits on the persistent kernel: the automatic plan's
+    longest split is 32 blocks for head groups of up to 4 and 24 above (a
+    wider group's block costs about twice the arithmetic, so shorter units
+    keep the tail of the launch short)."""
+    w3, w5 = synth.make_workload(3), synth.make_workload(5)
+    for w, want in ((w3, 32 * 64), (w5, 24 * 64)):
+        d = _desc(batch=w.batch, maxb=w.max_blocks, phys=w.num_phys_blocks, hkv=w.num_kv_heads,
+                  hq=w.num_q_heads)
+        L = int(w.lens.max())
+        tokens, ns = hk.hyb_decode_plan(d, L, 0)
+        nblk = -(-(L - 32) // 64)
+        assert tokens == want and ns == -(-(nblk + 1) // (want // 64)), (w.name, tokens, ns)
+        assert hk.hyb_decode_launch_info(d, L, 0)[0] == "persistent"
+
+
 @pytest.mark.parametrize("block,hot", [(32, 16), (128, 64), (64, 128)])
 def test_plan_other_block_and_hot_sizes(block, hot):
     """Splits count blocks of the descriptor's size; the cold range is the
