@@ -37,3 +37,16 @@ def test_config_object(qb, hot, blk):
     # every sequence has a physical block for each of its cold blocks
     need = w.cold_blocks()
     assert all((w.block_table[b, :need[b]] >= 0).all() for b in range(w.batch))
+
+
+def test_split_descriptions():
+    """The configuration's split text says what the launched kernel does: runs
+    of the split length on the one-CTA-per-split kernels, near-equal splits of
+    at most that length per sequence on the persistent one, at least n
+    near-equal splits for split_tokens = -n."""
+    assert bench.split_desc(0, 384, 6) == "automatic: 6 splits of 384 tokens"
+    assert bench.split_desc(512, 512, 5) == "5 splits of 512 tokens"
+    d = bench.split_desc(0, 2048, 4, persistent=True)
+    assert d.startswith("automatic: ") and "near-equal" in d and "<= 2048 tokens" in d
+    d = bench.split_desc(-64, 2048, 65, persistent=True)
+    assert "at least 64 near-equal splits" in d and "65 splits" in d
