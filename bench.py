@@ -76,6 +76,11 @@ DECODE_KERNELS = {"persistent": "hyb::decode_persist_kernel", "split_cta": "hyb:
 DECODE_LAUNCHES = {"persistent": 1, "split_cta": 1, "cluster": 1, "persistent+combine": 2}
 
 
+def is_persistent(kind):
+    """The launch kind (hyb_decode_launch_info's name) runs the persistent kernel."""
+    return kind in ("persistent", "persistent+combine")
+
+
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
@@ -557,7 +562,7 @@ def run_config(args, wl, rank, world, local_rank, clocks=None, cpu=True):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": {8: "int8", 4: "int4", 0: "f16"}[qb],
         "data": "synthetic (seeded N(0,1) FP16 K/V/q; caches built by the library's own appends)",
-        "config": workload_config(w, split, ns, qb, split_len, persistent=launch_kind >= 2),
+        "config": workload_config(w, split, ns, qb, split_len, persistent=is_persistent(launch_kind)),
         "tokens_per_s": round(tokens_s, 1),
         "tokens_per_s_model_equiv": round(tokens_s / layers, 1),
         "kv_bytes_per_step": kvb,

@@ -50,3 +50,14 @@ def test_split_descriptions():
     assert d.startswith("automatic: ") and "near-equal" in d and "<= 2048 tokens" in d
     d = bench.split_desc(-64, 2048, 65, persistent=True)
     assert "at least 64 near-equal splits" in d and "65 splits" in d
+
+
+def test_launch_kinds_are_known():
+    """Every launch kind the library reports has a kernel name and a launch
+    count in the bench, and the persistent ones are told apart by name."""
+    from int8_paged_kv_hybrid_b200 import _lib
+    for kind in _lib.KERNEL_NAMES.values():
+        assert kind in bench.DECODE_KERNELS and kind in bench.DECODE_LAUNCHES
+        assert bench.is_persistent(kind) == kind.startswith("persistent")
+        cfg = bench.workload_config(synth.make_workload(3), 0, 4, 8, 2048, persistent=bench.is_persistent(kind))
+        assert ("near-equal" in cfg["splits"]) == bench.is_persistent(kind)
